@@ -1,0 +1,124 @@
+"""Seeded synthetic inputs for the LSA path.
+
+This module only draws inputs; it holds none of the method's arithmetic.  It
+is the one piece the CUDA library's tests / benchmark and the CPU oracle both
+use.  Recipe (a stand-in for the long-context prefill/decode workloads the
+LSA pages measure on real models, whose weights and datasets are not used):
+
+* centres: ``n_centres`` unit vectors (normalised N(0, I_d));
+* keys:    k_{t,h} = 4 * mu_{c} + N(0, I_d), c uniform per (token, kv-head);
+* queries: q_{t,h} = mu_{c'} + N(0, I_d), c' uniform per (token, q-head);
+* values:  N(0, 1);
+* W_k, W_q: independent random orthonormal d x d_latent matrices (QR of a
+  Gaussian, signs fixed so diag(R) > 0), fp32;
+* everything drawn in fp32 and rounded to bf16 (ties to even).
+
+Streams are numpy PCG64 generators keyed by (seed, tensor tag), so any tensor
+can be regenerated alone and in token chunks.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+# The five workloads (shapes of the pages' single-layer prefill / decode
+# measurements).  T = context tokens, hkv / hq = KV / query heads.
+CONFIGS = {
+    "prefill-4k": dict(T=4096, hkv=1, hq=4, d=128, dl=64, n_centres=32, k=512,
+                       sinks=4, window=256, mode=0, agg=0, beam=2),
+    "prefill-128k": dict(T=131072, hkv=8, hq=32, d=128, dl=64, n_centres=1024,
+                         k=2048, sinks=4, window=1024, mode=0, agg=0, beam=2),
+    "prefill-1m": dict(T=1 << 20, hkv=8, hq=32, d=128, dl=64, n_centres=8192,
+                       k=2048, sinks=4, window=1024, mode=0, agg=0, beam=2),
+    "decode-32x1m": dict(T=1 << 20, batch=32, hkv=8, hq=32, d=128, dl=64,
+                         n_centres=8192, k=2048, sinks=4, window=1024, mode=0,
+                         agg=0, beam=2),
+    "decode-4x10m": dict(T=10_000_000, batch=4, hkv=8, hq=32, d=128, dl=64,
+                         n_centres=65536, k=2048, sinks=4, window=1024, mode=0,
+                         agg=0, beam=2),
+}
+
+_TAGS = {"centres": 1, "kc": 2, "kn": 3, "qc": 4, "qn": 5, "v": 6, "wk": 7, "wq": 8}
+
+
+def _rng(seed: int, tag: str, chunk: int = 0) -> np.random.Generator:
+    return np.random.Generator(np.random.PCG64(np.random.SeedSequence([seed, _TAGS[tag], chunk])))
+
+
+def f32_to_bf16_bits(x: np.ndarray) -> np.ndarray:
+    """fp32 -> bf16 bit patterns, round to nearest even (finite inputs)."""
+    u = np.ascontiguousarray(x, dtype=np.float32).view(np.uint32)
+    r = (u + np.uint32(0x7FFF) + ((u >> np.uint32(16)) & np.uint32(1))) >> np.uint32(16)
+    return r.astype(np.uint16)
+
+
+def bf16_bits_to_f32(b: np.ndarray) -> np.ndarray:
+    return (np.ascontiguousarray(b, dtype=np.uint16).astype(np.uint32) << np.uint32(16)).view(np.float32)
+
+
+def centres(seed: int, n: int, d: int) -> np.ndarray:
+    c = _rng(seed, "centres").standard_normal((n, d), dtype=np.float32)
+    c /= np.linalg.norm(c, axis=1, keepdims=True)
+    return c
+
+
+def orthonormal(seed: int, tag: str, d: int, dl: int) -> np.ndarray:
+    g = _rng(seed, tag).standard_normal((d, dl))
+    q, r = np.linalg.qr(g)
+    q = q * np.sign(np.diag(r))[None, :]
+    return np.ascontiguousarray(q, dtype=np.float32)
+
+
+def projections(seed: int = 0, d: int = 128, dl: int = 64):
+    """(W_k, W_q), fp32 [d, dl] row-major."""
+    return orthonormal(seed, "wk", d, dl), orthonormal(seed, "wq", d, dl)
+
+
+_CHUNK = 8192  # tokens per generator chunk (tensors are drawn chunk by chunk)
+
+
+def _tokens(seed, kind, t0, t1, heads, d, mu, scale):
+    """bf16 bits [t1 - t0, heads, d] of `scale * mu_c + N(0, I)` (kind k/q)
+    or N(0, 1) (kind v), drawn chunk-wise so any token range is reproducible."""
+    out = np.empty((t1 - t0, heads, d), np.uint16)
+    c0 = t0 // _CHUNK
+    c1 = (t1 + _CHUNK - 1) // _CHUNK
+    for c in range(c0, c1):
+        a, b = c * _CHUNK, (c + 1) * _CHUNK
+        if kind == "v":
+            x = _rng(seed, "v", c).standard_normal((_CHUNK, heads, d), dtype=np.float32)
+        else:
+            ci = _rng(seed, kind + "c", c).integers(0, mu.shape[0], size=(_CHUNK, heads))
+            x = _rng(seed, kind + "n", c).standard_normal((_CHUNK, heads, d), dtype=np.float32)
+            x += np.float32(scale) * mu[ci]
+        lo, hi = max(a, t0), min(b, t1)
+        out[lo - t0:hi - t0] = f32_to_bf16_bits(x[lo - a:hi - a])
+    return out
+
+
+def layer_inputs(name: str = "prefill-4k", seed: int = 0, T: int | None = None,
+                 parts=("Q", "K", "V")) -> dict:
+    """Q [T, hq, d], K/V [T, hkv, d] as bf16 bits, W_k/W_q fp32 [d, dl].
+    `T` overrides the configuration's length (a prefix of the same stream)."""
+    c = CONFIGS[name]
+    T = c["T"] if T is None else T
+    mu = centres(seed, c["n_centres"], c["d"])
+    Wk, Wq = projections(seed, c["d"], c["dl"])
+    out = dict(Wk=Wk, Wq=Wq, cfg=dict(c, T=T))
+    if "K" in parts:
+        out["K"] = _tokens(seed, "k", 0, T, c["hkv"], c["d"], mu, 4.0)
+    if "V" in parts:
+        out["V"] = _tokens(seed, "v", 0, T, c["hkv"], c["d"], mu, 0.0)
+    if "Q" in parts:
+        out["Q"] = _tokens(seed, "q", 0, T, c["hq"], c["d"], mu, 1.0)
+    return out
+
+
+def query_rows(name: str, tpos, seed: int = 0) -> np.ndarray:
+    """The Q rows at positions `tpos` (same values as layer_inputs' Q)."""
+    c = CONFIGS[name]
+    mu = centres(seed, c["n_centres"], c["d"])
+    tpos = np.asarray(tpos, np.int64)
+    out = np.empty((tpos.size, c["hq"], c["d"]), np.uint16)
+    for i, t in enumerate(tpos):
+        out[i] = _tokens(seed, "q", int(t), int(t) + 1, c["hq"], c["d"], mu, 1.0)[0]
+    return out
