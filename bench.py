@@ -1,0 +1,350 @@
+#!/usr/bin/env python
+"""LSA single-layer prefill throughput on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl lsa|reference]
+                    [--workload prefill-128k|prefill-4k|prefill-1m] [--mode flat|tree]
+                    [--agg mean|max]
+
+A step is one whole LSA attention layer over a T-token prompt (key build:
+latents + Ward buckets; [tree]; per query chunk: query latents, centroid
+scoring, selection + assembly, sparse attention), inputs already in HBM.
+`value` = tokens/s summed over ranks (each rank runs its own layer: weak
+scaling, no collective on the data path).  `e2e` repeats the measurement
+through the whole-layer C-ABI call (lsa_prefill) from pinned host buffers,
+with the Q/K/V upload and the O download inside the timed region.
+
+--impl reference times the CPU oracle (the method restated in plain fp64 C)
+on a bounded sample of the same workload, extrapolated to the same metric.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+METRIC = "LSA layer prefill tokens/s"
+UNIT = "tokens/s"
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=5)
+    p.add_argument("--warmup", type=int, default=3)
+    p.add_argument("--impl", default="lsa", choices=["lsa", "reference"])
+    p.add_argument("--workload", default="prefill-128k",
+                   choices=["prefill-4k", "prefill-128k", "prefill-1m"])
+    p.add_argument("--mode", default=None, choices=["flat", "tree"])
+    p.add_argument("--agg", default=None, choices=["mean", "max"])
+    p.add_argument("--chunk", type=int, default=16384)
+    p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--no-cpu", action="store_true")
+    return p.parse_args()
+
+
+def workload_cfg(args):
+    c = dict(synth.CONFIGS[args.workload])
+    if args.mode:
+        c["mode"] = 0 if args.mode == "flat" else 1
+    if args.agg:
+        c["agg"] = 0 if args.agg == "mean" else 1
+    return c
+
+
+def config_json(args, c, world):
+    return {
+        "workload": args.workload, "T": c["T"], "hkv": c["hkv"], "hq": c["hq"], "d_head": c["d"],
+        "d_latent": c["dl"], "k": c["k"], "sinks": c["sinks"], "window": c["window"],
+        "search": "flat" if c["mode"] == 0 else f"tree(beam={c['beam']})",
+        "query_score": "group-mean" if c["agg"] == 0 else "max-over-heads (native)",
+        "query_chunk": args.chunk, "parallelism": f"replicas x{world} (one layer per GPU)",
+        "l2": "no flush: per-step inputs (Q/K/V) are larger than L2",
+    }
+
+
+# --------------------------------------------------------------- helpers
+
+class Clocks:
+    """nvidia-smi samples during the timed region."""
+
+    def __init__(self, dev_index: int):
+        self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+        try:
+            self.p = subprocess.Popen(["nvidia-smi", f"--query-gpu={q}", "--format=csv,noheader,nounits",
+                                       "-lms", "200", "-i", str(dev_index)], stdout=self.f,
+                                      stderr=subprocess.DEVNULL)
+        except OSError:
+            self.p = None
+
+    def stop(self) -> dict:
+        if self.p is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.p.terminate()
+        self.p.wait()
+        self.f.seek(0)
+        rows = [r.split(",") for r in self.f.read().strip().splitlines() if r.count(",") >= 8]
+        os.unlink(self.f.name)
+        sm = [float(r[1]) for r in rows if r[1].strip().replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].strip().replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if "Active" in v and "Not" not in v})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+def peaks():
+    try:
+        return json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json"))), "measured"
+    except (OSError, ValueError):
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}, "fallback"
+
+
+# ------------------------------------------------------------ CPU oracle
+
+def oracle_sample(inp, c, n_blocks=None, n_queries=32, seed=0):
+    """Time the oracle on one kv-head: the build of `n_blocks` cluster blocks
+    (all if None) and select + attention for `n_queries` stratified positions.
+    Returns (seconds per layer extrapolated to T x hkv, description)."""
+    import oracle
+    T, hkv = c["T"], c["hkv"]
+    G = c["hq"] // hkv
+    ocfg = oracle.Cfg(k=c["k"], sinks=c["sinks"], window=c["window"], beam=c["beam"],
+                      mode=c["mode"], agg=c["agg"])
+    Tb = T if n_blocks is None else min(T, 512 * n_blocks)
+    K1 = np.ascontiguousarray(inp["K"][:, :1])
+    t0 = time.perf_counter()
+    U = oracle.key_latent_pool(K1[:Tb], inp["Wk"], 4)
+    cache = oracle.build_cache(U, Tb, ocfg)
+    tree = oracle.build_tree(cache) if c["mode"] == 1 else None
+    t_build = time.perf_counter() - t0
+    if Tb < T:  # the query sample needs the whole head's cache
+        U = oracle.key_latent_pool(K1, inp["Wk"], 4)
+        cache = oracle.build_cache(U, T, ocfg)
+        tree = oracle.build_tree(cache) if c["mode"] == 1 else None
+    rng = np.random.default_rng(seed)
+    lo = c["window"] + c["sinks"]
+    tpos = np.sort(rng.choice(np.arange(lo, T), size=n_queries, replace=False))
+    Qs = np.ascontiguousarray(inp["Q"][tpos][:, :G])
+    t1 = time.perf_counter()
+    Y = oracle.query_latent(Qs, inp["Wq"], 1, c["agg"])
+    idx, _, _ = oracle.select(cache, Y, tpos, ocfg, tree=tree, G=G)
+    oracle.attention(Qs, K1, np.ascontiguousarray(inp["V"][:, :1]), idx)
+    t_q = (time.perf_counter() - t1) / n_queries
+    per_layer = t_build * (T / Tb) * hkv + t_q * T * hkv
+    desc = (f"1 of {hkv} kv-heads: build of {Tb // 512} blocks ({Tb} keys) + select/attention of "
+            f"{n_queries} stratified query positions (G={G} heads), extrapolated to T={T} x {hkv} heads")
+    return per_layer, desc, t_build + t_q * n_queries
+
+
+# ------------------------------------------------------------------ main
+
+def dist_setup(args):
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600),
+                                device_id=torch.device("cuda", local))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def run_reference(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    c = workload_cfg(args)
+    inp = synth.layer_inputs(args.workload, seed=0, parts=("Q", "K", "V"))
+    vals = []
+    desc = ""
+    for i in range(args.warmup + args.steps):
+        per_layer, desc, _ = oracle_sample(inp, c, n_blocks=8, n_queries=4, seed=i)
+        if i >= args.warmup:
+            vals.append(c["T"] / per_layer)
+    v = statistics.median(vals)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * c["T"] / v,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": config_json(args, c, 1),
+        "cpu_baseline": {"value": v, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": desc},
+        "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def run_lsa(args):
+    import torch
+
+    import torch.distributed as dist
+
+    import clustered_key_indexing_b200 as lsa
+    from clustered_key_indexing_b200._lib import lib
+
+    world, rank, local = dist_setup(args)
+    c = workload_cfg(args)
+    T, hkv, hq = c["T"], c["hkv"], c["hq"]
+    cfg = lsa.Config(k=c["k"], sinks=c["sinks"], window=c["window"], beam=c["beam"],
+                     mode=c["mode"], agg=c["agg"])
+    inp = synth.layer_inputs(args.workload, seed=rank)
+    dev = torch.device("cuda", torch.cuda.current_device())
+
+    def pinned(bits):
+        return torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).pin_memory()
+
+    hQ, hK, hV = pinned(inp["Q"]), pinned(inp["K"]), pinned(inp["V"])
+    Q, K, V = hQ.to(dev), hK.to(dev), hV.to(dev)
+    Wk, Wq = torch.from_numpy(inp["Wk"]).to(dev), torch.from_numpy(inp["Wq"]).to(dev)
+    cache = lsa.Cache(hkv, T, cfg, device=dev)
+    tree = lsa.Tree(cache, device=dev) if cfg.mode == 1 else None
+    O = torch.empty_like(Q)
+    chunk = min(args.chunk, T)
+    row = cfg.row
+    idx = torch.empty((chunk, hkv, row), dtype=torch.int32, device=dev)
+    sws = torch.empty(lsa.select_workspace_bytes(cfg, chunk, hq, cache) or 1, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    chunks = [(t0, min(chunk, T - t0)) for t0 in range(0, T, chunk)]
+    attn_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in chunks]
+
+    def step(timed_attn=False):
+        lsa.build_buckets(K, Wk, cfg, cache)
+        if tree is not None:
+            lsa.build_tree(cache, cfg, tree)
+        for ci, (t0, n) in enumerate(chunks):
+            lsa.select(Q[t0:t0 + n], t0, Wq, cache, cfg, tree=tree, idx=idx[:n], ws=sws)
+            if timed_attn:
+                attn_ev[ci][0].record(stream)
+            lsa.sparse_attn(Q[t0:t0 + n], K, V, idx[:n], T, O=O[t0:t0 + n])
+            if timed_attn:
+                attn_ev[ci][1].record(stream)
+
+    # algorithmic bytes of the attention launches: every valid index entry
+    # gathers one K row and one V row (2 x 256 B); plus Q read and O write
+    step()
+    torch.cuda.synchronize()
+    valid = 0
+    lsa.build_buckets(K, Wk, cfg, cache)
+    if tree is not None:
+        lsa.build_tree(cache, cfg, tree)
+    for t0, n in chunks:
+        lsa.select(Q[t0:t0 + n], t0, Wq, cache, cfg, tree=tree, idx=idx[:n], ws=sws)
+        valid += int((idx[:n] >= 0).sum().item())
+    lsa.check_device_error()
+    attn_bytes = valid * 2 * 256 + 2 * T * hq * 128 * 2
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clocks = Clocks(torch.cuda.current_device())
+    n0 = lib().lsa_launch_count()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    ev0.record(stream)
+    attn_ms = 0.0
+    for _ in range(args.steps):
+        step(timed_attn=True)
+        torch.cuda.synchronize()  # read this step's attention events
+        attn_ms += sum(a.elapsed_time(b) for a, b in attn_ev)
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    launches = lib().lsa_launch_count() - n0
+    ms = ev0.elapsed_time(ev1)
+    if world > 1:
+        tt = torch.tensor([ms], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms = float(tt.item())
+        dist.barrier()
+    lsa.check_device_error()
+    ms_step = ms / args.steps
+    value = world * T / (ms_step / 1e3)
+
+    # e2e: the whole-layer C-ABI call from pinned host buffers
+    e2e = None
+    if not args.no_e2e:
+        hO = torch.empty_like(hQ).pin_memory()
+        pws = torch.empty(lsa.prefill_workspace_bytes(cfg, T, hq, hkv, chunk), dtype=torch.uint8, device=dev)
+
+        def e2e_step():
+            Q.copy_(hQ, non_blocking=True)
+            K.copy_(hK, non_blocking=True)
+            V.copy_(hV, non_blocking=True)
+            lsa.prefill(Q, K, V, Wk, Wq, cfg, cache=cache, tree=tree, O=O, chunk=chunk, ws=pws)
+            hO.copy_(O, non_blocking=True)
+
+        for _ in range(max(1, args.warmup)):
+            e2e_step()
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ems = e0.elapsed_time(e1)
+        if world > 1:
+            tt = torch.tensor([ems], device=dev)
+            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+            ems = float(tt.item())
+        e2e = {"value": world * T / (ems / args.steps / 1e3), "unit": UNIT,
+               "h2d_bytes_per_step": hQ.numel() * 2 + hK.numel() * 2 + hV.numel() * 2,
+               "d2h_bytes_per_step": hO.numel() * 2}
+
+    pk, src = peaks()
+    attn_ms_launch = attn_ms / (args.steps * len(chunks))
+    achieved = (attn_bytes / len(chunks)) / (attn_ms_launch / 1e3) / 1e9
+    roofline = {"kernel": "attn_kernel", "bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"],
+                "unit": "GB/s", "frac": achieved / pk["hbm_gbs"], "traffic": None,
+                "peak_source": src, "attn_share_of_step": attn_ms / ms if ms > 0 else None,
+                "bytes_per_launch": attn_bytes / len(chunks)}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu:
+        per_layer, desc, spent = oracle_sample(inp, c, n_blocks=None if T <= 131072 else 64, n_queries=16)
+        cpu = {"value": T / per_layer, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": desc,
+               "sample_seconds": spent}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": config_json(args, c, world), "clocks": clk, "e2e": e2e,
+            "gpu_launches": int(launches), "roofline": roofline, "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    a = parse()
+    if a.impl == "reference":
+        run_reference(a)
+    else:
+        run_lsa(a)

@@ -1,0 +1,208 @@
+"""PyTorch-facing calls of the LSA library (marshalling only).
+
+Tensors are CUDA tensors: Q/K/V/O torch.bfloat16, W_k/W_q torch.float32
+[128, 64], index lists torch.int32.  Streams default to torch's current
+stream.  Each call maps one-to-one onto an entry point of include/lsa.h.
+"""
+from __future__ import annotations
+
+import ctypes
+from dataclasses import dataclass, fields
+
+import torch
+
+from . import _lib
+from ._lib import check, lib
+
+
+def _ptr(t):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else None
+
+
+def _stream(stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _need_cuda(*ts):
+    for t in ts:
+        if t is not None and not t.is_cuda:
+            raise ValueError("LSA calls take CUDA tensors (there is no CPU implementation)")
+        if t is not None and not t.is_contiguous():
+            raise ValueError("LSA calls take contiguous tensors")
+
+
+@dataclass
+class Config:
+    """Method parameters (see lsa_cfg in include/lsa.h)."""
+    d_head: int = 128
+    d_latent: int = 64
+    pool: int = 4
+    block: int = 512
+    bucket_mean: int = 8
+    bucket_max: int = 16
+    k: int = 2048
+    sinks: int = 4
+    window: int = 1024
+    beam: int = 2
+    mode: int = 0   # 0 flat, 1 tree
+    agg: int = 0    # 0 group mean, 1 max over heads (native)
+
+    def c(self) -> _lib.lsa_cfg:
+        return _lib.lsa_cfg(*[getattr(self, f.name) for f in fields(self)])
+
+    @property
+    def row(self) -> int:
+        return self.sinks + self.k + self.window
+
+
+class Cache:
+    """Device arrays of one layer's bucket cache (lsa_cache), sized for
+    `cap_tokens` tokens per head."""
+
+    def __init__(self, hkv: int, cap_tokens: int, cfg: Config | None = None, device="cuda"):
+        cfg = cfg or Config()
+        cc = cfg.c()
+        L = lib()
+        self.hkv = hkv
+        self.cap_units = int(L.lsa_cache_units(ctypes.byref(cc), cap_tokens))
+        self.cap_buckets = int(L.lsa_cache_buckets(ctypes.byref(cc), cap_tokens))
+        dl = cfg.d_latent
+        z = dict(device=device)
+        self.U = torch.zeros((hkv, self.cap_units, dl), dtype=torch.float64, **z)
+        self.bucket_of_unit = torch.full((hkv, self.cap_units), -1, dtype=torch.int32, **z)
+        self.members = torch.full((hkv, self.cap_units), -1, dtype=torch.int32, **z)
+        self.offsets = torch.zeros((hkv, self.cap_buckets + 1), dtype=torch.int32, **z)
+        self.cnt_lr = torch.zeros((hkv, self.cap_buckets), dtype=torch.int32, **z)
+        self.minlr = torch.zeros((hkv, self.cap_buckets), dtype=torch.int32, **z)
+        self.maxpos = torch.zeros((hkv, self.cap_buckets), dtype=torch.int32, **z)
+        self.sum = torch.zeros((hkv, self.cap_buckets, dl), dtype=torch.float64, **z)
+        self.cent = torch.zeros((hkv, self.cap_buckets, dl), dtype=torch.bfloat16, **z)
+        self.c = _lib.lsa_cache(hkv, 0, self.cap_units, self.cap_buckets, *[
+            t.data_ptr() for t in (self.U, self.bucket_of_unit, self.members, self.offsets,
+                                   self.cnt_lr, self.minlr, self.maxpos, self.sum, self.cent)])
+
+    @property
+    def n_tokens(self) -> int:
+        return int(self.c.n_tokens)
+
+    @property
+    def n_buckets(self) -> int:
+        nu = -(-self.n_tokens // 4)
+        return -(-nu // 128) * 64
+
+
+class Tree:
+    """Device arrays of the binary centroid tree (lsa_tree) over a cache."""
+
+    def __init__(self, cache: Cache, device="cuda"):
+        self.t = _lib.lsa_tree()
+        check(lib().lsa_tree_layout(cache.cap_buckets, ctypes.byref(self.t)), "lsa_tree_layout")
+        n, hkv = int(self.t.n_nodes), cache.hkv
+        self.sum = torch.zeros((hkv, n, 64), dtype=torch.float64, device=device)
+        self.minlr = torch.zeros((hkv, n), dtype=torch.int32, device=device)
+        self.cent = torch.zeros((hkv, n, 64), dtype=torch.bfloat16, device=device)
+        self.t.sum, self.t.minlr, self.t.cent = self.sum.data_ptr(), self.minlr.data_ptr(), self.cent.data_ptr()
+
+    @property
+    def levels(self):
+        return int(self.t.levels)
+
+    @property
+    def level_n(self):
+        return [int(self.t.level_n[i]) for i in range(self.levels)]
+
+    @property
+    def level_off(self):
+        return [int(self.t.level_off[i]) for i in range(self.levels)]
+
+
+def check_device_error():
+    """Raise if a kernel set the device-side error word (synchronous)."""
+    check(lib().lsa_check_device_error(), "device")
+
+
+def build_buckets(K: torch.Tensor, W_k: torch.Tensor, cfg: Config, cache: Cache, stream=None):
+    """lsa_build_buckets: key latents, pooling, Ward buckets, centroids."""
+    _need_cuda(K, W_k)
+    T, hkv, _ = K.shape
+    check(lib().lsa_build_buckets(_ptr(K), T, hkv, _ptr(W_k), ctypes.byref(cfg.c()),
+                                  ctypes.byref(cache.c), _stream(stream)), "lsa_build_buckets")
+    return cache
+
+
+def build_tree(cache: Cache, cfg: Config, tree: Tree | None = None, stream=None) -> Tree:
+    """lsa_build_tree: binary tree of merged centroids."""
+    tree = tree or Tree(cache)
+    check(lib().lsa_build_tree(ctypes.byref(cache.c), ctypes.byref(cfg.c()), ctypes.byref(tree.t),
+                               _stream(stream)), "lsa_build_tree")
+    return tree
+
+
+def query_latent(Q: torch.Tensor, W_q: torch.Tensor, hkv: int, cfg: Config, stream=None):
+    """lsa_query_latent: bf16 latents [nq, hkv, 64] (mean) or [nq, hq, 64] (native)."""
+    _need_cuda(Q, W_q)
+    nq, hq, _ = Q.shape
+    Y = torch.empty((nq, hkv if cfg.agg == 0 else hq, cfg.d_latent), dtype=torch.bfloat16, device=Q.device)
+    check(lib().lsa_query_latent(_ptr(Q), nq, hq, hkv, _ptr(W_q), ctypes.byref(cfg.c()), _ptr(Y),
+                                 _stream(stream)), "lsa_query_latent")
+    return Y
+
+
+def select_workspace_bytes(cfg: Config, nq: int, hq: int, cache: Cache) -> int:
+    return int(lib().lsa_select_workspace_bytes(ctypes.byref(cfg.c()), nq, hq, ctypes.byref(cache.c)))
+
+
+def select(Q: torch.Tensor, t0: int, W_q: torch.Tensor, cache: Cache, cfg: Config,
+           tree: Tree | None = None, idx: torch.Tensor | None = None, Y_out: torch.Tensor | None = None,
+           ws: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """lsa_select: index lists [nq, hkv, S + k + W] for positions t0 .. t0+nq-1."""
+    _need_cuda(Q, W_q)
+    nq, hq, _ = Q.shape
+    if idx is None:
+        idx = torch.empty((nq, cache.hkv, cfg.row), dtype=torch.int32, device=Q.device)
+    need = select_workspace_bytes(cfg, nq, hq, cache)
+    if ws is None or ws.numel() < need:
+        ws = torch.empty(max(need, 1), dtype=torch.uint8, device=Q.device)
+    check(lib().lsa_select(_ptr(Q), t0, nq, hq, _ptr(W_q), ctypes.byref(cache.c),
+                           ctypes.byref(tree.t) if tree is not None else None, ctypes.byref(cfg.c()),
+                           _ptr(idx), _ptr(Y_out), _ptr(ws), ws.numel(), _stream(stream)), "lsa_select")
+    return idx
+
+
+def sparse_attn(Q, K, V, idx, T: int | None = None, O=None, stream=None) -> torch.Tensor:
+    """lsa_sparse_attn: exact softmax attention over index lists."""
+    _need_cuda(Q, K, V, idx)
+    nq, hq, d = Q.shape
+    hkv = K.shape[1]
+    if O is None:
+        O = torch.empty((nq, hq, d), dtype=torch.bfloat16, device=Q.device)
+    T = K.shape[0] if T is None else T
+    check(lib().lsa_sparse_attn(_ptr(Q), _ptr(K), _ptr(V), _ptr(idx), nq, hq, hkv, idx.shape[2], T,
+                                _ptr(O), _stream(stream)), "lsa_sparse_attn")
+    return O
+
+
+def prefill_workspace_bytes(cfg: Config, T: int, hq: int, hkv: int, chunk: int) -> int:
+    return int(lib().lsa_prefill_workspace_bytes(ctypes.byref(cfg.c()), T, hq, hkv, chunk))
+
+
+def prefill(Q, K, V, W_k, W_q, cfg: Config, cache: Cache | None = None, tree: Tree | None = None,
+            O=None, chunk: int = 16384, ws=None, stream=None) -> torch.Tensor:
+    """lsa_prefill: a whole LSA attention layer over a T-token prompt."""
+    _need_cuda(Q, K, V, W_k, W_q)
+    T, hq, d = Q.shape
+    hkv = K.shape[1]
+    cache = cache or Cache(hkv, T, cfg, device=Q.device)
+    if cfg.mode == 1 and tree is None:
+        tree = Tree(cache, device=Q.device)
+    if O is None:
+        O = torch.empty_like(Q)
+    need = prefill_workspace_bytes(cfg, T, hq, hkv, chunk)
+    if ws is None or ws.numel() < need:
+        ws = torch.empty(need, dtype=torch.uint8, device=Q.device)
+    check(lib().lsa_prefill(_ptr(Q), _ptr(K), _ptr(V), T, hq, hkv, _ptr(W_k), _ptr(W_q),
+                            ctypes.byref(cfg.c()), ctypes.byref(cache.c),
+                            ctypes.byref(tree.t) if tree is not None else None, _ptr(O), chunk,
+                            _ptr(ws), ws.numel(), _stream(stream)), "lsa_prefill")
+    return O

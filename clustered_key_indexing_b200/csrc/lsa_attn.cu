@@ -1,0 +1,218 @@
+// lsa_attn.cu -- exact softmax attention over gathered index lists
+// [tutorial "隐空间稀疏注意力 (LSA)" (diosapp.com.cn), section 二: the attention
+// formula is unchanged, only the set of keys read changes; project card
+// "Prefrontal-AI/latent-sparse-attention", 项目介绍].
+//
+// One warp per (query, kv-head).  The G <= 8 query heads of the GQA group
+// share the index list, so the warp computes S^T = K_sel Q^T with the keys as
+// the MMA's M dimension (16 keys per tile) and the heads as N (8 columns),
+// then O^T += V_sel^T P^T.  Keys are gathered 16 at a time with 16-byte
+// cp.async copies into a per-warp 3-stage shared-memory ring (16-byte chunks
+// XOR-swizzled by row so ldmatrix reads are conflict-free); index tiles with
+// no valid entry are skipped.  Online softmax in fp32 (exp2 with the
+// log2(e)/sqrt(d) scale folded in), P rounded to bf16 for the PV product.
+// Warps are ordered kv-head-major so the warps resident at one time read one
+// head's K/V, which keeps that head's rows in L2.
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "lsa_common.cuh"
+#include "lsa_mma.cuh"
+
+namespace lsa {
+
+constexpr int kAttnWarps = 4;
+constexpr int kStages = 3;
+constexpr int kTileKeys = 16;
+constexpr int kTileBytes = kTileKeys * kD * 2;           // 4 KB per tensor
+constexpr int kStageBytes = 2 * kTileBytes;              // K + V
+constexpr int kWarpBytes = kStages * kStageBytes;        // 24 KB
+
+struct AttnArgs {
+    const uint16_t* Q;
+    const uint16_t* K;
+    const uint16_t* V;
+    const int32_t* idx;
+    int64_t nq;
+    int32_t hq, hkv, n_idx;
+    int64_t T;
+    uint16_t* O;
+    float scale_log2;
+};
+
+__device__ __forceinline__ uint32_t swz(int row, int chunk) {
+    return (uint32_t)(row * (kD * 2) + ((chunk ^ (row & 7)) << 4));
+}
+
+__global__ void __launch_bounds__(32 * kAttnWarps) attn_kernel(AttnArgs a) {
+    extern __shared__ __align__(128) uint8_t asmem[];
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    const int64_t wg = (int64_t)blockIdx.x * kAttnWarps + wid;
+    if (wg >= a.nq * a.hkv) return;
+    const int64_t g = wg / a.nq, q = wg % a.nq;  // kv-head major
+    const int G = a.hq / a.hkv;
+    const int32_t* list = a.idx + (q * a.hkv + g) * (int64_t)a.n_idx;
+    uint8_t* wbuf = asmem + wid * kWarpBytes;
+    const uint32_t wbase = smem_u32(wbuf);
+
+    // Q^T as B fragments (k = dim, n = head)
+    const int gq = lane >> 2, tq = lane & 3;
+    uint32_t qb[8][2];
+    {
+        const uint16_t* qrow = a.Q + ((q * a.hq) + g * G + (gq < G ? gq : 0)) * (int64_t)kD;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+            qb[kk][0] = gq < G ? *reinterpret_cast<const uint32_t*>(qrow + kk * 16 + 2 * tq) : 0u;
+            qb[kk][1] = gq < G ? *reinterpret_cast<const uint32_t*>(qrow + kk * 16 + 2 * tq + 8) : 0u;
+        }
+    }
+
+    const int ntiles = (a.n_idx + kTileKeys - 1) / kTileKeys;
+    const int64_t kv_stride = (int64_t)a.hkv * kD;
+    const uint16_t* Kg = a.K + g * kD;
+    const uint16_t* Vg = a.V + g * kD;
+
+    auto tile_pos = [&](int tile) -> int {
+        const int e = tile * kTileKeys + (lane & 15);
+        int p = e < a.n_idx ? __ldg(list + e) : -1;
+        if (p >= a.T) {
+            raise_device_error(kErrIndexRange);
+            p = -1;
+        }
+        return p;
+    };
+    auto issue = [&](int tile, int stage) {
+        if (tile < ntiles) {
+            const int p = tile_pos(tile);
+            const uint32_t kb = wbase + stage * kStageBytes, vb = kb + kTileBytes;
+#pragma unroll
+            for (int m = 0; m < 8; ++m) {
+                const int r = 2 * m + (lane >> 4), part = lane & 15;
+                const int pr = __shfl_sync(0xffffffffu, p, r);
+                const int64_t off = (pr >= 0 ? (int64_t)pr : 0) * kv_stride + part * 8;
+                cp_async_16(kb + swz(r, part), Kg + off, pr >= 0 ? 16 : 0);
+                cp_async_16(vb + swz(r, part), Vg + off, pr >= 0 ? 16 : 0);
+            }
+        }
+        cp_async_commit();
+    };
+
+    float o[8][4];
+#pragma unroll
+    for (int mt = 0; mt < 8; ++mt)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) o[mt][i] = 0.f;
+    float m_run[2] = {-CUDART_INF_F, -CUDART_INF_F};
+    float l_run[2] = {0.f, 0.f};
+
+#pragma unroll
+    for (int s = 0; s < kStages - 1; ++s) issue(s, s);
+
+    for (int i = 0; i < ntiles; ++i) {
+        issue(i + kStages - 1, (i + kStages - 1) % kStages);
+        const int p = tile_pos(i);
+        const unsigned vmask = __ballot_sync(0xffffffffu, p >= 0) & 0xFFFFu;
+        cp_async_wait<kStages - 1>();
+        __syncwarp();
+        if (vmask != 0) {
+            const int stage = i % kStages;
+            const uint32_t kb = wbase + stage * kStageBytes, vb = kb + kTileBytes;
+            // S^T (16 keys x 8 heads)
+            float s[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+                uint32_t af[4];
+                const int row = ((lane >> 3) & 1) * 8 + (lane & 7);
+                const int chunk = 2 * kk + (lane >> 4);
+                ldsm_x4(af, kb + swz(row, chunk));
+                mma_16816(s, af, qb[kk][0], qb[kk][1]);
+            }
+            const bool v0 = (vmask >> gq) & 1u, v1 = (vmask >> (gq + 8)) & 1u;
+            s[0] = v0 ? s[0] * a.scale_log2 : -CUDART_INF_F;
+            s[1] = v0 ? s[1] * a.scale_log2 : -CUDART_INF_F;
+            s[2] = v1 ? s[2] * a.scale_log2 : -CUDART_INF_F;
+            s[3] = v1 ? s[3] * a.scale_log2 : -CUDART_INF_F;
+            float mx0 = fmaxf(s[0], s[2]), mx1 = fmaxf(s[1], s[3]);
+#pragma unroll
+            for (int off = 4; off < 32; off <<= 1) {
+                mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
+                mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
+            }
+            const float mn0 = fmaxf(m_run[0], mx0), mn1 = fmaxf(m_run[1], mx1);
+            const float al0 = exp2f(m_run[0] - mn0), al1 = exp2f(m_run[1] - mn1);
+            m_run[0] = mn0;
+            m_run[1] = mn1;
+            const float p0 = exp2f(s[0] - mn0), p1 = exp2f(s[1] - mn1);
+            const float p2 = exp2f(s[2] - mn0), p3 = exp2f(s[3] - mn1);
+            l_run[0] = l_run[0] * al0 + (p0 + p2);
+            l_run[1] = l_run[1] * al1 + (p1 + p3);
+#pragma unroll
+            for (int mt = 0; mt < 8; ++mt) {
+                o[mt][0] *= al0; o[mt][1] *= al1; o[mt][2] *= al0; o[mt][3] *= al1;
+            }
+            // P^T as B fragments: lane (head gq, tq) needs keys 2tq, 2tq+1, 2tq+8, 2tq+9
+            const uint32_t pk_lo = pack_bf16x2(p0, p1), pk_hi = pack_bf16x2(p2, p3);
+            const int src1 = (2 * tq) * 4 + (gq >> 1), src2 = (2 * tq + 1) * 4 + (gq >> 1);
+            const uint32_t x1 = __shfl_sync(0xffffffffu, pk_lo, src1);
+            const uint32_t x2 = __shfl_sync(0xffffffffu, pk_lo, src2);
+            const uint32_t y1 = __shfl_sync(0xffffffffu, pk_hi, src1);
+            const uint32_t y2 = __shfl_sync(0xffffffffu, pk_hi, src2);
+            const uint32_t sel = (gq & 1) ? 0x7632u : 0x5410u;
+            uint32_t b0 = __byte_perm(x1, x2, sel), b1 = __byte_perm(y1, y2, sel);
+            if (gq >= G) { b0 = 0u; b1 = 0u; }
+#pragma unroll
+            for (int mt = 0; mt < 8; ++mt) {
+                uint32_t af[4];
+                const int row = (lane >> 4) * 8 + (lane & 7);
+                const int chunk = 2 * mt + ((lane >> 3) & 1);
+                ldsm_x4_t(af, vb + swz(row, chunk));
+                mma_16816(o[mt], af, b0, b1);
+            }
+        }
+        __syncwarp();
+    }
+    cp_async_wait<0>();
+    __syncwarp();
+
+    // normalise and stage O (heads x dims, bf16) for a coalesced store
+#pragma unroll
+    for (int off = 4; off < 32; off <<= 1) {
+        l_run[0] += __shfl_xor_sync(0xffffffffu, l_run[0], off);
+        l_run[1] += __shfl_xor_sync(0xffffffffu, l_run[1], off);
+    }
+    const float inv0 = l_run[0] > 0.f ? 1.f / l_run[0] : 0.f;
+    const float inv1 = l_run[1] > 0.f ? 1.f / l_run[1] : 0.f;
+    uint16_t* os = reinterpret_cast<uint16_t*>(wbuf);  // [8][128]
+#pragma unroll
+    for (int mt = 0; mt < 8; ++mt) {
+        const int d0 = mt * 16 + gq;
+        const uint32_t lo = pack_bf16x2(o[mt][0] * inv0, o[mt][1] * inv1);
+        const uint32_t hi = pack_bf16x2(o[mt][2] * inv0, o[mt][3] * inv1);
+        os[(2 * tq) * kD + d0] = (uint16_t)(lo & 0xFFFF);
+        os[(2 * tq + 1) * kD + d0] = (uint16_t)(lo >> 16);
+        os[(2 * tq) * kD + d0 + 8] = (uint16_t)(hi & 0xFFFF);
+        os[(2 * tq + 1) * kD + d0 + 8] = (uint16_t)(hi >> 16);
+    }
+    __syncwarp();
+    uint16_t* orow = a.O + (q * a.hq + g * G) * (int64_t)kD;
+    const int nchunk = G * kD / 8;  // 16-byte chunks
+    for (int c = lane; c < nchunk; c += 32)
+        reinterpret_cast<uint4*>(orow)[c] = reinterpret_cast<const uint4*>(os)[c];
+}
+
+lsa_status launch_attn(const uint16_t* Q, const uint16_t* K, const uint16_t* V, const int32_t* idx,
+                       int64_t nq, int32_t hq, int32_t hkv, int32_t n_idx, int64_t T, uint16_t* O,
+                       cudaStream_t st) {
+    if (nq <= 0) return LSA_OK;
+    AttnArgs a{};
+    a.Q = Q; a.K = K; a.V = V; a.idx = idx; a.nq = nq; a.hq = hq; a.hkv = hkv; a.n_idx = n_idx;
+    a.T = T; a.O = O;
+    a.scale_log2 = 1.4426950408889634f / sqrtf((float)kD);
+    const size_t smem = (size_t)kAttnWarps * kWarpBytes;
+    cudaFuncSetAttribute(attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    const int64_t warps = nq * hkv;
+    attn_kernel<<<(unsigned)ceil_div<int64_t>(warps, kAttnWarps), 32 * kAttnWarps, smem, st>>>(a);
+    return check_launch("attn_kernel");
+}
+
+}  // namespace lsa

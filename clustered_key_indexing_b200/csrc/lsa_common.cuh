@@ -1,0 +1,93 @@
+// lsa_common.cuh -- shared device helpers of the LSA CUDA library (sm_100a).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <math_constants.h>
+#include <stdint.h>
+
+#include "lsa.h"
+
+namespace lsa {
+
+// Geometry fixed by the LSA pages (essay "《卡片柜》", ch. 2): 64-d latent,
+// 4 keys pooled per unit, 512-key cluster blocks (128 units) split into
+// buckets of mean 8 keys (64 per block) and at most 16 keys (4 units).
+constexpr int kD = 128;            // d_head
+constexpr int kDL = 64;            // d_latent
+constexpr int kPool = 4;
+constexpr int kBlockKeys = 512;
+constexpr int kUnitsPerBlock = 128;
+constexpr int kBucketsPerBlock = 64;
+constexpr int kMaxUnits = 4;
+constexpr int kIMax = 2147483647;
+
+// Device-side error word (one per device; the library is one translation
+// unit, lsa_lib.cu): kernels that detect an
+// inconsistency store a code here instead of trapping; the host reads it
+// with lsa_check_device_error().
+__device__ int g_lsa_device_error = 0;
+
+enum DeviceError : int {
+    kErrNone = 0,
+    kErrWardInfeasible = 1,   // no eligible pair before the target count
+    kErrSelectOverflow = 2,   // candidate list exceeded its capacity
+    kErrIndexRange = 3,       // an index list entry was >= T
+};
+
+__device__ __forceinline__ void raise_device_error(int code) {
+    atomicCAS(&g_lsa_device_error, 0, code);
+}
+
+__device__ __forceinline__ float bf16_to_f32(uint16_t h) {
+    return __uint_as_float(((uint32_t)h) << 16);
+}
+
+__device__ __forceinline__ double bf16_to_f64(uint16_t h) {
+    return (double)bf16_to_f32(h);
+}
+
+// Round a double directly to bf16 (8 significant bits), ties to even: add
+// half an ulp minus one (plus the kept lsb) to the bit pattern and truncate
+// the 45 dropped mantissa bits; tiny magnitudes use bf16's fixed subnormal
+// spacing 2^-133.
+__device__ __forceinline__ uint16_t f64_to_bf16_rne(double x) {
+    if (isnan(x)) return 0x7FC0;
+    const uint16_t sign = signbit(x) ? 0x8000 : 0;
+    const double a = fabs(x);
+    if (a == 0.0) return sign;
+    if (isinf(a)) return (uint16_t)(sign | 0x7F80);
+    const unsigned long long b = (unsigned long long)__double_as_longlong(a);
+    const int e = (int)(b >> 52) - 1023;
+    double y;
+    if (e >= -126) {
+        unsigned long long r = b + ((1ull << 44) - 1ull) + ((b >> 45) & 1ull);
+        r &= ~((1ull << 45) - 1ull);
+        y = __longlong_as_double((long long)r);
+    } else {
+        y = rint(a * 0x1p133) * 0x1p-133;  // exact power-of-two scalings
+    }
+    const float f = __double2float_rn(y);  // exact, or inf past the bf16 range
+    return (uint16_t)(sign | (uint16_t)(__float_as_uint(f) >> 16));
+}
+
+// Exact score of two bf16 latents: every product of two bf16 values is exact
+// in fp64; the sum runs in ascending index order.
+__device__ __forceinline__ double dot_bf16_exact(const uint16_t* __restrict__ y,
+                                                 const uint16_t* __restrict__ c) {
+    double s = 0.0;
+#pragma unroll 8
+    for (int i = 0; i < kDL; ++i) s = fma(bf16_to_f64(y[i]), bf16_to_f64(c[i]), s);
+    return s;
+}
+
+template <typename T>
+__host__ __device__ __forceinline__ T ceil_div(T a, T b) { return (a + b - 1) / b; }
+
+}  // namespace lsa
+
+// Host-side launch helpers (defined in lsa_api.cu).
+namespace lsa {
+lsa_status set_error(lsa_status st, const char* fmt, ...);
+lsa_status check_launch(const char* what);
+int num_sms();
+}  // namespace lsa

@@ -1,0 +1,6 @@
+// lsa_lib.cu -- single translation unit of liblsa.so (one copy of the
+// device-side error word, no separate device link step).
+#include "lsa_build.cu"
+#include "lsa_select.cu"
+#include "lsa_attn.cu"
+#include "lsa_api.cu"

@@ -1,0 +1,245 @@
+/*
+ * lsa.h -- C ABI of the B200 (sm_100a) Latent Sparse Attention library
+ * (liblsa.so).
+ *
+ * The library implements the data-parallel path of "Latent Sparse Attention:
+ * Towards Subquadratic Ultra-Long Context Attention" (arXiv:2610.42147) as the
+ * LSA web pages describe it:
+ *   (1) key build -- every key is projected by W_k into a 64-d latent, L2
+ *       normalised; every 4 consecutive keys are pooled; every 512-key cluster
+ *       block is Ward-clustered into buckets (mean 8 keys, max 16) whose
+ *       normalised centroids form the bucket cache  [essay "《卡片柜》——当注意力
+ *       学会先查目录再翻书" (zhichai.net), ch. 2 "卡片柜的灵感——语义聚类"];
+ *   (2) query scoring -- the query is projected by W_q into the same space and
+ *       scored against every centroid (flat search), or taken down a complete
+ *       binary tree of merged centroids by beam search (tree search); the top
+ *       buckets are expanded until k long-range keys are filled
+ *       [same essay, ch. 3 "查询来了怎么办" and ch. 4 "树——当卡片柜变成楼层图"];
+ *       the native variant scores a bucket by the max over the group's heads
+ *       [same essay, ch. 5 "两种生产方式"];
+ *   (3) assembly of sinks + long-range keys + local window under a causal
+ *       mask [ch. 3];
+ *   (4) exact softmax attention over that index set [tutorial "隐空间稀疏注意力
+ *       (LSA)" (diosapp.com.cn), section 二 "LSA 怎么工作"].
+ *
+ * Conventions (all entry points):
+ *   - Every tensor argument is a DEVICE pointer owned by the caller, unless
+ *     stated otherwise.  The library allocates no device memory and keeps no
+ *     state between calls; scratch space is passed in as `ws`/`ws_bytes`.
+ *   - bf16 tensors are passed as uint16_t bit patterns.  Layouts are
+ *     row-major; K/V are token-major [T, hkv, d_head]; Q is [nq, hq, d_head]
+ *     with query head h reading kv-head h / (hq / hkv).
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Calls are
+ *     asynchronous: a return of LSA_OK means the work was enqueued.
+ *   - Every call returns an lsa_status; on failure nothing is enqueued and
+ *     lsa_last_error() (thread-local) describes the reason.  Errors found by
+ *     kernels at run time (LSA_EDEVICE) are reported through
+ *     lsa_check_device_error().
+ *   - Supported geometry: d_head 128, d_latent 64, pool 4, block 512,
+ *     bucket_mean 8, bucket_max 16, hq / hkv in {1,2,4,8}; other values give
+ *     LSA_EUNSUPPORTED.
+ */
+#ifndef LSA_H_
+#define LSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef int32_t lsa_status;
+#define LSA_OK            0
+#define LSA_EINVAL        1  /* bad argument (null pointer, size, range)     */
+#define LSA_EUNSUPPORTED  2  /* valid but not implemented on this library    */
+#define LSA_ECUDA         3  /* a CUDA runtime call failed                   */
+#define LSA_ENOSPACE      4  /* workspace or capacity too small              */
+#define LSA_EDEVICE       5  /* a kernel raised its device-side error word   */
+
+/* Method parameters; names follow the pages' notation. */
+typedef struct lsa_cfg {
+    int32_t d_head;      /* key/query width (128)                                 */
+    int32_t d_latent;    /* latent width (64)                 [ch. 2]             */
+    int32_t pool;        /* consecutive keys pooled per unit (4)  [ch. 2]         */
+    int32_t block;       /* keys per cluster block (512)      [ch. 2]             */
+    int32_t bucket_mean; /* mean keys per bucket (8)          [ch. 2]             */
+    int32_t bucket_max;  /* max keys per bucket (16)          [ch. 2]             */
+    int32_t k;           /* long-range keys per query         [ch. 3]             */
+    int32_t sinks;       /* S: keys 0..S-1 always attended    [ch. 3]             */
+    int32_t window;      /* W: keys t-W+1..t always attended  [ch. 3], >= 1       */
+    int32_t beam;        /* beam width of tree search, 1..8   [ch. 4]             */
+    int32_t mode;        /* 0 flat search, 1 tree search      [ch. 3, ch. 4]      */
+    int32_t agg;         /* 0 group-mean query latent, 1 max over heads (native)  */
+} lsa_cfg;
+
+/*
+ * Bucket cache of one layer (all kv-heads), caller-owned device arrays.
+ * Sizes per head: cap_units >= ceil(n_tokens / pool) units and cap_buckets =
+ * (block / bucket_mean) * ceil(cap_units / (block / pool)) bucket slots.
+ * Bucket b of block beta is slot beta*64 + local; local ids are ordered by the
+ * bucket's lowest unit; unused slots are empty (cnt_lr 0, minlr INT32_MAX,
+ * maxpos -1, zero sum/centroid).
+ */
+typedef struct lsa_cache {
+    int32_t   hkv;
+    int64_t   n_tokens;        /* tokens clustered (set by the build calls)       */
+    int64_t   cap_units;       /* allocated units per head                        */
+    int64_t   cap_buckets;     /* allocated bucket slots per head                 */
+    double*   U;               /* [hkv, cap_units, d_latent] pooled unit latents  */
+    int32_t*  bucket_of_unit;  /* [hkv, cap_units]                                */
+    int32_t*  members;         /* [hkv, cap_units] unit ids grouped by bucket     */
+    int32_t*  offsets;         /* [hkv, cap_buckets + 1] CSR into members         */
+    int32_t*  cnt_lr;          /* [hkv, cap_buckets] keys at positions >= sinks   */
+    int32_t*  minlr;           /* [hkv, cap_buckets] smallest key >= sinks        */
+    int32_t*  maxpos;          /* [hkv, cap_buckets] largest key                  */
+    double*   sum;             /* [hkv, cap_buckets, d_latent] fp64 unit sums     */
+    uint16_t* cent;            /* [hkv, cap_buckets, d_latent] bf16 centroids     */
+} lsa_cache;
+
+#define LSA_MAX_LEVELS 48
+
+/*
+ * Complete binary tree over the bucket slots of a cache [ch. 4]: level 0 =
+ * the cap_buckets slots, level l+1 has ceil(n_l / 2) nodes, node i merging
+ * children 2i and 2i+1.  lsa_tree_layout() fills levels/level_n/level_off/
+ * n_nodes; the caller then allocates the arrays (per head n_nodes entries).
+ */
+typedef struct lsa_tree {
+    int32_t   levels;
+    int64_t   level_n[LSA_MAX_LEVELS];
+    int64_t   level_off[LSA_MAX_LEVELS];
+    int64_t   n_nodes;         /* nodes per head                                   */
+    double*   sum;             /* [hkv, n_nodes, d_latent]                         */
+    int32_t*  minlr;           /* [hkv, n_nodes]                                   */
+    uint16_t* cent;            /* [hkv, n_nodes, d_latent] bf16                    */
+} lsa_tree;
+
+/* ---------------------------------------------------------------- misc */
+
+/* Human-readable reason of the last failure on this thread ("" if none). */
+const char* lsa_last_error(void);
+/* Library version string. */
+const char* lsa_version(void);
+/* Fill *cfg with the pages' parameters (d 128, latent 64, pool 4, block 512,
+ * bucket mean 8 / max 16, k 2048, S 4, W 1024, beam 2, flat, mean). */
+lsa_status lsa_cfg_default(lsa_cfg* cfg);
+/* LSA_OK if *cfg is supported by this library, else the reason. */
+lsa_status lsa_cfg_check(const lsa_cfg* cfg);
+/* Units ceil(n_tokens / pool) and bucket slots for a capacity of n_tokens. */
+int64_t lsa_cache_units(const lsa_cfg* cfg, int64_t n_tokens);
+int64_t lsa_cache_buckets(const lsa_cfg* cfg, int64_t n_tokens);
+/* Fill the tree geometry for `n_buckets` leaf slots (host-only, no CUDA). */
+lsa_status lsa_tree_layout(int64_t n_buckets, lsa_tree* tree);
+/* Kernels this library has launched in this process (host-side counter,
+ * for diagnostics and launch accounting). */
+int64_t lsa_launch_count(void);
+/* Read back and clear the device-side error word of the current device:
+ * LSA_OK, or LSA_EDEVICE with a description in lsa_last_error(). Synchronous. */
+lsa_status lsa_check_device_error(void);
+
+/* ------------------------------------------------------------ (1) build */
+
+/*
+ * lsa_build_buckets -- key build [ch. 2].
+ * K [T, hkv, d_head] bf16, W_k [d_head, d_latent] fp32 row-major (one matrix
+ * per layer, shared by all heads [ch. 5]).  For every head: pooled unit
+ * latents u_j = mean of normalise(k W_k) over keys 4j..4j+3 (fp64, not
+ * re-normalised) -> cache->U; every 128-unit block (a 512-key cluster block;
+ * a ragged last block of n units gets ceil(n/2) buckets) is Ward-clustered:
+ * greedy least-Delta-SSE merges of units, clusters capped at 4 units (16
+ * keys), ties to the lowest (id_A, id_B), until 64 clusters remain.  Fills
+ * every cache array for tokens [0, T) and sets cache->n_tokens = T.
+ * Requires cache->cap_units >= ceil(T/4) (else LSA_ENOSPACE).
+ */
+lsa_status lsa_build_buckets(const uint16_t* K, int64_t T, int32_t hkv,
+                             const float* W_k, const lsa_cfg* cfg,
+                             lsa_cache* cache, void* stream);
+
+/*
+ * lsa_build_tree -- complete binary tree over the cache's bucket slots
+ * [ch. 4]: node sum = sum of its two children (fp64), minlr = min of the
+ * children, centroid = bf16(sum / |sum|) (the normalised mean of every key
+ * below it).  `tree` must carry lsa_tree_layout(cache->cap_buckets, ...).
+ */
+lsa_status lsa_build_tree(const lsa_cache* cache, const lsa_cfg* cfg,
+                          lsa_tree* tree, void* stream);
+
+/* ------------------------------------------------------ (2)+(3) select */
+
+/*
+ * lsa_query_latent -- query latents [tutorial section 二; ch. 5]:
+ * y_{t,h} = normalise(q_{t,h} W_q) in fp64; agg 0 writes the group mean
+ * rounded to bf16, Y [nq, hkv, d_latent]; agg 1 writes every head,
+ * Y [nq, hq, d_latent].
+ */
+lsa_status lsa_query_latent(const uint16_t* Q, int64_t nq, int32_t hq,
+                            int32_t hkv, const float* W_q, const lsa_cfg* cfg,
+                            uint16_t* Y, void* stream);
+
+/* Workspace bytes lsa_select needs for nq queries over `cache`. */
+size_t lsa_select_workspace_bytes(const lsa_cfg* cfg, int64_t nq, int32_t hq,
+                                  const lsa_cache* cache);
+
+/*
+ * lsa_select -- long-range key selection and index assembly [ch. 3, ch. 4].
+ * Queries are the positions t = t0 .. t0+nq-1 with rows Q [nq, hq, d_head].
+ * A bucket is eligible for t iff minlr <= t - W; its weight is its number of
+ * keys in [S, t - W].  Flat (cfg->mode 0): eligible buckets ranked by exact
+ * score (desc; lower bucket id first on ties) are expanded until exactly k
+ * keys are taken, the last bucket truncated to its lowest keys.  Tree
+ * (cfg->mode 1, `tree` built): beam descent from the root to level
+ * L* = min{l : beam * bucket_mean * 2^l >= k}, keeping the best `beam`
+ * eligible children per level, then the same fill over the buckets below the
+ * final beam.  Output idx [nq, hkv, S + k + W] int32:
+ *   [0,S) sinks 0..min(S,t+1)-1 | [S,S+k) long-range keys, chosen buckets in
+ *   ascending id, keys ascending | [S+k, S+k+W) window max(S,t-W+1)..t;
+ *   every part padded with -1.
+ * Y_out (optional, may be NULL) receives the bf16 query latents.
+ * ws / ws_bytes: scratch of at least lsa_select_workspace_bytes().
+ */
+lsa_status lsa_select(const uint16_t* Q, int64_t t0, int64_t nq, int32_t hq,
+                      const float* W_q, const lsa_cache* cache,
+                      const lsa_tree* tree, const lsa_cfg* cfg, int32_t* idx,
+                      uint16_t* Y_out, void* ws, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------- (4) attention */
+
+/*
+ * lsa_sparse_attn -- exact softmax attention over index lists [tutorial
+ * section 二]: O_{q,h} = sum_j softmax_j(q_{q,h} . k_j / sqrt(d_head)) v_j
+ * over the entries j >= 0 of idx[q, h / G, 0:n_idx] (G = hq / hkv; the G
+ * query heads of a group share the list).  Q [nq, hq, d_head], K/V
+ * [T, hkv, d_head] bf16, idx [nq, hkv, n_idx] int32 (-1 = padding; entries
+ * must be < T), O [nq, hq, d_head] bf16.  fp32 accumulation; a list with no
+ * valid entry gives O = 0.
+ */
+lsa_status lsa_sparse_attn(const uint16_t* Q, const uint16_t* K,
+                           const uint16_t* V, const int32_t* idx, int64_t nq,
+                           int32_t hq, int32_t hkv, int32_t n_idx, int64_t T,
+                           uint16_t* O, void* stream);
+
+/* --------------------------------------------------- whole-layer prefill */
+
+/* Workspace bytes lsa_prefill needs (T tokens, queries processed in chunks
+ * of `chunk` positions). */
+size_t lsa_prefill_workspace_bytes(const lsa_cfg* cfg, int64_t T, int32_t hq,
+                                   int32_t hkv, int64_t chunk);
+
+/*
+ * lsa_prefill -- one LSA attention layer over a prompt of T tokens:
+ * lsa_build_buckets, lsa_build_tree (tree mode), then per chunk of `chunk`
+ * query positions lsa_select + lsa_sparse_attn.  Q [T, hq, d], K/V
+ * [T, hkv, d], O [T, hq, d] bf16; cache/tree as for the calls above.
+ */
+lsa_status lsa_prefill(const uint16_t* Q, const uint16_t* K, const uint16_t* V,
+                       int64_t T, int32_t hq, int32_t hkv, const float* W_k,
+                       const float* W_q, const lsa_cfg* cfg, lsa_cache* cache,
+                       lsa_tree* tree, uint16_t* O, int64_t chunk, void* ws,
+                       size_t ws_bytes, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LSA_H_ */

@@ -1,0 +1,83 @@
+"""C ABI checks that need no GPU: liblsa.so loads, exports every function
+include/lsa.h declares, and its host-only calls and argument validation
+behave as documented (no compute call is made here)."""
+import ctypes
+import os
+import subprocess
+
+import pytest
+
+from clustered_key_indexing_b200 import _lib
+from clustered_key_indexing_b200._lib import (LSA_EINVAL, LSA_EUNSUPPORTED, LSA_OK, lsa_cache,
+                                              lsa_cfg, lsa_tree)
+
+
+@pytest.fixture(scope="module")
+def L():
+    from clustered_key_indexing_b200.build import build
+    build()
+    return _lib.lib()
+
+
+def test_every_declared_symbol_is_exported(L):
+    names = _lib.exported_names()
+    assert len(names) >= 15
+    out = subprocess.run(["nm", "-D", "--defined-only", _lib.SO], capture_output=True, text=True).stdout
+    exported = {line.split()[-1] for line in out.splitlines() if " T " in line}
+    missing = [n for n in names if n not in exported]
+    assert not missing, missing
+    for n in names:
+        getattr(L, n)
+
+
+def test_defaults_and_checks(L):
+    c = lsa_cfg()
+    assert L.lsa_cfg_default(ctypes.byref(c)) == LSA_OK
+    assert (c.d_head, c.d_latent, c.pool, c.block, c.bucket_mean, c.bucket_max) == (128, 64, 4, 512, 8, 16)
+    assert (c.k, c.sinks, c.window, c.beam, c.mode, c.agg) == (2048, 4, 1024, 2, 0, 0)
+    assert L.lsa_cfg_check(ctypes.byref(c)) == LSA_OK
+    bad = lsa_cfg.from_buffer_copy(c)
+    bad.d_latent = 32
+    assert L.lsa_cfg_check(ctypes.byref(bad)) == LSA_EUNSUPPORTED
+    assert b"d_latent" in L.lsa_last_error()
+    bad = lsa_cfg.from_buffer_copy(c)
+    bad.window = 0
+    assert L.lsa_cfg_check(ctypes.byref(bad)) == LSA_EINVAL
+    bad = lsa_cfg.from_buffer_copy(c)
+    bad.mode = 3
+    assert L.lsa_cfg_check(ctypes.byref(bad)) == LSA_EINVAL
+    assert L.lsa_cfg_check(None) == LSA_EINVAL
+
+
+def test_sizes_and_tree_layout(L):
+    c = lsa_cfg()
+    L.lsa_cfg_default(ctypes.byref(c))
+    assert L.lsa_cache_units(ctypes.byref(c), 4097) == 1025
+    assert L.lsa_cache_buckets(ctypes.byref(c), 4096) == 512
+    assert L.lsa_cache_buckets(ctypes.byref(c), 4097) == 576
+    assert L.lsa_cache_buckets(ctypes.byref(c), 1 << 20) == 131072
+    t = lsa_tree()
+    assert L.lsa_tree_layout(131072, ctypes.byref(t)) == LSA_OK
+    assert t.levels == 18 and t.level_n[17] == 1 and t.n_nodes == 2 * 131072 - 1
+    assert L.lsa_tree_layout(5, ctypes.byref(t)) == LSA_OK
+    assert [t.level_n[i] for i in range(t.levels)] == [5, 3, 2, 1]
+    assert [t.level_off[i] for i in range(t.levels)] == [0, 5, 8, 10]
+    assert L.lsa_tree_layout(0, ctypes.byref(t)) == LSA_EINVAL
+    cache = lsa_cache(8, 131072, 32768, 16384, *([16] * 9))
+    assert L.lsa_select_workspace_bytes(ctypes.byref(c), 131072, 32, ctypes.byref(cache)) > 0
+    assert L.lsa_prefill_workspace_bytes(ctypes.byref(c), 131072, 32, 8, 16384) > 0
+
+
+def test_compute_calls_reject_bad_arguments_before_any_launch(L):
+    c = lsa_cfg()
+    L.lsa_cfg_default(ctypes.byref(c))
+    # NULL cache / NULL tensors / bad head ratio: refused on the host
+    assert L.lsa_build_buckets(None, 16, 1, None, ctypes.byref(c), None, None) == LSA_EINVAL
+    cache = lsa_cache(1, 0, 4, 64, *([0] * 9))
+    assert L.lsa_build_buckets(None, 16, 1, None, ctypes.byref(c), ctypes.byref(cache), None) == LSA_EINVAL
+    assert L.lsa_sparse_attn(None, None, None, None, 1, 3, 2, 8, 16, None, None) == LSA_EINVAL
+    assert L.lsa_sparse_attn(None, None, None, None, 1, 48, 4, 8, 16, None, None) == LSA_EUNSUPPORTED
+    assert L.lsa_query_latent(None, 1, 4, 1, None, ctypes.byref(c), None, None) == LSA_EINVAL
+    assert L.lsa_select(None, 0, 1, 4, None, None, None, ctypes.byref(c), None, None, None, 0, None) == LSA_EINVAL
+    assert L.lsa_prefill(None, None, None, 16, 4, 1, None, None, ctypes.byref(c), None, None, None, 0,
+                         None, 0, None) == LSA_EINVAL

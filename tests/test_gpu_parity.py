@@ -1,0 +1,226 @@
+"""GPU parity: every stage of the CUDA path (through the C ABI) against the
+CPU oracle on the same seeded inputs.
+
+Bar: bucket cache, tree, query latents and index lists bit-exact (the
+library takes every quantising or ranking decision on the same fp64 values
+as the oracle); attention output within max |err| 2e-2 and mean |err| 2e-3
+of the fp64 oracle (bf16 inputs/outputs, fp32 accumulation).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from gpu_util import bits, cache_arrays, oracle_cfg, to_dev, to_dev_bf16
+
+pytestmark = pytest.mark.gpu
+
+CACHE_KEYS = ("bucket_of_unit", "members", "offsets", "cnt_lr", "minlr", "maxpos", "cent")
+ATOL_MAX, ATOL_MEAN = 2e-2, 2e-3
+
+
+@pytest.fixture(scope="module")
+def lsa():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import clustered_key_indexing_b200 as m
+    return m
+
+
+def _build_both(lsa, name, T, cfg, seed=0):
+    inp = synth.layer_inputs(name, seed=seed, T=T)
+    hkv = inp["K"].shape[1]
+    K = to_dev_bf16(inp["K"])
+    cache = lsa.Cache(hkv, T, cfg)
+    lsa.build_buckets(K, to_dev(inp["Wk"]), cfg, cache)
+    torch.cuda.synchronize()
+    lsa.check_device_error()
+    U = oracle.key_latent_pool(inp["K"], inp["Wk"], 4)
+    oc = oracle.build_cache(U, T, oracle_cfg(cfg))
+    return inp, cache, U, oc
+
+
+def _assert_cache_equal(cache, U, oc):
+    g = cache_arrays(cache, oc["NB"])
+    assert np.array_equal(g["U"].view(np.uint64), U.view(np.uint64)), "pooled latents differ"
+    assert np.array_equal(g["sum"].view(np.uint64), oc["sum"].view(np.uint64)), "bucket sums differ"
+    for key in CACHE_KEYS:
+        assert np.array_equal(g[key], oc[key]), key
+
+
+@pytest.mark.parametrize("T", [4096, 4099, 1000, 513, 512, 7, 4, 1])
+def test_build_bit_exact(lsa, T):
+    cfg = lsa.Config(k=512, sinks=4, window=256)
+    _, cache, U, oc = _build_both(lsa, "prefill-4k", T, cfg)
+    _assert_cache_equal(cache, U, oc)
+
+
+def test_build_bit_exact_8_heads(lsa):
+    cfg = lsa.Config(k=2048, sinks=4, window=1024)
+    _, cache, U, oc = _build_both(lsa, "prefill-128k", 8192 + 100, cfg)
+    _assert_cache_equal(cache, U, oc)
+
+
+def test_build_degenerate_keys(lsa):
+    """All-zero keys: zero latents, every Delta 0, ties broken by index."""
+    cfg = lsa.Config(k=512, sinks=4, window=256)
+    T = 1024
+    K = np.zeros((T, 1, 128), np.uint16)
+    Wk, _ = synth.projections(0)
+    cache = lsa.Cache(1, T, cfg)
+    lsa.build_buckets(to_dev_bf16(K), to_dev(Wk), cfg, cache)
+    torch.cuda.synchronize()
+    lsa.check_device_error()
+    U = oracle.key_latent_pool(K, Wk, 4)
+    oc = oracle.build_cache(U, T, oracle_cfg(cfg))
+    _assert_cache_equal(cache, U, oc)
+
+
+@pytest.mark.parametrize("agg", [0, 1])
+def test_query_latent_bit_exact(lsa, agg):
+    cfg = lsa.Config(agg=agg)
+    inp = synth.layer_inputs("prefill-128k", T=300)
+    Y = lsa.query_latent(to_dev_bf16(inp["Q"]), to_dev(inp["Wq"]), 8, cfg)
+    torch.cuda.synchronize()
+    want = oracle.query_latent(inp["Q"], inp["Wq"], 8, agg)
+    assert np.array_equal(bits(Y), want)
+
+
+def test_tree_bit_exact(lsa):
+    cfg = lsa.Config(k=512, sinks=4, window=256, mode=1)
+    _, cache, U, oc = _build_both(lsa, "prefill-4k", 4096 + 600, cfg)
+    tree = lsa.build_tree(cache, cfg)
+    torch.cuda.synchronize()
+    ot = oracle.build_tree(oc)
+    # the library's tree spans the capacity; it equals the oracle's on every
+    # level where the oracle has nodes
+    for lvl, (n, off) in enumerate(zip(ot["level_n"], ot["level_off"])):
+        goff = tree.level_off[lvl]
+        assert np.array_equal(tree.minlr[:, goff:goff + n].cpu().numpy(), ot["minlr"][:, off:off + n])
+        assert np.array_equal(bits(tree.cent[:, goff:goff + n]), ot["cent"][:, off:off + n])
+        assert np.array_equal(tree.sum[:, goff:goff + n].cpu().numpy().view(np.uint64),
+                              ot["sum"][:, off:off + n].view(np.uint64))
+
+
+def _select_both(lsa, name, T, cfg, tpos=None, seed=0):
+    inp, cache, U, oc = _build_both(lsa, name, T, cfg, seed=seed)
+    tree = lsa.build_tree(cache, cfg) if cfg.mode == 1 else None
+    Q = to_dev_bf16(inp["Q"])
+    Wq = to_dev(inp["Wq"])
+    idx = lsa.select(Q, 0, Wq, cache, cfg, tree=tree)
+    torch.cuda.synchronize()
+    lsa.check_device_error()
+    hkv, hq = inp["K"].shape[1], inp["Q"].shape[1]
+    if tpos is None:
+        tpos = np.arange(T)
+    Y = oracle.query_latent(inp["Q"][tpos], inp["Wq"], hkv, cfg.agg)
+    oidx, mg, nc = oracle.select(oc, Y, tpos, oracle_cfg(cfg), G=hq // hkv)
+    return inp, idx.cpu().numpy()[tpos], oidx, mg
+
+
+@pytest.mark.parametrize("mode,agg", [(0, 0), (0, 1), (1, 0), (1, 1)])
+def test_select_bit_exact_4k(lsa, mode, agg):
+    cfg = lsa.Config(k=512, sinks=4, window=256, mode=mode, agg=agg)
+    _, g, o, _ = _select_both(lsa, "prefill-4k", 4096, cfg)
+    bad = np.where((g != o).any(axis=(1, 2)))[0]
+    assert bad.size == 0, f"{bad.size} rows differ, first t={bad[:5]}"
+
+
+@pytest.mark.parametrize("T,k,W", [(1000, 64, 8), (777, 4096, 16), (130, 512, 1), (5, 16, 2)])
+def test_select_edge_cases(lsa, T, k, W):
+    """Ragged lengths, k above every eligible key (take-all), window 1,
+    prompts shorter than the sinks + window."""
+    for mode in (0, 1):
+        cfg = lsa.Config(k=k, sinks=4, window=W, mode=mode, beam=2)
+        _, g, o, _ = _select_both(lsa, "prefill-4k", T, cfg)
+        assert np.array_equal(g, o), (mode, np.where((g != o).any(axis=(1, 2)))[0][:5])
+
+
+def test_select_degenerate_ties(lsa):
+    """All-zero keys give all-zero centroids: every score ties and the fill
+    takes buckets in ascending id (the band overflow path included)."""
+    cfg = lsa.Config(k=64, sinks=4, window=16)
+    T = 4096
+    K = np.zeros((T, 1, 128), np.uint16)
+    inp = synth.layer_inputs("prefill-4k", T=T)
+    cache = lsa.Cache(1, T, cfg)
+    lsa.build_buckets(to_dev_bf16(K), to_dev(inp["Wk"]), cfg, cache)
+    idx = lsa.select(to_dev_bf16(inp["Q"]), 0, to_dev(inp["Wq"]), cache, cfg).cpu().numpy()
+    torch.cuda.synchronize()
+    lsa.check_device_error()
+    oc = oracle.build_cache(oracle.key_latent_pool(K, inp["Wk"], 4), T, oracle_cfg(cfg))
+    Y = oracle.query_latent(inp["Q"], inp["Wq"], 1, 0)
+    oidx, _, _ = oracle.select(oc, Y, np.arange(T), oracle_cfg(cfg), G=4)
+    assert np.array_equal(idx, oidx)
+
+
+def _attn_err(O_dev, O_ref):
+    g = O_dev.float().cpu().numpy().astype(np.float64)
+    e = np.abs(g - O_ref)
+    return e.max(), e.mean()
+
+
+def test_sparse_attn_matches_oracle(lsa):
+    inp = synth.layer_inputs("prefill-128k", T=3000)
+    rng = np.random.default_rng(5)
+    nq, n = 96, 700
+    idx = rng.integers(0, 3000, size=(nq, 8, n)).astype(np.int32)
+    idx[rng.random(idx.shape) < 0.2] = -1
+    idx[3, 2, :] = -1                  # an empty list -> zeros
+    idx[4, 1, :] = -1
+    idx[4, 1, 17] = 123                # a single key -> its value row
+    Q = inp["Q"][:nq]
+    O = lsa.sparse_attn(to_dev_bf16(Q), to_dev_bf16(inp["K"]), to_dev_bf16(inp["V"]), to_dev(idx))
+    torch.cuda.synchronize()
+    lsa.check_device_error()
+    ref = oracle.attention(Q, inp["K"], inp["V"], idx)
+    mx, mean = _attn_err(O, ref)
+    assert mx <= ATOL_MAX and mean <= ATOL_MEAN, (mx, mean)
+    assert np.all(O[3, 8:12].float().cpu().numpy() == 0)
+
+
+def test_prefill_end_to_end_4k(lsa):
+    """The whole layer (lsa_prefill) against the oracle layer."""
+    cfg = lsa.Config(k=512, sinks=4, window=256)
+    inp = synth.layer_inputs("prefill-4k")
+    O = lsa.prefill(to_dev_bf16(inp["Q"]), to_dev_bf16(inp["K"]), to_dev_bf16(inp["V"]),
+                    to_dev(inp["Wk"]), to_dev(inp["Wq"]), cfg, chunk=1000)
+    torch.cuda.synchronize()
+    lsa.check_device_error()
+    ref = oracle.layer(inp["Q"], inp["K"], inp["V"], inp["Wk"], inp["Wq"], oracle_cfg(cfg))["O"]
+    mx, mean = _attn_err(O, ref)
+    assert mx <= ATOL_MAX and mean <= ATOL_MEAN, (mx, mean)
+
+
+def test_prefill_all_keys_is_full_causal_attention(lsa):
+    """k >= T: LSA reduces to exact causal attention (torch SDPA in fp32)."""
+    T = 2000
+    cfg = lsa.Config(k=4096, sinks=4, window=64)
+    inp = synth.layer_inputs("prefill-4k", T=T)
+    Q, K, V = (to_dev_bf16(inp[x]) for x in "QKV")
+    O = lsa.prefill(Q, K, V, to_dev(inp["Wk"]), to_dev(inp["Wq"]), cfg)
+    torch.cuda.synchronize()
+    q = Q.float().permute(1, 0, 2)
+    k = K.float().permute(1, 0, 2).expand(4, T, 128)
+    v = V.float().permute(1, 0, 2).expand(4, T, 128)
+    ref = torch.nn.functional.scaled_dot_product_attention(q, k, v, is_causal=True).permute(1, 0, 2)
+    e = (O.float() - ref).abs()
+    assert e.max().item() <= ATOL_MAX and e.mean().item() <= ATOL_MEAN
+
+
+def test_bad_arguments_return_status(lsa):
+    from clustered_key_indexing_b200._lib import LSAError, LSA_EINVAL, LSA_EUNSUPPORTED, LSA_ENOSPACE
+    cfg = lsa.Config(k=512, sinks=4, window=256)
+    inp = synth.layer_inputs("prefill-4k", T=64)
+    K = to_dev_bf16(inp["K"])
+    small = lsa.Cache(1, 16, cfg)
+    with pytest.raises(LSAError) as e:
+        lsa.build_buckets(K, to_dev(inp["Wk"]), cfg, small)
+    assert e.value.status == LSA_ENOSPACE
+    with pytest.raises(LSAError) as e:
+        lsa.build_buckets(K, to_dev(inp["Wk"]), lsa.Config(d_latent=32), lsa.Cache(1, 64, cfg))
+    assert e.value.status == LSA_EUNSUPPORTED
+    with pytest.raises(LSAError) as e:
+        lsa.build_buckets(K, to_dev(inp["Wk"]), lsa.Config(window=0), lsa.Cache(1, 64, cfg))
+    assert e.value.status == LSA_EINVAL
