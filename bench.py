@@ -49,6 +49,7 @@ def parse():
     p.add_argument("--mode", default=None, choices=["flat", "tree"])
     p.add_argument("--agg", default=None, choices=["mean", "max"])
     p.add_argument("--chunk", type=int, default=16384)
+    p.add_argument("--T", type=int, default=None, help="prefix length of the workload (profiling runs)")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu", action="store_true")
     return p.parse_args()
@@ -56,6 +57,8 @@ def parse():
 
 def workload_cfg(args):
     c = dict(synth.CONFIGS[args.workload])
+    if args.T:
+        c["T"] = args.T
     if args.mode:
         c["mode"] = 0 if args.mode == "flat" else 1
     if args.agg:
@@ -175,7 +178,7 @@ def run_reference(args):
     if rank != 0:
         return
     c = workload_cfg(args)
-    inp = synth.layer_inputs(args.workload, seed=0, parts=("Q", "K", "V"))
+    inp = synth.layer_inputs(args.workload, seed=0, T=c["T"], parts=("Q", "K", "V"))
     vals = []
     desc = ""
     for i in range(args.warmup + args.steps):
@@ -207,7 +210,7 @@ def run_lsa(args):
     T, hkv, hq = c["T"], c["hkv"], c["hq"]
     cfg = lsa.Config(k=c["k"], sinks=c["sinks"], window=c["window"], beam=c["beam"],
                      mode=c["mode"], agg=c["agg"])
-    inp = synth.layer_inputs(args.workload, seed=rank)
+    inp = synth.layer_inputs(args.workload, seed=rank, T=T)
     dev = torch.device("cuda", torch.cuda.current_device())
 
     def pinned(bits):
@@ -225,15 +228,27 @@ def run_lsa(args):
     sws = torch.empty(lsa.select_workspace_bytes(cfg, chunk, hq, cache) or 1, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
     chunks = [(t0, min(chunk, T - t0)) for t0 in range(0, T, chunk)]
-    attn_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in chunks]
+    def ev():
+        return torch.cuda.Event(enable_timing=True)
+
+    attn_ev = [(ev(), ev()) for _ in chunks]
+    sel_ev = [(ev(), ev()) for _ in chunks]
+    build_ev = (ev(), ev())
 
     def step(timed_attn=False):
+        if timed_attn:
+            build_ev[0].record(stream)
         lsa.build_buckets(K, Wk, cfg, cache)
         if tree is not None:
             lsa.build_tree(cache, cfg, tree)
+        if timed_attn:
+            build_ev[1].record(stream)
         for ci, (t0, n) in enumerate(chunks):
+            if timed_attn:
+                sel_ev[ci][0].record(stream)
             lsa.select(Q[t0:t0 + n], t0, Wq, cache, cfg, tree=tree, idx=idx[:n], ws=sws)
             if timed_attn:
+                sel_ev[ci][1].record(stream)
                 attn_ev[ci][0].record(stream)
             lsa.sparse_attn(Q[t0:t0 + n], K, V, idx[:n], T, O=O[t0:t0 + n])
             if timed_attn:
@@ -263,11 +278,13 @@ def run_lsa(args):
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     torch.cuda.synchronize()
     ev0.record(stream)
-    attn_ms = 0.0
+    attn_ms = sel_ms = build_ms = 0.0
     for _ in range(args.steps):
         step(timed_attn=True)
-        torch.cuda.synchronize()  # read this step's attention events
+        torch.cuda.synchronize()  # read this step's stage events
         attn_ms += sum(a.elapsed_time(b) for a, b in attn_ev)
+        sel_ms += sum(a.elapsed_time(b) for a, b in sel_ev)
+        build_ms += build_ev[0].elapsed_time(build_ev[1])
     ev1.record(stream)
     torch.cuda.synchronize()
     clk = clocks.stop()
@@ -325,7 +342,7 @@ def run_lsa(args):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu:
-        per_layer, desc, spent = oracle_sample(inp, c, n_blocks=None if T <= 131072 else 64, n_queries=16)
+        per_layer, desc, spent = oracle_sample(inp, c, n_blocks=None if T <= 131072 else 64, n_queries=256)
         cpu = {"value": T / per_layer, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": desc,
                "sample_seconds": spent}
 
@@ -336,6 +353,8 @@ def run_lsa(args):
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": config_json(args, c, world), "clocks": clk, "e2e": e2e,
             "gpu_launches": int(launches), "roofline": roofline, "cpu_baseline": cpu,
+            "stages_ms_per_step": {"build": build_ms / args.steps, "select": sel_ms / args.steps,
+                                   "attention": attn_ms / args.steps},
         }
         print(json.dumps(line), flush=True)
     if world > 1:

@@ -26,26 +26,10 @@
 #include <stdint.h>
 
 #include "lsa_common.cuh"
+#include "lsa_flat.cuh"
 #include "lsa_mma.cuh"
 
 namespace lsa {
-
-// --------------------------------------------------------------- scoring
-
-constexpr int kScoreCols = 128;  // centroid columns per CTA tile
-constexpr int kScoreRows = 64;   // MMA rows per CTA (4 warps x 16)
-
-struct ScoreArgs {
-    const uint16_t* Y;    // chunk query latents: [nqc, hkv, 64] (mean) / [nqc, hq, 64] (native)
-    const uint16_t* cent; // [hkv, cap_buckets, 64]
-    int64_t cap_buckets;
-    int64_t NB;
-    int64_t nqc;
-    int64_t t_first;
-    int32_t W, hkv, G, agg;
-    float* S;             // [nqc * hkv, ld]
-    int64_t ld;
-};
 
 // Columns (bucket slots) that can hold an eligible bucket for query t: only
 // blocks that start at or before t - W.
@@ -54,95 +38,6 @@ __host__ __device__ __forceinline__ int64_t flat_ncol(int64_t t, int32_t W, int6
     if (lim < 0) return 0;
     const int64_t n = (int64_t)kBucketsPerBlock * (lim / kBlockKeys + 1);
     return n < NB ? n : NB;
-}
-
-__global__ void __launch_bounds__(128) score_kernel(ScoreArgs a) {
-    __shared__ __align__(128) uint16_t ctile[kScoreCols * kDL];  // 16 KB, 16B-chunk swizzled
-    const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
-    const int h = blockIdx.z;
-    const int G = a.agg ? a.G : 1;
-    const int64_t n0 = (int64_t)blockIdx.x * kScoreCols;
-    const int64_t qrow0 = (int64_t)blockIdx.y * (kScoreRows / G);  // first query of the tile
-    if (qrow0 >= a.nqc) return;
-    const int64_t qlast = min(a.nqc - 1, qrow0 + kScoreRows / G - 1);
-    if (n0 >= flat_ncol(a.t_first + qlast, a.W, a.NB)) return;
-
-    // centroid tile -> shared (chunk c of row n at position c ^ (n & 7))
-    const uint16_t* cb = a.cent + ((int64_t)h * a.cap_buckets + n0) * kDL;
-#pragma unroll
-    for (int i = 0; i < (kScoreCols * 8) / 128; ++i) {
-        const int idx = tid + 128 * i;
-        const int n = idx >> 3, c = idx & 7;
-        const bool ok = n0 + n < a.NB;
-        cp_async_16(smem_u32(ctile + n * kDL + ((c ^ (n & 7)) << 3)),
-                    ok ? (const void*)(cb + (int64_t)n * kDL + c * 8) : (const void*)cb, ok ? 16 : 0);
-    }
-    cp_async_commit();
-
-    // A fragments straight from global: MMA row r of this warp
-    const int g = lane >> 2, tq = lane & 3;
-    uint32_t af[4][4];
-    const uint16_t* rowp[2];
-    bool rowok[2];
-#pragma unroll
-    for (int hh = 0; hh < 2; ++hh) {
-        const int r = w * 16 + g + 8 * hh;
-        const int64_t q = qrow0 + r / G;
-        rowok[hh] = q < a.nqc;
-        const int64_t yrow = a.agg ? (q * (int64_t)a.hkv * G + (int64_t)h * G + r % G)
-                                   : (q * (int64_t)a.hkv + h);
-        rowp[hh] = a.Y + (rowok[hh] ? yrow : 0) * kDL;
-    }
-#pragma unroll
-    for (int kk = 0; kk < 4; ++kk) {
-        const int c0 = kk * 16 + 2 * tq;
-        af[kk][0] = rowok[0] ? *reinterpret_cast<const uint32_t*>(rowp[0] + c0) : 0u;
-        af[kk][1] = rowok[1] ? *reinterpret_cast<const uint32_t*>(rowp[1] + c0) : 0u;
-        af[kk][2] = rowok[0] ? *reinterpret_cast<const uint32_t*>(rowp[0] + c0 + 8) : 0u;
-        af[kk][3] = rowok[1] ? *reinterpret_cast<const uint32_t*>(rowp[1] + c0 + 8) : 0u;
-    }
-    cp_async_wait<0>();
-    __syncthreads();
-
-    float acc[16][4];
-#pragma unroll
-    for (int j = 0; j < 16; ++j)
-#pragma unroll
-        for (int i = 0; i < 4; ++i) acc[j][i] = 0.f;
-    const uint32_t base = smem_u32(ctile);
-#pragma unroll
-    for (int kk = 0; kk < 4; ++kk) {
-#pragma unroll
-        for (int jp = 0; jp < 8; ++jp) {
-            // matrices: (n-tile 2jp, k lo), (2jp, k hi), (2jp+1, k lo), (2jp+1, k hi)
-            const int mi = lane >> 3, ri = lane & 7;
-            const int n = (2 * jp + (mi >> 1)) * 8 + ri;
-            const int c = 2 * kk + (mi & 1);
-            uint32_t b[4];
-            ldsm_x4(b, base + (uint32_t)(n * kDL + ((c ^ (n & 7)) << 3)) * 2u);
-            mma_16816(acc[2 * jp], af[kk], b[0], b[1]);
-            mma_16816(acc[2 * jp + 1], af[kk], b[2], b[3]);
-        }
-    }
-
-    // epilogue: rows g and g+8 of this warp (native: max over the G heads)
-#pragma unroll
-    for (int j = 0; j < 16; ++j) {
-        float v[4] = {acc[j][0], acc[j][1], acc[j][2], acc[j][3]};
-        for (int off = 4; off < 4 * G; off <<= 1)
-#pragma unroll
-            for (int i = 0; i < 4; ++i) v[i] = fmaxf(v[i], __shfl_xor_sync(0xffffffffu, v[i], off));
-        if ((g % G) != 0) continue;
-        const int64_t col = n0 + j * 8 + 2 * tq;
-#pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-            const int r = w * 16 + g + 8 * hh;
-            const int64_t q = qrow0 + r / G;
-            if (q >= a.nqc) continue;
-            float2* dst = reinterpret_cast<float2*>(a.S + (q * a.hkv + h) * a.ld + col);
-            *dst = make_float2(v[2 * hh], v[2 * hh + 1]);
-        }
-    }
 }
 
 // ------------------------------------------------------------- selection
@@ -252,18 +147,19 @@ __device__ __forceinline__ int block_exscan(int v, int* total, int* sh4) {
 }
 
 struct SelShared {
+    // 8-byte members first: every field below stays naturally aligned
     unsigned long long hist[kBins];   // packed (count << 32 | weight)
-    int cid[kCap];
     double csc[kCap];
-    int cw[kCap];
-    int ctk[kCap];
-    uint16_t ylat[8 * kDL];
-    int sh4[4];
     long long beam_id[16];
     double beam_sc[16];
+    long long above;                  // radix select: weight strictly above the prefix
+    int cid[kCap];
+    int cw[kCap];
+    int ctk[kCap];
+    int sh4[4];
     int nbeam;
-    int misc[8];
-    unsigned long long thr;
+    int misc[4];
+    uint16_t ylat[8 * kDL];
 };
 
 // Weighted radix select on exact scores of n candidates (id order) with
@@ -310,12 +206,12 @@ __device__ void radix_fill(int64_t n, int k, GetS gs, GetW gw, SetTk st, SelShar
                     cum += h256[dd];
                 }
                 sh.misc[0] = dig;
-                reinterpret_cast<long long*>(sh.misc)[1] = cum;  // weight strictly above
+                sh.above = cum;  // weight strictly above the chosen digit
             }
         }
         __syncthreads();
         prefix |= (unsigned long long)sh.misc[0] << shift;
-        above = reinterpret_cast<long long*>(sh.misc)[1];
+        above = sh.above;
         __syncthreads();
     }
     // ties at the cut: lowest ids first
@@ -516,7 +412,8 @@ __device__ int tree_candidates(const SelectArgs& a, const RowInfo& r, SelShared&
     return n;
 }
 
-__global__ void __launch_bounds__(kSelThreads) select_kernel(SelectArgs a) {
+// Tree search [essay ch. 4]: one CTA per (query, kv-head).
+__global__ void __launch_bounds__(kSelThreads) tree_select_kernel(SelectArgs a) {
     __shared__ SelShared sh;
     const int tid = threadIdx.x;
     const int64_t row = blockIdx.x;
@@ -527,10 +424,7 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(SelectArgs a) {
         return;
     }
     load_latents(a, r, sh);
-    const int ng = a.agg ? a.G : 1;
-    const int64_t hb0 = (int64_t)r.h * a.cap_buckets;
-
-    if (a.mode == 1) {
+    {
         __syncthreads();
         const int n = tree_candidates(a, r, sh);
         if (n > kCap) {
@@ -551,98 +445,6 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(SelectArgs a) {
         return;
     }
 
-    // ---- flat: pass 1, weighted histogram of the fp32 scores
-    const int64_t ncol = flat_ncol(r.t, a.W, a.NB);
-    const float* srow = a.scores + row * a.ld;
-    for (int i = tid; i < kBins; i += kSelThreads) sh.hist[i] = 0ull;
-    __syncthreads();
-    long long myw = 0;
-    for (int64_t b = tid; b < ncol; b += kSelThreads) {
-        if ((int64_t)a.minlr[hb0 + b] > r.lim) continue;
-        const int w = bucket_weight(a, r.h, b, r.lim);
-        myw += w;
-        atomicAdd(&sh.hist[score_bin(srow[b])], (1ull << 32) | (unsigned long long)w);
-    }
-    // total weight
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) myw += __shfl_xor_sync(0xffffffffu, myw, off);
-    __shared__ long long wsum[4];
-    if ((tid & 31) == 0) wsum[tid >> 5] = myw;
-    __syncthreads();
-    const long long totw = wsum[0] + wsum[1] + wsum[2] + wsum[3];
-    if (totw <= a.k) {
-        emit_range(a, r, ncol,
-                   [&](int64_t b) -> int {
-                       return ((int64_t)a.minlr[hb0 + b] <= r.lim) ? bucket_weight(a, r.h, b, r.lim) : 0;
-                   },
-                   sh);
-        return;
-    }
-    // cut bin: highest j with weight(bins >= j) >= k; keep bins >= j - 1
-    if (tid < 32) {
-        const int lane = tid;
-        long long s = 0, c = 0;
-        for (int d = 0; d < kBins / 32; ++d) {
-            const unsigned long long v = sh.hist[kBins - 1 - (kBins / 32) * lane - d];
-            s += (long long)(v & 0xffffffffull);
-            c += (long long)(v >> 32);
-        }
-        long long incl = s;
-#pragma unroll
-        for (int off = 1; off < 32; off <<= 1) {
-            const long long y = __shfl_up_sync(0xffffffffu, incl, off);
-            if (lane >= off) incl += y;
-        }
-        const long long excl = incl - s;
-        const unsigned mask = __ballot_sync(0xffffffffu, incl >= a.k && excl < a.k);
-        const int src = __ffs(mask) - 1;
-        if (lane == src) {
-            long long cum = excl;
-            int j = kBins - 1 - (kBins / 32) * lane;
-            for (int d = 0; d < kBins / 32; ++d) {
-                const int jj = kBins - 1 - (kBins / 32) * lane - d;
-                cum += (long long)(sh.hist[jj] & 0xffffffffull);
-                if (cum >= a.k) { j = jj; break; }
-            }
-            sh.misc[0] = j > 0 ? j - 1 : 0;
-        }
-    }
-    __syncthreads();
-    const int jt = sh.misc[0];
-    // candidate count
-    int cnt = 0;
-    for (int i = jt + tid; i < kBins; i += kSelThreads) cnt += (int)(sh.hist[i] >> 32);
-    int ncand;
-    block_exscan(cnt, &ncand, sh.sh4);
-    if (ncand > kCap) {
-        if (tid == 0) {
-            const int slot = atomicAdd(a.ovf_count, 1);
-            if (slot < a.ovf_cap) a.ovf_rows[slot] = (int)row;
-            else raise_device_error(kErrSelectOverflow);
-        }
-        return;
-    }
-    // pass 2: ordered compaction of the band, then exact rescoring
-    int n = 0;
-    for (int64_t c0 = 0; c0 < ncol; c0 += kSelThreads) {
-        const int64_t b = c0 + tid;
-        const bool el = b < ncol && (int64_t)a.minlr[hb0 + b] <= r.lim && score_bin(srow[b]) >= jt;
-        int tot;
-        const int o = block_exscan(el ? 1 : 0, &tot, sh.sh4);
-        if (el) sh.cid[n + o] = (int)b;
-        n += tot;
-    }
-    __syncthreads();
-    for (int i = tid; i < n; i += kSelThreads) {
-        const int64_t b = sh.cid[i];
-        sh.csc[i] = exact_score(sh.ylat, ng, a.cent + (hb0 + b) * kDL);
-        sh.cw[i] = bucket_weight(a, r.h, b, r.lim);
-    }
-    __syncthreads();
-    radix_fill(
-        n, a.k, [&](int64_t i) { return sh.csc[i]; }, [&](int64_t i) { return sh.cw[i]; },
-        [&](int64_t i, int tk) { sh.ctk[i] = tk; }, sh);
-    emit_candidates(a, r, n, sh);
 }
 
 // Rows whose candidate band overflowed: exact scores of every eligible
@@ -680,7 +482,7 @@ __global__ void __launch_bounds__(kSelThreads) select_fallback_kernel(SelectArgs
 // ------------------------------------------------------------ host side
 
 struct SelectPlan {
-    int64_t ld;        // score row stride (floats)
+    int64_t ld;        // fallback slot stride (bucket slots, rounded up)
     int64_t chunk;     // query positions per chunk
     int32_t hy;        // latent rows per query
     int32_t fb_slots;
@@ -688,10 +490,11 @@ struct SelectPlan {
 
 static SelectPlan plan_select(const lsa_cfg* cfg, int64_t nq, int32_t hq, int32_t hkv, int64_t NB) {
     SelectPlan p;
-    p.ld = ceil_div<int64_t>(NB > 0 ? NB : 1, kScoreCols) * kScoreCols;
+    p.ld = ceil_div<int64_t>(NB > 0 ? NB : 1, 128) * 128;
     p.hy = cfg->agg ? hq : hkv;
-    const int64_t budget = (int64_t)512 << 20;  // score rows per chunk
-    int64_t c = budget / (hkv * p.ld * (int64_t)sizeof(float));
+    // candidate lists: kCandCap x 8 bytes per (query, kv-head)
+    const int64_t budget = (int64_t)512 << 20;
+    int64_t c = budget / (hkv * (int64_t)kCandCap * 8);
     c = c / 64 * 64;
     if (c < 64) c = 64;
     if (c > nq) c = nq;
@@ -705,7 +508,10 @@ static size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 struct SelectWs {
     uint16_t* Y;
-    float* S;
+    float* tau;
+    int32_t* cand_col;
+    float* cand_s;
+    int32_t* cand_n;
     int32_t* ovf_rows;
     int32_t* ovf_count;
     double* fb_score;
@@ -716,10 +522,14 @@ struct SelectWs {
 static SelectWs carve_select(const SelectPlan& p, int32_t hkv, int mode, char* base) {
     SelectWs w{};
     size_t o = 0;
+    const size_t rows = (size_t)p.chunk * hkv;
     w.Y = (uint16_t*)(base + o); o += align256((size_t)p.chunk * p.hy * kDL * 2);
     if (mode == 0) {
-        w.S = (float*)(base + o); o += align256((size_t)p.chunk * hkv * p.ld * 4);
-        w.ovf_rows = (int32_t*)(base + o); o += align256((size_t)p.chunk * hkv * 4);
+        w.tau = (float*)(base + o); o += align256(rows * 4);
+        w.cand_col = (int32_t*)(base + o); o += align256(rows * kCandCap * 4);
+        w.cand_s = (float*)(base + o); o += align256(rows * kCandCap * 4);
+        w.cand_n = (int32_t*)(base + o); o += align256(rows * 4);
+        w.ovf_rows = (int32_t*)(base + o); o += align256(rows * 4);
         w.ovf_count = (int32_t*)(base + o); o += 256;
         w.fb_score = (double*)(base + o); o += align256((size_t)p.fb_slots * p.ld * 8);
         w.fb_w = (int32_t*)(base + o); o += align256((size_t)p.fb_slots * p.ld * 4);
@@ -766,7 +576,6 @@ lsa_status run_select(const uint16_t* Q, int64_t t0, int64_t nq, int32_t hq, con
         for (int l = 0; l < tree->levels; ++l) { a.level_n[l] = tree->level_n[l]; a.level_off[l] = tree->level_off[l]; }
     }
     a.ld = p.ld;
-    a.scores = w.S;
     a.ovf_rows = w.ovf_rows; a.ovf_count = w.ovf_count; a.ovf_cap = (int32_t)(p.chunk * hkv);
     a.fb_score = w.fb_score; a.fb_w = w.fb_w;
 
@@ -776,28 +585,29 @@ lsa_status run_select(const uint16_t* Q, int64_t t0, int64_t nq, int32_t hq, con
         lsa_status s = launch_query_latent(Q + c0 * hq * kD, nqc, hq, hkv, W_q, cfg->agg, Y, st);
         if (s != LSA_OK) return s;
         a.Y = Y; a.nqc = nqc; a.t_first = t0 + c0; a.idx = idx + c0 * hkv * row_len;
-        if (cfg->mode == 0) {
-            ScoreArgs sa{};
-            sa.Y = Y; sa.cent = c->cent; sa.cap_buckets = c->cap_buckets; sa.NB = NB; sa.nqc = nqc;
-            sa.t_first = t0 + c0; sa.W = cfg->window; sa.hkv = hkv; sa.G = hq / hkv; sa.agg = cfg->agg;
-            sa.S = w.S; sa.ld = p.ld;
-            const int64_t ncol = flat_ncol(t0 + c0 + nqc - 1, cfg->window, NB);
-            if (ncol > 0) {
-                const int qpt = kScoreRows / (cfg->agg ? hq / hkv : 1);
-                dim3 grid((unsigned)ceil_div<int64_t>(ncol, kScoreCols),
-                          (unsigned)ceil_div<int64_t>(nqc, qpt), (unsigned)hkv);
-                score_kernel<<<grid, 128, 0, st>>>(sa);
-                if ((s = check_launch("score_kernel")) != LSA_OK) return s;
-            }
-            if (cudaMemsetAsync(w.ovf_count, 0, sizeof(int32_t), st) != cudaSuccess)
-                return set_error(LSA_ECUDA, "lsa_select: memset failed");
+        if (cfg->mode == 1) {
+            tree_select_kernel<<<(unsigned)(nqc * hkv), kSelThreads, 0, st>>>(a);
+            if ((s = check_launch("tree_select_kernel")) != LSA_OK) return s;
+            continue;
         }
-        select_kernel<<<(unsigned)(nqc * hkv), kSelThreads, 0, st>>>(a);
-        if ((s = check_launch("select_kernel")) != LSA_OK) return s;
-        if (cfg->mode == 0) {
-            select_fallback_kernel<<<(unsigned)p.fb_slots, kSelThreads, 0, st>>>(a);
-            if ((s = check_launch("select_fallback_kernel")) != LSA_OK) return s;
-        }
+        if (cudaMemsetAsync(w.ovf_count, 0, sizeof(int32_t), st) != cudaSuccess)
+            return set_error(LSA_ECUDA, "lsa_select: memset failed");
+        PassArgs pa{};
+        pa.Y = Y; pa.cent = c->cent; pa.minlr = c->minlr; pa.cnt_lr = c->cnt_lr;
+        pa.cap_buckets = c->cap_buckets; pa.NB = NB; pa.nqc = nqc; pa.t_first = t0 + c0;
+        pa.W = cfg->window; pa.hkv = hkv; pa.G = hq / hkv; pa.agg = cfg->agg; pa.k = cfg->k;
+        pa.tau = w.tau; pa.cand_col = w.cand_col; pa.cand_s = w.cand_s; pa.cand_n = w.cand_n;
+        ResolveArgs ra{};
+        ra.offsets = c->offsets; ra.members = c->members; ra.cnt_lr = c->cnt_lr; ra.minlr = c->minlr;
+        ra.maxpos = c->maxpos; ra.cent = c->cent; ra.cap_units = c->cap_units;
+        ra.cap_buckets = c->cap_buckets; ra.NB = NB; ra.T_built = c->n_tokens;
+        ra.hkv = hkv; ra.G = hq / hkv; ra.agg = cfg->agg; ra.k = cfg->k; ra.S = cfg->sinks;
+        ra.W = cfg->window; ra.Y = Y; ra.nqc = nqc; ra.t_first = t0 + c0; ra.tau = w.tau;
+        ra.cand_col = w.cand_col; ra.cand_s = w.cand_s; ra.cand_n = w.cand_n; ra.idx = a.idx;
+        ra.ovf_rows = w.ovf_rows; ra.ovf_count = w.ovf_count; ra.ovf_cap = a.ovf_cap;
+        if ((s = launch_flat(pa, ra, st)) != LSA_OK) return s;
+        select_fallback_kernel<<<(unsigned)p.fb_slots, kSelThreads, 0, st>>>(a);
+        if ((s = check_launch("select_fallback_kernel")) != LSA_OK) return s;
     }
     return LSA_OK;
 }
