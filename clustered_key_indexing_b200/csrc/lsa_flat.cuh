@@ -5,19 +5,23 @@
 // Three kernels per chunk of query positions:
 //   flat_pass_kernel<sample=true>   bf16 tensor-core scores (mma.sync
 //       m16n8k16, fp32 accumulate) of 64 query rows against every 16th
-//       centroid; a per-row weighted histogram of those scores gives a
-//       threshold tau expected to keep about twice the k keys needed;
+//       centroid; a per-row weighted histogram of those scores (bins scaled to
+//       the row's latent norm, which bounds its scores) gives a threshold tau
+//       expected to keep about twice the k keys needed;
 //   flat_pass_kernel<sample=false>  the same contraction over every eligible
-//       centroid; scores >= tau are appended to the row's candidate list;
+//       centroid; scores >= tau are appended to the row's candidate list in
+//       ascending bucket id;
 //   flat_resolve_kernel             one warp per (query, kv-head): eligibility
-//       and exact key counts, exact fp64 rescoring, weighted radix select on
-//       the exact scores (score desc, bucket id asc), sort of the chosen
-//       buckets by id, key emission, sinks and window.
-// The resolve step checks that the buckets with fp32 score >= tau + 2e
-// already hold k keys (e = 1e-4 bounds the fp32 score error, which is below
-// 64 * 2^-23 * |y||c|): then every bucket that can rank above the exact cut
-// is a candidate.  Rows that fail the check, or whose list overflowed, go to
-// the exact fallback kernel (exact scores of every eligible bucket).
+//       and exact key counts, weighted radix select on the fp32 scores for the
+//       cut c32, exact fp64 rescoring of the buckets within 2e of c32 only,
+//       key emission in bucket id order, sinks and window.
+// Exactness: |fp32 score - exact score| < e = 1e-4 (the error is below
+// 64 * 2^-23 * |y||c|).  The exact score E* of the k-th key then lies in
+// [c32 - e, c32 + e]: buckets with fp32 score > c32 + 2e rank strictly above
+// it, buckets below c32 - 2e strictly below, and only the band between is
+// ranked on exact fp64 scores (score desc, bucket id asc).  The band must lie
+// above tau (every bucket in it is then a candidate); rows where it does not,
+// or whose list overflowed, go to the exact fallback kernel.
 #pragma once
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -29,9 +33,7 @@ namespace lsa {
 
 constexpr int kCandCap = 1024;       // candidates kept per (query, kv-head)
 constexpr int kSampleStride = 16;    // every 16th bucket scored by the sample pass
-constexpr int kSBins = 256;          // sample histogram bins over [-1.0625, 1.0625)
-constexpr float kSBinLo = -1.0625f;
-constexpr float kSBinW = 2.125f / kSBins;
+constexpr int kSBins = 256;          // sample histogram bins over [-R, R], R = row latent norm
 constexpr int kOversample = 2;       // tau targets kOversample * k keys
 constexpr float kScoreErr = 1e-4f;   // bound on |fp32 score - exact score|
 constexpr int kPassCols = 128;
@@ -66,7 +68,8 @@ __global__ void __launch_bounds__(128) flat_pass_kernel(PassArgs a) {
     uint16_t* ctile = reinterpret_cast<uint16_t*>(psm);                       // [2][128*64]
     int32_t* mminlr = reinterpret_cast<int32_t*>(psm + 2 * kPassCols * kDL * 2);  // [2][128]
     int32_t* mcnt = mminlr + 2 * kPassCols;                                   // [2][128]
-    uint32_t* hist = reinterpret_cast<uint32_t*>(mcnt + 2 * kPassCols);       // sample: [qpt][256]; full: [qpt]
+    float* rads = reinterpret_cast<float*>(mcnt + 2 * kPassCols);             // [64] row radii
+    uint32_t* hist = reinterpret_cast<uint32_t*>(rads + 64);                  // sample: [qpt][256]; full: [qpt]
 
     const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
     const int h = blockIdx.y;
@@ -86,7 +89,7 @@ __global__ void __launch_bounds__(128) flat_pass_kernel(PassArgs a) {
     const int g = lane >> 2, tq = lane & 3;
     uint32_t af[4][4];
     int64_t lim[2], ncol[2], row[2];
-    float tau[2];
+    float tau[2], rad[2];
     int qloc[2];
     bool rowok[2];
 #pragma unroll
@@ -102,12 +105,25 @@ __global__ void __launch_bounds__(128) flat_pass_kernel(PassArgs a) {
         tau[hh] = SAMPLE ? 0.f : a.tau[row[hh]];
         const int64_t yrow = a.agg ? ((rowok[hh] ? q : 0) * (int64_t)a.hkv * G + (int64_t)h * G + r % G) : row[hh];
         const uint16_t* yp = a.Y + yrow * kDL;
+        float n2 = 0.f;
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {
             const int c0 = kk * 16 + 2 * tq;
             af[kk][hh] = rowok[hh] ? *reinterpret_cast<const uint32_t*>(yp + c0) : 0u;
             af[kk][hh + 2] = rowok[hh] ? *reinterpret_cast<const uint32_t*>(yp + c0 + 8) : 0u;
+            const uint32_t u[2] = {af[kk][hh], af[kk][hh + 2]};
+#pragma unroll
+            for (int x = 0; x < 2; ++x) {
+                const float lo = __uint_as_float(u[x] << 16), hi = __uint_as_float(u[x] & 0xFFFF0000u);
+                n2 += lo * lo + hi * hi;
+            }
         }
+        // |y| of the row (native: max over the group's heads) bounds |score|
+        n2 += __shfl_xor_sync(0xffffffffu, n2, 1);
+        n2 += __shfl_xor_sync(0xffffffffu, n2, 2);
+        for (int off = 4; off < 4 * G; off <<= 1) n2 = fmaxf(n2, __shfl_xor_sync(0xffffffffu, n2, off));
+        rad[hh] = fminf(1.0625f, sqrtf(n2) * 1.01f + 1e-6f);
+        if (SAMPLE && rowok[hh] && (g % G) == 0 && tq == 0) rads[qloc[hh]] = rad[hh];
     }
 
     const uint16_t* cb = a.cent + (int64_t)h * a.cap_buckets * kDL;
@@ -161,12 +177,15 @@ __global__ void __launch_bounds__(128) flat_pass_kernel(PassArgs a) {
             }
         }
         const int64_t v0 = (int64_t)tile * kPassCols;
+        uint32_t hit[2] = {0u, 0u};  // bit 2j+e: element (n8 tile j, column e) kept
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
             float v[4] = {acc[j][0], acc[j][1], acc[j][2], acc[j][3]};
             for (int off = 4; off < 4 * G; off <<= 1)
 #pragma unroll
                 for (int i = 0; i < 4; ++i) v[i] = fmaxf(v[i], __shfl_xor_sync(0xffffffffu, v[i], off));
+#pragma unroll
+            for (int i = 0; i < 4; ++i) acc[j][i] = v[i];
             if ((g % G) != 0) continue;
 #pragma unroll
             for (int hh = 0; hh < 2; ++hh) {
@@ -175,18 +194,52 @@ __global__ void __launch_bounds__(128) flat_pass_kernel(PassArgs a) {
                 for (int e = 0; e < 2; ++e) {
                     const int cl = j * 8 + 2 * tq + e;
                     const int64_t vc = v0 + cl;
-                    const float s = v[2 * hh + e];
+                    const float sc = v[2 * hh + e];
                     if (SAMPLE) {
                         if (vc * kSampleStride < ncol[hh] && (int64_t)mminlr[buf * kPassCols + cl] <= lim[hh]) {
-                            int bin = __float2int_rd((s - kSBinLo) * (1.0f / kSBinW));
+                            int bin = __float2int_rd((sc + rad[hh]) * ((float)kSBins / (2.f * rad[hh])));
                             bin = bin < 0 ? 0 : (bin >= kSBins ? kSBins - 1 : bin);
                             atomicAdd(&hist[qloc[hh] * kSBins + bin], (uint32_t)mcnt[buf * kPassCols + cl]);
                         }
-                    } else if (s >= tau[hh] && vc < ncol[hh]) {
-                        const uint32_t slot = atomicAdd(&hist[qloc[hh]], 1u);
-                        if (slot < (uint32_t)kCandCap) {
-                            a.cand_col[row[hh] * kCandCap + slot] = (int32_t)vc;
-                            a.cand_s[row[hh] * kCandCap + slot] = s;
+                    } else if (sc >= tau[hh] && vc < ncol[hh]) {
+                        hit[hh] |= 1u << (2 * j + e);
+                    }
+                }
+            }
+        }
+        if (!SAMPLE) {
+            // ordered append: the 4 lanes of a quad hold one row's columns
+            // 8j + 2tq + e; a hit's rank in the tile counts the quad's hits
+            // in earlier n8 tiles and in earlier lanes of its own tile
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+                const int qb = lane & ~3;
+                const uint32_t m0 = __shfl_sync(0xffffffffu, hit[hh], qb);
+                const uint32_t m1 = __shfl_sync(0xffffffffu, hit[hh], qb | 1);
+                const uint32_t m2 = __shfl_sync(0xffffffffu, hit[hh], qb | 2);
+                const uint32_t m3 = __shfl_sync(0xffffffffu, hit[hh], qb | 3);
+                const int tot = __popc(m0) + __popc(m1) + __popc(m2) + __popc(m3);
+                int base = 0;
+                if (tq == 0 && tot > 0) base = (int)atomicAdd(&hist[qloc[hh]], (uint32_t)tot);
+                base = __shfl_sync(0xffffffffu, base, qb);
+                if (tot == 0) continue;
+                const uint32_t mine = hit[hh];
+#pragma unroll
+                for (int j = 0; j < 16; ++j) {
+#pragma unroll
+                    for (int e = 0; e < 2; ++e) {
+                        if (!((mine >> (2 * j + e)) & 1u)) continue;
+                        const uint32_t below = (1u << (2 * j)) - 1u, here = 3u << (2 * j);
+                        int pos = __popc(m0 & below) + __popc(m1 & below) + __popc(m2 & below) +
+                                  __popc(m3 & below);
+                        if (tq > 0) pos += __popc(m0 & here);
+                        if (tq > 1) pos += __popc(m1 & here);
+                        if (tq > 2) pos += __popc(m2 & here);
+                        if (e) pos += (mine >> (2 * j)) & 1u;
+                        const int slot = base + pos;
+                        if (slot < kCandCap) {
+                            a.cand_col[row[hh] * kCandCap + slot] = (int32_t)(v0 + j * 8 + 2 * tq + e);
+                            a.cand_s[row[hh] * kCandCap + slot] = acc[j][2 * hh + e];
                         }
                     }
                 }
@@ -201,11 +254,12 @@ __global__ void __launch_bounds__(128) flat_pass_kernel(PassArgs a) {
         if (SAMPLE) {
             // tau: lower edge of the bin where the scaled sample weight from
             // the top first reaches kOversample * k; -inf if it never does
+            const float R = rads[tid];
             float t = -CUDART_INF_F;
             long long cum = 0;
             for (int b = kSBins - 1; b >= 0; --b) {
                 cum += (long long)hist[tid * kSBins + b] * kSampleStride;
-                if (cum >= (long long)kOversample * a.k) { t = kSBinLo + b * kSBinW; break; }
+                if (cum >= (long long)kOversample * a.k) { t = -R + b * (2.f * R / kSBins); break; }
             }
             a.tau[r] = t;
         } else {
@@ -239,18 +293,21 @@ struct ResolveArgs {
     int32_t ovf_cap;
 };
 
+constexpr int kBandCap = 128;  // buckets ranked on exact scores per row
+
 struct ResWarp {
-    double ex[kCandCap];      // exact scores
-    int32_t col[kCandCap];    // bucket ids; later packed (id << 5 | taken)
-    int32_t w[kCandCap];      // key weights; later taken counts (negative = tied)
+    double bex[kBandCap];     // exact scores of the band
+    int32_t col[kCandCap];    // eligible candidates, ascending bucket id
+    float sc[kCandCap];       // their fp32 scores
+    int32_t w[kCandCap];      // key weights, then taken counts
+    int32_t bidx[kBandCap];   // band members (index into col)
     uint32_t hist[256];
     uint16_t ylat[8 * kDL];
 };
 
-__device__ __forceinline__ unsigned long long order_key_d(double s) {
-    s = s + 0.0;
-    const unsigned long long u = (unsigned long long)__double_as_longlong(s);
-    return (u >> 63) ? ~u : (u | 0x8000000000000000ull);
+__device__ __forceinline__ uint32_t order_key_f(float s) {
+    const uint32_t u = __float_as_uint(s + 0.0f);
+    return (u >> 31) ? ~u : (u | 0x80000000u);
 }
 
 __device__ int weight_of(const ResolveArgs& a, int h, int64_t b, int64_t lim) {
@@ -267,11 +324,26 @@ __device__ int weight_of(const ResolveArgs& a, int h, int64_t b, int64_t lim) {
     return w;
 }
 
+// First `tk` keys of bucket b in [S, lim], ascending.  Fast path: a bucket
+// that is taken whole, lies entirely inside [S, lim] and has full units
+// writes 4 consecutive positions per member unit.
 __device__ void emit_keys(const ResolveArgs& a, int h, int64_t b, int tk, int64_t lim, int32_t* out) {
     const int32_t* off = a.offsets + (int64_t)h * (a.cap_buckets + 1);
     const int32_t* mem = a.members + (int64_t)h * a.cap_units;
+    const int64_t hb = (int64_t)h * a.cap_buckets + b;
+    const int32_t m0 = off[b], m1 = off[b + 1];
+    if (tk == (m1 - m0) * kPool && (int64_t)a.maxpos[hb] <= lim && a.minlr[hb] == mem[m0] * kPool &&
+        a.maxpos[hb] < a.T_built) {
+        int o = 0;
+        for (int32_t m = m0; m < m1; ++m) {
+            const int32_t p = mem[m] * kPool;
+            out[o] = p; out[o + 1] = p + 1; out[o + 2] = p + 2; out[o + 3] = p + 3;
+            o += 4;
+        }
+        return;
+    }
     int o = 0;
-    for (int32_t m = off[b]; m < off[b + 1] && o < tk; ++m) {
+    for (int32_t m = m0; m < m1 && o < tk; ++m) {
         const int64_t j = mem[m];
         for (int64_t p = j * kPool; p < j * kPool + kPool && p < a.T_built && o < tk; ++p)
             if (p >= a.S && p <= lim) out[o++] = (int32_t)p;
@@ -308,7 +380,7 @@ __device__ __forceinline__ void push_fallback(const ResolveArgs& a, int64_t row)
     else raise_device_error(kErrSelectOverflow);
 }
 
-__global__ void __launch_bounds__(32 * kResWarps) flat_resolve_kernel(ResolveArgs a) {
+__global__ void __launch_bounds__(32 * kResWarps, 4) flat_resolve_kernel(ResolveArgs a) {
     extern __shared__ __align__(16) uint8_t rsm[];
     const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
     ResWarp& sw = reinterpret_cast<ResWarp*>(rsm)[wid];
@@ -335,64 +407,51 @@ __global__ void __launch_bounds__(32 * kResWarps) flat_resolve_kernel(ResolveArg
         return;
     }
     const float tau = a.tau[row];
-    const int ng = a.agg ? a.G : 1;
-    const uint16_t* ysrc = a.agg ? a.Y + (q * (int64_t)a.hkv * a.G + (int64_t)h * a.G) * kDL
-                                 : a.Y + row * kDL;
-    for (int i = lane; i < ng * kDL; i += 32) sw.ylat[i] = ysrc[i];
-    __syncwarp();
 
-    // eligible candidates, exact weights and scores
+    // eligible candidates (kept in ascending bucket id) and their key counts
     const int64_t hb0 = (int64_t)h * a.cap_buckets;
     int m = 0;
-    long long whi = 0, wtot = 0;
+    long long wtot = 0;
     for (int base = 0; base < n; base += 32) {
         const int i = base + lane;
         bool el = false;
         int col = 0, wgt = 0;
-        float s = 0.f;
+        float sc = 0.f;
         if (i < n) {
             col = a.cand_col[row * kCandCap + i];
-            s = a.cand_s[row * kCandCap + i];
+            sc = a.cand_s[row * kCandCap + i];
             el = (int64_t)a.minlr[hb0 + col] <= lim;
         }
         if (el) {
             wgt = weight_of(a, h, col, lim);
             wtot += wgt;
-            if (s >= tau + 2.0f * kScoreErr) whi += wgt;
         }
         const unsigned bal = __ballot_sync(0xffffffffu, el);
-        const int pos = m + __popc(bal & ((1u << lane) - 1u));
         if (el) {
+            const int pos = m + __popc(bal & ((1u << lane) - 1u));
             sw.col[pos] = col;
+            sw.sc[pos] = sc;
             sw.w[pos] = wgt;
-            sw.ex[pos] = exact_row(sw.ylat, ng, a.cent + (hb0 + col) * kDL);
         }
         m += __popc(bal);
     }
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) {
-        whi += __shfl_xor_sync(0xffffffffu, whi, off);
-        wtot += __shfl_xor_sync(0xffffffffu, wtot, off);
-    }
-    // tau = -inf means every eligible bucket is in the list
-    if (tau > -CUDART_INF_F && whi < a.k) {
-        if (lane == 0) push_fallback(a, row);
-        return;
-    }
+    for (int off = 16; off > 0; off >>= 1) wtot += __shfl_xor_sync(0xffffffffu, wtot, off);
     __syncwarp();
 
     if (wtot > a.k) {
-        // weighted radix select on the exact scores (8 digits of 8 bits)
-        unsigned long long prefix = 0;
+        // weighted radix select on the fp32 scores: cut key K32 with
+        // weight(key > K32) < k <= weight(key >= K32)
+        uint32_t prefix = 0;
         long long above = 0;
-        for (int pass = 0; pass < 8; ++pass) {
-            const int shift = 56 - 8 * pass;
+        for (int pass = 0; pass < 4; ++pass) {
+            const int shift = 24 - 8 * pass;
             for (int i = lane; i < 256; i += 32) sw.hist[i] = 0u;
             __syncwarp();
             for (int i = lane; i < m; i += 32) {
-                const unsigned long long key = order_key_d(sw.ex[i]);
+                const uint32_t key = order_key_f(sw.sc[i]);
                 if (pass > 0 && (key >> (shift + 8)) != (prefix >> (shift + 8))) continue;
-                atomicAdd(&sw.hist[(key >> shift) & 255ull], (unsigned)sw.w[i]);
+                atomicAdd(&sw.hist[(key >> shift) & 255u], (unsigned)sw.w[i]);
             }
             __syncwarp();
             long long s8 = 0;
@@ -405,7 +464,7 @@ __global__ void __launch_bounds__(32 * kResWarps) flat_resolve_kernel(ResolveArg
             }
             const long long excl = incl - s8;
             const unsigned hitm = __ballot_sync(0xffffffffu, above + incl >= a.k && above + excl < a.k);
-            if (hitm == 0u) {  // cannot happen while the weights above the prefix reach k
+            if (hitm == 0u) {  // cannot happen while the weight above the prefix reaches k
                 if (lane == 0) push_fallback(a, row);
                 return;
             }
@@ -423,80 +482,97 @@ __global__ void __launch_bounds__(32 * kResWarps) flat_resolve_kernel(ResolveArg
             }
             dig = __shfl_sync(0xffffffffu, dig, src);
             above = __shfl_sync(0xffffffffu, cum, src);
-            prefix |= (unsigned long long)dig << shift;
+            prefix |= (uint32_t)dig << shift;
             __syncwarp();
         }
-        // taken counts: above the cut fully, below not at all, ties pending
+        const float c32 = __uint_as_float((prefix >> 31) ? (prefix & 0x7FFFFFFFu) : ~prefix);
+        const float hi = c32 + 2.f * kScoreErr, lo = c32 - 2.f * kScoreErr;
+        // every bucket that can rank above the exact cut must be a candidate
+        if (tau > -CUDART_INF_F && !(lo >= tau)) {
+            if (lane == 0) push_fallback(a, row);
+            return;
+        }
+        // in (> hi): taken whole; out (< lo): not taken; band: exact ranking
+        long long win = 0;
+        int nb = 0;
+        for (int base = 0; base < m; base += 32) {
+            const int i = base + lane;
+            const float sc = i < m ? sw.sc[i] : -CUDART_INF_F;
+            const bool band = i < m && sc >= lo && sc <= hi;
+            if (i < m && sc > hi) win += sw.w[i];
+            const unsigned bal = __ballot_sync(0xffffffffu, band);
+            if (band) {
+                const int pos = nb + __popc(bal & ((1u << lane) - 1u));
+                if (pos < kBandCap) sw.bidx[pos] = i;
+            }
+            nb += __popc(bal);
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) win += __shfl_xor_sync(0xffffffffu, win, off);
+        if (nb > kBandCap) {
+            if (lane == 0) push_fallback(a, row);
+            return;
+        }
+        const int ng = a.agg ? a.G : 1;
+        const uint16_t* ysrc = a.agg ? a.Y + (q * (int64_t)a.hkv * a.G + (int64_t)h * a.G) * kDL
+                                     : a.Y + row * kDL;
+        for (int i = lane; i < ng * kDL; i += 32) sw.ylat[i] = ysrc[i];
+        __syncwarp();
+        for (int i = lane; i < nb; i += 32)
+            sw.bex[i] = exact_row(sw.ylat, ng, a.cent + (hb0 + sw.col[sw.bidx[i]]) * kDL);
+        __syncwarp();
+        // taken counts: in -> whole, out -> 0, band -> pending (negative)
         for (int i = lane; i < m; i += 32) {
-            const unsigned long long key = order_key_d(sw.ex[i]);
-            sw.w[i] = key > prefix ? sw.w[i] : (key == prefix ? -sw.w[i] : 0);
+            const float sc = sw.sc[i];
+            sw.w[i] = sc > hi ? sw.w[i] : (sc >= lo ? -sw.w[i] : 0);
         }
         __syncwarp();
-        // ties at the cut: lowest bucket ids first
-        long long need = a.k - above;
+        long long need = a.k - win;
         while (need > 0) {
-            int best = 0x7FFFFFFF, bi = -1;
-            for (int i = lane; i < m; i += 32)
-                if (sw.w[i] < 0 && sw.col[i] < best) { best = sw.col[i]; bi = i; }
+            // best pending band bucket: exact score desc, bucket id asc
+            double bs = -CUDART_INF;
+            int bb = -1, bcol = 0x7FFFFFFF;
+            for (int i = lane; i < nb; i += 32) {
+                const int ci = sw.bidx[i];
+                if (sw.w[ci] >= 0) continue;
+                const double e = sw.bex[i];
+                if (bb < 0 || e > bs || (e == bs && sw.col[ci] < bcol)) { bs = e; bb = ci; bcol = sw.col[ci]; }
+            }
 #pragma unroll
             for (int off = 16; off > 0; off >>= 1) {
-                const int ob = __shfl_xor_sync(0xffffffffu, best, off);
-                const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
-                if (ob < best) { best = ob; bi = oi; }
+                const double os = __shfl_xor_sync(0xffffffffu, bs, off);
+                const int ob = __shfl_xor_sync(0xffffffffu, bb, off);
+                const int oc = __shfl_xor_sync(0xffffffffu, bcol, off);
+                if (ob >= 0 && (bb < 0 || os > bs || (os == bs && oc < bcol))) { bs = os; bb = ob; bcol = oc; }
             }
-            if (bi < 0) break;
-            const int wv = -sw.w[bi];
+            if (bb < 0) break;
+            const int wv = -sw.w[bb];
             const int tk = wv < need ? wv : (int)need;
             __syncwarp();
-            if (lane == 0) sw.w[bi] = tk;
+            if (lane == 0) sw.w[bb] = tk;
             need -= tk;
             __syncwarp();
         }
         for (int i = lane; i < m; i += 32)
             if (sw.w[i] < 0) sw.w[i] = 0;
         __syncwarp();
+    } else if (tau > -CUDART_INF_F) {
+        // fewer than k keys among the candidates, but buckets below tau exist
+        if (lane == 0) push_fallback(a, row);
+        return;
     }
-    // chosen buckets packed (id << 5 | taken), compacted, sorted by id
-    int nsel = 0;
+    // emit keys in ascending bucket id (candidates are already in that order)
+    int run = 0;
     for (int base = 0; base < m; base += 32) {
         const int i = base + lane;
         const int tk = i < m ? sw.w[i] : 0;
-        const int col = i < m ? sw.col[i] : 0;
-        const unsigned bal = __ballot_sync(0xffffffffu, tk > 0);
-        __syncwarp();
-        if (tk > 0) sw.col[nsel + __popc(bal & ((1u << lane) - 1u))] = (col << 5) | tk;
-        nsel += __popc(bal);
-        __syncwarp();
-    }
-    int P = 1;
-    while (P < nsel) P <<= 1;
-    for (int i = nsel + lane; i < P; i += 32) sw.col[i] = 0x7FFFFFFF;
-    __syncwarp();
-    for (int k2 = 2; k2 <= P; k2 <<= 1) {
-        for (int j = k2 >> 1; j > 0; j >>= 1) {
-            for (int i = lane; i < P; i += 32) {
-                const int ixj = i ^ j;
-                if (ixj > i) {
-                    const int x = sw.col[i], y = sw.col[ixj];
-                    if ((x > y) == ((i & k2) == 0)) { sw.col[i] = y; sw.col[ixj] = x; }
-                }
-            }
-            __syncwarp();
-        }
-    }
-    // emit keys in ascending bucket id
-    int run = 0;
-    for (int base = 0; base < nsel; base += 32) {
-        const int i = base + lane;
-        const int pk = i < nsel ? sw.col[i] : 0;
-        const int tk = i < nsel ? (pk & 31) : 0;
         int incl = tk;
 #pragma unroll
         for (int off = 1; off < 32; off <<= 1) {
             const int y = __shfl_up_sync(0xffffffffu, incl, off);
             if (lane >= off) incl += y;
         }
-        if (tk > 0) emit_keys(a, h, pk >> 5, tk, lim, out + a.S + run + incl - tk);
+        if (tk > 0) emit_keys(a, h, sw.col[i], tk, lim, out + a.S + run + incl - tk);
         run += __shfl_sync(0xffffffffu, incl, 31);
     }
     for (int i = run + lane; i < a.k; i += 32) out[a.S + i] = -1;
@@ -508,7 +584,7 @@ lsa_status launch_flat(const PassArgs& pa, const ResolveArgs& ra, cudaStream_t s
     const int G = pa.agg ? pa.G : 1;
     const int qpt = 64 / G;
     dim3 grid((unsigned)ceil_div<int64_t>(pa.nqc, qpt), (unsigned)pa.hkv);
-    const size_t base = 2 * kPassCols * kDL * 2 + 4 * kPassCols * 4;
+    const size_t base = 2 * kPassCols * kDL * 2 + 4 * kPassCols * 4 + 64 * 4;
     const size_t smem_s = base + (size_t)qpt * kSBins * 4;
     const size_t smem_f = base + (size_t)qpt * 4;
     cudaFuncSetAttribute(flat_pass_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_s);
