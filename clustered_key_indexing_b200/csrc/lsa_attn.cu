@@ -72,18 +72,18 @@ __global__ void __launch_bounds__(32 * kAttnWarps) attn_kernel(AttnArgs a) {
     const uint16_t* Kg = a.K + g * kD;
     const uint16_t* Vg = a.V + g * kD;
 
+    // positions of one 16-key tile: lanes l and l+16 both hold entry l
     auto tile_pos = [&](int tile) -> int {
         const int e = tile * kTileKeys + (lane & 15);
-        int p = e < a.n_idx ? __ldg(list + e) : -1;
+        int p = (tile < ntiles && e < a.n_idx) ? __ldg(list + e) : -1;
         if (p >= a.T) {
             raise_device_error(kErrIndexRange);
             p = -1;
         }
         return p;
     };
-    auto issue = [&](int tile, int stage) {
+    auto issue = [&](int tile, int stage, int p) {
         if (tile < ntiles) {
-            const int p = tile_pos(tile);
             const uint32_t kb = wbase + stage * kStageBytes, vb = kb + kTileBytes;
 #pragma unroll
             for (int m = 0; m < 8; ++m) {
@@ -105,28 +105,34 @@ __global__ void __launch_bounds__(32 * kAttnWarps) attn_kernel(AttnArgs a) {
     float m_run[2] = {-CUDART_INF_F, -CUDART_INF_F};
     float l_run[2] = {0.f, 0.f};
 
-#pragma unroll
-    for (int s = 0; s < kStages - 1; ++s) issue(s, s);
+    static_assert(kStages == 3, "the position ring below holds 3 tiles");
+    // p0: tile i (being computed), p1: tile i+1, p2: tile i+2 (next to issue)
+    int p0 = tile_pos(0), p1 = tile_pos(1);
+    issue(0, 0, p0);
+    issue(1, 1, p1);
+    int p2 = tile_pos(2);
 
     for (int i = 0; i < ntiles; ++i) {
-        issue(i + kStages - 1, (i + kStages - 1) % kStages);
-        const int p = tile_pos(i);
-        const unsigned vmask = __ballot_sync(0xffffffffu, p >= 0) & 0xFFFFu;
+        issue(i + 2, (i + 2) % kStages, p2);
+        const int p3 = tile_pos(i + 3);  // consumed one iteration later
+        const unsigned vmask = __ballot_sync(0xffffffffu, p0 >= 0) & 0xFFFFu;
         cp_async_wait<kStages - 1>();
         __syncwarp();
         if (vmask != 0) {
             const int stage = i % kStages;
             const uint32_t kb = wbase + stage * kStageBytes, vb = kb + kTileBytes;
-            // S^T (16 keys x 8 heads)
-            float s[4] = {0.f, 0.f, 0.f, 0.f};
+            // S^T (16 keys x 8 heads): two independent accumulation chains
+            float sa[4] = {0.f, 0.f, 0.f, 0.f}, sb[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk) {
                 uint32_t af[4];
                 const int row = ((lane >> 3) & 1) * 8 + (lane & 7);
                 const int chunk = 2 * kk + (lane >> 4);
                 ldsm_x4(af, kb + swz(row, chunk));
-                mma_16816(s, af, qb[kk][0], qb[kk][1]);
+                if (kk & 1) mma_16816(sb, af, qb[kk][0], qb[kk][1]);
+                else mma_16816(sa, af, qb[kk][0], qb[kk][1]);
             }
+            float s[4] = {sa[0] + sb[0], sa[1] + sb[1], sa[2] + sb[2], sa[3] + sb[3]};
             const bool v0 = (vmask >> gq) & 1u, v1 = (vmask >> (gq + 8)) & 1u;
             s[0] = v0 ? s[0] * a.scale_log2 : -CUDART_INF_F;
             s[1] = v0 ? s[1] * a.scale_log2 : -CUDART_INF_F;
@@ -139,19 +145,24 @@ __global__ void __launch_bounds__(32 * kAttnWarps) attn_kernel(AttnArgs a) {
                 mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
             }
             const float mn0 = fmaxf(m_run[0], mx0), mn1 = fmaxf(m_run[1], mx1);
-            const float al0 = exp2f(m_run[0] - mn0), al1 = exp2f(m_run[1] - mn1);
-            m_run[0] = mn0;
-            m_run[1] = mn1;
-            const float p0 = exp2f(s[0] - mn0), p1 = exp2f(s[1] - mn1);
-            const float p2 = exp2f(s[2] - mn0), p3 = exp2f(s[3] - mn1);
-            l_run[0] = l_run[0] * al0 + (p0 + p2);
-            l_run[1] = l_run[1] * al1 + (p1 + p3);
+            const bool grew = __any_sync(0xffffffffu, mn0 != m_run[0] || mn1 != m_run[1]);
+            if (grew) {
+                const float al0 = exp2f(m_run[0] - mn0), al1 = exp2f(m_run[1] - mn1);
+                l_run[0] *= al0;
+                l_run[1] *= al1;
 #pragma unroll
-            for (int mt = 0; mt < 8; ++mt) {
-                o[mt][0] *= al0; o[mt][1] *= al1; o[mt][2] *= al0; o[mt][3] *= al1;
+                for (int mt = 0; mt < 8; ++mt) {
+                    o[mt][0] *= al0; o[mt][1] *= al1; o[mt][2] *= al0; o[mt][3] *= al1;
+                }
+                m_run[0] = mn0;
+                m_run[1] = mn1;
             }
+            const float e0 = exp2f(s[0] - mn0), e1 = exp2f(s[1] - mn1);
+            const float e2 = exp2f(s[2] - mn0), e3 = exp2f(s[3] - mn1);
+            l_run[0] += e0 + e2;
+            l_run[1] += e1 + e3;
             // P^T as B fragments: lane (head gq, tq) needs keys 2tq, 2tq+1, 2tq+8, 2tq+9
-            const uint32_t pk_lo = pack_bf16x2(p0, p1), pk_hi = pack_bf16x2(p2, p3);
+            const uint32_t pk_lo = pack_bf16x2(e0, e1), pk_hi = pack_bf16x2(e2, e3);
             const int src1 = (2 * tq) * 4 + (gq >> 1), src2 = (2 * tq + 1) * 4 + (gq >> 1);
             const uint32_t x1 = __shfl_sync(0xffffffffu, pk_lo, src1);
             const uint32_t x2 = __shfl_sync(0xffffffffu, pk_lo, src2);
@@ -170,6 +181,9 @@ __global__ void __launch_bounds__(32 * kAttnWarps) attn_kernel(AttnArgs a) {
             }
         }
         __syncwarp();
+        p0 = p1;
+        p1 = p2;
+        p2 = p3;
     }
     cp_async_wait<0>();
     __syncwarp();
