@@ -275,6 +275,7 @@ def run_lsa(args):
         dist.barrier()
     clocks = Clocks(torch.cuda.current_device())
     n0 = lib().lsa_launch_count()
+    lib().lsa_fallback_rows()  # reset the counter
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     torch.cuda.synchronize()
     ev0.record(stream)
@@ -289,6 +290,7 @@ def run_lsa(args):
     torch.cuda.synchronize()
     clk = clocks.stop()
     launches = lib().lsa_launch_count() - n0
+    fallback_rows = int(lib().lsa_fallback_rows())
     ms = ev0.elapsed_time(ev1)
     if world > 1:
         tt = torch.tensor([ms], device=dev)
@@ -355,6 +357,7 @@ def run_lsa(args):
             "gpu_launches": int(launches), "roofline": roofline, "cpu_baseline": cpu,
             "stages_ms_per_step": {"build": build_ms / args.steps, "select": sel_ms / args.steps,
                                    "attention": attn_ms / args.steps},
+            "select_fallback_rows_per_step": fallback_rows / args.steps,
         }
         print(json.dumps(line), flush=True)
     if world > 1:

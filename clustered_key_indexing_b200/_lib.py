@@ -60,6 +60,7 @@ def lib():
         L.lsa_last_error.restype = ctypes.c_char_p
         L.lsa_version.restype = ctypes.c_char_p
         L.lsa_launch_count.restype = i64
+        L.lsa_fallback_rows.restype = i64
         L.lsa_cfg_default.argtypes = [P(lsa_cfg)]
         L.lsa_cfg_check.argtypes = [P(lsa_cfg)]
         L.lsa_cache_units.argtypes = [P(lsa_cfg), i64]

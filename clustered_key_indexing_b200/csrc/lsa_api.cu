@@ -157,6 +157,13 @@ lsa_status lsa_tree_layout(int64_t n_buckets, lsa_tree* t) {
     return LSA_OK;
 }
 
+int64_t lsa_fallback_rows(void) {
+    unsigned long long v = 0ull, zero = 0ull;
+    if (cudaMemcpyFromSymbol(&v, g_lsa_fallback_rows, sizeof(v)) != cudaSuccess) return -1;
+    cudaMemcpyToSymbol(g_lsa_fallback_rows, &zero, sizeof(zero));
+    return (int64_t)v;
+}
+
 lsa_status lsa_check_device_error(void) {
     int v = 0;
     cudaError_t e = cudaMemcpyFromSymbol(&v, g_lsa_device_error, sizeof(int));

@@ -7,7 +7,7 @@
 // share the index list, so the warp computes S^T = K_sel Q^T with the keys as
 // the MMA's M dimension (16 keys per tile) and the heads as N (8 columns),
 // then O^T += V_sel^T P^T.  Keys are gathered 16 at a time with 16-byte
-// cp.async copies into a per-warp 3-stage shared-memory ring (16-byte chunks
+// cp.async copies into a per-warp 2-stage shared-memory ring (16-byte chunks
 // XOR-swizzled by row so ldmatrix reads are conflict-free); index tiles with
 // no valid entry are skipped.  Online softmax in fp32 (exp2 with the
 // log2(e)/sqrt(d) scale folded in), P rounded to bf16 for the PV product.
@@ -22,7 +22,7 @@
 namespace lsa {
 
 constexpr int kAttnWarps = 4;
-constexpr int kStages = 3;
+constexpr int kStages = 2;
 constexpr int kTileKeys = 16;
 constexpr int kTileBytes = kTileKeys * kD * 2;           // 4 KB per tensor
 constexpr int kStageBytes = 2 * kTileBytes;              // K + V
@@ -105,16 +105,15 @@ __global__ void __launch_bounds__(32 * kAttnWarps) attn_kernel(AttnArgs a) {
     float m_run[2] = {-CUDART_INF_F, -CUDART_INF_F};
     float l_run[2] = {0.f, 0.f};
 
-    static_assert(kStages == 3, "the position ring below holds 3 tiles");
-    // p0: tile i (being computed), p1: tile i+1, p2: tile i+2 (next to issue)
-    int p0 = tile_pos(0), p1 = tile_pos(1);
+    static_assert(kStages == 2, "the position ring below holds 2 tiles");
+    // p0: tile i (being computed), p1: tile i+1 (next to issue)
+    int p0 = tile_pos(0);
     issue(0, 0, p0);
-    issue(1, 1, p1);
-    int p2 = tile_pos(2);
+    int p1 = tile_pos(1);
 
     for (int i = 0; i < ntiles; ++i) {
-        issue(i + 2, (i + 2) % kStages, p2);
-        const int p3 = tile_pos(i + 3);  // consumed one iteration later
+        issue(i + 1, (i + 1) % kStages, p1);
+        const int p2 = tile_pos(i + 2);  // consumed one iteration later
         const unsigned vmask = __ballot_sync(0xffffffffu, p0 >= 0) & 0xFFFFu;
         cp_async_wait<kStages - 1>();
         __syncwarp();
@@ -183,7 +182,6 @@ __global__ void __launch_bounds__(32 * kAttnWarps) attn_kernel(AttnArgs a) {
         __syncwarp();
         p0 = p1;
         p1 = p2;
-        p2 = p3;
     }
     cp_async_wait<0>();
     __syncwarp();

@@ -34,6 +34,9 @@ enum DeviceError : int {
     kErrIndexRange = 3,       // an index list entry was >= T
 };
 
+// Rows of the flat search that took the exact fallback (diagnostics).
+__device__ unsigned long long g_lsa_fallback_rows = 0ull;
+
 __device__ __forceinline__ void raise_device_error(int code) {
     atomicCAS(&g_lsa_device_error, 0, code);
 }

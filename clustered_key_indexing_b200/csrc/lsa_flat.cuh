@@ -375,6 +375,7 @@ __device__ __forceinline__ double exact_row(const uint16_t* ylat, int ng, const 
 }
 
 __device__ __forceinline__ void push_fallback(const ResolveArgs& a, int64_t row) {
+    atomicAdd(&g_lsa_fallback_rows, 1ull);
     const int slot = atomicAdd(a.ovf_count, 1);
     if (slot < a.ovf_cap) a.ovf_rows[slot] = (int32_t)row;
     else raise_device_error(kErrSelectOverflow);

@@ -467,7 +467,7 @@ __global__ void __launch_bounds__(kSelThreads) select_fallback_kernel(SelectArgs
         for (int64_t b = tid; b < ncol; b += kSelThreads) {
             const bool el = (int64_t)a.minlr[hb0 + b] <= r.lim;
             fw[b] = el ? bucket_weight(a, r.h, b, r.lim) : 0;
-            fs[b] = el ? exact_score(sh.ylat, ng, a.cent + (hb0 + b) * kDL) : 0.0;
+            fs[b] = el ? exact_row(sh.ylat, ng, a.cent + (hb0 + b) * kDL) : 0.0;
         }
         __syncthreads();
         // taken counts are written back into fw

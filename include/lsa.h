@@ -134,6 +134,9 @@ lsa_status lsa_tree_layout(int64_t n_buckets, lsa_tree* tree);
 /* Kernels this library has launched in this process (host-side counter,
  * for diagnostics and launch accounting). */
 int64_t lsa_launch_count(void);
+/* Flat-search rows (query, kv-head) that took the exact fallback since the
+ * last call, on the current device (diagnostics; synchronous; -1 on error). */
+int64_t lsa_fallback_rows(void);
 /* Read back and clear the device-side error word of the current device:
  * LSA_OK, or LSA_EDEVICE with a description in lsa_last_error(). Synchronous. */
 lsa_status lsa_check_device_error(void);
