@@ -78,9 +78,11 @@ class Cache:
         self.maxpos = torch.zeros((hkv, self.cap_buckets), dtype=torch.int32, **z)
         self.sum = torch.zeros((hkv, self.cap_buckets, dl), dtype=torch.float64, **z)
         self.cent = torch.zeros((hkv, self.cap_buckets, dl), dtype=torch.bfloat16, **z)
+        self.units = torch.zeros((hkv, self.cap_buckets), dtype=torch.int32, **z)
         self.c = _lib.lsa_cache(hkv, 0, self.cap_units, self.cap_buckets, *[
             t.data_ptr() for t in (self.U, self.bucket_of_unit, self.members, self.offsets,
-                                   self.cnt_lr, self.minlr, self.maxpos, self.sum, self.cent)])
+                                   self.cnt_lr, self.minlr, self.maxpos, self.sum, self.cent,
+                                   self.units)])
 
     @property
     def n_tokens(self) -> int:

@@ -91,7 +91,7 @@ static lsa_status check_cache(const lsa_cache* c, bool need_built) {
     if (!c) return set_error(LSA_EINVAL, "cache is NULL");
     if (c->hkv <= 0) return set_error(LSA_EINVAL, "cache: hkv must be positive");
     if (!c->U || !c->bucket_of_unit || !c->members || !c->offsets || !c->cnt_lr || !c->minlr ||
-        !c->maxpos || !c->sum || !c->cent)
+        !c->maxpos || !c->sum || !c->cent || !c->units)
         return set_error(LSA_EINVAL, "cache: a device array is NULL");
     if (c->cap_units <= 0 || c->cap_buckets <= 0) return set_error(LSA_EINVAL, "cache: capacities must be positive");
     if (c->cap_buckets < ceil_div<int64_t>(c->cap_units, kUnitsPerBlock) * kBucketsPerBlock)

@@ -234,6 +234,7 @@ struct WardArgs {
     int32_t* maxpos;
     double* sum;
     uint16_t* cent;
+    int32_t* units;
 };
 
 __device__ __forceinline__ int tri_index(int i, int j) {  // i < j < 128
@@ -461,6 +462,9 @@ __global__ void __launch_bounds__(128, 1) ward_kernel(WardArgs a) {
                 if (p >= a.sinks) { ++c_lr; if (p < mlr) mlr = (int32_t)p; }
             }
         }
+        int32_t pk = sz << 28;
+        for (int i = 0; i < sz; ++i) pk |= mem_[tid][i] << (7 * i);
+        a.units[hb0 + b] = pk;
         a.cnt_lr[hb0 + b] = c_lr;
         a.minlr[hb0 + b] = mlr;
         a.maxpos[hb0 + b] = mxp;
@@ -483,6 +487,7 @@ __global__ void __launch_bounds__(128, 1) ward_kernel(WardArgs a) {
         a.cnt_lr[hb0 + b] = 0;
         a.minlr[hb0 + b] = kIMax;
         a.maxpos[hb0 + b] = -1;
+        a.units[hb0 + b] = 0;
         for (int c = 0; c < kDL; ++c) {
             a.sum[(hb0 + b) * kDL + c] = 0.0;
             a.cent[(hb0 + b) * kDL + c] = 0;
@@ -499,6 +504,7 @@ lsa_status launch_ward(const lsa_cache* c, int64_t T, int32_t sinks, int64_t blk
     a.NU = ceil_div<int64_t>(T, kPool); a.T = T; a.sinks = sinks; a.blk0 = blk0;
     a.bucket_of_unit = c->bucket_of_unit; a.members = c->members; a.offsets = c->offsets;
     a.cnt_lr = c->cnt_lr; a.minlr = c->minlr; a.maxpos = c->maxpos; a.sum = c->sum; a.cent = c->cent;
+    a.units = c->units;
     const size_t smem = sizeof(double) * (2 * kDL * kWT + kUnitsPerBlock * (kUnitsPerBlock - 1) / 2);
     cudaFuncSetAttribute(ward_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     dim3 grid((unsigned)(blk1 - blk0), (unsigned)c->hkv);
@@ -508,8 +514,8 @@ lsa_status launch_ward(const lsa_cache* c, int64_t T, int32_t sinks, int64_t blk
 
 // Mark bucket slots [b0, b1) of every head empty.
 __global__ void clear_slots_kernel(int32_t* cnt_lr, int32_t* minlr, int32_t* maxpos, double* sum,
-                                   uint16_t* cent, int64_t cap_buckets, int64_t b0, int64_t b1,
-                                   int32_t hkv) {
+                                   uint16_t* cent, int32_t* units, int64_t cap_buckets, int64_t b0,
+                                   int64_t b1, int32_t hkv) {
     const int64_t span = b1 - b0;
     const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     if (i >= span * hkv * kDL) return;
@@ -522,6 +528,7 @@ __global__ void clear_slots_kernel(int32_t* cnt_lr, int32_t* minlr, int32_t* max
         cnt_lr[hb] = 0;
         minlr[hb] = kIMax;
         maxpos[hb] = -1;
+        units[hb] = 0;
     }
 }
 
@@ -529,7 +536,7 @@ lsa_status launch_clear_slots(const lsa_cache* c, int64_t b0, int64_t b1, cudaSt
     if (b1 <= b0) return LSA_OK;
     const int64_t n = (b1 - b0) * c->hkv * kDL;
     clear_slots_kernel<<<(unsigned)ceil_div<int64_t>(n, 256), 256, 0, st>>>(
-        c->cnt_lr, c->minlr, c->maxpos, c->sum, c->cent, c->cap_buckets, b0, b1, c->hkv);
+        c->cnt_lr, c->minlr, c->maxpos, c->sum, c->cent, c->units, c->cap_buckets, b0, b1, c->hkv);
     return check_launch("clear_slots_kernel");
 }
 

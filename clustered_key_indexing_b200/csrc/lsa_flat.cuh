@@ -4,7 +4,7 @@
 //
 // Three kernels per chunk of query positions:
 //   flat_pass_kernel<sample=true>   bf16 tensor-core scores (mma.sync
-//       m16n8k16, fp32 accumulate) of 64 query rows against every 16th
+//       m16n8k16, fp32 accumulate) of 64 query rows against every 8th
 //       centroid; a per-row weighted histogram of those scores (bins scaled to
 //       the row's latent norm, which bounds its scores) gives a threshold tau
 //       expected to keep about twice the k keys needed;
@@ -32,7 +32,7 @@
 namespace lsa {
 
 constexpr int kCandCap = 1024;       // candidates kept per (query, kv-head)
-constexpr int kSampleStride = 16;    // every 16th bucket scored by the sample pass
+constexpr int kSampleStride = 8;     // every 8th bucket scored by the sample pass
 constexpr int kSBins = 256;          // sample histogram bins over [-R, R], R = row latent norm
 constexpr int kOversample = 2;       // tau targets kOversample * k keys
 constexpr float kScoreErr = 1e-4f;   // bound on |fp32 score - exact score|
@@ -273,6 +273,7 @@ __global__ void __launch_bounds__(128) flat_pass_kernel(PassArgs a) {
 constexpr int kResWarps = 4;
 
 struct ResolveArgs {
+    const int32_t* units;
     const int32_t* offsets;
     const int32_t* members;
     const int32_t* cnt_lr;
@@ -300,6 +301,7 @@ struct ResWarp {
     int32_t col[kCandCap];    // eligible candidates, ascending bucket id
     float sc[kCandCap];       // their fp32 scores
     int32_t w[kCandCap];      // key weights, then taken counts
+    int32_t pk[kCandCap];     // packed member units
     int32_t bidx[kBandCap];   // band members (index into col)
     uint32_t hist[256];
     uint16_t ylat[8 * kDL];
@@ -310,41 +312,39 @@ __device__ __forceinline__ uint32_t order_key_f(float s) {
     return (u >> 31) ? ~u : (u | 0x80000000u);
 }
 
-__device__ int weight_of(const ResolveArgs& a, int h, int64_t b, int64_t lim) {
-    const int64_t hb = (int64_t)h * a.cap_buckets + b;
-    if ((int64_t)a.maxpos[hb] <= lim) return a.cnt_lr[hb];
-    const int32_t* off = a.offsets + (int64_t)h * (a.cap_buckets + 1);
-    const int32_t* mem = a.members + (int64_t)h * a.cap_units;
+// Keys of bucket b in [S, lim]; `pk` is the bucket's packed member units.
+__device__ __forceinline__ int weight_packed(const ResolveArgs& a, int64_t b, int32_t pk, int64_t lim) {
+    const int64_t ubase = (b / kBucketsPerBlock) * kUnitsPerBlock;
+    const int cnt = (pk >> 28) & 7;
     int w = 0;
-    for (int32_t m = off[b]; m < off[b + 1]; ++m) {
-        const int64_t j = mem[m];
+    for (int i = 0; i < cnt; ++i) {
+        const int64_t j = ubase + ((pk >> (7 * i)) & 127);
         for (int64_t p = j * kPool; p < j * kPool + kPool && p < a.T_built; ++p)
             if (p >= a.S && p <= lim) ++w;
     }
     return w;
 }
 
-// First `tk` keys of bucket b in [S, lim], ascending.  Fast path: a bucket
-// that is taken whole, lies entirely inside [S, lim] and has full units
-// writes 4 consecutive positions per member unit.
-__device__ void emit_keys(const ResolveArgs& a, int h, int64_t b, int tk, int64_t lim, int32_t* out) {
-    const int32_t* off = a.offsets + (int64_t)h * (a.cap_buckets + 1);
-    const int32_t* mem = a.members + (int64_t)h * a.cap_units;
-    const int64_t hb = (int64_t)h * a.cap_buckets + b;
-    const int32_t m0 = off[b], m1 = off[b + 1];
-    if (tk == (m1 - m0) * kPool && (int64_t)a.maxpos[hb] <= lim && a.minlr[hb] == mem[m0] * kPool &&
-        a.maxpos[hb] < a.T_built) {
+// First `tk` keys of bucket b in [S, lim], ascending (member units are
+// packed in ascending order).  Fast path: a bucket taken whole that lies
+// inside [S, lim] with full units writes 4 consecutive positions per unit.
+__device__ void emit_keys(const ResolveArgs& a, int64_t b, int32_t pk, int tk, int64_t lim,
+                          int32_t* out) {
+    const int64_t ubase = (b / kBucketsPerBlock) * kUnitsPerBlock;
+    const int cnt = (pk >> 28) & 7;
+    const int64_t j0 = ubase + (pk & 127);
+    if (tk == cnt * kPool && j0 * kPool >= a.S) {
         int o = 0;
-        for (int32_t m = m0; m < m1; ++m) {
-            const int32_t p = mem[m] * kPool;
+        for (int i = 0; i < cnt; ++i) {
+            const int32_t p = (int32_t)((ubase + ((pk >> (7 * i)) & 127)) * kPool);
             out[o] = p; out[o + 1] = p + 1; out[o + 2] = p + 2; out[o + 3] = p + 3;
             o += 4;
         }
         return;
     }
     int o = 0;
-    for (int32_t m = m0; m < m1 && o < tk; ++m) {
-        const int64_t j = mem[m];
+    for (int i = 0; i < cnt && o < tk; ++i) {
+        const int64_t j = ubase + ((pk >> (7 * i)) & 127);
         for (int64_t p = j * kPool; p < j * kPool + kPool && p < a.T_built && o < tk; ++p)
             if (p >= a.S && p <= lim) out[o++] = (int32_t)p;
     }
@@ -418,21 +418,24 @@ __global__ void __launch_bounds__(32 * kResWarps, 4) flat_resolve_kernel(Resolve
         bool el = false;
         int col = 0, wgt = 0;
         float sc = 0.f;
+        int32_t pk = 0;
         if (i < n) {
             col = a.cand_col[row * kCandCap + i];
             sc = a.cand_s[row * kCandCap + i];
-            el = (int64_t)a.minlr[hb0 + col] <= lim;
+            const int64_t hb = hb0 + col;
+            const int32_t mlr = a.minlr[hb], mxp = a.maxpos[hb], clr = a.cnt_lr[hb];
+            pk = a.units[hb];
+            el = (int64_t)mlr <= lim;
+            wgt = (int64_t)mxp <= lim ? clr : weight_packed(a, col, pk, lim);
         }
-        if (el) {
-            wgt = weight_of(a, h, col, lim);
-            wtot += wgt;
-        }
+        if (el) wtot += wgt;
         const unsigned bal = __ballot_sync(0xffffffffu, el);
         if (el) {
             const int pos = m + __popc(bal & ((1u << lane) - 1u));
             sw.col[pos] = col;
             sw.sc[pos] = sc;
             sw.w[pos] = wgt;
+            sw.pk[pos] = pk;
         }
         m += __popc(bal);
     }
@@ -573,7 +576,7 @@ __global__ void __launch_bounds__(32 * kResWarps, 4) flat_resolve_kernel(Resolve
             const int y = __shfl_up_sync(0xffffffffu, incl, off);
             if (lane >= off) incl += y;
         }
-        if (tk > 0) emit_keys(a, h, sw.col[i], tk, lim, out + a.S + run + incl - tk);
+        if (tk > 0) emit_keys(a, sw.col[i], sw.pk[i], tk, lim, out + a.S + run + incl - tk);
         run += __shfl_sync(0xffffffffu, incl, 31);
     }
     for (int i = run + lane; i < a.k; i += 32) out[a.S + i] = -1;

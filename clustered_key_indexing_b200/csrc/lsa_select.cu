@@ -598,7 +598,7 @@ lsa_status run_select(const uint16_t* Q, int64_t t0, int64_t nq, int32_t hq, con
         pa.W = cfg->window; pa.hkv = hkv; pa.G = hq / hkv; pa.agg = cfg->agg; pa.k = cfg->k;
         pa.tau = w.tau; pa.cand_col = w.cand_col; pa.cand_s = w.cand_s; pa.cand_n = w.cand_n;
         ResolveArgs ra{};
-        ra.offsets = c->offsets; ra.members = c->members; ra.cnt_lr = c->cnt_lr; ra.minlr = c->minlr;
+        ra.units = c->units; ra.offsets = c->offsets; ra.members = c->members; ra.cnt_lr = c->cnt_lr; ra.minlr = c->minlr;
         ra.maxpos = c->maxpos; ra.cent = c->cent; ra.cap_units = c->cap_units;
         ra.cap_buckets = c->cap_buckets; ra.NB = NB; ra.T_built = c->n_tokens;
         ra.hkv = hkv; ra.G = hq / hkv; ra.agg = cfg->agg; ra.k = cfg->k; ra.S = cfg->sinks;

@@ -95,6 +95,9 @@ typedef struct lsa_cache {
     int32_t*  maxpos;          /* [hkv, cap_buckets] largest key                  */
     double*   sum;             /* [hkv, cap_buckets, d_latent] fp64 unit sums     */
     uint16_t* cent;            /* [hkv, cap_buckets, d_latent] bf16 centroids     */
+    int32_t*  units;           /* [hkv, cap_buckets] member units packed: bits
+                                  7i..7i+6 = i-th member's unit index within its
+                                  128-unit block (ascending), bits 28..30 = count */
 } lsa_cache;
 
 #define LSA_MAX_LEVELS 48

@@ -63,7 +63,7 @@ def test_sizes_and_tree_layout(L):
     assert [t.level_n[i] for i in range(t.levels)] == [5, 3, 2, 1]
     assert [t.level_off[i] for i in range(t.levels)] == [0, 5, 8, 10]
     assert L.lsa_tree_layout(0, ctypes.byref(t)) == LSA_EINVAL
-    cache = lsa_cache(8, 131072, 32768, 16384, *([16] * 9))
+    cache = lsa_cache(8, 131072, 32768, 16384, *([16] * 10))
     assert L.lsa_select_workspace_bytes(ctypes.byref(c), 131072, 32, ctypes.byref(cache)) > 0
     assert L.lsa_prefill_workspace_bytes(ctypes.byref(c), 131072, 32, 8, 16384) > 0
 
@@ -73,7 +73,7 @@ def test_compute_calls_reject_bad_arguments_before_any_launch(L):
     L.lsa_cfg_default(ctypes.byref(c))
     # NULL cache / NULL tensors / bad head ratio: refused on the host
     assert L.lsa_build_buckets(None, 16, 1, None, ctypes.byref(c), None, None) == LSA_EINVAL
-    cache = lsa_cache(1, 0, 4, 64, *([0] * 9))
+    cache = lsa_cache(1, 0, 4, 64, *([0] * 10))
     assert L.lsa_build_buckets(None, 16, 1, None, ctypes.byref(c), ctypes.byref(cache), None) == LSA_EINVAL
     assert L.lsa_sparse_attn(None, None, None, None, 1, 3, 2, 8, 16, None, None) == LSA_EINVAL
     assert L.lsa_sparse_attn(None, None, None, None, 1, 48, 4, 8, 16, None, None) == LSA_EUNSUPPORTED

@@ -41,7 +41,20 @@ def _build_both(lsa, name, T, cfg, seed=0):
     return inp, cache, U, oc
 
 
+def _assert_units_match_members(cache, oc):
+    """The packed member-unit words decode to the oracle's CSR members."""
+    units = cache.units[:, :oc["NB"]].cpu().numpy()
+    for h in range(units.shape[0]):
+        for b in range(oc["NB"]):
+            pk = int(units[h, b])
+            cnt = (pk >> 28) & 7
+            got = [(b // 64) * 128 + ((pk >> (7 * i)) & 127) for i in range(cnt)]
+            want = oc["members"][h, oc["offsets"][h, b]:oc["offsets"][h, b + 1]].tolist()
+            assert got == want, (h, b)
+
+
 def _assert_cache_equal(cache, U, oc):
+    _assert_units_match_members(cache, oc)
     g = cache_arrays(cache, oc["NB"])
     assert np.array_equal(g["U"].view(np.uint64), U.view(np.uint64)), "pooled latents differ"
     assert np.array_equal(g["sum"].view(np.uint64), oc["sum"].view(np.uint64)), "bucket sums differ"
