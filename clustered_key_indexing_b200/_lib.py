@@ -76,6 +76,9 @@ def lib():
         L.lsa_select_workspace_bytes.restype = sz
         L.lsa_select.argtypes = [vp, i64, i64, i32, vp, P(lsa_cache), P(lsa_tree), P(lsa_cfg),
                                  vp, vp, vp, sz, vp]
+        L.lsa_select_noalloc.argtypes = [vp, i64, i64, i32, vp, P(lsa_cache), P(lsa_tree),
+                                         P(lsa_cfg), vp, vp]
+        L.lsa_select_noalloc_scratch_bytes.restype = sz
         L.lsa_sparse_attn.argtypes = [vp, vp, vp, vp, i64, i32, i32, i32, i64, vp, vp]
         L.lsa_prefill_workspace_bytes.argtypes = [P(lsa_cfg), i64, i32, i32, i64]
         L.lsa_prefill_workspace_bytes.restype = sz

@@ -4,3 +4,4 @@
 #include "lsa_select.cu"
 #include "lsa_attn.cu"
 #include "lsa_api.cu"
+#include "lsa_noalloc.cu"

@@ -225,6 +225,35 @@ lsa_status lsa_sparse_attn(const uint16_t* Q, const uint16_t* K,
                            int32_t hq, int32_t hkv, int32_t n_idx, int64_t T,
                            uint16_t* O, void* stream);
 
+/* ---------------------------------------------- selection without ws */
+
+/*
+ * lsa_select_noalloc -- lsa_select for callers that cannot allocate device
+ * memory (a host framework that owns all device memory through its own
+ * pool, or a latency-critical path that must not call cudaMalloc).  The
+ * pages have no counterpart of this call; it is a deployment convenience.
+ * Same arguments and results as lsa_select, minus Y_out and the workspace:
+ * the scratch is one built-in device array of
+ * lsa_select_noalloc_scratch_bytes() bytes (64 MiB) that every GPU loading
+ * this library reserves until the process exits.
+ *   - A request whose lsa_select_workspace_bytes() exceeds that size is
+ *     refused with LSA_ENOSPACE (split the query range into smaller calls;
+ *     e.g. 512 queries fit at 131072 keys x 8 kv-heads).
+ *   - The first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress, with that device current); make that first
+ *     call before any stream capture.
+ *   - Every call shares the one array: calls that can overlap on the GPU
+ *     (different streams, different host threads) race and must be
+ *     serialised by the caller.
+ *   - Allocates nothing: no cudaMalloc, cudaFree or allocating library call.
+ */
+lsa_status lsa_select_noalloc(const uint16_t* Q, int64_t t0, int64_t nq, int32_t hq,
+                              const float* W_q, const lsa_cache* cache,
+                              const lsa_tree* tree, const lsa_cfg* cfg, int32_t* idx,
+                              void* stream);
+/* Size in bytes of lsa_select_noalloc's built-in scratch array. */
+size_t lsa_select_noalloc_scratch_bytes(void);
+
 /* --------------------------------------------------- whole-layer prefill */
 
 /* Workspace bytes lsa_prefill needs (T tokens, queries processed in chunks
