@@ -37,6 +37,12 @@ import synth  # noqa: E402
 METRIC = "LSA layer prefill tokens/s"
 UNIT = "tokens/s"
 
+# DRAM bytes per (query, kv-head) of attn_kernel from the ncu capture in
+# profiles/attn_kernel_prefill-128k.md; reported as `traffic` only while the
+# kernel source is the one that capture measured.
+ATTN_TRAFFIC = {"sha256_prefix": "5fead07e225b0b47", "bytes_per_query_kvhead": 40295.4,
+                "source": "clustered_key_indexing_b200/csrc/lsa_attn.cu", "workload": "prefill-128k"}
+
 
 def parse():
     p = argparse.ArgumentParser()
@@ -337,8 +343,18 @@ def run_lsa(args):
     pk, src = peaks()
     attn_ms_launch = attn_ms / (args.steps * len(chunks))
     achieved = (attn_bytes / len(chunks)) / (attn_ms_launch / 1e3) / 1e9
+    traffic = None
+    try:
+        import hashlib
+        src = open(os.path.join(ROOT, ATTN_TRAFFIC["source"]), "rb").read()
+        if (hashlib.sha256(src).hexdigest()[:16] == ATTN_TRAFFIC["sha256_prefix"]
+                and args.workload == ATTN_TRAFFIC["workload"]):
+            traffic = ATTN_TRAFFIC["bytes_per_query_kvhead"] * chunk * hkv
+    except OSError:
+        pass
     roofline = {"kernel": "attn_kernel", "bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"],
-                "unit": "GB/s", "frac": achieved / pk["hbm_gbs"], "traffic": None,
+                "unit": "GB/s", "frac": achieved / pk["hbm_gbs"], "traffic": traffic,
+                "traffic_note": "ncu DRAM bytes per launch, scaled from a 2048-position launch",
                 "peak_source": src, "attn_share_of_step": attn_ms / ms if ms > 0 else None,
                 "bytes_per_launch": attn_bytes / len(chunks)}
 
