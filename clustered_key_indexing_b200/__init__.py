@@ -4,9 +4,9 @@ Thin PyTorch-facing binding of liblsa.so (include/lsa.h).  PyTorch only
 allocates device memory and provides streams; every step runs in the
 library's CUDA kernels.  See `api` for the calls.
 """
-from .api import (Cache, Config, Tree, build_buckets, build_tree, prefill, prefill_workspace_bytes,
+from .api import (Cache, Config, Decode, Tree, build_buckets, build_tree, prefill, prefill_workspace_bytes,
                   query_latent, select, select_workspace_bytes, sparse_attn, check_device_error)
 
-__all__ = ["Cache", "Config", "Tree", "build_buckets", "build_tree", "prefill",
+__all__ = ["Cache", "Config", "Decode", "Tree", "build_buckets", "build_tree", "prefill",
            "prefill_workspace_bytes", "query_latent", "select", "select_workspace_bytes",
            "sparse_attn", "check_device_error"]

@@ -39,6 +39,14 @@ class lsa_tree(ctypes.Structure):
                 ("n_nodes", i64), ("sum", vp), ("minlr", vp), ("cent", vp)]
 
 
+MAX_BATCH = 128
+
+
+class lsa_decode(ctypes.Structure):
+    _fields_ = [("batch", i32), ("hkv", i32), ("hq", i32), ("cap", i64), ("K", vp), ("V", vp),
+                ("U_blk", vp), ("cache", lsa_cache), ("tree", lsa_tree), ("len", i64 * MAX_BATCH)]
+
+
 class LSAError(RuntimeError):
     def __init__(self, status: int, msg: str):
         super().__init__(f"{STATUS_NAMES.get(status, status)}: {msg}")
@@ -80,6 +88,10 @@ def lib():
                                          P(lsa_cfg), vp, vp]
         L.lsa_select_noalloc_scratch_bytes.restype = sz
         L.lsa_sparse_attn.argtypes = [vp, vp, vp, vp, i64, i32, i32, i32, i64, vp, vp]
+        L.lsa_decode_workspace_bytes.argtypes = [P(lsa_cfg), P(lsa_decode)]
+        L.lsa_decode_workspace_bytes.restype = sz
+        L.lsa_decode_load.argtypes = [P(lsa_decode), i32, i64, vp, P(lsa_cfg), vp, sz, vp]
+        L.lsa_decode_step.argtypes = [P(lsa_decode), vp, vp, vp, vp, vp, P(lsa_cfg), vp, vp, vp, sz, vp]
         L.lsa_prefill_workspace_bytes.argtypes = [P(lsa_cfg), i64, i32, i32, i64]
         L.lsa_prefill_workspace_bytes.restype = sz
         L.lsa_prefill.argtypes = [vp, vp, vp, i64, i32, i32, vp, vp, P(lsa_cfg), P(lsa_cache),

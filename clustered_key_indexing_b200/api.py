@@ -60,7 +60,8 @@ class Cache:
     """Device arrays of one layer's bucket cache (lsa_cache), sized for
     `cap_tokens` tokens per head."""
 
-    def __init__(self, hkv: int, cap_tokens: int, cfg: Config | None = None, device="cuda"):
+    def __init__(self, hkv: int, cap_tokens: int, cfg: Config | None = None, device="cuda",
+                 with_units: bool = True):
         cfg = cfg or Config()
         cc = cfg.c()
         L = lib()
@@ -69,7 +70,8 @@ class Cache:
         self.cap_buckets = int(L.lsa_cache_buckets(ctypes.byref(cc), cap_tokens))
         dl = cfg.d_latent
         z = dict(device=device)
-        self.U = torch.zeros((hkv, self.cap_units, dl), dtype=torch.float64, **z)
+        # pooled unit latents (the decode state keeps only a block ring instead)
+        self.U = torch.zeros((hkv, self.cap_units if with_units else 1, dl), dtype=torch.float64, **z)
         self.bucket_of_unit = torch.full((hkv, self.cap_units), -1, dtype=torch.int32, **z)
         self.members = torch.full((hkv, self.cap_units), -1, dtype=torch.int32, **z)
         self.offsets = torch.zeros((hkv, self.cap_buckets + 1), dtype=torch.int32, **z)
@@ -97,7 +99,7 @@ class Cache:
 class Tree:
     """Device arrays of the binary centroid tree (lsa_tree) over a cache."""
 
-    def __init__(self, cache: Cache, device="cuda"):
+    def __init__(self, cache: "Cache", device="cuda"):
         self.t = _lib.lsa_tree()
         check(lib().lsa_tree_layout(cache.cap_buckets, ctypes.byref(self.t)), "lsa_tree_layout")
         n, hkv = int(self.t.n_nodes), cache.hkv
@@ -208,3 +210,54 @@ def prefill(Q, K, V, W_k, W_q, cfg: Config, cache: Cache | None = None, tree: Tr
                             ctypes.byref(tree.t) if tree is not None else None, _ptr(O), chunk,
                             _ptr(ws), ws.numel(), _stream(stream)), "lsa_prefill")
     return O
+
+
+class Decode:
+    """Batched decode state (lsa_decode): `batch` requests of `cap` tokens,
+    K/V pools [batch, cap, hkv, 128], a cache whose heads are
+    (request, kv-head) pairs, the per-request block ring, and (tree mode) the
+    tree.  `load` installs a prompt, `step` decodes one token per request."""
+
+    def __init__(self, batch: int, hkv: int, hq: int, cap: int, cfg: Config, device="cuda"):
+        if cap % 512:
+            raise ValueError("cap must be a multiple of 512")
+        self.cfg = cfg
+        z = dict(device=device)
+        self.K = torch.zeros((batch, cap, hkv, 128), dtype=torch.bfloat16, **z)
+        self.V = torch.zeros((batch, cap, hkv, 128), dtype=torch.bfloat16, **z)
+        self.U_blk = torch.zeros((batch * hkv, 128, 64), dtype=torch.float64, **z)
+        self.cache = Cache(batch * hkv, cap, cfg, device=device, with_units=False)
+        self.tree = Tree(self.cache, device=device) if cfg.mode == 1 else None
+        d = _lib.lsa_decode()
+        d.batch, d.hkv, d.hq, d.cap = batch, hkv, hq, cap
+        d.K, d.V, d.U_blk = self.K.data_ptr(), self.V.data_ptr(), self.U_blk.data_ptr()
+        d.cache = self.cache.c
+        if self.tree is not None:
+            d.tree = self.tree.t
+        self.d = d
+        need = int(lib().lsa_decode_workspace_bytes(ctypes.byref(cfg.c()), ctypes.byref(d)))
+        if need == 0:
+            check(_lib.LSA_EINVAL, "lsa_decode_workspace_bytes")
+        self.ws = torch.empty(need, dtype=torch.uint8, **z)
+
+    @property
+    def len(self):
+        return [int(self.d.len[i]) for i in range(self.d.batch)]
+
+    def load(self, r: int, K: torch.Tensor, V: torch.Tensor, W_k: torch.Tensor, stream=None):
+        """Install a prompt (K/V [n, hkv, 128]) as request r."""
+        n = K.shape[0]
+        self.K[r, :n].copy_(K)
+        self.V[r, :n].copy_(V)
+        check(lib().lsa_decode_load(ctypes.byref(self.d), r, n, _ptr(W_k), ctypes.byref(self.cfg.c()),
+                                    _ptr(self.ws), self.ws.numel(), _stream(stream)), "lsa_decode_load")
+
+    def step(self, q, k, v, W_k, W_q, o=None, idx_out=None, stream=None):
+        """One token per request: q [batch, hq, 128], k/v [batch, hkv, 128]."""
+        _need_cuda(q, k, v, W_k, W_q)
+        if o is None:
+            o = torch.empty_like(q)
+        check(lib().lsa_decode_step(ctypes.byref(self.d), _ptr(q), _ptr(k), _ptr(v), _ptr(W_k), _ptr(W_q),
+                                    ctypes.byref(self.cfg.c()), _ptr(o), _ptr(idx_out), _ptr(self.ws),
+                                    self.ws.numel(), _stream(stream)), "lsa_decode_step")
+        return o

@@ -53,7 +53,7 @@ lsa_status run_select(const uint16_t* Q, int64_t t0, int64_t nq, int32_t hq, con
                       uint16_t* Y_out, void* ws, size_t ws_bytes, cudaStream_t st);
 lsa_status launch_attn(const uint16_t* Q, const uint16_t* K, const uint16_t* V, const int32_t* idx,
                        int64_t nq, int32_t hq, int32_t hkv, int32_t n_idx, int64_t T, uint16_t* O,
-                       cudaStream_t st);
+                       cudaStream_t st, int64_t kv_q_stride, int split);
 
 static lsa_status check_cfg(const lsa_cfg* c) {
     if (!c) return set_error(LSA_EINVAL, "cfg is NULL");

@@ -13,6 +13,7 @@
 // log2(e)/sqrt(d) scale folded in), P rounded to bf16 for the PV product.
 // Warps are ordered kv-head-major so the warps resident at one time read one
 // head's K/V, which keeps that head's rows in L2.
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -35,7 +36,8 @@ struct AttnArgs {
     const int32_t* idx;
     int64_t nq;
     int32_t hq, hkv, n_idx;
-    int64_t T;
+    int64_t T;            // index entries must be < T
+    int64_t kv_q_stride;  // token rows of K/V per query row (decode: each request's capacity); 0 = shared
     uint16_t* O;
     float scale_log2;
 };
@@ -44,10 +46,15 @@ __device__ __forceinline__ uint32_t swz(int row, int chunk) {
     return (uint32_t)(row * (kD * 2) + ((chunk ^ (row & 7)) << 4));
 }
 
-__global__ void __launch_bounds__(32 * kAttnWarps) attn_kernel(AttnArgs a) {
+// SPLIT == 1: one warp per (query, kv-head), 4 warps per CTA (prefill).
+// SPLIT > 1: SPLIT warps share one (query, kv-head) row, each taking a
+// contiguous slice of its index tiles; partial softmax states are combined
+// through shared memory (decode, where rows are few).
+template <int SPLIT>
+__global__ void __launch_bounds__(32 * (SPLIT == 1 ? kAttnWarps : SPLIT)) attn_kernel(AttnArgs a) {
     extern __shared__ __align__(128) uint8_t asmem[];
     const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
-    const int64_t wg = (int64_t)blockIdx.x * kAttnWarps + wid;
+    const int64_t wg = SPLIT == 1 ? (int64_t)blockIdx.x * kAttnWarps + wid : (int64_t)blockIdx.x;
     if (wg >= a.nq * a.hkv) return;
     const int64_t g = wg / a.nq, q = wg % a.nq;  // kv-head major
     const int G = a.hq / a.hkv;
@@ -67,10 +74,12 @@ __global__ void __launch_bounds__(32 * kAttnWarps) attn_kernel(AttnArgs a) {
         }
     }
 
-    const int ntiles = (a.n_idx + kTileKeys - 1) / kTileKeys;
+    const int ntot = (a.n_idx + kTileKeys - 1) / kTileKeys;
+    const int tbeg = SPLIT == 1 ? 0 : (int)(((int64_t)ntot * wid) / SPLIT);
+    const int ntiles = SPLIT == 1 ? ntot : (int)(((int64_t)ntot * (wid + 1)) / SPLIT);  // tile end
     const int64_t kv_stride = (int64_t)a.hkv * kD;
-    const uint16_t* Kg = a.K + g * kD;
-    const uint16_t* Vg = a.V + g * kD;
+    const uint16_t* Kg = a.K + (q * a.kv_q_stride * a.hkv + g) * kD;
+    const uint16_t* Vg = a.V + (q * a.kv_q_stride * a.hkv + g) * kD;
 
     // positions of one 16-key tile: lanes l and l+16 both hold entry l
     auto tile_pos = [&](int tile) -> int {
@@ -107,11 +116,11 @@ __global__ void __launch_bounds__(32 * kAttnWarps) attn_kernel(AttnArgs a) {
 
     static_assert(kStages == 2, "the position ring below holds 2 tiles");
     // p0: tile i (being computed), p1: tile i+1 (next to issue)
-    int p0 = tile_pos(0);
-    issue(0, 0, p0);
-    int p1 = tile_pos(1);
+    int p0 = tile_pos(tbeg);
+    issue(tbeg, tbeg % kStages, p0);
+    int p1 = tile_pos(tbeg + 1);
 
-    for (int i = 0; i < ntiles; ++i) {
+    for (int i = tbeg; i < ntiles; ++i) {
         issue(i + 1, (i + 1) % kStages, p1);
         const int p2 = tile_pos(i + 2);  // consumed one iteration later
         const unsigned vmask = __ballot_sync(0xffffffffu, p0 >= 0) & 0xFFFFu;
@@ -186,45 +195,89 @@ __global__ void __launch_bounds__(32 * kAttnWarps) attn_kernel(AttnArgs a) {
     cp_async_wait<0>();
     __syncwarp();
 
-    // normalise and stage O (heads x dims, bf16) for a coalesced store
 #pragma unroll
     for (int off = 4; off < 32; off <<= 1) {
         l_run[0] += __shfl_xor_sync(0xffffffffu, l_run[0], off);
         l_run[1] += __shfl_xor_sync(0xffffffffu, l_run[1], off);
     }
-    const float inv0 = l_run[0] > 0.f ? 1.f / l_run[0] : 0.f;
-    const float inv1 = l_run[1] > 0.f ? 1.f / l_run[1] : 0.f;
-    uint16_t* os = reinterpret_cast<uint16_t*>(wbuf);  // [8][128]
+    if constexpr (SPLIT == 1) {
+        // normalise and stage O (heads x dims, bf16) for a coalesced store
+        const float inv0 = l_run[0] > 0.f ? 1.f / l_run[0] : 0.f;
+        const float inv1 = l_run[1] > 0.f ? 1.f / l_run[1] : 0.f;
+        uint16_t* os = reinterpret_cast<uint16_t*>(wbuf);  // [8][128]
 #pragma unroll
-    for (int mt = 0; mt < 8; ++mt) {
-        const int d0 = mt * 16 + gq;
-        const uint32_t lo = pack_bf16x2(o[mt][0] * inv0, o[mt][1] * inv1);
-        const uint32_t hi = pack_bf16x2(o[mt][2] * inv0, o[mt][3] * inv1);
-        os[(2 * tq) * kD + d0] = (uint16_t)(lo & 0xFFFF);
-        os[(2 * tq + 1) * kD + d0] = (uint16_t)(lo >> 16);
-        os[(2 * tq) * kD + d0 + 8] = (uint16_t)(hi & 0xFFFF);
-        os[(2 * tq + 1) * kD + d0 + 8] = (uint16_t)(hi >> 16);
+        for (int mt = 0; mt < 8; ++mt) {
+            const int d0 = mt * 16 + gq;
+            const uint32_t lo = pack_bf16x2(o[mt][0] * inv0, o[mt][1] * inv1);
+            const uint32_t hi = pack_bf16x2(o[mt][2] * inv0, o[mt][3] * inv1);
+            os[(2 * tq) * kD + d0] = (uint16_t)(lo & 0xFFFF);
+            os[(2 * tq + 1) * kD + d0] = (uint16_t)(lo >> 16);
+            os[(2 * tq) * kD + d0 + 8] = (uint16_t)(hi & 0xFFFF);
+            os[(2 * tq + 1) * kD + d0 + 8] = (uint16_t)(hi >> 16);
+        }
+        __syncwarp();
+        uint16_t* orow = a.O + (q * a.hq + g * G) * (int64_t)kD;
+        const int nchunk = G * kD / 8;  // 16-byte chunks
+        for (int c = lane; c < nchunk; c += 32)
+            reinterpret_cast<uint4*>(orow)[c] = reinterpret_cast<const uint4*>(os)[c];
+    } else {
+        // partial states: unnormalised O [8 heads][128] fp32 per warp + (m, l)
+        __shared__ float ml[SPLIT][8][2];
+        float* op = reinterpret_cast<float*>(wbuf);
+#pragma unroll
+        for (int mt = 0; mt < 8; ++mt) {
+            const int d0 = mt * 16 + gq;
+            op[(2 * tq) * kD + d0] = o[mt][0];
+            op[(2 * tq + 1) * kD + d0] = o[mt][1];
+            op[(2 * tq) * kD + d0 + 8] = o[mt][2];
+            op[(2 * tq + 1) * kD + d0 + 8] = o[mt][3];
+        }
+        if (gq == 0) {
+            ml[wid][2 * tq][0] = m_run[0]; ml[wid][2 * tq][1] = l_run[0];
+            ml[wid][2 * tq + 1][0] = m_run[1]; ml[wid][2 * tq + 1][1] = l_run[1];
+        }
+        __syncthreads();
+        for (int e = threadIdx.x; e < G * kD; e += 32 * SPLIT) {
+            const int hh = e / kD, d = e % kD;
+            float mx = -CUDART_INF_F;
+            for (int w = 0; w < SPLIT; ++w) mx = fmaxf(mx, ml[w][hh][0]);
+            float l = 0.f, acc = 0.f;
+            if (mx > -CUDART_INF_F) {
+                for (int w = 0; w < SPLIT; ++w) {
+                    const float mw = ml[w][hh][0];
+                    if (!(mw > -CUDART_INF_F)) continue;
+                    const float sc = exp2f(mw - mx);
+                    l += ml[w][hh][1] * sc;
+                    acc += reinterpret_cast<const float*>(asmem + w * kWarpBytes)[hh * kD + d] * sc;
+                }
+            }
+            const float out = l > 0.f ? acc / l : 0.f;
+            const __nv_bfloat16 ob = __float2bfloat16_rn(out);
+            a.O[(q * a.hq + g * G + hh) * (int64_t)kD + d] = *reinterpret_cast<const uint16_t*>(&ob);
+        }
     }
-    __syncwarp();
-    uint16_t* orow = a.O + (q * a.hq + g * G) * (int64_t)kD;
-    const int nchunk = G * kD / 8;  // 16-byte chunks
-    for (int c = lane; c < nchunk; c += 32)
-        reinterpret_cast<uint4*>(orow)[c] = reinterpret_cast<const uint4*>(os)[c];
 }
 
 lsa_status launch_attn(const uint16_t* Q, const uint16_t* K, const uint16_t* V, const int32_t* idx,
                        int64_t nq, int32_t hq, int32_t hkv, int32_t n_idx, int64_t T, uint16_t* O,
-                       cudaStream_t st) {
+                       cudaStream_t st, int64_t kv_q_stride = 0, int split = 1) {
     if (nq <= 0) return LSA_OK;
     AttnArgs a{};
     a.Q = Q; a.K = K; a.V = V; a.idx = idx; a.nq = nq; a.hq = hq; a.hkv = hkv; a.n_idx = n_idx;
-    a.T = T; a.O = O;
+    a.T = T; a.O = O; a.kv_q_stride = kv_q_stride;
     a.scale_log2 = 1.4426950408889634f / sqrtf((float)kD);
-    const size_t smem = (size_t)kAttnWarps * kWarpBytes;
-    cudaFuncSetAttribute(attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    const int64_t warps = nq * hkv;
-    attn_kernel<<<(unsigned)ceil_div<int64_t>(warps, kAttnWarps), 32 * kAttnWarps, smem, st>>>(a);
-    return check_launch("attn_kernel");
+    const int64_t rows = nq * hkv;
+    if (split == 1) {
+        const size_t smem = (size_t)kAttnWarps * kWarpBytes;
+        cudaFuncSetAttribute(attn_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        attn_kernel<1><<<(unsigned)ceil_div<int64_t>(rows, kAttnWarps), 32 * kAttnWarps, smem, st>>>(a);
+        return check_launch("attn_kernel");
+    }
+    constexpr int kSplit = 8;
+    const size_t smem = (size_t)kSplit * kWarpBytes;
+    cudaFuncSetAttribute(attn_kernel<kSplit>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    attn_kernel<kSplit><<<(unsigned)rows, 32 * kSplit, smem, st>>>(a);
+    return check_launch("attn_kernel(split)");
 }
 
 }  // namespace lsa

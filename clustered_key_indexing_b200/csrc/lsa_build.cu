@@ -219,8 +219,15 @@ lsa_status launch_query_latent(const uint16_t* Q, int64_t nq, int32_t hq, int32_
 // that pointed at either merged cluster).
 constexpr int kWT = 129;  // padded stride of UT / MU (doubles)
 
+constexpr int kMaxWardJobs = 256;
+
 struct WardArgs {
     const double* U;
+    int64_t U_stride;    // units per head in U
+    int32_t U_local;     // 1: U holds only the clustered block (decode block ring)
+    int32_t n_jobs;      // > 0: decode jobs, blockIdx.x -> (head base, block) below
+    int32_t job_head0[kMaxWardJobs];
+    int64_t job_blk[kMaxWardJobs];
     int64_t cap_units, cap_buckets;
     int64_t NU;          // units in use
     int64_t T;           // tokens in use (key ranges clip to it)
@@ -279,12 +286,12 @@ __global__ void __launch_bounds__(128, 1) ward_kernel(WardArgs a) {
     __shared__ int scan2_[4];
 
     const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
-    const int h = blockIdx.y;
-    const int64_t blk = a.blk0 + blockIdx.x;
+    const int h = a.n_jobs > 0 ? a.job_head0[blockIdx.x] + (int)blockIdx.y : (int)blockIdx.y;
+    const int64_t blk = a.n_jobs > 0 ? a.job_blk[blockIdx.x] : a.blk0 + blockIdx.x;
     const int64_t u0 = blk * kUnitsPerBlock;
     const int n = (int)min((int64_t)kUnitsPerBlock, a.NU - u0);
     const int m = (n * kBucketsPerBlock + kUnitsPerBlock - 1) / kUnitsPerBlock;
-    const double* Ub = a.U + ((int64_t)h * a.cap_units + u0) * kDL;
+    const double* Ub = a.U + ((int64_t)h * a.U_stride + (a.U_local ? 0 : u0)) * kDL;
 
     for (int i = tid; i < n * kDL; i += 128) {
         const int unit = i / kDL, c = i % kDL;
@@ -496,20 +503,55 @@ __global__ void __launch_bounds__(128, 1) ward_kernel(WardArgs a) {
     if (tid == 0) offs[(blk + 1) * kBucketsPerBlock] = (int32_t)(u0 + n);
 }
 
-lsa_status launch_ward(const lsa_cache* c, int64_t T, int32_t sinks, int64_t blk0, int64_t blk1,
-                       cudaStream_t st) {
-    if (blk1 <= blk0) return LSA_OK;
-    WardArgs a{};
-    a.U = c->U; a.cap_units = c->cap_units; a.cap_buckets = c->cap_buckets;
-    a.NU = ceil_div<int64_t>(T, kPool); a.T = T; a.sinks = sinks; a.blk0 = blk0;
+static void fill_ward_cache(WardArgs& a, const lsa_cache* c) {
+    a.cap_units = c->cap_units; a.cap_buckets = c->cap_buckets;
     a.bucket_of_unit = c->bucket_of_unit; a.members = c->members; a.offsets = c->offsets;
     a.cnt_lr = c->cnt_lr; a.minlr = c->minlr; a.maxpos = c->maxpos; a.sum = c->sum; a.cent = c->cent;
     a.units = c->units;
-    const size_t smem = sizeof(double) * (2 * kDL * kWT + kUnitsPerBlock * (kUnitsPerBlock - 1) / 2);
+}
+
+static size_t ward_smem() {
+    return sizeof(double) * (2 * kDL * kWT + kUnitsPerBlock * (kUnitsPerBlock - 1) / 2);
+}
+
+// Blocks [blk0, blk1) of every head of `c`, units read from U (U_stride
+// units per head).
+lsa_status launch_ward_u(const lsa_cache* c, const double* U, int64_t U_stride, int64_t T,
+                         int32_t sinks, int64_t blk0, int64_t blk1, cudaStream_t st) {
+    if (blk1 <= blk0) return LSA_OK;
+    WardArgs a{};
+    fill_ward_cache(a, c);
+    a.U = U; a.U_stride = U_stride; a.U_local = 0; a.n_jobs = 0;
+    a.NU = ceil_div<int64_t>(T, kPool); a.T = T; a.sinks = sinks; a.blk0 = blk0;
+    const size_t smem = ward_smem();
     cudaFuncSetAttribute(ward_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     dim3 grid((unsigned)(blk1 - blk0), (unsigned)c->hkv);
     ward_kernel<<<grid, 128, smem, st>>>(a);
     return check_launch("ward_kernel");
+}
+
+lsa_status launch_ward(const lsa_cache* c, int64_t T, int32_t sinks, int64_t blk0, int64_t blk1,
+                       cudaStream_t st) {
+    return launch_ward_u(c, c->U, c->cap_units, T, sinks, blk0, blk1, st);
+}
+
+// Decode: cluster one completed block per job; job j covers heads
+// head0[j] .. head0[j] + hkv - 1 of the (request-combined) cache, and its
+// units come from the block ring U_blk [heads, 128, 64].
+lsa_status launch_ward_jobs(const lsa_cache* c, const double* U_blk, int32_t hkv, int32_t sinks,
+                            int n_jobs, const int32_t* head0, const int64_t* blk, cudaStream_t st) {
+    if (n_jobs <= 0) return LSA_OK;
+    if (n_jobs > kMaxWardJobs) return set_error(LSA_EUNSUPPORTED, "more than %d blocks completed in one step", kMaxWardJobs);
+    WardArgs a{};
+    fill_ward_cache(a, c);
+    a.U = U_blk; a.U_stride = kUnitsPerBlock; a.U_local = 1; a.n_jobs = n_jobs;
+    for (int j = 0; j < n_jobs; ++j) { a.job_head0[j] = head0[j]; a.job_blk[j] = blk[j]; }
+    a.NU = c->cap_units; a.T = c->cap_units * kPool; a.sinks = sinks; a.blk0 = 0;
+    const size_t smem = ward_smem();
+    cudaFuncSetAttribute(ward_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    dim3 grid((unsigned)n_jobs, (unsigned)hkv);
+    ward_kernel<<<grid, 128, smem, st>>>(a);
+    return check_launch("ward_kernel(decode)");
 }
 
 // Mark bucket slots [b0, b1) of every head empty.

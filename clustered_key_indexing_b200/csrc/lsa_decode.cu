@@ -1,0 +1,622 @@
+// lsa_decode.cu -- batched decode of the LSA path on sm_100a.
+//
+// One new token per request per step [essay "《卡片柜》——当注意力学会先查目录
+// 再翻书", ch. 2: clustering is done once per completed 512-key block while
+// streaming and never redone; ch. 3/4: the query then searches the bucket
+// cache flat or down the tree; tutorial "隐空间稀疏注意力 (LSA)", section 二:
+// exact attention over the selected keys].
+//
+// The cache of a decode batch is one lsa_cache whose heads are
+// (request, kv-head) pairs: head r*hkv + h.  Per step:
+//   decode_append_kernel   K/V rows of the new token; its key latent (fp64)
+//                          added to the pooled unit being filled (block ring
+//                          U_blk), divided by 4 when the unit completes;
+//   ward_kernel (jobs)     every request whose token completed a block
+//                          clusters it; the tree is updated above its slots;
+//   query latents, then flat (decode_score_kernel + decode_resolve_kernel)
+//                          or tree (tree_select_kernel) selection;
+//   attn_kernel<8>         eight warps share each (request, kv-head) row.
+// Flat scores: one HBM pass over the request's eligible centroids (fp32 dot
+// products from 16-byte loads, 8 lanes per centroid), then one CTA per row:
+// weighted histogram on bins of width >= 2e around the row's score range,
+// exact fp64 rescoring of the two top bins' buckets, weighted radix select,
+// key emission in bucket-id order; rows whose band overflows shared memory
+// take exact fp64 scores of every eligible bucket in a global slot.
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "lsa.h"
+#include "lsa_common.cuh"
+
+namespace lsa {
+
+lsa_status launch_key_latent(const uint16_t* K, int64_t T, int32_t hkv, const float* W, int64_t unit0,
+                             int64_t unit1, int64_t cap_units, double* U, cudaStream_t st);
+lsa_status launch_query_latent(const uint16_t* Q, int64_t nq, int32_t hq, int32_t hkv, const float* W,
+                               int agg, uint16_t* Y, cudaStream_t st);
+lsa_status launch_ward_u(const lsa_cache* c, const double* U, int64_t U_stride, int64_t T, int32_t sinks,
+                         int64_t blk0, int64_t blk1, cudaStream_t st);
+lsa_status launch_ward_jobs(const lsa_cache* c, const double* U_blk, int32_t hkv, int32_t sinks, int n_jobs,
+                            const int32_t* head0, const int64_t* blk, cudaStream_t st);
+lsa_status launch_clear_slots(const lsa_cache* c, int64_t b0, int64_t b1, cudaStream_t st);
+lsa_status launch_tree_update(const lsa_cache* c, lsa_tree* t, int64_t b0, int64_t b1, cudaStream_t st);
+lsa_status launch_attn(const uint16_t* Q, const uint16_t* K, const uint16_t* V, const int32_t* idx,
+                       int64_t nq, int32_t hq, int32_t hkv, int32_t n_idx, int64_t T, uint16_t* O,
+                       cudaStream_t st, int64_t kv_q_stride, int split);
+
+// ------------------------------------------------------------- key latent
+
+// z = normalise(k W) for one 128-value bf16 row held in shared memory as
+// doubles; lane computes dims c = lane, lane + 32; |v|^2 summed in ascending
+// dim order.  Returns z for the lane's two dims.
+__device__ __forceinline__ void latent_row(const double* krow, const float* __restrict__ W,
+                                           int lane, double& z0, double& z1) {
+    double v0 = 0.0, v1 = 0.0;
+    for (int e = 0; e < kD; ++e) {
+        const double k = krow[e];
+        v0 = fma(k, (double)__ldg(W + e * kDL + lane), v0);
+        v1 = fma(k, (double)__ldg(W + e * kDL + lane + 32), v1);
+    }
+    double n2 = 0.0;
+    for (int c = 0; c < kDL; ++c) {
+        const double v = __shfl_sync(0xffffffffu, c < 32 ? v0 : v1, c & 31);
+        n2 = __dadd_rn(n2, __dmul_rn(v, v));
+    }
+    const double nrm = sqrt(n2);
+    z0 = nrm > 0.0 ? __ddiv_rn(v0, nrm) : 0.0;
+    z1 = nrm > 0.0 ? __ddiv_rn(v1, nrm) : 0.0;
+}
+
+struct AppendArgs {
+    const uint16_t* k;   // [batch, hkv, 128] new keys
+    const uint16_t* v;   // [batch, hkv, 128] new values
+    uint16_t* K;         // [batch, cap, hkv, 128]
+    uint16_t* V;
+    const float* W;      // W_k [128, 64]
+    double* U_blk;       // [batch * hkv, 128, 64]
+    int64_t cap;
+    int32_t hkv, batch;
+    int64_t pos[LSA_MAX_BATCH];
+};
+
+// One warp per (request, kv-head).
+__global__ void __launch_bounds__(256) decode_append_kernel(AppendArgs a) {
+    __shared__ double krow[8][kD];
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    const int64_t w = (int64_t)blockIdx.x * 8 + wid;
+    if (w >= (int64_t)a.batch * a.hkv) return;
+    const int64_t r = w / a.hkv, h = w % a.hkv;
+    const int64_t t = a.pos[r];
+    const uint16_t* ks = a.k + w * kD;
+    const uint16_t* vs = a.v + w * kD;
+    const int64_t dst = ((r * a.cap + t) * a.hkv + h) * kD;
+    if (lane < 16) {
+        reinterpret_cast<uint4*>(a.K + dst)[lane] = reinterpret_cast<const uint4*>(ks)[lane];
+        reinterpret_cast<uint4*>(a.V + dst)[lane] = reinterpret_cast<const uint4*>(vs)[lane];
+    }
+    for (int e = lane; e < kD; e += 32) krow[wid][e] = bf16_to_f64(ks[e]);
+    __syncwarp();
+    double z0, z1;
+    latent_row(krow[wid], a.W, lane, z0, z1);
+    double* u = a.U_blk + (w * kUnitsPerBlock + (t / kPool) % kUnitsPerBlock) * kDL;
+    const int i = (int)(t % kPool);
+    double s0 = (i == 0) ? __dadd_rn(0.0, z0) : __dadd_rn(u[lane], z0);
+    double s1 = (i == 0) ? __dadd_rn(0.0, z1) : __dadd_rn(u[lane + 32], z1);
+    if (i == kPool - 1) {
+        s0 = __ddiv_rn(s0, (double)kPool);
+        s1 = __ddiv_rn(s1, (double)kPool);
+    }
+    u[lane] = s0;
+    u[lane + 32] = s1;
+}
+
+// Tail of a loaded prompt: pooled units [j0, j1) of one request into its
+// block ring (complete units divided by 4, the last partial unit left as the
+// running sum the next appends continue).  One warp per (head, unit).
+__global__ void __launch_bounds__(256) tail_units_kernel(const uint16_t* __restrict__ K,
+                                                         const float* __restrict__ W, double* U_blk,
+                                                         int64_t n, int64_t j0, int64_t j1, int32_t hkv,
+                                                         int64_t head0) {
+    __shared__ double krow[8][kD];
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    const int64_t w = (int64_t)blockIdx.x * 8 + wid;
+    if (w >= (j1 - j0) * hkv) return;
+    const int64_t j = j0 + w / hkv, h = w % hkv;
+    double s0 = 0.0, s1 = 0.0;
+    int cnt = 0;
+    for (int64_t t = j * kPool; t < j * kPool + kPool && t < n; ++t) {
+        const uint16_t* ks = K + (t * hkv + h) * kD;
+        __syncwarp();
+        for (int e = lane; e < kD; e += 32) krow[wid][e] = bf16_to_f64(ks[e]);
+        __syncwarp();
+        double z0, z1;
+        latent_row(krow[wid], W, lane, z0, z1);
+        s0 = __dadd_rn(s0, z0);
+        s1 = __dadd_rn(s1, z1);
+        ++cnt;
+    }
+    if (cnt == kPool) {
+        s0 = __ddiv_rn(s0, (double)kPool);
+        s1 = __ddiv_rn(s1, (double)kPool);
+    }
+    double* u = U_blk + ((head0 + h) * kUnitsPerBlock + j % kUnitsPerBlock) * kDL;
+    u[lane] = s0;
+    u[lane + 32] = s1;
+}
+
+// ------------------------------------------------------ flat decode scores
+
+constexpr int kDecScoreCols = 2048;  // bucket slots per CTA
+
+struct DecScoreArgs {
+    const uint16_t* Y;        // [batch, hkv, 64] (mean) / [batch, hq, 64] (native)
+    const uint16_t* cent;     // [heads, cap_buckets, 64]
+    const int32_t* minlr;
+    const int32_t* maxpos;
+    const int32_t* cnt_lr;
+    const int32_t* units;
+    int64_t cap_buckets, ld;
+    int32_t hkv, G, agg, S, W;
+    int64_t T_built;
+    float* sc;                // [rows, ld]
+    uint8_t* wt;              // [rows, ld]
+    int64_t pos[LSA_MAX_BATCH];
+};
+
+__device__ __forceinline__ int weight_units(int64_t b, int32_t pk, int64_t lim, int32_t S, int64_t T_built) {
+    const int64_t ubase = (b / kBucketsPerBlock) * kUnitsPerBlock;
+    const int cnt = (pk >> 28) & 7;
+    int w = 0;
+    for (int i = 0; i < cnt; ++i) {
+        const int64_t j = ubase + ((pk >> (7 * i)) & 127);
+        for (int64_t p = j * kPool; p < j * kPool + kPool && p < T_built; ++p)
+            if (p >= S && p <= lim) ++w;
+    }
+    return w;
+}
+
+// grid (column chunks, rows); 8 warps, each 256 buckets, 8 lanes per bucket.
+// NG = query latents per row (1 for the group mean, G for the native max).
+template <int NG>
+__global__ void __launch_bounds__(256) decode_score_kernel(DecScoreArgs a) {
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    const int64_t row = blockIdx.y;
+    const int64_t r = row / a.hkv;
+    const int64_t t = a.pos[r];
+    const int64_t lim = t - a.W;
+    const int64_t ncol = lim < 0 ? 0 : min(a.cap_buckets, (int64_t)kBucketsPerBlock * (lim / kBlockKeys + 1));
+    const int64_t c0 = (int64_t)blockIdx.x * kDecScoreCols;
+    if (c0 >= ncol) return;
+    const int part = lane & 7;
+    // this lane's 8 latent dims of each of the NG query latents
+    float y[NG][8];
+    const uint16_t* yb = a.Y + (row * NG) * kDL;  // native: row*G = r*hq + h*G
+#pragma unroll
+    for (int g = 0; g < NG; ++g) {
+        const uint4 yv = *reinterpret_cast<const uint4*>(yb + g * kDL + part * 8);
+        const uint32_t u[4] = {yv.x, yv.y, yv.z, yv.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            y[g][2 * e] = __uint_as_float(u[e] << 16);
+            y[g][2 * e + 1] = __uint_as_float(u[e] & 0xFFFF0000u);
+        }
+    }
+    const uint16_t* cb = a.cent + row * a.cap_buckets * kDL;
+    const int64_t hb0 = row * a.cap_buckets;
+    const int64_t wbase = c0 + (int64_t)wid * (kDecScoreCols / 8);
+#pragma unroll 4
+    for (int it = 0; it < kDecScoreCols / 8 / 4; ++it) {
+        const int64_t b = wbase + it * 4 + (lane >> 3);
+        const bool in = b < ncol;
+        uint4 cv = make_uint4(0, 0, 0, 0);
+        if (in) cv = __ldg(reinterpret_cast<const uint4*>(cb + b * kDL + part * 8));
+        const uint32_t u[4] = {cv.x, cv.y, cv.z, cv.w};
+        float c8[8];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            c8[2 * e] = __uint_as_float(u[e] << 16);
+            c8[2 * e + 1] = __uint_as_float(u[e] & 0xFFFF0000u);
+        }
+        float best = -CUDART_INF_F;
+#pragma unroll
+        for (int g = 0; g < NG; ++g) {
+            float s = 0.f;
+#pragma unroll
+            for (int e = 0; e < 8; ++e) s = fmaf(y[g][e], c8[e], s);
+            s += __shfl_xor_sync(0xffffffffu, s, 1);
+            s += __shfl_xor_sync(0xffffffffu, s, 2);
+            s += __shfl_xor_sync(0xffffffffu, s, 4);
+            best = fmaxf(best, s);
+        }
+        if (in && part == 0) {
+            const int32_t mlr = a.minlr[hb0 + b];
+            const bool el = (int64_t)mlr <= lim;
+            int w = 0;
+            if (el) {
+                const int32_t mxp = a.maxpos[hb0 + b];
+                w = (int64_t)mxp <= lim ? a.cnt_lr[hb0 + b] : weight_units(b, a.units[hb0 + b], lim, a.S, a.T_built);
+            }
+            a.sc[row * a.ld + b] = el ? best : -CUDART_INF_F;
+            a.wt[row * a.ld + b] = (uint8_t)w;
+        }
+    }
+}
+
+// ---------------------------------------------------- flat decode resolve
+
+constexpr float kDecErr = 1e-4f;   // bound on |fp32 score - exact score|
+constexpr int kDecBins = 2048;
+
+struct DecResolveArgs {
+    SelectArgs s;            // cache, cfg, idx, decode positions (row_info)
+    const float* sc;
+    uint8_t* wt;             // weights in, taken counts out (fallback rows)
+    double* slot;            // [rows, ld] exact scores (fallback rows)
+    int64_t ld;
+    int64_t cap_buckets;
+};
+
+__global__ void __launch_bounds__(kSelThreads) decode_resolve_kernel(DecResolveArgs d) {
+    __shared__ SelShared sh;
+    __shared__ float rad_s;
+    const SelectArgs& a = d.s;
+    const int tid = threadIdx.x;
+    const int64_t row = blockIdx.x;
+    const RowInfo r = row_info(a, row);
+    write_sinks_window(a, r);
+    if (r.lim < a.S) {
+        for (int i = tid; i < a.k; i += kSelThreads) r.out[a.S + i] = -1;
+        return;
+    }
+    load_latents(a, r, sh);
+    __syncthreads();
+    const int ng = a.agg ? a.G : 1;
+    if (tid == 0) {
+        // score range [-R, R]: |score| <= |y| (native: max over heads);
+        // R >= 0.25 keeps every bin >= 2e wide
+        float R = 0.f;
+        for (int g = 0; g < ng; ++g) {
+            float n2 = 0.f;
+            for (int i = 0; i < kDL; ++i) { const float v = bf16_to_f32(sh.ylat[g * kDL + i]); n2 += v * v; }
+            R = fmaxf(R, sqrtf(n2));
+        }
+        rad_s = fmaxf(0.25f, fminf(1.0625f, R * 1.01f + 1e-6f));
+    }
+    __syncthreads();
+    const float R = rad_s;
+    const float bscale = (float)kDecBins / (2.f * R);
+    const int64_t ncol = min(d.cap_buckets, (int64_t)kBucketsPerBlock * (r.lim / kBlockKeys + 1));
+    const float* srow = d.sc + row * d.ld;
+    uint8_t* wrow = d.wt + row * d.ld;
+    for (int i = tid; i < kDecBins; i += kSelThreads) sh.hist[i] = 0ull;
+    __syncthreads();
+    long long myw = 0;
+    for (int64_t b = tid; b < ncol; b += kSelThreads) {
+        const int w = wrow[b];
+        if (w == 0) continue;
+        myw += w;
+        int bin = __float2int_rd((srow[b] + R) * bscale);
+        bin = bin < 0 ? 0 : (bin >= kDecBins ? kDecBins - 1 : bin);
+        atomicAdd(&sh.hist[bin], (1ull << 32) | (unsigned long long)w);
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) myw += __shfl_xor_sync(0xffffffffu, myw, off);
+    __shared__ long long wsum[kSelThreads / 32];
+    if ((tid & 31) == 0) wsum[tid >> 5] = myw;
+    __syncthreads();
+    long long totw = 0;
+    for (int i = 0; i < kSelThreads / 32; ++i) totw += wsum[i];
+    if (totw <= a.k) {
+        emit_range(a, r, ncol, [&](int64_t b) -> int { return (int)wrow[b]; }, sh);
+        return;
+    }
+    // cut bin j*: highest bin whose weight from the top reaches k; keep bins >= j* - 1
+    if (tid < 32) {
+        const int lane = tid;
+        long long s = 0;
+        for (int dd = 0; dd < kDecBins / 32; ++dd)
+            s += (long long)(sh.hist[kDecBins - 1 - (kDecBins / 32) * lane - dd] & 0xffffffffull);
+        long long incl = s;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const long long y = __shfl_up_sync(0xffffffffu, incl, off);
+            if (lane >= off) incl += y;
+        }
+        const long long excl = incl - s;
+        const unsigned mask = __ballot_sync(0xffffffffu, incl >= a.k && excl < a.k);
+        const int src = __ffs(mask) - 1;
+        if (lane == src) {
+            long long cum = excl;
+            int j = kDecBins - 1 - (kDecBins / 32) * lane;
+            for (int dd = 0; dd < kDecBins / 32; ++dd) {
+                const int jj = kDecBins - 1 - (kDecBins / 32) * lane - dd;
+                cum += (long long)(sh.hist[jj] & 0xffffffffull);
+                if (cum >= a.k) { j = jj; break; }
+            }
+            sh.misc[0] = j > 0 ? j - 1 : 0;
+        }
+    }
+    __syncthreads();
+    const int jt = sh.misc[0];
+    int cnt = 0;
+    for (int i = jt + tid; i < kDecBins; i += kSelThreads) cnt += (int)(sh.hist[i] >> 32);
+    int ncand;
+    block_exscan(cnt, &ncand, sh.sh4);
+    if (ncand <= kCap) {
+        // ordered compaction of the kept bins, exact rescoring, radix fill
+        int n = 0;
+        for (int64_t c0 = 0; c0 < ncol; c0 += kSelThreads) {
+            const int64_t b = c0 + tid;
+            bool el = false;
+            if (b < ncol && wrow[b] > 0) {
+                int bin = __float2int_rd((srow[b] + R) * bscale);
+                bin = bin < 0 ? 0 : (bin >= kDecBins ? kDecBins - 1 : bin);
+                el = bin >= jt;
+            }
+            int tot;
+            const int o = block_exscan(el ? 1 : 0, &tot, sh.sh4);
+            if (el) sh.cid[n + o] = (int)b;
+            n += tot;
+        }
+        __syncthreads();
+        const int64_t hb0 = (int64_t)r.h * d.cap_buckets;
+        for (int i = tid; i < n; i += kSelThreads) {
+            const int64_t b = sh.cid[i];
+            sh.csc[i] = exact_row(sh.ylat, ng, a.cent + (hb0 + b) * kDL);
+            sh.cw[i] = wrow[b];
+        }
+        __syncthreads();
+        radix_fill(
+            n, a.k, [&](int64_t i) { return sh.csc[i]; }, [&](int64_t i) { return sh.cw[i]; },
+            [&](int64_t i, int tk) { sh.ctk[i] = tk; }, sh);
+        emit_candidates(a, r, n, sh);
+        return;
+    }
+    // band overflow (dense ties): exact scores of every eligible bucket
+    double* fs = d.slot + row * d.ld;
+    const int64_t hb0 = (int64_t)r.h * d.cap_buckets;
+    for (int64_t b = tid; b < ncol; b += kSelThreads)
+        fs[b] = wrow[b] > 0 ? exact_row(sh.ylat, ng, a.cent + (hb0 + b) * kDL) : 0.0;
+    __syncthreads();
+    radix_fill(
+        ncol, a.k, [&](int64_t i) { return fs[i]; }, [&](int64_t i) { return (int)wrow[i]; },
+        [&](int64_t i, int tk) { wrow[i] = (uint8_t)tk; }, sh);
+    __syncthreads();
+    emit_range(a, r, ncol, [&](int64_t b) -> int { return (int)wrow[b]; }, sh);
+}
+
+// ------------------------------------------------------------- host side
+
+static int64_t decode_row_len(const lsa_cfg* cfg) { return cfg->sinks + cfg->k + cfg->window; }
+
+struct DecodeWs {
+    uint16_t* Y;
+    int32_t* idx;
+    float* sc;
+    uint8_t* wt;
+    double* slot;
+    double* Utmp;
+    size_t step_bytes, load_bytes;
+};
+
+static DecodeWs carve_decode(const lsa_cfg* cfg, const lsa_decode* d, char* base) {
+    DecodeWs w{};
+    const int64_t rows = (int64_t)d->batch * d->hkv;
+    const int64_t ld = (d->cache.cap_buckets + 127) / 128 * 128;
+    const int32_t hy = cfg->agg ? d->hq : d->hkv;
+    size_t o = 0;
+    auto take = [&](size_t n) { size_t at = o; o += (n + 255) & ~(size_t)255; return base + at; };
+    w.Y = (uint16_t*)take((size_t)d->batch * hy * kDL * 2);
+    w.idx = (int32_t*)take((size_t)rows * decode_row_len(cfg) * 4);
+    if (cfg->mode == 0) {
+        w.sc = (float*)take((size_t)rows * ld * 4);
+        w.wt = (uint8_t*)take((size_t)rows * ld);
+        w.slot = (double*)take((size_t)rows * ld * 8);
+    }
+    w.step_bytes = o;
+    // a request load reuses the same bytes for its temporary pooled units
+    w.Utmp = (double*)base;
+    w.load_bytes = (size_t)d->hkv * (d->cap / kPool) * kDL * 8;
+    return w;
+}
+
+static lsa_cache request_view(const lsa_decode* d, int32_t r) {
+    lsa_cache v = d->cache;
+    const int64_t h0 = (int64_t)r * d->hkv;
+    v.hkv = d->hkv;
+    v.U = nullptr;
+    v.bucket_of_unit += h0 * v.cap_units;
+    v.members += h0 * v.cap_units;
+    v.offsets += h0 * (v.cap_buckets + 1);
+    v.cnt_lr += h0 * v.cap_buckets;
+    v.minlr += h0 * v.cap_buckets;
+    v.maxpos += h0 * v.cap_buckets;
+    v.sum += h0 * v.cap_buckets * kDL;
+    v.cent += h0 * v.cap_buckets * kDL;
+    v.units += h0 * v.cap_buckets;
+    return v;
+}
+
+static lsa_tree tree_view(const lsa_decode* d, int32_t r) {
+    lsa_tree t = d->tree;
+    const int64_t h0 = (int64_t)r * d->hkv;
+    t.sum += h0 * t.n_nodes * kDL;
+    t.minlr += h0 * t.n_nodes;
+    t.cent += h0 * t.n_nodes * kDL;
+    return t;
+}
+
+static lsa_status check_decode(const lsa_decode* d, const lsa_cfg* cfg) {
+    if (!d) return set_error(LSA_EINVAL, "decode state is NULL");
+    if (d->batch < 1 || d->batch > LSA_MAX_BATCH) return set_error(LSA_EUNSUPPORTED, "decode: batch must be 1..%d", LSA_MAX_BATCH);
+    if (d->hkv < 1 || d->hq < 1 || d->hq % d->hkv) return set_error(LSA_EINVAL, "decode: need hq %% hkv == 0");
+    const int G = d->hq / d->hkv;
+    if (G != 1 && G != 2 && G != 4 && G != 8) return set_error(LSA_EUNSUPPORTED, "decode: hq / hkv must be 1, 2, 4 or 8");
+    if (d->cap < kBlockKeys || d->cap % kBlockKeys) return set_error(LSA_EINVAL, "decode: cap must be a positive multiple of 512");
+    if (!d->K || !d->V || !d->U_blk) return set_error(LSA_EINVAL, "decode: K, V or U_blk is NULL");
+    const lsa_cache& c = d->cache;
+    if (c.hkv != d->batch * d->hkv) return set_error(LSA_EINVAL, "decode: cache.hkv must be batch * hkv");
+    if (c.cap_units != d->cap / kPool || c.cap_buckets != d->cap / kBlockKeys * kBucketsPerBlock)
+        return set_error(LSA_EINVAL, "decode: cache capacities must match cap");
+    if (!c.bucket_of_unit || !c.members || !c.offsets || !c.cnt_lr || !c.minlr || !c.maxpos || !c.sum ||
+        !c.cent || !c.units)
+        return set_error(LSA_EINVAL, "decode: a cache array is NULL");
+    if (cfg->mode == 1) {
+        lsa_tree ref;
+        lsa_tree_layout(c.cap_buckets, &ref);
+        if (!d->tree.sum || !d->tree.minlr || !d->tree.cent || d->tree.levels != ref.levels ||
+            d->tree.n_nodes != ref.n_nodes)
+            return set_error(LSA_EINVAL, "decode: tree mode needs a tree laid out over cache.cap_buckets");
+    }
+    return LSA_OK;
+}
+
+static int lstar_for(const lsa_cfg* cfg) {
+    int l = 0;
+    while ((int64_t)cfg->beam * cfg->bucket_mean * ((int64_t)1 << l) < cfg->k && l < 62) ++l;
+    return l;
+}
+
+static void fill_select_args(SelectArgs& a, const lsa_decode* d, const lsa_cfg* cfg, const uint16_t* Y,
+                             int32_t* idx) {
+    const lsa_cache& c = d->cache;
+    a.offsets = c.offsets; a.members = c.members; a.cnt_lr = c.cnt_lr; a.minlr = c.minlr;
+    a.maxpos = c.maxpos; a.cent = c.cent; a.cap_units = c.cap_units; a.cap_buckets = c.cap_buckets;
+    a.NB = c.cap_buckets; a.T_built = d->cap;
+    a.hkv = d->hkv; a.G = d->hq / d->hkv; a.agg = cfg->agg; a.k = cfg->k; a.S = cfg->sinks; a.W = cfg->window;
+    a.mode = cfg->mode;
+    if (cfg->mode == 1) {
+        a.tminlr = d->tree.minlr; a.tcent = d->tree.cent; a.n_nodes = d->tree.n_nodes;
+        a.levels = d->tree.levels; a.beam = cfg->beam; a.lstar = lstar_for(cfg);
+        for (int l = 0; l < d->tree.levels; ++l) { a.level_n[l] = d->tree.level_n[l]; a.level_off[l] = d->tree.level_off[l]; }
+    }
+    a.Y = Y; a.nqc = d->batch; a.t_first = 0; a.idx = idx;
+    a.decode = 1;
+    for (int r = 0; r < d->batch; ++r) a.pos[r] = d->len[r];
+}
+
+}  // namespace lsa
+
+using namespace lsa;
+
+extern "C" {
+
+size_t lsa_decode_workspace_bytes(const lsa_cfg* cfg, const lsa_decode* d) {
+    if (check_cfg(cfg) != LSA_OK || check_decode(d, cfg) != LSA_OK) return 0;
+    const DecodeWs w = carve_decode(cfg, d, nullptr);
+    return w.step_bytes > w.load_bytes ? w.step_bytes : w.load_bytes;
+}
+
+lsa_status lsa_decode_load(lsa_decode* d, int32_t r, int64_t n, const float* W_k, const lsa_cfg* cfg,
+                           void* ws, size_t ws_bytes, void* stream) {
+    lsa_status s;
+    if ((s = check_cfg(cfg)) != LSA_OK) return s;
+    if ((s = check_decode(d, cfg)) != LSA_OK) return s;
+    if (r < 0 || r >= d->batch) return set_error(LSA_EINVAL, "lsa_decode_load: request %d out of range", r);
+    if (n < 0 || n >= d->cap) return set_error(LSA_ENOSPACE, "lsa_decode_load: n must be in [0, cap)");
+    if (!W_k || !ws) return set_error(LSA_EINVAL, "lsa_decode_load: W_k or ws is NULL");
+    const DecodeWs w = carve_decode(cfg, d, (char*)ws);
+    if (ws_bytes < w.load_bytes || ws_bytes < w.step_bytes)
+        return set_error(LSA_ENOSPACE, "lsa_decode_load: workspace too small");
+    cudaStream_t st = (cudaStream_t)stream;
+    const lsa_cache view = request_view(d, r);
+    const uint16_t* Kr = d->K + (int64_t)r * d->cap * d->hkv * kD;
+    const int64_t nb = n / kBlockKeys, nc = nb * kBlockKeys;
+    if (nb > 0) {
+        if ((s = launch_key_latent(Kr, nc, d->hkv, W_k, 0, nc / kPool, nc / kPool, w.Utmp, st)) != LSA_OK) return s;
+        if ((s = launch_ward_u(&view, w.Utmp, nc / kPool, nc, cfg->sinks, 0, nb, st)) != LSA_OK) return s;
+    }
+    if ((s = launch_clear_slots(&view, nb * kBucketsPerBlock, view.cap_buckets, st)) != LSA_OK) return s;
+    const int64_t j0 = nc / kPool, j1 = (n + kPool - 1) / kPool;
+    if (j1 > j0) {
+        const int64_t warps = (j1 - j0) * d->hkv;
+        tail_units_kernel<<<(unsigned)ceil_div<int64_t>(warps, 8), 256, 0, st>>>(
+            Kr, W_k, d->U_blk, n, j0, j1, d->hkv, (int64_t)r * d->hkv);
+        if ((s = check_launch("tail_units_kernel")) != LSA_OK) return s;
+    }
+    if (cfg->mode == 1) {
+        lsa_tree tv = tree_view(d, r);
+        if ((s = launch_tree_update(&view, &tv, 0, view.cap_buckets, st)) != LSA_OK) return s;
+    }
+    d->len[r] = n;
+    return LSA_OK;
+}
+
+lsa_status lsa_decode_step(lsa_decode* d, const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                           const float* W_k, const float* W_q, const lsa_cfg* cfg, uint16_t* o,
+                           int32_t* idx_out, void* ws, size_t ws_bytes, void* stream) {
+    lsa_status s;
+    if ((s = check_cfg(cfg)) != LSA_OK) return s;
+    if ((s = check_decode(d, cfg)) != LSA_OK) return s;
+    if (!q || !k || !v || !W_k || !W_q || !o || !ws) return set_error(LSA_EINVAL, "lsa_decode_step: NULL pointer");
+    for (int r = 0; r < d->batch; ++r)
+        if (d->len[r] < 0 || d->len[r] >= d->cap)
+            return set_error(LSA_ENOSPACE, "lsa_decode_step: request %d is full (len %lld, cap %lld)", r,
+                             (long long)d->len[r], (long long)d->cap);
+    const DecodeWs w = carve_decode(cfg, d, (char*)ws);
+    if (ws_bytes < w.step_bytes) return set_error(LSA_ENOSPACE, "lsa_decode_step: workspace too small");
+    cudaStream_t st = (cudaStream_t)stream;
+    const int64_t rows = (int64_t)d->batch * d->hkv;
+
+    // (1) append k/v and pool the new key
+    AppendArgs ap{};
+    ap.k = k; ap.v = v; ap.K = d->K; ap.V = d->V; ap.W = W_k; ap.U_blk = d->U_blk; ap.cap = d->cap;
+    ap.hkv = d->hkv; ap.batch = d->batch;
+    for (int r = 0; r < d->batch; ++r) ap.pos[r] = d->len[r];
+    decode_append_kernel<<<(unsigned)ceil_div<int64_t>(rows, 8), 256, 0, st>>>(ap);
+    if ((s = check_launch("decode_append_kernel")) != LSA_OK) return s;
+
+    // (2) cluster every block this token completed
+    int32_t head0[LSA_MAX_BATCH];
+    int64_t blk[LSA_MAX_BATCH];
+    int nj = 0;
+    for (int r = 0; r < d->batch; ++r)
+        if ((d->len[r] + 1) % kBlockKeys == 0) { head0[nj] = r * d->hkv; blk[nj] = d->len[r] / kBlockKeys; ++nj; }
+    if ((s = launch_ward_jobs(&d->cache, d->U_blk, d->hkv, cfg->sinks, nj, head0, blk, st)) != LSA_OK) return s;
+    if (cfg->mode == 1) {
+        for (int j = 0; j < nj; ++j) {
+            const int r = head0[j] / d->hkv;
+            lsa_cache cv = request_view(d, r);
+            lsa_tree tv = tree_view(d, r);
+            if ((s = launch_tree_update(&cv, &tv, blk[j] * kBucketsPerBlock, (blk[j] + 1) * kBucketsPerBlock, st)) != LSA_OK)
+                return s;
+        }
+    }
+    // the new token is part of the context from here on
+    for (int r = 0; r < d->batch; ++r) d->len[r] += 1;
+
+    // (3) query latents, selection
+    if ((s = launch_query_latent(q, d->batch, d->hq, d->hkv, W_q, cfg->agg, w.Y, st)) != LSA_OK) return s;
+    int32_t* idx = idx_out ? idx_out : w.idx;
+    SelectArgs a{};
+    fill_select_args(a, d, cfg, w.Y, idx);
+    for (int r = 0; r < d->batch; ++r) a.pos[r] = d->len[r] - 1;
+    if (cfg->mode == 1) {
+        tree_select_kernel<<<(unsigned)rows, kSelThreads, 0, st>>>(a);
+        if ((s = check_launch("tree_select_kernel(decode)")) != LSA_OK) return s;
+    } else {
+        const int64_t ld = (d->cache.cap_buckets + 127) / 128 * 128;
+        DecScoreArgs sa{};
+        sa.Y = w.Y; sa.cent = d->cache.cent; sa.minlr = d->cache.minlr; sa.maxpos = d->cache.maxpos;
+        sa.cnt_lr = d->cache.cnt_lr; sa.units = d->cache.units; sa.cap_buckets = d->cache.cap_buckets;
+        sa.ld = ld; sa.hkv = d->hkv; sa.G = d->hq / d->hkv; sa.agg = cfg->agg; sa.S = cfg->sinks;
+        sa.W = cfg->window; sa.T_built = d->cap; sa.sc = w.sc; sa.wt = w.wt;
+        for (int r = 0; r < d->batch; ++r) sa.pos[r] = a.pos[r];
+        dim3 grid((unsigned)ceil_div<int64_t>(d->cache.cap_buckets, kDecScoreCols), (unsigned)rows);
+        const int ng = cfg->agg ? d->hq / d->hkv : 1;
+        if (ng == 1) decode_score_kernel<1><<<grid, 256, 0, st>>>(sa);
+        else if (ng == 2) decode_score_kernel<2><<<grid, 256, 0, st>>>(sa);
+        else if (ng == 4) decode_score_kernel<4><<<grid, 256, 0, st>>>(sa);
+        else decode_score_kernel<8><<<grid, 256, 0, st>>>(sa);
+        if ((s = check_launch("decode_score_kernel")) != LSA_OK) return s;
+        DecResolveArgs ra{};
+        ra.s = a; ra.sc = w.sc; ra.wt = w.wt; ra.slot = w.slot; ra.ld = ld; ra.cap_buckets = d->cache.cap_buckets;
+        decode_resolve_kernel<<<(unsigned)rows, kSelThreads, 0, st>>>(ra);
+        if ((s = check_launch("decode_resolve_kernel")) != LSA_OK) return s;
+    }
+    // (4) attention: each request reads its own K/V rows
+    return launch_attn(q, d->K, d->V, idx, d->batch, d->hq, d->hkv, (int32_t)decode_row_len(cfg), d->cap,
+                       o, st, d->cap, 8);
+}
+
+}  // extern "C"

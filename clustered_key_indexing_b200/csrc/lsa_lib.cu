@@ -4,4 +4,5 @@
 #include "lsa_select.cu"
 #include "lsa_attn.cu"
 #include "lsa_api.cu"
+#include "lsa_decode.cu"
 #include "lsa_noalloc.cu"

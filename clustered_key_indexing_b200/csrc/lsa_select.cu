@@ -74,6 +74,10 @@ struct SelectArgs {
     int32_t ovf_cap;
     double* fb_score;      // [n_slots, ld]
     int32_t* fb_w;         // [n_slots, ld]
+    // decode rows: row = request * hkv + head is also the cache head, and
+    // each request has its own position
+    int32_t decode;
+    int64_t pos[LSA_MAX_BATCH];
 };
 
 __device__ __forceinline__ unsigned long long order_key(double s) {
@@ -251,9 +255,15 @@ struct RowInfo {
 
 __device__ __forceinline__ RowInfo row_info(const SelectArgs& a, int64_t row) {
     RowInfo r;
-    r.q = row / a.hkv;
-    r.h = (int)(row % a.hkv);
-    r.t = a.t_first + r.q;
+    if (a.decode) {
+        r.q = 0;
+        r.h = (int)row;
+        r.t = a.pos[row / a.hkv];
+    } else {
+        r.q = row / a.hkv;
+        r.h = (int)(row % a.hkv);
+        r.t = a.t_first + r.q;
+    }
     r.lim = r.t - a.W;
     r.out = a.idx + row * (int64_t)(a.S + a.k + a.W);
     return r;

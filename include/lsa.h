@@ -101,6 +101,7 @@ typedef struct lsa_cache {
 } lsa_cache;
 
 #define LSA_MAX_LEVELS 48
+#define LSA_MAX_BATCH 128
 
 /*
  * Complete binary tree over the bucket slots of a cache [ch. 4]: level 0 =
@@ -224,6 +225,66 @@ lsa_status lsa_sparse_attn(const uint16_t* Q, const uint16_t* K,
                            const uint16_t* V, const int32_t* idx, int64_t nq,
                            int32_t hq, int32_t hkv, int32_t n_idx, int64_t T,
                            uint16_t* O, void* stream);
+
+/* ------------------------------------------------------------ decode */
+
+/*
+ * Batched decode state of one layer, `batch` requests of one geometry
+ * [essay ch. 2: each completed 512-key block is clustered once, while
+ * streaming].  All arrays are caller-owned device memory except `len`.
+ * The cache's heads are (request, kv-head) pairs: head r*hkv + h.
+ *   K, V    [batch, cap, hkv, d_head] bf16: request r's token t is row r*cap + t.
+ *   U_blk   [batch*hkv, 128, d_latent] fp64: pooled units of the block each
+ *           request is filling (a complete unit holds its mean, the unit in
+ *           progress the running sum of its key latents).
+ *   cache   lsa_cache with hkv = batch*hkv, cap_units = cap/4,
+ *           cap_buckets = 64*cap/512; cache.U is not used (may be NULL).
+ *   tree    tree mode only: lsa_tree_layout(cache.cap_buckets), arrays
+ *           [batch*hkv, n_nodes, ...].
+ *   len     tokens each request holds (host memory, in this struct); set by
+ *           lsa_decode_load and advanced by lsa_decode_step.
+ * cap must be a multiple of 512; batch <= LSA_MAX_BATCH.
+ */
+typedef struct lsa_decode {
+    int32_t   batch, hkv, hq;
+    int64_t   cap;
+    uint16_t* K;
+    uint16_t* V;
+    double*   U_blk;
+    lsa_cache cache;
+    lsa_tree  tree;
+    int64_t   len[LSA_MAX_BATCH];
+} lsa_decode;
+
+/* Workspace bytes of lsa_decode_load / lsa_decode_step for this state. */
+size_t lsa_decode_workspace_bytes(const lsa_cfg* cfg, const lsa_decode* d);
+
+/*
+ * lsa_decode_load -- make request r hold the n tokens whose K/V rows the
+ * caller has written at rows r*cap .. r*cap+n-1: clusters its complete
+ * blocks (as lsa_build_buckets), pools the keys of the block in progress into
+ * U_blk, empties the later bucket slots, builds its tree (tree mode) and
+ * sets len[r] = n.  Requires n < cap.
+ */
+lsa_status lsa_decode_load(lsa_decode* d, int32_t r, int64_t n, const float* W_k,
+                           const lsa_cfg* cfg, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * lsa_decode_step -- one new token per request [essay ch. 2-4; tutorial §二].
+ * q [batch, hq, d], k/v [batch, hkv, d] bf16 (token t = len[r] of request r),
+ * o [batch, hq, d] bf16.  Appends k/v at t; pools its key latent; clusters a
+ * block completed by t (Ward, exactly as prefill) and updates the tree above
+ * it; then selects for query position t over the clustered blocks (flat or
+ * tree, as lsa_select) and attends over sinks + long-range keys + window
+ * (the window includes the new token).  len[r] advances by one.  With
+ * W >= 512 the selection equals lsa_select's at the same position.
+ * idx_out (optional, may be NULL): [batch, hkv, S+k+W] receives the index
+ * rows (positions within each request), as lsa_select writes them.
+ */
+lsa_status lsa_decode_step(lsa_decode* d, const uint16_t* q, const uint16_t* k,
+                           const uint16_t* v, const float* W_k, const float* W_q,
+                           const lsa_cfg* cfg, uint16_t* o, int32_t* idx_out, void* ws,
+                           size_t ws_bytes, void* stream);
 
 /* ---------------------------------------------- selection without ws */
 

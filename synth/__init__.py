@@ -32,6 +32,8 @@ CONFIGS = {
     "decode-32x1m": dict(T=1 << 20, batch=32, hkv=8, hq=32, d=128, dl=64,
                          n_centres=8192, k=2048, sinks=4, window=1024, mode=0,
                          agg=0, beam=2),
+    "decode-small": dict(T=4096, batch=3, hkv=2, hq=8, d=128, dl=64, n_centres=64, k=256,
+                         sinks=4, window=600, mode=0, agg=0, beam=2),
     "decode-4x10m": dict(T=10_000_000, batch=4, hkv=8, hq=32, d=128, dl=64,
                          n_centres=65536, k=2048, sinks=4, window=1024, mode=0,
                          agg=0, beam=2),

@@ -1,0 +1,74 @@
+"""GPU parity of the batched decode step (lsa_decode_step) against the CPU
+oracle: at a decode position t the oracle clusters the blocks complete at t
+(streaming, essay "《卡片柜》" ch. 2), selects for query t (ch. 3-4) and
+attends over the keys 0..t (tutorial "隐空间稀疏注意力" §二).  Index rows
+bit-exact, outputs within max |err| 2e-2 / mean |err| 2e-3."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from gpu_util import oracle_cfg, to_dev, to_dev_bf16
+
+pytestmark = pytest.mark.gpu
+
+PROMPTS = (1000, 1530, 2047)   # request 2 completes a block on its first step
+STEPS = 40
+
+
+@pytest.fixture(scope="module")
+def lsa():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import clustered_key_indexing_b200 as m
+    return m
+
+
+@pytest.fixture(scope="module")
+def reqs():
+    return [synth.layer_inputs("decode-small", seed=r) for r in range(len(PROMPTS))]
+
+
+@pytest.mark.parametrize("mode,agg,W", [(0, 0, 600), (0, 1, 600), (1, 0, 600), (1, 1, 600), (0, 0, 128)])
+def test_decode_matches_oracle(lsa, reqs, mode, agg, W):
+    c = synth.CONFIGS["decode-small"]
+    hkv, hq, cap = c["hkv"], c["hq"], c["T"]
+    cfg = lsa.Config(k=c["k"], sinks=c["sinks"], window=W, beam=c["beam"], mode=mode, agg=agg)
+    Wk, Wq = to_dev(reqs[0]["Wk"]), to_dev(reqs[0]["Wq"])  # one W_k / W_q per layer
+    dec = lsa.Decode(len(PROMPTS), hkv, hq, cap, cfg)
+    for r, n in enumerate(PROMPTS):
+        dec.load(r, to_dev_bf16(reqs[r]["K"][:n]), to_dev_bf16(reqs[r]["V"][:n]), Wk)
+    check_at = {0, 1, 2, 19, STEPS - 1}
+    idx = torch.empty((len(PROMPTS), hkv, cfg.row), dtype=torch.int32, device="cuda")
+    ocfg = oracle_cfg(cfg)
+    caches = {}
+    for s in range(STEPS):
+        ts = [n + s for n in PROMPTS]
+        q = to_dev_bf16(np.stack([reqs[r]["Q"][t] for r, t in enumerate(ts)]))
+        k = to_dev_bf16(np.stack([reqs[r]["K"][t] for r, t in enumerate(ts)]))
+        v = to_dev_bf16(np.stack([reqs[r]["V"][t] for r, t in enumerate(ts)]))
+        o = dec.step(q, k, v, Wk, Wq, idx_out=idx)
+        completes = any((t + 1) % 512 == 0 or t % 512 == 0 for t in ts)
+        if s not in check_at and not completes:
+            continue
+        torch.cuda.synchronize()
+        lsa.check_device_error()
+        g_idx = idx.cpu().numpy()
+        g_o = o.float().cpu().numpy().astype(np.float64)
+        for r, t in enumerate(ts):
+            tb = 512 * ((t + 1) // 512)
+            key = (r, tb)
+            if key not in caches:
+                U = oracle.key_latent_pool(reqs[r]["K"][:tb], reqs[0]["Wk"], 4)
+                oc = oracle.build_cache(U, tb, ocfg)
+                caches[key] = (oc, oracle.build_tree(oc) if mode == 1 else None)
+            oc, ot = caches[key]
+            Qt = reqs[r]["Q"][t:t + 1]
+            Y = oracle.query_latent(Qt, reqs[0]["Wq"], hkv, agg)
+            oidx, _, _ = oracle.select(oc, Y, np.array([t]), ocfg, tree=ot, G=hq // hkv)
+            assert np.array_equal(g_idx[r], oidx[0]), (s, r, t)
+            ref = oracle.attention(Qt, reqs[r]["K"][:t + 1], reqs[r]["V"][:t + 1], oidx)[0]
+            e = np.abs(g_o[r] - ref)
+            assert e.max() <= 2e-2 and e.mean() <= 2e-3, (s, r, e.max(), e.mean())
+    assert dec.len == [n + STEPS for n in PROMPTS]
