@@ -51,7 +51,7 @@ def parse():
     p.add_argument("--warmup", type=int, default=3)
     p.add_argument("--impl", default="lsa", choices=["lsa", "reference"])
     p.add_argument("--workload", default="prefill-128k",
-                   choices=["prefill-4k", "prefill-128k", "prefill-1m"])
+                   choices=["prefill-4k", "prefill-128k", "prefill-1m", "decode-32x1m"])
     p.add_argument("--mode", default=None, choices=["flat", "tree"])
     p.add_argument("--agg", default=None, choices=["mean", "max"])
     p.add_argument("--chunk", type=int, default=16384)
@@ -80,6 +80,7 @@ def config_json(args, c, world):
         "query_score": "group-mean" if c["agg"] == 0 else "max-over-heads (native)",
         "query_chunk": args.chunk, "parallelism": f"replicas x{world} (one layer per GPU)",
         "l2": "no flush: per-step inputs (Q/K/V) are larger than L2",
+        "inputs": "host-drawn (numpy PCG64)" if c["T"] <= 131072 else "device-drawn (torch Philox), same recipe",
     }
 
 
@@ -160,7 +161,46 @@ def oracle_sample(inp, c, n_blocks=None, n_queries=32, seed=0):
     return per_layer, desc, t_build + t_q * n_queries
 
 
+# ------------------------------------------------- device-drawn inputs
+
+def device_tokens(n, heads, d, mu, scale, gen, dev, out=None, chunk=65536):
+    """bf16 [n, heads, d] of scale * mu_c + N(0, I) (scale 0: N(0, 1)), c
+    uniform per (token, head), drawn on the device by torch's seeded
+    generator (same recipe as synth, another random stream)."""
+    import torch
+    if out is None:
+        out = torch.empty((n, heads, d), dtype=torch.bfloat16, device=dev)
+    for t0 in range(0, n, chunk):
+        t1 = min(n, t0 + chunk)
+        x = torch.randn((t1 - t0, heads, d), generator=gen, device=dev, dtype=torch.float32)
+        if scale != 0.0:
+            ci = torch.randint(0, mu.shape[0], (t1 - t0, heads), generator=gen, device=dev)
+            x += scale * mu[ci]
+        out[t0:t1] = x.to(torch.bfloat16)
+    return out
+
+
+def device_layer(c, seed, dev):
+    import torch
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(seed)
+    mu = torch.from_numpy(synth.centres(seed, c["n_centres"], c["d"])).to(dev)
+    K = device_tokens(c["T"], c["hkv"], c["d"], mu, 4.0, gen, dev)
+    V = device_tokens(c["T"], c["hkv"], c["d"], mu, 0.0, gen, dev)
+    Q = device_tokens(c["T"], c["hq"], c["d"], mu, 1.0, gen, dev)
+    return Q, K, V
+
+
 # ------------------------------------------------------------------ main
+
+def bits_of(t):
+    return t.contiguous().view(torch_int16()).numpy().view(np.uint16)
+
+
+def torch_int16():
+    import torch
+    return torch.int16
+
 
 def dist_setup(args):
     import torch
@@ -216,15 +256,23 @@ def run_lsa(args):
     T, hkv, hq = c["T"], c["hkv"], c["hq"]
     cfg = lsa.Config(k=c["k"], sinks=c["sinks"], window=c["window"], beam=c["beam"],
                      mode=c["mode"], agg=c["agg"])
-    inp = synth.layer_inputs(args.workload, seed=rank, T=T)
     dev = torch.device("cuda", torch.cuda.current_device())
+    host_drawn = T <= 131072
+    if host_drawn:
+        inp = synth.layer_inputs(args.workload, seed=rank, T=T)
 
-    def pinned(bits):
-        return torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).pin_memory()
+        def pinned(bits):
+            return torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).pin_memory()
 
-    hQ, hK, hV = pinned(inp["Q"]), pinned(inp["K"]), pinned(inp["V"])
-    Q, K, V = hQ.to(dev), hK.to(dev), hV.to(dev)
-    Wk, Wq = torch.from_numpy(inp["Wk"]).to(dev), torch.from_numpy(inp["Wq"]).to(dev)
+        hQ, hK, hV = pinned(inp["Q"]), pinned(inp["K"]), pinned(inp["V"])
+        Q, K, V = hQ.to(dev), hK.to(dev), hV.to(dev)
+        Wk_np, Wq_np = inp["Wk"], inp["Wq"]
+    else:
+        Q, K, V = device_layer(c, rank, dev)
+        hQ, hK, hV = (x.cpu().pin_memory() for x in (Q, K, V))
+        Wk_np, Wq_np = synth.projections(rank, c["d"], c["dl"])
+        inp = {"Wk": Wk_np, "Wq": Wq_np}
+    Wk, Wq = torch.from_numpy(Wk_np).to(dev), torch.from_numpy(Wq_np).to(dev)
     cache = lsa.Cache(hkv, T, cfg, device=dev)
     tree = lsa.Tree(cache, device=dev) if cfg.mode == 1 else None
     O = torch.empty_like(Q)
@@ -360,7 +408,11 @@ def run_lsa(args):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu:
-        per_layer, desc, spent = oracle_sample(inp, c, n_blocks=None if T <= 131072 else 64, n_queries=256)
+        if not host_drawn:  # the oracle sample reads head 0's K/V and the query rows
+            inp = {"Wk": Wk_np, "Wq": Wq_np, "K": bits_of(hK[:, :1]), "V": bits_of(hV[:, :1]),
+                   "Q": bits_of(hQ)}
+        per_layer, desc, spent = oracle_sample(inp, c, n_blocks=None if T <= 131072 else 64,
+                                               n_queries=256 if T <= 131072 else 64)
         cpu = {"value": T / per_layer, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": desc,
                "sample_seconds": spent}
 
@@ -380,9 +432,118 @@ def run_lsa(args):
         dist.destroy_process_group()
 
 
+def run_decode(args):
+    """Batched decode: `batch` requests whose caches hold T - 32 tokens (built
+    with lsa_decode_load, outside the timing); a step is one lsa_decode_step
+    (one new token per request).  The 32nd step completes a 512-key block in
+    every request, so the timed steps include one streaming Ward pass."""
+    import torch
+    import torch.distributed as dist
+
+    import clustered_key_indexing_b200 as lsa
+    from clustered_key_indexing_b200._lib import check, lib
+
+    world, rank, local = dist_setup(args)
+    c = workload_cfg(args)
+    B, hkv, hq, T = c["batch"], c["hkv"], c["hq"], c["T"]
+    cfg = lsa.Config(k=c["k"], sinks=c["sinks"], window=c["window"], beam=c["beam"],
+                     mode=c["mode"], agg=c["agg"])
+    dev = torch.device("cuda", torch.cuda.current_device())
+    cap = T + 512
+    n0 = T - 32
+    dec = lsa.Decode(B, hkv, hq, cap, cfg, device=dev)
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(1000 * rank)
+    mu = torch.from_numpy(synth.centres(rank, c["n_centres"], c["d"])).to(dev)
+    Wk_np, Wq_np = synth.projections(rank, c["d"], c["dl"])
+    Wk, Wq = torch.from_numpy(Wk_np).to(dev), torch.from_numpy(Wq_np).to(dev)
+    ccfg = cfg.c()
+    for r in range(B):
+        device_tokens(n0, hkv, c["d"], mu, 4.0, gen, dev, out=dec.K[r, :n0])
+        device_tokens(n0, hkv, c["d"], mu, 0.0, gen, dev, out=dec.V[r, :n0])
+        check(lib().lsa_decode_load(ctypes_ref(dec.d), r, n0, ctypes_ptr(Wk), ctypes_ref(ccfg),
+                                    ctypes_ptr(dec.ws), dec.ws.numel(), None), "lsa_decode_load")
+    nsteps = args.warmup + args.steps
+    q = device_tokens(nsteps * B, hq, c["d"], mu, 1.0, gen, dev).view(nsteps, B, hq, c["d"])
+    kk = device_tokens(nsteps * B, hkv, c["d"], mu, 4.0, gen, dev).view(nsteps, B, hkv, c["d"])
+    vv = device_tokens(nsteps * B, hkv, c["d"], mu, 0.0, gen, dev).view(nsteps, B, hkv, c["d"])
+    o = torch.empty((B, hq, c["d"]), dtype=torch.bfloat16, device=dev)
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+    for s_ in range(args.warmup):
+        dec.step(q[s_], kk[s_], vv[s_], Wk, Wq, o=o)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    lens0 = dec.len
+    clocks = Clocks(torch.cuda.current_device())
+    nl0 = lib().lsa_launch_count()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for s_ in range(args.warmup, nsteps):
+        dec.step(q[s_], kk[s_], vv[s_], Wk, Wq, o=o)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    launches = lib().lsa_launch_count() - nl0
+    ms = e0.elapsed_time(e1)
+    if world > 1:
+        tt = torch.tensor([ms], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms = float(tt.item())
+    lsa.check_device_error()
+    ms_step = ms / args.steps
+    # algorithmic bytes per step: every eligible centroid (128 B) with its
+    # minlr word, the gathered K/V rows of every index entry (512 B), Q and O
+    row = cfg.row
+    byts = 0.0
+    for t in lens0:
+        for s_ in range(args.steps):
+            pos = t + s_
+            lim = pos - c["window"]
+            nb = min(cap // 512 * 64, 64 * (lim // 512 + 1))
+            nb = min(nb, 64 * ((pos + 1) // 512))
+            byts += hkv * (nb * 132 + row * 512) + 2 * hq * c["d"] * 2
+    byts /= args.steps
+    pk, src = peaks()
+    achieved = byts / (ms_step / 1e3) / 1e9
+    if rank == 0:
+        line = {
+            "metric": "LSA decode steps/s", "value": world / (ms_step / 1e3), "unit": "steps/s",
+            "tokens_per_s": world * B / (ms_step / 1e3), "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": args.workload, "batch": B, "context": T, "hkv": hkv, "hq": hq,
+                       "k": c["k"], "sinks": c["sinks"], "window": c["window"],
+                       "search": "flat" if c["mode"] == 0 else f"tree(beam={c['beam']})",
+                       "inputs": "device-drawn (torch Philox), same recipe as synth",
+                       "l2": "no flush: per-step centroid scan (4.3 GB) is larger than L2"},
+            "clocks": clk, "gpu_launches": int(launches),
+            "roofline": {"kernel": "decode step (centroid scan + gather + attention)", "bound": "hbm",
+                         "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                         "frac": achieved / pk["hbm_gbs"], "traffic": None, "peak_source": src,
+                         "bytes_per_step": byts},
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+def ctypes_ref(x):
+    import ctypes
+    return ctypes.byref(x)
+
+
+def ctypes_ptr(t):
+    import ctypes
+    return ctypes.c_void_p(t.data_ptr())
+
+
 if __name__ == "__main__":
     a = parse()
     if a.impl == "reference":
         run_reference(a)
+    elif a.workload.startswith("decode"):
+        run_decode(a)
     else:
         run_lsa(a)
