@@ -117,6 +117,23 @@ class Clocks:
                 "reasons": reasons, "samples": len(rows)}
 
 
+def emit_json(line):
+    """Print the result line; any non-JSON value (reported on stderr with its
+    key) is printed as text."""
+    def walk(o, path):
+        if isinstance(o, dict):
+            for k, v in o.items():
+                walk(v, f"{path}.{k}")
+        elif isinstance(o, (list, tuple)):
+            for i, v in enumerate(o):
+                walk(v, f"{path}[{i}]")
+        elif not isinstance(o, (str, int, float, bool, type(None))):
+            print(f"bench.py: non-JSON value at {path}: {type(o).__name__} {o!r:.80}", file=sys.stderr)
+    walk(line, "line")
+    print(json.dumps(line, default=lambda o: o.decode(errors="replace") if isinstance(o, bytes) else str(o)),
+          flush=True)
+
+
 def peaks():
     try:
         return json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json"))), "measured"
@@ -240,7 +257,7 @@ def run_reference(args):
         "cpu_baseline": {"value": v, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": desc},
         "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
-    print(json.dumps(line), flush=True)
+    emit_json(line)
 
 
 def run_lsa(args):
@@ -427,7 +444,7 @@ def run_lsa(args):
                                    "attention": attn_ms / args.steps},
             "select_fallback_rows_per_step": fallback_rows / args.steps,
         }
-        print(json.dumps(line), flush=True)
+        emit_json(line)
     if world > 1:
         dist.destroy_process_group()
 
@@ -524,7 +541,7 @@ def run_decode(args):
                          "frac": achieved / pk["hbm_gbs"], "traffic": None, "peak_source": src,
                          "bytes_per_step": byts},
         }
-        print(json.dumps(line), flush=True)
+        emit_json(line)
     if world > 1:
         dist.destroy_process_group()
 
