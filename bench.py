@@ -411,8 +411,8 @@ def run_lsa(args):
     traffic = None
     try:
         import hashlib
-        src = open(os.path.join(ROOT, ATTN_TRAFFIC["source"]), "rb").read()
-        if (hashlib.sha256(src).hexdigest()[:16] == ATTN_TRAFFIC["sha256_prefix"]
+        attn_src = open(os.path.join(ROOT, ATTN_TRAFFIC["source"]), "rb").read()
+        if (hashlib.sha256(attn_src).hexdigest()[:16] == ATTN_TRAFFIC["sha256_prefix"]
                 and args.workload == ATTN_TRAFFIC["workload"]):
             traffic = ATTN_TRAFFIC["bytes_per_query_kvhead"] * chunk * hkv
     except OSError:
