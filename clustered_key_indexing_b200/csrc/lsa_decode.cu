@@ -16,11 +16,12 @@
 //   query latents, then flat (decode_score_kernel + decode_resolve_kernel)
 //                          or tree (tree_select_kernel) selection;
 //   attn_kernel<8>         eight warps share each (request, kv-head) row.
-// Flat scores: one HBM pass over the request's eligible centroids (fp32 dot
-// products from 16-byte loads, 8 lanes per centroid), then one CTA per row:
-// weighted histogram on bins of width >= 2e around the row's score range,
-// exact fp64 rescoring of the two top bins' buckets, weighted radix select,
-// key emission in bucket-id order; rows whose band overflows shared memory
+// Flat scores: one HBM pass over the request's eligible centroids (one lane
+// per centroid, fp32 dot products) storing each slot's score bin (2048 bins
+// of width >= 2e over the row's score range) and key weight; then one CTA per
+// row: weighted histogram of the bins, the two bins around the k-th key kept
+// (warp-ordered compaction), exact fp64 rescoring, weighted radix select, key
+// emission in bucket-id order.  Rows whose kept bins overflow shared memory
 // take exact fp64 scores of every eligible bucket in a global slot.
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -147,6 +148,7 @@ __global__ void __launch_bounds__(256) tail_units_kernel(const uint16_t* __restr
 // ------------------------------------------------------ flat decode scores
 
 constexpr int kDecScoreCols = 2048;  // bucket slots per CTA
+constexpr int kDecBins = 2048;       // histogram bins over the row's score range
 
 struct DecScoreArgs {
     const uint16_t* Y;        // [batch, hkv, 64] (mean) / [batch, hq, 64] (native)
@@ -158,8 +160,8 @@ struct DecScoreArgs {
     int64_t cap_buckets, ld;
     int32_t hkv, G, agg, S, W;
     int64_t T_built;
-    float* sc;                // [rows, ld]
-    uint8_t* wt;              // [rows, ld]
+    uint16_t* bin;            // [rows, ld] score bin of every slot
+    uint8_t* wt;              // [rows, ld] keys of the slot in [S, t-W] (0 = not eligible)
     int64_t pos[LSA_MAX_BATCH];
 };
 
@@ -175,11 +177,30 @@ __device__ __forceinline__ int weight_units(int64_t b, int32_t pk, int64_t lim, 
     return w;
 }
 
-// grid (column chunks, rows); 8 warps, each 256 buckets, 8 lanes per bucket.
-// NG = query latents per row (1 for the group mean, G for the native max).
+// Score range of a row: |score| <= |y| (native: max over its heads); the
+// floor 0.25 keeps every one of the 2048 bins at least 2e = 2e-4 wide.
+__device__ __forceinline__ float row_radius(const uint16_t* y, int ng) {
+    float R = 0.f;
+    for (int g = 0; g < ng; ++g) {
+        float n2 = 0.f;
+        for (int i = 0; i < kDL; ++i) { const float v = bf16_to_f32(y[g * kDL + i]); n2 += v * v; }
+        R = fmaxf(R, sqrtf(n2));
+    }
+    return fmaxf(0.25f, fminf(1.0625f, R * 1.01f + 1e-6f));
+}
+
+__device__ __forceinline__ int score_to_bin(float s, float R) {
+    int bin = __float2int_rd((s + R) * ((float)kDecBins / (2.f * R)));
+    return bin < 0 ? 0 : (bin >= kDecBins ? kDecBins - 1 : bin);
+}
+
+// grid (column chunks, rows); one lane per bucket slot: eight 16-byte loads of
+// its centroid, a private fp32 dot product per query latent; coalesced
+// metadata loads and bin / weight stores.  NG = latents per row.
 template <int NG>
 __global__ void __launch_bounds__(256) decode_score_kernel(DecScoreArgs a) {
-    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    __shared__ float ys[NG][kDL];
+    __shared__ float rad;
     const int64_t row = blockIdx.y;
     const int64_t r = row / a.hkv;
     const int64_t t = a.pos[r];
@@ -187,69 +208,48 @@ __global__ void __launch_bounds__(256) decode_score_kernel(DecScoreArgs a) {
     const int64_t ncol = lim < 0 ? 0 : min(a.cap_buckets, (int64_t)kBucketsPerBlock * (lim / kBlockKeys + 1));
     const int64_t c0 = (int64_t)blockIdx.x * kDecScoreCols;
     if (c0 >= ncol) return;
-    const int part = lane & 7;
-    // this lane's 8 latent dims of each of the NG query latents
-    float y[NG][8];
     const uint16_t* yb = a.Y + (row * NG) * kDL;  // native: row*G = r*hq + h*G
-#pragma unroll
-    for (int g = 0; g < NG; ++g) {
-        const uint4 yv = *reinterpret_cast<const uint4*>(yb + g * kDL + part * 8);
-        const uint32_t u[4] = {yv.x, yv.y, yv.z, yv.w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            y[g][2 * e] = __uint_as_float(u[e] << 16);
-            y[g][2 * e + 1] = __uint_as_float(u[e] & 0xFFFF0000u);
-        }
-    }
+    for (int i = threadIdx.x; i < NG * kDL; i += blockDim.x) ys[i / kDL][i % kDL] = bf16_to_f32(yb[i]);
+    if (threadIdx.x == 0) rad = row_radius(yb, NG);
+    __syncthreads();
+    const float R = rad;
     const uint16_t* cb = a.cent + row * a.cap_buckets * kDL;
     const int64_t hb0 = row * a.cap_buckets;
-    const int64_t wbase = c0 + (int64_t)wid * (kDecScoreCols / 8);
-#pragma unroll 4
-    for (int it = 0; it < kDecScoreCols / 8 / 4; ++it) {
-        const int64_t b = wbase + it * 4 + (lane >> 3);
-        const bool in = b < ncol;
-        uint4 cv = make_uint4(0, 0, 0, 0);
-        if (in) cv = __ldg(reinterpret_cast<const uint4*>(cb + b * kDL + part * 8));
-        const uint32_t u[4] = {cv.x, cv.y, cv.z, cv.w};
-        float c8[8];
+    for (int64_t b = c0 + threadIdx.x; b < min(ncol, c0 + kDecScoreCols); b += blockDim.x) {
+        uint4 cv[8];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            c8[2 * e] = __uint_as_float(u[e] << 16);
-            c8[2 * e + 1] = __uint_as_float(u[e] & 0xFFFF0000u);
-        }
+        for (int i = 0; i < 8; ++i) cv[i] = __ldg(reinterpret_cast<const uint4*>(cb + b * kDL) + i);
+        const int32_t mlr = __ldg(a.minlr + hb0 + b);
+        const int32_t mxp = __ldg(a.maxpos + hb0 + b);
+        const int32_t clr = __ldg(a.cnt_lr + hb0 + b);
         float best = -CUDART_INF_F;
 #pragma unroll
         for (int g = 0; g < NG; ++g) {
             float s = 0.f;
 #pragma unroll
-            for (int e = 0; e < 8; ++e) s = fmaf(y[g][e], c8[e], s);
-            s += __shfl_xor_sync(0xffffffffu, s, 1);
-            s += __shfl_xor_sync(0xffffffffu, s, 2);
-            s += __shfl_xor_sync(0xffffffffu, s, 4);
+            for (int i = 0; i < 8; ++i) {
+                const uint32_t u[4] = {cv[i].x, cv[i].y, cv[i].z, cv[i].w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    s = fmaf(ys[g][8 * i + 2 * e], __uint_as_float(u[e] << 16), s);
+                    s = fmaf(ys[g][8 * i + 2 * e + 1], __uint_as_float(u[e] & 0xFFFF0000u), s);
+                }
+            }
             best = fmaxf(best, s);
         }
-        if (in && part == 0) {
-            const int32_t mlr = a.minlr[hb0 + b];
-            const bool el = (int64_t)mlr <= lim;
-            int w = 0;
-            if (el) {
-                const int32_t mxp = a.maxpos[hb0 + b];
-                w = (int64_t)mxp <= lim ? a.cnt_lr[hb0 + b] : weight_units(b, a.units[hb0 + b], lim, a.S, a.T_built);
-            }
-            a.sc[row * a.ld + b] = el ? best : -CUDART_INF_F;
-            a.wt[row * a.ld + b] = (uint8_t)w;
-        }
+        int w = 0;
+        if ((int64_t)mlr <= lim)
+            w = (int64_t)mxp <= lim ? clr : weight_units(b, __ldg(a.units + hb0 + b), lim, a.S, a.T_built);
+        a.bin[row * a.ld + b] = (uint16_t)score_to_bin(best, R);
+        a.wt[row * a.ld + b] = (uint8_t)w;
     }
 }
 
 // ---------------------------------------------------- flat decode resolve
 
-constexpr float kDecErr = 1e-4f;   // bound on |fp32 score - exact score|
-constexpr int kDecBins = 2048;
-
 struct DecResolveArgs {
     SelectArgs s;            // cache, cfg, idx, decode positions (row_info)
-    const float* sc;
+    const uint16_t* bin;
     uint8_t* wt;             // weights in, taken counts out (fallback rows)
     double* slot;            // [rows, ld] exact scores (fallback rows)
     int64_t ld;
@@ -258,9 +258,9 @@ struct DecResolveArgs {
 
 __global__ void __launch_bounds__(kSelThreads) decode_resolve_kernel(DecResolveArgs d) {
     __shared__ SelShared sh;
-    __shared__ float rad_s;
+    __shared__ int wcnt[kSelThreads / 32];
     const SelectArgs& a = d.s;
-    const int tid = threadIdx.x;
+    const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
     const int64_t row = blockIdx.x;
     const RowInfo r = row_info(a, row);
     write_sinks_window(a, r);
@@ -269,24 +269,9 @@ __global__ void __launch_bounds__(kSelThreads) decode_resolve_kernel(DecResolveA
         return;
     }
     load_latents(a, r, sh);
-    __syncthreads();
     const int ng = a.agg ? a.G : 1;
-    if (tid == 0) {
-        // score range [-R, R]: |score| <= |y| (native: max over heads);
-        // R >= 0.25 keeps every bin >= 2e wide
-        float R = 0.f;
-        for (int g = 0; g < ng; ++g) {
-            float n2 = 0.f;
-            for (int i = 0; i < kDL; ++i) { const float v = bf16_to_f32(sh.ylat[g * kDL + i]); n2 += v * v; }
-            R = fmaxf(R, sqrtf(n2));
-        }
-        rad_s = fmaxf(0.25f, fminf(1.0625f, R * 1.01f + 1e-6f));
-    }
-    __syncthreads();
-    const float R = rad_s;
-    const float bscale = (float)kDecBins / (2.f * R);
     const int64_t ncol = min(d.cap_buckets, (int64_t)kBucketsPerBlock * (r.lim / kBlockKeys + 1));
-    const float* srow = d.sc + row * d.ld;
+    const uint16_t* brow = d.bin + row * d.ld;
     uint8_t* wrow = d.wt + row * d.ld;
     for (int i = tid; i < kDecBins; i += kSelThreads) sh.hist[i] = 0ull;
     __syncthreads();
@@ -295,14 +280,12 @@ __global__ void __launch_bounds__(kSelThreads) decode_resolve_kernel(DecResolveA
         const int w = wrow[b];
         if (w == 0) continue;
         myw += w;
-        int bin = __float2int_rd((srow[b] + R) * bscale);
-        bin = bin < 0 ? 0 : (bin >= kDecBins ? kDecBins - 1 : bin);
-        atomicAdd(&sh.hist[bin], (1ull << 32) | (unsigned long long)w);
+        atomicAdd(&sh.hist[brow[b]], (1ull << 32) | (unsigned long long)w);
     }
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) myw += __shfl_xor_sync(0xffffffffu, myw, off);
     __shared__ long long wsum[kSelThreads / 32];
-    if ((tid & 31) == 0) wsum[tid >> 5] = myw;
+    if (lane == 0) wsum[wid] = myw;
     __syncthreads();
     long long totw = 0;
     for (int i = 0; i < kSelThreads / 32; ++i) totw += wsum[i];
@@ -312,7 +295,6 @@ __global__ void __launch_bounds__(kSelThreads) decode_resolve_kernel(DecResolveA
     }
     // cut bin j*: highest bin whose weight from the top reaches k; keep bins >= j* - 1
     if (tid < 32) {
-        const int lane = tid;
         long long s = 0;
         for (int dd = 0; dd < kDecBins / 32; ++dd)
             s += (long long)(sh.hist[kDecBins - 1 - (kDecBins / 32) * lane - dd] & 0xffffffffull);
@@ -343,22 +325,27 @@ __global__ void __launch_bounds__(kSelThreads) decode_resolve_kernel(DecResolveA
     int ncand;
     block_exscan(cnt, &ncand, sh.sh4);
     if (ncand <= kCap) {
-        // ordered compaction of the kept bins, exact rescoring, radix fill
-        int n = 0;
-        for (int64_t c0 = 0; c0 < ncol; c0 += kSelThreads) {
-            const int64_t b = c0 + tid;
-            bool el = false;
-            if (b < ncol && wrow[b] > 0) {
-                int bin = __float2int_rd((srow[b] + R) * bscale);
-                bin = bin < 0 ? 0 : (bin >= kDecBins ? kDecBins - 1 : bin);
-                el = bin >= jt;
-            }
-            int tot;
-            const int o = block_exscan(el ? 1 : 0, &tot, sh.sh4);
-            if (el) sh.cid[n + o] = (int)b;
-            n += tot;
+        // warp-ordered compaction: warp w takes a contiguous quarter of the
+        // slots, so concatenating the warps' lists keeps ascending ids
+        const int64_t per = (ncol + kSelThreads / 32 - 1) / (kSelThreads / 32);
+        const int64_t b_lo = wid * per, b_hi = min(ncol, b_lo + per);
+        int c = 0;
+        for (int64_t b = b_lo + lane; b < b_hi; b += 32) c += (wrow[b] > 0 && brow[b] >= jt);
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) c += __shfl_xor_sync(0xffffffffu, c, off);
+        if (lane == 0) wcnt[wid] = c;
+        __syncthreads();
+        int base = 0;
+        for (int i = 0; i < wid; ++i) base += wcnt[i];
+        for (int64_t b0 = b_lo; b0 < b_hi; b0 += 32) {
+            const int64_t b = b0 + lane;
+            const bool el = b < b_hi && wrow[b] > 0 && brow[b] >= jt;
+            const unsigned bal = __ballot_sync(0xffffffffu, el);
+            if (el) sh.cid[base + __popc(bal & ((1u << lane) - 1u))] = (int)b;
+            base += __popc(bal);
         }
         __syncthreads();
+        const int n = ncand;
         const int64_t hb0 = (int64_t)r.h * d.cap_buckets;
         for (int i = tid; i < n; i += kSelThreads) {
             const int64_t b = sh.cid[i];
@@ -392,7 +379,7 @@ static int64_t decode_row_len(const lsa_cfg* cfg) { return cfg->sinks + cfg->k +
 struct DecodeWs {
     uint16_t* Y;
     int32_t* idx;
-    float* sc;
+    uint16_t* bin;
     uint8_t* wt;
     double* slot;
     double* Utmp;
@@ -409,7 +396,7 @@ static DecodeWs carve_decode(const lsa_cfg* cfg, const lsa_decode* d, char* base
     w.Y = (uint16_t*)take((size_t)d->batch * hy * kDL * 2);
     w.idx = (int32_t*)take((size_t)rows * decode_row_len(cfg) * 4);
     if (cfg->mode == 0) {
-        w.sc = (float*)take((size_t)rows * ld * 4);
+        w.bin = (uint16_t*)take((size_t)rows * ld * 2);
         w.wt = (uint8_t*)take((size_t)rows * ld);
         w.slot = (double*)take((size_t)rows * ld * 8);
     }
@@ -600,7 +587,7 @@ lsa_status lsa_decode_step(lsa_decode* d, const uint16_t* q, const uint16_t* k, 
         sa.Y = w.Y; sa.cent = d->cache.cent; sa.minlr = d->cache.minlr; sa.maxpos = d->cache.maxpos;
         sa.cnt_lr = d->cache.cnt_lr; sa.units = d->cache.units; sa.cap_buckets = d->cache.cap_buckets;
         sa.ld = ld; sa.hkv = d->hkv; sa.G = d->hq / d->hkv; sa.agg = cfg->agg; sa.S = cfg->sinks;
-        sa.W = cfg->window; sa.T_built = d->cap; sa.sc = w.sc; sa.wt = w.wt;
+        sa.W = cfg->window; sa.T_built = d->cap; sa.bin = w.bin; sa.wt = w.wt;
         for (int r = 0; r < d->batch; ++r) sa.pos[r] = a.pos[r];
         dim3 grid((unsigned)ceil_div<int64_t>(d->cache.cap_buckets, kDecScoreCols), (unsigned)rows);
         const int ng = cfg->agg ? d->hq / d->hkv : 1;
@@ -610,7 +597,7 @@ lsa_status lsa_decode_step(lsa_decode* d, const uint16_t* q, const uint16_t* k, 
         else decode_score_kernel<8><<<grid, 256, 0, st>>>(sa);
         if ((s = check_launch("decode_score_kernel")) != LSA_OK) return s;
         DecResolveArgs ra{};
-        ra.s = a; ra.sc = w.sc; ra.wt = w.wt; ra.slot = w.slot; ra.ld = ld; ra.cap_buckets = d->cache.cap_buckets;
+        ra.s = a; ra.bin = w.bin; ra.wt = w.wt; ra.slot = w.slot; ra.ld = ld; ra.cap_buckets = d->cache.cap_buckets;
         decode_resolve_kernel<<<(unsigned)rows, kSelThreads, 0, st>>>(ra);
         if ((s = check_launch("decode_resolve_kernel")) != LSA_OK) return s;
     }
