@@ -215,33 +215,47 @@ __global__ void __launch_bounds__(256) decode_score_kernel(DecScoreArgs a) {
     const float R = rad;
     const uint16_t* cb = a.cent + row * a.cap_buckets * kDL;
     const int64_t hb0 = row * a.cap_buckets;
-    for (int64_t b = c0 + threadIdx.x; b < min(ncol, c0 + kDecScoreCols); b += blockDim.x) {
-        uint4 cv[8];
+    const int64_t cend = min(ncol, c0 + kDecScoreCols);
+    // two slots per thread per iteration: 16 loads of 16 bytes in flight
+    for (int64_t b0 = c0 + threadIdx.x; b0 < cend; b0 += 2 * blockDim.x) {
+        int64_t bb[2] = {b0, b0 + blockDim.x};
+        bool ok[2] = {true, b0 + blockDim.x < cend};
+        uint4 cv[2][8];
+        int32_t mlr[2], mxp[2], clr[2];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) cv[i] = __ldg(reinterpret_cast<const uint4*>(cb + b * kDL) + i);
-        const int32_t mlr = __ldg(a.minlr + hb0 + b);
-        const int32_t mxp = __ldg(a.maxpos + hb0 + b);
-        const int32_t clr = __ldg(a.cnt_lr + hb0 + b);
-        float best = -CUDART_INF_F;
+        for (int u2 = 0; u2 < 2; ++u2) {
+            const int64_t b = ok[u2] ? bb[u2] : b0;
 #pragma unroll
-        for (int g = 0; g < NG; ++g) {
-            float s = 0.f;
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const uint32_t u[4] = {cv[i].x, cv[i].y, cv[i].z, cv[i].w};
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    s = fmaf(ys[g][8 * i + 2 * e], __uint_as_float(u[e] << 16), s);
-                    s = fmaf(ys[g][8 * i + 2 * e + 1], __uint_as_float(u[e] & 0xFFFF0000u), s);
-                }
-            }
-            best = fmaxf(best, s);
+            for (int i = 0; i < 8; ++i) cv[u2][i] = __ldg(reinterpret_cast<const uint4*>(cb + b * kDL) + i);
+            mlr[u2] = __ldg(a.minlr + hb0 + b);
+            mxp[u2] = __ldg(a.maxpos + hb0 + b);
+            clr[u2] = __ldg(a.cnt_lr + hb0 + b);
         }
-        int w = 0;
-        if ((int64_t)mlr <= lim)
-            w = (int64_t)mxp <= lim ? clr : weight_units(b, __ldg(a.units + hb0 + b), lim, a.S, a.T_built);
-        a.bin[row * a.ld + b] = (uint16_t)score_to_bin(best, R);
-        a.wt[row * a.ld + b] = (uint8_t)w;
+#pragma unroll
+        for (int u2 = 0; u2 < 2; ++u2) {
+            if (!ok[u2]) continue;
+            const int64_t b = bb[u2];
+            float best = -CUDART_INF_F;
+#pragma unroll
+            for (int g = 0; g < NG; ++g) {
+                float sacc = 0.f;
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const uint32_t u[4] = {cv[u2][i].x, cv[u2][i].y, cv[u2][i].z, cv[u2][i].w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        sacc = fmaf(ys[g][8 * i + 2 * e], __uint_as_float(u[e] << 16), sacc);
+                        sacc = fmaf(ys[g][8 * i + 2 * e + 1], __uint_as_float(u[e] & 0xFFFF0000u), sacc);
+                    }
+                }
+                best = fmaxf(best, sacc);
+            }
+            int w = 0;
+            if ((int64_t)mlr[u2] <= lim)
+                w = (int64_t)mxp[u2] <= lim ? clr[u2] : weight_units(b, __ldg(a.units + hb0 + b), lim, a.S, a.T_built);
+            a.bin[row * a.ld + b] = (uint16_t)score_to_bin(best, R);
+            a.wt[row * a.ld + b] = (uint8_t)w;
+        }
     }
 }
 
@@ -275,12 +289,31 @@ __global__ void __launch_bounds__(kSelThreads) decode_resolve_kernel(DecResolveA
     uint8_t* wrow = d.wt + row * d.ld;
     for (int i = tid; i < kDecBins; i += kSelThreads) sh.hist[i] = 0ull;
     __syncthreads();
+    // 16 slots per lane per step: one 16-byte load of weights, two of bins
+    auto load16 = [&](int64_t g16, uint8_t (&w16)[16], uint16_t (&b16)[16]) {
+        const uint4 wv = *reinterpret_cast<const uint4*>(wrow + g16 * 16);
+        const uint4 bv0 = *reinterpret_cast<const uint4*>(brow + g16 * 16);
+        const uint4 bv1 = *reinterpret_cast<const uint4*>(brow + g16 * 16 + 8);
+        const uint32_t wu[4] = {wv.x, wv.y, wv.z, wv.w};
+        const uint32_t bu[8] = {bv0.x, bv0.y, bv0.z, bv0.w, bv1.x, bv1.y, bv1.z, bv1.w};
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            w16[i] = (g16 * 16 + i < ncol) ? (uint8_t)((wu[i >> 2] >> (8 * (i & 3))) & 0xFF) : 0;
+            b16[i] = (uint16_t)((bu[i >> 1] >> (16 * (i & 1))) & 0xFFFF);
+        }
+    };
+    const int64_t ng16 = (ncol + 15) / 16;
     long long myw = 0;
-    for (int64_t b = tid; b < ncol; b += kSelThreads) {
-        const int w = wrow[b];
-        if (w == 0) continue;
-        myw += w;
-        atomicAdd(&sh.hist[brow[b]], (1ull << 32) | (unsigned long long)w);
+    for (int64_t g16 = tid; g16 < ng16; g16 += kSelThreads) {
+        uint8_t w16[16];
+        uint16_t b16[16];
+        load16(g16, w16, b16);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            if (w16[i] == 0) continue;
+            myw += w16[i];
+            atomicAdd(&sh.hist[b16[i]], (1ull << 32) | (unsigned long long)w16[i]);
+        }
     }
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) myw += __shfl_xor_sync(0xffffffffu, myw, off);
@@ -326,23 +359,48 @@ __global__ void __launch_bounds__(kSelThreads) decode_resolve_kernel(DecResolveA
     block_exscan(cnt, &ncand, sh.sh4);
     if (ncand <= kCap) {
         // warp-ordered compaction: warp w takes a contiguous quarter of the
-        // slots, so concatenating the warps' lists keeps ascending ids
-        const int64_t per = (ncol + kSelThreads / 32 - 1) / (kSelThreads / 32);
-        const int64_t b_lo = wid * per, b_hi = min(ncol, b_lo + per);
+        // 16-slot groups and lane l the l-th group of each 512-slot stretch,
+        // so the concatenated lists keep ascending ids
+        const int64_t per = (ng16 + kSelThreads / 32 - 1) / (kSelThreads / 32);
+        const int64_t g_lo = wid * per, g_hi = min(ng16, g_lo + per);
         int c = 0;
-        for (int64_t b = b_lo + lane; b < b_hi; b += 32) c += (wrow[b] > 0 && brow[b] >= jt);
+        for (int64_t g16 = g_lo + lane; g16 < g_hi; g16 += 32) {
+            uint8_t w16[16];
+            uint16_t b16[16];
+            load16(g16, w16, b16);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) c += (w16[i] > 0 && b16[i] >= jt);
+        }
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) c += __shfl_xor_sync(0xffffffffu, c, off);
         if (lane == 0) wcnt[wid] = c;
         __syncthreads();
         int base = 0;
         for (int i = 0; i < wid; ++i) base += wcnt[i];
-        for (int64_t b0 = b_lo; b0 < b_hi; b0 += 32) {
-            const int64_t b = b0 + lane;
-            const bool el = b < b_hi && wrow[b] > 0 && brow[b] >= jt;
-            const unsigned bal = __ballot_sync(0xffffffffu, el);
-            if (el) sh.cid[base + __popc(bal & ((1u << lane) - 1u))] = (int)b;
-            base += __popc(bal);
+        for (int64_t s0 = g_lo; s0 < g_hi; s0 += 32) {
+            const int64_t g16 = s0 + lane;
+            uint32_t hits = 0;
+            if (g16 < g_hi) {
+                uint8_t w16[16];
+                uint16_t b16[16];
+                load16(g16, w16, b16);
+#pragma unroll
+                for (int i = 0; i < 16; ++i) hits |= (uint32_t)(w16[i] > 0 && b16[i] >= jt) << i;
+            }
+            const int nh = __popc(hits);
+            int incl = nh;
+#pragma unroll
+            for (int off = 1; off < 32; off <<= 1) {
+                const int y = __shfl_up_sync(0xffffffffu, incl, off);
+                if (lane >= off) incl += y;
+            }
+            int o = base + incl - nh;
+            while (hits) {
+                const int i = __ffs(hits) - 1;
+                hits &= hits - 1;
+                sh.cid[o++] = (int)(g16 * 16 + i);
+            }
+            base += __shfl_sync(0xffffffffu, incl, 31);
         }
         __syncthreads();
         const int n = ncand;
