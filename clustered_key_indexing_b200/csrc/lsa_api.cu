@@ -173,7 +173,8 @@ lsa_status lsa_check_device_error(void) {
     cudaMemcpyToSymbol(g_lsa_device_error, &zero, sizeof(int));
     const char* what = v == kErrWardInfeasible ? "Ward: no eligible merge left"
                      : v == kErrSelectOverflow ? "select: candidate list overflow"
-                     : v == kErrIndexRange ? "attention: index entry >= T" : "unknown";
+                     : v == kErrIndexRange ? "attention: index entry >= T"
+                     : v == kErrTcTimeout  ? "tensor-core pipeline wait timed out" : "unknown";
     return set_error(LSA_EDEVICE, "device error %d: %s", v, what);
 }
 
@@ -240,6 +241,7 @@ lsa_status lsa_select(const uint16_t* Q, int64_t t0, int64_t nq, int32_t hq, con
     if ((s = check_heads(hq, cache->hkv)) != LSA_OK) return s;
     if (!Q || !W_q || !idx) return set_error(LSA_EINVAL, "lsa_select: NULL pointer");
     if (!aligned16(Q)) return set_error(LSA_EINVAL, "lsa_select: Q must be 16-byte aligned");
+    if (Y_out && !aligned16(Y_out)) return set_error(LSA_EINVAL, "lsa_select: Y_out must be 16-byte aligned");
     if (nq <= 0 || t0 < 0) return set_error(LSA_EINVAL, "lsa_select: need nq > 0 and t0 >= 0");
     if (t0 + nq > (int64_t)INT32_MAX) return set_error(LSA_EUNSUPPORTED, "lsa_select: positions beyond 2^31");
     if (cfg->mode == 1) {

@@ -32,6 +32,7 @@ enum DeviceError : int {
     kErrWardInfeasible = 1,   // no eligible pair before the target count
     kErrSelectOverflow = 2,   // candidate list exceeded its capacity
     kErrIndexRange = 3,       // an index list entry was >= T
+    kErrTcTimeout = 4,        // a tensor-core pipeline wait ran out (mbarrier never completed)
 };
 
 // Rows of the flat search that took the exact fallback (diagnostics).

@@ -2,48 +2,65 @@
 // 当注意力学会先查目录再翻书", ch. 3: score every centroid, expand the best
 // buckets until k long-range keys are filled; ch. 5: native max over heads].
 //
-// Three kernels per chunk of query positions:
-//   flat_pass_kernel<sample=true>   bf16 tensor-core scores (mma.sync
-//       m16n8k16, fp32 accumulate) of 64 query rows against every 8th
-//       centroid; a per-row weighted histogram of those scores (bins scaled to
-//       the row's latent norm, which bounds its scores) gives a threshold tau
-//       expected to keep about twice the k keys needed;
-//   flat_pass_kernel<sample=false>  the same contraction over every eligible
-//       centroid; scores >= tau are appended to the row's candidate list in
-//       ascending bucket id;
-//   flat_resolve_kernel             one warp per (query, kv-head): eligibility
-//       and exact key counts, weighted radix select on the fp32 scores for the
+// Per chunk of query positions:
+//   sample_gather_kernel (once per call)  every 8th centroid of each kv-head
+//       and its (first eligible position, key count), packed contiguously;
+//   flat_tc_kernel  one CTA per 128 latent rows of one kv-head, on the 5th-
+//       generation tensor cores (TMA -> shared memory -> tcgen05.mma ->
+//       TMEM, bf16 in, fp32 accumulate).  Phase 1 scores the rows against the
+//       sampled centroids and builds a per-row weighted histogram (bins
+//       scaled to the row's latent norm, which bounds its scores) whose upper
+//       tail gives a threshold tau expected to keep about twice the k keys
+//       needed; phase 2 scores every eligible centroid and appends scores
+//       >= tau to the row's candidate list in ascending bucket id;
+//   flat_resolve_kernel  one warp per (query, kv-head): eligibility and
+//       exact key counts, weighted radix select on the fp32 scores for the
 //       cut c32, exact fp64 rescoring of the buckets within 2e of c32 only,
 //       key emission in bucket id order, sinks and window.
 // Exactness: |fp32 score - exact score| < e = 1e-4 (the error is below
-// 64 * 2^-23 * |y||c|).  The exact score E* of the k-th key then lies in
-// [c32 - e, c32 + e]: buckets with fp32 score > c32 + 2e rank strictly above
-// it, buckets below c32 - 2e strictly below, and only the band between is
-// ranked on exact fp64 scores (score desc, bucket id asc).  The band must lie
-// above tau (every bucket in it is then a candidate); rows where it does not,
-// or whose list overflowed, go to the exact fallback kernel.
+// 64 * 2^-23 * |y||c|, whatever order the tensor core sums in).  The exact
+// score E* of the k-th key then lies in [c32 - e, c32 + e]: buckets with fp32
+// score > c32 + 2e rank strictly above it, buckets below c32 - 2e strictly
+// below, and only the band between is ranked on exact fp64 scores (score
+// desc, bucket id asc).  The band must lie above tau (every bucket in it is
+// then a candidate); rows where it does not, or whose list overflowed, go to
+// the exact fallback kernel.
 #pragma once
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
 #include "lsa_common.cuh"
 #include "lsa_mma.cuh"
+#include "lsa_tc.cuh"
 
 namespace lsa {
 
 constexpr int kCandCap = 1024;       // candidates kept per (query, kv-head)
-constexpr int kSampleStride = 8;     // every 8th bucket scored by the sample pass
-constexpr int kSBins = 256;          // sample histogram bins over [-R, R], R = row latent norm
+constexpr int kSampleStride = 8;     // every 8th bucket scored by the sample phase
+constexpr int kSBins = 256;          // sample histogram bins over [-R, R], R = row latent norm bound
 constexpr int kOversample = 2;       // tau targets kOversample * k keys
 constexpr float kScoreErr = 1e-4f;   // bound on |fp32 score - exact score|
-constexpr int kPassCols = 128;
+
+// tcgen05 tile of the flat pass: M = 128 latent rows, N = 256 centroids,
+// K = 64 (four MMAs of K = 16), a 4-stage TMA ring of centroid tiles and two
+// TMEM accumulators (512 fp32 columns).
+constexpr int kTcRows = 128;
+constexpr int kTcCols = 256;
+constexpr int kTcStages = 4;
+constexpr int kTcThreads = 192;  // warp 0 TMA, warp 1 MMA + TMEM owner, warps 2-5 epilogue
+constexpr uint32_t kTcABytes = kTcRows * kDL * 2;  // 16 KB
+constexpr uint32_t kTcBBytes = kTcCols * kDL * 2;  // 32 KB
+constexpr uint32_t kTcTmemCols = 2 * kTcCols;
+constexpr uint32_t kTcHistBytes = kSBins * kTcRows * 2;  // uint16 bins [bin][row]
+constexpr size_t kTcSmemBytes = 1024 + kTcABytes + kTcStages * kTcBBytes + kTcHistBytes + 256;
+constexpr uint32_t kTcIdesc = umma_idesc_bf16(kTcRows, kTcCols);
+constexpr int kInfoPosBits = 27;     // packed sample info: count << 27 | min(first eligible position, 2^27 - 1)
 
 struct PassArgs {
     const uint16_t* Y;       // chunk latents [nqc, hkv, 64] (mean) / [nqc, hq, 64] (native)
-    const uint16_t* cent;    // [hkv, cap_buckets, 64]
-    const int32_t* minlr;    // [hkv, cap_buckets]
-    const int32_t* cnt_lr;   // [hkv, cap_buckets]
-    int64_t cap_buckets, NB, nqc, t_first;
+    const int32_t* info_s;   // [hkv, ns_cap] packed sample info of buckets 0, 8, 16, ...
+    int64_t cap_buckets, ns_cap, NB, nqc, t_first;
     int32_t W, hkv, G, agg, k;
     float* tau;              // [nqc * hkv]
     int32_t* cand_col;       // [nqc * hkv, kCandCap]
@@ -51,220 +68,274 @@ struct PassArgs {
     int32_t* cand_n;         // [nqc * hkv]
 };
 
-__device__ __forceinline__ int64_t flat_ncol_d(int64_t t, int32_t W, int64_t NB) {
+__host__ __device__ __forceinline__ int64_t flat_ncol_d(int64_t t, int32_t W, int64_t NB) {
     const int64_t lim = t - W;
     if (lim < 0) return 0;
     const int64_t n = (int64_t)kBucketsPerBlock * (lim / kBlockKeys + 1);
     return n < NB ? n : NB;
 }
 
-__device__ __forceinline__ void cp_async_4(uint32_t dst, const void* src, int src_bytes) {
-    asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;\n" ::"r"(dst), "l"(src), "r"(src_bytes));
+// cent_s[h, j] = cent[h, 8j] and info_s[h, j] = packed (minlr, cnt_lr) of
+// bucket 8j, for 8j < NB (zero centroid and no weight past it).
+__global__ void sample_gather_kernel(const uint16_t* __restrict__ cent, const int32_t* __restrict__ minlr,
+                                     const int32_t* __restrict__ cnt_lr, int64_t cap_buckets, int64_t NB,
+                                     int64_t ns_cap, int32_t hkv, uint16_t* __restrict__ cent_s,
+                                     int32_t* __restrict__ info_s) {
+    const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (idx >= (int64_t)hkv * ns_cap * 8) return;
+    const int64_t row = idx >> 3;
+    const int c = (int)(idx & 7);
+    const int64_t h = row / ns_cap, b = (row % ns_cap) * kSampleStride;
+    const bool ok = b < NB;
+    const int64_t src = h * cap_buckets + b;
+    reinterpret_cast<uint4*>(cent_s + row * kDL)[c] =
+        ok ? reinterpret_cast<const uint4*>(cent + src * kDL)[c] : make_uint4(0, 0, 0, 0);
+    if (c == 0) {
+        int32_t v = (1 << kInfoPosBits) - 1;
+        if (ok) {
+            const int32_t m = minlr[src], w = cnt_lr[src];
+            const int32_t mc = m < 0 ? 0 : (m > (1 << kInfoPosBits) - 1 ? (1 << kInfoPosBits) - 1 : m);
+            v = mc | ((w < 0 ? 0 : (w > 15 ? 15 : w)) << kInfoPosBits);
+        }
+        info_s[row] = v;
+    }
 }
 
-template <bool SAMPLE>
-__global__ void __launch_bounds__(128) flat_pass_kernel(PassArgs a) {
-    extern __shared__ __align__(128) uint8_t psm[];
-    uint16_t* ctile = reinterpret_cast<uint16_t*>(psm);                       // [2][128*64]
-    int32_t* mminlr = reinterpret_cast<int32_t*>(psm + 2 * kPassCols * kDL * 2);  // [2][128]
-    int32_t* mcnt = mminlr + 2 * kPassCols;                                   // [2][128]
-    float* rads = reinterpret_cast<float*>(mcnt + 2 * kPassCols);             // [64] row radii
-    uint32_t* hist = reinterpret_cast<uint32_t*>(rads + 64);                  // sample: [qpt][256]; full: [qpt]
+__global__ void __launch_bounds__(kTcThreads, 1)
+flat_tc_kernel(const __grid_constant__ CUtensorMap tmF, const __grid_constant__ CUtensorMap tmS, PassArgs a) {
+    extern __shared__ uint8_t tsm_raw[];
+    // 1024-byte alignment for the 128-byte swizzle atoms
+    uint8_t* tsm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(tsm_raw) + 1023) & ~(uintptr_t)1023);
+    uint8_t* sA = tsm;
+    uint8_t* sB = tsm + kTcABytes;
+    uint16_t* hist = reinterpret_cast<uint16_t*>(sB + kTcStages * kTcBBytes);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(hist) + kTcHistBytes);
+    // bars: full[S], empty[S], tfull[2], tempty[2], drain
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * kTcStages + 5);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
-    const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int h = blockIdx.y;
     const int G = a.agg ? a.G : 1;
-    const int qpt = 64 / G;
+    const int qpt = kTcRows / G;
     const int64_t q0 = (int64_t)blockIdx.x * qpt;
     if (q0 >= a.nqc) return;
     const int64_t qlast = min(a.nqc - 1, q0 + qpt - 1);
     const int64_t ncol_max = flat_ncol_d(a.t_first + qlast, a.W, a.NB);
-    const int64_t stride = SAMPLE ? kSampleStride : 1;
-    const int64_t nv = ceil_div<int64_t>(ncol_max, stride);
-    const int ntile = (int)ceil_div<int64_t>(nv, kPassCols);
+    const int ns_tiles = (int)ceil_div<int64_t>(ceil_div<int64_t>(ncol_max, kSampleStride), kTcCols);
+    const int ntiles = ns_tiles + (int)ceil_div<int64_t>(ncol_max, kTcCols);
 
-    for (int i = tid; i < qpt * (SAMPLE ? kSBins : 1); i += 128) hist[i] = 0u;
+    const uint32_t bar0 = smem_u32(bars);
+    const uint32_t drain = bar0 + 8u * (2 * kTcStages + 4);
+#define FULL(s) (bar0 + 8u * (uint32_t)(s))
+#define EMPTY(s) (bar0 + 8u * (uint32_t)(kTcStages + (s)))
+#define TFULL(b) (bar0 + 8u * (uint32_t)(2 * kTcStages + (b)))
+#define TEMPTY(b) (bar0 + 8u * (uint32_t)(2 * kTcStages + 2 + (b)))
 
-    // A fragments (rows of this warp) and per-row limits
-    const int g = lane >> 2, tq = lane & 3;
-    uint32_t af[4][4];
-    int64_t lim[2], ncol[2], row[2];
-    float tau[2], rad[2];
-    int qloc[2];
-    bool rowok[2];
-#pragma unroll
-    for (int hh = 0; hh < 2; ++hh) {
-        const int r = w * 16 + g + 8 * hh;
-        qloc[hh] = r / G;
-        const int64_t q = q0 + qloc[hh];
-        rowok[hh] = q < a.nqc;
-        const int64_t t = a.t_first + (rowok[hh] ? q : 0);
-        lim[hh] = t - a.W;
-        ncol[hh] = flat_ncol_d(t, a.W, a.NB);
-        row[hh] = (rowok[hh] ? q : 0) * a.hkv + h;
-        tau[hh] = SAMPLE ? 0.f : a.tau[row[hh]];
-        const int64_t yrow = a.agg ? ((rowok[hh] ? q : 0) * (int64_t)a.hkv * G + (int64_t)h * G + r % G) : row[hh];
-        const uint16_t* yp = a.Y + yrow * kDL;
-        float n2 = 0.f;
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
-            const int c0 = kk * 16 + 2 * tq;
-            af[kk][hh] = rowok[hh] ? *reinterpret_cast<const uint32_t*>(yp + c0) : 0u;
-            af[kk][hh + 2] = rowok[hh] ? *reinterpret_cast<const uint32_t*>(yp + c0 + 8) : 0u;
-            const uint32_t u[2] = {af[kk][hh], af[kk][hh + 2]};
-#pragma unroll
-            for (int x = 0; x < 2; ++x) {
-                const float lo = __uint_as_float(u[x] << 16), hi = __uint_as_float(u[x] & 0xFFFF0000u);
-                n2 += lo * lo + hi * hi;
-            }
-        }
-        // |y| of the row (native: max over the group's heads) bounds |score|
-        n2 += __shfl_xor_sync(0xffffffffu, n2, 1);
-        n2 += __shfl_xor_sync(0xffffffffu, n2, 2);
-        for (int off = 4; off < 4 * G; off <<= 1) n2 = fmaxf(n2, __shfl_xor_sync(0xffffffffu, n2, off));
-        rad[hh] = fminf(1.0625f, sqrtf(n2) * 1.01f + 1e-6f);
-        if (SAMPLE && rowok[hh] && (g % G) == 0 && tq == 0) rads[qloc[hh]] = rad[hh];
+    if (tid == 0) {
+        for (int s = 0; s < kTcStages; ++s) { mbar_init(FULL(s), 1); mbar_init(EMPTY(s), 1); }
+        for (int b = 0; b < 2; ++b) { mbar_init(TFULL(b), 1); mbar_init(TEMPTY(b), 4 * 32); }
+        mbar_init(drain, 1);
+        *abort_flag = 0;
+        fence_barrier_init();
     }
-
-    const uint16_t* cb = a.cent + (int64_t)h * a.cap_buckets * kDL;
-    auto load_tile = [&](int tile, int buf) {
-        const int64_t v0 = (int64_t)tile * kPassCols;
-        uint16_t* dst = ctile + buf * kPassCols * kDL;
+    if (warp == 1) tmem_alloc(smem_u32(tmem_slot), kTcTmemCols);
+    if (warp >= 2) {
+        // A: the CTA's 128 latent rows, 128-byte swizzled; rows past the
+        // chunk are zero
+        const int r = tid - 64;
+        const int64_t q = q0 + r / G;
+        uint4* dst = reinterpret_cast<uint4*>(sA + r * 128);
+        if (q < a.nqc) {
+            const int64_t yrow = a.agg ? (q * a.hkv + h) * G + r % G : q * a.hkv + h;
+            const uint4* src = reinterpret_cast<const uint4*>(a.Y + yrow * kDL);
 #pragma unroll
-        for (int i = 0; i < (kPassCols * 8) / 128; ++i) {
-            const int idx = tid + 128 * i;
-            const int n = idx >> 3, c = idx & 7;
-            const bool ok = v0 + n < nv;
-            const int64_t b = (v0 + n) * stride;
-            cp_async_16(smem_u32(dst + n * kDL + ((c ^ (n & 7)) << 3)),
-                        ok ? (const void*)(cb + b * kDL + c * 8) : (const void*)cb, ok ? 16 : 0);
-        }
-        if (SAMPLE) {
-            const bool ok = v0 + tid < nv;
-            const int64_t b = (v0 + tid) * stride;
-            const int64_t hb = (int64_t)h * a.cap_buckets + (ok ? b : 0);
-            cp_async_4(smem_u32(mminlr + buf * kPassCols + tid), a.minlr + hb, ok ? 4 : 0);
-            cp_async_4(smem_u32(mcnt + buf * kPassCols + tid), a.cnt_lr + hb, ok ? 4 : 0);
-        }
-        cp_async_commit();
-    };
-
-    if (ntile > 0) load_tile(0, 0);
-    __syncthreads();  // histogram / counters cleared
-    for (int tile = 0; tile < ntile; ++tile) {
-        const int buf = tile & 1;
-        if (tile + 1 < ntile) load_tile(tile + 1, buf ^ 1);
-        else cp_async_commit();
-        cp_async_wait<1>();
-        __syncthreads();
-        float acc[16][4];
-#pragma unroll
-        for (int j = 0; j < 16; ++j)
-#pragma unroll
-            for (int i = 0; i < 4; ++i) acc[j][i] = 0.f;
-        const uint32_t base = smem_u32(ctile + buf * kPassCols * kDL);
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
-#pragma unroll
-            for (int jp = 0; jp < 8; ++jp) {
-                const int mi = lane >> 3, ri = lane & 7;
-                const int n = (2 * jp + (mi >> 1)) * 8 + ri;
-                const int c = 2 * kk + (mi & 1);
-                uint32_t b[4];
-                ldsm_x4(b, base + (uint32_t)(n * kDL + ((c ^ (n & 7)) << 3)) * 2u);
-                mma_16816(acc[2 * jp], af[kk], b[0], b[1]);
-                mma_16816(acc[2 * jp + 1], af[kk], b[2], b[3]);
-            }
-        }
-        const int64_t v0 = (int64_t)tile * kPassCols;
-        uint32_t hit[2] = {0u, 0u};  // bit 2j+e: element (n8 tile j, column e) kept
-#pragma unroll
-        for (int j = 0; j < 16; ++j) {
-            float v[4] = {acc[j][0], acc[j][1], acc[j][2], acc[j][3]};
-            for (int off = 4; off < 4 * G; off <<= 1)
-#pragma unroll
-                for (int i = 0; i < 4; ++i) v[i] = fmaxf(v[i], __shfl_xor_sync(0xffffffffu, v[i], off));
-#pragma unroll
-            for (int i = 0; i < 4; ++i) acc[j][i] = v[i];
-            if ((g % G) != 0) continue;
-#pragma unroll
-            for (int hh = 0; hh < 2; ++hh) {
-                if (!rowok[hh]) continue;
-#pragma unroll
-                for (int e = 0; e < 2; ++e) {
-                    const int cl = j * 8 + 2 * tq + e;
-                    const int64_t vc = v0 + cl;
-                    const float sc = v[2 * hh + e];
-                    if (SAMPLE) {
-                        if (vc * kSampleStride < ncol[hh] && (int64_t)mminlr[buf * kPassCols + cl] <= lim[hh]) {
-                            int bin = __float2int_rd((sc + rad[hh]) * ((float)kSBins / (2.f * rad[hh])));
-                            bin = bin < 0 ? 0 : (bin >= kSBins ? kSBins - 1 : bin);
-                            atomicAdd(&hist[qloc[hh] * kSBins + bin], (uint32_t)mcnt[buf * kPassCols + cl]);
-                        }
-                    } else if (sc >= tau[hh] && vc < ncol[hh]) {
-                        hit[hh] |= 1u << (2 * j + e);
-                    }
-                }
-            }
-        }
-        if (!SAMPLE) {
-            // ordered append: the 4 lanes of a quad hold one row's columns
-            // 8j + 2tq + e; a hit's rank in the tile counts the quad's hits
-            // in earlier n8 tiles and in earlier lanes of its own tile
-#pragma unroll
-            for (int hh = 0; hh < 2; ++hh) {
-                const int qb = lane & ~3;
-                const uint32_t m0 = __shfl_sync(0xffffffffu, hit[hh], qb);
-                const uint32_t m1 = __shfl_sync(0xffffffffu, hit[hh], qb | 1);
-                const uint32_t m2 = __shfl_sync(0xffffffffu, hit[hh], qb | 2);
-                const uint32_t m3 = __shfl_sync(0xffffffffu, hit[hh], qb | 3);
-                const int tot = __popc(m0) + __popc(m1) + __popc(m2) + __popc(m3);
-                int base = 0;
-                if (tq == 0 && tot > 0) base = (int)atomicAdd(&hist[qloc[hh]], (uint32_t)tot);
-                base = __shfl_sync(0xffffffffu, base, qb);
-                if (tot == 0) continue;
-                const uint32_t mine = hit[hh];
-#pragma unroll
-                for (int j = 0; j < 16; ++j) {
-#pragma unroll
-                    for (int e = 0; e < 2; ++e) {
-                        if (!((mine >> (2 * j + e)) & 1u)) continue;
-                        const uint32_t below = (1u << (2 * j)) - 1u, here = 3u << (2 * j);
-                        int pos = __popc(m0 & below) + __popc(m1 & below) + __popc(m2 & below) +
-                                  __popc(m3 & below);
-                        if (tq > 0) pos += __popc(m0 & here);
-                        if (tq > 1) pos += __popc(m1 & here);
-                        if (tq > 2) pos += __popc(m2 & here);
-                        if (e) pos += (mine >> (2 * j)) & 1u;
-                        const int slot = base + pos;
-                        if (slot < kCandCap) {
-                            a.cand_col[row[hh] * kCandCap + slot] = (int32_t)(v0 + j * 8 + 2 * tq + e);
-                            a.cand_s[row[hh] * kCandCap + slot] = acc[j][2 * hh + e];
-                        }
-                    }
-                }
-            }
-        }
-        __syncthreads();  // buffer `buf` is refilled two iterations later
-    }
-    cp_async_wait<0>();
-    __syncthreads();
-    if (tid < qpt && q0 + tid < a.nqc) {
-        const int64_t r = (q0 + tid) * a.hkv + h;
-        if (SAMPLE) {
-            // tau: lower edge of the bin where the scaled sample weight from
-            // the top first reaches kOversample * k; -inf if it never does
-            const float R = rads[tid];
-            float t = -CUDART_INF_F;
-            long long cum = 0;
-            for (int b = kSBins - 1; b >= 0; --b) {
-                cum += (long long)hist[tid * kSBins + b] * kSampleStride;
-                if (cum >= (long long)kOversample * a.k) { t = -R + b * (2.f * R / kSBins); break; }
-            }
-            a.tau[r] = t;
+            for (int c = 0; c < 8; ++c) dst[c ^ (r & 7)] = src[c];
         } else {
-            a.cand_n[r] = (int32_t)hist[tid];
+#pragma unroll
+            for (int c = 0; c < 8; ++c) dst[c] = make_uint4(0, 0, 0, 0);
         }
+        fence_proxy_async_smem();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            // producer: sampled tiles first, then every eligible tile
+            int issued = 0;
+            for (int it = 0; it < ntiles; ++it) {
+                const int s = it % kTcStages;
+                if (!mbar_wait(EMPTY(s), ((uint32_t)(it / kTcStages) & 1u) ^ 1u, abort_flag)) break;
+                mbar_expect_tx(FULL(s), kTcBBytes);
+                if (it < ns_tiles)
+                    tma_load_2d(smem_u32(sB + s * kTcBBytes), &tmS, 0,
+                                (int32_t)((int64_t)h * a.ns_cap + (int64_t)it * kTcCols), FULL(s));
+                else
+                    tma_load_2d(smem_u32(sB + s * kTcBBytes), &tmF, 0,
+                                (int32_t)((int64_t)h * a.cap_buckets + (int64_t)(it - ns_tiles) * kTcCols), FULL(s));
+                ++issued;
+            }
+            // after an abort, let this thread's copies land before the CTA exits
+            if (*abort_flag)
+                for (int it = max(0, issued - kTcStages); it < issued; ++it)
+                    mbar_wait(FULL(it % kTcStages), (uint32_t)(it / kTcStages) & 1u, abort_flag, false);
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            const uint32_t a0 = smem_u32(sA);
+            for (int it = 0; it < ntiles; ++it) {
+                const int s = it % kTcStages, b = it & 1;
+                if (!mbar_wait(TEMPTY(b), ((uint32_t)(it >> 1) & 1u) ^ 1u, abort_flag)) break;
+                if (!mbar_wait(FULL(s), (uint32_t)(it / kTcStages) & 1u, abort_flag)) break;
+                tc_fence_after();
+                const uint32_t b0 = smem_u32(sB + s * kTcBBytes);
+#pragma unroll
+                for (int k = 0; k < kDL / 16; ++k)
+                    umma_bf16(tmem + (uint32_t)(b * kTcCols), sw128_desc(a0 + 32u * k), sw128_desc(b0 + 32u * k),
+                              kTcIdesc, k > 0 ? 1u : 0u);
+                umma_commit(EMPTY(s));
+                umma_commit(TFULL(b));
+            }
+            // every MMA this thread issued has completed once `drain` fires
+            umma_commit(drain);
+            mbar_wait(drain, 0, abort_flag, false);
+        }
+    } else {
+        // epilogue: TMEM lane quarter (warp % 4) holds rows 32 * (warp % 4) + lane
+        const int quarter = warp & 3;
+        const int r = quarter * 32 + lane;
+        const int64_t q = q0 + r / G;
+        const bool valid = q < a.nqc;
+        const bool owner = valid && (r % G) == 0;
+        const int64_t qq = valid ? q : 0;
+        const int64_t t = a.t_first + qq;
+        const int64_t lim = t - a.W;
+        const int64_t ncol = flat_ncol_d(t, a.W, a.NB);
+        const int64_t orow = qq * a.hkv + h;
+        const uint32_t trow = tmem + ((uint32_t)(quarter * 32) << 16);
+
+        // R bounds |score| of the row (native: the max over the group's heads)
+        float n2 = 0.f;
+        {
+            const int64_t yrow = a.agg ? (qq * a.hkv + h) * G + r % G : orow;
+            const uint4* yp = reinterpret_cast<const uint4*>(a.Y + yrow * kDL);
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+                const uint4 u = yp[c];
+                const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+                for (int x = 0; x < 4; ++x) {
+                    const float lo = __uint_as_float(w4[x] << 16), hi = __uint_as_float(w4[x] & 0xFFFF0000u);
+                    n2 += lo * lo + hi * hi;
+                }
+            }
+            for (int off = 1; off < G; off <<= 1) n2 = fmaxf(n2, __shfl_xor_sync(0xffffffffu, n2, off));
+        }
+        const float R = fminf(1.0625f, sqrtf(n2) * 1.01f + 1e-6f);
+        const float bscale = (float)kSBins / (2.f * R);
+        for (int b = 0; b < kSBins; ++b) hist[b * kTcRows + r] = 0;
+
+        // packed info of sampled column j, prefetched two 32-column chunks ahead
+        const int32_t* info = a.info_s + (int64_t)h * a.ns_cap;
+        auto load_info = [&](int64_t j) { return j < a.ns_cap ? __ldg(info + j) : (1 << kInfoPosBits) - 1; };
+        int pf0 = load_info(lane), pf1 = load_info(32 + lane);
+
+        int it = 0;
+        // phase 1: weighted histogram of the sampled scores
+        for (; it < ns_tiles; ++it) {
+            const int b = it & 1;
+            // warp-uniform outcome: tcgen05.ld below needs the whole warp
+            if (!__all_sync(0xffffffffu, mbar_wait(TFULL(b), (uint32_t)(it >> 1) & 1u, abort_flag))) break;
+            tc_fence_after();
+#pragma unroll 1
+            for (int c = 0; c < kTcCols / 32; ++c) {
+                const int64_t j0 = (int64_t)it * kTcCols + c * 32;
+                const int inf = pf0;
+                pf0 = pf1;
+                pf1 = load_info(j0 + 64 + lane);
+                float v[32];
+                tmem_ld32(trow + (uint32_t)(b * kTcCols + c * 32), v);
+#pragma unroll
+                for (int i = 0; i < 32; ++i)
+                    for (int off = 1; off < G; off <<= 1) v[i] = fmaxf(v[i], __shfl_xor_sync(0xffffffffu, v[i], off));
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    const int pk = __shfl_sync(0xffffffffu, inf, i);
+                    if (owner && (j0 + i) * kSampleStride < ncol && (int64_t)(pk & ((1 << kInfoPosBits) - 1)) <= lim) {
+                        int bin = __float2int_rd((v[i] + R) * bscale);
+                        bin = bin < 0 ? 0 : (bin >= kSBins ? kSBins - 1 : bin);
+                        uint16_t* hp = hist + bin * kTcRows + r;
+                        const uint32_t nv = (uint32_t)*hp + (uint32_t)(pk >> kInfoPosBits);
+                        *hp = (uint16_t)(nv > 65535u ? 65535u : nv);
+                    }
+                }
+            }
+            tc_fence_before();
+            mbar_arrive(TEMPTY(b));
+        }
+        // tau: lower edge of the bin where the scaled sample weight from the
+        // top first reaches kOversample * k (saturated bins only occur at or
+        // below that bin, since 65535 * 8 > kOversample * 4096); -inf if never
+        float tau = -CUDART_INF_F;
+        {
+            long long cum = 0;
+            for (int bn = kSBins - 1; bn >= 0; --bn) {
+                cum += (long long)hist[bn * kTcRows + r] * kSampleStride;
+                if (cum >= (long long)kOversample * a.k) { tau = -R + bn * (2.f * R / kSBins); break; }
+            }
+        }
+        if (owner) a.tau[orow] = tau;
+
+        // phase 2: candidates >= tau in ascending bucket id (the thread owns
+        // the row, so appends need no atomics)
+        int32_t* ccol = a.cand_col + orow * (int64_t)kCandCap;
+        float* cs = a.cand_s + orow * (int64_t)kCandCap;
+        int cnt = 0;
+        for (; it < ntiles; ++it) {
+            const int b = it & 1;
+            // warp-uniform outcome: tcgen05.ld below needs the whole warp
+            if (!__all_sync(0xffffffffu, mbar_wait(TFULL(b), (uint32_t)(it >> 1) & 1u, abort_flag))) break;
+            tc_fence_after();
+            const int64_t c_base = (int64_t)(it - ns_tiles) * kTcCols;
+#pragma unroll 1
+            for (int c = 0; c < kTcCols / 32; ++c) {
+                float v[32];
+                tmem_ld32(trow + (uint32_t)(b * kTcCols + c * 32), v);
+#pragma unroll
+                for (int i = 0; i < 32; ++i)
+                    for (int off = 1; off < G; off <<= 1) v[i] = fmaxf(v[i], __shfl_xor_sync(0xffffffffu, v[i], off));
+                float m = v[0];
+#pragma unroll
+                for (int i = 1; i < 32; ++i) m = fmaxf(m, v[i]);
+                const int64_t col0 = c_base + c * 32;
+                if (owner && m >= tau && col0 < ncol) {
+                    const int64_t rem = ncol - col0;
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) {
+                        if (v[i] >= tau && i < rem) {
+                            if (cnt < kCandCap) { ccol[cnt] = (int32_t)(col0 + i); cs[cnt] = v[i]; }
+                            ++cnt;
+                        }
+                    }
+                }
+            }
+            tc_fence_before();
+            mbar_arrive(TEMPTY(b));
+        }
+        if (owner) a.cand_n[orow] = cnt;
+    }
+#undef FULL
+#undef EMPTY
+#undef TFULL
+#undef TEMPTY
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kTcTmemCols);
     }
 }
 
@@ -584,20 +655,28 @@ __global__ void __launch_bounds__(32 * kResWarps, 4) flat_resolve_kernel(Resolve
 
 // ------------------------------------------------------------ host side
 
-lsa_status launch_flat(const PassArgs& pa, const ResolveArgs& ra, cudaStream_t st) {
+// Sampled centroids and their packed info, once per call (the cache does not
+// change between chunks).
+lsa_status launch_sample_gather(const uint16_t* cent, const int32_t* minlr, const int32_t* cnt_lr,
+                                int64_t cap_buckets, int64_t NB, int64_t ns_cap, int32_t hkv, uint16_t* cent_s,
+                                int32_t* info_s, cudaStream_t st) {
+    const int64_t n = (int64_t)hkv * ns_cap * 8;
+    sample_gather_kernel<<<(unsigned)ceil_div<int64_t>(n, 256), 256, 0, st>>>(cent, minlr, cnt_lr, cap_buckets, NB,
+                                                                              ns_cap, hkv, cent_s, info_s);
+    return check_launch("sample_gather_kernel");
+}
+
+// tmF: centroids [hkv * cap_buckets, 64]; tmS: sampled centroids
+// [hkv * ns_cap, 64]; both with 256-row boxes.
+lsa_status launch_flat(const PassArgs& pa, const ResolveArgs& ra, const CUtensorMap& tmF, const CUtensorMap& tmS,
+                       cudaStream_t st) {
     const int G = pa.agg ? pa.G : 1;
-    const int qpt = 64 / G;
+    const int qpt = kTcRows / G;
     dim3 grid((unsigned)ceil_div<int64_t>(pa.nqc, qpt), (unsigned)pa.hkv);
-    const size_t base = 2 * kPassCols * kDL * 2 + 4 * kPassCols * 4 + 64 * 4;
-    const size_t smem_s = base + (size_t)qpt * kSBins * 4;
-    const size_t smem_f = base + (size_t)qpt * 4;
-    cudaFuncSetAttribute(flat_pass_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_s);
-    cudaFuncSetAttribute(flat_pass_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_f);
-    flat_pass_kernel<true><<<grid, 128, smem_s, st>>>(pa);
-    lsa_status s = check_launch("flat_pass_kernel<sample>");
+    cudaFuncSetAttribute(flat_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kTcSmemBytes);
+    flat_tc_kernel<<<grid, kTcThreads, kTcSmemBytes, st>>>(tmF, tmS, pa);
+    lsa_status s = check_launch("flat_tc_kernel");
     if (s != LSA_OK) return s;
-    flat_pass_kernel<false><<<grid, 128, smem_f, st>>>(pa);
-    if ((s = check_launch("flat_pass_kernel<full>")) != LSA_OK) return s;
     const size_t smem_r = sizeof(ResWarp) * kResWarps;
     cudaFuncSetAttribute(flat_resolve_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_r);
     const int64_t rows = pa.nqc * pa.hkv;

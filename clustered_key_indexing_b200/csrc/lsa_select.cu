@@ -496,6 +496,7 @@ struct SelectPlan {
     int64_t chunk;     // query positions per chunk
     int32_t hy;        // latent rows per query
     int32_t fb_slots;
+    int64_t ns_cap;    // sampled buckets per kv-head (every 8th)
 };
 
 static SelectPlan plan_select(const lsa_cfg* cfg, int64_t nq, int32_t hq, int32_t hkv, int64_t NB) {
@@ -511,6 +512,7 @@ static SelectPlan plan_select(const lsa_cfg* cfg, int64_t nq, int32_t hq, int32_
     if (c < 1) c = 1;
     p.chunk = c;
     p.fb_slots = 64;
+    p.ns_cap = ceil_div<int64_t>(NB > 0 ? NB : 1, kSampleStride);
     return p;
 }
 
@@ -526,6 +528,8 @@ struct SelectWs {
     int32_t* ovf_count;
     double* fb_score;
     int32_t* fb_w;
+    uint16_t* cent_s;
+    int32_t* info_s;
     size_t bytes;
 };
 
@@ -543,6 +547,8 @@ static SelectWs carve_select(const SelectPlan& p, int32_t hkv, int mode, char* b
         w.ovf_count = (int32_t*)(base + o); o += 256;
         w.fb_score = (double*)(base + o); o += align256((size_t)p.fb_slots * p.ld * 8);
         w.fb_w = (int32_t*)(base + o); o += align256((size_t)p.fb_slots * p.ld * 4);
+        w.cent_s = (uint16_t*)(base + o); o += align256((size_t)hkv * p.ns_cap * kDL * 2);
+        w.info_s = (int32_t*)(base + o); o += align256((size_t)hkv * p.ns_cap * 4);
     }
     w.bytes = o;
     return w;
@@ -589,6 +595,15 @@ lsa_status run_select(const uint16_t* Q, int64_t t0, int64_t nq, int32_t hq, con
     a.ovf_rows = w.ovf_rows; a.ovf_count = w.ovf_count; a.ovf_cap = (int32_t)(p.chunk * hkv);
     a.fb_score = w.fb_score; a.fb_w = w.fb_w;
 
+    CUtensorMap tmF, tmS;
+    if (cfg->mode == 0) {
+        lsa_status s = launch_sample_gather(c->cent, c->minlr, c->cnt_lr, c->cap_buckets, NB, p.ns_cap, hkv,
+                                            w.cent_s, w.info_s, st);
+        if (s != LSA_OK) return s;
+        if ((s = make_rows64_map(&tmF, c->cent, (int64_t)hkv * c->cap_buckets, kTcCols)) != LSA_OK) return s;
+        if ((s = make_rows64_map(&tmS, w.cent_s, (int64_t)hkv * p.ns_cap, kTcCols)) != LSA_OK) return s;
+    }
+
     for (int64_t c0 = 0; c0 < nq; c0 += p.chunk) {
         const int64_t nqc = (nq - c0) < p.chunk ? (nq - c0) : p.chunk;
         uint16_t* Y = Y_out ? Y_out + c0 * p.hy * kDL : w.Y;
@@ -603,7 +618,7 @@ lsa_status run_select(const uint16_t* Q, int64_t t0, int64_t nq, int32_t hq, con
         if (cudaMemsetAsync(w.ovf_count, 0, sizeof(int32_t), st) != cudaSuccess)
             return set_error(LSA_ECUDA, "lsa_select: memset failed");
         PassArgs pa{};
-        pa.Y = Y; pa.cent = c->cent; pa.minlr = c->minlr; pa.cnt_lr = c->cnt_lr;
+        pa.Y = Y; pa.info_s = w.info_s; pa.ns_cap = p.ns_cap;
         pa.cap_buckets = c->cap_buckets; pa.NB = NB; pa.nqc = nqc; pa.t_first = t0 + c0;
         pa.W = cfg->window; pa.hkv = hkv; pa.G = hq / hkv; pa.agg = cfg->agg; pa.k = cfg->k;
         pa.tau = w.tau; pa.cand_col = w.cand_col; pa.cand_s = w.cand_s; pa.cand_n = w.cand_n;
@@ -615,7 +630,7 @@ lsa_status run_select(const uint16_t* Q, int64_t t0, int64_t nq, int32_t hq, con
         ra.W = cfg->window; ra.Y = Y; ra.nqc = nqc; ra.t_first = t0 + c0; ra.tau = w.tau;
         ra.cand_col = w.cand_col; ra.cand_s = w.cand_s; ra.cand_n = w.cand_n; ra.idx = a.idx;
         ra.ovf_rows = w.ovf_rows; ra.ovf_count = w.ovf_count; ra.ovf_cap = a.ovf_cap;
-        if ((s = launch_flat(pa, ra, st)) != LSA_OK) return s;
+        if ((s = launch_flat(pa, ra, tmF, tmS, st)) != LSA_OK) return s;
         select_fallback_kernel<<<(unsigned)p.fb_slots, kSelThreads, 0, st>>>(a);
         if ((s = check_launch("select_fallback_kernel")) != LSA_OK) return s;
     }

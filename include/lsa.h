@@ -202,7 +202,7 @@ size_t lsa_select_workspace_bytes(const lsa_cfg* cfg, int64_t nq, int32_t hq,
  *   [0,S) sinks 0..min(S,t+1)-1 | [S,S+k) long-range keys, chosen buckets in
  *   ascending id, keys ascending | [S+k, S+k+W) window max(S,t-W+1)..t;
  *   every part padded with -1.
- * Y_out (optional, may be NULL) receives the bf16 query latents.
+ * Y_out (optional, may be NULL, 16-byte aligned) receives the bf16 query latents.
  * ws / ws_bytes: scratch of at least lsa_select_workspace_bytes().
  */
 lsa_status lsa_select(const uint16_t* Q, int64_t t0, int64_t nq, int32_t hq,
