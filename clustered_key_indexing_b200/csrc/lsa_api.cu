@@ -39,6 +39,7 @@ int num_sms() {
 }
 
 // kernels (other translation units)
+int64_t select_chunk(const lsa_cfg* cfg, int32_t hq, int32_t hkv);
 lsa_status launch_key_latent(const uint16_t* K, int64_t T, int32_t hkv, const float* W, int64_t unit0,
                              int64_t unit1, int64_t cap_units, double* U, cudaStream_t st);
 lsa_status launch_query_latent(const uint16_t* Q, int64_t nq, int32_t hq, int32_t hkv, const float* W,
@@ -268,14 +269,21 @@ lsa_status lsa_sparse_attn(const uint16_t* Q, const uint16_t* K, const uint16_t*
     return launch_attn(Q, K, V, idx, nq, hq, hkv, n_idx, T, O, (cudaStream_t)stream);
 }
 
-static int64_t prefill_chunk(int64_t T, int64_t chunk) {
+// Query positions per prefill chunk: `chunk` (all of T if <= 0 or larger),
+// rounded down to a multiple of the flat search's own chunk when larger
+// than it, so that every select call but the last fills whole waves.
+static int64_t prefill_chunk(const lsa_cfg* cfg, int64_t T, int32_t hq, int32_t hkv, int64_t chunk) {
     if (chunk <= 0 || chunk > T) chunk = T;
+    if (cfg->mode == 0 && hkv > 0 && hq > 0) {
+        const int64_t sc = lsa::select_chunk(cfg, hq, hkv);
+        if (chunk > sc && chunk < T) chunk = chunk / sc * sc;
+    }
     return chunk;
 }
 
 size_t lsa_prefill_workspace_bytes(const lsa_cfg* cfg, int64_t T, int32_t hq, int32_t hkv, int64_t chunk) {
     if (check_cfg(cfg) != LSA_OK || T <= 0 || hkv <= 0) return 0;
-    chunk = prefill_chunk(T, chunk);
+    chunk = prefill_chunk(cfg, T, hq, hkv, chunk);
     const int64_t NU = ceil_div<int64_t>(T, kPool);
     const int64_t NB = ceil_div<int64_t>(NU, kUnitsPerBlock) * kBucketsPerBlock;
     const size_t idx_bytes = ((size_t)chunk * hkv * (cfg->sinks + cfg->k + cfg->window) * 4 + 255) & ~(size_t)255;
@@ -290,7 +298,7 @@ lsa_status lsa_prefill(const uint16_t* Q, const uint16_t* K, const uint16_t* V, 
     if ((s = check_cfg(cfg)) != LSA_OK) return s;
     if ((s = check_heads(hq, hkv)) != LSA_OK) return s;
     if (!Q || !K || !V || !O || !W_k || !W_q || !ws) return set_error(LSA_EINVAL, "lsa_prefill: NULL pointer");
-    chunk = prefill_chunk(T, chunk);
+    chunk = prefill_chunk(cfg, T, hq, hkv, chunk);
     const size_t need = lsa_prefill_workspace_bytes(cfg, T, hq, hkv, chunk);
     if (ws_bytes < need) return set_error(LSA_ENOSPACE, "lsa_prefill: workspace %zu < %zu bytes", ws_bytes, need);
     if ((s = lsa_build_buckets(K, T, hkv, W_k, cfg, cache, stream)) != LSA_OK) return s;

@@ -38,33 +38,44 @@ namespace lsa {
 
 constexpr int kCandCap = 1024;       // candidates kept per (query, kv-head)
 constexpr int kSampleStride = 8;     // every 8th bucket scored by the sample phase
-constexpr int kSBins = 256;          // sample histogram bins over [-R, R], R = row latent norm bound
 constexpr int kOversample = 2;       // tau targets kOversample * k keys
 constexpr float kScoreErr = 1e-4f;   // bound on |fp32 score - exact score|
 
-// tcgen05 tile of the flat pass: M = 128 latent rows, N = 256 centroids,
-// K = 64 (four MMAs of K = 16), a 4-stage TMA ring of centroid tiles and two
-// TMEM accumulators (512 fp32 columns).
-constexpr int kTcRows = 128;
-constexpr int kTcCols = 256;
-constexpr int kTcStages = 4;
-constexpr int kTcThreads = 192;  // warp 0 TMA, warp 1 MMA + TMEM owner, warps 2-5 epilogue
-constexpr uint32_t kTcABytes = kTcRows * kDL * 2;  // 16 KB
-constexpr uint32_t kTcBBytes = kTcCols * kDL * 2;  // 32 KB
-constexpr uint32_t kTcTmemCols = 2 * kTcCols;
-constexpr uint32_t kTcHistBytes = kSBins * kTcRows * 2;  // uint16 bins [bin][row]
-constexpr size_t kTcSmemBytes = 1024 + kTcABytes + kTcStages * kTcBBytes + kTcHistBytes + 256;
-constexpr uint32_t kTcIdesc = umma_idesc_bf16(kTcRows, kTcCols);
-constexpr int kInfoPosBits = 27;     // packed sample info: count << 27 | min(first eligible position, 2^27 - 1)
+// tcgen05 tile of the flat pass.  A CTA scores 256 latent rows (two M = 128
+// blocks, each its own MMA) against 128 centroids per tile: K = 64 (four MMAs
+// of K = 16) plus, in the candidate phase, one more K = 16 step that adds -tau
+// to every row (A holds -tau in its first extra column, B a 1 there), so TMEM
+// holds s - tau and a hit is a clear sign bit.  A 3-stage TMA ring of centroid
+// tiles; TMEM = 2 buffers x 2 blocks x 128 fp32 columns; eight epilogue warps,
+// each owning 32 rows of one block (TMEM lane quarter = warp % 4), a thread
+// per row.
+constexpr int kTcBlocks = 2;
+constexpr int kTcRows = 128 * kTcBlocks;
+constexpr int kTcCols = 128;
+constexpr int kTcStages = 3;
+constexpr int kTcEpi = 32 * 4 * kTcBlocks;         // epilogue threads, one per row
+constexpr int kTcThreads = 64 + kTcEpi;            // warp 0 TMA, warp 1 MMA + TMEM owner, warps 2-9 epilogue
+constexpr int kHBins = 128;                        // sample histogram bins per row
+constexpr uint32_t kTcABytes = 128 * kDL * 2;      // 16 KB per block, 128-byte swizzle
+constexpr uint32_t kTcAxBytes = 128 * 16 * 2;      // 4 KB per block, extra K = 16 of A, no swizzle
+constexpr uint32_t kTcBxBytes = kTcCols * 16 * 2;  // 4 KB, extra K = 16 of B, no swizzle
+constexpr uint32_t kTcBBytes = kTcCols * kDL * 2;  // 16 KB per stage
+constexpr uint32_t kTcTmemCols = 2 * kTcBlocks * kTcCols;
+constexpr uint32_t kTcHistBytes = kHBins * kTcRows * 4;       // [bin][row] counts (sample phase)
+constexpr int kTcStgStride = 36;                              // floats per row in the staging rows
+constexpr uint32_t kTcStgBytes = kTcRows * kTcStgStride * 4;  // candidate phase; shares the histogram's space
+constexpr uint32_t kTcScratchBytes = kTcHistBytes > kTcStgBytes ? kTcHistBytes : kTcStgBytes;
+constexpr size_t kTcSmemBytes = 1024 + kTcBlocks * (kTcABytes + kTcAxBytes) + kTcBxBytes + kTcStages * kTcBBytes +
+                                kTcScratchBytes + 256;
+constexpr uint32_t kTcIdesc = umma_idesc_bf16(128, kTcCols);
+static_assert(kTcSmemBytes <= 232448, "flat_tc_kernel shared memory");
 
 struct PassArgs {
     const uint16_t* Y;       // chunk latents [nqc, hkv, 64] (mean) / [nqc, hq, 64] (native)
-    const int32_t* info_s;   // [hkv, ns_cap] packed sample info of buckets 0, 8, 16, ...
     int64_t cap_buckets, ns_cap, NB, nqc, t_first;
-    int32_t W, hkv, G, agg, k;
+    int32_t W, hkv, G, agg, k, S;
     float* tau;              // [nqc * hkv]
-    int32_t* cand_col;       // [nqc * hkv, kCandCap]
-    float* cand_s;           // [nqc * hkv, kCandCap]
+    int2* cand;              // [nqc * hkv, kCandCap] (bucket id, fp32 score bits)
     int32_t* cand_n;         // [nqc * hkv]
 };
 
@@ -75,58 +86,76 @@ __host__ __device__ __forceinline__ int64_t flat_ncol_d(int64_t t, int32_t W, in
     return n < NB ? n : NB;
 }
 
-// cent_s[h, j] = cent[h, 8j] and info_s[h, j] = packed (minlr, cnt_lr) of
-// bucket 8j, for 8j < NB (zero centroid and no weight past it).
-__global__ void sample_gather_kernel(const uint16_t* __restrict__ cent, const int32_t* __restrict__ minlr,
-                                     const int32_t* __restrict__ cnt_lr, int64_t cap_buckets, int64_t NB,
-                                     int64_t ns_cap, int32_t hkv, uint16_t* __restrict__ cent_s,
-                                     int32_t* __restrict__ info_s) {
+// cent_s[h, j] = cent[h, 8j] for 8j < NB (zero past it).
+__global__ void sample_gather_kernel(const uint16_t* __restrict__ cent, int64_t cap_buckets, int64_t NB,
+                                     int64_t ns_cap, int32_t hkv, uint16_t* __restrict__ cent_s) {
     const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     if (idx >= (int64_t)hkv * ns_cap * 8) return;
     const int64_t row = idx >> 3;
     const int c = (int)(idx & 7);
     const int64_t h = row / ns_cap, b = (row % ns_cap) * kSampleStride;
-    const bool ok = b < NB;
-    const int64_t src = h * cap_buckets + b;
     reinterpret_cast<uint4*>(cent_s + row * kDL)[c] =
-        ok ? reinterpret_cast<const uint4*>(cent + src * kDL)[c] : make_uint4(0, 0, 0, 0);
-    if (c == 0) {
-        int32_t v = (1 << kInfoPosBits) - 1;
-        if (ok) {
-            const int32_t m = minlr[src], w = cnt_lr[src];
-            const int32_t mc = m < 0 ? 0 : (m > (1 << kInfoPosBits) - 1 ? (1 << kInfoPosBits) - 1 : m);
-            v = mc | ((w < 0 ? 0 : (w > 15 ? 15 : w)) << kInfoPosBits);
-        }
-        info_s[row] = v;
-    }
+        b < NB ? reinterpret_cast<const uint4*>(cent + (h * cap_buckets + b) * kDL)[c] : make_uint4(0, 0, 0, 0);
 }
 
+template <int G>
+__device__ __forceinline__ void group_max(uint32_t (&v)[32]) {
+#pragma unroll
+    for (int off = 1; off < G; off <<= 1)
+#pragma unroll
+        for (int i = 0; i < 32; ++i)
+            v[i] = __float_as_uint(fmaxf(__uint_as_float(v[i]), __uint_as_float(__shfl_xor_sync(0xffffffffu, v[i], off))));
+}
+
+// Largest bf16 value <= x (x finite or -inf).
+__device__ __forceinline__ float bf16_floor(float x) {
+    uint32_t u = __float_as_uint(x);
+    const uint32_t low = u & 0xFFFFu;
+    u &= 0xFFFF0000u;
+    if ((u >> 31) && low) u += 0x10000u;  // negative: truncation went up, step one ulp down
+    return __uint_as_float(u);
+}
+
+// Element (row, k) of a K = 16, no-swizzle K-major operand: 8-row x 16-byte
+// core matrices; 128 bytes between the two K halves, 256 between row groups.
+__device__ __forceinline__ uint32_t noswz_off(int row, int khalf) {
+    return (uint32_t)((row >> 3) * 256 + khalf * 128 + (row & 7) * 16);
+}
+
+// G: latent rows per query (1 for the group-mean score, hq / hkv for the
+// native per-head max).
+template <int G>
 __global__ void __launch_bounds__(kTcThreads, 1)
 flat_tc_kernel(const __grid_constant__ CUtensorMap tmF, const __grid_constant__ CUtensorMap tmS, PassArgs a) {
     extern __shared__ uint8_t tsm_raw[];
     // 1024-byte alignment for the 128-byte swizzle atoms
     uint8_t* tsm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(tsm_raw) + 1023) & ~(uintptr_t)1023);
-    uint8_t* sA = tsm;
-    uint8_t* sB = tsm + kTcABytes;
-    uint16_t* hist = reinterpret_cast<uint16_t*>(sB + kTcStages * kTcBBytes);
-    uint64_t* bars = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(hist) + kTcHistBytes);
-    // bars: full[S], empty[S], tfull[2], tempty[2], drain
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * kTcStages + 5);
+    uint8_t* sA = tsm;                                   // [block] 16 KB
+    uint8_t* sB = sA + kTcBlocks * kTcABytes;            // [stage] 16 KB
+    uint8_t* sAx = sB + kTcStages * kTcBBytes;           // [block] 4 KB
+    uint8_t* sBx = sAx + kTcBlocks * kTcAxBytes;         // 4 KB
+    uint8_t* scratch = sBx + kTcBxBytes;                 // histogram, then staging rows
+    uint32_t* hist = reinterpret_cast<uint32_t*>(scratch);
+    float* stg = reinterpret_cast<float*>(scratch);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(scratch + kTcScratchBytes);
+    // bars: full[S], empty[S], tfull[2], tempty[2], tau_ready, drain
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * kTcStages + 6);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int h = blockIdx.y;
-    const int G = a.agg ? a.G : 1;
-    const int qpt = kTcRows / G;
+    constexpr int qpt = kTcRows / G;
     const int64_t q0 = (int64_t)blockIdx.x * qpt;
     if (q0 >= a.nqc) return;
     const int64_t qlast = min(a.nqc - 1, q0 + qpt - 1);
     const int64_t ncol_max = flat_ncol_d(a.t_first + qlast, a.W, a.NB);
+    const int64_t ncol_min = flat_ncol_d(a.t_first + q0, a.W, a.NB);
     const int ns_tiles = (int)ceil_div<int64_t>(ceil_div<int64_t>(ncol_max, kSampleStride), kTcCols);
     const int ntiles = ns_tiles + (int)ceil_div<int64_t>(ncol_max, kTcCols);
 
     const uint32_t bar0 = smem_u32(bars);
-    const uint32_t drain = bar0 + 8u * (2 * kTcStages + 4);
+    const uint32_t tau_ready = bar0 + 8u * (2 * kTcStages + 4);
+    const uint32_t drain = bar0 + 8u * (2 * kTcStages + 5);
 #define FULL(s) (bar0 + 8u * (uint32_t)(s))
 #define EMPTY(s) (bar0 + 8u * (uint32_t)(kTcStages + (s)))
 #define TFULL(b) (bar0 + 8u * (uint32_t)(2 * kTcStages + (b)))
@@ -134,20 +163,27 @@ flat_tc_kernel(const __grid_constant__ CUtensorMap tmF, const __grid_constant__ 
 
     if (tid == 0) {
         for (int s = 0; s < kTcStages; ++s) { mbar_init(FULL(s), 1); mbar_init(EMPTY(s), 1); }
-        for (int b = 0; b < 2; ++b) { mbar_init(TFULL(b), 1); mbar_init(TEMPTY(b), 4 * 32); }
+        for (int b = 0; b < 2; ++b) { mbar_init(TFULL(b), 1); mbar_init(TEMPTY(b), kTcEpi); }
+        mbar_init(tau_ready, kTcEpi);
         mbar_init(drain, 1);
         *abort_flag = 0;
         fence_barrier_init();
     }
     if (warp == 1) tmem_alloc(smem_u32(tmem_slot), kTcTmemCols);
-    if (warp >= 2) {
-        // A: the CTA's 128 latent rows, 128-byte swizzled; rows past the
-        // chunk are zero
+    for (int i = tid; i < kHBins * kTcRows; i += kTcThreads) hist[i] = 0u;
+    // extra K step: B = 1 in its first column (bf16 0x3F80); A filled in once tau is known
+    for (int i = tid; i < kTcCols * 2; i += kTcThreads) {
+        const int n = i >> 1, kh = i & 1;
+        *reinterpret_cast<uint4*>(sBx + noswz_off(n, kh)) = make_uint4(kh == 0 ? 0x3F80u : 0u, 0u, 0u, 0u);
+    }
+    if (tid >= 64) {
+        // A: the CTA's 256 latent rows (block r / 128), 128-byte swizzled;
+        // rows past the chunk are zero
         const int r = tid - 64;
         const int64_t q = q0 + r / G;
-        uint4* dst = reinterpret_cast<uint4*>(sA + r * 128);
+        uint4* dst = reinterpret_cast<uint4*>(sA + (r >> 7) * kTcABytes + (r & 127) * 128);
         if (q < a.nqc) {
-            const int64_t yrow = a.agg ? (q * a.hkv + h) * G + r % G : q * a.hkv + h;
+            const int64_t yrow = G > 1 ? (q * a.hkv + h) * G + r % G : q * a.hkv + h;
             const uint4* src = reinterpret_cast<const uint4*>(a.Y + yrow * kDL);
 #pragma unroll
             for (int c = 0; c < 8; ++c) dst[c ^ (r & 7)] = src[c];
@@ -155,8 +191,8 @@ flat_tc_kernel(const __grid_constant__ CUtensorMap tmF, const __grid_constant__ 
 #pragma unroll
             for (int c = 0; c < 8; ++c) dst[c] = make_uint4(0, 0, 0, 0);
         }
-        fence_proxy_async_smem();
     }
+    fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -185,17 +221,24 @@ flat_tc_kernel(const __grid_constant__ CUtensorMap tmF, const __grid_constant__ 
         }
     } else if (warp == 1) {
         if (lane == 0) {
-            const uint32_t a0 = smem_u32(sA);
+            const uint64_t bxd = noswz_desc(smem_u32(sBx), 128, 256);
             for (int it = 0; it < ntiles; ++it) {
                 const int s = it % kTcStages, b = it & 1;
                 if (!mbar_wait(TEMPTY(b), ((uint32_t)(it >> 1) & 1u) ^ 1u, abort_flag)) break;
                 if (!mbar_wait(FULL(s), (uint32_t)(it / kTcStages) & 1u, abort_flag)) break;
+                if (it == ns_tiles && !mbar_wait(tau_ready, 0, abort_flag)) break;
                 tc_fence_after();
                 const uint32_t b0 = smem_u32(sB + s * kTcBBytes);
 #pragma unroll
-                for (int k = 0; k < kDL / 16; ++k)
-                    umma_bf16(tmem + (uint32_t)(b * kTcCols), sw128_desc(a0 + 32u * k), sw128_desc(b0 + 32u * k),
-                              kTcIdesc, k > 0 ? 1u : 0u);
+                for (int blk = 0; blk < kTcBlocks; ++blk) {
+                    const uint32_t d = tmem + (uint32_t)((b * kTcBlocks + blk) * kTcCols);
+                    const uint32_t a0 = smem_u32(sA + blk * kTcABytes);
+#pragma unroll
+                    for (int k = 0; k < kDL / 16; ++k)
+                        umma_bf16(d, sw128_desc(a0 + 32u * k), sw128_desc(b0 + 32u * k), kTcIdesc, k > 0 ? 1u : 0u);
+                    if (it >= ns_tiles)
+                        umma_bf16(d, noswz_desc(smem_u32(sAx + blk * kTcAxBytes), 128, 256), bxd, kTcIdesc, 1u);
+                }
                 umma_commit(EMPTY(s));
                 umma_commit(TFULL(b));
             }
@@ -204,23 +247,23 @@ flat_tc_kernel(const __grid_constant__ CUtensorMap tmF, const __grid_constant__ 
             mbar_wait(drain, 0, abort_flag, false);
         }
     } else {
-        // epilogue: TMEM lane quarter (warp % 4) holds rows 32 * (warp % 4) + lane
-        const int quarter = warp & 3;
-        const int r = quarter * 32 + lane;
+        // epilogue: warp w owns rows 128 * blk + 32 * (w % 4) + lane of block
+        // blk = (w - 2) / 4 (TMEM lane quarter w % 4)
+        const int quarter = warp & 3, blk = (warp - 2) >> 2;
+        const int r = blk * 128 + quarter * 32 + lane;
         const int64_t q = q0 + r / G;
         const bool valid = q < a.nqc;
         const bool owner = valid && (r % G) == 0;
         const int64_t qq = valid ? q : 0;
         const int64_t t = a.t_first + qq;
-        const int64_t lim = t - a.W;
-        const int64_t ncol = flat_ncol_d(t, a.W, a.NB);
+        const int ncol = (int)flat_ncol_d(t, a.W, a.NB);
         const int64_t orow = qq * a.hkv + h;
-        const uint32_t trow = tmem + ((uint32_t)(quarter * 32) << 16);
+        const uint32_t trow = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(blk * kTcCols);
 
-        // R bounds |score| of the row (native: the max over the group's heads)
+        // R bounds |score| of the row: |s| <= |y| |c| < 1.01 |y| (|c| <= 1 + 2^-8)
         float n2 = 0.f;
         {
-            const int64_t yrow = a.agg ? (qq * a.hkv + h) * G + r % G : orow;
+            const int64_t yrow = G > 1 ? (qq * a.hkv + h) * G + r % G : orow;
             const uint4* yp = reinterpret_cast<const uint4*>(a.Y + yrow * kDL);
 #pragma unroll
             for (int c = 0; c < 8; ++c) {
@@ -232,95 +275,132 @@ flat_tc_kernel(const __grid_constant__ CUtensorMap tmF, const __grid_constant__ 
                     n2 += lo * lo + hi * hi;
                 }
             }
+#pragma unroll
             for (int off = 1; off < G; off <<= 1) n2 = fmaxf(n2, __shfl_xor_sync(0xffffffffu, n2, off));
         }
-        const float R = fminf(1.0625f, sqrtf(n2) * 1.01f + 1e-6f);
-        const float bscale = (float)kSBins / (2.f * R);
-        for (int b = 0; b < kSBins; ++b) hist[b * kTcRows + r] = 0;
+        const float R = sqrtf(n2) * 1.01f + 1e-6f;
+        // Eligible long-range keys of the row: positions S .. t - W.  Rows
+        // with at most kOversample * k of them and no more than kCandCap
+        // buckets in range take every bucket (tau = -inf).  Histogram range
+        // [lo, R): rows with at least four times that target bin [0, R) only
+        // (their tau lies in the upper tail), others the whole [-R, R).  Bin of s:
+        // round(s * bsc + boff - 0.5), computed by adding 1.5 * 2^23 (the
+        // float's last place is then 1) and clamped to [0, kHBins).
+        const long long n_elig = max(0LL, (long long)(t - a.W) - a.S + 1);
+        const bool take_all = n_elig <= (long long)kOversample * a.k && ncol <= kCandCap;
+        const bool upper = n_elig >= 4LL * kOversample * a.k;
+        const float lo = upper ? 0.f : -R;
+        const float bsc = (float)kHBins / (R - lo);
+        const float boff = -lo * bsc - 0.5f + 12582912.0f;
 
-        // packed info of sampled column j, prefetched two 32-column chunks ahead
-        const int32_t* info = a.info_s + (int64_t)h * a.ns_cap;
-        auto load_info = [&](int64_t j) { return j < a.ns_cap ? __ldg(info + j) : (1 << kInfoPosBits) - 1; };
-        int pf0 = load_info(lane), pf1 = load_info(32 + lane);
-
+        uint32_t va[32], vb[32];
         int it = 0;
-        // phase 1: weighted histogram of the sampled scores
+        // phase 1: histogram of the sampled scores, one count per sampled
+        // bucket (buckets hold 8 keys on average, a block's 512 keys in 64)
         for (; it < ns_tiles; ++it) {
             const int b = it & 1;
-            // warp-uniform outcome: tcgen05.ld below needs the whole warp
             if (!__all_sync(0xffffffffu, mbar_wait(TFULL(b), (uint32_t)(it >> 1) & 1u, abort_flag))) break;
             tc_fence_after();
-#pragma unroll 1
-            for (int c = 0; c < kTcCols / 32; ++c) {
-                const int64_t j0 = (int64_t)it * kTcCols + c * 32;
-                const int inf = pf0;
-                pf0 = pf1;
-                pf1 = load_info(j0 + 64 + lane);
-                float v[32];
-                tmem_ld32(trow + (uint32_t)(b * kTcCols + c * 32), v);
-#pragma unroll
-                for (int i = 0; i < 32; ++i)
-                    for (int off = 1; off < G; off <<= 1) v[i] = fmaxf(v[i], __shfl_xor_sync(0xffffffffu, v[i], off));
+            const uint32_t tb = trow + (uint32_t)(b * kTcBlocks * kTcCols);
+            auto sample_chunk = [&](uint32_t (&v)[32], uint32_t (&vn)[32], int c) {
+                if (c + 1 < kTcCols / 32) tmem_ld32_async(tb + (uint32_t)((c + 1) * 32), vn);
+                group_max<G>(v);
+                const int j0 = it * kTcCols + c * 32;  // sampled column; its bucket is 8 j
+                // columns a row may score: 8 j < ncol
+                const int nval = !owner ? 0 : min(32, max(0, (ncol + kSampleStride - 1) / kSampleStride - j0));
 #pragma unroll
                 for (int i = 0; i < 32; ++i) {
-                    const int pk = __shfl_sync(0xffffffffu, inf, i);
-                    if (owner && (j0 + i) * kSampleStride < ncol && (int64_t)(pk & ((1 << kInfoPosBits) - 1)) <= lim) {
-                        int bin = __float2int_rd((v[i] + R) * bscale);
-                        bin = bin < 0 ? 0 : (bin >= kSBins ? kSBins - 1 : bin);
-                        uint16_t* hp = hist + bin * kTcRows + r;
-                        const uint32_t nv = (uint32_t)*hp + (uint32_t)(pk >> kInfoPosBits);
-                        *hp = (uint16_t)(nv > 65535u ? 65535u : nv);
-                    }
+                    const int bin = min(kHBins - 1, max(0, __float_as_int(fmaf(__uint_as_float(v[i]), bsc, boff)) - 0x4B400000));
+                    if (i < nval) atomicAdd(&hist[bin * kTcRows + r], 1u);
                 }
+                if (c + 1 < kTcCols / 32) tmem_wait_ld(vn);
+            };
+            tmem_ld32_async(tb, va);
+            tmem_wait_ld(va);
+#pragma unroll 1
+            for (int c = 0; c < kTcCols / 32; c += 2) {
+                sample_chunk(va, vb, c);
+                sample_chunk(vb, va, c + 1);
             }
             tc_fence_before();
             mbar_arrive(TEMPTY(b));
         }
-        // tau: lower edge of the bin where the scaled sample weight from the
-        // top first reaches kOversample * k (saturated bins only occur at or
-        // below that bin, since 65535 * 8 > kOversample * 4096); -inf if never
+        // tau: lower edge of the bin where the sampled key estimate (8 keys
+        // per bucket, every 8th bucket) from the top first reaches
+        // kOversample * k, rounded down to bf16 (it enters the extra K step);
+        // -inf if never (the upper-only range then still reports the whole
+        // count at bin 0, so an upper row whose target lies below 0 gets 0)
         float tau = -CUDART_INF_F;
-        {
+        if (!take_all) {
             long long cum = 0;
-            for (int bn = kSBins - 1; bn >= 0; --bn) {
-                cum += (long long)hist[bn * kTcRows + r] * kSampleStride;
-                if (cum >= (long long)kOversample * a.k) { tau = -R + bn * (2.f * R / kSBins); break; }
+            const long long need = ((long long)kOversample * a.k + 63) / 64;  // sampled buckets
+            for (int bn = kHBins - 1; bn >= 0; --bn) {
+                cum += hist[bn * kTcRows + r];
+                if (cum >= need) { tau = lo + bn * ((R - lo) / kHBins); break; }
             }
         }
+        tau = bf16_floor(tau);
+        if (G > 1) tau = __shfl_sync(0xffffffffu, tau, lane & ~(G - 1));  // the query's owner lane
+        const bool tau_inf = tau == -CUDART_INF_F;
+        const float tau_add = tau_inf ? 0.f : tau;
         if (owner) a.tau[orow] = tau;
+        {
+            uint8_t* ax = sAx + blk * kTcAxBytes;
+            const int rb = quarter * 32 + lane;
+            const uint32_t nb = (uint32_t)(__float_as_uint(-tau_add) >> 16);  // exact: tau_add is a bf16 value
+            *reinterpret_cast<uint4*>(ax + noswz_off(rb, 0)) = make_uint4(nb, 0u, 0u, 0u);
+            *reinterpret_cast<uint4*>(ax + noswz_off(rb, 1)) = make_uint4(0u, 0u, 0u, 0u);
+            fence_proxy_async_smem();
+            mbar_arrive(tau_ready);
+        }
+        // the histogram's space becomes the staging rows: every epilogue
+        // thread has read its bins past this barrier
+        asm volatile("bar.sync 1, %0;\n" ::"n"(kTcEpi) : "memory");
+        float* my_stg = stg + r * kTcStgStride;
 
-        // phase 2: candidates >= tau in ascending bucket id (the thread owns
-        // the row, so appends need no atomics)
-        int32_t* ccol = a.cand_col + orow * (int64_t)kCandCap;
-        float* cs = a.cand_s + orow * (int64_t)kCandCap;
+        // phase 2: TMEM holds s - tau_add; candidates (score >= tau) are
+        // appended in ascending bucket id (the thread owns its row)
+        int2* cand = a.cand + orow * (int64_t)kCandCap;
         int cnt = 0;
         for (; it < ntiles; ++it) {
             const int b = it & 1;
-            // warp-uniform outcome: tcgen05.ld below needs the whole warp
             if (!__all_sync(0xffffffffu, mbar_wait(TFULL(b), (uint32_t)(it >> 1) & 1u, abort_flag))) break;
             tc_fence_after();
-            const int64_t c_base = (int64_t)(it - ns_tiles) * kTcCols;
-#pragma unroll 1
-            for (int c = 0; c < kTcCols / 32; ++c) {
-                float v[32];
-                tmem_ld32(trow + (uint32_t)(b * kTcCols + c * 32), v);
+            const uint32_t tb = trow + (uint32_t)(b * kTcBlocks * kTcCols);
+            const int tbase = (it - ns_tiles) * kTcCols;
+            auto cand_chunk = [&](uint32_t (&v)[32], uint32_t (&vn)[32], int c) {
+                if (c + 1 < kTcCols / 32) tmem_ld32_async(tb + (uint32_t)((c + 1) * 32), vn);
+                group_max<G>(v);
+                const int col0 = tbase + c * 32;
+                const int rem = ncol - col0;
+                const uint32_t lm = !owner || rem <= 0 ? 0u : (rem >= 32 ? 0xffffffffu : ((1u << rem) - 1u));
+                // sign bits of s - tau: bit i set = miss
+                uint32_t shi = 0u, slo = 0u;
 #pragma unroll
-                for (int i = 0; i < 32; ++i)
-                    for (int off = 1; off < G; off <<= 1) v[i] = fmaxf(v[i], __shfl_xor_sync(0xffffffffu, v[i], off));
-                float m = v[0];
+                for (int i = 15; i >= 0; --i) {
+                    shi = __funnelshift_l(v[16 + i], shi, 1);
+                    slo = __funnelshift_l(v[i], slo, 1);
+                }
+                uint32_t hits = (tau_inf ? 0xffffffffu : ~((shi << 16) | slo)) & lm;
+                if (__any_sync(0xffffffffu, hits)) {
 #pragma unroll
-                for (int i = 1; i < 32; ++i) m = fmaxf(m, v[i]);
-                const int64_t col0 = c_base + c * 32;
-                if (owner && m >= tau && col0 < ncol) {
-                    const int64_t rem = ncol - col0;
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) {
-                        if (v[i] >= tau && i < rem) {
-                            if (cnt < kCandCap) { ccol[cnt] = (int32_t)(col0 + i); cs[cnt] = v[i]; }
-                            ++cnt;
-                        }
+                    for (int j = 0; j < 8; ++j)
+                        reinterpret_cast<uint4*>(my_stg)[j] = make_uint4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+                    while (hits) {
+                        const int i = __ffs(hits) - 1;
+                        hits &= hits - 1u;
+                        if (cnt < kCandCap) cand[cnt] = make_int2(col0 + i, __float_as_int(my_stg[i] + tau_add));
+                        ++cnt;
                     }
                 }
+                if (c + 1 < kTcCols / 32) tmem_wait_ld(vn);
+            };
+            tmem_ld32_async(tb, va);
+            tmem_wait_ld(va);
+#pragma unroll 1
+            for (int c = 0; c < kTcCols / 32; c += 2) {
+                cand_chunk(va, vb, c);
+                cand_chunk(vb, va, c + 1);
             }
             tc_fence_before();
             mbar_arrive(TEMPTY(b));
@@ -356,8 +436,7 @@ struct ResolveArgs {
     const uint16_t* Y;
     int64_t nqc, t_first;
     const float* tau;
-    const int32_t* cand_col;
-    const float* cand_s;
+    const int2* cand;
     const int32_t* cand_n;
     int32_t* idx;
     int32_t* ovf_rows;
@@ -491,8 +570,9 @@ __global__ void __launch_bounds__(32 * kResWarps, 4) flat_resolve_kernel(Resolve
         float sc = 0.f;
         int32_t pk = 0;
         if (i < n) {
-            col = a.cand_col[row * kCandCap + i];
-            sc = a.cand_s[row * kCandCap + i];
+            const int2 cv = a.cand[row * kCandCap + i];
+            col = cv.x;
+            sc = __int_as_float(cv.y);
             const int64_t hb = hb0 + col;
             const int32_t mlr = a.minlr[hb], mxp = a.maxpos[hb], clr = a.cnt_lr[hb];
             pk = a.units[hb];
@@ -562,8 +642,9 @@ __global__ void __launch_bounds__(32 * kResWarps, 4) flat_resolve_kernel(Resolve
         }
         const float c32 = __uint_as_float((prefix >> 31) ? (prefix & 0x7FFFFFFFu) : ~prefix);
         const float hi = c32 + 2.f * kScoreErr, lo = c32 - 2.f * kScoreErr;
-        // every bucket that can rank above the exact cut must be a candidate
-        if (tau > -CUDART_INF_F && !(lo >= tau)) {
+        // every bucket that can rank above the exact cut must be a candidate:
+        // non-candidates score <= tau (s - tau < 0 rounds to at most tau)
+        if (tau > -CUDART_INF_F && !(lo > tau)) {
             if (lane == 0) push_fallback(a, row);
             return;
         }
@@ -655,26 +736,24 @@ __global__ void __launch_bounds__(32 * kResWarps, 4) flat_resolve_kernel(Resolve
 
 // ------------------------------------------------------------ host side
 
-// Sampled centroids and their packed info, once per call (the cache does not
-// change between chunks).
-lsa_status launch_sample_gather(const uint16_t* cent, const int32_t* minlr, const int32_t* cnt_lr,
-                                int64_t cap_buckets, int64_t NB, int64_t ns_cap, int32_t hkv, uint16_t* cent_s,
-                                int32_t* info_s, cudaStream_t st) {
+// Sampled centroids, once per call (the cache does not change between
+// chunks).
+lsa_status launch_sample_gather(const uint16_t* cent, int64_t cap_buckets, int64_t NB, int64_t ns_cap, int32_t hkv,
+                                uint16_t* cent_s, cudaStream_t st) {
     const int64_t n = (int64_t)hkv * ns_cap * 8;
-    sample_gather_kernel<<<(unsigned)ceil_div<int64_t>(n, 256), 256, 0, st>>>(cent, minlr, cnt_lr, cap_buckets, NB,
-                                                                              ns_cap, hkv, cent_s, info_s);
+    sample_gather_kernel<<<(unsigned)ceil_div<int64_t>(n, 256), 256, 0, st>>>(cent, cap_buckets, NB, ns_cap, hkv,
+                                                                              cent_s);
     return check_launch("sample_gather_kernel");
 }
 
-// tmF: centroids [hkv * cap_buckets, 64]; tmS: sampled centroids
-// [hkv * ns_cap, 64]; both with 256-row boxes.
 lsa_status launch_flat(const PassArgs& pa, const ResolveArgs& ra, const CUtensorMap& tmF, const CUtensorMap& tmS,
                        cudaStream_t st) {
     const int G = pa.agg ? pa.G : 1;
     const int qpt = kTcRows / G;
     dim3 grid((unsigned)ceil_div<int64_t>(pa.nqc, qpt), (unsigned)pa.hkv);
-    cudaFuncSetAttribute(flat_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kTcSmemBytes);
-    flat_tc_kernel<<<grid, kTcThreads, kTcSmemBytes, st>>>(tmF, tmS, pa);
+    auto kern = G == 1 ? flat_tc_kernel<1> : G == 2 ? flat_tc_kernel<2> : G == 4 ? flat_tc_kernel<4> : flat_tc_kernel<8>;
+    cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kTcSmemBytes);
+    kern<<<grid, kTcThreads, kTcSmemBytes, st>>>(tmF, tmS, pa);
     lsa_status s = check_launch("flat_tc_kernel");
     if (s != LSA_OK) return s;
     const size_t smem_r = sizeof(ResWarp) * kResWarps;

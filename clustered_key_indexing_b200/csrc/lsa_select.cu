@@ -474,16 +474,22 @@ __global__ void __launch_bounds__(kSelThreads) select_fallback_kernel(SelectArgs
         const int ng = a.agg ? a.G : 1;
         const int64_t hb0 = (int64_t)r.h * a.cap_buckets;
         const int64_t ncol = flat_ncol(r.t, a.W, a.NB);
+        int myw = 0;
         for (int64_t b = tid; b < ncol; b += kSelThreads) {
             const bool el = (int64_t)a.minlr[hb0 + b] <= r.lim;
             fw[b] = el ? bucket_weight(a, r.h, b, r.lim) : 0;
             fs[b] = el ? exact_row(sh.ylat, ng, a.cent + (hb0 + b) * kDL) : 0.0;
+            myw += fw[b];
         }
+        int totw;
+        block_exscan(myw, &totw, sh.sh4);
         __syncthreads();
-        // taken counts are written back into fw
-        radix_fill(
-            ncol, a.k, [&](int64_t i) { return fs[i]; }, [&](int64_t i) { return (int)fw[i]; },
-            [&](int64_t i, int tk) { fw[i] = tk; }, sh);
+        // taken counts are written back into fw (every eligible key when
+        // there are no more than k of them)
+        if (totw > a.k)
+            radix_fill(
+                ncol, a.k, [&](int64_t i) { return fs[i]; }, [&](int64_t i) { return (int)fw[i]; },
+                [&](int64_t i, int tk) { fw[i] = tk; }, sh);
         __syncthreads();
         emit_range(a, r, ncol, [&](int64_t b) -> int { return fw[b]; }, sh);
     }
@@ -499,15 +505,26 @@ struct SelectPlan {
     int64_t ns_cap;    // sampled buckets per kv-head (every 8th)
 };
 
+// Query positions per flat-search chunk: the flat pass launches one CTA per
+// (256 / G latent rows, kv-head), so a chunk of a multiple of
+// num_sms / gcd(num_sms, hkv) CTA row blocks fills whole waves; candidate
+// lists (kCandCap x 8 bytes per query and kv-head) stay within 1 GiB.
+int64_t select_chunk(const lsa_cfg* cfg, int32_t hq, int32_t hkv) {
+    const int64_t qpt = kTcRows / (cfg->agg ? hq / hkv : 1);
+    int64_t g = num_sms(), x = hkv;
+    while (x) { const int64_t y = g % x; g = x; x = y; }
+    const int64_t unit = num_sms() / g;
+    const int64_t per_block = qpt * hkv * (int64_t)kCandCap * 8;
+    int64_t m = ((int64_t)1 << 30) / per_block / unit;
+    if (m < 1) m = 1;
+    return qpt * unit * m;
+}
+
 static SelectPlan plan_select(const lsa_cfg* cfg, int64_t nq, int32_t hq, int32_t hkv, int64_t NB) {
     SelectPlan p;
     p.ld = ceil_div<int64_t>(NB > 0 ? NB : 1, 128) * 128;
     p.hy = cfg->agg ? hq : hkv;
-    // candidate lists: kCandCap x 8 bytes per (query, kv-head)
-    const int64_t budget = (int64_t)512 << 20;
-    int64_t c = budget / (hkv * (int64_t)kCandCap * 8);
-    c = c / 64 * 64;
-    if (c < 64) c = 64;
+    int64_t c = select_chunk(cfg, hq, hkv);
     if (c > nq) c = nq;
     if (c < 1) c = 1;
     p.chunk = c;
@@ -521,15 +538,13 @@ static size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 struct SelectWs {
     uint16_t* Y;
     float* tau;
-    int32_t* cand_col;
-    float* cand_s;
+    int2* cand;
     int32_t* cand_n;
     int32_t* ovf_rows;
     int32_t* ovf_count;
     double* fb_score;
     int32_t* fb_w;
     uint16_t* cent_s;
-    int32_t* info_s;
     size_t bytes;
 };
 
@@ -540,15 +555,13 @@ static SelectWs carve_select(const SelectPlan& p, int32_t hkv, int mode, char* b
     w.Y = (uint16_t*)(base + o); o += align256((size_t)p.chunk * p.hy * kDL * 2);
     if (mode == 0) {
         w.tau = (float*)(base + o); o += align256(rows * 4);
-        w.cand_col = (int32_t*)(base + o); o += align256(rows * kCandCap * 4);
-        w.cand_s = (float*)(base + o); o += align256(rows * kCandCap * 4);
+        w.cand = (int2*)(base + o); o += align256(rows * kCandCap * 8);
         w.cand_n = (int32_t*)(base + o); o += align256(rows * 4);
         w.ovf_rows = (int32_t*)(base + o); o += align256(rows * 4);
         w.ovf_count = (int32_t*)(base + o); o += 256;
         w.fb_score = (double*)(base + o); o += align256((size_t)p.fb_slots * p.ld * 8);
         w.fb_w = (int32_t*)(base + o); o += align256((size_t)p.fb_slots * p.ld * 4);
         w.cent_s = (uint16_t*)(base + o); o += align256((size_t)hkv * p.ns_cap * kDL * 2);
-        w.info_s = (int32_t*)(base + o); o += align256((size_t)hkv * p.ns_cap * 4);
     }
     w.bytes = o;
     return w;
@@ -597,8 +610,7 @@ lsa_status run_select(const uint16_t* Q, int64_t t0, int64_t nq, int32_t hq, con
 
     CUtensorMap tmF, tmS;
     if (cfg->mode == 0) {
-        lsa_status s = launch_sample_gather(c->cent, c->minlr, c->cnt_lr, c->cap_buckets, NB, p.ns_cap, hkv,
-                                            w.cent_s, w.info_s, st);
+        lsa_status s = launch_sample_gather(c->cent, c->cap_buckets, NB, p.ns_cap, hkv, w.cent_s, st);
         if (s != LSA_OK) return s;
         if ((s = make_rows64_map(&tmF, c->cent, (int64_t)hkv * c->cap_buckets, kTcCols)) != LSA_OK) return s;
         if ((s = make_rows64_map(&tmS, w.cent_s, (int64_t)hkv * p.ns_cap, kTcCols)) != LSA_OK) return s;
@@ -618,17 +630,17 @@ lsa_status run_select(const uint16_t* Q, int64_t t0, int64_t nq, int32_t hq, con
         if (cudaMemsetAsync(w.ovf_count, 0, sizeof(int32_t), st) != cudaSuccess)
             return set_error(LSA_ECUDA, "lsa_select: memset failed");
         PassArgs pa{};
-        pa.Y = Y; pa.info_s = w.info_s; pa.ns_cap = p.ns_cap;
+        pa.Y = Y; pa.ns_cap = p.ns_cap;
         pa.cap_buckets = c->cap_buckets; pa.NB = NB; pa.nqc = nqc; pa.t_first = t0 + c0;
-        pa.W = cfg->window; pa.hkv = hkv; pa.G = hq / hkv; pa.agg = cfg->agg; pa.k = cfg->k;
-        pa.tau = w.tau; pa.cand_col = w.cand_col; pa.cand_s = w.cand_s; pa.cand_n = w.cand_n;
+        pa.W = cfg->window; pa.S = cfg->sinks; pa.hkv = hkv; pa.G = hq / hkv; pa.agg = cfg->agg; pa.k = cfg->k;
+        pa.tau = w.tau; pa.cand = w.cand; pa.cand_n = w.cand_n;
         ResolveArgs ra{};
         ra.units = c->units; ra.offsets = c->offsets; ra.members = c->members; ra.cnt_lr = c->cnt_lr; ra.minlr = c->minlr;
         ra.maxpos = c->maxpos; ra.cent = c->cent; ra.cap_units = c->cap_units;
         ra.cap_buckets = c->cap_buckets; ra.NB = NB; ra.T_built = c->n_tokens;
         ra.hkv = hkv; ra.G = hq / hkv; ra.agg = cfg->agg; ra.k = cfg->k; ra.S = cfg->sinks;
         ra.W = cfg->window; ra.Y = Y; ra.nqc = nqc; ra.t_first = t0 + c0; ra.tau = w.tau;
-        ra.cand_col = w.cand_col; ra.cand_s = w.cand_s; ra.cand_n = w.cand_n; ra.idx = a.idx;
+        ra.cand = w.cand; ra.cand_n = w.cand_n; ra.idx = a.idx;
         ra.ovf_rows = w.ovf_rows; ra.ovf_count = w.ovf_count; ra.ovf_cap = a.ovf_cap;
         if ((s = launch_flat(pa, ra, tmF, tmS, st)) != LSA_OK) return s;
         select_fallback_kernel<<<(unsigned)p.fb_slots, kSelThreads, 0, st>>>(a);
