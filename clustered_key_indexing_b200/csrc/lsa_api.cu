@@ -269,14 +269,17 @@ lsa_status lsa_sparse_attn(const uint16_t* Q, const uint16_t* K, const uint16_t*
     return launch_attn(Q, K, V, idx, nq, hq, hkv, n_idx, T, O, (cudaStream_t)stream);
 }
 
-// Query positions per prefill chunk: `chunk` (all of T if <= 0 or larger),
-// rounded down to a multiple of the flat search's own chunk when larger
-// than it, so that every select call but the last fills whole waves.
+// Query positions per prefill chunk: `chunk` (all of T if <= 0 or larger);
+// in flat mode the nearest multiple of the flat search's own wave-aligned
+// chunk (at least one, at most T), so every select call but the last fills
+// whole waves.
 static int64_t prefill_chunk(const lsa_cfg* cfg, int64_t T, int32_t hq, int32_t hkv, int64_t chunk) {
     if (chunk <= 0 || chunk > T) chunk = T;
-    if (cfg->mode == 0 && hkv > 0 && hq > 0) {
+    if (cfg->mode == 0 && hkv > 0 && hq > 0 && chunk < T) {
         const int64_t sc = lsa::select_chunk(cfg, hq, hkv);
-        if (chunk > sc && chunk < T) chunk = chunk / sc * sc;
+        int64_t m = (chunk + sc / 2) / sc;
+        if (m < 1) m = 1;
+        chunk = m * sc < T ? m * sc : T;
     }
     return chunk;
 }

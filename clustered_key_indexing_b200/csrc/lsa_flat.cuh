@@ -3,16 +3,15 @@
 // buckets until k long-range keys are filled; ch. 5: native max over heads].
 //
 // Per chunk of query positions:
-//   sample_gather_kernel (once per call)  every 8th centroid of each kv-head
-//       and its (first eligible position, key count), packed contiguously;
-//   flat_tc_kernel  one CTA per 128 latent rows of one kv-head, on the 5th-
-//       generation tensor cores (TMA -> shared memory -> tcgen05.mma ->
-//       TMEM, bf16 in, fp32 accumulate).  Phase 1 scores the rows against the
-//       sampled centroids and builds a per-row weighted histogram (bins
-//       scaled to the row's latent norm, which bounds its scores) whose upper
-//       tail gives a threshold tau expected to keep about twice the k keys
-//       needed; phase 2 scores every eligible centroid and appends scores
-//       >= tau to the row's candidate list in ascending bucket id;
+//   sample_gather_kernel (once per call)  every 8th centroid of each kv-head,
+//       packed contiguously;
+//   flat_sample_kernel  tensor-core scores of the rows against the sampled
+//       centroids; a per-row histogram (bins scaled to the row's latent norm,
+//       which bounds its scores) whose upper tail gives a threshold tau
+//       expected to keep about twice the k keys needed;
+//   flat_cand_kernel  tensor-core scores against every eligible centroid;
+//       scores >= tau are appended to the row's candidate list in ascending
+//       bucket id;
 //   flat_resolve_kernel  one warp per (query, kv-head): eligibility and
 //       exact key counts, weighted radix select on the fp32 scores for the
 //       cut c32, exact fp64 rescoring of the buckets within 2e of c32 only,
@@ -41,34 +40,40 @@ constexpr int kSampleStride = 8;     // every 8th bucket scored by the sample ph
 constexpr int kOversample = 2;       // tau targets kOversample * k keys
 constexpr float kScoreErr = 1e-4f;   // bound on |fp32 score - exact score|
 
-// tcgen05 tile of the flat pass.  A CTA scores 256 latent rows (two M = 128
-// blocks, each its own MMA) against 128 centroids per tile: K = 64 (four MMAs
-// of K = 16) plus, in the candidate phase, one more K = 16 step that adds -tau
-// to every row (A holds -tau in its first extra column, B a 1 there), so TMEM
-// holds s - tau and a hit is a clear sign bit.  A 3-stage TMA ring of centroid
-// tiles; TMEM = 2 buffers x 2 blocks x 128 fp32 columns; eight epilogue warps,
-// each owning 32 rows of one block (TMEM lane quarter = warp % 4), a thread
-// per row.
-constexpr int kTcBlocks = 2;
-constexpr int kTcRows = 128 * kTcBlocks;
-constexpr int kTcCols = 128;
-constexpr int kTcStages = 3;
-constexpr int kTcEpi = 32 * 4 * kTcBlocks;         // epilogue threads, one per row
-constexpr int kTcThreads = 64 + kTcEpi;            // warp 0 TMA, warp 1 MMA + TMEM owner, warps 2-9 epilogue
-constexpr int kHBins = 128;                        // sample histogram bins per row
-constexpr uint32_t kTcABytes = 128 * kDL * 2;      // 16 KB per block, 128-byte swizzle
-constexpr uint32_t kTcAxBytes = 128 * 16 * 2;      // 4 KB per block, extra K = 16 of A, no swizzle
-constexpr uint32_t kTcBxBytes = kTcCols * 16 * 2;  // 4 KB, extra K = 16 of B, no swizzle
-constexpr uint32_t kTcBBytes = kTcCols * kDL * 2;  // 16 KB per stage
-constexpr uint32_t kTcTmemCols = 2 * kTcBlocks * kTcCols;
-constexpr uint32_t kTcHistBytes = kHBins * kTcRows * 4;       // [bin][row] counts (sample phase)
-constexpr int kTcStgStride = 36;                              // floats per row in the staging rows
-constexpr uint32_t kTcStgBytes = kTcRows * kTcStgStride * 4;  // candidate phase; shares the histogram's space
-constexpr uint32_t kTcScratchBytes = kTcHistBytes > kTcStgBytes ? kTcHistBytes : kTcStgBytes;
-constexpr size_t kTcSmemBytes = 1024 + kTcBlocks * (kTcABytes + kTcAxBytes) + kTcBxBytes + kTcStages * kTcBBytes +
-                                kTcScratchBytes + 256;
-constexpr uint32_t kTcIdesc = umma_idesc_bf16(128, kTcCols);
-static_assert(kTcSmemBytes <= 232448, "flat_tc_kernel shared memory");
+// The flat pass runs on the 5th-generation tensor cores in two kernels per
+// chunk, both TMA -> shared memory -> tcgen05.mma (bf16 in, fp32 accumulate
+// in TMEM) -> tcgen05.ld, with one producer thread (warp 0), one MMA thread
+// (warp 1, which also owns the TMEM allocation) and epilogue warps that own
+// one latent row per thread (TMEM lane quarter = warp % 4):
+//   flat_sample_kernel  256 rows (two M = 128 blocks) x 128 sampled centroids
+//       per tile; per-row histogram of the sampled scores -> tau;
+//   flat_cand_kernel    512 rows (four blocks) x 64 centroids per tile, plus
+//       one K = 16 step that adds -tau to every row (A holds -tau in its first
+//       extra column, B a 1 there), so TMEM holds s - tau and a hit is a clear
+//       sign bit; hits are appended in ascending bucket id.
+constexpr uint32_t kTcABytes = 128 * kDL * 2;      // one M = 128 block of latents, 128-byte swizzle
+constexpr uint32_t kTcAxBytes = 128 * 16 * 2;      // extra K = 16 of a block, no swizzle
+constexpr int kHBins = 256;                        // sample histogram bins per row (16-bit counts)
+
+constexpr int kSmBlocks = 2, kSmCols = 128, kSmStages = 3;
+constexpr int kSmRows = 128 * kSmBlocks;
+constexpr int kSmThreads = 64 + kSmRows;
+constexpr uint32_t kSmBBytes = kSmCols * kDL * 2;
+constexpr uint32_t kSmHistBytes = kHBins / 2 * kSmRows * 4;  // [bin / 2][row] words, two counts each
+constexpr size_t kSmSmemBytes = 1024 + kSmBlocks * kTcABytes + kSmStages * kSmBBytes + kSmHistBytes + 256;
+static_assert(kSmSmemBytes <= 232448, "flat_sample_kernel shared memory");
+
+constexpr int kCdBlocks = 4, kCdCols = 64, kCdStages = 4;
+constexpr int kCdRows = 128 * kCdBlocks;
+constexpr int kCdThreads = 64 + kCdRows;
+constexpr uint32_t kCdBBytes = kCdCols * kDL * 2;
+constexpr uint32_t kCdBxBytes = kCdCols * 16 * 2;
+constexpr int kTcStgStride = 36;                               // floats per row in the staging rows
+constexpr uint32_t kCdStgBytes = kCdRows * kTcStgStride * 4;
+constexpr size_t kCdSmemBytes = 1024 + kCdBlocks * (kTcABytes + kTcAxBytes) + kCdStages * kCdBBytes + kCdBxBytes +
+                                kCdStgBytes + 256;
+static_assert(kCdSmemBytes <= 232448, "flat_cand_kernel shared memory");
+static_assert(2 * kSmBlocks * kSmCols <= 512 && 2 * kCdBlocks * kCdCols <= 512, "TMEM columns");
 
 struct PassArgs {
     const uint16_t* Y;       // chunk latents [nqc, hkv, 64] (mean) / [nqc, hq, 64] (native)
@@ -122,76 +127,146 @@ __device__ __forceinline__ uint32_t noswz_off(int row, int khalf) {
     return (uint32_t)((row >> 3) * 256 + khalf * 128 + (row & 7) * 16);
 }
 
+// Latent row r of the CTA (query q0 + r / G) into block r / 128 of A,
+// 128-byte swizzled (16-byte chunk c of row i at c ^ (i & 7)); zero past the chunk.
+template <int G>
+__device__ __forceinline__ void fill_a_row(uint8_t* sA, const PassArgs& a, int64_t q0, int h, int r) {
+    const int64_t q = q0 + r / G;
+    uint4* dst = reinterpret_cast<uint4*>(sA + (r >> 7) * kTcABytes + (r & 127) * 128);
+    if (q < a.nqc) {
+        const int64_t yrow = G > 1 ? (q * a.hkv + h) * G + r % G : q * a.hkv + h;
+        const uint4* src = reinterpret_cast<const uint4*>(a.Y + yrow * kDL);
+#pragma unroll
+        for (int c = 0; c < 8; ++c) dst[c ^ (r & 7)] = src[c];
+    } else {
+#pragma unroll
+        for (int c = 0; c < 8; ++c) dst[c] = make_uint4(0, 0, 0, 0);
+    }
+}
+
+// Barrier layout shared by both kernels: full[S], empty[S], tfull[2],
+// tempty[2], drain.
+template <int STAGES>
+struct TcBars {
+    uint32_t b0;
+    __device__ uint32_t full(int s) const { return b0 + 8u * (uint32_t)s; }
+    __device__ uint32_t empty(int s) const { return b0 + 8u * (uint32_t)(STAGES + s); }
+    __device__ uint32_t tfull(int b) const { return b0 + 8u * (uint32_t)(2 * STAGES + b); }
+    __device__ uint32_t tempty(int b) const { return b0 + 8u * (uint32_t)(2 * STAGES + 2 + b); }
+    __device__ uint32_t drain() const { return b0 + 8u * (uint32_t)(2 * STAGES + 4); }
+    static constexpr int kCount = 2 * STAGES + 5;
+    __device__ void init(int epi_threads) const {
+        for (int s = 0; s < STAGES; ++s) { mbar_init(full(s), 1); mbar_init(empty(s), 1); }
+        for (int b = 0; b < 2; ++b) { mbar_init(tfull(b), 1); mbar_init(tempty(b), (uint32_t)epi_threads); }
+        mbar_init(drain(), 1);
+    }
+};
+
+// Producer (one thread): tile `it` is rows row0 + it * ROWS of `map`.
+template <int STAGES, int ROWS>
+__device__ void tc_produce(const CUtensorMap* map, int64_t row0, int ntiles, uint8_t* sB, const TcBars<STAGES>& bar,
+                           volatile int* abort_flag) {
+    constexpr uint32_t bytes = ROWS * kDL * 2;
+    int issued = 0;
+    for (int it = 0; it < ntiles; ++it) {
+        const int s = it % STAGES;
+        if (!mbar_wait(bar.empty(s), ((uint32_t)(it / STAGES) & 1u) ^ 1u, abort_flag)) break;
+        mbar_expect_tx(bar.full(s), bytes);
+        tma_load_2d(smem_u32(sB + s * bytes), map, 0, (int32_t)(row0 + (int64_t)it * ROWS), bar.full(s));
+        ++issued;
+    }
+    // after an abort, let this thread's copies land before the CTA exits
+    if (*abort_flag)
+        for (int it = max(0, issued - STAGES); it < issued; ++it)
+            mbar_wait(bar.full(it % STAGES), (uint32_t)(it / STAGES) & 1u, abort_flag, false);
+}
+
+// MMA issuer (one thread): per tile and block, D[(buf * BLK + blk) * N] =
+// A_blk * B_tile^T over K = 64 (+ the extra K = 16 step when EXTRA).
+template <int BLK, int N, int STAGES, bool EXTRA>
+__device__ void tc_mma(uint32_t tmem, const uint8_t* sA, const uint8_t* sB, const uint8_t* sAx, const uint8_t* sBx,
+                       int ntiles, const TcBars<STAGES>& bar, volatile int* abort_flag) {
+    constexpr uint32_t idesc = umma_idesc_bf16(128, N);
+    constexpr uint32_t bbytes = N * kDL * 2;
+    for (int it = 0; it < ntiles; ++it) {
+        const int s = it % STAGES, b = it & 1;
+        if (!mbar_wait(bar.tempty(b), ((uint32_t)(it >> 1) & 1u) ^ 1u, abort_flag)) break;
+        if (!mbar_wait(bar.full(s), (uint32_t)(it / STAGES) & 1u, abort_flag)) break;
+        tc_fence_after();
+        const uint32_t b0 = smem_u32(sB + s * bbytes);
+#pragma unroll
+        for (int blk = 0; blk < BLK; ++blk) {
+            const uint32_t d = tmem + (uint32_t)((b * BLK + blk) * N);
+            const uint32_t a0 = smem_u32(sA + blk * kTcABytes);
+#pragma unroll
+            for (int k = 0; k < kDL / 16; ++k)
+                umma_bf16(d, sw128_desc(a0 + 32u * k), sw128_desc(b0 + 32u * k), idesc, k > 0 ? 1u : 0u);
+            if (EXTRA)
+                umma_bf16(d, noswz_desc(smem_u32(sAx + blk * kTcAxBytes), 128, 256), noswz_desc(smem_u32(sBx), 128, 256),
+                          idesc, 1u);
+        }
+        umma_commit(bar.empty(s));
+        umma_commit(bar.tfull(b));
+    }
+    // every MMA this thread issued has completed once `drain` fires
+    umma_commit(bar.drain());
+    mbar_wait(bar.drain(), 0, abort_flag, false);
+}
+
+// Epilogue row of a CTA: row r of the CTA's latent rows.
+struct EpiRow {
+    int64_t q, qq, t, orow;
+    int ncol;
+    bool valid, owner;
+};
+
+template <int G>
+__device__ __forceinline__ EpiRow epi_row(const PassArgs& a, int64_t q0, int h, int r) {
+    EpiRow e;
+    e.q = q0 + r / G;
+    e.valid = e.q < a.nqc;
+    e.owner = e.valid && (r % G) == 0;
+    e.qq = e.valid ? e.q : 0;
+    e.t = a.t_first + e.qq;
+    e.ncol = (int)flat_ncol_d(e.t, a.W, a.NB);
+    e.orow = e.qq * a.hkv + h;
+    return e;
+}
+
 // G: latent rows per query (1 for the group-mean score, hq / hkv for the
 // native per-head max).
 template <int G>
-__global__ void __launch_bounds__(kTcThreads, 1)
-flat_tc_kernel(const __grid_constant__ CUtensorMap tmF, const __grid_constant__ CUtensorMap tmS, PassArgs a) {
+__global__ void __launch_bounds__(kSmThreads, 1)
+flat_sample_kernel(const __grid_constant__ CUtensorMap tmS, PassArgs a) {
     extern __shared__ uint8_t tsm_raw[];
-    // 1024-byte alignment for the 128-byte swizzle atoms
     uint8_t* tsm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(tsm_raw) + 1023) & ~(uintptr_t)1023);
     uint8_t* sA = tsm;                                   // [block] 16 KB
-    uint8_t* sB = sA + kTcBlocks * kTcABytes;            // [stage] 16 KB
-    uint8_t* sAx = sB + kTcStages * kTcBBytes;           // [block] 4 KB
-    uint8_t* sBx = sAx + kTcBlocks * kTcAxBytes;         // 4 KB
-    uint8_t* scratch = sBx + kTcBxBytes;                 // histogram, then staging rows
-    uint32_t* hist = reinterpret_cast<uint32_t*>(scratch);
-    float* stg = reinterpret_cast<float*>(scratch);
-    uint64_t* bars = reinterpret_cast<uint64_t*>(scratch + kTcScratchBytes);
-    // bars: full[S], empty[S], tfull[2], tempty[2], tau_ready, drain
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * kTcStages + 6);
+    uint8_t* sB = sA + kSmBlocks * kTcABytes;            // [stage] 16 KB
+    uint32_t* hist = reinterpret_cast<uint32_t*>(sB + kSmStages * kSmBBytes);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(hist) + kSmHistBytes);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + TcBars<kSmStages>::kCount);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+    const TcBars<kSmStages> bar{smem_u32(bars)};
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int h = blockIdx.y;
-    constexpr int qpt = kTcRows / G;
+    constexpr int qpt = kSmRows / G;
     const int64_t q0 = (int64_t)blockIdx.x * qpt;
     if (q0 >= a.nqc) return;
     const int64_t qlast = min(a.nqc - 1, q0 + qpt - 1);
     const int64_t ncol_max = flat_ncol_d(a.t_first + qlast, a.W, a.NB);
-    const int64_t ncol_min = flat_ncol_d(a.t_first + q0, a.W, a.NB);
-    const int ns_tiles = (int)ceil_div<int64_t>(ceil_div<int64_t>(ncol_max, kSampleStride), kTcCols);
-    const int ntiles = ns_tiles + (int)ceil_div<int64_t>(ncol_max, kTcCols);
-
-    const uint32_t bar0 = smem_u32(bars);
-    const uint32_t tau_ready = bar0 + 8u * (2 * kTcStages + 4);
-    const uint32_t drain = bar0 + 8u * (2 * kTcStages + 5);
-#define FULL(s) (bar0 + 8u * (uint32_t)(s))
-#define EMPTY(s) (bar0 + 8u * (uint32_t)(kTcStages + (s)))
-#define TFULL(b) (bar0 + 8u * (uint32_t)(2 * kTcStages + (b)))
-#define TEMPTY(b) (bar0 + 8u * (uint32_t)(2 * kTcStages + 2 + (b)))
+    const int ntiles = (int)ceil_div<int64_t>(ceil_div<int64_t>(ncol_max, kSampleStride), kSmCols);
 
     if (tid == 0) {
-        for (int s = 0; s < kTcStages; ++s) { mbar_init(FULL(s), 1); mbar_init(EMPTY(s), 1); }
-        for (int b = 0; b < 2; ++b) { mbar_init(TFULL(b), 1); mbar_init(TEMPTY(b), kTcEpi); }
-        mbar_init(tau_ready, kTcEpi);
-        mbar_init(drain, 1);
+        bar.init(kSmRows);
         *abort_flag = 0;
         fence_barrier_init();
     }
-    if (warp == 1) tmem_alloc(smem_u32(tmem_slot), kTcTmemCols);
-    for (int i = tid; i < kHBins * kTcRows; i += kTcThreads) hist[i] = 0u;
-    // extra K step: B = 1 in its first column (bf16 0x3F80); A filled in once tau is known
-    for (int i = tid; i < kTcCols * 2; i += kTcThreads) {
-        const int n = i >> 1, kh = i & 1;
-        *reinterpret_cast<uint4*>(sBx + noswz_off(n, kh)) = make_uint4(kh == 0 ? 0x3F80u : 0u, 0u, 0u, 0u);
-    }
-    if (tid >= 64) {
-        // A: the CTA's 256 latent rows (block r / 128), 128-byte swizzled;
-        // rows past the chunk are zero
-        const int r = tid - 64;
-        const int64_t q = q0 + r / G;
-        uint4* dst = reinterpret_cast<uint4*>(sA + (r >> 7) * kTcABytes + (r & 127) * 128);
-        if (q < a.nqc) {
-            const int64_t yrow = G > 1 ? (q * a.hkv + h) * G + r % G : q * a.hkv + h;
-            const uint4* src = reinterpret_cast<const uint4*>(a.Y + yrow * kDL);
-#pragma unroll
-            for (int c = 0; c < 8; ++c) dst[c ^ (r & 7)] = src[c];
-        } else {
-#pragma unroll
-            for (int c = 0; c < 8; ++c) dst[c] = make_uint4(0, 0, 0, 0);
-        }
-    }
+    if (warp == 1) tmem_alloc(smem_u32(tmem_slot), 512);
+    for (int i = tid; i < kHBins / 2 * kSmRows; i += kSmThreads) hist[i] = 0u;
+    const int quarter = warp & 3, blk = (warp - 2) >> 2;
+    const int r = blk * 128 + quarter * 32 + lane;  // epilogue row of this thread
+    if (warp >= 2) fill_a_row<G>(sA, a, q0, h, r);
     fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
@@ -199,71 +274,16 @@ flat_tc_kernel(const __grid_constant__ CUtensorMap tmF, const __grid_constant__ 
     const uint32_t tmem = *tmem_slot;
 
     if (warp == 0) {
-        if (lane == 0) {
-            // producer: sampled tiles first, then every eligible tile
-            int issued = 0;
-            for (int it = 0; it < ntiles; ++it) {
-                const int s = it % kTcStages;
-                if (!mbar_wait(EMPTY(s), ((uint32_t)(it / kTcStages) & 1u) ^ 1u, abort_flag)) break;
-                mbar_expect_tx(FULL(s), kTcBBytes);
-                if (it < ns_tiles)
-                    tma_load_2d(smem_u32(sB + s * kTcBBytes), &tmS, 0,
-                                (int32_t)((int64_t)h * a.ns_cap + (int64_t)it * kTcCols), FULL(s));
-                else
-                    tma_load_2d(smem_u32(sB + s * kTcBBytes), &tmF, 0,
-                                (int32_t)((int64_t)h * a.cap_buckets + (int64_t)(it - ns_tiles) * kTcCols), FULL(s));
-                ++issued;
-            }
-            // after an abort, let this thread's copies land before the CTA exits
-            if (*abort_flag)
-                for (int it = max(0, issued - kTcStages); it < issued; ++it)
-                    mbar_wait(FULL(it % kTcStages), (uint32_t)(it / kTcStages) & 1u, abort_flag, false);
-        }
+        if (lane == 0) tc_produce<kSmStages, kSmCols>(&tmS, (int64_t)h * a.ns_cap, ntiles, sB, bar, abort_flag);
     } else if (warp == 1) {
-        if (lane == 0) {
-            const uint64_t bxd = noswz_desc(smem_u32(sBx), 128, 256);
-            for (int it = 0; it < ntiles; ++it) {
-                const int s = it % kTcStages, b = it & 1;
-                if (!mbar_wait(TEMPTY(b), ((uint32_t)(it >> 1) & 1u) ^ 1u, abort_flag)) break;
-                if (!mbar_wait(FULL(s), (uint32_t)(it / kTcStages) & 1u, abort_flag)) break;
-                if (it == ns_tiles && !mbar_wait(tau_ready, 0, abort_flag)) break;
-                tc_fence_after();
-                const uint32_t b0 = smem_u32(sB + s * kTcBBytes);
-#pragma unroll
-                for (int blk = 0; blk < kTcBlocks; ++blk) {
-                    const uint32_t d = tmem + (uint32_t)((b * kTcBlocks + blk) * kTcCols);
-                    const uint32_t a0 = smem_u32(sA + blk * kTcABytes);
-#pragma unroll
-                    for (int k = 0; k < kDL / 16; ++k)
-                        umma_bf16(d, sw128_desc(a0 + 32u * k), sw128_desc(b0 + 32u * k), kTcIdesc, k > 0 ? 1u : 0u);
-                    if (it >= ns_tiles)
-                        umma_bf16(d, noswz_desc(smem_u32(sAx + blk * kTcAxBytes), 128, 256), bxd, kTcIdesc, 1u);
-                }
-                umma_commit(EMPTY(s));
-                umma_commit(TFULL(b));
-            }
-            // every MMA this thread issued has completed once `drain` fires
-            umma_commit(drain);
-            mbar_wait(drain, 0, abort_flag, false);
-        }
+        if (lane == 0) tc_mma<kSmBlocks, kSmCols, kSmStages, false>(tmem, sA, sB, nullptr, nullptr, ntiles, bar, abort_flag);
     } else {
-        // epilogue: warp w owns rows 128 * blk + 32 * (w % 4) + lane of block
-        // blk = (w - 2) / 4 (TMEM lane quarter w % 4)
-        const int quarter = warp & 3, blk = (warp - 2) >> 2;
-        const int r = blk * 128 + quarter * 32 + lane;
-        const int64_t q = q0 + r / G;
-        const bool valid = q < a.nqc;
-        const bool owner = valid && (r % G) == 0;
-        const int64_t qq = valid ? q : 0;
-        const int64_t t = a.t_first + qq;
-        const int ncol = (int)flat_ncol_d(t, a.W, a.NB);
-        const int64_t orow = qq * a.hkv + h;
-        const uint32_t trow = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(blk * kTcCols);
-
+        const EpiRow e = epi_row<G>(a, q0, h, r);
+        const uint32_t trow = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(blk * kSmCols);
         // R bounds |score| of the row: |s| <= |y| |c| < 1.01 |y| (|c| <= 1 + 2^-8)
         float n2 = 0.f;
         {
-            const int64_t yrow = G > 1 ? (qq * a.hkv + h) * G + r % G : orow;
+            const int64_t yrow = G > 1 ? (e.qq * a.hkv + h) * G + r % G : e.orow;
             const uint4* yp = reinterpret_cast<const uint4*>(a.Y + yrow * kDL);
 #pragma unroll
             for (int c = 0; c < 8; ++c) {
@@ -283,105 +303,160 @@ flat_tc_kernel(const __grid_constant__ CUtensorMap tmF, const __grid_constant__ 
         // with at most kOversample * k of them and no more than kCandCap
         // buckets in range take every bucket (tau = -inf).  Histogram range
         // [lo, R): rows with at least four times that target bin [0, R) only
-        // (their tau lies in the upper tail), others the whole [-R, R).  Bin of s:
-        // round(s * bsc + boff - 0.5), computed by adding 1.5 * 2^23 (the
-        // float's last place is then 1) and clamped to [0, kHBins).
-        const long long n_elig = max(0LL, (long long)(t - a.W) - a.S + 1);
-        const bool take_all = n_elig <= (long long)kOversample * a.k && ncol <= kCandCap;
+        // (their tau lies in the upper tail), others the whole [-R, R).  Bin
+        // of s: round(s * bsc + boff - 0.5), computed by adding 1.5 * 2^23
+        // (the float's last place is then 1) and clamped to [0, kHBins).
+        const long long n_elig = max(0LL, (long long)(e.t - a.W) - a.S + 1);
+        const bool take_all = n_elig <= (long long)kOversample * a.k && e.ncol <= kCandCap;
         const bool upper = n_elig >= 4LL * kOversample * a.k;
         const float lo = upper ? 0.f : -R;
         const float bsc = (float)kHBins / (R - lo);
         const float boff = -lo * bsc - 0.5f + 12582912.0f;
+        const int ns_row = e.owner ? (e.ncol + kSampleStride - 1) / kSampleStride : 0;
 
         uint32_t va[32], vb[32];
-        int it = 0;
-        // phase 1: histogram of the sampled scores, one count per sampled
-        // bucket (buckets hold 8 keys on average, a block's 512 keys in 64)
-        for (; it < ns_tiles; ++it) {
+        // one count per sampled bucket (buckets hold 8 keys on average: a
+        // block's 512 keys in 64); 16-bit counts, two bins per word
+        for (int it = 0; it < ntiles; ++it) {
             const int b = it & 1;
-            if (!__all_sync(0xffffffffu, mbar_wait(TFULL(b), (uint32_t)(it >> 1) & 1u, abort_flag))) break;
+            if (!__all_sync(0xffffffffu, mbar_wait(bar.tfull(b), (uint32_t)(it >> 1) & 1u, abort_flag))) break;
             tc_fence_after();
-            const uint32_t tb = trow + (uint32_t)(b * kTcBlocks * kTcCols);
-            auto sample_chunk = [&](uint32_t (&v)[32], uint32_t (&vn)[32], int c) {
-                if (c + 1 < kTcCols / 32) tmem_ld32_async(tb + (uint32_t)((c + 1) * 32), vn);
+            const uint32_t tb = trow + (uint32_t)(b * kSmBlocks * kSmCols);
+            auto chunk = [&](uint32_t (&v)[32], uint32_t (&vn)[32], int c) {
+                if (c + 1 < kSmCols / 32) tmem_ld32_async(tb + (uint32_t)((c + 1) * 32), vn);
                 group_max<G>(v);
-                const int j0 = it * kTcCols + c * 32;  // sampled column; its bucket is 8 j
-                // columns a row may score: 8 j < ncol
-                const int nval = !owner ? 0 : min(32, max(0, (ncol + kSampleStride - 1) / kSampleStride - j0));
+                const int nval = min(32, max(0, ns_row - (it * kSmCols + c * 32)));
 #pragma unroll
                 for (int i = 0; i < 32; ++i) {
-                    const int bin = min(kHBins - 1, max(0, __float_as_int(fmaf(__uint_as_float(v[i]), bsc, boff)) - 0x4B400000));
-                    if (i < nval) atomicAdd(&hist[bin * kTcRows + r], 1u);
+                    const int bin =
+                        min(kHBins - 1, max(0, __float_as_int(fmaf(__uint_as_float(v[i]), bsc, boff)) - 0x4B400000));
+                    if (i < nval) atomicAdd(&hist[(bin >> 1) * kSmRows + r], 1u << ((bin & 1) << 4));
                 }
-                if (c + 1 < kTcCols / 32) tmem_wait_ld(vn);
+                if (c + 1 < kSmCols / 32) tmem_wait_ld(vn);
             };
             tmem_ld32_async(tb, va);
             tmem_wait_ld(va);
 #pragma unroll 1
-            for (int c = 0; c < kTcCols / 32; c += 2) {
-                sample_chunk(va, vb, c);
-                sample_chunk(vb, va, c + 1);
+            for (int c = 0; c < kSmCols / 32; c += 2) {
+                chunk(va, vb, c);
+                chunk(vb, va, c + 1);
             }
             tc_fence_before();
-            mbar_arrive(TEMPTY(b));
+            mbar_arrive(bar.tempty(b));
         }
         // tau: lower edge of the bin where the sampled key estimate (8 keys
         // per bucket, every 8th bucket) from the top first reaches
-        // kOversample * k, rounded down to bf16 (it enters the extra K step);
-        // -inf if never (the upper-only range then still reports the whole
-        // count at bin 0, so an upper row whose target lies below 0 gets 0)
+        // kOversample * k, rounded down to bf16 (it enters the extra K step
+        // of the candidate kernel); -inf if never (an upper-range row whose
+        // target lies below 0 gets 0: bin 0 holds every score below 0)
         float tau = -CUDART_INF_F;
         if (!take_all) {
             long long cum = 0;
             const long long need = ((long long)kOversample * a.k + 63) / 64;  // sampled buckets
             for (int bn = kHBins - 1; bn >= 0; --bn) {
-                cum += hist[bn * kTcRows + r];
+                cum += (hist[(bn >> 1) * kSmRows + r] >> ((bn & 1) << 4)) & 0xFFFFu;
                 if (cum >= need) { tau = lo + bn * ((R - lo) / kHBins); break; }
             }
         }
-        tau = bf16_floor(tau);
-        if (G > 1) tau = __shfl_sync(0xffffffffu, tau, lane & ~(G - 1));  // the query's owner lane
+        if (e.owner) a.tau[e.orow] = bf16_floor(tau);
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+template <int G>
+__global__ void __launch_bounds__(kCdThreads, 1)
+flat_cand_kernel(const __grid_constant__ CUtensorMap tmF, PassArgs a) {
+    extern __shared__ uint8_t tsm_raw[];
+    uint8_t* tsm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(tsm_raw) + 1023) & ~(uintptr_t)1023);
+    uint8_t* sA = tsm;                                   // [block] 16 KB
+    uint8_t* sB = sA + kCdBlocks * kTcABytes;            // [stage] 8 KB
+    uint8_t* sAx = sB + kCdStages * kCdBBytes;           // [block] 4 KB
+    uint8_t* sBx = sAx + kCdBlocks * kTcAxBytes;         // 2 KB
+    float* stg = reinterpret_cast<float*>(sBx + kCdBxBytes);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(stg) + kCdStgBytes);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + TcBars<kCdStages>::kCount);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+    const TcBars<kCdStages> bar{smem_u32(bars)};
+
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int h = blockIdx.y;
+    constexpr int qpt = kCdRows / G;
+    const int64_t q0 = (int64_t)blockIdx.x * qpt;
+    if (q0 >= a.nqc) return;
+    const int64_t qlast = min(a.nqc - 1, q0 + qpt - 1);
+    const int ntiles = (int)ceil_div<int64_t>(flat_ncol_d(a.t_first + qlast, a.W, a.NB), kCdCols);
+
+    if (tid == 0) {
+        bar.init(kCdRows);
+        *abort_flag = 0;
+        fence_barrier_init();
+    }
+    if (warp == 1) tmem_alloc(smem_u32(tmem_slot), 512);
+    // extra K step: B = 1 in its first column (bf16 0x3F80)
+    for (int i = tid; i < kCdCols * 2; i += kCdThreads) {
+        const int n = i >> 1, kh = i & 1;
+        *reinterpret_cast<uint4*>(sBx + noswz_off(n, kh)) = make_uint4(kh == 0 ? 0x3F80u : 0u, 0u, 0u, 0u);
+    }
+    const int quarter = warp & 3, blk = (warp - 2) >> 2;
+    const int r = blk * 128 + quarter * 32 + lane;  // epilogue row of this thread
+    float tau = -CUDART_INF_F;
+    EpiRow e{};
+    if (warp >= 2) {
+        fill_a_row<G>(sA, a, q0, h, r);
+        e = epi_row<G>(a, q0, h, r);
+        tau = e.valid ? a.tau[e.orow] : -CUDART_INF_F;
+        // A's extra column: -tau (exact: tau is a bf16 value), 0 when tau = -inf
+        const float tau_add = tau == -CUDART_INF_F ? 0.f : tau;
+        uint8_t* ax = sAx + blk * kTcAxBytes;
+        const int rb = r & 127;
+        *reinterpret_cast<uint4*>(ax + noswz_off(rb, 0)) =
+            make_uint4((uint32_t)(__float_as_uint(-tau_add) >> 16), 0u, 0u, 0u);
+        *reinterpret_cast<uint4*>(ax + noswz_off(rb, 1)) = make_uint4(0u, 0u, 0u, 0u);
+    }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        if (lane == 0) tc_produce<kCdStages, kCdCols>(&tmF, (int64_t)h * a.cap_buckets, ntiles, sB, bar, abort_flag);
+    } else if (warp == 1) {
+        if (lane == 0) tc_mma<kCdBlocks, kCdCols, kCdStages, true>(tmem, sA, sB, sAx, sBx, ntiles, bar, abort_flag);
+    } else {
+        const uint32_t trow = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(blk * kCdCols);
         const bool tau_inf = tau == -CUDART_INF_F;
         const float tau_add = tau_inf ? 0.f : tau;
-        if (owner) a.tau[orow] = tau;
-        {
-            uint8_t* ax = sAx + blk * kTcAxBytes;
-            const int rb = quarter * 32 + lane;
-            const uint32_t nb = (uint32_t)(__float_as_uint(-tau_add) >> 16);  // exact: tau_add is a bf16 value
-            *reinterpret_cast<uint4*>(ax + noswz_off(rb, 0)) = make_uint4(nb, 0u, 0u, 0u);
-            *reinterpret_cast<uint4*>(ax + noswz_off(rb, 1)) = make_uint4(0u, 0u, 0u, 0u);
-            fence_proxy_async_smem();
-            mbar_arrive(tau_ready);
-        }
-        // the histogram's space becomes the staging rows: every epilogue
-        // thread has read its bins past this barrier
-        asm volatile("bar.sync 1, %0;\n" ::"n"(kTcEpi) : "memory");
         float* my_stg = stg + r * kTcStgStride;
-
-        // phase 2: TMEM holds s - tau_add; candidates (score >= tau) are
-        // appended in ascending bucket id (the thread owns its row)
-        int2* cand = a.cand + orow * (int64_t)kCandCap;
+        int2* cand = a.cand + e.orow * (int64_t)kCandCap;
         int cnt = 0;
-        for (; it < ntiles; ++it) {
+        uint32_t va[32], vb[32];
+        // TMEM holds s - tau_add; candidates (score >= tau) are appended in
+        // ascending bucket id (the thread owns its row)
+        for (int it = 0; it < ntiles; ++it) {
             const int b = it & 1;
-            if (!__all_sync(0xffffffffu, mbar_wait(TFULL(b), (uint32_t)(it >> 1) & 1u, abort_flag))) break;
+            if (!__all_sync(0xffffffffu, mbar_wait(bar.tfull(b), (uint32_t)(it >> 1) & 1u, abort_flag))) break;
             tc_fence_after();
-            const uint32_t tb = trow + (uint32_t)(b * kTcBlocks * kTcCols);
-            const int tbase = (it - ns_tiles) * kTcCols;
-            auto cand_chunk = [&](uint32_t (&v)[32], uint32_t (&vn)[32], int c) {
-                if (c + 1 < kTcCols / 32) tmem_ld32_async(tb + (uint32_t)((c + 1) * 32), vn);
+            const uint32_t tb = trow + (uint32_t)(b * kCdBlocks * kCdCols);
+            auto chunk = [&](uint32_t (&v)[32], uint32_t (&vn)[32], int c) {
+                if (c + 1 < kCdCols / 32) tmem_ld32_async(tb + (uint32_t)((c + 1) * 32), vn);
                 group_max<G>(v);
-                const int col0 = tbase + c * 32;
-                const int rem = ncol - col0;
-                const uint32_t lm = !owner || rem <= 0 ? 0u : (rem >= 32 ? 0xffffffffu : ((1u << rem) - 1u));
-                // sign bits of s - tau: bit i set = miss
-                uint32_t shi = 0u, slo = 0u;
+                const int col0 = it * kCdCols + c * 32;
+                const int rem = e.ncol - col0;
+                const uint32_t lm = !e.owner || rem <= 0 ? 0u : (rem >= 32 ? 0xffffffffu : ((1u << rem) - 1u));
+                // sign bits of s - tau (bit i set = miss), four independent chains
+                uint32_t sg[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
-                for (int i = 15; i >= 0; --i) {
-                    shi = __funnelshift_l(v[16 + i], shi, 1);
-                    slo = __funnelshift_l(v[i], slo, 1);
-                }
-                uint32_t hits = (tau_inf ? 0xffffffffu : ~((shi << 16) | slo)) & lm;
+                for (int i = 7; i >= 0; --i)
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) sg[j] = __funnelshift_l(v[8 * j + i], sg[j], 1);
+                const uint32_t miss = sg[0] | (sg[1] << 8) | (sg[2] << 16) | (sg[3] << 24);
+                uint32_t hits = (tau_inf ? 0xffffffffu : ~miss) & lm;
                 if (__any_sync(0xffffffffu, hits)) {
 #pragma unroll
                     for (int j = 0; j < 8; ++j)
@@ -393,45 +468,34 @@ flat_tc_kernel(const __grid_constant__ CUtensorMap tmF, const __grid_constant__ 
                         ++cnt;
                     }
                 }
-                if (c + 1 < kTcCols / 32) tmem_wait_ld(vn);
+                if (c + 1 < kCdCols / 32) tmem_wait_ld(vn);
             };
             tmem_ld32_async(tb, va);
             tmem_wait_ld(va);
-#pragma unroll 1
-            for (int c = 0; c < kTcCols / 32; c += 2) {
-                cand_chunk(va, vb, c);
-                cand_chunk(vb, va, c + 1);
-            }
+            chunk(va, vb, 0);
+            chunk(vb, va, 1);
             tc_fence_before();
-            mbar_arrive(TEMPTY(b));
+            mbar_arrive(bar.tempty(b));
         }
-        if (owner) a.cand_n[orow] = cnt;
+        if (e.owner) a.cand_n[e.orow] = cnt;
     }
-#undef FULL
-#undef EMPTY
-#undef TFULL
-#undef TEMPTY
     tc_fence_before();
     __syncthreads();
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem, kTcTmemCols);
+        tmem_dealloc(tmem, 512);
     }
 }
 
 // --------------------------------------------------------------- resolve
 
 constexpr int kResWarps = 4;
+constexpr int kBandCap = 128;  // buckets ranked on exact scores per row
 
 struct ResolveArgs {
-    const int32_t* units;
-    const int32_t* offsets;
-    const int32_t* members;
-    const int32_t* cnt_lr;
-    const int32_t* minlr;
-    const int32_t* maxpos;
+    const int4* meta;        // [hkv, NB] (minlr, maxpos, cnt_lr, packed member units)
     const uint16_t* cent;
-    int64_t cap_units, cap_buckets, NB, T_built;
+    int64_t cap_buckets, NB, T_built;
     int32_t hkv, G, agg, k, S, W;
     const uint16_t* Y;
     int64_t nqc, t_first;
@@ -444,33 +508,35 @@ struct ResolveArgs {
     int32_t ovf_cap;
 };
 
-constexpr int kBandCap = 128;  // buckets ranked on exact scores per row
+// meta[h * NB + b] = (minlr, maxpos, cnt_lr, units) of bucket b < NB: one 16-byte
+// record per bucket for the resolve's gathers.
+__global__ void meta_gather_kernel(const int32_t* __restrict__ minlr, const int32_t* __restrict__ maxpos,
+                                   const int32_t* __restrict__ cnt_lr, const int32_t* __restrict__ units,
+                                   int64_t cap_buckets, int64_t NB, int32_t hkv, int4* __restrict__ meta) {
+    const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (idx >= (int64_t)hkv * NB) return;
+    const int64_t hb = (idx / NB) * cap_buckets + idx % NB;
+    meta[idx] = make_int4(minlr[hb], maxpos[hb], cnt_lr[hb], units[hb]);
+}
 
 struct ResWarp {
     double bex[kBandCap];     // exact scores of the band
-    int32_t col[kCandCap];    // eligible candidates, ascending bucket id
-    float sc[kCandCap];       // their fp32 scores
-    int32_t w[kCandCap];      // key weights, then taken counts
-    int32_t pk[kCandCap];     // packed member units
-    int32_t bidx[kBandCap];   // band members (index into col)
+    int2 cs[kCandCap];        // eligible candidates (bucket id, fp32 score bits), ascending id
+    uint8_t w[kCandCap];      // key weights (<= 16), then taken counts
+    int16_t bidx[kBandCap];   // band members (index into cs)
     uint32_t hist[256];
     uint16_t ylat[8 * kDL];
 };
 
-__device__ __forceinline__ uint32_t order_key_f(float s) {
-    const uint32_t u = __float_as_uint(s + 0.0f);
-    return (u >> 31) ? ~u : (u | 0x80000000u);
-}
-
 // Keys of bucket b in [S, lim]; `pk` is the bucket's packed member units.
-__device__ __forceinline__ int weight_packed(const ResolveArgs& a, int64_t b, int32_t pk, int64_t lim) {
+__device__ __noinline__ int weight_packed(int64_t b, int32_t pk, int64_t lim, int32_t S, int64_t T_built) {
     const int64_t ubase = (b / kBucketsPerBlock) * kUnitsPerBlock;
     const int cnt = (pk >> 28) & 7;
     int w = 0;
     for (int i = 0; i < cnt; ++i) {
         const int64_t j = ubase + ((pk >> (7 * i)) & 127);
-        for (int64_t p = j * kPool; p < j * kPool + kPool && p < a.T_built; ++p)
-            if (p >= a.S && p <= lim) ++w;
+        for (int64_t p = j * kPool; p < j * kPool + kPool && p < T_built; ++p)
+            if (p >= S && p <= lim) ++w;
     }
     return w;
 }
@@ -478,12 +544,12 @@ __device__ __forceinline__ int weight_packed(const ResolveArgs& a, int64_t b, in
 // First `tk` keys of bucket b in [S, lim], ascending (member units are
 // packed in ascending order).  Fast path: a bucket taken whole that lies
 // inside [S, lim] with full units writes 4 consecutive positions per unit.
-__device__ void emit_keys(const ResolveArgs& a, int64_t b, int32_t pk, int tk, int64_t lim,
-                          int32_t* out) {
+__device__ __noinline__ void emit_keys(int64_t b, int32_t pk, int tk, int64_t lim, int32_t S, int64_t T_built,
+                                      int32_t* out) {
     const int64_t ubase = (b / kBucketsPerBlock) * kUnitsPerBlock;
     const int cnt = (pk >> 28) & 7;
     const int64_t j0 = ubase + (pk & 127);
-    if (tk == cnt * kPool && j0 * kPool >= a.S) {
+    if (tk == cnt * kPool && j0 * kPool >= S) {
         int o = 0;
         for (int i = 0; i < cnt; ++i) {
             const int32_t p = (int32_t)((ubase + ((pk >> (7 * i)) & 127)) * kPool);
@@ -495,8 +561,8 @@ __device__ void emit_keys(const ResolveArgs& a, int64_t b, int32_t pk, int tk, i
     int o = 0;
     for (int i = 0; i < cnt && o < tk; ++i) {
         const int64_t j = ubase + ((pk >> (7 * i)) & 127);
-        for (int64_t p = j * kPool; p < j * kPool + kPool && p < a.T_built && o < tk; ++p)
-            if (p >= a.S && p <= lim) out[o++] = (int32_t)p;
+        for (int64_t p = j * kPool; p < j * kPool + kPool && p < T_built && o < tk; ++p)
+            if (p >= S && p <= lim) out[o++] = (int32_t)p;
     }
 }
 
@@ -531,7 +597,51 @@ __device__ __forceinline__ void push_fallback(const ResolveArgs& a, int64_t row)
     else raise_device_error(kErrSelectOverflow);
 }
 
-__global__ void __launch_bounds__(32 * kResWarps, 4) flat_resolve_kernel(ResolveArgs a) {
+// Weighted cut over 256 bins (descending): the bin where the weight from the
+// top first reaches `need`; *above = the weight of the bins above it.
+// -1 if the bins hold less than `need`.
+__device__ __forceinline__ int cut_bin(const uint32_t* hist, long long need, long long* above) {
+    const int lane = threadIdx.x & 31;
+    long long s8 = 0;
+#pragma unroll
+    for (int d = 0; d < 8; ++d) s8 += hist[255 - 8 * lane - d];
+    long long incl = s8;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const long long y = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += y;
+    }
+    const long long excl = incl - s8;
+    const unsigned hitm = __ballot_sync(0xffffffffu, incl >= need && excl < need);
+    if (hitm == 0u) return -1;
+    const int src = __ffs(hitm) - 1;
+    int dig = 0;
+    long long cum = 0;
+    if (lane == src) {
+        cum = excl;
+        dig = 255 - 8 * lane;
+        for (int d = 0; d < 8; ++d) {
+            const int dd = 255 - 8 * lane - d;
+            if (cum + hist[dd] >= need) { dig = dd; break; }
+            cum += hist[dd];
+        }
+    }
+    *above = __shfl_sync(0xffffffffu, cum, src);
+    return __shfl_sync(0xffffffffu, dig, src);
+}
+
+__device__ __forceinline__ float warp_minf(float v) {
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) v = fminf(v, __shfl_xor_sync(0xffffffffu, v, off));
+    return v;
+}
+__device__ __forceinline__ float warp_maxf(float v) {
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, off));
+    return v;
+}
+
+__global__ void __launch_bounds__(32 * kResWarps, 3) flat_resolve_kernel(ResolveArgs a) {
     extern __shared__ __align__(16) uint8_t rsm[];
     const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
     ResWarp& sw = reinterpret_cast<ResWarp*>(rsm)[wid];
@@ -559,89 +669,79 @@ __global__ void __launch_bounds__(32 * kResWarps, 4) flat_resolve_kernel(Resolve
     }
     const float tau = a.tau[row];
 
-    // eligible candidates (kept in ascending bucket id) and their key counts
+    // eligible candidates (kept in ascending bucket id), their key counts
+    // and score range
     const int64_t hb0 = (int64_t)h * a.cap_buckets;
+    const int4* mrow = a.meta + (int64_t)h * a.NB;
+    const int2* crow = a.cand + row * kCandCap;
     int m = 0;
     long long wtot = 0;
+    float smin = CUDART_INF_F, smax = -CUDART_INF_F;
     for (int base = 0; base < n; base += 32) {
         const int i = base + lane;
         bool el = false;
-        int col = 0, wgt = 0;
-        float sc = 0.f;
-        int32_t pk = 0;
+        int2 cv = make_int2(0, 0);
+        int wgt = 0;
         if (i < n) {
-            const int2 cv = a.cand[row * kCandCap + i];
-            col = cv.x;
-            sc = __int_as_float(cv.y);
-            const int64_t hb = hb0 + col;
-            const int32_t mlr = a.minlr[hb], mxp = a.maxpos[hb], clr = a.cnt_lr[hb];
-            pk = a.units[hb];
-            el = (int64_t)mlr <= lim;
-            wgt = (int64_t)mxp <= lim ? clr : weight_packed(a, col, pk, lim);
+            cv = crow[i];
+            const int4 md = __ldg(mrow + cv.x);
+            el = (int64_t)md.x <= lim;
+            wgt = (int64_t)md.y <= lim ? md.z : weight_packed(cv.x, md.w, lim, a.S, a.T_built);
         }
-        if (el) wtot += wgt;
+        if (el) {
+            wtot += wgt;
+            smin = fminf(smin, __int_as_float(cv.y));
+            smax = fmaxf(smax, __int_as_float(cv.y));
+        }
         const unsigned bal = __ballot_sync(0xffffffffu, el);
         if (el) {
             const int pos = m + __popc(bal & ((1u << lane) - 1u));
-            sw.col[pos] = col;
-            sw.sc[pos] = sc;
-            sw.w[pos] = wgt;
-            sw.pk[pos] = pk;
+            sw.cs[pos] = cv;
+            sw.w[pos] = (uint8_t)wgt;
         }
         m += __popc(bal);
     }
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) wtot += __shfl_xor_sync(0xffffffffu, wtot, off);
+    smin = warp_minf(smin);
+    smax = warp_maxf(smax);
     __syncwarp();
 
     if (wtot > a.k) {
-        // weighted radix select on the fp32 scores: cut key K32 with
-        // weight(key > K32) < k <= weight(key >= K32)
-        uint32_t prefix = 0;
+        // the fp32 score of the k-th key lies in [lo_s, hi_s], the score
+        // range of the members of the cut bin: two passes of 256 linear bins
+        // over [smin, smax] (the second inside the first pass's cut bin)
+        const float inv = smax > smin ? 256.f / (smax - smin) : 0.f;
+        auto bin1 = [&](float s) { return min(255, (int)((s - smin) * inv)); };
+        for (int i = lane; i < 256; i += 32) sw.hist[i] = 0u;
+        __syncwarp();
+        for (int i = lane; i < m; i += 32) atomicAdd(&sw.hist[bin1(__int_as_float(sw.cs[i].y))], (unsigned)sw.w[i]);
+        __syncwarp();
         long long above = 0;
-        for (int pass = 0; pass < 4; ++pass) {
-            const int shift = 24 - 8 * pass;
-            for (int i = lane; i < 256; i += 32) sw.hist[i] = 0u;
-            __syncwarp();
-            for (int i = lane; i < m; i += 32) {
-                const uint32_t key = order_key_f(sw.sc[i]);
-                if (pass > 0 && (key >> (shift + 8)) != (prefix >> (shift + 8))) continue;
-                atomicAdd(&sw.hist[(key >> shift) & 255u], (unsigned)sw.w[i]);
-            }
-            __syncwarp();
-            long long s8 = 0;
-            for (int d = 0; d < 8; ++d) s8 += sw.hist[255 - 8 * lane - d];
-            long long incl = s8;
-#pragma unroll
-            for (int off = 1; off < 32; off <<= 1) {
-                const long long y = __shfl_up_sync(0xffffffffu, incl, off);
-                if (lane >= off) incl += y;
-            }
-            const long long excl = incl - s8;
-            const unsigned hitm = __ballot_sync(0xffffffffu, above + incl >= a.k && above + excl < a.k);
-            if (hitm == 0u) {  // cannot happen while the weight above the prefix reaches k
-                if (lane == 0) push_fallback(a, row);
-                return;
-            }
-            const int src = __ffs(hitm) - 1;
-            int dig = 0;
-            long long cum = 0;
-            if (lane == src) {
-                cum = above + excl;
-                dig = 255 - 8 * lane;
-                for (int d = 0; d < 8; ++d) {
-                    const int dd = 255 - 8 * lane - d;
-                    if (cum + sw.hist[dd] >= a.k) { dig = dd; break; }
-                    cum += sw.hist[dd];
-                }
-            }
-            dig = __shfl_sync(0xffffffffu, dig, src);
-            above = __shfl_sync(0xffffffffu, cum, src);
-            prefix |= (uint32_t)dig << shift;
-            __syncwarp();
+        const int b1 = cut_bin(sw.hist, a.k, &above);
+        __syncwarp();
+        auto bin2 = [&](float s) { return min(255, max(0, (int)(((s - smin) * inv - (float)b1) * 256.f))); };
+        for (int i = lane; i < 256; i += 32) sw.hist[i] = 0u;
+        __syncwarp();
+        for (int i = lane; i < m; i += 32) {
+            const float s = __int_as_float(sw.cs[i].y);
+            if (bin1(s) == b1) atomicAdd(&sw.hist[bin2(s)], (unsigned)sw.w[i]);
         }
-        const float c32 = __uint_as_float((prefix >> 31) ? (prefix & 0x7FFFFFFFu) : ~prefix);
-        const float hi = c32 + 2.f * kScoreErr, lo = c32 - 2.f * kScoreErr;
+        __syncwarp();
+        long long above2 = 0;
+        const int b2 = cut_bin(sw.hist, a.k - above, &above2);
+        if (b1 < 0 || b2 < 0) {  // cannot happen while the weights above reach k
+            if (lane == 0) push_fallback(a, row);
+            return;
+        }
+        float lo_s = CUDART_INF_F, hi_s = -CUDART_INF_F;
+        for (int i = lane; i < m; i += 32) {
+            const float s = __int_as_float(sw.cs[i].y);
+            if (bin1(s) == b1 && bin2(s) == b2) { lo_s = fminf(lo_s, s); hi_s = fmaxf(hi_s, s); }
+        }
+        lo_s = warp_minf(lo_s);
+        hi_s = warp_maxf(hi_s);
+        const float hi = hi_s + 2.f * kScoreErr, lo = lo_s - 2.f * kScoreErr;
         // every bucket that can rank above the exact cut must be a candidate:
         // non-candidates score <= tau (s - tau < 0 rounds to at most tau)
         if (tau > -CUDART_INF_F && !(lo > tau)) {
@@ -653,13 +753,13 @@ __global__ void __launch_bounds__(32 * kResWarps, 4) flat_resolve_kernel(Resolve
         int nb = 0;
         for (int base = 0; base < m; base += 32) {
             const int i = base + lane;
-            const float sc = i < m ? sw.sc[i] : -CUDART_INF_F;
+            const float sc = i < m ? __int_as_float(sw.cs[i].y) : -CUDART_INF_F;
             const bool band = i < m && sc >= lo && sc <= hi;
             if (i < m && sc > hi) win += sw.w[i];
             const unsigned bal = __ballot_sync(0xffffffffu, band);
             if (band) {
                 const int pos = nb + __popc(bal & ((1u << lane) - 1u));
-                if (pos < kBandCap) sw.bidx[pos] = i;
+                if (pos < kBandCap) sw.bidx[pos] = (int16_t)i;
             }
             nb += __popc(bal);
         }
@@ -675,12 +775,12 @@ __global__ void __launch_bounds__(32 * kResWarps, 4) flat_resolve_kernel(Resolve
         for (int i = lane; i < ng * kDL; i += 32) sw.ylat[i] = ysrc[i];
         __syncwarp();
         for (int i = lane; i < nb; i += 32)
-            sw.bex[i] = exact_row(sw.ylat, ng, a.cent + (hb0 + sw.col[sw.bidx[i]]) * kDL);
+            sw.bex[i] = exact_row(sw.ylat, ng, a.cent + (hb0 + sw.cs[sw.bidx[i]].x) * kDL);
         __syncwarp();
-        // taken counts: in -> whole, out -> 0, band -> pending (negative)
+        // taken counts: in -> whole, out -> 0, band -> pending (marked 0x80 | w)
         for (int i = lane; i < m; i += 32) {
-            const float sc = sw.sc[i];
-            sw.w[i] = sc > hi ? sw.w[i] : (sc >= lo ? -sw.w[i] : 0);
+            const float sc = __int_as_float(sw.cs[i].y);
+            sw.w[i] = sc > hi ? sw.w[i] : (sc >= lo ? (uint8_t)(0x80u | sw.w[i]) : (uint8_t)0);
         }
         __syncwarp();
         long long need = a.k - win;
@@ -690,9 +790,10 @@ __global__ void __launch_bounds__(32 * kResWarps, 4) flat_resolve_kernel(Resolve
             int bb = -1, bcol = 0x7FFFFFFF;
             for (int i = lane; i < nb; i += 32) {
                 const int ci = sw.bidx[i];
-                if (sw.w[ci] >= 0) continue;
+                if (!(sw.w[ci] & 0x80u)) continue;
                 const double e = sw.bex[i];
-                if (bb < 0 || e > bs || (e == bs && sw.col[ci] < bcol)) { bs = e; bb = ci; bcol = sw.col[ci]; }
+                const int col = sw.cs[ci].x;
+                if (bb < 0 || e > bs || (e == bs && col < bcol)) { bs = e; bb = ci; bcol = col; }
             }
 #pragma unroll
             for (int off = 16; off > 0; off >>= 1) {
@@ -702,15 +803,15 @@ __global__ void __launch_bounds__(32 * kResWarps, 4) flat_resolve_kernel(Resolve
                 if (ob >= 0 && (bb < 0 || os > bs || (os == bs && oc < bcol))) { bs = os; bb = ob; bcol = oc; }
             }
             if (bb < 0) break;
-            const int wv = -sw.w[bb];
+            const int wv = sw.w[bb] & 0x7F;
             const int tk = wv < need ? wv : (int)need;
             __syncwarp();
-            if (lane == 0) sw.w[bb] = tk;
+            if (lane == 0) sw.w[bb] = (uint8_t)tk;
             need -= tk;
             __syncwarp();
         }
         for (int i = lane; i < m; i += 32)
-            if (sw.w[i] < 0) sw.w[i] = 0;
+            if (sw.w[i] & 0x80u) sw.w[i] = 0;
         __syncwarp();
     } else if (tau > -CUDART_INF_F) {
         // fewer than k keys among the candidates, but buckets below tau exist
@@ -728,7 +829,10 @@ __global__ void __launch_bounds__(32 * kResWarps, 4) flat_resolve_kernel(Resolve
             const int y = __shfl_up_sync(0xffffffffu, incl, off);
             if (lane >= off) incl += y;
         }
-        if (tk > 0) emit_keys(a, sw.col[i], sw.pk[i], tk, lim, out + a.S + run + incl - tk);
+        if (tk > 0) {
+            const int col = sw.cs[i].x;
+            emit_keys(col, __ldg(&mrow[col].w), tk, lim, a.S, a.T_built, out + a.S + run + incl - tk);
+        }
         run += __shfl_sync(0xffffffffu, incl, 31);
     }
     for (int i = run + lane; i < a.k; i += 32) out[a.S + i] = -1;
@@ -746,16 +850,33 @@ lsa_status launch_sample_gather(const uint16_t* cent, int64_t cap_buckets, int64
     return check_launch("sample_gather_kernel");
 }
 
+// Packed bucket records for the resolve, once per call.
+lsa_status launch_meta_gather(const lsa_cache* c, int64_t NB, int4* meta, cudaStream_t st) {
+    const int64_t n = (int64_t)c->hkv * NB;
+    if (n == 0) return LSA_OK;
+    meta_gather_kernel<<<(unsigned)ceil_div<int64_t>(n, 256), 256, 0, st>>>(c->minlr, c->maxpos, c->cnt_lr, c->units,
+                                                                            c->cap_buckets, NB, c->hkv, meta);
+    return check_launch("meta_gather_kernel");
+}
+
+// tmF: centroids [hkv * cap_buckets, 64] in 64-row boxes; tmS: sampled
+// centroids [hkv * ns_cap, 64] in 128-row boxes.
 lsa_status launch_flat(const PassArgs& pa, const ResolveArgs& ra, const CUtensorMap& tmF, const CUtensorMap& tmS,
                        cudaStream_t st) {
     const int G = pa.agg ? pa.G : 1;
-    const int qpt = kTcRows / G;
-    dim3 grid((unsigned)ceil_div<int64_t>(pa.nqc, qpt), (unsigned)pa.hkv);
-    auto kern = G == 1 ? flat_tc_kernel<1> : G == 2 ? flat_tc_kernel<2> : G == 4 ? flat_tc_kernel<4> : flat_tc_kernel<8>;
-    cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kTcSmemBytes);
-    kern<<<grid, kTcThreads, kTcSmemBytes, st>>>(tmF, tmS, pa);
-    lsa_status s = check_launch("flat_tc_kernel");
+    auto ks = G == 1 ? flat_sample_kernel<1> : G == 2 ? flat_sample_kernel<2> : G == 4 ? flat_sample_kernel<4>
+                                                                                          : flat_sample_kernel<8>;
+    auto kc = G == 1 ? flat_cand_kernel<1> : G == 2 ? flat_cand_kernel<2> : G == 4 ? flat_cand_kernel<4>
+                                                                                    : flat_cand_kernel<8>;
+    cudaFuncSetAttribute(ks, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmSmemBytes);
+    cudaFuncSetAttribute(kc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kCdSmemBytes);
+    ks<<<dim3((unsigned)ceil_div<int64_t>(pa.nqc, kSmRows / G), (unsigned)pa.hkv), kSmThreads, kSmSmemBytes, st>>>(tmS,
+                                                                                                               pa);
+    lsa_status s = check_launch("flat_sample_kernel");
     if (s != LSA_OK) return s;
+    kc<<<dim3((unsigned)ceil_div<int64_t>(pa.nqc, kCdRows / G), (unsigned)pa.hkv), kCdThreads, kCdSmemBytes, st>>>(tmF,
+                                                                                                               pa);
+    if ((s = check_launch("flat_cand_kernel")) != LSA_OK) return s;
     const size_t smem_r = sizeof(ResWarp) * kResWarps;
     cudaFuncSetAttribute(flat_resolve_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_r);
     const int64_t rows = pa.nqc * pa.hkv;

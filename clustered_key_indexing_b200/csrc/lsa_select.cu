@@ -503,19 +503,20 @@ struct SelectPlan {
     int32_t hy;        // latent rows per query
     int32_t fb_slots;
     int64_t ns_cap;    // sampled buckets per kv-head (every 8th)
+    int64_t nb;        // buckets per kv-head (packed records)
 };
 
-// Query positions per flat-search chunk: the flat pass launches one CTA per
-// (256 / G latent rows, kv-head), so a chunk of a multiple of
+// Query positions per flat-search chunk: the candidate kernel launches one CTA
+// per (512 / G latent rows, kv-head), so a chunk of a multiple of
 // num_sms / gcd(num_sms, hkv) CTA row blocks fills whole waves; candidate
-// lists (kCandCap x 8 bytes per query and kv-head) stay within 1 GiB.
+// lists (kCandCap x 8 bytes per query and kv-head) stay within 2 GiB.
 int64_t select_chunk(const lsa_cfg* cfg, int32_t hq, int32_t hkv) {
-    const int64_t qpt = kTcRows / (cfg->agg ? hq / hkv : 1);
+    const int64_t qpt = kCdRows / (cfg->agg ? hq / hkv : 1);
     int64_t g = num_sms(), x = hkv;
     while (x) { const int64_t y = g % x; g = x; x = y; }
     const int64_t unit = num_sms() / g;
     const int64_t per_block = qpt * hkv * (int64_t)kCandCap * 8;
-    int64_t m = ((int64_t)1 << 30) / per_block / unit;
+    int64_t m = ((int64_t)2 << 30) / per_block / unit;
     if (m < 1) m = 1;
     return qpt * unit * m;
 }
@@ -530,6 +531,7 @@ static SelectPlan plan_select(const lsa_cfg* cfg, int64_t nq, int32_t hq, int32_
     p.chunk = c;
     p.fb_slots = 64;
     p.ns_cap = ceil_div<int64_t>(NB > 0 ? NB : 1, kSampleStride);
+    p.nb = NB > 0 ? NB : 1;
     return p;
 }
 
@@ -545,6 +547,7 @@ struct SelectWs {
     double* fb_score;
     int32_t* fb_w;
     uint16_t* cent_s;
+    int4* meta;
     size_t bytes;
 };
 
@@ -562,6 +565,7 @@ static SelectWs carve_select(const SelectPlan& p, int32_t hkv, int mode, char* b
         w.fb_score = (double*)(base + o); o += align256((size_t)p.fb_slots * p.ld * 8);
         w.fb_w = (int32_t*)(base + o); o += align256((size_t)p.fb_slots * p.ld * 4);
         w.cent_s = (uint16_t*)(base + o); o += align256((size_t)hkv * p.ns_cap * kDL * 2);
+        w.meta = (int4*)(base + o); o += align256((size_t)hkv * p.nb * 16);
     }
     w.bytes = o;
     return w;
@@ -612,8 +616,9 @@ lsa_status run_select(const uint16_t* Q, int64_t t0, int64_t nq, int32_t hq, con
     if (cfg->mode == 0) {
         lsa_status s = launch_sample_gather(c->cent, c->cap_buckets, NB, p.ns_cap, hkv, w.cent_s, st);
         if (s != LSA_OK) return s;
-        if ((s = make_rows64_map(&tmF, c->cent, (int64_t)hkv * c->cap_buckets, kTcCols)) != LSA_OK) return s;
-        if ((s = make_rows64_map(&tmS, w.cent_s, (int64_t)hkv * p.ns_cap, kTcCols)) != LSA_OK) return s;
+        if ((s = launch_meta_gather(c, NB, w.meta, st)) != LSA_OK) return s;
+        if ((s = make_rows64_map(&tmF, c->cent, (int64_t)hkv * c->cap_buckets, kCdCols)) != LSA_OK) return s;
+        if ((s = make_rows64_map(&tmS, w.cent_s, (int64_t)hkv * p.ns_cap, kSmCols)) != LSA_OK) return s;
     }
 
     for (int64_t c0 = 0; c0 < nq; c0 += p.chunk) {
@@ -635,8 +640,7 @@ lsa_status run_select(const uint16_t* Q, int64_t t0, int64_t nq, int32_t hq, con
         pa.W = cfg->window; pa.S = cfg->sinks; pa.hkv = hkv; pa.G = hq / hkv; pa.agg = cfg->agg; pa.k = cfg->k;
         pa.tau = w.tau; pa.cand = w.cand; pa.cand_n = w.cand_n;
         ResolveArgs ra{};
-        ra.units = c->units; ra.offsets = c->offsets; ra.members = c->members; ra.cnt_lr = c->cnt_lr; ra.minlr = c->minlr;
-        ra.maxpos = c->maxpos; ra.cent = c->cent; ra.cap_units = c->cap_units;
+        ra.meta = w.meta; ra.cent = c->cent;
         ra.cap_buckets = c->cap_buckets; ra.NB = NB; ra.T_built = c->n_tokens;
         ra.hkv = hkv; ra.G = hq / hkv; ra.agg = cfg->agg; ra.k = cfg->k; ra.S = cfg->sinks;
         ra.W = cfg->window; ra.Y = Y; ra.nqc = nqc; ra.t_first = t0 + c0; ra.tau = w.tau;

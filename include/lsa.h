@@ -318,9 +318,9 @@ size_t lsa_select_noalloc_scratch_bytes(void);
 /* --------------------------------------------------- whole-layer prefill */
 
 /* Workspace bytes lsa_prefill needs (T tokens, queries processed in chunks
- * of `chunk` positions; chunk <= 0 means all of T; in flat mode a chunk
- * larger than the flat search's wave-aligned chunk is rounded down to a
- * multiple of it). */
+ * of `chunk` positions; chunk <= 0 means all of T; in flat mode the chunk
+ * becomes the nearest multiple of the flat search's wave-aligned chunk,
+ * at least one and at most T). */
 size_t lsa_prefill_workspace_bytes(const lsa_cfg* cfg, int64_t T, int32_t hq,
                                    int32_t hkv, int64_t chunk);
 
