@@ -72,13 +72,13 @@ def workload_cfg(args):
     return c
 
 
-def config_json(args, c, world):
+def config_json(args, c, world, chunk=None):
     return {
         "workload": args.workload, "T": c["T"], "hkv": c["hkv"], "hq": c["hq"], "d_head": c["d"],
         "d_latent": c["dl"], "k": c["k"], "sinks": c["sinks"], "window": c["window"],
         "search": "flat" if c["mode"] == 0 else f"tree(beam={c['beam']})",
         "query_score": "group-mean" if c["agg"] == 0 else "max-over-heads (native)",
-        "query_chunk": args.chunk, "parallelism": f"replicas x{world} (one layer per GPU)",
+        "query_chunk": chunk or args.chunk, "parallelism": f"replicas x{world} (one layer per GPU)",
         "l2": "no flush: per-step inputs (Q/K/V) are larger than L2",
         "inputs": "host-drawn (numpy PCG64)" if c["T"] <= 131072 else "device-drawn (torch Philox), same recipe",
     }
@@ -293,10 +293,11 @@ def run_lsa(args):
     cache = lsa.Cache(hkv, T, cfg, device=dev)
     tree = lsa.Tree(cache, device=dev) if cfg.mode == 1 else None
     O = torch.empty_like(Q)
-    chunk = min(args.chunk, T)
+    chunk = lsa.prefill_chunk(cfg, T, hq, hkv, args.chunk)
     row = cfg.row
     idx = torch.empty((chunk, hkv, row), dtype=torch.int32, device=dev)
     sws = torch.empty(lsa.select_workspace_bytes(cfg, chunk, hq, cache) or 1, dtype=torch.uint8, device=dev)
+    aws = torch.empty(lsa.select_attn_workspace_bytes(chunk, hq) or 1, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
     chunks = [(t0, min(chunk, T - t0)) for t0 in range(0, T, chunk)]
     def ev():
@@ -321,7 +322,7 @@ def run_lsa(args):
             if timed_attn:
                 sel_ev[ci][1].record(stream)
                 attn_ev[ci][0].record(stream)
-            lsa.sparse_attn(Q[t0:t0 + n], K, V, idx[:n], T, O=O[t0:t0 + n])
+            lsa.select_attn(Q[t0:t0 + n], K, V, idx[:n], t0, cfg, T, O=O[t0:t0 + n], ws=aws)
             if timed_attn:
                 attn_ev[ci][1].record(stream)
 
@@ -438,7 +439,7 @@ def run_lsa(args):
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": config_json(args, c, world), "clocks": clk, "e2e": e2e,
+            "config": config_json(args, c, world, chunk), "clocks": clk, "e2e": e2e,
             "gpu_launches": int(launches), "roofline": roofline, "cpu_baseline": cpu,
             "stages_ms_per_step": {"build": build_ms / args.steps, "select": sel_ms / args.steps,
                                    "attention": attn_ms / args.steps},

@@ -88,6 +88,11 @@ def lib():
                                          P(lsa_cfg), vp, vp]
         L.lsa_select_noalloc_scratch_bytes.restype = sz
         L.lsa_sparse_attn.argtypes = [vp, vp, vp, vp, i64, i32, i32, i32, i64, vp, vp]
+        L.lsa_select_attn_workspace_bytes.argtypes = [i64, i32]
+        L.lsa_select_attn_workspace_bytes.restype = sz
+        L.lsa_select_attn.argtypes = [vp, vp, vp, vp, i64, i64, i32, i32, i64, P(lsa_cfg), vp, vp, sz, vp]
+        L.lsa_prefill_chunk.argtypes = [P(lsa_cfg), i64, i32, i32, i64]
+        L.lsa_prefill_chunk.restype = i64
         L.lsa_decode_workspace_bytes.argtypes = [P(lsa_cfg), P(lsa_decode)]
         L.lsa_decode_workspace_bytes.restype = sz
         L.lsa_decode_load.argtypes = [P(lsa_decode), i32, i64, vp, P(lsa_cfg), vp, sz, vp]

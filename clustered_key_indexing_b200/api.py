@@ -187,6 +187,33 @@ def sparse_attn(Q, K, V, idx, T: int | None = None, O=None, stream=None) -> torc
     return O
 
 
+def select_attn_workspace_bytes(nq: int, hq: int) -> int:
+    return int(lib().lsa_select_attn_workspace_bytes(nq, hq))
+
+
+def select_attn(Q, K, V, idx, t0: int, cfg: Config, T: int | None = None, O=None, ws=None,
+                stream=None) -> torch.Tensor:
+    """lsa_select_attn: attention over lsa_select's index rows (window as a band)."""
+    _need_cuda(Q, K, V, idx)
+    nq, hq, d = Q.shape
+    hkv = K.shape[1]
+    if O is None:
+        O = torch.empty((nq, hq, d), dtype=torch.bfloat16, device=Q.device)
+    T = K.shape[0] if T is None else T
+    need = select_attn_workspace_bytes(nq, hq)
+    if ws is None:
+        ws = torch.empty(max(need, 1), dtype=torch.uint8, device=Q.device)
+    check(lib().lsa_select_attn(_ptr(Q), _ptr(K), _ptr(V), _ptr(idx), t0, nq, hq, hkv, T,
+                                ctypes.byref(cfg.c()), _ptr(O), _ptr(ws), ws.numel(), _stream(stream)),
+          "lsa_select_attn")
+    return O
+
+
+def prefill_chunk(cfg: Config, T: int, hq: int, hkv: int, chunk: int = 0) -> int:
+    """The query chunk lsa_prefill uses for a requested chunk (0: its own choice)."""
+    return int(lib().lsa_prefill_chunk(ctypes.byref(cfg.c()), T, hq, hkv, chunk))
+
+
 def prefill_workspace_bytes(cfg: Config, T: int, hq: int, hkv: int, chunk: int) -> int:
     return int(lib().lsa_prefill_workspace_bytes(ctypes.byref(cfg.c()), T, hq, hkv, chunk))
 

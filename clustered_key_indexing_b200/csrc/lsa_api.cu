@@ -54,7 +54,11 @@ lsa_status run_select(const uint16_t* Q, int64_t t0, int64_t nq, int32_t hq, con
                       uint16_t* Y_out, void* ws, size_t ws_bytes, cudaStream_t st);
 lsa_status launch_attn(const uint16_t* Q, const uint16_t* K, const uint16_t* V, const int32_t* idx,
                        int64_t nq, int32_t hq, int32_t hkv, int32_t n_idx, int64_t T, uint16_t* O,
-                       cudaStream_t st, int64_t kv_q_stride, int split);
+                       cudaStream_t st, int64_t kv_q_stride, int split, int32_t n_use, const float* Ow,
+                       const float* lse);
+lsa_status launch_band_attn(const uint16_t* Q, const uint16_t* K, const uint16_t* V, int64_t nq, int64_t t0,
+                            int64_t T, int32_t hq, int32_t hkv, int32_t S, int32_t W, float* Ow, float* lse,
+                            cudaStream_t st);
 
 static lsa_status check_cfg(const lsa_cfg* c) {
     if (!c) return set_error(LSA_EINVAL, "cfg is NULL");
@@ -266,13 +270,60 @@ lsa_status lsa_sparse_attn(const uint16_t* Q, const uint16_t* K, const uint16_t*
     if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O))
         return set_error(LSA_EINVAL, "lsa_sparse_attn: Q, K, V, O must be 16-byte aligned");
     if (T > (int64_t)INT32_MAX) return set_error(LSA_EUNSUPPORTED, "lsa_sparse_attn: T beyond 2^31");
-    return launch_attn(Q, K, V, idx, nq, hq, hkv, n_idx, T, O, (cudaStream_t)stream);
+    return launch_attn(Q, K, V, idx, nq, hq, hkv, n_idx, T, O, (cudaStream_t)stream, 0, 1, -1, nullptr, nullptr);
 }
+
+size_t lsa_select_attn_workspace_bytes(int64_t nq, int32_t hq) {
+    if (nq <= 0 || hq <= 0) return 0;
+    return (((size_t)nq * hq * kD * 4 + 255) & ~(size_t)255) + (((size_t)nq * hq * 4 + 255) & ~(size_t)255);
+}
+
+lsa_status lsa_select_attn(const uint16_t* Q, const uint16_t* K, const uint16_t* V, const int32_t* idx, int64_t t0,
+                           int64_t nq, int32_t hq, int32_t hkv, int64_t T, const lsa_cfg* cfg, uint16_t* O, void* ws,
+                           size_t ws_bytes, void* stream) {
+    lsa_status s;
+    if ((s = check_cfg(cfg)) != LSA_OK) return s;
+    if ((s = check_heads(hq, hkv)) != LSA_OK) return s;
+    if (!Q || !K || !V || !idx || !O || (!ws && nq > 0)) return set_error(LSA_EINVAL, "lsa_select_attn: NULL pointer");
+    if (nq < 0 || t0 < 0 || T < 0) return set_error(LSA_EINVAL, "lsa_select_attn: negative size");
+    if (t0 + nq > T) return set_error(LSA_EINVAL, "lsa_select_attn: query positions beyond T");
+    if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(ws))
+        return set_error(LSA_EINVAL, "lsa_select_attn: Q, K, V, O, ws must be 16-byte aligned");
+    if (T > (int64_t)INT32_MAX) return set_error(LSA_EUNSUPPORTED, "lsa_select_attn: T beyond 2^31");
+    if (nq == 0) return LSA_OK;
+    const size_t need = lsa_select_attn_workspace_bytes(nq, hq);
+    if (ws_bytes < need) return set_error(LSA_ENOSPACE, "lsa_select_attn: workspace %zu < %zu bytes", ws_bytes, need);
+    float* Ow = (float*)ws;
+    float* lse = (float*)((char*)ws + (((size_t)nq * hq * kD * 4 + 255) & ~(size_t)255));
+    const cudaStream_t st = (cudaStream_t)stream;
+    const int32_t row = cfg->sinks + cfg->k + cfg->window;
+    // the rows' window part [S + k, S + k + W) is the contiguous range
+    // max(S, t - W + 1) .. t: attend to it as a band, then gather the sinks
+    // and long-range entries and merge the two softmax states
+    if ((s = launch_band_attn(Q, K, V, nq, t0, T, hq, hkv, cfg->sinks, cfg->window, Ow, lse, st)) != LSA_OK) return s;
+    return launch_attn(Q, K, V, idx, nq, hq, hkv, row, T, O, st, 0, 1, cfg->sinks + cfg->k, Ow, lse);
+}
+
 
 // Query positions per prefill chunk: `chunk` (all of T if <= 0 or larger);
 // in flat mode the nearest multiple of the flat search's own wave-aligned
 // chunk (at least one, at most T), so every select call but the last fills
 // whole waves.
+// Prefill workspace ahead of the select workspace: the chunk's index rows,
+// then the sliding-window partial output (fp32) and its log-sum-exp.
+struct PrefillWs {
+    size_t idx_bytes, ow_bytes, lse_bytes, total;
+};
+static PrefillWs prefill_ws_layout(const lsa_cfg* cfg, int64_t chunk, int32_t hq, int32_t hkv) {
+    auto al = [](size_t x) { return (x + 255) & ~(size_t)255; };
+    PrefillWs w;
+    w.idx_bytes = al((size_t)chunk * hkv * (cfg->sinks + cfg->k + cfg->window) * 4);
+    w.ow_bytes = al((size_t)chunk * hq * kD * 4);
+    w.lse_bytes = al((size_t)chunk * hq * 4);
+    w.total = w.idx_bytes + w.ow_bytes + w.lse_bytes;
+    return w;
+}
+
 static int64_t prefill_chunk(const lsa_cfg* cfg, int64_t T, int32_t hq, int32_t hkv, int64_t chunk) {
     if (chunk <= 0 || chunk > T) chunk = T;
     if (cfg->mode == 0 && hkv > 0 && hq > 0 && chunk < T) {
@@ -284,13 +335,17 @@ static int64_t prefill_chunk(const lsa_cfg* cfg, int64_t T, int32_t hq, int32_t 
     return chunk;
 }
 
+int64_t lsa_prefill_chunk(const lsa_cfg* cfg, int64_t T, int32_t hq, int32_t hkv, int64_t chunk) {
+    if (check_cfg(cfg) != LSA_OK || T <= 0 || hq <= 0 || hkv <= 0) return -1;
+    return prefill_chunk(cfg, T, hq, hkv, chunk);
+}
+
 size_t lsa_prefill_workspace_bytes(const lsa_cfg* cfg, int64_t T, int32_t hq, int32_t hkv, int64_t chunk) {
     if (check_cfg(cfg) != LSA_OK || T <= 0 || hkv <= 0) return 0;
     chunk = prefill_chunk(cfg, T, hq, hkv, chunk);
     const int64_t NU = ceil_div<int64_t>(T, kPool);
     const int64_t NB = ceil_div<int64_t>(NU, kUnitsPerBlock) * kBucketsPerBlock;
-    const size_t idx_bytes = ((size_t)chunk * hkv * (cfg->sinks + cfg->k + cfg->window) * 4 + 255) & ~(size_t)255;
-    return idx_bytes + select_ws_bytes(cfg, chunk, hq, hkv, NB);
+    return prefill_ws_layout(cfg, chunk, hq, hkv).total + select_ws_bytes(cfg, chunk, hq, hkv, NB);
 }
 
 lsa_status lsa_prefill(const uint16_t* Q, const uint16_t* K, const uint16_t* V, int64_t T, int32_t hq,
@@ -306,17 +361,18 @@ lsa_status lsa_prefill(const uint16_t* Q, const uint16_t* K, const uint16_t* V, 
     if (ws_bytes < need) return set_error(LSA_ENOSPACE, "lsa_prefill: workspace %zu < %zu bytes", ws_bytes, need);
     if ((s = lsa_build_buckets(K, T, hkv, W_k, cfg, cache, stream)) != LSA_OK) return s;
     if (cfg->mode == 1 && (s = lsa_build_tree(cache, cfg, tree, stream)) != LSA_OK) return s;
-    const int32_t row = cfg->sinks + cfg->k + cfg->window;
-    const size_t idx_bytes = ((size_t)chunk * hkv * row * 4 + 255) & ~(size_t)255;
+    const PrefillWs pw = prefill_ws_layout(cfg, chunk, hq, hkv);
     int32_t* idx = (int32_t*)ws;
-    void* sws = (char*)ws + idx_bytes;
-    const size_t sws_bytes = ws_bytes - idx_bytes;
+    void* aws = (char*)ws + pw.idx_bytes;
+    void* sws = (char*)ws + pw.total;
+    const size_t sws_bytes = ws_bytes - pw.total;
     for (int64_t t0 = 0; t0 < T; t0 += chunk) {
         const int64_t n = (T - t0) < chunk ? (T - t0) : chunk;
-        if ((s = lsa_select(Q + t0 * hq * kD, t0, n, hq, W_q, cache, tree, cfg, idx, nullptr, sws, sws_bytes,
-                            stream)) != LSA_OK)
+        const uint16_t* Qc = Q + t0 * hq * kD;
+        if ((s = lsa_select(Qc, t0, n, hq, W_q, cache, tree, cfg, idx, nullptr, sws, sws_bytes, stream)) != LSA_OK)
             return s;
-        if ((s = lsa_sparse_attn(Q + t0 * hq * kD, K, V, idx, n, hq, hkv, row, T, O + t0 * hq * kD, stream)) != LSA_OK)
+        if ((s = lsa_select_attn(Qc, K, V, idx, t0, n, hq, hkv, T, cfg, O + t0 * hq * kD, aws,
+                                 pw.ow_bytes + pw.lse_bytes, stream)) != LSA_OK)
             return s;
     }
     return LSA_OK;

@@ -27,7 +27,7 @@ constexpr int kStages = 2;
 constexpr int kTileKeys = 16;
 constexpr int kTileBytes = kTileKeys * kD * 2;           // 4 KB per tensor
 constexpr int kStageBytes = 2 * kTileBytes;              // K + V
-constexpr int kWarpBytes = kStages * kStageBytes;        // 24 KB
+constexpr int kWarpBytes = kStages * kStageBytes;        // per-warp ring
 
 struct AttnArgs {
     const uint16_t* Q;
@@ -36,6 +36,9 @@ struct AttnArgs {
     const int32_t* idx;
     int64_t nq;
     int32_t hq, hkv, n_idx;
+    int32_t n_use;        // entries of each list to attend to (<= n_idx, the list stride)
+    const float* Ow;      // optional [nq, hq, 128] partial output over other keys (normalised) ...
+    const float* lse;     // ... and its log2-domain log-sum-exp, merged into the result
     int64_t T;            // index entries must be < T
     int64_t kv_q_stride;  // token rows of K/V per query row (decode: each request's capacity); 0 = shared
     uint16_t* O;
@@ -74,7 +77,7 @@ __global__ void __launch_bounds__(32 * (SPLIT == 1 ? kAttnWarps : SPLIT)) attn_k
         }
     }
 
-    const int ntot = (a.n_idx + kTileKeys - 1) / kTileKeys;
+    const int ntot = (a.n_use + kTileKeys - 1) / kTileKeys;
     const int tbeg = SPLIT == 1 ? 0 : (int)(((int64_t)ntot * wid) / SPLIT);
     const int ntiles = SPLIT == 1 ? ntot : (int)(((int64_t)ntot * (wid + 1)) / SPLIT);  // tile end
     const int64_t kv_stride = (int64_t)a.hkv * kD;
@@ -84,7 +87,7 @@ __global__ void __launch_bounds__(32 * (SPLIT == 1 ? kAttnWarps : SPLIT)) attn_k
     // positions of one 16-key tile: lanes l and l+16 both hold entry l
     auto tile_pos = [&](int tile) -> int {
         const int e = tile * kTileKeys + (lane & 15);
-        int p = (tile < ntiles && e < a.n_idx) ? __ldg(list + e) : -1;
+        int p = (tile < ntiles && e < a.n_use) ? __ldg(list + e) : -1;
         if (p >= a.T) {
             raise_device_error(kErrIndexRange);
             p = -1;
@@ -114,16 +117,19 @@ __global__ void __launch_bounds__(32 * (SPLIT == 1 ? kAttnWarps : SPLIT)) attn_k
     float m_run[2] = {-CUDART_INF_F, -CUDART_INF_F};
     float l_run[2] = {0.f, 0.f};
 
-    static_assert(kStages == 2, "the position ring below holds 2 tiles");
-    // p0: tile i (being computed), p1: tile i+1 (next to issue)
-    int p0 = tile_pos(tbeg);
-    issue(tbeg, tbeg % kStages, p0);
-    int p1 = tile_pos(tbeg + 1);
+    // pr[j]: positions of tile i + j (tiles i .. i + kStages - 2 are in
+    // flight, tile i + kStages - 1 is issued at the top of iteration i)
+    int pr[kStages];
+#pragma unroll
+    for (int j = 0; j < kStages; ++j) {
+        pr[j] = tile_pos(tbeg + j);
+        if (j < kStages - 1) issue(tbeg + j, (tbeg + j) % kStages, pr[j]);
+    }
 
     for (int i = tbeg; i < ntiles; ++i) {
-        issue(i + 1, (i + 1) % kStages, p1);
-        const int p2 = tile_pos(i + 2);  // consumed one iteration later
-        const unsigned vmask = __ballot_sync(0xffffffffu, p0 >= 0) & 0xFFFFu;
+        issue(i + kStages - 1, (i + kStages - 1) % kStages, pr[kStages - 1]);
+        const int pnext = tile_pos(i + kStages);  // consumed kStages - 1 iterations later
+        const unsigned vmask = __ballot_sync(0xffffffffu, pr[0] >= 0) & 0xFFFFu;
         cp_async_wait<kStages - 1>();
         __syncwarp();
         if (vmask != 0) {
@@ -189,8 +195,9 @@ __global__ void __launch_bounds__(32 * (SPLIT == 1 ? kAttnWarps : SPLIT)) attn_k
             }
         }
         __syncwarp();
-        p0 = p1;
-        p1 = p2;
+#pragma unroll
+        for (int j = 0; j + 1 < kStages; ++j) pr[j] = pr[j + 1];
+        pr[kStages - 1] = pnext;
     }
     cp_async_wait<0>();
     __syncwarp();
@@ -200,7 +207,40 @@ __global__ void __launch_bounds__(32 * (SPLIT == 1 ? kAttnWarps : SPLIT)) attn_k
         l_run[0] += __shfl_xor_sync(0xffffffffu, l_run[0], off);
         l_run[1] += __shfl_xor_sync(0xffffffffu, l_run[1], off);
     }
-    if constexpr (SPLIT == 1) {
+    if (SPLIT == 1 && a.Ow != nullptr) {
+        // merge with the partial (O_w, lse) of the other keys: stage the
+        // unnormalised O [8 heads][128] fp32 and (m, l) per head, then each
+        // lane combines (head, dim) elements with coalesced reads and writes
+        float* op = reinterpret_cast<float*>(wbuf);
+        float* ml = op + 8 * kD;  // [8][2]
+#pragma unroll
+        for (int mt = 0; mt < 8; ++mt) {
+            const int d0 = mt * 16 + gq;
+            op[(2 * tq) * kD + d0] = o[mt][0];
+            op[(2 * tq + 1) * kD + d0] = o[mt][1];
+            op[(2 * tq) * kD + d0 + 8] = o[mt][2];
+            op[(2 * tq + 1) * kD + d0 + 8] = o[mt][3];
+        }
+        if (gq == 0) {
+            ml[4 * tq] = m_run[0]; ml[4 * tq + 1] = l_run[0];
+            ml[4 * tq + 2] = m_run[1]; ml[4 * tq + 3] = l_run[1];
+        }
+        __syncwarp();
+        const int64_t r0 = q * a.hq + g * G;
+        for (int e = lane; e < G * kD; e += 32) {
+            const int hh = e / kD, d = e % kD;
+            const float mb = ml[2 * hh], lb = ml[2 * hh + 1];
+            const float la = a.lse[r0 + hh];
+            const float M = fmaxf(mb, la);
+            float out = 0.f;
+            if (M > -CUDART_INF_F) {
+                const float wb = exp2f(mb - M), wa = exp2f(la - M);
+                out = (op[hh * kD + d] * wb + a.Ow[(r0 + hh) * kD + d] * wa) / (lb * wb + wa);
+            }
+            const __nv_bfloat16 ob = __float2bfloat16_rn(out);
+            a.O[(r0 + hh) * kD + d] = *reinterpret_cast<const uint16_t*>(&ob);
+        }
+    } else if constexpr (SPLIT == 1) {
         // normalise and stage O (heads x dims, bf16) for a coalesced store
         const float inv0 = l_run[0] > 0.f ? 1.f / l_run[0] : 0.f;
         const float inv1 = l_run[1] > 0.f ? 1.f / l_run[1] : 0.f;
@@ -258,12 +298,18 @@ __global__ void __launch_bounds__(32 * (SPLIT == 1 ? kAttnWarps : SPLIT)) attn_k
     }
 }
 
+// n_use < 0: every entry of each list; Ow / lse: optional partial state of
+// other keys to merge (prefill: the sliding window, from the band kernel).
 lsa_status launch_attn(const uint16_t* Q, const uint16_t* K, const uint16_t* V, const int32_t* idx,
                        int64_t nq, int32_t hq, int32_t hkv, int32_t n_idx, int64_t T, uint16_t* O,
-                       cudaStream_t st, int64_t kv_q_stride = 0, int split = 1) {
+                       cudaStream_t st, int64_t kv_q_stride = 0, int split = 1, int32_t n_use = -1,
+                       const float* Ow = nullptr, const float* lse = nullptr) {
     if (nq <= 0) return LSA_OK;
     AttnArgs a{};
     a.Q = Q; a.K = K; a.V = V; a.idx = idx; a.nq = nq; a.hq = hq; a.hkv = hkv; a.n_idx = n_idx;
+    a.n_use = n_use < 0 || n_use > n_idx ? n_idx : n_use;
+    a.Ow = split == 1 ? Ow : nullptr;
+    a.lse = split == 1 ? lse : nullptr;
     a.T = T; a.O = O; a.kv_q_stride = kv_q_stride;
     a.scale_log2 = 1.4426950408889634f / sqrtf((float)kD);
     const int64_t rows = nq * hkv;

@@ -43,7 +43,8 @@ lsa_status launch_clear_slots(const lsa_cache* c, int64_t b0, int64_t b1, cudaSt
 lsa_status launch_tree_update(const lsa_cache* c, lsa_tree* t, int64_t b0, int64_t b1, cudaStream_t st);
 lsa_status launch_attn(const uint16_t* Q, const uint16_t* K, const uint16_t* V, const int32_t* idx,
                        int64_t nq, int32_t hq, int32_t hkv, int32_t n_idx, int64_t T, uint16_t* O,
-                       cudaStream_t st, int64_t kv_q_stride, int split);
+                       cudaStream_t st, int64_t kv_q_stride, int split, int32_t n_use, const float* Ow,
+                       const float* lse);
 
 // ------------------------------------------------------------- key latent
 
@@ -661,7 +662,7 @@ lsa_status lsa_decode_step(lsa_decode* d, const uint16_t* q, const uint16_t* k, 
     }
     // (4) attention: each request reads its own K/V rows
     return launch_attn(q, d->K, d->V, idx, d->batch, d->hq, d->hkv, (int32_t)decode_row_len(cfg), d->cap,
-                       o, st, d->cap, 8);
+                       o, st, d->cap, 8, -1, nullptr, nullptr);
 }
 
 }  // extern "C"

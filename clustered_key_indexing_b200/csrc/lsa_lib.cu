@@ -3,6 +3,7 @@
 #include "lsa_build.cu"
 #include "lsa_select.cu"
 #include "lsa_attn.cu"
+#include "lsa_band.cu"
 #include "lsa_api.cu"
 #include "lsa_decode.cu"
 #include "lsa_noalloc.cu"

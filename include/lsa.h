@@ -226,6 +226,28 @@ lsa_status lsa_sparse_attn(const uint16_t* Q, const uint16_t* K,
                            int32_t hq, int32_t hkv, int32_t n_idx, int64_t T,
                            uint16_t* O, void* stream);
 
+/* Workspace bytes lsa_select_attn needs for nq query positions (the
+ * window's fp32 partial output and its log-sum-exp). */
+size_t lsa_select_attn_workspace_bytes(int64_t nq, int32_t hq);
+
+/*
+ * lsa_select_attn -- lsa_sparse_attn for index rows in lsa_select's layout
+ * (same cfg): the same result over the same entries, computed in two parts
+ * [tutorial section 二: sinks and the local window are always attended].
+ * The window part [S + k, S + k + W) of a row is by construction the
+ * contiguous range max(S, t - W + 1) .. t, so it is not read: queries
+ * t0 .. t0 + nq - 1 attend to their windows as a band (consecutive queries
+ * share K/V tiles), then the sinks and long-range entries [0, S + k) are
+ * gathered and the two softmax states merged.  Q [nq, hq, d_head], K/V
+ * [T, hkv, d_head], O [nq, hq, d_head] bf16; idx [nq, hkv, S + k + W];
+ * ws (16-byte aligned): at least lsa_select_attn_workspace_bytes(nq, hq).
+ */
+lsa_status lsa_select_attn(const uint16_t* Q, const uint16_t* K,
+                           const uint16_t* V, const int32_t* idx, int64_t t0,
+                           int64_t nq, int32_t hq, int32_t hkv, int64_t T,
+                           const lsa_cfg* cfg, uint16_t* O, void* ws,
+                           size_t ws_bytes, void* stream);
+
 /* ------------------------------------------------------------ decode */
 
 /*
@@ -317,6 +339,11 @@ size_t lsa_select_noalloc_scratch_bytes(void);
 
 /* --------------------------------------------------- whole-layer prefill */
 
+/* The query chunk lsa_prefill uses for a requested `chunk` (see below);
+ * -1 on invalid arguments. */
+int64_t lsa_prefill_chunk(const lsa_cfg* cfg, int64_t T, int32_t hq,
+                          int32_t hkv, int64_t chunk);
+
 /* Workspace bytes lsa_prefill needs (T tokens, queries processed in chunks
  * of `chunk` positions; chunk <= 0 means all of T; in flat mode the chunk
  * becomes the nearest multiple of the flat search's wave-aligned chunk,
@@ -327,7 +354,7 @@ size_t lsa_prefill_workspace_bytes(const lsa_cfg* cfg, int64_t T, int32_t hq,
 /*
  * lsa_prefill -- one LSA attention layer over a prompt of T tokens:
  * lsa_build_buckets, lsa_build_tree (tree mode), then per chunk of `chunk`
- * query positions lsa_select + lsa_sparse_attn.  Q [T, hq, d], K/V
+ * query positions lsa_select + lsa_select_attn.  Q [T, hq, d], K/V
  * [T, hkv, d], O [T, hq, d] bf16; cache/tree as for the calls above.
  */
 lsa_status lsa_prefill(const uint16_t* Q, const uint16_t* K, const uint16_t* V,

@@ -193,6 +193,35 @@ def test_sparse_attn_matches_oracle(lsa):
     assert np.all(O[3, 8:12].float().cpu().numpy() == 0)
 
 
+@pytest.mark.parametrize("G,t0,nq,W", [(1, 1500, 700, 300), (2, 0, 333, 300), (4, 900, 515, 1),
+                                        (8, 0, 300, 5000)])
+def test_select_attn_matches_gather_and_oracle(lsa, G, t0, nq, W):
+    """lsa_select_attn (window as a band + gathered sinks / long-range
+    entries, merged) against lsa_sparse_attn over the same index rows and
+    against the oracle attention: every GQA group size, ragged query ranges,
+    windows of 1 and longer than the prompt, queries from position 0."""
+    T, hkv = 3000, 2
+    inp = synth.layer_inputs("prefill-128k", T=T)
+    Q = np.ascontiguousarray(inp["Q"][:, :hkv * G])
+    K = np.ascontiguousarray(inp["K"][:, :hkv])
+    V = np.ascontiguousarray(inp["V"][:, :hkv])
+    cfg = lsa.Config(k=256, sinks=4, window=W)
+    dK, dV = to_dev_bf16(K), to_dev_bf16(V)
+    cache = lsa.Cache(hkv, T, cfg)
+    lsa.build_buckets(dK, to_dev(inp["Wk"]), cfg, cache)
+    dQ = to_dev_bf16(Q[t0:t0 + nq])
+    idx = lsa.select(dQ, t0, to_dev(inp["Wq"]), cache, cfg)
+    O = lsa.select_attn(dQ, dK, dV, idx, t0, cfg, T)
+    Og = lsa.sparse_attn(dQ, dK, dV, idx, T)
+    torch.cuda.synchronize()
+    lsa.check_device_error()
+    d = (O.float() - Og.float()).abs()
+    assert d.max().item() <= ATOL_MAX and d.mean().item() <= ATOL_MEAN, (d.max().item(), d.mean().item())
+    ref = oracle.attention(Q[t0:t0 + nq], K, V, idx.cpu().numpy())
+    mx, mean = _attn_err(O, ref)
+    assert mx <= ATOL_MAX and mean <= ATOL_MEAN, (mx, mean)
+
+
 def test_prefill_end_to_end_4k(lsa):
     """The whole layer (lsa_prefill) against the oracle layer."""
     cfg = lsa.Config(k=512, sinks=4, window=256)
