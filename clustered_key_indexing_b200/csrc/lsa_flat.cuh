@@ -542,27 +542,30 @@ __device__ __noinline__ int weight_packed(int64_t b, int32_t pk, int64_t lim, in
 }
 
 // First `tk` keys of bucket b in [S, lim], ascending (member units are
-// packed in ascending order).  Fast path: a bucket taken whole that lies
-// inside [S, lim] with full units writes 4 consecutive positions per unit.
-__device__ __noinline__ void emit_keys(int64_t b, int32_t pk, int tk, int64_t lim, int32_t S, int64_t T_built,
-                                      int32_t* out) {
+// packed in ascending order), written to out[o ..].  Fast path: a bucket
+// taken whole whose units are full and >= S writes 4 consecutive positions
+// per unit, as one 16-byte store where out + o is 16-byte aligned.
+__device__ __forceinline__ void emit_keys(int64_t b, int32_t pk, int tk, int64_t lim, int32_t S, int64_t T_built,
+                                          int32_t* out, int o) {
     const int64_t ubase = (b / kBucketsPerBlock) * kUnitsPerBlock;
     const int cnt = (pk >> 28) & 7;
     const int64_t j0 = ubase + (pk & 127);
     if (tk == cnt * kPool && j0 * kPool >= S) {
-        int o = 0;
+        const bool al = ((((uintptr_t)(out + o)) & 15u) == 0u);
         for (int i = 0; i < cnt; ++i) {
             const int32_t p = (int32_t)((ubase + ((pk >> (7 * i)) & 127)) * kPool);
-            out[o] = p; out[o + 1] = p + 1; out[o + 2] = p + 2; out[o + 3] = p + 3;
-            o += 4;
+            if (al) {
+                reinterpret_cast<int4*>(out + o)[i] = make_int4(p, p + 1, p + 2, p + 3);
+            } else {
+                out[o + 4 * i] = p; out[o + 4 * i + 1] = p + 1; out[o + 4 * i + 2] = p + 2; out[o + 4 * i + 3] = p + 3;
+            }
         }
         return;
     }
-    int o = 0;
-    for (int i = 0; i < cnt && o < tk; ++i) {
+    for (int i = 0; i < cnt && tk > 0; ++i) {
         const int64_t j = ubase + ((pk >> (7 * i)) & 127);
-        for (int64_t p = j * kPool; p < j * kPool + kPool && p < T_built && o < tk; ++p)
-            if (p >= S && p <= lim) out[o++] = (int32_t)p;
+        for (int64_t p = j * kPool; p < j * kPool + kPool && p < T_built && tk > 0; ++p)
+            if (p >= S && p <= lim) { out[o++] = (int32_t)p; --tk; }
     }
 }
 
@@ -653,11 +656,21 @@ __global__ void __launch_bounds__(32 * kResWarps, 3) flat_resolve_kernel(Resolve
     const int64_t lim = t - a.W;
     int32_t* out = a.idx + row * (int64_t)(a.S + a.k + a.W);
 
-    // sinks and window
+    // sinks and window (16-byte stores when the row layout keeps them aligned)
     for (int i = lane; i < a.S; i += 32) out[i] = (i <= t) ? i : -1;
     const int64_t w0 = max((int64_t)a.S, t - a.W + 1);
-    const int64_t nw = t >= a.S ? t - w0 + 1 : 0;
-    for (int i = lane; i < a.W; i += 32) out[a.S + a.k + i] = i < nw ? (int32_t)(w0 + i) : -1;
+    const int nw = t >= a.S ? (int)(t - w0 + 1) : 0;
+    int32_t* wout = out + a.S + a.k;
+    if ((((uintptr_t)wout) & 15u) == 0u && (a.W & 3) == 0) {
+        for (int i4 = lane; i4 < a.W / 4; i4 += 32) {
+            const int i = 4 * i4;
+            reinterpret_cast<int4*>(wout)[i4] =
+                make_int4(i < nw ? (int)w0 + i : -1, i + 1 < nw ? (int)w0 + i + 1 : -1,
+                          i + 2 < nw ? (int)w0 + i + 2 : -1, i + 3 < nw ? (int)w0 + i + 3 : -1);
+        }
+    } else {
+        for (int i = lane; i < a.W; i += 32) wout[i] = i < nw ? (int32_t)(w0 + i) : -1;
+    }
     if (lim < a.S) {
         for (int i = lane; i < a.k; i += 32) out[a.S + i] = -1;
         return;
@@ -674,26 +687,37 @@ __global__ void __launch_bounds__(32 * kResWarps, 3) flat_resolve_kernel(Resolve
     const int64_t hb0 = (int64_t)h * a.cap_buckets;
     const int4* mrow = a.meta + (int64_t)h * a.NB;
     const int2* crow = a.cand + row * kCandCap;
+    // (1) the candidate list into shared memory, (2) every candidate's
+    // record gathered with the loads of a lane in flight together, its key
+    // count (0: not eligible) kept, (3) in-place compaction of the eligible
+    // ones (a chunk's reads precede its writes, which land at or below it)
+#pragma unroll 4
+    for (int i = lane; i < n; i += 32) sw.cs[i] = crow[i];
+    __syncwarp();
+#pragma unroll 4
+    for (int i = lane; i < n; i += 32) {
+        const int col = sw.cs[i].x;
+        const int4 md = __ldg(mrow + col);
+        int wgt = 0;
+        if ((int64_t)md.x <= lim) wgt = (int64_t)md.y <= lim ? md.z : weight_packed(col, md.w, lim, a.S, a.T_built);
+        sw.w[i] = (uint8_t)wgt;
+    }
+    __syncwarp();
     int m = 0;
     long long wtot = 0;
     float smin = CUDART_INF_F, smax = -CUDART_INF_F;
     for (int base = 0; base < n; base += 32) {
         const int i = base + lane;
-        bool el = false;
-        int2 cv = make_int2(0, 0);
-        int wgt = 0;
-        if (i < n) {
-            cv = crow[i];
-            const int4 md = __ldg(mrow + cv.x);
-            el = (int64_t)md.x <= lim;
-            wgt = (int64_t)md.y <= lim ? md.z : weight_packed(cv.x, md.w, lim, a.S, a.T_built);
-        }
+        const int2 cv = i < n ? sw.cs[i] : make_int2(0, 0);
+        const int wgt = i < n ? sw.w[i] : 0;
+        const bool el = wgt > 0;
         if (el) {
             wtot += wgt;
             smin = fminf(smin, __int_as_float(cv.y));
             smax = fmaxf(smax, __int_as_float(cv.y));
         }
         const unsigned bal = __ballot_sync(0xffffffffu, el);
+        __syncwarp();
         if (el) {
             const int pos = m + __popc(bal & ((1u << lane) - 1u));
             sw.cs[pos] = cv;
@@ -831,7 +855,7 @@ __global__ void __launch_bounds__(32 * kResWarps, 3) flat_resolve_kernel(Resolve
         }
         if (tk > 0) {
             const int col = sw.cs[i].x;
-            emit_keys(col, __ldg(&mrow[col].w), tk, lim, a.S, a.T_built, out + a.S + run + incl - tk);
+            emit_keys(col, __ldg(&mrow[col].w), tk, lim, a.S, a.T_built, out, a.S + run + incl - tk);
         }
         run += __shfl_sync(0xffffffffu, incl, 31);
     }
