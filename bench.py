@@ -40,8 +40,18 @@ UNIT = "tokens/s"
 # DRAM bytes per (query, kv-head) of attn_kernel from the ncu capture in
 # profiles/attn_kernel_prefill-128k.md; reported as `traffic` only while the
 # kernel source is the one that capture measured.
-ATTN_TRAFFIC = {"sha256_prefix": "5fead07e225b0b47", "bytes_per_query_kvhead": 40295.4,
-                "source": "clustered_key_indexing_b200/csrc/lsa_attn.cu", "workload": "prefill-128k"}
+# ncu DRAM bytes (read + write) per (query, kv-head) of the gather attention
+# kernel on a workload, valid while the kernel's source (the text from its
+# template header to its launcher, hashed) is unchanged since the capture.
+ATTN_TRAFFIC = {"kernel_sha256_prefix": "090d2ce0e8c877bc", "bytes_per_query_kvhead": 21345.1,
+                "workload": "prefill-128k"}
+
+
+def attn_kernel_hash():
+    import hashlib
+    src = open(os.path.join(ROOT, "clustered_key_indexing_b200/csrc/lsa_attn.cu")).read()
+    a, b = src.find("template <int SPLIT>"), src.find("lsa_status launch_attn(")
+    return hashlib.sha256(src[a:b].encode()).hexdigest()[:16] if a >= 0 and b > a else None
 
 
 def parse():
@@ -326,19 +336,19 @@ def run_lsa(args):
             if timed_attn:
                 attn_ev[ci][1].record(stream)
 
-    # algorithmic bytes of the attention launches: every valid index entry
-    # gathers one K row and one V row (2 x 256 B); plus Q read and O write
+    # index entries per step: gathered (sinks + long range) and window
     step()
     torch.cuda.synchronize()
-    valid = 0
+    valid_g = valid_w = 0
     lsa.build_buckets(K, Wk, cfg, cache)
     if tree is not None:
         lsa.build_tree(cache, cfg, tree)
+    ng = c["sinks"] + c["k"]
     for t0, n in chunks:
         lsa.select(Q[t0:t0 + n], t0, Wq, cache, cfg, tree=tree, idx=idx[:n], ws=sws)
-        valid += int((idx[:n] >= 0).sum().item())
+        valid_g += int((idx[:n, :, :ng] >= 0).sum().item())
+        valid_w += int((idx[:n, :, ng:] >= 0).sum().item())
     lsa.check_device_error()
-    attn_bytes = valid * 2 * 256 + 2 * T * hq * 128 * 2
 
     for _ in range(args.warmup):
         step()
@@ -350,16 +360,25 @@ def run_lsa(args):
     lib().lsa_fallback_rows()  # reset the counter
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     torch.cuda.synchronize()
+    kt = lsa.KernelTimer()
     ev0.record(stream)
     attn_ms = sel_ms = build_ms = 0.0
-    for _ in range(args.steps):
-        step(timed_attn=True)
-        torch.cuda.synchronize()  # read this step's stage events
-        attn_ms += sum(a.elapsed_time(b) for a, b in attn_ev)
-        sel_ms += sum(a.elapsed_time(b) for a, b in sel_ev)
-        build_ms += build_ev[0].elapsed_time(build_ev[1])
-    ev1.record(stream)
-    torch.cuda.synchronize()
+    with kt:
+        for _ in range(args.steps):
+            step(timed_attn=True)
+            torch.cuda.synchronize()  # read this step's stage events
+            attn_ms += sum(a.elapsed_time(b) for a, b in attn_ev)
+            sel_ms += sum(a.elapsed_time(b) for a, b in sel_ev)
+            build_ms += build_ev[0].elapsed_time(build_ev[1])
+        ev1.record(stream)
+        torch.cuda.synchronize()
+    kernels = {}
+    for name in ("attn_kernel", "band_attn_kernel", "flat_cand_kernel", "flat_sample_kernel", "flat_resolve_kernel",
+                 "latent_kernel", "ward_kernel", "select_fallback_kernel", "tree_select_kernel"):
+        kms, kn = kt.get(name)
+        if kn:
+            kernels[name] = {"ms_per_step": kms / args.steps, "launches_per_step": kn / args.steps,
+                             "ms_per_launch": kms / kn}
     clk = clocks.stop()
     launches = lib().lsa_launch_count() - n0
     fallback_rows = int(lib().lsa_fallback_rows())
@@ -407,23 +426,56 @@ def run_lsa(args):
                "d2h_bytes_per_step": hO.numel() * 2}
 
     pk, src = peaks()
-    attn_ms_launch = attn_ms / (args.steps * len(chunks))
-    achieved = (attn_bytes / len(chunks)) / (attn_ms_launch / 1e3) / 1e9
-    traffic = None
-    try:
-        import hashlib
-        attn_src = open(os.path.join(ROOT, ATTN_TRAFFIC["source"]), "rb").read()
-        if (hashlib.sha256(attn_src).hexdigest()[:16] == ATTN_TRAFFIC["sha256_prefix"]
-                and args.workload == ATTN_TRAFFIC["workload"]):
-            traffic = ATTN_TRAFFIC["bytes_per_query_kvhead"] * chunk * hkv
-    except OSError:
-        pass
-    roofline = {"kernel": "attn_kernel", "bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"],
-                "unit": "GB/s", "frac": achieved / pk["hbm_gbs"], "traffic": traffic,
-                "traffic_note": "ncu DRAM bytes per launch, scaled from a 2048-position launch",
-                "peak_source": src, "attn_share_of_step": attn_ms / ms if ms > 0 else None,
-                "bytes_per_launch": attn_bytes / len(chunks)}
+    for kv in kernels.values():
+        kv["share_of_step"] = kv["ms_per_step"] / ms_step if ms_step > 0 else None
+    # algorithmic work per step of the kernels with a roofline:
+    #   attn_kernel: K and V rows of every gathered entry (2 x 256 B), its
+    #     index entries (4 B), Q read, O write, the window partial (fp32 O and
+    #     lse) read -- HBM-bound;
+    #   band_attn_kernel: 4 x 128 FLOP per (window entry, query head) -- mma.sync;
+    #   flat_cand_kernel / flat_sample_kernel: 2 x 64 FLOP per (row, scored
+    #     centroid), every eligible / every 8th centroid -- tensor cores.
+    G = hq // hkv
+    rows_per_q = hq if cfg.agg else hkv
+    NB = ((T + 3) // 4 + 127) // 128 * 64  # buckets per kv-head
+    tt = np.arange(T, dtype=np.int64)
+    lim = tt - c["window"]
+    ncol = np.where(lim >= 0, np.minimum(NB, 64 * (np.maximum(lim, 0) // 512 + 1)), 0)
+    work = {
+        "attn_kernel": ("hbm", valid_g * (2 * 256 + 4) + T * hq * (2 * 256 + 4 * 129)),
+        "band_attn_kernel": ("tensor", valid_w * G * 4 * 128),
+        "flat_cand_kernel": ("tensor", 2 * 64 * rows_per_q * int(ncol.sum())),
+        "flat_sample_kernel": ("tensor", 2 * 64 * rows_per_q * int(((ncol + 7) // 8).sum())),
+    }
 
+    def roof(name):
+        bound, w = work[name]
+        k = kernels.get(name)
+        if not k:
+            return None
+        per_launch = w / k["launches_per_step"]
+        sec = k["ms_per_launch"] / 1e3
+        if bound == "hbm":
+            ach, peak, unit = per_launch / sec / 1e9, pk["hbm_gbs"], "GB/s"
+        else:
+            ach, unit = per_launch / sec / 1e12, "TFLOP/s"
+            peak = pk.get("bf16_tflops_sustained", pk["bf16_tflops"])
+        r = {"kernel": name, "bound": bound, "achieved": ach, "peak": peak, "unit": unit, "frac": ach / peak,
+             "traffic": None, "peak_source": src + (" (sustained)" if bound == "tensor" else ""),
+             "work_per_launch": per_launch, "ms_per_launch": k["ms_per_launch"],
+             "share_of_step": k["share_of_step"]}
+        if name == "attn_kernel":
+            h = attn_kernel_hash()
+            if (h and h == ATTN_TRAFFIC["kernel_sha256_prefix"] and args.workload == ATTN_TRAFFIC["workload"]
+                    and ATTN_TRAFFIC["bytes_per_query_kvhead"]):
+                r["traffic"] = ATTN_TRAFFIC["bytes_per_query_kvhead"] * T * hkv / k["launches_per_step"]
+            r["note"] = ("gathered K/V rows are served mostly from L2 (one kv-head's K/V per wave), so the "
+                         "algorithmic bytes can exceed the HBM copy peak; traffic = ncu DRAM bytes")
+        return r
+
+    ranked = sorted((n for n in work if n in kernels), key=lambda n: -kernels[n]["ms_per_step"])
+    roofline = roof(ranked[0]) if ranked else None
+    roofline_scoring = roof("flat_cand_kernel")
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu:
         if not host_drawn:  # the oracle sample reads head 0's K/V and the query rows
@@ -440,7 +492,8 @@ def run_lsa(args):
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": config_json(args, c, world, chunk), "clocks": clk, "e2e": e2e,
-            "gpu_launches": int(launches), "roofline": roofline, "cpu_baseline": cpu,
+            "gpu_launches": int(launches), "roofline": roofline, "roofline_scoring": roofline_scoring,
+            "kernels": kernels, "cpu_baseline": cpu,
             "stages_ms_per_step": {"build": build_ms / args.steps, "select": sel_ms / args.steps,
                                    "attention": attn_ms / args.steps},
             "select_fallback_rows_per_step": fallback_rows / args.steps,

@@ -91,6 +91,7 @@ def lib():
         L.lsa_select_attn_workspace_bytes.argtypes = [i64, i32]
         L.lsa_select_attn_workspace_bytes.restype = sz
         L.lsa_select_attn.argtypes = [vp, vp, vp, vp, i64, i64, i32, i32, i64, P(lsa_cfg), vp, vp, sz, vp]
+        L.lsa_timing_get.argtypes = [ctypes.c_char_p, P(ctypes.c_double), P(i64)]
         L.lsa_prefill_chunk.argtypes = [P(lsa_cfg), i64, i32, i32, i64]
         L.lsa_prefill_chunk.restype = i64
         L.lsa_decode_workspace_bytes.argtypes = [P(lsa_cfg), P(lsa_decode)]

@@ -288,3 +288,22 @@ class Decode:
                                     ctypes.byref(self.cfg.c()), _ptr(o), _ptr(idx_out), _ptr(self.ws),
                                     self.ws.numel(), _stream(stream)), "lsa_decode_step")
         return o
+
+
+class KernelTimer:
+    """Context manager around lsa_timing_begin / lsa_timing_end; get(name)
+    returns (total ms, launches) of one kernel recorded inside it."""
+
+    def __enter__(self):
+        lib().lsa_timing_begin()
+        return self
+
+    def __exit__(self, *exc):
+        lib().lsa_timing_end()
+        return False
+
+    @staticmethod
+    def get(name: str):
+        ms, n = ctypes.c_double(0.0), ctypes.c_int64(0)
+        check(lib().lsa_timing_get(name.encode(), ctypes.byref(ms), ctypes.byref(n)), "lsa_timing_get")
+        return ms.value, n.value

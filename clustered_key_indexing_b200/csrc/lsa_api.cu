@@ -5,7 +5,9 @@
 #include <stdarg.h>
 
 #include <atomic>
+#include <mutex>
 #include <stdint.h>
+#include <vector>
 #include <stdio.h>
 #include <string.h>
 
@@ -30,6 +32,46 @@ lsa_status check_launch(const char* what) {
     const cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return set_error(LSA_ECUDA, "%s: %s", what, cudaGetErrorString(e));
     return LSA_OK;
+}
+
+// ---------------------------------------------------------- kernel timing
+
+struct TimerRec {
+    const char* name;
+    std::vector<cudaEvent_t> start, stop;
+    size_t used = 0;
+};
+static std::atomic<bool> g_timing{false};
+static std::mutex g_tmu;
+static std::vector<TimerRec> g_trec;
+
+KTime::KTime(const char* name, cudaStream_t s) : st(s) {
+    if (!g_timing.load(std::memory_order_relaxed)) return;
+    std::lock_guard<std::mutex> lk(g_tmu);
+    int r = -1;
+    for (size_t i = 0; i < g_trec.size(); ++i)
+        if (strcmp(g_trec[i].name, name) == 0) { r = (int)i; break; }
+    if (r < 0) {
+        g_trec.push_back(TimerRec{name, {}, {}, 0});
+        r = (int)g_trec.size() - 1;
+    }
+    TimerRec& t = g_trec[r];
+    if (t.used == t.start.size()) {
+        cudaEvent_t a, b;
+        if (cudaEventCreate(&a) != cudaSuccess) return;
+        if (cudaEventCreate(&b) != cudaSuccess) { cudaEventDestroy(a); return; }
+        t.start.push_back(a);
+        t.stop.push_back(b);
+    }
+    rec = r;
+    slot = (int)t.used++;
+    cudaEventRecord(t.start[slot], st);
+}
+
+KTime::~KTime() {
+    if (slot < 0) return;
+    std::lock_guard<std::mutex> lk(g_tmu);
+    cudaEventRecord(g_trec[rec].stop[slot], st);
 }
 
 int num_sms() {
@@ -118,6 +160,34 @@ extern "C" {
 const char* lsa_last_error(void) { return g_err; }
 
 int64_t lsa_launch_count(void) { return (int64_t)g_launches.load(std::memory_order_relaxed); }
+
+void lsa_timing_begin(void) {
+    std::lock_guard<std::mutex> lk(g_tmu);
+    for (auto& t : g_trec) t.used = 0;
+    g_timing.store(true, std::memory_order_relaxed);
+}
+
+void lsa_timing_end(void) { g_timing.store(false, std::memory_order_relaxed); }
+
+lsa_status lsa_timing_get(const char* name, double* total_ms, int64_t* launches) {
+    if (!name || !total_ms || !launches) return set_error(LSA_EINVAL, "lsa_timing_get: NULL pointer");
+    std::lock_guard<std::mutex> lk(g_tmu);
+    *total_ms = 0.0;
+    *launches = 0;
+    for (auto& t : g_trec) {
+        if (strcmp(t.name, name) != 0) continue;
+        for (size_t i = 0; i < t.used; ++i) {
+            if (cudaEventSynchronize(t.stop[i]) != cudaSuccess)
+                return set_error(LSA_ECUDA, "lsa_timing_get: event synchronize failed");
+            float ms = 0.f;
+            if (cudaEventElapsedTime(&ms, t.start[i], t.stop[i]) != cudaSuccess)
+                return set_error(LSA_ECUDA, "lsa_timing_get: elapsed time failed");
+            *total_ms += ms;
+        }
+        *launches = (int64_t)t.used;
+    }
+    return LSA_OK;
+}
 
 const char* lsa_version(void) { return "lsa-b200 0.1 (sm_100a)"; }
 

@@ -316,13 +316,19 @@ lsa_status launch_attn(const uint16_t* Q, const uint16_t* K, const uint16_t* V, 
     if (split == 1) {
         const size_t smem = (size_t)kAttnWarps * kWarpBytes;
         cudaFuncSetAttribute(attn_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        attn_kernel<1><<<(unsigned)ceil_div<int64_t>(rows, kAttnWarps), 32 * kAttnWarps, smem, st>>>(a);
+        {
+            KTime kt_("attn_kernel", st);
+            attn_kernel<1><<<(unsigned)ceil_div<int64_t>(rows, kAttnWarps), 32 * kAttnWarps, smem, st>>>(a);
+        }
         return check_launch("attn_kernel");
     }
     constexpr int kSplit = 8;
     const size_t smem = (size_t)kSplit * kWarpBytes;
     cudaFuncSetAttribute(attn_kernel<kSplit>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    attn_kernel<kSplit><<<(unsigned)rows, 32 * kSplit, smem, st>>>(a);
+    {
+        KTime kt_("attn_kernel_split", st);
+        attn_kernel<kSplit><<<(unsigned)rows, 32 * kSplit, smem, st>>>(a);
+    }
     return check_launch("attn_kernel(split)");
 }
 

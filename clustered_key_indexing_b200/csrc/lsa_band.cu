@@ -239,8 +239,11 @@ lsa_status launch_band_attn(const uint16_t* Q, const uint16_t* K, const uint16_t
     auto kern = G == 1 ? band_attn_kernel<1> : G == 2 ? band_attn_kernel<2> : G == 4 ? band_attn_kernel<4>
                                                                                      : band_attn_kernel<8>;
     cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kBandSmemBytes);
-    kern<<<dim3((unsigned)ceil_div<int64_t>(nq, kBandRows / G), (unsigned)hkv), 32 * kBandWarps, kBandSmemBytes,
-           st>>>(a);
+    {
+        KTime kt_("band_attn_kernel", st);
+        kern<<<dim3((unsigned)ceil_div<int64_t>(nq, kBandRows / G), (unsigned)hkv), 32 * kBandWarps, kBandSmemBytes,
+               st>>>(a);
+    }
     return check_launch("band_attn_kernel");
 }
 

@@ -182,7 +182,10 @@ static lsa_status launch_latent(const LatentArgs& a, cudaStream_t st) {
     int64_t grid = ceil_div<int64_t>(iters, kLatWarps);
     const int64_t cap = (int64_t)num_sms() * 4;
     if (grid > cap) grid = cap;
-    latent_kernel<MODE><<<(unsigned)grid, 32 * kLatWarps, smem, st>>>(a);
+    {
+        KTime kt_("latent_kernel", st);
+        latent_kernel<MODE><<<(unsigned)grid, 32 * kLatWarps, smem, st>>>(a);
+    }
     return check_launch("latent_kernel");
 }
 
@@ -526,7 +529,10 @@ lsa_status launch_ward_u(const lsa_cache* c, const double* U, int64_t U_stride, 
     const size_t smem = ward_smem();
     cudaFuncSetAttribute(ward_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     dim3 grid((unsigned)(blk1 - blk0), (unsigned)c->hkv);
-    ward_kernel<<<grid, 128, smem, st>>>(a);
+    {
+        KTime kt_("ward_kernel", st);
+        ward_kernel<<<grid, 128, smem, st>>>(a);
+    }
     return check_launch("ward_kernel");
 }
 
@@ -550,7 +556,10 @@ lsa_status launch_ward_jobs(const lsa_cache* c, const double* U_blk, int32_t hkv
     const size_t smem = ward_smem();
     cudaFuncSetAttribute(ward_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     dim3 grid((unsigned)n_jobs, (unsigned)hkv);
-    ward_kernel<<<grid, 128, smem, st>>>(a);
+    {
+        KTime kt_("ward_kernel", st);
+        ward_kernel<<<grid, 128, smem, st>>>(a);
+    }
     return check_launch("ward_kernel(decode)");
 }
 

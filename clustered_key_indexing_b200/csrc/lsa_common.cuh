@@ -94,4 +94,14 @@ namespace lsa {
 lsa_status set_error(lsa_status st, const char* fmt, ...);
 lsa_status check_launch(const char* what);
 int num_sms();
+
+// Kernel timing: while lsa_timing_begin() is in effect, the launch inside a
+// KTime's scope is bracketed by two CUDA events on its stream, filed under
+// `name` (read back with lsa_timing_get).  Otherwise it does nothing.
+struct KTime {
+    int rec = -1, slot = -1;
+    cudaStream_t st = nullptr;
+    KTime(const char* name, cudaStream_t s);
+    ~KTime();
+};
 }  // namespace lsa

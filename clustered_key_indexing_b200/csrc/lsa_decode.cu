@@ -609,7 +609,10 @@ lsa_status lsa_decode_step(lsa_decode* d, const uint16_t* q, const uint16_t* k, 
     ap.k = k; ap.v = v; ap.K = d->K; ap.V = d->V; ap.W = W_k; ap.U_blk = d->U_blk; ap.cap = d->cap;
     ap.hkv = d->hkv; ap.batch = d->batch;
     for (int r = 0; r < d->batch; ++r) ap.pos[r] = d->len[r];
-    decode_append_kernel<<<(unsigned)ceil_div<int64_t>(rows, 8), 256, 0, st>>>(ap);
+    {
+        KTime kt_("decode_append_kernel", st);
+        decode_append_kernel<<<(unsigned)ceil_div<int64_t>(rows, 8), 256, 0, st>>>(ap);
+    }
     if ((s = check_launch("decode_append_kernel")) != LSA_OK) return s;
 
     // (2) cluster every block this token completed
@@ -650,14 +653,20 @@ lsa_status lsa_decode_step(lsa_decode* d, const uint16_t* q, const uint16_t* k, 
         for (int r = 0; r < d->batch; ++r) sa.pos[r] = a.pos[r];
         dim3 grid((unsigned)ceil_div<int64_t>(d->cache.cap_buckets, kDecScoreCols), (unsigned)rows);
         const int ng = cfg->agg ? d->hq / d->hkv : 1;
-        if (ng == 1) decode_score_kernel<1><<<grid, 256, 0, st>>>(sa);
-        else if (ng == 2) decode_score_kernel<2><<<grid, 256, 0, st>>>(sa);
-        else if (ng == 4) decode_score_kernel<4><<<grid, 256, 0, st>>>(sa);
-        else decode_score_kernel<8><<<grid, 256, 0, st>>>(sa);
+        {
+            KTime kt_("decode_score_kernel", st);
+            if (ng == 1) decode_score_kernel<1><<<grid, 256, 0, st>>>(sa);
+            else if (ng == 2) decode_score_kernel<2><<<grid, 256, 0, st>>>(sa);
+            else if (ng == 4) decode_score_kernel<4><<<grid, 256, 0, st>>>(sa);
+            else decode_score_kernel<8><<<grid, 256, 0, st>>>(sa);
+        }
         if ((s = check_launch("decode_score_kernel")) != LSA_OK) return s;
         DecResolveArgs ra{};
         ra.s = a; ra.bin = w.bin; ra.wt = w.wt; ra.slot = w.slot; ra.ld = ld; ra.cap_buckets = d->cache.cap_buckets;
-        decode_resolve_kernel<<<(unsigned)rows, kSelThreads, 0, st>>>(ra);
+        {
+            KTime kt_("decode_resolve_kernel", st);
+            decode_resolve_kernel<<<(unsigned)rows, kSelThreads, 0, st>>>(ra);
+        }
         if ((s = check_launch("decode_resolve_kernel")) != LSA_OK) return s;
     }
     // (4) attention: each request reads its own K/V rows

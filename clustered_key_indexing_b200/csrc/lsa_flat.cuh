@@ -894,17 +894,26 @@ lsa_status launch_flat(const PassArgs& pa, const ResolveArgs& ra, const CUtensor
                                                                                     : flat_cand_kernel<8>;
     cudaFuncSetAttribute(ks, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmSmemBytes);
     cudaFuncSetAttribute(kc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kCdSmemBytes);
-    ks<<<dim3((unsigned)ceil_div<int64_t>(pa.nqc, kSmRows / G), (unsigned)pa.hkv), kSmThreads, kSmSmemBytes, st>>>(tmS,
-                                                                                                               pa);
+    {
+        KTime kt_("flat_sample_kernel", st);
+        ks<<<dim3((unsigned)ceil_div<int64_t>(pa.nqc, kSmRows / G), (unsigned)pa.hkv), kSmThreads, kSmSmemBytes, st>>>(tmS,
+                                                                                                                   pa);
+    }
     lsa_status s = check_launch("flat_sample_kernel");
     if (s != LSA_OK) return s;
-    kc<<<dim3((unsigned)ceil_div<int64_t>(pa.nqc, kCdRows / G), (unsigned)pa.hkv), kCdThreads, kCdSmemBytes, st>>>(tmF,
-                                                                                                               pa);
+    {
+        KTime kt_("flat_cand_kernel", st);
+        kc<<<dim3((unsigned)ceil_div<int64_t>(pa.nqc, kCdRows / G), (unsigned)pa.hkv), kCdThreads, kCdSmemBytes, st>>>(tmF,
+                                                                                                                   pa);
+    }
     if ((s = check_launch("flat_cand_kernel")) != LSA_OK) return s;
     const size_t smem_r = sizeof(ResWarp) * kResWarps;
     cudaFuncSetAttribute(flat_resolve_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_r);
     const int64_t rows = pa.nqc * pa.hkv;
-    flat_resolve_kernel<<<(unsigned)ceil_div<int64_t>(rows, kResWarps), 32 * kResWarps, smem_r, st>>>(ra);
+    {
+        KTime kt_("flat_resolve_kernel", st);
+        flat_resolve_kernel<<<(unsigned)ceil_div<int64_t>(rows, kResWarps), 32 * kResWarps, smem_r, st>>>(ra);
+    }
     return check_launch("flat_resolve_kernel");
 }
 

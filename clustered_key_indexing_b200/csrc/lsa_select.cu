@@ -628,7 +628,10 @@ lsa_status run_select(const uint16_t* Q, int64_t t0, int64_t nq, int32_t hq, con
         if (s != LSA_OK) return s;
         a.Y = Y; a.nqc = nqc; a.t_first = t0 + c0; a.idx = idx + c0 * hkv * row_len;
         if (cfg->mode == 1) {
-            tree_select_kernel<<<(unsigned)(nqc * hkv), kSelThreads, 0, st>>>(a);
+            {
+                KTime kt_("tree_select_kernel", st);
+                tree_select_kernel<<<(unsigned)(nqc * hkv), kSelThreads, 0, st>>>(a);
+            }
             if ((s = check_launch("tree_select_kernel")) != LSA_OK) return s;
             continue;
         }
@@ -647,7 +650,10 @@ lsa_status run_select(const uint16_t* Q, int64_t t0, int64_t nq, int32_t hq, con
         ra.cand = w.cand; ra.cand_n = w.cand_n; ra.idx = a.idx;
         ra.ovf_rows = w.ovf_rows; ra.ovf_count = w.ovf_count; ra.ovf_cap = a.ovf_cap;
         if ((s = launch_flat(pa, ra, tmF, tmS, st)) != LSA_OK) return s;
-        select_fallback_kernel<<<(unsigned)p.fb_slots, kSelThreads, 0, st>>>(a);
+        {
+            KTime kt_("select_fallback_kernel", st);
+            select_fallback_kernel<<<(unsigned)p.fb_slots, kSelThreads, 0, st>>>(a);
+        }
         if ((s = check_launch("select_fallback_kernel")) != LSA_OK) return s;
     }
     return LSA_OK;

@@ -210,6 +210,22 @@ lsa_status lsa_select(const uint16_t* Q, int64_t t0, int64_t nq, int32_t hq,
                       const lsa_tree* tree, const lsa_cfg* cfg, int32_t* idx,
                       uint16_t* Y_out, void* ws, size_t ws_bytes, void* stream);
 
+/* --------------------------------------------------------- kernel timing */
+
+/*
+ * Kernel timing (tracing; no counterpart on the pages).  Between
+ * lsa_timing_begin() and lsa_timing_end(), every launch of the library's
+ * compute kernels is bracketed by two CUDA events recorded on its stream;
+ * lsa_timing_get() synchronises on them and returns, for one kernel name
+ * (e.g. "flat_cand_kernel", "attn_kernel"), the summed duration in ms and
+ * the number of launches recorded since the last begin.  Events are created
+ * on first use and reused.  A name never launched gives 0 and 0.  Host
+ * thread safe; one device per process.
+ */
+void lsa_timing_begin(void);
+void lsa_timing_end(void);
+lsa_status lsa_timing_get(const char* name, double* total_ms, int64_t* launches);
+
 /* ------------------------------------------------------- (4) attention */
 
 /*
