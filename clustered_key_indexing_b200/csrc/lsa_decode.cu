@@ -14,7 +14,7 @@
 //   ward_kernel (jobs)     every request whose token completed a block
 //                          clusters it; the tree is updated above its slots;
 //   query latents, then flat (decode_score_kernel + decode_resolve_kernel)
-//                          or tree (tree_select_kernel) selection;
+//                          or tree (tree_warp_kernel) selection;
 //   attn_kernel<8>         eight warps share each (request, kv-head) row.
 // Flat scores: one HBM pass over the request's eligible centroids (one lane
 // per centroid, fp32 dot products) storing each slot's score bin (2048 bins
@@ -641,8 +641,7 @@ lsa_status lsa_decode_step(lsa_decode* d, const uint16_t* q, const uint16_t* k, 
     fill_select_args(a, d, cfg, w.Y, idx);
     for (int r = 0; r < d->batch; ++r) a.pos[r] = d->len[r] - 1;
     if (cfg->mode == 1) {
-        tree_select_kernel<<<(unsigned)rows, kSelThreads, 0, st>>>(a);
-        if ((s = check_launch("tree_select_kernel(decode)")) != LSA_OK) return s;
+        if ((s = launch_tree_select(a, rows, st)) != LSA_OK) return s;
     } else {
         const int64_t ld = (d->cache.cap_buckets + 127) / 128 * 128;
         DecScoreArgs sa{};

@@ -154,14 +154,11 @@ struct SelShared {
     // 8-byte members first: every field below stays naturally aligned
     unsigned long long hist[kBins];   // packed (count << 32 | weight)
     double csc[kCap];
-    long long beam_id[16];
-    double beam_sc[16];
     long long above;                  // radix select: weight strictly above the prefix
     int cid[kCap];
     int cw[kCap];
     int ctk[kCap];
     int sh4[4];
-    int nbeam;
     int misc[4];
     uint16_t ylat[8 * kDL];
 };
@@ -327,134 +324,216 @@ __device__ void emit_range(const SelectArgs& a, const RowInfo& r, int64_t ncol, 
     for (int64_t i = base + threadIdx.x; i < a.k; i += kSelThreads) r.out[a.S + i] = -1;
 }
 
-// Beam descent [essay ch. 4]: leaves end up as candidates (id order) in
-// sh.cid / sh.csc / sh.cw; returns their count.
-__device__ int tree_candidates(const SelectArgs& a, const RowInfo& r, SelShared& sh) {
-    const int tid = threadIdx.x;
+// Tree search [essay ch. 4]: one warp per (query, kv-head).
+//   descent: from the root down to level L*, the children of the beam are
+//     scored exactly (fp64, ascending dims, one child per lane) and the best
+//     `beam` eligible ones kept (score desc, node index asc), then ordered by
+//     node index;
+//   leaves: the eligible buckets below the final beam, ascending id, scored
+//     exactly, weighted by their keys in [S, t - W];
+//   fill: exactly k keys from the best (score desc, id asc) by a warp radix
+//     select on the fp64 order keys (8 digits of 8 bits); at the cut the
+//     lowest ids first; keys emitted in ascending bucket id.
+constexpr int kTreeWarps = 4;
+
+// Leaves a row can reach: at most beam subtrees of 2^L* buckets.
+static inline int tree_max_cands(int beam, int lstar) { return beam << lstar; }
+
+__host__ __device__ inline size_t tree_warp_bytes(int maxn) {
+    return (((size_t)maxn * 16 + 256 * 4 + 8 * kDL * 2) + 15) & ~(size_t)15;
+}
+
+__global__ void __launch_bounds__(32 * kTreeWarps) tree_warp_kernel(SelectArgs a, int64_t nrows, int maxn) {
+    extern __shared__ __align__(16) uint8_t tsm[];
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    const int64_t row = (int64_t)blockIdx.x * kTreeWarps + wid;
+    if (row >= nrows) return;
+    uint8_t* base = tsm + (size_t)wid * tree_warp_bytes(maxn);
+    double* sc = reinterpret_cast<double*>(base);          // exact leaf scores
+    int* id = reinterpret_cast<int*>(sc + maxn);          // leaf bucket ids, ascending
+    int* wt = id + maxn;                                  // key weights, then taken counts
+    uint32_t* hist = reinterpret_cast<uint32_t*>(wt + maxn);
+    uint16_t* ylat = reinterpret_cast<uint16_t*>(hist + 256);
+    const RowInfo r = row_info(a, row);
+
+    for (int i = lane; i < a.S; i += 32) r.out[i] = (i <= r.t) ? i : -1;
+    const int64_t w0 = max((int64_t)a.S, r.t - a.W + 1);
+    const int64_t nw = r.t >= a.S ? r.t - w0 + 1 : 0;
+    for (int i = lane; i < a.W; i += 32) r.out[a.S + a.k + i] = i < nw ? (int32_t)(w0 + i) : -1;
+    if (r.lim < a.S) {
+        for (int i = lane; i < a.k; i += 32) r.out[a.S + i] = -1;
+        return;
+    }
     const int ng = a.agg ? a.G : 1;
+    const uint16_t* ysrc = a.agg ? a.Y + (r.q * (int64_t)a.hkv * a.G + (int64_t)r.h * a.G) * kDL
+                                 : a.Y + (r.q * (int64_t)a.hkv + r.h) * kDL;
+    for (int i = lane; i < ng * kDL; i += 32) ylat[i] = ysrc[i];
+    __syncwarp();
+
+    // descent: lane i < nbeam holds beam node i (ascending index)
     const int64_t hn = (int64_t)r.h * a.n_nodes;
     const int top = a.levels - 1;
-    if (tid == 0) {
-        sh.nbeam = 0;
-        if (top <= a.lstar) {
-            sh.beam_id[0] = 0;
-            sh.nbeam = 1;
-        } else if ((int64_t)a.tminlr[hn + a.level_off[top]] <= r.lim) {
-            sh.beam_id[0] = 0;
-            sh.nbeam = 1;
-        }
+    int nbeam = 0;
+    long long mybeam = -1;
+    if (top <= a.lstar || (int64_t)a.tminlr[hn + a.level_off[top]] <= r.lim) {
+        nbeam = 1;
+        mybeam = lane == 0 ? 0 : -1;
     }
-    __syncthreads();
-    int lvl = top;
-    while (lvl > a.lstar && sh.nbeam > 0) {
-        const int nb = sh.nbeam;
+    for (int lvl = top; lvl > a.lstar && nbeam > 0; --lvl) {
         const int64_t nl = a.level_n[lvl - 1];
-        double sc = -CUDART_INF;
+        const int nc = 2 * nbeam;  // children of the beam (<= 16)
+        const long long par = __shfl_sync(0xffffffffu, mybeam, (lane >> 1) & 31);
+        double s = -CUDART_INF;
         long long node = -1;
-        if (tid < 2 * nb) {
-            const long long ch = 2 * sh.beam_id[tid >> 1] + (tid & 1);
+        if (lane < nc) {
+            const long long ch = 2 * par + (lane & 1);
             if (ch < nl) {
                 const int64_t gi = hn + a.level_off[lvl - 1] + ch;
                 if ((int64_t)a.tminlr[gi] <= r.lim) {
-                    sc = exact_score(sh.ylat, ng, a.tcent + gi * kDL);
+                    s = exact_row(ylat, ng, a.tcent + gi * kDL);
                     node = ch;
                 }
             }
         }
-        __syncthreads();
-        if (tid < 16) { sh.beam_sc[tid] = sc; sh.beam_id[tid] = node; }
-        __syncthreads();
-        if (tid == 0) {
-            // keep the best `beam` eligible children (score desc, index asc)
-            double bs[16];
-            long long bi[16];
-            int m = 0;
-            for (int i = 0; i < 2 * nb; ++i) {
-                if (sh.beam_id[i] < 0) continue;
-                int j = m++;
-                while (j > 0 && (bs[j - 1] < sh.beam_sc[i] ||
-                                 (bs[j - 1] == sh.beam_sc[i] && bi[j - 1] > sh.beam_id[i]))) {
-                    bs[j] = bs[j - 1];
-                    bi[j] = bi[j - 1];
-                    --j;
-                }
-                bs[j] = sh.beam_sc[i];
-                bi[j] = sh.beam_id[i];
-            }
-            const int keep = m < a.beam ? m : a.beam;
-            // ascending node index for the next level / the leaf list
-            for (int i = 1; i < keep; ++i)
-                for (int j = i; j > 0 && bi[j - 1] > bi[j]; --j) {
-                    long long t2 = bi[j]; bi[j] = bi[j - 1]; bi[j - 1] = t2;
-                }
-            for (int i = 0; i < keep; ++i) sh.beam_id[i] = bi[i];
-            sh.nbeam = keep;
+        // rank among the eligible children (score desc, index asc)
+        int rank = 0;
+        for (int j = 0; j < nc; ++j) {
+            const double sj = __shfl_sync(0xffffffffu, s, j);
+            const long long nj = __shfl_sync(0xffffffffu, node, j);
+            if (nj >= 0 && (sj > s || (sj == s && nj < node))) ++rank;
         }
-        __syncthreads();
-        --lvl;
+        const bool keep = node >= 0 && rank < a.beam;
+        const unsigned km = __ballot_sync(0xffffffffu, keep);
+        // the kept nodes, ascending index, into lanes 0 .. popc(km) - 1
+        int pos = 0;
+        for (int j = 0; j < nc; ++j) {
+            const long long nj = __shfl_sync(0xffffffffu, node, j);
+            if (((km >> j) & 1u) && nj < node) ++pos;
+        }
+        long long nb_new = -1;
+        for (int j = 0; j < nc; ++j) {
+            const int pj = __shfl_sync(0xffffffffu, pos, j);
+            const long long nj = __shfl_sync(0xffffffffu, node, j);
+            if (((km >> j) & 1u) && pj == lane) nb_new = nj;
+        }
+        mybeam = nb_new;
+        nbeam = __popc(km);
     }
-    // leaves below the final beam, ascending
-    const int nb = sh.nbeam;
+
+    // leaves below the final beam (the whole cache when the tree is not
+    // taller than L*), eligible ones in ascending id
     const int64_t span = (int64_t)1 << a.lstar;
+    const int64_t hb0 = (int64_t)r.h * a.cap_buckets;
     int n = 0;
-    for (int i = 0; i < nb; ++i) {
-        const int64_t b0 = (top <= a.lstar) ? 0 : (int64_t)sh.beam_id[i] * span;
+    for (int i = 0; i < nbeam; ++i) {
+        const long long bnode = __shfl_sync(0xffffffffu, mybeam, i);
+        const int64_t b0 = (top <= a.lstar) ? 0 : (int64_t)bnode * span;
         const int64_t b1 = (top <= a.lstar) ? a.NB : min(a.NB, b0 + span);
-        for (int64_t c0 = b0; c0 < b1; c0 += kSelThreads) {
-            const int64_t b = c0 + tid;
-            const bool el = b < b1 && (int64_t)a.minlr[(int64_t)r.h * a.cap_buckets + b] <= r.lim;
+        for (int64_t c0 = b0; c0 < b1; c0 += 32) {
+            const int64_t b = c0 + lane;
+            const bool el = b < b1 && (int64_t)a.minlr[hb0 + b] <= r.lim;
             const unsigned bal = __ballot_sync(0xffffffffu, el);
-            int tot;
-            const int o = block_exscan(el ? 1 : 0, &tot, sh.sh4);
-            (void)bal;
-            if (el && n + o < kCap) sh.cid[n + o] = (int)b;
-            n += tot;
+            const int o = n + __popc(bal & ((1u << lane) - 1u));
+            if (el && o < maxn) id[o] = (int)b;
+            n += __popc(bal);
         }
     }
-    __syncthreads();
-    if (n > kCap) return n;
-    for (int i = tid; i < n; i += kSelThreads) {
-        const int64_t b = sh.cid[i];
-        sh.csc[i] = exact_score(sh.ylat, ng, a.cent + ((int64_t)r.h * a.cap_buckets + b) * kDL);
-        sh.cw[i] = bucket_weight(a, r.h, b, r.lim);
+    if (n > maxn) {  // cannot happen: at most beam subtrees of 2^L* leaves
+        if (lane == 0) raise_device_error(kErrSelectOverflow);
+        return;
     }
-    __syncthreads();
-    return n;
+    __syncwarp();
+    long long totw = 0;
+    for (int i = lane; i < n; i += 32) {
+        const int64_t b = id[i];
+        sc[i] = exact_row(ylat, ng, a.cent + (hb0 + b) * kDL);
+        wt[i] = bucket_weight(a, r.h, b, r.lim);
+        totw += wt[i];
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) totw += __shfl_xor_sync(0xffffffffu, totw, off);
+    __syncwarp();
+
+    if (totw > a.k) {
+        // weighted radix select: prefix = the order key of the k-th key,
+        // above = the weight strictly above it
+        unsigned long long prefix = 0ull;
+        long long above = 0;
+        for (int pass = 0; pass < 8; ++pass) {
+            const int shift = 56 - 8 * pass;
+            for (int i = lane; i < 256; i += 32) hist[i] = 0u;
+            __syncwarp();
+            for (int i = lane; i < n; i += 32) {
+                const int w = wt[i];
+                if (w <= 0) continue;
+                const unsigned long long key = order_key(sc[i]);
+                if (pass > 0 && (key >> (shift + 8)) != (prefix >> (shift + 8))) continue;
+                atomicAdd(&hist[(key >> shift) & 255ull], (unsigned)w);
+            }
+            __syncwarp();
+            long long ab = 0;
+            const int dig = cut_bin(hist, a.k - above, &ab);
+            if (dig < 0) {  // cannot happen while the weight above the prefix reaches k
+                if (lane == 0) raise_device_error(kErrSelectOverflow);
+                return;
+            }
+            above += ab;
+            prefix |= (unsigned long long)dig << shift;
+            __syncwarp();
+        }
+        // taken counts: above the cut whole, at the cut lowest ids first
+        const long long need = a.k - above;
+        long long run = 0;
+        for (int b0 = 0; b0 < n; b0 += 32) {
+            const int i = b0 + lane;
+            const int w = i < n ? wt[i] : 0;
+            const unsigned long long key = i < n ? order_key(sc[i]) : 0ull;
+            const long long eq = (w > 0 && key == prefix) ? w : 0;
+            long long incl = eq;
+#pragma unroll
+            for (int off = 1; off < 32; off <<= 1) {
+                const long long y = __shfl_up_sync(0xffffffffu, incl, off);
+                if (lane >= off) incl += y;
+            }
+            int tk = 0;
+            if (w > 0) {
+                if (key > prefix) tk = w;
+                else if (key == prefix) tk = (int)max(0LL, min((long long)w, need - (run + incl - eq)));
+            }
+            __syncwarp();
+            if (i < n) wt[i] = tk;
+            run += __shfl_sync(0xffffffffu, incl, 31);
+        }
+        __syncwarp();
+    }
+    // emit the taken keys in ascending bucket id
+    int o = 0;
+    for (int b0 = 0; b0 < n; b0 += 32) {
+        const int i = b0 + lane;
+        const int tk = i < n ? wt[i] : 0;
+        int incl = tk;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, incl, off);
+            if (lane >= off) incl += y;
+        }
+        if (tk > 0) emit_bucket(a, r.h, id[i], tk, r.lim, r.out + a.S + o + incl - tk);
+        o += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    for (int i = o + lane; i < a.k; i += 32) r.out[a.S + i] = -1;
 }
 
-// Tree search [essay ch. 4]: one CTA per (query, kv-head).
-__global__ void __launch_bounds__(kSelThreads) tree_select_kernel(SelectArgs a) {
-    __shared__ SelShared sh;
-    const int tid = threadIdx.x;
-    const int64_t row = blockIdx.x;
-    const RowInfo r = row_info(a, row);
-    write_sinks_window(a, r);
-    if (r.lim < a.S) {
-        for (int i = tid; i < a.k; i += kSelThreads) r.out[a.S + i] = -1;
-        return;
-    }
-    load_latents(a, r, sh);
+lsa_status launch_tree_select(const SelectArgs& a, int64_t nrows, cudaStream_t st) {
+    const int maxn = tree_max_cands(a.beam, a.lstar);
+    const size_t smem = (size_t)kTreeWarps * tree_warp_bytes(maxn);
+    if (smem > 227 * 1024) return set_error(LSA_EUNSUPPORTED, "tree search: beam * 2^L* = %d leaves too many", maxn);
+    cudaFuncSetAttribute(tree_warp_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     {
-        __syncthreads();
-        const int n = tree_candidates(a, r, sh);
-        if (n > kCap) {
-            if (tid == 0) raise_device_error(kErrSelectOverflow);
-            return;
-        }
-        long long totw = 0;
-        for (int i = 0; i < n; ++i) totw += sh.cw[i];
-        if (totw <= a.k) {
-            for (int i = tid; i < n; i += kSelThreads) sh.ctk[i] = sh.cw[i];
-            __syncthreads();
-        } else {
-            radix_fill(
-                n, a.k, [&](int64_t i) { return sh.csc[i]; }, [&](int64_t i) { return sh.cw[i]; },
-                [&](int64_t i, int tk) { sh.ctk[i] = tk; }, sh);
-        }
-        emit_candidates(a, r, n, sh);
-        return;
+        KTime kt_("tree_select_kernel", st);
+        tree_warp_kernel<<<(unsigned)ceil_div<int64_t>(nrows, kTreeWarps), 32 * kTreeWarps, smem, st>>>(a, nrows,
+                                                                                                       maxn);
     }
-
+    return check_launch("tree_warp_kernel");
 }
 
 // Rows whose candidate band overflowed: exact scores of every eligible
@@ -628,11 +707,7 @@ lsa_status run_select(const uint16_t* Q, int64_t t0, int64_t nq, int32_t hq, con
         if (s != LSA_OK) return s;
         a.Y = Y; a.nqc = nqc; a.t_first = t0 + c0; a.idx = idx + c0 * hkv * row_len;
         if (cfg->mode == 1) {
-            {
-                KTime kt_("tree_select_kernel", st);
-                tree_select_kernel<<<(unsigned)(nqc * hkv), kSelThreads, 0, st>>>(a);
-            }
-            if ((s = check_launch("tree_select_kernel")) != LSA_OK) return s;
+            if ((s = launch_tree_select(a, nqc * hkv, st)) != LSA_OK) return s;
             continue;
         }
         if (cudaMemsetAsync(w.ovf_count, 0, sizeof(int32_t), st) != cudaSuccess)

@@ -132,6 +132,16 @@ def _select_both(lsa, name, T, cfg, tpos=None, seed=0):
     return inp, idx.cpu().numpy()[tpos], oidx, mg
 
 
+@pytest.mark.parametrize("beam,k,agg", [(1, 512, 0), (3, 300, 1), (8, 512, 0)])
+def test_tree_beams_bit_exact(lsa, beam, k, agg):
+    """Tree search with beam 1 (greedy), 3 (native scores) and 8 (16 children
+    scored per level) against the oracle."""
+    cfg = lsa.Config(k=k, sinks=4, window=256, mode=1, beam=beam, agg=agg)
+    _, g, o, _ = _select_both(lsa, "prefill-4k", 4096, cfg)
+    bad = np.where((g != o).any(axis=(1, 2)))[0]
+    assert bad.size == 0, f"{bad.size} rows differ, first t={bad[:5]}"
+
+
 @pytest.mark.parametrize("mode,agg", [(0, 0), (0, 1), (1, 0), (1, 1)])
 def test_select_bit_exact_4k(lsa, mode, agg):
     cfg = lsa.Config(k=512, sinks=4, window=256, mode=mode, agg=agg)
