@@ -550,12 +550,20 @@ def run_decode(args):
     clocks = Clocks(torch.cuda.current_device())
     nl0 = lib().lsa_launch_count()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for s_ in range(args.warmup, nsteps):
-        dec.step(q[s_], kk[s_], vv[s_], Wk, Wq, o=o)
-    e1.record(stream)
-    torch.cuda.synchronize()
+    kt = lsa.KernelTimer()
+    with kt:
+        e0.record(stream)
+        for s_ in range(args.warmup, nsteps):
+            dec.step(q[s_], kk[s_], vv[s_], Wk, Wq, o=o)
+        e1.record(stream)
+        torch.cuda.synchronize()
     clk = clocks.stop()
+    kernels = {}
+    for name in ("decode_score_kernel", "decode_resolve_kernel", "attn_kernel_split", "decode_append_kernel",
+                 "latent_kernel", "ward_kernel", "tree_select_kernel"):
+        kms, kn = kt.get(name)
+        if kn:
+            kernels[name] = {"ms_per_step": kms / args.steps, "launches_per_step": kn / args.steps}
     launches = lib().lsa_launch_count() - nl0
     ms = e0.elapsed_time(e1)
     if world > 1:
@@ -589,7 +597,7 @@ def run_decode(args):
                        "search": "flat" if c["mode"] == 0 else f"tree(beam={c['beam']})",
                        "inputs": "device-drawn (torch Philox), same recipe as synth",
                        "l2": "no flush: per-step centroid scan (4.3 GB) is larger than L2"},
-            "clocks": clk, "gpu_launches": int(launches),
+            "clocks": clk, "gpu_launches": int(launches), "kernels": kernels,
             "roofline": {"kernel": "decode step (centroid scan + gather + attention)", "bound": "hbm",
                          "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
                          "frac": achieved / pk["hbm_gbs"], "traffic": None, "peak_source": src,

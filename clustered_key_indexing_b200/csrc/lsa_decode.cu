@@ -28,6 +28,8 @@
 
 #include "lsa.h"
 #include "lsa_common.cuh"
+#include "lsa_mma.cuh"
+#include "lsa_tc.cuh"
 
 namespace lsa {
 
@@ -148,7 +150,6 @@ __global__ void __launch_bounds__(256) tail_units_kernel(const uint16_t* __restr
 
 // ------------------------------------------------------ flat decode scores
 
-constexpr int kDecScoreCols = 2048;  // bucket slots per CTA
 constexpr int kDecBins = 2048;       // histogram bins over the row's score range
 
 struct DecScoreArgs {
@@ -195,68 +196,133 @@ __device__ __forceinline__ int score_to_bin(float s, float R) {
     return bin < 0 ? 0 : (bin >= kDecBins ? kDecBins - 1 : bin);
 }
 
-// grid (column chunks, rows); one lane per bucket slot: eight 16-byte loads of
-// its centroid, a private fp32 dot product per query latent; coalesced
-// metadata loads and bin / weight stores.  NG = latents per row.
+// grid (column chunks, rows), 4 warps.  The chunk's centroids stream through
+// a 3-stage shared-memory ring of 256-row tiles (TMA, 128-byte swizzle, one
+// thread issues; bounded mbarrier waits, no multicast).  Each warp scores 64
+// centroids of a tile with mma.sync m16n8k16 (centroids as M, the row's NG
+// query latents as N, fp32 accumulate), the lane pairs' scores are reduced
+// to the max over latents, binned, and the tile's bins and weights are
+// written with coalesced stores (weights from cnt_lr, and below the frontier
+// block no minlr / maxpos reads: those buckets lie wholly in [S, t - W]).
+constexpr int kDecScanCols = 4096;   // bucket slots per CTA
+constexpr int kDecTile = 256;        // centroids per ring stage (32 KB)
+constexpr int kDecStages = 3;
+constexpr size_t kDecScanSmem = 1024 + (size_t)kDecStages * kDecTile * kDL * 2 + kDecTile * 4 + 64;
+
 template <int NG>
-__global__ void __launch_bounds__(256) decode_score_kernel(DecScoreArgs a) {
-    __shared__ float ys[NG][kDL];
+__global__ void __launch_bounds__(128) decode_score_kernel(const __grid_constant__ CUtensorMap tmC, DecScoreArgs a) {
+    extern __shared__ uint8_t dsm_raw[];
+    uint8_t* dsm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsm_raw) + 1023) & ~(uintptr_t)1023);
+    uint8_t* ring = dsm;
+    float* best_s = reinterpret_cast<float*>(ring + kDecStages * kDecTile * kDL * 2);  // [kDecTile]
+    uint64_t* bars = reinterpret_cast<uint64_t*>(best_s + kDecTile);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + kDecStages);
     __shared__ float rad;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int64_t row = blockIdx.y;
     const int64_t r = row / a.hkv;
     const int64_t t = a.pos[r];
     const int64_t lim = t - a.W;
     const int64_t ncol = lim < 0 ? 0 : min(a.cap_buckets, (int64_t)kBucketsPerBlock * (lim / kBlockKeys + 1));
-    const int64_t c0 = (int64_t)blockIdx.x * kDecScoreCols;
+    const int64_t c0 = (int64_t)blockIdx.x * kDecScanCols;
     if (c0 >= ncol) return;
+    const int64_t cend = min(ncol, c0 + kDecScanCols);
+    const int ntiles = (int)((cend - c0 + kDecTile - 1) / kDecTile);
+    const uint32_t bar0 = smem_u32(bars);
+    if (tid == 0) {
+        for (int s = 0; s < kDecStages; ++s) mbar_init(bar0 + 8u * s, 1);
+        *abort_flag = 0;
+        fence_barrier_init();
+    }
     const uint16_t* yb = a.Y + (row * NG) * kDL;  // native: row*G = r*hq + h*G
-    for (int i = threadIdx.x; i < NG * kDL; i += blockDim.x) ys[i / kDL][i % kDL] = bf16_to_f32(yb[i]);
-    if (threadIdx.x == 0) rad = row_radius(yb, NG);
+    if (tid == 0) rad = row_radius(yb, NG);
+    // B operand: Y^T (k = dims, n = latent rows, zero past NG)
+    const int gq = lane >> 2, tq = lane & 3;
+    uint32_t yq[4][2];
+#pragma unroll
+    for (int kk = 0; kk < 4; ++kk) {
+        yq[kk][0] = gq < NG ? *reinterpret_cast<const uint32_t*>(yb + gq * kDL + kk * 16 + 2 * tq) : 0u;
+        yq[kk][1] = gq < NG ? *reinterpret_cast<const uint32_t*>(yb + gq * kDL + kk * 16 + 8 + 2 * tq) : 0u;
+    }
     __syncthreads();
-    const float R = rad;
-    const uint16_t* cb = a.cent + row * a.cap_buckets * kDL;
-    const int64_t hb0 = row * a.cap_buckets;
-    const int64_t cend = min(ncol, c0 + kDecScoreCols);
-    // two slots per thread per iteration: 16 loads of 16 bytes in flight
-    for (int64_t b0 = c0 + threadIdx.x; b0 < cend; b0 += 2 * blockDim.x) {
-        int64_t bb[2] = {b0, b0 + blockDim.x};
-        bool ok[2] = {true, b0 + blockDim.x < cend};
-        uint4 cv[2][8];
-        int32_t mlr[2], mxp[2], clr[2];
-#pragma unroll
-        for (int u2 = 0; u2 < 2; ++u2) {
-            const int64_t b = ok[u2] ? bb[u2] : b0;
-#pragma unroll
-            for (int i = 0; i < 8; ++i) cv[u2][i] = __ldg(reinterpret_cast<const uint4*>(cb + b * kDL) + i);
-            mlr[u2] = __ldg(a.minlr + hb0 + b);
-            mxp[u2] = __ldg(a.maxpos + hb0 + b);
-            clr[u2] = __ldg(a.cnt_lr + hb0 + b);
+    const int64_t rowbase = row * a.cap_buckets;
+    if (tid == 0) {
+        for (int i = 0; i < kDecStages && i < ntiles; ++i) {
+            mbar_expect_tx(bar0 + 8u * i, kDecTile * kDL * 2);
+            tma_load_2d(smem_u32(ring + i * kDecTile * kDL * 2), &tmC, 0, (int32_t)(rowbase + c0 + i * kDecTile),
+                        bar0 + 8u * i);
         }
+    }
+    const float R = rad;
+    const int64_t hb0 = rowbase;
+    const int64_t frontier = ncol - kBucketsPerBlock;  // first bucket of the last block in range
+    int done = 0;  // tiles consumed
+    for (int it = 0; it < ntiles; ++it) {
+        const int s = it % kDecStages;
+        const bool ok = mbar_wait(bar0 + 8u * s, (uint32_t)(it / kDecStages) & 1u, abort_flag);
+        if (!__syncthreads_and(ok)) break;
+        const uint32_t tb = smem_u32(ring + s * kDecTile * kDL * 2);
+        // warp w: centroids 64 w .. 64 w + 63 of the tile, four m16 tiles
 #pragma unroll
-        for (int u2 = 0; u2 < 2; ++u2) {
-            if (!ok[u2]) continue;
-            const int64_t b = bb[u2];
-            float best = -CUDART_INF_F;
+        for (int mt = 0; mt < 4; ++mt) {
+            float acc[4] = {0.f, 0.f, 0.f, 0.f};
+            const int m0 = 64 * warp + 16 * mt;
 #pragma unroll
-            for (int g = 0; g < NG; ++g) {
-                float sacc = 0.f;
-#pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    const uint32_t u[4] = {cv[u2][i].x, cv[u2][i].y, cv[u2][i].z, cv[u2][i].w};
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        sacc = fmaf(ys[g][8 * i + 2 * e], __uint_as_float(u[e] << 16), sacc);
-                        sacc = fmaf(ys[g][8 * i + 2 * e + 1], __uint_as_float(u[e] & 0xFFFF0000u), sacc);
-                    }
-                }
-                best = fmaxf(best, sacc);
+            for (int kk = 0; kk < 4; ++kk) {
+                uint32_t af[4];
+                const int rr = m0 + (lane & 15);
+                const int ch = 2 * kk + (lane >> 4);
+                ldsm_x4(af, tb + (uint32_t)(rr * 128 + ((ch ^ (rr & 7)) << 4)));
+                mma_16816(acc, af, yq[kk][0], yq[kk][1]);
             }
-            int w = 0;
-            if ((int64_t)mlr[u2] <= lim)
-                w = (int64_t)mxp[u2] <= lim ? clr[u2] : weight_units(b, __ldg(a.units + hb0 + b), lim, a.S, a.T_built);
-            a.bin[row * a.ld + b] = (uint16_t)score_to_bin(best, R);
+            // acc: (centroid gq, latents 2tq, 2tq+1), (centroid gq + 8, same)
+            float b0 = NG > 1 ? fmaxf(acc[0], acc[1]) : acc[0];
+            float b1 = NG > 1 ? fmaxf(acc[2], acc[3]) : acc[2];
+            if (NG > 2) {
+                b0 = fmaxf(b0, __shfl_xor_sync(0xffffffffu, b0, 1));
+                b1 = fmaxf(b1, __shfl_xor_sync(0xffffffffu, b1, 1));
+            }
+            if (NG > 4) {
+                b0 = fmaxf(b0, __shfl_xor_sync(0xffffffffu, b0, 2));
+                b1 = fmaxf(b1, __shfl_xor_sync(0xffffffffu, b1, 2));
+            }
+            if (tq == 0) {
+                best_s[m0 + gq] = b0;
+                best_s[m0 + gq + 8] = b1;
+            }
+        }
+        __syncthreads();
+        // the stage is free: the next tile of the chunk into it
+        if (tid == 0 && it + kDecStages < ntiles) {
+            fence_proxy_async_smem();
+            mbar_expect_tx(bar0 + 8u * s, kDecTile * kDL * 2);
+            tma_load_2d(smem_u32(ring + s * kDecTile * kDL * 2), &tmC, 0,
+                        (int32_t)(rowbase + c0 + (it + kDecStages) * kDecTile), bar0 + 8u * s);
+        }
+        // bins and weights of the tile, coalesced
+        const int64_t tb0 = c0 + (int64_t)it * kDecTile;
+        for (int j = tid; j < kDecTile; j += 128) {
+            const int64_t b = tb0 + j;
+            if (b >= cend) break;
+            const int32_t clr = __ldg(a.cnt_lr + hb0 + b);
+            int w = clr;
+            if (b >= frontier) {
+                const int32_t mlr = __ldg(a.minlr + hb0 + b), mxp = __ldg(a.maxpos + hb0 + b);
+                w = 0;
+                if ((int64_t)mlr <= lim)
+                    w = (int64_t)mxp <= lim ? clr : weight_units(b, __ldg(a.units + hb0 + b), lim, a.S, a.T_built);
+            }
+            a.bin[row * a.ld + b] = (uint16_t)score_to_bin(best_s[j], R);
             a.wt[row * a.ld + b] = (uint8_t)w;
         }
+        __syncthreads();  // best_s is rewritten by the next tile
+        done = it + 1;
+    }
+    // after an abort, let the copies already issued land before the CTA exits
+    if (tid == 0 && *abort_flag) {
+        const int issued = min(ntiles, done + kDecStages);
+        for (int i = done; i < issued; ++i)
+            mbar_wait(bar0 + 8u * (i % kDecStages), (uint32_t)(i / kDecStages) & 1u, abort_flag, false);
     }
 }
 
@@ -305,6 +371,7 @@ __global__ void __launch_bounds__(kSelThreads) decode_resolve_kernel(DecResolveA
     };
     const int64_t ng16 = (ncol + 15) / 16;
     long long myw = 0;
+#pragma unroll 4
     for (int64_t g16 = tid; g16 < ng16; g16 += kSelThreads) {
         uint8_t w16[16];
         uint16_t b16[16];
@@ -365,6 +432,7 @@ __global__ void __launch_bounds__(kSelThreads) decode_resolve_kernel(DecResolveA
         const int64_t per = (ng16 + kSelThreads / 32 - 1) / (kSelThreads / 32);
         const int64_t g_lo = wid * per, g_hi = min(ng16, g_lo + per);
         int c = 0;
+#pragma unroll 4
         for (int64_t g16 = g_lo + lane; g16 < g_hi; g16 += 32) {
             uint8_t w16[16];
             uint16_t b16[16];
@@ -650,14 +718,16 @@ lsa_status lsa_decode_step(lsa_decode* d, const uint16_t* q, const uint16_t* k, 
         sa.ld = ld; sa.hkv = d->hkv; sa.G = d->hq / d->hkv; sa.agg = cfg->agg; sa.S = cfg->sinks;
         sa.W = cfg->window; sa.T_built = d->cap; sa.bin = w.bin; sa.wt = w.wt;
         for (int r = 0; r < d->batch; ++r) sa.pos[r] = a.pos[r];
-        dim3 grid((unsigned)ceil_div<int64_t>(d->cache.cap_buckets, kDecScoreCols), (unsigned)rows);
+        dim3 grid((unsigned)ceil_div<int64_t>(d->cache.cap_buckets, kDecScanCols), (unsigned)rows);
         const int ng = cfg->agg ? d->hq / d->hkv : 1;
+        CUtensorMap tmC;
+        if ((s = make_rows64_map(&tmC, d->cache.cent, rows * d->cache.cap_buckets, kDecTile)) != LSA_OK) return s;
+        auto kern = ng == 1 ? decode_score_kernel<1> : ng == 2 ? decode_score_kernel<2>
+                  : ng == 4 ? decode_score_kernel<4> : decode_score_kernel<8>;
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kDecScanSmem);
         {
             KTime kt_("decode_score_kernel", st);
-            if (ng == 1) decode_score_kernel<1><<<grid, 256, 0, st>>>(sa);
-            else if (ng == 2) decode_score_kernel<2><<<grid, 256, 0, st>>>(sa);
-            else if (ng == 4) decode_score_kernel<4><<<grid, 256, 0, st>>>(sa);
-            else decode_score_kernel<8><<<grid, 256, 0, st>>>(sa);
+            kern<<<grid, 128, kDecScanSmem, st>>>(tmC, sa);
         }
         if ((s = check_launch("decode_score_kernel")) != LSA_OK) return s;
         DecResolveArgs ra{};
