@@ -354,7 +354,10 @@ __global__ void __launch_bounds__(kSelThreads) decode_resolve_kernel(DecResolveA
     const int64_t ncol = min(d.cap_buckets, (int64_t)kBucketsPerBlock * (r.lim / kBlockKeys + 1));
     const uint16_t* brow = d.bin + row * d.ld;
     uint8_t* wrow = d.wt + row * d.ld;
-    for (int i = tid; i < kDecBins; i += kSelThreads) sh.hist[i] = 0ull;
+    // key weights per bin (32-bit counters; the candidate count comes from
+    // the compaction's own count)
+    uint32_t* h32 = reinterpret_cast<uint32_t*>(sh.hist);
+    for (int i = tid; i < kDecBins; i += kSelThreads) h32[i] = 0u;
     __syncthreads();
     // 16 slots per lane per step: one 16-byte load of weights, two of bins
     auto load16 = [&](int64_t g16, uint8_t (&w16)[16], uint16_t (&b16)[16]) {
@@ -380,7 +383,7 @@ __global__ void __launch_bounds__(kSelThreads) decode_resolve_kernel(DecResolveA
         for (int i = 0; i < 16; ++i) {
             if (w16[i] == 0) continue;
             myw += w16[i];
-            atomicAdd(&sh.hist[b16[i]], (1ull << 32) | (unsigned long long)w16[i]);
+            atomicAdd(&h32[b16[i]], (uint32_t)w16[i]);
         }
     }
 #pragma unroll
@@ -398,7 +401,7 @@ __global__ void __launch_bounds__(kSelThreads) decode_resolve_kernel(DecResolveA
     if (tid < 32) {
         long long s = 0;
         for (int dd = 0; dd < kDecBins / 32; ++dd)
-            s += (long long)(sh.hist[kDecBins - 1 - (kDecBins / 32) * lane - dd] & 0xffffffffull);
+            s += (long long)h32[kDecBins - 1 - (kDecBins / 32) * lane - dd];
         long long incl = s;
 #pragma unroll
         for (int off = 1; off < 32; off <<= 1) {
@@ -413,7 +416,7 @@ __global__ void __launch_bounds__(kSelThreads) decode_resolve_kernel(DecResolveA
             int j = kDecBins - 1 - (kDecBins / 32) * lane;
             for (int dd = 0; dd < kDecBins / 32; ++dd) {
                 const int jj = kDecBins - 1 - (kDecBins / 32) * lane - dd;
-                cum += (long long)(sh.hist[jj] & 0xffffffffull);
+                cum += (long long)h32[jj];
                 if (cum >= a.k) { j = jj; break; }
             }
             sh.misc[0] = j > 0 ? j - 1 : 0;
@@ -421,16 +424,12 @@ __global__ void __launch_bounds__(kSelThreads) decode_resolve_kernel(DecResolveA
     }
     __syncthreads();
     const int jt = sh.misc[0];
-    int cnt = 0;
-    for (int i = jt + tid; i < kDecBins; i += kSelThreads) cnt += (int)(sh.hist[i] >> 32);
-    int ncand;
-    block_exscan(cnt, &ncand, sh.sh4);
-    if (ncand <= kCap) {
-        // warp-ordered compaction: warp w takes a contiguous quarter of the
-        // 16-slot groups and lane l the l-th group of each 512-slot stretch,
-        // so the concatenated lists keep ascending ids
-        const int64_t per = (ng16 + kSelThreads / 32 - 1) / (kSelThreads / 32);
-        const int64_t g_lo = wid * per, g_hi = min(ng16, g_lo + per);
+    // warp-ordered compaction: warp w takes a contiguous quarter of the
+    // 16-slot groups and lane l the l-th group of each 512-slot stretch, so
+    // the concatenated lists keep ascending ids; first each warp's count
+    const int64_t per = (ng16 + kSelThreads / 32 - 1) / (kSelThreads / 32);
+    const int64_t g_lo = wid * per, g_hi = min(ng16, g_lo + per);
+    {
         int c = 0;
 #pragma unroll 4
         for (int64_t g16 = g_lo + lane; g16 < g_hi; g16 += 32) {
@@ -443,7 +442,11 @@ __global__ void __launch_bounds__(kSelThreads) decode_resolve_kernel(DecResolveA
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) c += __shfl_xor_sync(0xffffffffu, c, off);
         if (lane == 0) wcnt[wid] = c;
-        __syncthreads();
+    }
+    __syncthreads();
+    int ncand = 0;
+    for (int i = 0; i < kSelThreads / 32; ++i) ncand += wcnt[i];
+    if (ncand <= kCap) {
         int base = 0;
         for (int i = 0; i < wid; ++i) base += wcnt[i];
         for (int64_t s0 = g_lo; s0 < g_hi; s0 += 32) {

@@ -158,7 +158,7 @@ struct SelShared {
     int cid[kCap];
     int cw[kCap];
     int ctk[kCap];
-    int sh4[4];
+    int sh4[kSelThreads / 32];
     int misc[4];
     uint16_t ylat[8 * kDL];
 };
