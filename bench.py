@@ -188,36 +188,6 @@ def oracle_sample(inp, c, n_blocks=None, n_queries=32, seed=0):
     return per_layer, desc, t_build + t_q * n_queries
 
 
-# ------------------------------------------------- device-drawn inputs
-
-def device_tokens(n, heads, d, mu, scale, gen, dev, out=None, chunk=65536):
-    """bf16 [n, heads, d] of scale * mu_c + N(0, I) (scale 0: N(0, 1)), c
-    uniform per (token, head), drawn on the device by torch's seeded
-    generator (same recipe as synth, another random stream)."""
-    import torch
-    if out is None:
-        out = torch.empty((n, heads, d), dtype=torch.bfloat16, device=dev)
-    for t0 in range(0, n, chunk):
-        t1 = min(n, t0 + chunk)
-        x = torch.randn((t1 - t0, heads, d), generator=gen, device=dev, dtype=torch.float32)
-        if scale != 0.0:
-            ci = torch.randint(0, mu.shape[0], (t1 - t0, heads), generator=gen, device=dev)
-            x += scale * mu[ci]
-        out[t0:t1] = x.to(torch.bfloat16)
-    return out
-
-
-def device_layer(c, seed, dev):
-    import torch
-    gen = torch.Generator(device=dev)
-    gen.manual_seed(seed)
-    mu = torch.from_numpy(synth.centres(seed, c["n_centres"], c["d"])).to(dev)
-    K = device_tokens(c["T"], c["hkv"], c["d"], mu, 4.0, gen, dev)
-    V = device_tokens(c["T"], c["hkv"], c["d"], mu, 0.0, gen, dev)
-    Q = device_tokens(c["T"], c["hq"], c["d"], mu, 1.0, gen, dev)
-    return Q, K, V
-
-
 # ------------------------------------------------------------------ main
 
 def bits_of(t):
@@ -295,7 +265,7 @@ def run_lsa(args):
         Q, K, V = hQ.to(dev), hK.to(dev), hV.to(dev)
         Wk_np, Wq_np = inp["Wk"], inp["Wq"]
     else:
-        Q, K, V = device_layer(c, rank, dev)
+        Q, K, V = synth.device_layer(c, rank, dev)
         hQ, hK, hV = (x.cpu().pin_memory() for x in (Q, K, V))
         Wk_np, Wq_np = synth.projections(rank, c["d"], c["dl"])
         inp = {"Wk": Wk_np, "Wq": Wq_np}
@@ -504,10 +474,11 @@ def run_lsa(args):
 
 
 def run_decode(args):
-    """Batched decode: `batch` requests whose caches hold T - 32 tokens (built
-    with lsa_decode_load, outside the timing); a step is one lsa_decode_step
-    (one new token per request).  The 32nd step completes a 512-key block in
-    every request, so the timed steps include one streaming Ward pass."""
+    """Batched decode: `batch` requests whose prompts (built with
+    lsa_decode_load, outside the timing) end so that the middle timed step
+    appends the last key of a 512-key block in every request: the timed
+    steps include one streaming Ward pass per request (with 512 timed steps
+    that is exactly the steady-state rate of one block per 512 tokens)."""
     import torch
     import torch.distributed as dist
 
@@ -520,24 +491,17 @@ def run_decode(args):
     cfg = lsa.Config(k=c["k"], sinks=c["sinks"], window=c["window"], beam=c["beam"],
                      mode=c["mode"], agg=c["agg"])
     dev = torch.device("cuda", torch.cuda.current_device())
-    cap = T + 512
-    n0 = T - 32
+    nsteps = args.warmup + args.steps
+    n0 = decode_prompt_len(T, args.warmup, args.steps)
+    cap = -(-(n0 + nsteps) // 512) * 512
     dec = lsa.Decode(B, hkv, hq, cap, cfg, device=dev)
-    gen = torch.Generator(device=dev)
-    gen.manual_seed(1000 * rank)
-    mu = torch.from_numpy(synth.centres(rank, c["n_centres"], c["d"])).to(dev)
     Wk_np, Wq_np = synth.projections(rank, c["d"], c["dl"])
     Wk, Wq = torch.from_numpy(Wk_np).to(dev), torch.from_numpy(Wq_np).to(dev)
     ccfg = cfg.c()
+    q, kk, vv = synth.device_decode(c, rank, dev, n0, nsteps, dec.K, dec.V)
     for r in range(B):
-        device_tokens(n0, hkv, c["d"], mu, 4.0, gen, dev, out=dec.K[r, :n0])
-        device_tokens(n0, hkv, c["d"], mu, 0.0, gen, dev, out=dec.V[r, :n0])
         check(lib().lsa_decode_load(ctypes_ref(dec.d), r, n0, ctypes_ptr(Wk), ctypes_ref(ccfg),
                                     ctypes_ptr(dec.ws), dec.ws.numel(), None), "lsa_decode_load")
-    nsteps = args.warmup + args.steps
-    q = device_tokens(nsteps * B, hq, c["d"], mu, 1.0, gen, dev).view(nsteps, B, hq, c["d"])
-    kk = device_tokens(nsteps * B, hkv, c["d"], mu, 4.0, gen, dev).view(nsteps, B, hkv, c["d"])
-    vv = device_tokens(nsteps * B, hkv, c["d"], mu, 0.0, gen, dev).view(nsteps, B, hkv, c["d"])
     o = torch.empty((B, hq, c["d"]), dtype=torch.bfloat16, device=dev)
     torch.cuda.synchronize()
     stream = torch.cuda.current_stream()
@@ -550,13 +514,21 @@ def run_decode(args):
     clocks = Clocks(torch.cuda.current_device())
     nl0 = lib().lsa_launch_count()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sev = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
     kt = lsa.KernelTimer()
     with kt:
         e0.record(stream)
-        for s_ in range(args.warmup, nsteps):
+        sev[0].record(stream)
+        for i, s_ in enumerate(range(args.warmup, nsteps)):
             dec.step(q[s_], kk[s_], vv[s_], Wk, Wq, o=o)
+            sev[i + 1].record(stream)
         e1.record(stream)
         torch.cuda.synchronize()
+    step_ms = [sev[i].elapsed_time(sev[i + 1]) for i in range(args.steps)]
+    # steps that append the last key of a block run the streaming Ward pass
+    cl = [(n0 + args.warmup + i + 1) % 512 == 0 for i in range(args.steps)]
+    plain = [m for m, f in zip(step_ms, cl) if not f]
+    clus = [m for m, f in zip(step_ms, cl) if f]
     clk = clocks.stop()
     kernels = {}
     for name in ("decode_score_kernel", "decode_resolve_kernel", "attn_kernel_split", "decode_append_kernel",
@@ -598,6 +570,9 @@ def run_decode(args):
                        "inputs": "device-drawn (torch Philox), same recipe as synth",
                        "l2": "no flush: per-step centroid scan (4.3 GB) is larger than L2"},
             "clocks": clk, "gpu_launches": int(launches), "kernels": kernels,
+            "ms_per_step_without_clustering": float(np.mean(plain)) if plain else None,
+            "ms_per_clustering_step": float(np.mean(clus)) if clus else None,
+            "clustering_steps": len(clus),
             "roofline": {"kernel": "decode step (centroid scan + gather + attention)", "bound": "hbm",
                          "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
                          "frac": achieved / pk["hbm_gbs"], "traffic": None, "peak_source": src,
@@ -606,6 +581,12 @@ def run_decode(args):
         emit_json(line)
     if world > 1:
         dist.destroy_process_group()
+
+
+def decode_prompt_len(T, warmup, steps):
+    """Prompt length after which step warmup + steps // 2 appends position
+    T - 1 (T a multiple of 512: the last key of a cluster block)."""
+    return T - 1 - warmup - steps // 2
 
 
 def ctypes_ref(x):

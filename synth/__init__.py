@@ -124,3 +124,56 @@ def query_rows(name: str, tpos, seed: int = 0) -> np.ndarray:
     for i, t in enumerate(tpos):
         out[i] = _tokens(seed, "q", int(t), int(t) + 1, c["hq"], c["d"], mu, 1.0)[0]
     return out
+
+
+# ----------------------------------------------------- device-drawn inputs
+#
+# The 1M-token and decode workloads are too large to draw on the host; they
+# use the same recipe with torch's seeded device generator (another random
+# stream than the host tensors above).  Both the benchmark and the full-size
+# tests draw through these two functions, so they see identical bytes.
+
+def device_tokens(n, heads, d, mu, scale, gen, device, out=None, chunk=65536):
+    """bf16 [n, heads, d] of scale * mu_c + N(0, I) (scale 0: N(0, 1)), c
+    uniform per (token, head), drawn by the seeded device generator `gen`."""
+    import torch
+    if out is None:
+        out = torch.empty((n, heads, d), dtype=torch.bfloat16, device=device)
+    for t0 in range(0, n, chunk):
+        t1 = min(n, t0 + chunk)
+        x = torch.randn((t1 - t0, heads, d), generator=gen, device=device, dtype=torch.float32)
+        if scale != 0.0:
+            ci = torch.randint(0, mu.shape[0], (t1 - t0, heads), generator=gen, device=device)
+            x += scale * mu[ci]
+        out[t0:t1] = x.to(torch.bfloat16)
+    return out
+
+
+def device_layer(c: dict, seed: int, device):
+    """(Q [T, hq, d], K/V [T, hkv, d]) bf16 on `device` for configuration `c`."""
+    import torch
+    gen = torch.Generator(device=device)
+    gen.manual_seed(seed)
+    mu = torch.from_numpy(centres(seed, c["n_centres"], c["d"])).to(device)
+    K = device_tokens(c["T"], c["hkv"], c["d"], mu, 4.0, gen, device)
+    V = device_tokens(c["T"], c["hkv"], c["d"], mu, 0.0, gen, device)
+    Q = device_tokens(c["T"], c["hq"], c["d"], mu, 1.0, gen, device)
+    return Q, K, V
+
+
+def device_decode(c: dict, seed: int, device, n0: int, steps: int, K_out, V_out):
+    """Decode inputs: prompts of n0 tokens per request written into
+    K_out[r, :n0] / V_out[r, :n0], then (q, k, v) for `steps` steps,
+    [steps, batch, heads, d] each."""
+    import torch
+    B, hkv, hq, d = c["batch"], c["hkv"], c["hq"], c["d"]
+    gen = torch.Generator(device=device)
+    gen.manual_seed(1000 * seed)
+    mu = torch.from_numpy(centres(seed, c["n_centres"], d)).to(device)
+    for r in range(B):
+        device_tokens(n0, hkv, d, mu, 4.0, gen, device, out=K_out[r, :n0])
+        device_tokens(n0, hkv, d, mu, 0.0, gen, device, out=V_out[r, :n0])
+    q = device_tokens(steps * B, hq, d, mu, 1.0, gen, device).view(steps, B, hq, d)
+    k = device_tokens(steps * B, hkv, d, mu, 4.0, gen, device).view(steps, B, hkv, d)
+    v = device_tokens(steps * B, hkv, d, mu, 0.0, gen, device).view(steps, B, hkv, d)
+    return q, k, v
