@@ -66,6 +66,7 @@ def parse():
     p.add_argument("--agg", default=None, choices=["mean", "max"])
     p.add_argument("--chunk", type=int, default=16384)
     p.add_argument("--T", type=int, default=None, help="prefix length of the workload (profiling runs)")
+    p.add_argument("--batch", type=int, default=None, help="decode requests (profiling runs)")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu", action="store_true")
     return p.parse_args()
@@ -75,6 +76,8 @@ def workload_cfg(args):
     c = dict(synth.CONFIGS[args.workload])
     if args.T:
         c["T"] = args.T
+    if args.batch and "batch" in c:
+        c["batch"] = args.batch
     if args.mode:
         c["mode"] = 0 if args.mode == "flat" else 1
     if args.agg:

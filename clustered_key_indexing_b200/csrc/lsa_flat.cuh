@@ -435,7 +435,6 @@ flat_cand_kernel(const __grid_constant__ CUtensorMap tmF, PassArgs a) {
         float* my_stg = stg + r * kTcStgStride;
         int2* cand = a.cand + e.orow * (int64_t)kCandCap;
         int cnt = 0;
-        uint32_t va[32], vb[32];
         // TMEM holds s - tau_add; candidates (score >= tau) are appended in
         // ascending bucket id (the thread owns its row)
         for (int it = 0; it < ntiles; ++it) {
@@ -443,9 +442,20 @@ flat_cand_kernel(const __grid_constant__ CUtensorMap tmF, PassArgs a) {
             if (!__all_sync(0xffffffffu, mbar_wait(bar.tfull(b), (uint32_t)(it >> 1) & 1u, abort_flag))) break;
             tc_fence_after();
             const uint32_t tb = trow + (uint32_t)(b * kCdBlocks * kCdCols);
-            auto chunk = [&](uint32_t (&v)[32], uint32_t (&vn)[32], int c) {
-                if (c + 1 < kCdCols / 32) tmem_ld32_async(tb + (uint32_t)((c + 1) * 32), vn);
-                group_max<G>(v);
+            uint32_t v[64];
+            tmem_ld64(tb, v);
+            // the whole tile is in registers: its TMEM buffer goes back to the
+            // MMA thread before the scan
+            tc_fence_before();
+            mbar_arrive(bar.tempty(b));
+#pragma unroll
+            for (int c = 0; c < 2; ++c) {
+                uint32_t* vv = v + 32 * c;
+#pragma unroll
+                for (int off = 1; off < G; off <<= 1)   // native: max over the query's head rows
+#pragma unroll
+                    for (int i = 0; i < 32; ++i)
+                        vv[i] = __float_as_uint(fmaxf(__uint_as_float(vv[i]), __uint_as_float(__shfl_xor_sync(0xffffffffu, vv[i], off))));
                 const int col0 = it * kCdCols + c * 32;
                 const int rem = e.ncol - col0;
                 const uint32_t lm = !e.owner || rem <= 0 ? 0u : (rem >= 32 ? 0xffffffffu : ((1u << rem) - 1u));
@@ -454,13 +464,13 @@ flat_cand_kernel(const __grid_constant__ CUtensorMap tmF, PassArgs a) {
 #pragma unroll
                 for (int i = 7; i >= 0; --i)
 #pragma unroll
-                    for (int j = 0; j < 4; ++j) sg[j] = __funnelshift_l(v[8 * j + i], sg[j], 1);
+                    for (int j = 0; j < 4; ++j) sg[j] = __funnelshift_l(vv[8 * j + i], sg[j], 1);
                 const uint32_t miss = sg[0] | (sg[1] << 8) | (sg[2] << 16) | (sg[3] << 24);
                 uint32_t hits = (tau_inf ? 0xffffffffu : ~miss) & lm;
                 if (__any_sync(0xffffffffu, hits)) {
 #pragma unroll
                     for (int j = 0; j < 8; ++j)
-                        reinterpret_cast<uint4*>(my_stg)[j] = make_uint4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+                        reinterpret_cast<uint4*>(my_stg)[j] = make_uint4(vv[4 * j], vv[4 * j + 1], vv[4 * j + 2], vv[4 * j + 3]);
                     while (hits) {
                         const int i = __ffs(hits) - 1;
                         hits &= hits - 1u;
@@ -468,14 +478,7 @@ flat_cand_kernel(const __grid_constant__ CUtensorMap tmF, PassArgs a) {
                         ++cnt;
                     }
                 }
-                if (c + 1 < kCdCols / 32) tmem_wait_ld(vn);
-            };
-            tmem_ld32_async(tb, va);
-            tmem_wait_ld(va);
-            chunk(va, vb, 0);
-            chunk(vb, va, 1);
-            tc_fence_before();
-            mbar_arrive(bar.tempty(b));
+            }
         }
         if (e.owner) a.cand_n[e.orow] = cnt;
     }
