@@ -202,6 +202,24 @@ def torch_int16():
     return torch.int16
 
 
+def max_over_ranks(ms, world, dev=None):
+    """The slowest rank's time: every rank takes this one collective, in the
+    same place (weak scaling, one independent layer or batch per rank)."""
+    if world == 1:
+        return ms
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([ms], dtype=torch.float64, device=dev if dev is not None else "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_rate(world, units_per_rank, ms_per_step):
+    """Whole-job throughput: the units all ranks processed per second, timed
+    by the slowest rank."""
+    return world * units_per_rank / (ms_per_step / 1e3)
+
+
 def dist_setup(args):
     import torch
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -355,15 +373,12 @@ def run_lsa(args):
     clk = clocks.stop()
     launches = lib().lsa_launch_count() - n0
     fallback_rows = int(lib().lsa_fallback_rows())
-    ms = ev0.elapsed_time(ev1)
+    ms = max_over_ranks(ev0.elapsed_time(ev1), world, dev)
     if world > 1:
-        tt = torch.tensor([ms], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms = float(tt.item())
         dist.barrier()
     lsa.check_device_error()
     ms_step = ms / args.steps
-    value = world * T / (ms_step / 1e3)
+    value = job_rate(world, T, ms_step)
 
     # e2e: the whole-layer C-ABI call from pinned host buffers
     e2e = None
@@ -389,12 +404,8 @@ def run_lsa(args):
             e2e_step()
         e1.record(stream)
         torch.cuda.synchronize()
-        ems = e0.elapsed_time(e1)
-        if world > 1:
-            tt = torch.tensor([ems], device=dev)
-            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-            ems = float(tt.item())
-        e2e = {"value": world * T / (ems / args.steps / 1e3), "unit": UNIT,
+        ems = max_over_ranks(e0.elapsed_time(e1), world, dev)
+        e2e = {"value": job_rate(world, T, ems / args.steps), "unit": UNIT,
                "h2d_bytes_per_step": hQ.numel() * 2 + hK.numel() * 2 + hV.numel() * 2,
                "d2h_bytes_per_step": hO.numel() * 2}
 
@@ -540,11 +551,7 @@ def run_decode(args):
         if kn:
             kernels[name] = {"ms_per_step": kms / args.steps, "launches_per_step": kn / args.steps}
     launches = lib().lsa_launch_count() - nl0
-    ms = e0.elapsed_time(e1)
-    if world > 1:
-        tt = torch.tensor([ms], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms = float(tt.item())
+    ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
     lsa.check_device_error()
     ms_step = ms / args.steps
     # algorithmic bytes per step: every eligible centroid (128 B) with its
@@ -563,8 +570,8 @@ def run_decode(args):
     achieved = byts / (ms_step / 1e3) / 1e9
     if rank == 0:
         line = {
-            "metric": "LSA decode steps/s", "value": world / (ms_step / 1e3), "unit": "steps/s",
-            "tokens_per_s": world * B / (ms_step / 1e3), "n_gpus": world, "steps": args.steps,
+            "metric": "LSA decode steps/s", "value": job_rate(world, 1, ms_step), "unit": "steps/s",
+            "tokens_per_s": job_rate(world, B, ms_step), "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": {"workload": args.workload, "batch": B, "context": T, "hkv": hkv, "hq": hq,

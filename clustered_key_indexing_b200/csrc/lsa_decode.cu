@@ -16,13 +16,14 @@
 //   query latents, then flat (decode_score_kernel + decode_resolve_kernel)
 //                          or tree (tree_warp_kernel) selection;
 //   attn_kernel<8>         eight warps share each (request, kv-head) row.
-// Flat scores: one HBM pass over the request's eligible centroids (one lane
-// per centroid, fp32 dot products) storing each slot's score bin (2048 bins
-// of width >= 2e over the row's score range) and key weight; then one CTA per
-// row: weighted histogram of the bins, the two bins around the k-th key kept
-// (warp-ordered compaction), exact fp64 rescoring, weighted radix select, key
-// emission in bucket-id order.  Rows whose kept bins overflow shared memory
-// take exact fp64 scores of every eligible bucket in a global slot.
+// Flat scores: one HBM pass over the request's eligible centroids (TMA into a
+// shared-memory ring, mma.sync bf16 scores with fp32 accumulation) storing
+// each slot's score bin (2048 bins of width >= 2e over the row's score range)
+// and key weight; then one CTA per row: weighted histogram of the bins, the
+// two bins around the k-th key kept (warp-ordered compaction), exact fp64
+// rescoring, weighted radix select, key emission in bucket-id order.  Rows
+// whose kept bins overflow shared memory take exact fp64 scores of every
+// eligible bucket in a global slot.
 #include <cuda_runtime.h>
 #include <stdint.h>
 
