@@ -82,6 +82,7 @@ int num_sms() {
 
 // kernels (other translation units)
 int64_t select_chunk(const lsa_cfg* cfg, int32_t hq, int32_t hkv);
+int64_t select_wave_rows(const lsa_cfg* cfg, int32_t hq, int32_t hkv);
 lsa_status launch_key_latent(const uint16_t* K, int64_t T, int32_t hkv, const float* W, int64_t unit0,
                              int64_t unit1, int64_t cap_units, double* U, cudaStream_t st);
 lsa_status launch_query_latent(const uint16_t* Q, int64_t nq, int32_t hq, int32_t hkv, const float* W,
@@ -397,7 +398,7 @@ static PrefillWs prefill_ws_layout(const lsa_cfg* cfg, int64_t chunk, int32_t hq
 static int64_t prefill_chunk(const lsa_cfg* cfg, int64_t T, int32_t hq, int32_t hkv, int64_t chunk) {
     if (chunk <= 0 || chunk > T) chunk = T;
     if (cfg->mode == 0 && hkv > 0 && hq > 0 && chunk < T) {
-        const int64_t sc = lsa::select_chunk(cfg, hq, hkv);
+        const int64_t sc = lsa::select_wave_rows(cfg, hq, hkv);
         int64_t m = (chunk + sc / 2) / sc;
         if (m < 1) m = 1;
         chunk = m * sc < T ? m * sc : T;

@@ -50,7 +50,11 @@ constexpr float kScoreErr = 1e-4f;   // bound on |fp32 score - exact score|
 //   flat_cand_kernel    512 rows (four blocks) x 64 centroids per tile, plus
 //       one K = 16 step that adds -tau to every row (A holds -tau in its first
 //       extra column, B a 1 there), so TMEM holds s - tau and a hit is a clear
-//       sign bit; hits are appended in ascending bucket id.
+//       sign bit; hits are appended in ascending bucket id.  Each epilogue
+//       thread takes a whole tile row into registers with one TMEM load, and
+//       the buffer goes back to the MMA thread before the scan.  (Two blocks
+//       of 128 columns halve the operand bytes per score but leave half the
+//       epilogue warps, which then bound the kernel.)
 constexpr uint32_t kTcABytes = 128 * kDL * 2;      // one M = 128 block of latents, 128-byte swizzle
 constexpr uint32_t kTcAxBytes = 128 * 16 * 2;      // extra K = 16 of a block, no swizzle
 constexpr int kHBins = 256;                        // sample histogram bins per row (16-bit counts)
@@ -63,7 +67,7 @@ constexpr uint32_t kSmHistBytes = kHBins / 2 * kSmRows * 4;  // [bin / 2][row] w
 constexpr size_t kSmSmemBytes = 1024 + kSmBlocks * kTcABytes + kSmStages * kSmBBytes + kSmHistBytes + 256;
 static_assert(kSmSmemBytes <= 232448, "flat_sample_kernel shared memory");
 
-constexpr int kCdBlocks = 4, kCdCols = 64, kCdStages = 4;
+constexpr int kCdBlocks = 4, kCdCols = 64, kCdStages = 4;  // the epilogue scans a tile as two 32-column halves
 constexpr int kCdRows = 128 * kCdBlocks;
 constexpr int kCdThreads = 64 + kCdRows;
 constexpr uint32_t kCdBBytes = kCdCols * kDL * 2;
@@ -73,6 +77,7 @@ constexpr uint32_t kCdStgBytes = kCdRows * kTcStgStride * 4;
 constexpr size_t kCdSmemBytes = 1024 + kCdBlocks * (kTcABytes + kTcAxBytes) + kCdStages * kCdBBytes + kCdBxBytes +
                                 kCdStgBytes + 256;
 static_assert(kCdSmemBytes <= 232448, "flat_cand_kernel shared memory");
+static_assert(kCdCols == 64, "flat_cand_kernel epilogue: one 64-column TMEM load per tile");
 static_assert(2 * kSmBlocks * kSmCols <= 512 && 2 * kCdBlocks * kCdCols <= 512, "TMEM columns");
 
 struct PassArgs {

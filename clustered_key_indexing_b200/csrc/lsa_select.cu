@@ -589,15 +589,19 @@ struct SelectPlan {
 // per (512 / G latent rows, kv-head), so a chunk of a multiple of
 // num_sms / gcd(num_sms, hkv) CTA row blocks fills whole waves; candidate
 // lists (kCandCap x 8 bytes per query and kv-head) stay within 2 GiB.
-int64_t select_chunk(const lsa_cfg* cfg, int32_t hq, int32_t hkv) {
+int64_t select_wave_rows(const lsa_cfg* cfg, int32_t hq, int32_t hkv) {
     const int64_t qpt = kCdRows / (cfg->agg ? hq / hkv : 1);
     int64_t g = num_sms(), x = hkv;
     while (x) { const int64_t y = g % x; g = x; x = y; }
-    const int64_t unit = num_sms() / g;
-    const int64_t per_block = qpt * hkv * (int64_t)kCandCap * 8;
-    int64_t m = ((int64_t)2 << 30) / per_block / unit;
+    return qpt * (num_sms() / g);
+}
+
+int64_t select_chunk(const lsa_cfg* cfg, int32_t hq, int32_t hkv) {
+    const int64_t wave = select_wave_rows(cfg, hq, hkv);
+    const int64_t per_wave = wave * hkv * (int64_t)kCandCap * 8;
+    int64_t m = ((int64_t)2 << 30) / per_wave;
     if (m < 1) m = 1;
-    return qpt * unit * m;
+    return wave * m;
 }
 
 static SelectPlan plan_select(const lsa_cfg* cfg, int64_t nq, int32_t hq, int32_t hkv, int64_t NB) {
