@@ -61,7 +61,7 @@ def parse():
     p.add_argument("--warmup", type=int, default=3)
     p.add_argument("--impl", default="lsa", choices=["lsa", "reference"])
     p.add_argument("--workload", default="prefill-128k",
-                   choices=["prefill-4k", "prefill-128k", "prefill-1m", "decode-32x1m"])
+                   choices=["prefill-4k", "prefill-128k", "prefill-1m", "decode-32x1m", "decode-4x10m"])
     p.add_argument("--mode", default=None, choices=["flat", "tree"])
     p.add_argument("--agg", default=None, choices=["mean", "max"])
     p.add_argument("--chunk", type=int, default=16384)
@@ -508,11 +508,20 @@ def run_decode(args):
     nsteps = args.warmup + args.steps
     n0 = decode_prompt_len(T, args.warmup, args.steps)
     cap = -(-(n0 + nsteps) // 512) * 512
-    dec = lsa.Decode(B, hkv, hq, cap, cfg, device=dev)
     Wk_np, Wq_np = synth.projections(rank, c["d"], c["dl"])
     Wk, Wq = torch.from_numpy(Wk_np).to(dev), torch.from_numpy(Wq_np).to(dev)
     ccfg = cfg.c()
-    q, kk, vv = synth.device_decode(c, rank, dev, n0, nsteps, dec.K, dec.V)
+    if c.get("shared_prefix"):
+        # one shared K/V for the prompt's whole blocks but the last, every
+        # request's own tokens after it
+        sl = 512 * ((n0 - 512) // 512)
+        shared = synth.device_shared_prefix(c, rank, dev, sl)
+        dec = lsa.Decode(B, hkv, hq, cap, cfg, device=dev, shared=shared)
+        q, kk, vv = synth.device_decode_tails(c, rank, dev, sl, n0, nsteps, dec.K, dec.V)
+    else:
+        sl = 0
+        dec = lsa.Decode(B, hkv, hq, cap, cfg, device=dev)
+        q, kk, vv = synth.device_decode(c, rank, dev, n0, nsteps, dec.K, dec.V)
     for r in range(B):
         check(lib().lsa_decode_load(ctypes_ref(dec.d), r, n0, ctypes_ptr(Wk), ctypes_ref(ccfg),
                                     ctypes_ptr(dec.ws), dec.ws.numel(), None), "lsa_decode_load")
@@ -545,8 +554,8 @@ def run_decode(args):
     clus = [m for m, f in zip(step_ms, cl) if f]
     clk = clocks.stop()
     kernels = {}
-    for name in ("decode_score_kernel", "decode_resolve_kernel", "attn_kernel_split", "decode_append_kernel",
-                 "latent_kernel", "ward_kernel", "tree_select_kernel"):
+    for name in ("decode_score_kernel", "decode_keep_kernel", "decode_resolve_kernel", "attn_kernel_split",
+                 "decode_append_kernel", "latent_kernel", "ward_kernel", "tree_select_kernel"):
         kms, kn = kt.get(name)
         if kn:
             kernels[name] = {"ms_per_step": kms / args.steps, "launches_per_step": kn / args.steps}
@@ -554,9 +563,16 @@ def run_decode(args):
     ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
     lsa.check_device_error()
     ms_step = ms / args.steps
-    # algorithmic bytes per step: every eligible centroid (128 B) with its
-    # minlr word, the gathered K/V rows of every index entry (512 B), Q and O
+    # algorithmic bytes per step: the centroids the search must read (128 B,
+    # with a 4-byte record) -- flat: every eligible bucket; tree: the children
+    # of the beam at every level above L* plus the B * 2^L* leaves under the
+    # final beam -- the gathered K/V rows of every index entry (512 B), Q and O
     row = cfg.row
+    if cfg.mode == 1:
+        lstar = 0
+        while c["beam"] * 8 * (1 << lstar) < c["k"]:
+            lstar += 1
+        tree_nodes = 2 * c["beam"] * (dec.tree.levels - 1 - lstar) + c["beam"] * (1 << lstar)
     byts = 0.0
     for t in lens0:
         for s_ in range(args.steps):
@@ -564,6 +580,8 @@ def run_decode(args):
             lim = pos - c["window"]
             nb = min(cap // 512 * 64, 64 * (lim // 512 + 1))
             nb = min(nb, 64 * ((pos + 1) // 512))
+            if cfg.mode == 1:
+                nb = min(nb, tree_nodes)
             byts += hkv * (nb * 132 + row * 512) + 2 * hq * c["d"] * 2
     byts /= args.steps
     pk, src = peaks()
@@ -574,11 +592,11 @@ def run_decode(args):
             "tokens_per_s": job_rate(world, B, ms_step), "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": args.workload, "batch": B, "context": T, "hkv": hkv, "hq": hq,
+            "config": {"workload": args.workload, "batch": B, "context": T, "shared_prefix": sl, "hkv": hkv, "hq": hq,
                        "k": c["k"], "sinks": c["sinks"], "window": c["window"],
                        "search": "flat" if c["mode"] == 0 else f"tree(beam={c['beam']})",
                        "inputs": "device-drawn (torch Philox), same recipe as synth",
-                       "l2": "no flush: per-step centroid scan (4.3 GB) is larger than L2"},
+                       "l2": f"no flush: per-step centroid scan ({byts / 1e9:.1f} GB) is larger than L2"},
             "clocks": clk, "gpu_launches": int(launches), "kernels": kernels,
             "ms_per_step_without_clustering": float(np.mean(plain)) if plain else None,
             "ms_per_clustering_step": float(np.mean(clus)) if clus else None,

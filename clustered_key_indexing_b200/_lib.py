@@ -44,7 +44,8 @@ MAX_BATCH = 128
 
 class lsa_decode(ctypes.Structure):
     _fields_ = [("batch", i32), ("hkv", i32), ("hq", i32), ("cap", i64), ("K", vp), ("V", vp),
-                ("U_blk", vp), ("cache", lsa_cache), ("tree", lsa_tree), ("len", i64 * MAX_BATCH)]
+                ("U_blk", vp), ("cache", lsa_cache), ("tree", lsa_tree), ("len", i64 * MAX_BATCH),
+                ("K_shared", vp), ("V_shared", vp), ("shared_len", i64)]
 
 
 class LSAError(RuntimeError):

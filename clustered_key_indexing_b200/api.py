@@ -245,19 +245,28 @@ class Decode:
     (request, kv-head) pairs, the per-request block ring, and (tree mode) the
     tree.  `load` installs a prompt, `step` decodes one token per request."""
 
-    def __init__(self, batch: int, hkv: int, hq: int, cap: int, cfg: Config, device="cuda"):
+    def __init__(self, batch: int, hkv: int, hq: int, cap: int, cfg: Config, device="cuda", shared=None):
+        """`shared`: optional (K_shared, V_shared) [shared_len, hkv, 128], a
+        prefix every request starts with (shared_len a multiple of 512); the
+        pools then hold each request's tokens from shared_len on."""
         if cap % 512:
             raise ValueError("cap must be a multiple of 512")
         self.cfg = cfg
         z = dict(device=device)
-        self.K = torch.zeros((batch, cap, hkv, 128), dtype=torch.bfloat16, **z)
-        self.V = torch.zeros((batch, cap, hkv, 128), dtype=torch.bfloat16, **z)
+        self.shared = shared
+        sl = 0 if shared is None else int(shared[0].shape[0])
+        self.shared_len = sl
+        self.K = torch.zeros((batch, cap - sl, hkv, 128), dtype=torch.bfloat16, **z)
+        self.V = torch.zeros((batch, cap - sl, hkv, 128), dtype=torch.bfloat16, **z)
         self.U_blk = torch.zeros((batch * hkv, 128, 64), dtype=torch.float64, **z)
         self.cache = Cache(batch * hkv, cap, cfg, device=device, with_units=False)
         self.tree = Tree(self.cache, device=device) if cfg.mode == 1 else None
         d = _lib.lsa_decode()
         d.batch, d.hkv, d.hq, d.cap = batch, hkv, hq, cap
         d.K, d.V, d.U_blk = self.K.data_ptr(), self.V.data_ptr(), self.U_blk.data_ptr()
+        if shared is not None:
+            _need_cuda(*shared)
+            d.K_shared, d.V_shared, d.shared_len = shared[0].data_ptr(), shared[1].data_ptr(), sl
         d.cache = self.cache.c
         if self.tree is not None:
             d.tree = self.tree.t
@@ -272,12 +281,14 @@ class Decode:
         return [int(self.d.len[i]) for i in range(self.d.batch)]
 
     def load(self, r: int, K: torch.Tensor, V: torch.Tensor, W_k: torch.Tensor, stream=None):
-        """Install a prompt (K/V [n, hkv, 128]) as request r."""
+        """Install a prompt as request r: K/V [n, hkv, 128], or with a shared
+        prefix the prompt's tokens after it (the prompt holds shared_len + n)."""
         n = K.shape[0]
         self.K[r, :n].copy_(K)
         self.V[r, :n].copy_(V)
-        check(lib().lsa_decode_load(ctypes.byref(self.d), r, n, _ptr(W_k), ctypes.byref(self.cfg.c()),
-                                    _ptr(self.ws), self.ws.numel(), _stream(stream)), "lsa_decode_load")
+        check(lib().lsa_decode_load(ctypes.byref(self.d), r, self.shared_len + n, _ptr(W_k),
+                                    ctypes.byref(self.cfg.c()), _ptr(self.ws), self.ws.numel(), _stream(stream)),
+              "lsa_decode_load")
 
     def step(self, q, k, v, W_k, W_q, o=None, idx_out=None, stream=None):
         """One token per request: q [batch, hq, 128], k/v [batch, hkv, 128]."""

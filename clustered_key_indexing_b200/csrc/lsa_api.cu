@@ -98,7 +98,7 @@ lsa_status run_select(const uint16_t* Q, int64_t t0, int64_t nq, int32_t hq, con
 lsa_status launch_attn(const uint16_t* Q, const uint16_t* K, const uint16_t* V, const int32_t* idx,
                        int64_t nq, int32_t hq, int32_t hkv, int32_t n_idx, int64_t T, uint16_t* O,
                        cudaStream_t st, int64_t kv_q_stride, int split, int32_t n_use, const float* Ow,
-                       const float* lse);
+                       const float* lse, const uint16_t* Ks, const uint16_t* Vs, int64_t shared_len);
 lsa_status launch_band_attn(const uint16_t* Q, const uint16_t* K, const uint16_t* V, int64_t nq, int64_t t0,
                             int64_t T, int32_t hq, int32_t hkv, int32_t S, int32_t W, float* Ow, float* lse,
                             cudaStream_t st);
@@ -341,7 +341,8 @@ lsa_status lsa_sparse_attn(const uint16_t* Q, const uint16_t* K, const uint16_t*
     if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O))
         return set_error(LSA_EINVAL, "lsa_sparse_attn: Q, K, V, O must be 16-byte aligned");
     if (T > (int64_t)INT32_MAX) return set_error(LSA_EUNSUPPORTED, "lsa_sparse_attn: T beyond 2^31");
-    return launch_attn(Q, K, V, idx, nq, hq, hkv, n_idx, T, O, (cudaStream_t)stream, 0, 1, -1, nullptr, nullptr);
+    return launch_attn(Q, K, V, idx, nq, hq, hkv, n_idx, T, O, (cudaStream_t)stream, 0, 1, -1, nullptr, nullptr,
+                       nullptr, nullptr, 0);
 }
 
 size_t lsa_select_attn_workspace_bytes(int64_t nq, int32_t hq) {
@@ -372,7 +373,8 @@ lsa_status lsa_select_attn(const uint16_t* Q, const uint16_t* K, const uint16_t*
     // max(S, t - W + 1) .. t: attend to it as a band, then gather the sinks
     // and long-range entries and merge the two softmax states
     if ((s = launch_band_attn(Q, K, V, nq, t0, T, hq, hkv, cfg->sinks, cfg->window, Ow, lse, st)) != LSA_OK) return s;
-    return launch_attn(Q, K, V, idx, nq, hq, hkv, row, T, O, st, 0, 1, cfg->sinks + cfg->k, Ow, lse);
+    return launch_attn(Q, K, V, idx, nq, hq, hkv, row, T, O, st, 0, 1, cfg->sinks + cfg->k, Ow, lse,
+                       nullptr, nullptr, 0);
 }
 
 

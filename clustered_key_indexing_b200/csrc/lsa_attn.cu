@@ -41,6 +41,9 @@ struct AttnArgs {
     const float* lse;     // ... and its log2-domain log-sum-exp, merged into the result
     int64_t T;            // index entries must be < T
     int64_t kv_q_stride;  // token rows of K/V per query row (decode: each request's capacity); 0 = shared
+    const uint16_t* Ks;   // decode's shared prefix [shared_len, hkv, 128] (SPLIT > 1 only) ...
+    const uint16_t* Vs;
+    int64_t shared_len;   // ... positions below it are read there; 0 = none
     uint16_t* O;
     float scale_log2;
 };
@@ -83,6 +86,8 @@ __global__ void __launch_bounds__(32 * (SPLIT == 1 ? kAttnWarps : SPLIT)) attn_k
     const int64_t kv_stride = (int64_t)a.hkv * kD;
     const uint16_t* Kg = a.K + (q * a.kv_q_stride * a.hkv + g) * kD;
     const uint16_t* Vg = a.V + (q * a.kv_q_stride * a.hkv + g) * kD;
+    const uint16_t* Ksg = SPLIT > 1 && a.shared_len > 0 ? a.Ks + (int64_t)g * kD : Kg;
+    const uint16_t* Vsg = SPLIT > 1 && a.shared_len > 0 ? a.Vs + (int64_t)g * kD : Vg;
 
     // positions of one 16-key tile: lanes l and l+16 both hold entry l
     auto tile_pos = [&](int tile) -> int {
@@ -101,9 +106,17 @@ __global__ void __launch_bounds__(32 * (SPLIT == 1 ? kAttnWarps : SPLIT)) attn_k
             for (int m = 0; m < 8; ++m) {
                 const int r = 2 * m + (lane >> 4), part = lane & 15;
                 const int pr = __shfl_sync(0xffffffffu, p, r);
-                const int64_t off = (pr >= 0 ? (int64_t)pr : 0) * kv_stride + part * 8;
-                cp_async_16(kb + swz(r, part), Kg + off, pr >= 0 ? 16 : 0);
-                cp_async_16(vb + swz(r, part), Vg + off, pr >= 0 ? 16 : 0);
+                if constexpr (SPLIT == 1) {
+                    const int64_t off = (pr >= 0 ? (int64_t)pr : 0) * kv_stride + part * 8;
+                    cp_async_16(kb + swz(r, part), Kg + off, pr >= 0 ? 16 : 0);
+                    cp_async_16(vb + swz(r, part), Vg + off, pr >= 0 ? 16 : 0);
+                } else {  // decode: the shared prefix, then the request's own rows
+                    const bool sh = pr >= 0 && pr < a.shared_len;
+                    const int64_t row = pr < 0 ? 0 : (sh ? (int64_t)pr : (int64_t)pr - a.shared_len);
+                    const int64_t off = row * kv_stride + part * 8;
+                    cp_async_16(kb + swz(r, part), (sh ? Ksg : Kg) + off, pr >= 0 ? 16 : 0);
+                    cp_async_16(vb + swz(r, part), (sh ? Vsg : Vg) + off, pr >= 0 ? 16 : 0);
+                }
             }
         }
         cp_async_commit();
@@ -299,11 +312,13 @@ __global__ void __launch_bounds__(32 * (SPLIT == 1 ? kAttnWarps : SPLIT)) attn_k
 }
 
 // n_use < 0: every entry of each list; Ow / lse: optional partial state of
-// other keys to merge (prefill: the sliding window, from the band kernel).
+// other keys to merge (prefill: the sliding window, from the band kernel);
+// Ks / Vs / shared_len: decode's shared prefix (positions below shared_len
+// read Ks / Vs, the others row p - shared_len of the query row's own K / V).
 lsa_status launch_attn(const uint16_t* Q, const uint16_t* K, const uint16_t* V, const int32_t* idx,
                        int64_t nq, int32_t hq, int32_t hkv, int32_t n_idx, int64_t T, uint16_t* O,
-                       cudaStream_t st, int64_t kv_q_stride = 0, int split = 1, int32_t n_use = -1,
-                       const float* Ow = nullptr, const float* lse = nullptr) {
+                       cudaStream_t st, int64_t kv_q_stride, int split, int32_t n_use, const float* Ow,
+                       const float* lse, const uint16_t* Ks, const uint16_t* Vs, int64_t shared_len) {
     if (nq <= 0) return LSA_OK;
     AttnArgs a{};
     a.Q = Q; a.K = K; a.V = V; a.idx = idx; a.nq = nq; a.hq = hq; a.hkv = hkv; a.n_idx = n_idx;
@@ -311,6 +326,8 @@ lsa_status launch_attn(const uint16_t* Q, const uint16_t* K, const uint16_t* V, 
     a.Ow = split == 1 ? Ow : nullptr;
     a.lse = split == 1 ? lse : nullptr;
     a.T = T; a.O = O; a.kv_q_stride = kv_q_stride;
+    if (split == 1 && shared_len > 0) return set_error(LSA_EUNSUPPORTED, "attention: shared prefix is decode only");
+    a.Ks = Ks; a.Vs = Vs; a.shared_len = shared_len;
     a.scale_log2 = 1.4426950408889634f / sqrtf((float)kD);
     const int64_t rows = nq * hkv;
     if (split == 1) {

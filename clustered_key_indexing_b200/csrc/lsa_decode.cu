@@ -47,7 +47,7 @@ lsa_status launch_tree_update(const lsa_cache* c, lsa_tree* t, int64_t b0, int64
 lsa_status launch_attn(const uint16_t* Q, const uint16_t* K, const uint16_t* V, const int32_t* idx,
                        int64_t nq, int32_t hq, int32_t hkv, int32_t n_idx, int64_t T, uint16_t* O,
                        cudaStream_t st, int64_t kv_q_stride, int split, int32_t n_use, const float* Ow,
-                       const float* lse);
+                       const float* lse, const uint16_t* Ks, const uint16_t* Vs, int64_t shared_len);
 
 // ------------------------------------------------------------- key latent
 
@@ -72,15 +72,19 @@ __device__ __forceinline__ void latent_row(const double* krow, const float* __re
     z1 = nrm > 0.0 ? __ddiv_rn(v1, nrm) : 0.0;
 }
 
+constexpr int kDecBins = 2048;       // histogram bins over the row's score range
+
 struct AppendArgs {
     const uint16_t* k;   // [batch, hkv, 128] new keys
     const uint16_t* v;   // [batch, hkv, 128] new values
-    uint16_t* K;         // [batch, cap, hkv, 128]
+    uint16_t* K;         // [batch, tail, hkv, 128] (tail = cap - shared_len)
     uint16_t* V;
     const float* W;      // W_k [128, 64]
     double* U_blk;       // [batch * hkv, 128, 64]
-    int64_t cap;
+    int64_t tail, shared_len;
     int32_t hkv, batch;
+    uint32_t* hist;      // flat search: [batch * hkv, kDecBins] zeroed here for this step's scores ...
+    unsigned long long* tot;  // ... and [batch * hkv] row totals
     int64_t pos[LSA_MAX_BATCH];
 };
 
@@ -92,9 +96,13 @@ __global__ void __launch_bounds__(256) decode_append_kernel(AppendArgs a) {
     if (w >= (int64_t)a.batch * a.hkv) return;
     const int64_t r = w / a.hkv, h = w % a.hkv;
     const int64_t t = a.pos[r];
+    if (a.hist) {
+        for (int i = lane; i < kDecBins; i += 32) a.hist[w * kDecBins + i] = 0u;
+        if (lane == 0) a.tot[w] = 0ull;
+    }
     const uint16_t* ks = a.k + w * kD;
     const uint16_t* vs = a.v + w * kD;
-    const int64_t dst = ((r * a.cap + t) * a.hkv + h) * kD;
+    const int64_t dst = ((r * a.tail + (t - a.shared_len)) * a.hkv + h) * kD;
     if (lane < 16) {
         reinterpret_cast<uint4*>(a.K + dst)[lane] = reinterpret_cast<const uint4*>(ks)[lane];
         reinterpret_cast<uint4*>(a.V + dst)[lane] = reinterpret_cast<const uint4*>(vs)[lane];
@@ -121,7 +129,7 @@ __global__ void __launch_bounds__(256) decode_append_kernel(AppendArgs a) {
 __global__ void __launch_bounds__(256) tail_units_kernel(const uint16_t* __restrict__ K,
                                                          const float* __restrict__ W, double* U_blk,
                                                          int64_t n, int64_t j0, int64_t j1, int32_t hkv,
-                                                         int64_t head0) {
+                                                         int64_t head0, int64_t row0) {
     __shared__ double krow[8][kD];
     const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
     const int64_t w = (int64_t)blockIdx.x * 8 + wid;
@@ -130,7 +138,7 @@ __global__ void __launch_bounds__(256) tail_units_kernel(const uint16_t* __restr
     double s0 = 0.0, s1 = 0.0;
     int cnt = 0;
     for (int64_t t = j * kPool; t < j * kPool + kPool && t < n; ++t) {
-        const uint16_t* ks = K + (t * hkv + h) * kD;
+        const uint16_t* ks = K + ((t - row0) * hkv + h) * kD;   // K holds positions row0 ..
         __syncwarp();
         for (int e = lane; e < kD; e += 32) krow[wid][e] = bf16_to_f64(ks[e]);
         __syncwarp();
@@ -151,7 +159,6 @@ __global__ void __launch_bounds__(256) tail_units_kernel(const uint16_t* __restr
 
 // ------------------------------------------------------ flat decode scores
 
-constexpr int kDecBins = 2048;       // histogram bins over the row's score range
 
 struct DecScoreArgs {
     const uint16_t* Y;        // [batch, hkv, 64] (mean) / [batch, hq, 64] (native)
@@ -161,10 +168,12 @@ struct DecScoreArgs {
     const int32_t* cnt_lr;
     const int32_t* units;
     int64_t cap_buckets, ld;
-    int32_t hkv, G, agg, S, W;
+    int32_t hkv, G, agg, S, W, k;
     int64_t T_built;
     uint16_t* bin;            // [rows, ld] score bin of every slot
     uint8_t* wt;              // [rows, ld] keys of the slot in [S, t-W] (0 = not eligible)
+    uint32_t* hist;           // [rows, kDecBins] key weight per bin (zeroed by the append kernel)
+    unsigned long long* tot;  // [rows] key weight of the row (zeroed by the append kernel)
     int64_t pos[LSA_MAX_BATCH];
 };
 
@@ -197,6 +206,49 @@ __device__ __forceinline__ int score_to_bin(float s, float R) {
     return bin < 0 ? 0 : (bin >= kDecBins ? kDecBins - 1 : bin);
 }
 
+// Cut of a key-weight histogram h (kDecBins bins in shared memory, bin
+// kDecBins - 1 the highest scores), computed by all 128 threads of a block
+// (each sums 16 bins, then a block scan): returns j - 1 (not below 0) for the
+// highest bin j whose weight counted from the top reaches k, and in *tot the
+// histogram's total weight.  Every slot in bins >= j - 1 is kept for exact
+// rescoring: the k-th key's exact score lies in bin j or j - 1 (bins are at
+// least 2e wide).  Contains __syncthreads: every thread of the block calls it.
+__device__ int dec_cut_block(const uint32_t* h, int64_t k, long long* tot) {
+    __shared__ long long wsum[4];
+    __shared__ int s_j;
+    const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+    const int top = kDecBins - 1 - 16 * tid;  // this thread's bins: top, top - 1, .., top - 15
+    long long s = 0;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) s += (long long)h[top - i];
+    long long incl = s;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const long long y = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += y;
+    }
+    if (lane == 31) wsum[wid] = incl;
+    if (tid == 0) s_j = 1;  // no bin reaches k: cut 0
+    __syncthreads();
+    for (int i = 0; i < wid; ++i) incl += wsum[i];
+    const long long all = wsum[0] + wsum[1] + wsum[2] + wsum[3];
+    const long long excl = incl - s;
+    if (excl < k && incl >= k) {
+        long long cum = excl;
+        int j = top;
+        for (int i = 0; i < 16; ++i) {
+            cum += (long long)h[top - i];
+            if (cum >= k) { j = top - i; break; }
+        }
+        s_j = j;
+    }
+    __syncthreads();
+    const int j = s_j;
+    __syncthreads();  // s_j and wsum are reused by the next call
+    *tot = all;
+    return j > 0 ? j - 1 : 0;
+}
+
 // grid (column chunks, rows), 4 warps.  The chunk's centroids stream through
 // a 3-stage shared-memory ring of 256-row tiles (TMA, 128-byte swizzle, one
 // thread issues; bounded mbarrier waits, no multicast).  Each warp scores 64
@@ -205,7 +257,7 @@ __device__ __forceinline__ int score_to_bin(float s, float R) {
 // to the max over latents, binned, and the tile's bins and weights are
 // written with coalesced stores (weights from cnt_lr, and below the frontier
 // block no minlr / maxpos reads: those buckets lie wholly in [S, t - W]).
-constexpr int kDecScanCols = 4096;   // bucket slots per CTA
+constexpr int kDecScanCols = 16384;   // bucket slots per CTA
 constexpr int kDecTile = 256;        // centroids per ring stage (32 KB)
 constexpr int kDecStages = 3;
 constexpr size_t kDecScanSmem = 1024 + (size_t)kDecStages * kDecTile * kDL * 2 + kDecTile * 4 + 64;
@@ -219,6 +271,7 @@ __global__ void __launch_bounds__(128) decode_score_kernel(const __grid_constant
     uint64_t* bars = reinterpret_cast<uint64_t*>(best_s + kDecTile);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + kDecStages);
     __shared__ float rad;
+    __shared__ uint32_t shist[kDecBins];  // key weight per score bin over this CTA's slots
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int64_t row = blockIdx.y;
     const int64_t r = row / a.hkv;
@@ -230,6 +283,7 @@ __global__ void __launch_bounds__(128) decode_score_kernel(const __grid_constant
     const int64_t cend = min(ncol, c0 + kDecScanCols);
     const int ntiles = (int)((cend - c0 + kDecTile - 1) / kDecTile);
     const uint32_t bar0 = smem_u32(bars);
+    for (int i = tid; i < kDecBins; i += 128) shist[i] = 0u;
     if (tid == 0) {
         for (int s = 0; s < kDecStages; ++s) mbar_init(bar0 + 8u * s, 1);
         *abort_flag = 0;
@@ -313,8 +367,10 @@ __global__ void __launch_bounds__(128) decode_score_kernel(const __grid_constant
                 if ((int64_t)mlr <= lim)
                     w = (int64_t)mxp <= lim ? clr : weight_units(b, __ldg(a.units + hb0 + b), lim, a.S, a.T_built);
             }
-            a.bin[row * a.ld + b] = (uint16_t)score_to_bin(best_s[j], R);
+            const int bn = score_to_bin(best_s[j], R);
+            a.bin[row * a.ld + b] = (uint16_t)bn;
             a.wt[row * a.ld + b] = (uint8_t)w;
+            if (w > 0) atomicAdd(&shist[bn], (uint32_t)w);
         }
         __syncthreads();  // best_s is rewritten by the next tile
         done = it + 1;
@@ -324,6 +380,116 @@ __global__ void __launch_bounds__(128) decode_score_kernel(const __grid_constant
         const int issued = min(ntiles, done + kDecStages);
         for (int i = done; i < issued; ++i)
             mbar_wait(bar0 + 8u * (i % kDecStages), (uint32_t)(i / kDecStages) & 1u, abort_flag, false);
+    }
+    // The CTA's bin weights into the row's histogram, from its own cut bin
+    // down by one: the row's cut bin j (where the weight from the top reaches
+    // k) is at or above every CTA's, so the row histogram is exact on every
+    // bin >= j - 1, the only bins the cut and the kept slots read.  The
+    // total weight goes into the row total.
+    __syncthreads();
+    long long tc;
+    const int jc = dec_cut_block(shist, a.k, &tc);
+    if (tid == 0 && tc) atomicAdd(a.tot + row, (unsigned long long)tc);
+    for (int i = jc + tid; i < kDecBins; i += 128)
+        if (shist[i]) atomicAdd(a.hist + row * kDecBins + i, shist[i]);
+}
+
+// ------------------------------------------------------ flat decode cut
+
+// Slots of chunk [c0, c0 + kDecScanCols) of a row with a key in [S, t - W]
+// and a bin >= the row's cut, in ascending id, into the chunk's segment
+// (kCap ids; the count is stored whole, so an overflow shows).  grid
+// (chunks, rows), 4 warps; warp w takes a contiguous quarter of the chunk.
+struct DecKeepArgs {
+    const uint32_t* hist;    // [rows, kDecBins]
+    const unsigned long long* tot;  // [rows]
+    const uint16_t* bin;     // [rows, ld]
+    const uint8_t* wt;       // [rows, ld]
+    int32_t* seg;            // [rows, nch, kCap]
+    int32_t* segn;           // [rows, nch]
+    int64_t ld, cap_buckets, nch;
+    int32_t hkv, k, S, W;
+    int64_t pos[LSA_MAX_BATCH];
+};
+
+__device__ __forceinline__ int64_t dec_ncol(int64_t t, int32_t S, int32_t W, int64_t cap_buckets) {
+    const int64_t lim = t - W;
+    if (lim < S) return 0;
+    return min(cap_buckets, (int64_t)kBucketsPerBlock * (lim / kBlockKeys + 1));
+}
+
+__global__ void __launch_bounds__(128) decode_keep_kernel(DecKeepArgs a) {
+    __shared__ int wc[4];
+    __shared__ __align__(16) uint32_t h[kDecBins];
+    const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+    const int64_t row = blockIdx.y, chunk = blockIdx.x;
+    const int64_t ncol = dec_ncol(a.pos[row / a.hkv], a.S, a.W, a.cap_buckets);
+    int32_t* nout = a.segn + row * a.nch + chunk;
+    const int64_t c0 = chunk * (int64_t)kDecScanCols;
+    if (c0 >= ncol) {
+        if (tid == 0) *nout = 0;
+        return;
+    }
+    if ((long long)a.tot[row] <= a.k) {  // the resolve takes every eligible key
+        if (tid == 0) *nout = 0;
+        return;
+    }
+    for (int i = tid; i < kDecBins / 4; i += 128)
+        reinterpret_cast<uint4*>(h)[i] = reinterpret_cast<const uint4*>(a.hist + row * kDecBins)[i];
+    __syncthreads();
+    long long hsum;
+    const int jt = dec_cut_block(h, a.k, &hsum);
+    const uint16_t* brow = a.bin + row * a.ld;
+    const uint8_t* wrow = a.wt + row * a.ld;
+    auto hits16 = [&](int64_t g16) -> uint32_t {
+        const uint4 wv = *reinterpret_cast<const uint4*>(wrow + g16 * 16);
+        const uint4 bv0 = *reinterpret_cast<const uint4*>(brow + g16 * 16);
+        const uint4 bv1 = *reinterpret_cast<const uint4*>(brow + g16 * 16 + 8);
+        const uint32_t wu[4] = {wv.x, wv.y, wv.z, wv.w};
+        const uint32_t bu[8] = {bv0.x, bv0.y, bv0.z, bv0.w, bv1.x, bv1.y, bv1.z, bv1.w};
+        uint32_t m = 0;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            const uint32_t w = (wu[i >> 2] >> (8 * (i & 3))) & 0xFFu;
+            const int b = (int)((bu[i >> 1] >> (16 * (i & 1))) & 0xFFFFu);
+            m |= (uint32_t)(w > 0 && b >= jt && g16 * 16 + i < ncol) << i;
+        }
+        return m;
+    };
+    const int64_t g0 = c0 / 16, g1 = (min(ncol, c0 + (int64_t)kDecScanCols) + 15) / 16;
+    const int64_t per = (g1 - g0 + 3) / 4;
+    const int64_t g_lo = g0 + wid * per, g_hi = min(g1, g_lo + per);
+    int c = 0;
+    for (int64_t g = g_lo + lane; g < g_hi; g += 32) c += __popc(hits16(g));
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) c += __shfl_xor_sync(0xffffffffu, c, off);
+    if (lane == 0) wc[wid] = c;
+    __syncthreads();
+    int base = 0, total = 0;
+    for (int i = 0; i < 4; ++i) {
+        if (i < wid) base += wc[i];
+        total += wc[i];
+    }
+    if (tid == 0) *nout = total;
+    if (total > kCap) return;  // the resolve falls back to exact scores
+    int32_t* out = a.seg + (row * a.nch + chunk) * (int64_t)kCap;
+    for (int64_t s0 = g_lo; s0 < g_hi; s0 += 32) {
+        const int64_t g = s0 + lane;
+        uint32_t m = g < g_hi ? hits16(g) : 0u;
+        const int nh = __popc(m);
+        int incl = nh;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, incl, off);
+            if (lane >= off) incl += y;
+        }
+        int o = base + incl - nh;
+        while (m) {
+            const int i = __ffs(m) - 1;
+            m &= m - 1;
+            out[o++] = (int32_t)(g * 16 + i);
+        }
+        base += __shfl_sync(0xffffffffu, incl, 31);
     }
 }
 
@@ -336,6 +502,10 @@ struct DecResolveArgs {
     double* slot;            // [rows, ld] exact scores (fallback rows)
     int64_t ld;
     int64_t cap_buckets;
+    const unsigned long long* tot;  // [rows] key weight of the row
+    const int32_t* seg;      // [rows, nch, kCap] kept slots per chunk (decode_keep_kernel)
+    const int32_t* segn;     // [rows, nch]
+    int64_t nch;
 };
 
 __global__ void __launch_bounds__(kSelThreads) decode_resolve_kernel(DecResolveArgs d) {
@@ -353,127 +523,51 @@ __global__ void __launch_bounds__(kSelThreads) decode_resolve_kernel(DecResolveA
     load_latents(a, r, sh);
     const int ng = a.agg ? a.G : 1;
     const int64_t ncol = min(d.cap_buckets, (int64_t)kBucketsPerBlock * (r.lim / kBlockKeys + 1));
-    const uint16_t* brow = d.bin + row * d.ld;
     uint8_t* wrow = d.wt + row * d.ld;
-    // key weights per bin (32-bit counters; the candidate count comes from
-    // the compaction's own count)
-    uint32_t* h32 = reinterpret_cast<uint32_t*>(sh.hist);
-    for (int i = tid; i < kDecBins; i += kSelThreads) h32[i] = 0u;
-    __syncthreads();
-    // 16 slots per lane per step: one 16-byte load of weights, two of bins
-    auto load16 = [&](int64_t g16, uint8_t (&w16)[16], uint16_t (&b16)[16]) {
-        const uint4 wv = *reinterpret_cast<const uint4*>(wrow + g16 * 16);
-        const uint4 bv0 = *reinterpret_cast<const uint4*>(brow + g16 * 16);
-        const uint4 bv1 = *reinterpret_cast<const uint4*>(brow + g16 * 16 + 8);
-        const uint32_t wu[4] = {wv.x, wv.y, wv.z, wv.w};
-        const uint32_t bu[8] = {bv0.x, bv0.y, bv0.z, bv0.w, bv1.x, bv1.y, bv1.z, bv1.w};
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            w16[i] = (g16 * 16 + i < ncol) ? (uint8_t)((wu[i >> 2] >> (8 * (i & 3))) & 0xFF) : 0;
-            b16[i] = (uint16_t)((bu[i >> 1] >> (16 * (i & 1))) & 0xFFFF);
-        }
-    };
-    const int64_t ng16 = (ncol + 15) / 16;
-    long long myw = 0;
-#pragma unroll 4
-    for (int64_t g16 = tid; g16 < ng16; g16 += kSelThreads) {
-        uint8_t w16[16];
-        uint16_t b16[16];
-        load16(g16, w16, b16);
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            if (w16[i] == 0) continue;
-            myw += w16[i];
-            atomicAdd(&h32[b16[i]], (uint32_t)w16[i]);
-        }
-    }
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) myw += __shfl_xor_sync(0xffffffffu, myw, off);
-    __shared__ long long wsum[kSelThreads / 32];
-    if (lane == 0) wsum[wid] = myw;
-    __syncthreads();
-    long long totw = 0;
-    for (int i = 0; i < kSelThreads / 32; ++i) totw += wsum[i];
+    // the row's key weight (summed by the score kernel); the cut itself is
+    // the keep kernel's, which left the kept slots in per-chunk segments
+    const long long totw = (long long)d.tot[row];
     if (totw <= a.k) {
         emit_range(a, r, ncol, [&](int64_t b) -> int { return (int)wrow[b]; }, sh);
         return;
     }
-    // cut bin j*: highest bin whose weight from the top reaches k; keep bins >= j* - 1
-    if (tid < 32) {
-        long long s = 0;
-        for (int dd = 0; dd < kDecBins / 32; ++dd)
-            s += (long long)h32[kDecBins - 1 - (kDecBins / 32) * lane - dd];
-        long long incl = s;
+    // candidates: the keep kernel's per-chunk segments, concatenated in
+    // chunk order (ascending ids)
+    const int64_t nch = (ncol + kDecScanCols - 1) / kDecScanCols;
+    const int32_t* sn = d.segn + row * d.nch;
+    int my = 0;
+    for (int64_t c = tid; c < nch; c += kSelThreads) my += sn[c];
 #pragma unroll
-        for (int off = 1; off < 32; off <<= 1) {
-            const long long y = __shfl_up_sync(0xffffffffu, incl, off);
-            if (lane >= off) incl += y;
-        }
-        const long long excl = incl - s;
-        const unsigned mask = __ballot_sync(0xffffffffu, incl >= a.k && excl < a.k);
-        const int src = __ffs(mask) - 1;
-        if (lane == src) {
-            long long cum = excl;
-            int j = kDecBins - 1 - (kDecBins / 32) * lane;
-            for (int dd = 0; dd < kDecBins / 32; ++dd) {
-                const int jj = kDecBins - 1 - (kDecBins / 32) * lane - dd;
-                cum += (long long)h32[jj];
-                if (cum >= a.k) { j = jj; break; }
-            }
-            sh.misc[0] = j > 0 ? j - 1 : 0;
-        }
-    }
-    __syncthreads();
-    const int jt = sh.misc[0];
-    // warp-ordered compaction: warp w takes a contiguous quarter of the
-    // 16-slot groups and lane l the l-th group of each 512-slot stretch, so
-    // the concatenated lists keep ascending ids; first each warp's count
-    const int64_t per = (ng16 + kSelThreads / 32 - 1) / (kSelThreads / 32);
-    const int64_t g_lo = wid * per, g_hi = min(ng16, g_lo + per);
-    {
-        int c = 0;
-#pragma unroll 4
-        for (int64_t g16 = g_lo + lane; g16 < g_hi; g16 += 32) {
-            uint8_t w16[16];
-            uint16_t b16[16];
-            load16(g16, w16, b16);
-#pragma unroll
-            for (int i = 0; i < 16; ++i) c += (w16[i] > 0 && b16[i] >= jt);
-        }
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) c += __shfl_xor_sync(0xffffffffu, c, off);
-        if (lane == 0) wcnt[wid] = c;
-    }
+    for (int off = 16; off > 0; off >>= 1) my += __shfl_xor_sync(0xffffffffu, my, off);
+    if (lane == 0) wcnt[wid] = my;
     __syncthreads();
     int ncand = 0;
     for (int i = 0; i < kSelThreads / 32; ++i) ncand += wcnt[i];
+    __syncthreads();
     if (ncand <= kCap) {
         int base = 0;
-        for (int i = 0; i < wid; ++i) base += wcnt[i];
-        for (int64_t s0 = g_lo; s0 < g_hi; s0 += 32) {
-            const int64_t g16 = s0 + lane;
-            uint32_t hits = 0;
-            if (g16 < g_hi) {
-                uint8_t w16[16];
-                uint16_t b16[16];
-                load16(g16, w16, b16);
-#pragma unroll
-                for (int i = 0; i < 16; ++i) hits |= (uint32_t)(w16[i] > 0 && b16[i] >= jt) << i;
-            }
-            const int nh = __popc(hits);
-            int incl = nh;
+        for (int64_t cb = 0; cb < nch; cb += kSelThreads) {
+            const int64_t c = cb + tid;
+            const int n = c < nch ? sn[c] : 0;
+            int incl = n;
 #pragma unroll
             for (int off = 1; off < 32; off <<= 1) {
                 const int y = __shfl_up_sync(0xffffffffu, incl, off);
                 if (lane >= off) incl += y;
             }
-            int o = base + incl - nh;
-            while (hits) {
-                const int i = __ffs(hits) - 1;
-                hits &= hits - 1;
-                sh.cid[o++] = (int)(g16 * 16 + i);
+            if (lane == 31) wcnt[wid] = incl;
+            __syncthreads();
+            int wbase = base;
+            int gtot = 0;
+            for (int i = 0; i < kSelThreads / 32; ++i) {
+                if (i < wid) wbase += wcnt[i];
+                gtot += wcnt[i];
             }
-            base += __shfl_sync(0xffffffffu, incl, 31);
+            const int32_t* src = d.seg + (row * d.nch + c) * (int64_t)kCap;
+            const int o = wbase + incl - n;
+            for (int j = 0; j < n; ++j) sh.cid[o + j] = src[j];
+            base += gtot;
+            __syncthreads();
         }
         __syncthreads();
         const int n = ncand;
@@ -513,6 +607,11 @@ struct DecodeWs {
     uint16_t* bin;
     uint8_t* wt;
     double* slot;
+    uint32_t* hist;
+    unsigned long long* tot;
+    int32_t* seg;
+    int32_t* segn;
+    int64_t nch;
     double* Utmp;
     size_t step_bytes, load_bytes;
 };
@@ -530,6 +629,11 @@ static DecodeWs carve_decode(const lsa_cfg* cfg, const lsa_decode* d, char* base
         w.bin = (uint16_t*)take((size_t)rows * ld * 2);
         w.wt = (uint8_t*)take((size_t)rows * ld);
         w.slot = (double*)take((size_t)rows * ld * 8);
+        w.nch = (d->cache.cap_buckets + kDecScanCols - 1) / kDecScanCols;
+        w.hist = (uint32_t*)take((size_t)rows * kDecBins * 4);
+        w.tot = (unsigned long long*)take((size_t)rows * 8);
+        w.seg = (int32_t*)take((size_t)rows * w.nch * kCap * 4);
+        w.segn = (int32_t*)take((size_t)rows * w.nch * 4);
     }
     w.step_bytes = o;
     // a request load reuses the same bytes for its temporary pooled units
@@ -572,6 +676,10 @@ static lsa_status check_decode(const lsa_decode* d, const lsa_cfg* cfg) {
     if (G != 1 && G != 2 && G != 4 && G != 8) return set_error(LSA_EUNSUPPORTED, "decode: hq / hkv must be 1, 2, 4 or 8");
     if (d->cap < kBlockKeys || d->cap % kBlockKeys) return set_error(LSA_EINVAL, "decode: cap must be a positive multiple of 512");
     if (!d->K || !d->V || !d->U_blk) return set_error(LSA_EINVAL, "decode: K, V or U_blk is NULL");
+    if (d->shared_len < 0 || d->shared_len % kBlockKeys || d->shared_len >= d->cap)
+        return set_error(LSA_EINVAL, "decode: shared_len must be a multiple of 512 in [0, cap)");
+    if (d->shared_len > 0 && (!d->K_shared || !d->V_shared))
+        return set_error(LSA_EINVAL, "decode: shared_len > 0 needs K_shared and V_shared");
     const lsa_cache& c = d->cache;
     if (c.hkv != d->batch * d->hkv) return set_error(LSA_EINVAL, "decode: cache.hkv must be batch * hkv");
     if (c.cap_units != d->cap / kPool || c.cap_buckets != d->cap / kBlockKeys * kBucketsPerBlock)
@@ -632,16 +740,23 @@ lsa_status lsa_decode_load(lsa_decode* d, int32_t r, int64_t n, const float* W_k
     if ((s = check_decode(d, cfg)) != LSA_OK) return s;
     if (r < 0 || r >= d->batch) return set_error(LSA_EINVAL, "lsa_decode_load: request %d out of range", r);
     if (n < 0 || n >= d->cap) return set_error(LSA_ENOSPACE, "lsa_decode_load: n must be in [0, cap)");
+    if (n < d->shared_len) return set_error(LSA_EINVAL, "lsa_decode_load: n below the shared prefix");
     if (!W_k || !ws) return set_error(LSA_EINVAL, "lsa_decode_load: W_k or ws is NULL");
     const DecodeWs w = carve_decode(cfg, d, (char*)ws);
     if (ws_bytes < w.load_bytes || ws_bytes < w.step_bytes)
         return set_error(LSA_ENOSPACE, "lsa_decode_load: workspace too small");
     cudaStream_t st = (cudaStream_t)stream;
     const lsa_cache view = request_view(d, r);
-    const uint16_t* Kr = d->K + (int64_t)r * d->cap * d->hkv * kD;
-    const int64_t nb = n / kBlockKeys, nc = nb * kBlockKeys;
+    const int64_t sl = d->shared_len;
+    const uint16_t* Kr = d->K + (int64_t)r * (d->cap - sl) * d->hkv * kD;   // the request's rows from sl on
+    const int64_t nb = n / kBlockKeys, nc = nb * kBlockKeys;                 // nc >= sl (sl is whole blocks)
     if (nb > 0) {
-        if ((s = launch_key_latent(Kr, nc, d->hkv, W_k, 0, nc / kPool, nc / kPool, w.Utmp, st)) != LSA_OK) return s;
+        if (sl > 0 &&
+            (s = launch_key_latent(d->K_shared, sl, d->hkv, W_k, 0, sl / kPool, nc / kPool, w.Utmp, st)) != LSA_OK)
+            return s;
+        if (nc > sl && (s = launch_key_latent(Kr, nc - sl, d->hkv, W_k, 0, (nc - sl) / kPool, nc / kPool,
+                                              w.Utmp + (sl / kPool) * kDL, st)) != LSA_OK)
+            return s;
         if ((s = launch_ward_u(&view, w.Utmp, nc / kPool, nc, cfg->sinks, 0, nb, st)) != LSA_OK) return s;
     }
     if ((s = launch_clear_slots(&view, nb * kBucketsPerBlock, view.cap_buckets, st)) != LSA_OK) return s;
@@ -649,7 +764,7 @@ lsa_status lsa_decode_load(lsa_decode* d, int32_t r, int64_t n, const float* W_k
     if (j1 > j0) {
         const int64_t warps = (j1 - j0) * d->hkv;
         tail_units_kernel<<<(unsigned)ceil_div<int64_t>(warps, 8), 256, 0, st>>>(
-            Kr, W_k, d->U_blk, n, j0, j1, d->hkv, (int64_t)r * d->hkv);
+            Kr, W_k, d->U_blk, n, j0, j1, d->hkv, (int64_t)r * d->hkv, sl);
         if ((s = check_launch("tail_units_kernel")) != LSA_OK) return s;
     }
     if (cfg->mode == 1) {
@@ -678,8 +793,11 @@ lsa_status lsa_decode_step(lsa_decode* d, const uint16_t* q, const uint16_t* k, 
 
     // (1) append k/v and pool the new key
     AppendArgs ap{};
-    ap.k = k; ap.v = v; ap.K = d->K; ap.V = d->V; ap.W = W_k; ap.U_blk = d->U_blk; ap.cap = d->cap;
+    ap.k = k; ap.v = v; ap.K = d->K; ap.V = d->V; ap.W = W_k; ap.U_blk = d->U_blk;
+    ap.tail = d->cap - d->shared_len; ap.shared_len = d->shared_len;
     ap.hkv = d->hkv; ap.batch = d->batch;
+    ap.hist = cfg->mode == 0 ? w.hist : nullptr;
+    ap.tot = w.tot;
     for (int r = 0; r < d->batch; ++r) ap.pos[r] = d->len[r];
     {
         KTime kt_("decode_append_kernel", st);
@@ -720,7 +838,8 @@ lsa_status lsa_decode_step(lsa_decode* d, const uint16_t* q, const uint16_t* k, 
         sa.Y = w.Y; sa.cent = d->cache.cent; sa.minlr = d->cache.minlr; sa.maxpos = d->cache.maxpos;
         sa.cnt_lr = d->cache.cnt_lr; sa.units = d->cache.units; sa.cap_buckets = d->cache.cap_buckets;
         sa.ld = ld; sa.hkv = d->hkv; sa.G = d->hq / d->hkv; sa.agg = cfg->agg; sa.S = cfg->sinks;
-        sa.W = cfg->window; sa.T_built = d->cap; sa.bin = w.bin; sa.wt = w.wt;
+        sa.W = cfg->window; sa.T_built = d->cap; sa.bin = w.bin; sa.wt = w.wt; sa.hist = w.hist;
+        sa.tot = w.tot; sa.k = cfg->k;
         for (int r = 0; r < d->batch; ++r) sa.pos[r] = a.pos[r];
         dim3 grid((unsigned)ceil_div<int64_t>(d->cache.cap_buckets, kDecScanCols), (unsigned)rows);
         const int ng = cfg->agg ? d->hq / d->hkv : 1;
@@ -734,8 +853,19 @@ lsa_status lsa_decode_step(lsa_decode* d, const uint16_t* q, const uint16_t* k, 
             kern<<<grid, 128, kDecScanSmem, st>>>(tmC, sa);
         }
         if ((s = check_launch("decode_score_kernel")) != LSA_OK) return s;
+        DecKeepArgs ka{};
+        ka.hist = w.hist; ka.tot = w.tot; ka.bin = w.bin; ka.wt = w.wt; ka.seg = w.seg; ka.segn = w.segn; ka.ld = ld;
+        ka.cap_buckets = d->cache.cap_buckets; ka.nch = w.nch; ka.hkv = d->hkv; ka.k = cfg->k; ka.S = cfg->sinks;
+        ka.W = cfg->window;
+        for (int r = 0; r < d->batch; ++r) ka.pos[r] = a.pos[r];
+        {
+            KTime kt_("decode_keep_kernel", st);
+            decode_keep_kernel<<<dim3((unsigned)w.nch, (unsigned)rows), 128, 0, st>>>(ka);
+        }
+        if ((s = check_launch("decode_keep_kernel")) != LSA_OK) return s;
         DecResolveArgs ra{};
         ra.s = a; ra.bin = w.bin; ra.wt = w.wt; ra.slot = w.slot; ra.ld = ld; ra.cap_buckets = d->cache.cap_buckets;
+        ra.tot = w.tot; ra.seg = w.seg; ra.segn = w.segn; ra.nch = w.nch;
         {
             KTime kt_("decode_resolve_kernel", st);
             decode_resolve_kernel<<<(unsigned)rows, kSelThreads, 0, st>>>(ra);
@@ -744,7 +874,8 @@ lsa_status lsa_decode_step(lsa_decode* d, const uint16_t* q, const uint16_t* k, 
     }
     // (4) attention: each request reads its own K/V rows
     return launch_attn(q, d->K, d->V, idx, d->batch, d->hq, d->hkv, (int32_t)decode_row_len(cfg), d->cap,
-                       o, st, d->cap, 8, -1, nullptr, nullptr);
+                       o, st, d->cap - d->shared_len, 8, -1, nullptr, nullptr, d->K_shared, d->V_shared,
+                       d->shared_len);
 }
 
 }  // extern "C"

@@ -282,6 +282,15 @@ lsa_status lsa_select_attn(const uint16_t* Q, const uint16_t* K,
  *   len     tokens each request holds (host memory, in this struct); set by
  *           lsa_decode_load and advanced by lsa_decode_step.
  * cap must be a multiple of 512; batch <= LSA_MAX_BATCH.
+ *
+ * Shared prefix (optional; K_shared = V_shared = NULL, shared_len = 0 for
+ * none): every request starts with the same shared_len tokens, whose rows
+ * are read from K_shared / V_shared [shared_len, hkv, d_head] (caller-owned,
+ * read only).  The pools K, V then hold only each request's tail:
+ * [batch, cap - shared_len, hkv, d_head], request r's token t >= shared_len
+ * at row r*(cap - shared_len) + (t - shared_len).  shared_len is a multiple
+ * of 512 below cap, and lsa_decode_load needs n >= shared_len.  Each request
+ * keeps its own cache (its blocks are clustered once per request).
  */
 typedef struct lsa_decode {
     int32_t   batch, hkv, hq;
@@ -292,6 +301,9 @@ typedef struct lsa_decode {
     lsa_cache cache;
     lsa_tree  tree;
     int64_t   len[LSA_MAX_BATCH];
+    const uint16_t* K_shared;
+    const uint16_t* V_shared;
+    int64_t   shared_len;
 } lsa_decode;
 
 /* Workspace bytes of lsa_decode_load / lsa_decode_step for this state. */

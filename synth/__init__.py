@@ -36,7 +36,7 @@ CONFIGS = {
                          sinks=4, window=600, mode=0, agg=0, beam=2),
     "decode-4x10m": dict(T=10_000_000, batch=4, hkv=8, hq=32, d=128, dl=64,
                          n_centres=65536, k=2048, sinks=4, window=1024, mode=0,
-                         agg=0, beam=2),
+                         agg=0, beam=2, shared_prefix=True),
 }
 
 _TAGS = {"centres": 1, "kc": 2, "kn": 3, "qc": 4, "qn": 5, "v": 6, "wk": 7, "wq": 8}
@@ -173,6 +173,35 @@ def device_decode(c: dict, seed: int, device, n0: int, steps: int, K_out, V_out)
     for r in range(B):
         device_tokens(n0, hkv, d, mu, 4.0, gen, device, out=K_out[r, :n0])
         device_tokens(n0, hkv, d, mu, 0.0, gen, device, out=V_out[r, :n0])
+    q = device_tokens(steps * B, hq, d, mu, 1.0, gen, device).view(steps, B, hq, d)
+    k = device_tokens(steps * B, hkv, d, mu, 4.0, gen, device).view(steps, B, hkv, d)
+    v = device_tokens(steps * B, hkv, d, mu, 0.0, gen, device).view(steps, B, hkv, d)
+    return q, k, v
+
+
+def device_shared_prefix(c: dict, seed: int, device, shared_len: int):
+    """K/V [shared_len, hkv, d] of a prefix every decode request shares."""
+    import torch
+    gen = torch.Generator(device=device)
+    gen.manual_seed(1000 * seed + 1)
+    mu = torch.from_numpy(centres(seed, c["n_centres"], c["d"])).to(device)
+    Ks = device_tokens(shared_len, c["hkv"], c["d"], mu, 4.0, gen, device)
+    Vs = device_tokens(shared_len, c["hkv"], c["d"], mu, 0.0, gen, device)
+    return Ks, Vs
+
+
+def device_decode_tails(c: dict, seed: int, device, shared_len: int, n0: int, steps: int, K_tail, V_tail):
+    """Each request's prompt tokens shared_len .. n0 - 1 written into
+    K_tail[r] / V_tail[r] (rows from 0), then (q, k, v) for `steps` steps,
+    [steps, batch, heads, d] each."""
+    import torch
+    B, hkv, hq, d = c["batch"], c["hkv"], c["hq"], c["d"]
+    gen = torch.Generator(device=device)
+    gen.manual_seed(1000 * seed + 2)
+    mu = torch.from_numpy(centres(seed, c["n_centres"], d)).to(device)
+    for r in range(B):
+        device_tokens(n0 - shared_len, hkv, d, mu, 4.0, gen, device, out=K_tail[r, :n0 - shared_len])
+        device_tokens(n0 - shared_len, hkv, d, mu, 0.0, gen, device, out=V_tail[r, :n0 - shared_len])
     q = device_tokens(steps * B, hq, d, mu, 1.0, gen, device).view(steps, B, hq, d)
     k = device_tokens(steps * B, hkv, d, mu, 4.0, gen, device).view(steps, B, hkv, d)
     v = device_tokens(steps * B, hkv, d, mu, 0.0, gen, device).view(steps, B, hkv, d)

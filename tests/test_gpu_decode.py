@@ -30,24 +30,28 @@ def reqs():
     return [synth.layer_inputs("decode-small", seed=r) for r in range(len(PROMPTS))]
 
 
-@pytest.mark.parametrize("mode,agg,W", [(0, 0, 600), (0, 1, 600), (1, 0, 600), (1, 1, 600), (0, 0, 128)])
-def test_decode_matches_oracle(lsa, reqs, mode, agg, W):
+def _run_decode(lsa, Kl, Vl, Ql, Wk_np, Wq_np, cfg, shared_len=0):
+    """Decode STEPS tokens per request after PROMPTS, checking index rows and
+    outputs against the oracle over the logical keys Kl[r] (the shared prefix
+    then the request's own tokens)."""
     c = synth.CONFIGS["decode-small"]
     hkv, hq, cap = c["hkv"], c["hq"], c["T"]
-    cfg = lsa.Config(k=c["k"], sinks=c["sinks"], window=W, beam=c["beam"], mode=mode, agg=agg)
-    Wk, Wq = to_dev(reqs[0]["Wk"]), to_dev(reqs[0]["Wq"])  # one W_k / W_q per layer
-    dec = lsa.Decode(len(PROMPTS), hkv, hq, cap, cfg)
+    Wk, Wq = to_dev(Wk_np), to_dev(Wq_np)  # one W_k / W_q per layer
+    shared = None
+    if shared_len:
+        shared = (to_dev_bf16(Kl[0][:shared_len]), to_dev_bf16(Vl[0][:shared_len]))
+    dec = lsa.Decode(len(PROMPTS), hkv, hq, cap, cfg, shared=shared)
     for r, n in enumerate(PROMPTS):
-        dec.load(r, to_dev_bf16(reqs[r]["K"][:n]), to_dev_bf16(reqs[r]["V"][:n]), Wk)
+        dec.load(r, to_dev_bf16(Kl[r][shared_len:n]), to_dev_bf16(Vl[r][shared_len:n]), Wk)
     check_at = {0, 1, 2, 19, STEPS - 1}
     idx = torch.empty((len(PROMPTS), hkv, cfg.row), dtype=torch.int32, device="cuda")
     ocfg = oracle_cfg(cfg)
     caches = {}
     for s in range(STEPS):
         ts = [n + s for n in PROMPTS]
-        q = to_dev_bf16(np.stack([reqs[r]["Q"][t] for r, t in enumerate(ts)]))
-        k = to_dev_bf16(np.stack([reqs[r]["K"][t] for r, t in enumerate(ts)]))
-        v = to_dev_bf16(np.stack([reqs[r]["V"][t] for r, t in enumerate(ts)]))
+        q = to_dev_bf16(np.stack([Ql[r][t] for r, t in enumerate(ts)]))
+        k = to_dev_bf16(np.stack([Kl[r][t] for r, t in enumerate(ts)]))
+        v = to_dev_bf16(np.stack([Vl[r][t] for r, t in enumerate(ts)]))
         o = dec.step(q, k, v, Wk, Wq, idx_out=idx)
         completes = any((t + 1) % 512 == 0 or t % 512 == 0 for t in ts)
         if s not in check_at and not completes:
@@ -60,15 +64,36 @@ def test_decode_matches_oracle(lsa, reqs, mode, agg, W):
             tb = 512 * ((t + 1) // 512)
             key = (r, tb)
             if key not in caches:
-                U = oracle.key_latent_pool(reqs[r]["K"][:tb], reqs[0]["Wk"], 4)
+                U = oracle.key_latent_pool(Kl[r][:tb], Wk_np, 4)
                 oc = oracle.build_cache(U, tb, ocfg)
-                caches[key] = (oc, oracle.build_tree(oc) if mode == 1 else None)
+                caches[key] = (oc, oracle.build_tree(oc) if cfg.mode == 1 else None)
             oc, ot = caches[key]
-            Qt = reqs[r]["Q"][t:t + 1]
-            Y = oracle.query_latent(Qt, reqs[0]["Wq"], hkv, agg)
+            Qt = Ql[r][t:t + 1]
+            Y = oracle.query_latent(Qt, Wq_np, hkv, cfg.agg)
             oidx, _, _ = oracle.select(oc, Y, np.array([t]), ocfg, tree=ot, G=hq // hkv)
             assert np.array_equal(g_idx[r], oidx[0]), (s, r, t)
-            ref = oracle.attention(Qt, reqs[r]["K"][:t + 1], reqs[r]["V"][:t + 1], oidx)[0]
+            ref = oracle.attention(Qt, Kl[r][:t + 1], Vl[r][:t + 1], oidx)[0]
             e = np.abs(g_o[r] - ref)
             assert e.max() <= 2e-2 and e.mean() <= 2e-3, (s, r, e.max(), e.mean())
     assert dec.len == [n + STEPS for n in PROMPTS]
+
+
+@pytest.mark.parametrize("mode,agg,W", [(0, 0, 600), (0, 1, 600), (1, 0, 600), (1, 1, 600), (0, 0, 128)])
+def test_decode_matches_oracle(lsa, reqs, mode, agg, W):
+    c = synth.CONFIGS["decode-small"]
+    cfg = lsa.Config(k=c["k"], sinks=c["sinks"], window=W, beam=c["beam"], mode=mode, agg=agg)
+    _run_decode(lsa, [x["K"] for x in reqs], [x["V"] for x in reqs], [x["Q"] for x in reqs],
+                reqs[0]["Wk"], reqs[0]["Wq"], cfg)
+
+
+@pytest.mark.parametrize("mode", [0, 1])
+def test_decode_shared_prefix_matches_oracle(lsa, reqs, mode):
+    """Requests that share their first 512 tokens (read from one shared
+    K/V, the pools holding only each request's tail) decode exactly as if
+    each held the whole prefix itself."""
+    c = synth.CONFIGS["decode-small"]
+    cfg = lsa.Config(k=c["k"], sinks=c["sinks"], window=600, beam=c["beam"], mode=mode, agg=0)
+    sl = 512
+    Kl = [np.concatenate([reqs[0]["K"][:sl], x["K"][sl:]]) for x in reqs]
+    Vl = [np.concatenate([reqs[0]["V"][:sl], x["V"][sl:]]) for x in reqs]
+    _run_decode(lsa, Kl, Vl, [x["Q"] for x in reqs], reqs[0]["Wk"], reqs[0]["Wq"], cfg, shared_len=sl)
