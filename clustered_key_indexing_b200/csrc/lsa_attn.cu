@@ -22,7 +22,7 @@
 
 namespace lsa {
 
-constexpr int kAttnWarps = 4;
+constexpr int kAttnWarps = 7;  // 16 KB of ring each: two CTAs, 14 warps per SM
 constexpr int kStages = 2;
 constexpr int kTileKeys = 16;
 constexpr int kTileBytes = kTileKeys * kD * 2;           // 4 KB per tensor
