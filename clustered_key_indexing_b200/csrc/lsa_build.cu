@@ -26,7 +26,7 @@ namespace lsa {
 // cg, cg+16, cg+32, cg+48): 32 fp64 accumulators, one fma per (row, dim, e).
 // The product of a bf16 key and an fp32 weight is exact in fp64, so the fma
 // chain equals "sum of products in ascending e, one rounding per add".
-constexpr int kLatWarps = 4;
+constexpr int kLatWarps = 8;  // 204 KB of shared memory: one CTA, 8 warps per SM
 constexpr int kKT = 17;        // padded row stride (doubles) of the staged tile
 constexpr int kVS = 65;        // padded row stride of the projected rows
 
