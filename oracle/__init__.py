@@ -310,3 +310,34 @@ def layer(Q, K, V, Wk, Wq, cfg: Cfg, tpos=None, cache=None, tree=None):
     idx, mg, nc = select(cache, Y, tpos, cfg, tree=tree, G=G)
     O = attention(Qs, K, V, idx)
     return dict(U=U, cache=cache, tree=tree, Y=Y, idx=idx, margin=mg, ncmp=nc, O=O)
+
+
+# ------------------------------------------- training-free PCA projection
+
+def fit_pca(K: np.ndarray, d_latent: int = 64):
+    """Training-free projection of the distilled variant: the first d_latent
+    principal directions of the layer's keys (tutorial "隐空间稀疏注意力
+    (LSA)" and the essay's closing remarks: PCA of the keys, the leading 64
+    directions taken as the projection, no training).
+
+    Readings: the covariance is the centred one, (1/N) sum (k - mean)(k -
+    mean)^T over the keys of every kv-head (one projection per layer);
+    directions are ordered by eigenvalue, largest first, equal eigenvalues by
+    eigh's order; each direction's sign makes its largest-magnitude component
+    (the first such) positive.
+
+    K: bf16 bits [T, hkv, d].  Returns (W fp32 [d, d_latent] with the
+    directions as columns, eigenvalues fp64 [d] descending, V fp64 [d, d])."""
+    X = bf16_to_f64(np.asarray(K, np.uint16)).reshape(-1, K.shape[-1])
+    N = X.shape[0]
+    mean = X.sum(axis=0) / N
+    Xc = X - mean
+    C = (Xc.T @ Xc) / N
+    lam, V = np.linalg.eigh(C)                    # ascending
+    order = np.argsort(-lam, kind="stable")
+    lam, V = lam[order], V[:, order]
+    for j in range(V.shape[1]):
+        i = int(np.argmax(np.abs(V[:, j])))
+        if V[i, j] < 0:
+            V[:, j] = -V[:, j]
+    return np.ascontiguousarray(V[:, :d_latent], dtype=np.float32), lam, V

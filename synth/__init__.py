@@ -206,3 +206,17 @@ def device_decode_tails(c: dict, seed: int, device, shared_len: int, n0: int, st
     k = device_tokens(steps * B, hkv, d, mu, 4.0, gen, device).view(steps, B, hkv, d)
     v = device_tokens(steps * B, hkv, d, mu, 0.0, gen, device).view(steps, B, hkv, d)
     return q, k, v
+
+
+def pca_keys(seed: int, T: int, hkv: int, d: int = 128, decay: float = 0.97) -> np.ndarray:
+    """bf16 bits [T, hkv, d] of keys with a known, well-separated spectrum:
+    k = R (s * g) + m, with R a random orthogonal d x d matrix, s_i =
+    4 * decay^i, g ~ N(0, I) and a fixed offset m (the principal directions
+    are R's columns in order)."""
+    rng = _rng(seed, "kn", 7777)
+    R = orthonormal(seed, "wk", d, d)
+    s = (4.0 * decay ** np.arange(d)).astype(np.float32)
+    g = rng.standard_normal((T * hkv, d), dtype=np.float32)
+    m = rng.standard_normal(d, dtype=np.float32)
+    x = (g * s[None, :]) @ R.T + m[None, :]
+    return f32_to_bf16_bits(x.astype(np.float32)).reshape(T, hkv, d)
