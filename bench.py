@@ -68,6 +68,7 @@ def parse():
     p.add_argument("--batch", type=int, default=None, help="decode requests (profiling runs)")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu", action="store_true")
+    p.add_argument("--pca", action="store_true", help="time the training-free projection fit on the workload's keys")
     return p.parse_args()
 
 
@@ -616,6 +617,64 @@ def decode_prompt_len(T, warmup, steps):
     return T - 1 - warmup - steps // 2
 
 
+def run_pca(args):
+    """The training-free projection (lsa_fit_pca) on the workload's keys: one
+    step = one fit over all T * hkv keys (fp64 second moments + Jacobi)."""
+    import torch
+
+    import clustered_key_indexing_b200 as lsa
+
+    world, rank, local = dist_setup(args)
+    c = workload_cfg(args)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    if c["T"] <= 131072:
+        K = torch.from_numpy(synth.layer_inputs(args.workload, seed=rank, T=c["T"], parts=("K",))["K"]
+                             .view(np.int16)).view(torch.bfloat16).to(dev)
+    else:
+        _, K, _ = synth.device_layer(dict(c, hq=c["hkv"]), rank, dev)
+    N = K.shape[0] * K.shape[1]
+    for _ in range(args.warmup):
+        lsa.fit_pca(K)
+    torch.cuda.synchronize()
+    clocks = Clocks(torch.cuda.current_device())
+    kt = lsa.KernelTimer()
+    stream = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with kt:
+        e0.record(stream)
+        for _ in range(args.steps):
+            W, eig = lsa.fit_pca(K)
+        e1.record(stream)
+        torch.cuda.synchronize()
+    clk = clocks.stop()
+    lsa.check_device_error()
+    ms = max_over_ranks(e0.elapsed_time(e1), world, dev) / args.steps
+    kms, kn = kt.get("pca_moments_kernel")
+    jms, jn = kt.get("pca_jacobi_kernel")
+    # algorithmic work of the moments: one fp64 FMA per key and per entry of
+    # the symmetric 128 x 128 matrix's upper triangle; peak: 148 SMs x 64
+    # fp64 FMA per clock x 2 FLOP x 1965 MHz
+    flops = N * (128 * 129 // 2) * 2.0
+    peak = 148 * 64 * 2 * 1.965e9 / 1e12
+    mom_ms = kms / max(kn, 1)
+    achieved = flops / (mom_ms / 1e3) / 1e12
+    if rank == 0:
+        emit_json({
+            "metric": "LSA PCA projection fit keys/s", "value": job_rate(world, N, ms), "unit": "keys/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": {"workload": args.workload, "T": c["T"], "hkv": c["hkv"], "keys": N,
+                                            "d_latent": 64, "l2": "no flush: the keys are larger than L2"},
+            "clocks": clk, "gpu_launches": 3 * args.steps,
+            "kernels": {"pca_moments_kernel": mom_ms, "pca_jacobi_kernel": jms / max(jn, 1)},
+            "roofline": {"kernel": "pca_moments_kernel", "bound": "alu", "achieved": achieved, "peak": peak,
+                         "unit": "TFLOP/s", "frac": achieved / peak, "traffic": None,
+                         "peak_source": "derived: 148 SMs x 64 fp64 FMA/clk x 2 x 1965 MHz",
+                         "work_per_launch": flops},
+            "eigenvalues_top4": [float(x) for x in eig[:4].cpu()],
+        })
+
+
 def ctypes_ref(x):
     import ctypes
     return ctypes.byref(x)
@@ -630,6 +689,8 @@ if __name__ == "__main__":
     a = parse()
     if a.impl == "reference":
         run_reference(a)
+    elif a.pca:
+        run_pca(a)
     elif a.workload.startswith("decode"):
         run_decode(a)
     else:

@@ -209,6 +209,20 @@ def select_attn(Q, K, V, idx, t0: int, cfg: Config, T: int | None = None, O=None
     return O
 
 
+def fit_pca(K: torch.Tensor, d_latent: int = 64, stream=None):
+    """lsa_fit_pca: the training-free projection, the leading d_latent
+    principal directions of the keys K [T, hkv, 128] (all heads).  Returns
+    (W fp32 [128, d_latent], eigenvalues fp64 [128], descending)."""
+    _need_cuda(K)
+    T, hkv = int(K.shape[0]), int(K.shape[1])
+    W = torch.empty((128, d_latent), dtype=torch.float32, device=K.device)
+    eig = torch.empty(128, dtype=torch.float64, device=K.device)
+    ws = torch.empty(int(lib().lsa_fit_pca_workspace_bytes(T, hkv)) or 1, dtype=torch.uint8, device=K.device)
+    check(lib().lsa_fit_pca(_ptr(K), T, hkv, d_latent, _ptr(W), _ptr(eig), _ptr(ws), ws.numel(), _stream(stream)),
+          "lsa_fit_pca")
+    return W, eig
+
+
 def prefill_chunk(cfg: Config, T: int, hq: int, hkv: int, chunk: int = 0) -> int:
     """The query chunk lsa_prefill uses for a requested chunk (0: its own choice)."""
     return int(lib().lsa_prefill_chunk(ctypes.byref(cfg.c()), T, hq, hkv, chunk))

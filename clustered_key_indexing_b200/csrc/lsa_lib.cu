@@ -7,3 +7,4 @@
 #include "lsa_api.cu"
 #include "lsa_decode.cu"
 #include "lsa_noalloc.cu"
+#include "lsa_pca.cu"

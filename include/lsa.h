@@ -391,6 +391,31 @@ lsa_status lsa_prefill(const uint16_t* Q, const uint16_t* K, const uint16_t* V,
                        lsa_tree* tree, uint16_t* O, int64_t chunk, void* ws,
                        size_t ws_bytes, void* stream);
 
+/* ------------------------------------------- training-free projection */
+
+/* Workspace bytes of lsa_fit_pca (independent of T beyond T > 0). */
+size_t lsa_fit_pca_workspace_bytes(int64_t T, int32_t hkv);
+
+/*
+ * lsa_fit_pca -- the training-free projection of the distilled variant: the
+ * leading d_latent principal directions of the layer's keys, used as W_k
+ * (and as W_q: queries are projected onto the same directions)
+ * [tutorial "隐空间稀疏注意力 (LSA)"; essay ch. 5 and closing remarks: PCA of
+ * the keys, the leading 64 directions as the projection, no training].
+ * K [T, hkv, d_head] bf16, 16-byte aligned; every key of every kv-head
+ * counts once.  Computes the centred covariance C = (1/N) sum (k - mean)
+ * (k - mean)^T (fp64, N = T*hkv) and its eigen-decomposition (cyclic Jacobi,
+ * fp64); directions ordered by eigenvalue, largest first (equal eigenvalues:
+ * lower Jacobi index first); each direction's first largest-magnitude
+ * component is positive.  W_out [d_head, d_latent] fp32 row-major, column r
+ * = direction r (rounded to nearest).  eig_out (optional, may be NULL):
+ * [d_head] fp64 eigenvalues, descending.  Requires ws_bytes >=
+ * lsa_fit_pca_workspace_bytes(T, hkv).
+ */
+lsa_status lsa_fit_pca(const uint16_t* K, int64_t T, int32_t hkv, int32_t d_latent,
+                       float* W_out, double* eig_out, void* ws, size_t ws_bytes,
+                       void* stream);
+
 #ifdef __cplusplus
 }
 #endif
