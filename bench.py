@@ -385,13 +385,12 @@ def run_lsa(args):
     if not args.no_e2e:
         hO = torch.empty_like(hQ).pin_memory()
         pws = torch.empty(lsa.prefill_workspace_bytes(cfg, T, hq, hkv, chunk), dtype=torch.uint8, device=dev)
+        up, down = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
 
         def e2e_step():
-            Q.copy_(hQ, non_blocking=True)
-            K.copy_(hK, non_blocking=True)
-            V.copy_(hV, non_blocking=True)
-            lsa.prefill(Q, K, V, Wk, Wq, cfg, cache=cache, tree=tree, O=O, chunk=chunk, ws=pws)
-            hO.copy_(O, non_blocking=True)
+            # lsa_prefill_host: uploads, the layer and the copy back, overlapped
+            lsa.prefill_host(hQ, hK, hV, Wk, Wq, cfg, hO=hO, dev_bufs=(Q, K, V, O), cache=cache, tree=tree,
+                             chunk=chunk, ws=pws, stream=stream, h2d_stream=up, d2h_stream=down)
 
         for _ in range(max(1, args.warmup)):
             e2e_step()

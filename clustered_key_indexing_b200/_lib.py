@@ -103,6 +103,8 @@ def lib():
         L.lsa_prefill_workspace_bytes.restype = sz
         L.lsa_prefill.argtypes = [vp, vp, vp, i64, i32, i32, vp, vp, P(lsa_cfg), P(lsa_cache),
                                   P(lsa_tree), vp, i64, vp, sz, vp]
+        L.lsa_prefill_host.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i64, i32, i32, vp, vp, P(lsa_cfg),
+                                       P(lsa_cache), P(lsa_tree), i64, vp, sz, vp, vp, vp]
         L.lsa_fit_pca_workspace_bytes.argtypes = [i64, i32]
         L.lsa_fit_pca_workspace_bytes.restype = sz
         L.lsa_fit_pca.argtypes = [vp, i64, i32, i32, vp, vp, vp, sz, vp]

@@ -253,6 +253,41 @@ def prefill(Q, K, V, W_k, W_q, cfg: Config, cache: Cache | None = None, tree: Tr
     return O
 
 
+def prefill_host(hQ, hK, hV, W_k, W_q, cfg: Config, hO=None, dev_bufs=None, cache: Cache | None = None,
+                 tree: Tree | None = None, chunk: int = 16384, ws=None, stream=None, h2d_stream=None,
+                 d2h_stream=None) -> torch.Tensor:
+    """lsa_prefill_host: the whole layer from pinned host Q/K/V into pinned
+    host O, uploads and downloads overlapped with the compute.  dev_bufs:
+    optional (Q, K, V, O) device buffers; streams: the compute stream (default
+    current) and two copy streams (default: new ones)."""
+    _need_cuda(W_k, W_q)
+    for t in (hQ, hK, hV):
+        if t.is_cuda or not t.is_pinned():
+            raise ValueError("lsa_prefill_host takes pinned host tensors")
+    T, hq, d = hQ.shape
+    hkv = hK.shape[1]
+    dev = W_k.device
+    if hO is None:
+        hO = torch.empty_like(hQ).pin_memory()
+    if dev_bufs is None:
+        dev_bufs = (torch.empty(hQ.shape, dtype=hQ.dtype, device=dev), torch.empty(hK.shape, dtype=hK.dtype, device=dev),
+                    torch.empty(hV.shape, dtype=hV.dtype, device=dev), torch.empty(hQ.shape, dtype=hQ.dtype, device=dev))
+    Q, K, V, O = dev_bufs
+    cache = cache or Cache(hkv, T, cfg, device=dev)
+    if cfg.mode == 1 and tree is None:
+        tree = Tree(cache, device=dev)
+    need = prefill_workspace_bytes(cfg, T, hq, hkv, chunk)
+    if ws is None or ws.numel() < need:
+        ws = torch.empty(need, dtype=torch.uint8, device=dev)
+    up = h2d_stream or torch.cuda.Stream(device=dev)
+    down = d2h_stream or torch.cuda.Stream(device=dev)
+    check(lib().lsa_prefill_host(_ptr(hQ), _ptr(hK), _ptr(hV), _ptr(hO), _ptr(Q), _ptr(K), _ptr(V), _ptr(O), T, hq,
+                                 hkv, _ptr(W_k), _ptr(W_q), ctypes.byref(cfg.c()), ctypes.byref(cache.c),
+                                 ctypes.byref(tree.t) if tree is not None else None, chunk, _ptr(ws), ws.numel(),
+                                 _stream(stream), _stream(up), _stream(down)), "lsa_prefill_host")
+    return hO
+
+
 class Decode:
     """Batched decode state (lsa_decode): `batch` requests of `cap` tokens,
     K/V pools [batch, cap, hkv, 128], a cache whose heads are

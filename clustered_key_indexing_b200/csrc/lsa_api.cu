@@ -451,4 +451,88 @@ lsa_status lsa_prefill(const uint16_t* Q, const uint16_t* K, const uint16_t* V, 
     return LSA_OK;
 }
 
+lsa_status lsa_prefill_host(const uint16_t* hQ, const uint16_t* hK, const uint16_t* hV, uint16_t* hO,
+                            uint16_t* Q, uint16_t* K, uint16_t* V, uint16_t* O, int64_t T, int32_t hq,
+                            int32_t hkv, const float* W_k, const float* W_q, const lsa_cfg* cfg,
+                            lsa_cache* cache, lsa_tree* tree, int64_t chunk, void* ws, size_t ws_bytes,
+                            void* stream, void* h2d_stream, void* d2h_stream) {
+    lsa_status s;
+    if ((s = check_cfg(cfg)) != LSA_OK) return s;
+    if ((s = check_heads(hq, hkv)) != LSA_OK) return s;
+    if (!hQ || !hK || !hV || !hO) return set_error(LSA_EINVAL, "lsa_prefill_host: NULL host pointer");
+    if (!Q || !K || !V || !O || !W_k || !W_q || !ws) return set_error(LSA_EINVAL, "lsa_prefill_host: NULL pointer");
+    if (T <= 0) return set_error(LSA_EINVAL, "lsa_prefill_host: T must be positive");
+    chunk = prefill_chunk(cfg, T, hq, hkv, chunk);
+    const size_t need = lsa_prefill_workspace_bytes(cfg, T, hq, hkv, chunk);
+    if (ws_bytes < need) return set_error(LSA_ENOSPACE, "lsa_prefill_host: workspace %zu < %zu bytes", ws_bytes, need);
+    cudaStream_t st = (cudaStream_t)stream, up = (cudaStream_t)h2d_stream, down = (cudaStream_t)d2h_stream;
+    const int64_t nch = (T + chunk - 1) / chunk;
+    const size_t qrow = (size_t)hq * kD * 2, kvrow = (size_t)hkv * kD * 2;
+    // events: start, K landed, per chunk (Q and V rows landed, O written, O copied back)
+    std::vector<cudaEvent_t> ev((size_t)(2 + 3 * nch), nullptr);
+    auto cleanup = [&]() {
+        for (auto& e : ev)
+            if (e) cudaEventDestroy(e);  // released once complete
+    };
+    for (auto& e : ev)
+        if (cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess) {
+            e = nullptr;
+            cleanup();
+            return set_error(LSA_ECUDA, "lsa_prefill_host: cudaEventCreate failed");
+        }
+    cudaEvent_t e_start = ev[0], e_k = ev[1];
+    auto e_in = [&](int64_t i) { return ev[2 + 3 * i]; };
+    auto e_out = [&](int64_t i) { return ev[3 + 3 * i]; };
+    auto e_back = [&](int64_t i) { return ev[4 + 3 * i]; };
+    auto fail = [&](const char* what) {
+        cleanup();
+        return set_error(LSA_ECUDA, "lsa_prefill_host: %s: %s", what, cudaGetErrorString(cudaGetLastError()));
+    };
+    // uploads: K whole (the build needs every key), then per chunk its Q rows
+    // and V rows; they start after the work already queued on `stream`
+    if (cudaEventRecord(e_start, st) != cudaSuccess || cudaStreamWaitEvent(up, e_start, 0) != cudaSuccess)
+        return fail("event");
+    if (cudaMemcpyAsync(K, hK, (size_t)T * kvrow, cudaMemcpyHostToDevice, up) != cudaSuccess) return fail("K upload");
+    if (cudaEventRecord(e_k, up) != cudaSuccess) return fail("event");
+    for (int64_t i = 0; i < nch; ++i) {
+        const int64_t t0 = i * chunk, n = (T - t0) < chunk ? (T - t0) : chunk;
+        if (cudaMemcpyAsync(Q + t0 * hq * kD, hQ + t0 * hq * kD, (size_t)n * qrow, cudaMemcpyHostToDevice, up) !=
+                cudaSuccess ||
+            cudaMemcpyAsync(V + t0 * hkv * kD, hV + t0 * hkv * kD, (size_t)n * kvrow, cudaMemcpyHostToDevice, up) !=
+                cudaSuccess)
+            return fail("Q/V upload");
+        if (cudaEventRecord(e_in(i), up) != cudaSuccess) return fail("event");
+    }
+    // compute, with each chunk's output copied back as soon as it is written
+    if (cudaStreamWaitEvent(st, e_k, 0) != cudaSuccess) return fail("event");
+    if ((s = lsa_build_buckets(K, T, hkv, W_k, cfg, cache, stream)) != LSA_OK) { cleanup(); return s; }
+    if (cfg->mode == 1 && (s = lsa_build_tree(cache, cfg, tree, stream)) != LSA_OK) { cleanup(); return s; }
+    const PrefillWs pw = prefill_ws_layout(cfg, chunk, hq, hkv);
+    int32_t* idx = (int32_t*)ws;
+    void* aws = (char*)ws + pw.idx_bytes;
+    void* sws = (char*)ws + pw.total;
+    const size_t sws_bytes = ws_bytes - pw.total;
+    for (int64_t i = 0; i < nch; ++i) {
+        const int64_t t0 = i * chunk, n = (T - t0) < chunk ? (T - t0) : chunk;
+        if (cudaStreamWaitEvent(st, e_in(i), 0) != cudaSuccess) return fail("event");
+        const uint16_t* Qc = Q + t0 * hq * kD;
+        if ((s = lsa_select(Qc, t0, n, hq, W_q, cache, tree, cfg, idx, nullptr, sws, sws_bytes, stream)) != LSA_OK ||
+            (s = lsa_select_attn(Qc, K, V, idx, t0, n, hq, hkv, T, cfg, O + t0 * hq * kD, aws,
+                                 pw.ow_bytes + pw.lse_bytes, stream)) != LSA_OK) {
+            cleanup();
+            return s;
+        }
+        if (cudaEventRecord(e_out(i), st) != cudaSuccess || cudaStreamWaitEvent(down, e_out(i), 0) != cudaSuccess)
+            return fail("event");
+        if (cudaMemcpyAsync(hO + t0 * hq * kD, O + t0 * hq * kD, (size_t)n * qrow, cudaMemcpyDeviceToHost, down) !=
+            cudaSuccess)
+            return fail("O download");
+        if (cudaEventRecord(e_back(i), down) != cudaSuccess) return fail("event");
+    }
+    // the call is complete on `stream` once the last copy back has landed
+    if (cudaStreamWaitEvent(st, e_back(nch - 1), 0) != cudaSuccess) return fail("event");
+    cleanup();
+    return LSA_OK;
+}
+
 }  // extern "C"

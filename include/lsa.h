@@ -391,6 +391,26 @@ lsa_status lsa_prefill(const uint16_t* Q, const uint16_t* K, const uint16_t* V,
                        lsa_tree* tree, uint16_t* O, int64_t chunk, void* ws,
                        size_t ws_bytes, void* stream);
 
+/*
+ * lsa_prefill_host -- lsa_prefill from pinned HOST buffers hQ, hK, hV into
+ * the pinned host buffer hO, with the transfers overlapped with the compute:
+ * on `h2d_stream` K is uploaded whole (the build needs every key), then per
+ * chunk its Q rows and V rows; the layer runs on `stream` (each chunk waits
+ * for its rows only); each chunk's O rows go back on `d2h_stream` as soon as
+ * they are written.  Q, K, V, O are the caller's device buffers for the
+ * layer ([T, hq or hkv, d] bf16), the rest as for lsa_prefill.  The uploads
+ * start after the work already queued on `stream`, and the call is complete
+ * on `stream` once the last O rows are on the host.  The three streams
+ * should be distinct for the copies to overlap (NULL = the legacy default
+ * stream, which serialises them).  Events are created and released inside.
+ */
+lsa_status lsa_prefill_host(const uint16_t* hQ, const uint16_t* hK, const uint16_t* hV,
+                            uint16_t* hO, uint16_t* Q, uint16_t* K, uint16_t* V, uint16_t* O,
+                            int64_t T, int32_t hq, int32_t hkv, const float* W_k,
+                            const float* W_q, const lsa_cfg* cfg, lsa_cache* cache,
+                            lsa_tree* tree, int64_t chunk, void* ws, size_t ws_bytes,
+                            void* stream, void* h2d_stream, void* d2h_stream);
+
 /* ------------------------------------------- training-free projection */
 
 /* Workspace bytes of lsa_fit_pca (independent of T beyond T > 0). */

@@ -276,3 +276,20 @@ def test_bad_arguments_return_status(lsa):
     with pytest.raises(LSAError) as e:
         lsa.build_buckets(K, to_dev(inp["Wk"]), lsa.Config(window=0), lsa.Cache(1, 64, cfg))
     assert e.value.status == LSA_EINVAL
+
+
+@pytest.mark.parametrize("mode", [0, 1])
+def test_prefill_host_equals_prefill(lsa, mode):
+    """lsa_prefill_host (pinned host buffers, overlapped copies on two extra
+    streams) gives the bits of lsa_prefill on the same inputs."""
+    T = 3000
+    cfg = lsa.Config(k=256, sinks=4, window=300, mode=mode)
+    inp = synth.layer_inputs("prefill-128k", T=T)
+    Qh, Kh, Vh = (np.ascontiguousarray(inp[x][:, :n]) for x, n in (("Q", 8), ("K", 2), ("V", 2)))
+    Wk, Wq = to_dev(inp["Wk"]), to_dev(inp["Wq"])
+    O_dev = lsa.prefill(to_dev_bf16(Qh), to_dev_bf16(Kh), to_dev_bf16(Vh), Wk, Wq, cfg, chunk=700)
+    pin = [torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).pin_memory() for x in (Qh, Kh, Vh)]
+    hO = lsa.prefill_host(*pin, Wk, Wq, cfg, chunk=700)
+    torch.cuda.synchronize()
+    lsa.check_device_error()
+    assert torch.equal(hO.view(torch.int16), O_dev.cpu().view(torch.int16))
