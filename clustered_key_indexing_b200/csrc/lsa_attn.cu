@@ -7,9 +7,11 @@
 // share the index list, so the warp computes S^T = K_sel Q^T with the keys as
 // the MMA's M dimension (16 keys per tile) and the heads as N (8 columns),
 // then O^T += V_sel^T P^T.  Keys are gathered 16 at a time with 16-byte
-// cp.async copies into a per-warp 2-stage shared-memory ring (16-byte chunks
-// XOR-swizzled by row so ldmatrix reads are conflict-free); index tiles with
-// no valid entry are skipped.  Online softmax in fp32 (exp2 with the
+// cp.async copies into a per-warp 12 KB shared-memory ring: two K tiles and
+// one V tile (16-byte chunks XOR-swizzled by row so ldmatrix reads are
+// conflict-free), so that 16 warps fit on an SM; the next V tile is fetched
+// while the next tile's scores are computed.  Index tiles with no valid
+// entry are skipped.  Online softmax in fp32 (exp2 with the
 // log2(e)/sqrt(d) scale folded in), P rounded to bf16 for the PV product.
 // Warps are ordered kv-head-major so the warps resident at one time read one
 // head's K/V, which keeps that head's rows in L2.
@@ -22,12 +24,10 @@
 
 namespace lsa {
 
-constexpr int kAttnWarps = 7;  // 16 KB of ring each: two CTAs, 14 warps per SM
-constexpr int kStages = 2;
+constexpr int kAttnWarps = 8;  // 12 KB of ring each: two CTAs, 16 warps per SM
 constexpr int kTileKeys = 16;
 constexpr int kTileBytes = kTileKeys * kD * 2;           // 4 KB per tensor
-constexpr int kStageBytes = 2 * kTileBytes;              // K + V
-constexpr int kWarpBytes = kStages * kStageBytes;        // per-warp ring
+constexpr int kWarpBytes = 3 * kTileBytes;               // per-warp ring: K twice, V once
 
 struct AttnArgs {
     const uint16_t* Q;
@@ -57,7 +57,7 @@ __device__ __forceinline__ uint32_t swz(int row, int chunk) {
 // contiguous slice of its index tiles; partial softmax states are combined
 // through shared memory (decode, where rows are few).
 template <int SPLIT>
-__global__ void __launch_bounds__(32 * (SPLIT == 1 ? kAttnWarps : SPLIT)) attn_kernel(AttnArgs a) {
+__global__ void __launch_bounds__(32 * (SPLIT == 1 ? kAttnWarps : SPLIT), SPLIT == 1 ? 2 : 1) attn_kernel(AttnArgs a) {
     extern __shared__ __align__(128) uint8_t asmem[];
     const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
     const int64_t wg = SPLIT == 1 ? (int64_t)blockIdx.x * kAttnWarps + wid : (int64_t)blockIdx.x;
@@ -99,28 +99,30 @@ __global__ void __launch_bounds__(32 * (SPLIT == 1 ? kAttnWarps : SPLIT)) attn_k
         }
         return p;
     };
-    auto issue = [&](int tile, int stage, int p) {
+    // one 16-key tile of K (into K slot `slot`) or of V (its one slot), as a
+    // cp.async group of its own
+    auto issue = [&](int tile, uint32_t dst, const uint16_t* src, const uint16_t* src_sh, int p) {
         if (tile < ntiles) {
-            const uint32_t kb = wbase + stage * kStageBytes, vb = kb + kTileBytes;
 #pragma unroll
             for (int m = 0; m < 8; ++m) {
                 const int r = 2 * m + (lane >> 4), part = lane & 15;
                 const int pr = __shfl_sync(0xffffffffu, p, r);
                 if constexpr (SPLIT == 1) {
                     const int64_t off = (pr >= 0 ? (int64_t)pr : 0) * kv_stride + part * 8;
-                    cp_async_16(kb + swz(r, part), Kg + off, pr >= 0 ? 16 : 0);
-                    cp_async_16(vb + swz(r, part), Vg + off, pr >= 0 ? 16 : 0);
+                    cp_async_16(dst + swz(r, part), src + off, pr >= 0 ? 16 : 0);
                 } else {  // decode: the shared prefix, then the request's own rows
                     const bool sh = pr >= 0 && pr < a.shared_len;
                     const int64_t row = pr < 0 ? 0 : (sh ? (int64_t)pr : (int64_t)pr - a.shared_len);
                     const int64_t off = row * kv_stride + part * 8;
-                    cp_async_16(kb + swz(r, part), (sh ? Ksg : Kg) + off, pr >= 0 ? 16 : 0);
-                    cp_async_16(vb + swz(r, part), (sh ? Vsg : Vg) + off, pr >= 0 ? 16 : 0);
+                    cp_async_16(dst + swz(r, part), (sh ? src_sh : src) + off, pr >= 0 ? 16 : 0);
                 }
             }
         }
         cp_async_commit();
     };
+    const uint32_t vslot = wbase + 2 * kTileBytes;
+    auto issue_k = [&](int tile, int p) { issue(tile, wbase + (tile & 1) * kTileBytes, Kg, Ksg, p); };
+    auto issue_v = [&](int tile, int p) { issue(tile, vslot, Vg, Vsg, p); };
 
     float o[8][4];
 #pragma unroll
@@ -130,24 +132,22 @@ __global__ void __launch_bounds__(32 * (SPLIT == 1 ? kAttnWarps : SPLIT)) attn_k
     float m_run[2] = {-CUDART_INF_F, -CUDART_INF_F};
     float l_run[2] = {0.f, 0.f};
 
-    // pr[j]: positions of tile i + j (tiles i .. i + kStages - 2 are in
-    // flight, tile i + kStages - 1 is issued at the top of iteration i)
-    int pr[kStages];
-#pragma unroll
-    for (int j = 0; j < kStages; ++j) {
-        pr[j] = tile_pos(tbeg + j);
-        if (j < kStages - 1) issue(tbeg + j, (tbeg + j) % kStages, pr[j]);
-    }
+    // Tile i: K in slot i % 2, V in the one V slot.  Groups are committed in
+    // the order K(i), V(i), K(i + 1): S and the softmax of tile i wait for
+    // K(i) only, the PV product for V(i); then V(i + 1) and K(i + 2) go out.
+    int pr0 = tile_pos(tbeg), pr1 = tile_pos(tbeg + 1);
+    issue_k(tbeg, pr0);
+    issue_v(tbeg, pr0);
+    issue_k(tbeg + 1, pr1);
 
     for (int i = tbeg; i < ntiles; ++i) {
-        issue(i + kStages - 1, (i + kStages - 1) % kStages, pr[kStages - 1]);
-        const int pnext = tile_pos(i + kStages);  // consumed kStages - 1 iterations later
-        const unsigned vmask = __ballot_sync(0xffffffffu, pr[0] >= 0) & 0xFFFFu;
-        cp_async_wait<kStages - 1>();
+        const int pnext = tile_pos(i + 2);
+        const unsigned vmask = __ballot_sync(0xffffffffu, pr0 >= 0) & 0xFFFFu;
+        const uint32_t kb = wbase + (i & 1) * kTileBytes, vb = vslot;
+        uint32_t b0 = 0u, b1 = 0u;
+        cp_async_wait<2>();
         __syncwarp();
         if (vmask != 0) {
-            const int stage = i % kStages;
-            const uint32_t kb = wbase + stage * kStageBytes, vb = kb + kTileBytes;
             // S^T (16 keys x 8 heads): two independent accumulation chains
             float sa[4] = {0.f, 0.f, 0.f, 0.f}, sb[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
@@ -196,8 +196,13 @@ __global__ void __launch_bounds__(32 * (SPLIT == 1 ? kAttnWarps : SPLIT)) attn_k
             const uint32_t y1 = __shfl_sync(0xffffffffu, pk_hi, src1);
             const uint32_t y2 = __shfl_sync(0xffffffffu, pk_hi, src2);
             const uint32_t sel = (gq & 1) ? 0x7632u : 0x5410u;
-            uint32_t b0 = __byte_perm(x1, x2, sel), b1 = __byte_perm(y1, y2, sel);
+            b0 = __byte_perm(x1, x2, sel);
+            b1 = __byte_perm(y1, y2, sel);
             if (gq >= G) { b0 = 0u; b1 = 0u; }
+        }
+        cp_async_wait<1>();
+        __syncwarp();
+        if (vmask != 0) {
 #pragma unroll
             for (int mt = 0; mt < 8; ++mt) {
                 uint32_t af[4];
@@ -208,9 +213,10 @@ __global__ void __launch_bounds__(32 * (SPLIT == 1 ? kAttnWarps : SPLIT)) attn_k
             }
         }
         __syncwarp();
-#pragma unroll
-        for (int j = 0; j + 1 < kStages; ++j) pr[j] = pr[j + 1];
-        pr[kStages - 1] = pnext;
+        issue_v(i + 1, pr1);
+        issue_k(i + 2, pnext);
+        pr0 = pr1;
+        pr1 = pnext;
     }
     cp_async_wait<0>();
     __syncwarp();
