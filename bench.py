@@ -42,7 +42,7 @@ UNIT = "tokens/s"
 # (the committed ncu summary of attn_kernel gives the command); reported as
 # `traffic` only while the kernel's source (the text from its template header
 # to its launcher, hashed) is the one that capture measured.
-ATTN_TRAFFIC = {"kernel_sha256_prefix": "de8295bbc85d176c", "bytes_per_query_kvhead": 21968.7,
+ATTN_TRAFFIC = {"kernel_sha256_prefix": "d24e17fa489f0fb0", "bytes_per_query_kvhead": 19224.3,
                 "workload": "prefill-128k"}
 
 
@@ -459,6 +459,11 @@ def run_lsa(args):
     ranked = sorted((n for n in work if n in kernels), key=lambda n: -kernels[n]["ms_per_step"])
     roofline = roof(ranked[0]) if ranked else None
     roofline_scoring = roof("flat_cand_kernel")
+    if roofline_scoring:
+        roofline_scoring["note"] = ("tcgen05 scores of every eligible centroid; the epilogue appends the candidates "
+                                    "(score >= tau, about 2k keys' buckets per row), so the share of scores that are "
+                                    "candidates -- high at short contexts -- bounds it with the tensor core's "
+                                    "shared-memory operand reads")
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu:
         if not host_drawn:  # the oracle sample reads head 0's K/V and the query rows
