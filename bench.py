@@ -46,6 +46,12 @@ ATTN_TRAFFIC = {"kernel_sha256_prefix": "d24e17fa489f0fb0", "bytes_per_query_kvh
                 "workload": "prefill-128k"}
 
 
+# Peak of the L2-to-SM read path on this machine's B200s, from ncu's
+# l1tex__m_xbar2l1tex_read_bytes.sum.per_second (12.905 TB/s) and its
+# pct_of_peak_sustained_elapsed (37.04%) for the gather attention kernel.
+L2_TO_SM_PEAK_GBS = 12904.99 / 0.3703643
+
+
 def attn_kernel_hash():
     import hashlib
     src = open(os.path.join(ROOT, "clustered_key_indexing_b200/csrc/lsa_attn.cu")).read()
@@ -454,6 +460,12 @@ def run_lsa(args):
                 r["traffic"] = ATTN_TRAFFIC["bytes_per_query_kvhead"] * T * hkv / k["launches_per_step"]
             r["note"] = ("gathered K/V rows are served mostly from L2 (one kv-head's K/V per wave), so the "
                          "algorithmic bytes can exceed the HBM copy peak; traffic = ncu DRAM bytes")
+            # the same bytes against the L2-to-SM read path, whose peak ncu
+            # gives as l1tex__m_xbar2l1tex_read_bytes' pct_of_peak (12.90
+            # TB/s measured = 37.04% of peak in the 256K-prefix capture)
+            l2_peak = L2_TO_SM_PEAK_GBS
+            r["l2_view"] = {"achieved": ach, "peak": l2_peak, "unit": "GB/s", "frac": ach / l2_peak,
+                            "peak_source": "ncu: l1tex__m_xbar2l1tex_read_bytes per second / its pct_of_peak"}
         return r
 
     ranked = sorted((n for n in work if n in kernels), key=lambda n: -kernels[n]["ms_per_step"])
