@@ -601,6 +601,36 @@ __device__ __forceinline__ double exact_row(const uint16_t* ylat, int ng, const 
     return best;
 }
 
+// exact_row for four centroids at once: four independent fma chains (each
+// in ascending dimension order, so every score equals exact_row's).
+__device__ __forceinline__ void exact_rows4(const uint16_t* ylat, int ng, const uint16_t* const (&c)[4],
+                                            double (&out)[4]) {
+#pragma unroll
+    for (int j = 0; j < 4; ++j) out[j] = -CUDART_INF;
+    for (int g = 0; g < ng; ++g) {
+        const uint16_t* y = ylat + g * kDL;
+        double s[4] = {0.0, 0.0, 0.0, 0.0};
+#pragma unroll 2
+        for (int i = 0; i < 8; ++i) {
+            uint4 cv[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) cv[j] = __ldg(reinterpret_cast<const uint4*>(c[j]) + i);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const double y0 = bf16_to_f64(y[8 * i + 2 * e]), y1 = bf16_to_f64(y[8 * i + 2 * e + 1]);
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const uint32_t w = e == 0 ? cv[j].x : e == 1 ? cv[j].y : e == 2 ? cv[j].z : cv[j].w;
+                    s[j] = fma(y0, (double)__uint_as_float(w << 16), s[j]);
+                    s[j] = fma(y1, (double)__uint_as_float(w & 0xFFFF0000u), s[j]);
+                }
+            }
+        }
+#pragma unroll
+        for (int j = 0; j < 4; ++j) out[j] = s[j] > out[j] ? s[j] : out[j];
+    }
+}
+
 __device__ __forceinline__ void push_fallback(const ResolveArgs& a, int64_t row) {
     atomicAdd(&g_lsa_fallback_rows, 1ull);
     const int slot = atomicAdd(a.ovf_count, 1);

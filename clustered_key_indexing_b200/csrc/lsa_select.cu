@@ -343,7 +343,7 @@ __host__ __device__ inline size_t tree_warp_bytes(int maxn) {
     return (((size_t)maxn * 16 + 256 * 4 + 8 * kDL * 2) + 15) & ~(size_t)15;
 }
 
-__global__ void __launch_bounds__(32 * kTreeWarps) tree_warp_kernel(SelectArgs a, int64_t nrows, int maxn) {
+__global__ void __launch_bounds__(32 * kTreeWarps, 4) tree_warp_kernel(SelectArgs a, int64_t nrows, int maxn) {
     extern __shared__ __align__(16) uint8_t tsm[];
     const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
     const int64_t row = (int64_t)blockIdx.x * kTreeWarps + wid;
@@ -444,11 +444,25 @@ __global__ void __launch_bounds__(32 * kTreeWarps) tree_warp_kernel(SelectArgs a
     }
     __syncwarp();
     long long totw = 0;
-    for (int i = lane; i < n; i += 32) {
-        const int64_t b = id[i];
-        sc[i] = exact_row(ylat, ng, a.cent + (hb0 + b) * kDL);
-        wt[i] = bucket_weight(a, r.h, b, r.lim);
-        totw += wt[i];
+    // leaves four per lane at a time (i, i + 32, i + 64, i + 96): four
+    // independent exact-score chains in flight
+    for (int i0 = 0; i0 < n; i0 += 128) {
+        const uint16_t* cp[4];
+        int ii[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            ii[j] = i0 + lane + 32 * j;
+            cp[j] = a.cent + (hb0 + (ii[j] < n ? id[ii[j]] : id[0])) * kDL;
+        }
+        double sv[4];
+        exact_rows4(ylat, ng, cp, sv);
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+            if (ii[j] < n) {
+                sc[ii[j]] = sv[j];
+                wt[ii[j]] = bucket_weight(a, r.h, id[ii[j]], r.lim);
+                totw += wt[ii[j]];
+            }
     }
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) totw += __shfl_xor_sync(0xffffffffu, totw, off);
