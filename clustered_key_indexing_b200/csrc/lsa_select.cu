@@ -339,6 +339,36 @@ constexpr int kTreeWarps = 4;
 // Leaves a row can reach: at most beam subtrees of 2^L* buckets.
 static inline int tree_max_cands(int beam, int lstar) { return beam << lstar; }
 
+// Exponent spread of the nonzero bf16 values among `b` (biased exponents,
+// subnormals counted as exponent 1): returns (max << 8) | min, or 0 if all
+// are zero.
+__device__ __forceinline__ uint32_t bf16_exp_span(uint32_t lo_bits, uint32_t hi_bits) {
+    uint32_t mn = 255u, mx = 0u;
+    const uint32_t v[2] = {lo_bits, hi_bits};
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+        const uint32_t b = v[i] & 0xFFFFu;
+        if (b & 0x7FFFu) {
+            const uint32_t e = max(1u, (b >> 7) & 0xFFu);
+            mn = min(mn, e);
+            mx = max(mx, e);
+        }
+    }
+    return mx ? (mx << 8) | mn : 0u;
+}
+
+// Exactness test of a dot product of two bf16 vectors in fp64: with every
+// product exact (8-bit significands) and the spreads of the two vectors'
+// nonzero exponents summing to at most 30, every partial sum is an integer
+// multiple of the smallest product quantum below 2^53 of them, so any order
+// of summation gives the exact sum -- the ascending sequential sum included.
+__device__ __forceinline__ int exp_range(uint32_t span) { return span ? (int)(span >> 8) - (int)(span & 0xFFu) : 0; }
+__device__ __forceinline__ uint32_t span_merge(uint32_t a, uint32_t b) {
+    if (!a) return b;
+    if (!b) return a;
+    return (max(a >> 8, b >> 8) << 8) | min(a & 0xFFu, b & 0xFFu);
+}
+
 __host__ __device__ inline size_t tree_warp_bytes(int maxn) {
     return (((size_t)maxn * 16 + 256 * 4 + 8 * kDL * 2) + 15) & ~(size_t)15;
 }
@@ -369,6 +399,14 @@ __global__ void __launch_bounds__(32 * kTreeWarps, 4) tree_warp_kernel(SelectArg
                                  : a.Y + (r.q * (int64_t)a.hkv + r.h) * kDL;
     for (int i = lane; i < ng * kDL; i += 32) ylat[i] = ysrc[i];
     __syncwarp();
+    // the widest exponent spread over the row's latent(s), for the exactness test
+    int yrange = 0;
+    for (int g = 0; g < ng; ++g) {
+        uint32_t sp = bf16_exp_span(ylat[g * kDL + 2 * lane], ylat[g * kDL + 2 * lane + 1]);
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) sp = span_merge(sp, __shfl_xor_sync(0xffffffffu, sp, off));
+        yrange = max(yrange, exp_range(sp));
+    }
 
     // descent: lane i < nbeam holds beam node i (ascending index)
     const int64_t hn = (int64_t)r.h * a.n_nodes;
@@ -382,6 +420,44 @@ __global__ void __launch_bounds__(32 * kTreeWarps, 4) tree_warp_kernel(SelectArg
     for (int lvl = top; lvl > a.lstar && nbeam > 0; --lvl) {
         const int64_t nl = a.level_n[lvl - 1];
         const int nc = 2 * nbeam;  // children of the beam (<= 16)
+        // exact scores of the children, 8 lanes per child (8 dimensions each,
+        // combined in a fixed tree), four children per pass; a child whose
+        // vectors fail the exactness test is scored sequentially instead
+        double s_all = -CUDART_INF;  // lane j < nc: child j's score
+        for (int p0 = 0; p0 < nc; p0 += 4) {
+            const int j = p0 + (lane >> 3), part = lane & 7;
+            const long long parj = __shfl_sync(0xffffffffu, mybeam, (j >> 1) & 31);
+            const long long chj = 2 * parj + (j & 1);
+            const bool act = j < nc && chj < nl;
+            const int64_t gj = hn + a.level_off[lvl - 1] + (act ? chj : 0);
+            const uint4 cv = act ? __ldg(reinterpret_cast<const uint4*>(a.tcent + gj * kDL) + part)
+                                 : make_uint4(0u, 0u, 0u, 0u);
+            const uint32_t cw[4] = {cv.x, cv.y, cv.z, cv.w};
+            uint32_t sp = 0u;
+#pragma unroll
+            for (int e = 0; e < 4; ++e) sp = span_merge(sp, bf16_exp_span(cw[e] & 0xFFFFu, cw[e] >> 16));
+#pragma unroll
+            for (int off = 1; off < 8; off <<= 1) sp = span_merge(sp, __shfl_xor_sync(0xffffffffu, sp, off));
+            double best = -CUDART_INF;
+            for (int g = 0; g < ng; ++g) {
+                const uint16_t* y = ylat + g * kDL + 8 * part;
+                double ps = 0.0;
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    ps = fma(bf16_to_f64(y[2 * e]), (double)__uint_as_float(cw[e] << 16), ps);
+                    ps = fma(bf16_to_f64(y[2 * e + 1]), (double)__uint_as_float(cw[e] & 0xFFFF0000u), ps);
+                }
+#pragma unroll
+                for (int off = 1; off < 8; off <<= 1) ps += __shfl_xor_sync(0xffffffffu, ps, off);
+                best = ps > best ? ps : best;
+            }
+            if (act && part == 0 && yrange + exp_range(sp) > 30) best = exact_row(ylat, ng, a.tcent + gj * kDL);
+#pragma unroll
+            for (int q4 = 0; q4 < 4; ++q4) {
+                const double v = __shfl_sync(0xffffffffu, best, 8 * q4);
+                if (lane == p0 + q4) s_all = v;
+            }
+        }
         const long long par = __shfl_sync(0xffffffffu, mybeam, (lane >> 1) & 31);
         double s = -CUDART_INF;
         long long node = -1;
@@ -390,7 +466,7 @@ __global__ void __launch_bounds__(32 * kTreeWarps, 4) tree_warp_kernel(SelectArg
             if (ch < nl) {
                 const int64_t gi = hn + a.level_off[lvl - 1] + ch;
                 if ((int64_t)a.tminlr[gi] <= r.lim) {
-                    s = exact_row(ylat, ng, a.tcent + gi * kDL);
+                    s = s_all;
                     node = ch;
                 }
             }
