@@ -293,3 +293,30 @@ def test_prefill_host_equals_prefill(lsa, mode):
     torch.cuda.synchronize()
     lsa.check_device_error()
     assert torch.equal(hO.view(torch.int16), O_dev.cpu().view(torch.int16))
+
+
+@pytest.mark.parametrize("scale_q,scale_k", [(2.0 ** -40, 1.0), (1.0, 2.0 ** -40), (2.0 ** -20, 2.0 ** -20)])
+def test_tree_exponent_spread_fallback(lsa, scale_q, scale_k):
+    """Latents with a component ~2^-40 of the others (one column of W_q or W_k
+    scaled) fail the exponent-spread test of the parallel tree descent, so the
+    children are scored sequentially; selections stay bit-exact."""
+    T = 4096
+    cfg = lsa.Config(k=512, sinks=4, window=256, mode=1)
+    inp = synth.layer_inputs("prefill-4k", T=T)
+    Wk, Wq = inp["Wk"].copy(), inp["Wq"].copy()
+    Wk[:, 5] *= np.float32(scale_k)
+    Wq[:, 5] *= np.float32(scale_q)
+    K, Q = to_dev_bf16(inp["K"]), to_dev_bf16(inp["Q"])
+    cache = lsa.Cache(1, T, cfg)
+    lsa.build_buckets(K, to_dev(Wk), cfg, cache)
+    tree = lsa.build_tree(cache, cfg)
+    idx = lsa.select(Q, 0, to_dev(Wq), cache, cfg, tree=tree)
+    torch.cuda.synchronize()
+    lsa.check_device_error()
+    ocfg = oracle_cfg(cfg)
+    U = oracle.key_latent_pool(inp["K"], Wk, 4)
+    oc = oracle.build_cache(U, T, ocfg)
+    tpos = np.arange(0, T, 7)
+    Y = oracle.query_latent(inp["Q"][tpos], Wq, 1, 0)
+    oidx, _, _ = oracle.select(oc, Y, tpos, ocfg, tree=oracle.build_tree(oc), G=4)
+    assert np.array_equal(idx.cpu().numpy()[tpos], oidx)

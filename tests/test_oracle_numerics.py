@@ -2,6 +2,8 @@
 key / query latents (essay "《卡片柜》", ch. 2; tutorial "隐空间稀疏注意力",
 section 二).  Each check compares with something other than the oracle itself:
 brute force over all bf16 values, closed forms, or invariances."""
+import math
+
 import numpy as np
 import pytest
 
@@ -123,3 +125,38 @@ def test_query_latent_closed_form_and_group_mean():
     # the group mean is rounded once; fp64 summation order can differ only by
     # an ulp, which moves a bf16 rounding only at an exact midpoint
     assert np.mean(Ym == oracle.bf16_rne(zm.reshape(-1)).reshape(zm.shape)) > 0.999
+
+
+def test_bf16_dot_exact_in_any_order_when_exponent_spread_is_small():
+    """The lemma behind the tree descent's parallel exact scores: with bf16
+    factors (8-bit significands) and nonzero-exponent spreads summing to at
+    most 30 over the two vectors, every fp64 partial sum is exact, so any
+    summation order equals the ascending sequential fma chain."""
+    import random
+    rng = np.random.default_rng(5)
+
+    def bf16_vec(lo_exp, hi_exp):
+        e = rng.integers(lo_exp, hi_exp + 1, size=64)
+        m = rng.integers(128, 256, size=64)
+        s = rng.choice([-1.0, 1.0], size=64)
+        return s * m * np.exp2(e - 7.0)
+
+    def seq(y, c):
+        acc = 0.0
+        for a, b in zip(y, c):
+            acc = acc + a * b  # each product is exact in fp64
+        return acc
+
+    for _ in range(200):
+        y = bf16_vec(-12, 0)     # spread 12
+        c = bf16_vec(-18, 0)     # spread 18: total 30
+        ref = seq(y, c)
+        prods = list(y * c)
+        for _ in range(5):
+            random.shuffle(prods)
+            assert sum(prods) == ref
+            assert math.fsum(prods) == ref
+    # and the bound is needed: widely spread exponents lose the exactness
+    y = np.array([1.0, 2.0 ** -60, -1.0] + [0.0] * 61)
+    c = np.ones(64)
+    assert seq(y, c) != math.fsum(list(y * c))
