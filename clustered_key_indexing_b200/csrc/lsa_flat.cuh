@@ -531,6 +531,7 @@ struct ResWarp {
     double bex[kBandCap];     // exact scores of the band
     int2 cs[kCandCap];        // eligible candidates (bucket id, fp32 score bits), ascending id
     uint8_t w[kCandCap];      // key weights (<= 16), then taken counts
+    int32_t pk[kCandCap];     // packed member units of each candidate (from its record)
     int16_t bidx[kBandCap];   // band members (index into cs)
     uint32_t hist[256];
     uint16_t ylat[8 * kDL];
@@ -739,6 +740,7 @@ __global__ void __launch_bounds__(32 * kResWarps, 3) flat_resolve_kernel(Resolve
         int wgt = 0;
         if ((int64_t)md.x <= lim) wgt = (int64_t)md.y <= lim ? md.z : weight_packed(col, md.w, lim, a.S, a.T_built);
         sw.w[i] = (uint8_t)wgt;
+        sw.pk[i] = md.w;
     }
     __syncwarp();
     int m = 0;
@@ -748,6 +750,7 @@ __global__ void __launch_bounds__(32 * kResWarps, 3) flat_resolve_kernel(Resolve
         const int i = base + lane;
         const int2 cv = i < n ? sw.cs[i] : make_int2(0, 0);
         const int wgt = i < n ? sw.w[i] : 0;
+        const int32_t pkv = i < n ? sw.pk[i] : 0;
         const bool el = wgt > 0;
         if (el) {
             wtot += wgt;
@@ -760,6 +763,7 @@ __global__ void __launch_bounds__(32 * kResWarps, 3) flat_resolve_kernel(Resolve
             const int pos = m + __popc(bal & ((1u << lane) - 1u));
             sw.cs[pos] = cv;
             sw.w[pos] = (uint8_t)wgt;
+            sw.pk[pos] = pkv;
         }
         m += __popc(bal);
     }
@@ -845,33 +849,37 @@ __global__ void __launch_bounds__(32 * kResWarps, 3) flat_resolve_kernel(Resolve
             sw.w[i] = sc > hi ? sw.w[i] : (sc >= lo ? (uint8_t)(0x80u | sw.w[i]) : (uint8_t)0);
         }
         __syncwarp();
-        long long need = a.k - win;
-        while (need > 0) {
-            // best pending band bucket: exact score desc, bucket id asc
-            double bs = -CUDART_INF;
-            int bb = -1, bcol = 0x7FFFFFFF;
-            for (int i = lane; i < nb; i += 32) {
-                const int ci = sw.bidx[i];
-                if (!(sw.w[ci] & 0x80u)) continue;
-                const double e = sw.bex[i];
-                const int col = sw.cs[ci].x;
-                if (bb < 0 || e > bs || (e == bs && col < bcol)) { bs = e; bb = ci; bcol = col; }
-            }
+        // the greedy fill of the band (best exact score first, lower bucket id
+        // on ties) in closed form: a band bucket takes what is left of the
+        // need after the weight of every band bucket ranked above it
+        const long long need = a.k - win;
+        int tk_reg[kBandCap / 32];
 #pragma unroll
-            for (int off = 16; off > 0; off >>= 1) {
-                const double os = __shfl_xor_sync(0xffffffffu, bs, off);
-                const int ob = __shfl_xor_sync(0xffffffffu, bb, off);
-                const int oc = __shfl_xor_sync(0xffffffffu, bcol, off);
-                if (ob >= 0 && (bb < 0 || os > bs || (os == bs && oc < bcol))) { bs = os; bb = ob; bcol = oc; }
+        for (int u = 0; u < kBandCap / 32; ++u) {
+            const int i = lane + 32 * u;
+            tk_reg[u] = 0;
+            if (i < nb) {
+                const int ci = sw.bidx[i];
+                const double ei = sw.bex[i];
+                const int coli = sw.cs[ci].x;
+                long long above = 0;
+                for (int j = 0; j < nb; ++j) {
+                    const double ej = sw.bex[j];
+                    const int cj = sw.bidx[j];
+                    if (ej > ei || (ej == ei && sw.cs[cj].x < coli)) above += sw.w[cj] & 0x7F;
+                }
+                const long long left = need - above;
+                const int wv = sw.w[ci] & 0x7F;
+                tk_reg[u] = left <= 0 ? 0 : (left < wv ? (int)left : wv);
             }
-            if (bb < 0) break;
-            const int wv = sw.w[bb] & 0x7F;
-            const int tk = wv < need ? wv : (int)need;
-            __syncwarp();
-            if (lane == 0) sw.w[bb] = (uint8_t)tk;
-            need -= tk;
-            __syncwarp();
         }
+        __syncwarp();
+#pragma unroll
+        for (int u = 0; u < kBandCap / 32; ++u) {
+            const int i = lane + 32 * u;
+            if (i < nb) sw.w[sw.bidx[i]] = (uint8_t)tk_reg[u];
+        }
+        __syncwarp();
         for (int i = lane; i < m; i += 32)
             if (sw.w[i] & 0x80u) sw.w[i] = 0;
         __syncwarp();
@@ -893,7 +901,7 @@ __global__ void __launch_bounds__(32 * kResWarps, 3) flat_resolve_kernel(Resolve
         }
         if (tk > 0) {
             const int col = sw.cs[i].x;
-            emit_keys(col, __ldg(&mrow[col].w), tk, lim, a.S, a.T_built, out, a.S + run + incl - tk);
+            emit_keys(col, sw.pk[i], tk, lim, a.S, a.T_built, out, a.S + run + incl - tk);
         }
         run += __shfl_sync(0xffffffffu, incl, 31);
     }
