@@ -733,14 +733,25 @@ __global__ void __launch_bounds__(32 * kResWarps, 3) flat_resolve_kernel(Resolve
 #pragma unroll 4
     for (int i = lane; i < n; i += 32) sw.cs[i] = crow[i];
     __syncwarp();
-#pragma unroll 4
-    for (int i = lane; i < n; i += 32) {
-        const int col = sw.cs[i].x;
-        const int4 md = __ldg(mrow + col);
-        int wgt = 0;
-        if ((int64_t)md.x <= lim) wgt = (int64_t)md.y <= lim ? md.z : weight_packed(col, md.w, lim, a.S, a.T_built);
-        sw.w[i] = (uint8_t)wgt;
-        sw.pk[i] = md.w;
+    // the records of 8 candidates per lane are requested before any is used
+    for (int i0 = lane; i0 < n; i0 += 32 * 8) {
+        int4 md[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const int i = i0 + 32 * u;
+            md[u] = i < n ? __ldg(mrow + sw.cs[i].x) : make_int4(0, 0, 0, 0);
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const int i = i0 + 32 * u;
+            if (i < n) {
+                int wgt = 0;
+                if ((int64_t)md[u].x <= lim)
+                    wgt = (int64_t)md[u].y <= lim ? md[u].z : weight_packed(sw.cs[i].x, md[u].w, lim, a.S, a.T_built);
+                sw.w[i] = (uint8_t)wgt;
+                sw.pk[i] = md[u].w;
+            }
+        }
     }
     __syncwarp();
     int m = 0;
