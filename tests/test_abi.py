@@ -5,6 +5,7 @@ import ctypes
 import os
 import subprocess
 
+import numpy as np
 import pytest
 
 from clustered_key_indexing_b200 import _lib
@@ -81,3 +82,24 @@ def test_compute_calls_reject_bad_arguments_before_any_launch(L):
     assert L.lsa_select(None, 0, 1, 4, None, None, None, ctypes.byref(c), None, None, None, 0, None) == LSA_EINVAL
     assert L.lsa_prefill(None, None, None, 16, 4, 1, None, None, ctypes.byref(c), None, None, None, 0,
                          None, 0, None) == LSA_EINVAL
+
+
+def test_prefill_chunk_is_whole_waves_of_the_candidate_kernel(L):
+    """Host logic: in flat mode the query chunk is a whole number of waves of
+    the candidate kernel (512 / G latent rows per CTA, CTAs a multiple of the
+    148 SMs), the nearest to the request; tree mode keeps the request."""
+    import clustered_key_indexing_b200 as lsa
+    for agg, G in ((0, 1), (1, 4)):
+        cfg = lsa.Config(k=2048, sinks=4, window=1024, agg=agg)
+        for T, hkv, hq in ((131072, 8, 32), (1 << 20, 8, 32), (50000, 2, 8)):
+            ch = lsa.prefill_chunk(cfg, T, hq, hkv, 16384)
+            if ch == T:
+                continue
+            rows_per_cta = 512 // (hq // hkv if agg else 1)
+            assert ch % rows_per_cta == 0
+            assert (ch // rows_per_cta * hkv) % 148 == 0, (agg, T, ch)
+            wave = rows_per_cta * 148 // np.gcd(148, hkv)
+            assert abs(ch - 16384) <= wave // 2 + 1 or ch == wave
+    tree = lsa.Config(k=2048, sinks=4, window=1024, mode=1)
+    assert lsa.prefill_chunk(tree, 131072, 32, 8, 16384) == 16384
+    assert lsa.prefill_chunk(tree, 3000, 8, 2, 700) == 700
