@@ -314,6 +314,15 @@ __global__ void __launch_bounds__(128) decode_score_kernel(const __grid_constant
     int done = 0;  // tiles consumed
     for (int it = 0; it < ntiles; ++it) {
         const int s = it % kDecStages;
+        // this tile's key counts, requested before the scores so that their
+        // latency overlaps the MMAs (two slots per thread)
+        const int64_t tb0 = c0 + (int64_t)it * kDecTile;
+        int32_t clr_pre[kDecTile / 128];
+#pragma unroll
+        for (int u = 0; u < kDecTile / 128; ++u) {
+            const int64_t b = tb0 + tid + 128 * u;
+            clr_pre[u] = b < cend ? __ldg(a.cnt_lr + hb0 + b) : 0;
+        }
         const bool ok = mbar_wait(bar0 + 8u * s, (uint32_t)(it / kDecStages) & 1u, abort_flag);
         if (!__syncthreads_and(ok)) break;
         const uint32_t tb = smem_u32(ring + s * kDecTile * kDL * 2);
@@ -355,11 +364,12 @@ __global__ void __launch_bounds__(128) decode_score_kernel(const __grid_constant
                         (int32_t)(rowbase + c0 + (it + kDecStages) * kDecTile), bar0 + 8u * s);
         }
         // bins and weights of the tile, coalesced
-        const int64_t tb0 = c0 + (int64_t)it * kDecTile;
-        for (int j = tid; j < kDecTile; j += 128) {
+#pragma unroll
+        for (int u = 0; u < kDecTile / 128; ++u) {
+            const int j = tid + 128 * u;
             const int64_t b = tb0 + j;
             if (b >= cend) break;
-            const int32_t clr = __ldg(a.cnt_lr + hb0 + b);
+            const int32_t clr = clr_pre[u];
             int w = clr;
             if (b >= frontier) {
                 const int32_t mlr = __ldg(a.minlr + hb0 + b), mxp = __ldg(a.maxpos + hb0 + b);
