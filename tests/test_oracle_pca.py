@@ -89,6 +89,9 @@ def test_structure():
     Xc = X - X.mean(axis=0)
     C = Xc.T @ Xc / X.shape[0]
     assert np.abs(C @ V - V * lam[None, :]).max() < 1e-12 * np.abs(C).max() * 128
+    # the projection holds the leading directions as its columns (fp32)
+    Wd = W.astype(np.float64)
+    assert np.abs(C @ Wd - Wd * lam[None, :64]).max() < 1e-5 * lam[0]
     for j in range(128):  # sign convention: the largest-magnitude entry is positive
         i = int(np.argmax(np.abs(V[:, j])))
         assert V[i, j] > 0

@@ -2,10 +2,13 @@
 attention (essay "《卡片柜》", ch. 3-5; tutorial "隐空间稀疏注意力", section 二).
 
 Independent checks: the all-buckets case reduces to full causal attention
-(torch's scaled_dot_product_attention in fp64); the flat fill is a top set
+(torch's scaled_dot_product_attention in fp64), with one and with 8 kv-heads
+of 4 query heads; single-key lists (a closed form); the flat fill is a top set
 under independently computed exact scores; structural invariants of each index
-row; tree with a beam wider than every level equals flat; beam 1 equals a
-greedy single-path descent written here; comparison counts O(T/8) vs O(log T).
+row; rows written out by hand on a hand-built cache (a bucket holding sink
+keys, exact score ties); tree with a beam wider than every level equals flat;
+beam 1 equals a greedy single-path descent written here; comparison counts
+O(T/8) vs O(log T).
 """
 import numpy as np
 import pytest
@@ -234,3 +237,126 @@ def test_tree_structure_and_log_comparisons(built):
     _, _, nc = oracle.select(cache, Y, tpos, c2, tree=tr, G=4)
     H = len(ln) - 1  # 9 levels above the leaves for 512 buckets
     assert nc[0, 0] <= 2 * 2 * (H - 5) + 2 * 2 ** 5
+
+
+@pytest.fixture(scope="module")
+def gqa_inputs():
+    """160 tokens of the 8 kv-head / 32 query-head layer."""
+    return _inputs(160, hkv=8, hq=32, name="prefill-128k")
+
+
+def test_full_causal_attention_with_gqa_groups(gqa_inputs):
+    """k >= T with 8 kv-heads of 4 query heads each: query head h attends
+    with kv-head h // 4 (the GQA grouping), checked against SDPA in fp64."""
+    T = 160
+    inp = gqa_inputs
+    cfg = oracle.Cfg(k=T, sinks=4, window=16)
+    r = oracle.layer(inp["Q"], inp["K"], inp["V"], inp["Wk"], inp["Wq"], cfg)
+    q = torch.tensor(oracle.bf16_to_f64(inp["Q"])).permute(1, 0, 2)      # [32, T, d]
+    k = torch.tensor(oracle.bf16_to_f64(inp["K"])).permute(1, 0, 2).repeat_interleave(4, dim=0)
+    v = torch.tensor(oracle.bf16_to_f64(inp["V"])).permute(1, 0, 2).repeat_interleave(4, dim=0)
+    ref = torch.nn.functional.scaled_dot_product_attention(q, k, v, is_causal=True)
+    assert np.allclose(r["O"], ref.permute(1, 0, 2).numpy(), atol=1e-12, rtol=0)
+
+
+def test_each_query_head_reads_its_groups_list(gqa_inputs):
+    """One distinct key per kv-head list: a softmax over one key is 1, so
+    query head h returns the V row of its group's key, V[key(h // 4), h // 4]."""
+    inp = gqa_inputs
+    idx = np.full((1, 8, 5), -1, np.int32)
+    keys = [3 * g + 1 for g in range(8)]
+    for g in range(8):
+        idx[0, g, 2] = keys[g]
+    O = oracle.attention(inp["Q"][:1], inp["K"], inp["V"], idx)
+    Vf = oracle.bf16_to_f64(inp["V"])
+    for h in range(32):
+        assert np.array_equal(O[0, h], Vf[keys[h // 4], h // 4]), h
+
+
+def _hand_cache(groups, T, S, vecs, dl=64, pool=4):
+    """A one-head bucket cache made from explicit member lists; the bucket
+    metadata follows its definition (unit j holds keys pool*j .. pool*j+3),
+    and both the sum and the centroid of bucket b are the bf16-exact vector
+    vecs[b] (the flat fill reads only the centroid; the tree reads sums)."""
+    NU = (T + pool - 1) // pool
+    NB = len(groups)
+    members, offsets, cnt, mlr, mxp = [], [0], [], [], []
+    bou = np.full((1, NU), -1, np.int32)
+    for b, g in enumerate(groups):
+        g = sorted(g)
+        members += g
+        offsets.append(len(members))
+        keys = [p for j in g for p in range(pool * j, min(pool * j + pool, T))]
+        lr = [p for p in keys if p >= S]
+        cnt.append(len(lr))
+        mlr.append(min(lr) if lr else oracle.IMAX)
+        mxp.append(max(keys) if keys else -1)
+        bou[0, g] = b
+    assert sorted(members) == list(range(NU))
+    V = np.zeros((1, NB, dl))
+    V[0, :, :len(vecs[0])] = np.asarray(vecs, np.float64)
+    cent = synth.f32_to_bf16_bits(V.astype(np.float32))
+    assert np.array_equal(oracle.bf16_to_f64(cent), V)
+    i32 = lambda a: np.asarray(a, np.int32)[None, :]
+    return dict(T=T, H=1, NU=NU, NB=NB, nblk=1, bucket_of_unit=bou,
+                members=i32(members), offsets=i32(offsets), cnt_lr=i32(cnt),
+                minlr=i32(mlr), maxpos=i32(mxp), sum=V, cent=cent,
+                ward_margin=np.zeros((1, 1)))
+
+
+def _e0(dl=64):
+    y = np.zeros((1, 1, dl), np.float32)
+    y[0, 0, 0] = 1.0
+    return synth.f32_to_bf16_bits(y)
+
+
+def test_flat_fill_on_a_hand_built_cache():
+    """Rows written out by hand from the definition of the flat fill.
+
+    Bucket 0 holds the sink keys 0-3, keys 20-23 and keys 56-59, so at t = 40
+    (R_t = [4, 32]) only its 4 keys 20-23 count. Buckets 1 and 2 score
+    exactly the same; the lower bucket id wins the tie."""
+    groups = [[0, 5, 14], [1, 2], [3, 4], [6, 7, 8, 9, 10, 11, 12, 13, 15]]
+    c = _hand_cache(groups, 64, 4, [[1.0], [0.5], [0.5], [0.25]])
+    y = _e0()
+    cfg = oracle.Cfg(k=8, sinks=4, window=8)
+    idx, _, _ = oracle.select(c, y, np.array([40]), cfg, G=1)
+    assert idx[0, 0].tolist() == [0, 1, 2, 3,
+                                  20, 21, 22, 23, 4, 5, 6, 7,
+                                  33, 34, 35, 36, 37, 38, 39, 40]
+    cfg = oracle.Cfg(k=24, sinks=4, window=8)
+    rows = {}
+    for t in (63, 5, 2):
+        idx, _, _ = oracle.select(c, y, np.array([t]), cfg, G=1)
+        rows[t] = idx[0, 0].tolist()
+    # t = 63: R_t = [4, 55]; bucket 0 gives 20-23, bucket 1 (tie won) 4-11,
+    # bucket 2 12-19, bucket 3 the lowest 4 of its keys in R_t
+    assert rows[63] == [0, 1, 2, 3,
+                        20, 21, 22, 23, *range(4, 12), *range(12, 20), 24, 25, 26, 27,
+                        *range(56, 64)]
+    # t = 5: no long-range key yet; window 4-5.  t = 2: sinks 0-2 only.
+    assert rows[5] == [0, 1, 2, 3] + [-1] * 24 + [4, 5] + [-1] * 6
+    assert rows[2] == [0, 1, 2, -1] + [-1] * 24 + [-1] * 8
+
+
+def test_ties_take_the_lower_id_in_flat_and_tree():
+    """Buckets 0 and 3 have one centroid, buckets 1 and 2 another, so both
+    level-1 tree nodes have the same centroid: the beam of 1 keeps node 0 and
+    the flat fill breaks both ties by the lower bucket id."""
+    groups = [[0, 1], [2, 3], [4, 5], [6, 7]]
+    c = _hand_cache(groups, 32, 4, [[2.0, 1.0], [1.0, 2.0], [1.0, 2.0], [2.0, 1.0]])
+    # the flat fill reads centroids: make them the normalised sums, in bf16
+    s = c["sum"][0]
+    c["cent"] = oracle.bf16_rne(s / np.linalg.norm(s, axis=1, keepdims=True)).reshape(1, 4, 64)
+    y = _e0()
+    tr = oracle.build_tree(c)
+    lo = tr["level_off"]
+    assert np.array_equal(tr["cent"][0, lo[1]], tr["cent"][0, lo[1] + 1])
+    t = np.array([31])                                  # R_t = [4, 27]
+    flat = oracle.select(c, y, t, oracle.Cfg(k=16, sinks=4, window=4), G=1)[0][0, 0]
+    # b0 and b3 tie first (b0 4-7, b3 24-27), then b1 beats b2 for the last 8
+    assert flat.tolist() == [0, 1, 2, 3, *range(4, 16), 24, 25, 26, 27, 28, 29, 30, 31]
+    cfg = oracle.Cfg(k=16, sinks=4, window=4, beam=1, mode=1)   # L* = 1
+    tree = oracle.select(c, y, t, cfg, tree=tr, G=1)[0][0, 0]
+    # node 0 (buckets 0, 1) wins the tie at level 1; both buckets fit
+    assert tree.tolist() == [0, 1, 2, 3, *range(4, 16), -1, -1, -1, -1, 28, 29, 30, 31]

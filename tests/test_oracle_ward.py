@@ -110,7 +110,7 @@ def _brute_bucket_meta(c, h, b, pool, T, S):
     return mem, keys, lr
 
 
-@pytest.mark.parametrize("T", [4096, 1000, 513, 4])
+@pytest.mark.parametrize("T", [4096, 1000, 777, 524, 513, 4])
 def test_bucket_cache_invariants(T):
     inp = synth.layer_inputs("prefill-4k", seed=3, T=T, parts=("K",))
     cfg = oracle.Cfg(k=512, sinks=4, window=256)
@@ -124,7 +124,10 @@ def test_bucket_cache_invariants(T):
     assert sorted(c["members"][h].tolist()) == list(range(NU))
     for blk in range(nblk):
         n = min(128, NU - 128 * blk)
-        want_m = -(-n * 64 // 128)
+        # a block's bucket count is the least that keeps its mean bucket at
+        # most 8 keys (2 pooled units): 64 for a full block, and for a ragged
+        # last block of n units the least m with n <= 2 m
+        want_m = min(m for m in range(1, 65) if n <= 2 * m)
         sizes = np.diff(c["offsets"][h, 64 * blk:64 * blk + 65])
         assert (sizes[:want_m] >= 1).all() and (sizes[:want_m] <= 4).all()
         assert (sizes[want_m:] == 0).all()
