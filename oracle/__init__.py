@@ -13,7 +13,8 @@ arrays in and out of it.  Each function names the passage it restates:
 * essay "《卡片柜》——当注意力学会先查目录再翻书" (zhichai.net), ch. 2
   (key latent, pool, Ward buckets, centroids), ch. 3 (flat search, sinks,
   window), ch. 4 (binary tree, beam descent), ch. 5 (one W_k/W_q pair per
-  layer; native max over heads);
+  layer; native max over heads), ch. 6 (the natively trained variant's
+  backward over saved key indices);
 * tutorial "隐空间稀疏注意力 (LSA)" (diosapp.com.cn), section 二 (query in the
   same latent space; exact softmax attention over the selected keys);
 * Ward (1963), cited by the essay: least increase of within-cluster SSE.
@@ -75,8 +76,11 @@ def _L():
                                     P, i32, P, i64, i32, i32, i32, i32, i32, i32, i32,
                                     P, P, P]
         lib.lsao_attention.argtypes = [P, P, P, P, i64, i32, i32, i32, i32, P]
+        lib.lsao_attention_backward.argtypes = [P, P, P, P, P, i64, i32, i32, i32, i32, i64,
+                                                P, P, P]
         for f in ("lsao_key_latent_pool", "lsao_query_latent", "lsao_ward_block",
-                  "lsao_build", "lsao_build_tree", "lsao_select", "lsao_attention"):
+                  "lsao_build", "lsao_build_tree", "lsao_select", "lsao_attention",
+                  "lsao_attention_backward"):
             getattr(lib, f).restype = i32
         _lib = lib
     return _lib
@@ -285,6 +289,35 @@ def attention(Q: np.ndarray, K: np.ndarray, V: np.ndarray, idx: np.ndarray) -> n
     rc = _L().lsao_attention(_p(Q), _p(K), _p(V), _p(idx), nq, hq, hkv, d, idx.shape[2], _p(O))
     assert rc == 0
     return O
+
+
+def _f64(x) -> np.ndarray:
+    """bf16 bits (uint16) to fp64; any other array is taken as real values."""
+    x = np.asarray(x)
+    return bf16_to_f64(x) if x.dtype == np.uint16 else _c(x, np.float64)
+
+
+def attention_backward(Q, K, V, idx: np.ndarray, dO):
+    """Gradients (dQ, dK, dV) of the exact sparse attention over saved index
+    lists, in fp64 (tutorial section 二 for the attention; essay ch. 6: the
+    natively trained variant keeps each query's selected key indices for its
+    backward pass).  The discrete selection carries no gradient.
+
+    Q, dO [nq, hq, d]; K, V [T, hkv, d]; each as bf16 bits or real values.
+    idx [nq, hkv, n] as for ``attention``.  Returns dQ [nq, hq, d] and
+    dK, dV [T, hkv, d], fp64."""
+    Qf, Kf, Vf, gf = _f64(Q), _f64(K), _f64(V), _f64(dO)
+    idx = _c(idx, np.int32)
+    nq, hq, d = Qf.shape
+    T, hkv, _ = Kf.shape
+    assert gf.shape == Qf.shape and Vf.shape == Kf.shape and idx.shape[:2] == (nq, hkv)
+    dQ = np.empty_like(Qf)
+    dK = np.empty_like(Kf)
+    dV = np.empty_like(Vf)
+    rc = _L().lsao_attention_backward(_p(Qf), _p(Kf), _p(Vf), _p(gf), _p(idx), nq, hq, hkv, d,
+                                      idx.shape[2], T, _p(dQ), _p(dK), _p(dV))
+    assert rc == 0
+    return dQ, dK, dV
 
 
 # ------------------------------------------------------------ whole layer

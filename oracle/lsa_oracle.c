@@ -21,6 +21,9 @@
  *         its keys, beam descent, O(log T) comparisons.
  *   [CC5] same essay, ch. 5 "两种生产方式": one W_k / W_q pair per layer;
  *         native variant scores a bucket by the max over heads.
+ *   [CC6] same essay, ch. 6 "数字不说谎": natively trained LSA (N-LSA) runs
+ *         forward + backward per layer; its backward keeps every query's
+ *         selected key indices.
  *   [DA2] tutorial "隐空间稀疏注意力 (LSA)" (diosapp.com.cn), section 二
  *         "LSA 怎么工作": the query is projected into the same latent space;
  *         exact softmax attention over the gathered keys, scale 1/sqrt(d).
@@ -743,5 +746,89 @@ int lsao_attention(const uint16_t* Q, const uint16_t* K, const uint16_t* V,
         }
     }
     free(lg);
+    return 0;
+}
+
+/* ------------------------------------------ attention backward [DA2][CC6] */
+
+/*
+ * Gradient of the exact sparse attention above with respect to Q, K and V,
+ * for saved index lists [CC6].  The selection is a discrete choice and
+ * carries no gradient.  For one (query, head) with valid entries i of its list,
+ * s_i = sc q.k_i (sc = 1/sqrt(d)), p = softmax(s), O = sum_i p_i v_i and the
+ * output gradient g = dO:
+ *   dV[k_i] += p_i g
+ *   dp_i     = g . v_i,   D = g . O
+ *   ds_i     = p_i (dp_i - D)
+ *   dQ       = sc sum_i ds_i k_i
+ *   dK[k_i] += sc ds_i q
+ * Q, dO [nq, hq, d], K, V [T, hkv, d] as fp64; idx [nq, hkv, n_idx] (entries
+ * < 0 are padding; every valid entry < T).  dQ [nq, hq, d], dK, dV
+ * [T, hkv, d] are overwritten.  Order: queries ascending, heads ascending,
+ * list entries in list order; every sum from +0.0 in ascending index order.
+ */
+int lsao_attention_backward(const double* Q, const double* K, const double* V,
+                            const double* dO, const int32_t* idx, int64_t nq,
+                            int32_t hq, int32_t hkv, int32_t d, int32_t n_idx,
+                            int64_t T, double* dQ, double* dK, double* dV)
+{
+    if (hkv <= 0 || hq % hkv != 0 || d <= 0 || n_idx < 0 || nq < 0 || T < 0) return -1;
+    int32_t G = hq / hkv;
+    for (int64_t i = 0; i < T * hkv * d; ++i) { dK[i] = 0.0; dV[i] = 0.0; }
+    double* p = (double*)malloc(sizeof(double) * (n_idx > 0 ? n_idx : 1));
+    double* o = (double*)malloc(sizeof(double) * d);
+    double sc = 1.0 / sqrt((double)d);
+    for (int64_t q = 0; q < nq; ++q) {
+        for (int32_t h = 0; h < hq; ++h) {
+            int32_t g = h / G;
+            const int32_t* list = idx + (q * hkv + g) * (int64_t)n_idx;
+            const double* qv = Q + (q * hq + h) * (int64_t)d;
+            const double* gv = dO + (q * hq + h) * (int64_t)d;
+            double* dq = dQ + (q * hq + h) * (int64_t)d;
+            for (int32_t e = 0; e < d; ++e) dq[e] = 0.0;
+            /* forward again: probabilities and output */
+            double mx = -INFINITY;
+            for (int32_t i = 0; i < n_idx; ++i) {
+                if (list[i] < 0) continue;
+                if (list[i] >= T) { free(p); free(o); return -1; }
+                const double* kv = K + ((int64_t)list[i] * hkv + g) * d;
+                double s = 0.0;
+                for (int32_t e = 0; e < d; ++e) s = s + qv[e] * kv[e];
+                p[i] = s * sc;
+                if (p[i] > mx) mx = p[i];
+            }
+            double den = 0.0;
+            for (int32_t i = 0; i < n_idx; ++i) {
+                if (list[i] < 0) continue;
+                p[i] = exp(p[i] - mx);
+                den = den + p[i];
+            }
+            if (!(den > 0.0)) continue;             /* empty list: no gradient */
+            for (int32_t e = 0; e < d; ++e) o[e] = 0.0;
+            for (int32_t i = 0; i < n_idx; ++i) {
+                if (list[i] < 0) continue;
+                p[i] = p[i] / den;
+                const double* vv = V + ((int64_t)list[i] * hkv + g) * d;
+                for (int32_t e = 0; e < d; ++e) o[e] = o[e] + p[i] * vv[e];
+            }
+            double D = 0.0;
+            for (int32_t e = 0; e < d; ++e) D = D + gv[e] * o[e];
+            /* backward */
+            for (int32_t i = 0; i < n_idx; ++i) {
+                if (list[i] < 0) continue;
+                int64_t r = ((int64_t)list[i] * hkv + g) * d;
+                double dp = 0.0;
+                for (int32_t e = 0; e < d; ++e) dp = dp + gv[e] * V[r + e];
+                double ds = p[i] * (dp - D);
+                for (int32_t e = 0; e < d; ++e) {
+                    dV[r + e] = dV[r + e] + p[i] * gv[e];
+                    dq[e] = dq[e] + ds * K[r + e];
+                    dK[r + e] = dK[r + e] + (sc * ds) * qv[e];
+                }
+            }
+            for (int32_t e = 0; e < d; ++e) dq[e] = sc * dq[e];
+        }
+    }
+    free(p); free(o);
     return 0;
 }

@@ -24,6 +24,7 @@ NUM = "test_oracle_numerics.py"
 WARD = "test_oracle_ward.py"
 SEL = "test_oracle_select_attn.py"
 PCA = "test_oracle_pca.py"
+BWD = "test_oracle_backward.py"
 
 # (name, file, original text, mutated text, pin file that must fail)
 MUTANTS = [
@@ -111,7 +112,9 @@ MUTANTS = [
      "if (p >= S && p <= lim && rem > 1) { out[o++] = (int32_t)p; --rem; }"
      " else if (p >= S && p <= lim) { out[o++] = (int32_t)(lim); --rem; }", SEL),
     # attention (tutorial section 二)
-    ("attention_scale_1_over_d", C, "double sc = 1.0 / sqrt((double)d);", "double sc = 1.0 / (double)d;", SEL),
+    ("attention_scale_1_over_d", C,
+     "double* lg = (double*)malloc(sizeof(double) * (n_idx > 0 ? n_idx : 1));\n    double sc = 1.0 / sqrt((double)d);",
+     "double* lg = (double*)malloc(sizeof(double) * (n_idx > 0 ? n_idx : 1));\n    double sc = 1.0 / (double)d;", SEL),
     ("attention_list_of_wrong_group", C,
      "const int32_t* list = idx + (q * hkv + h / G) * (int64_t)n_idx;",
      "const int32_t* list = idx + (q * hkv + h % hkv) * (int64_t)n_idx;", SEL),
@@ -123,6 +126,21 @@ MUTANTS = [
     ("attention_values_from_keys", C,
      "const uint16_t* vv = V + ((int64_t)list[i] * hkv + h / G) * d;",
      "const uint16_t* vv = K + ((int64_t)list[i] * hkv + h / G) * d;", SEL),
+    # sparse-attention backward
+    ("backward_scale_1_over_d", C,
+     "double* o = (double*)malloc(sizeof(double) * d);\n    double sc = 1.0 / sqrt((double)d);",
+     "double* o = (double*)malloc(sizeof(double) * d);\n    double sc = 1.0 / (double)d;", BWD),
+    ("backward_drops_D", C, "double ds = p[i] * (dp - D);", "double ds = p[i] * dp;", BWD),
+    ("backward_dK_unscaled", C, "dK[r + e] = dK[r + e] + (sc * ds) * qv[e];",
+     "dK[r + e] = dK[r + e] + ds * qv[e];", BWD),
+    ("backward_dQ_unscaled", C, "for (int32_t e = 0; e < d; ++e) dq[e] = sc * dq[e];",
+     "for (int32_t e = 0; e < d; ++e) dq[e] = dq[e];", BWD),
+    ("backward_dQ_from_values", C, "dq[e] = dq[e] + ds * K[r + e];", "dq[e] = dq[e] + ds * V[r + e];", BWD),
+    ("backward_dV_unweighted", C, "dV[r + e] = dV[r + e] + p[i] * gv[e];", "dV[r + e] = dV[r + e] + gv[e];", BWD),
+    ("backward_wrong_group", C, "int32_t g = h / G;\n            const int32_t* list",
+     "int32_t g = h % hkv;\n            const int32_t* list", BWD),
+    ("backward_D_from_gradient_only", C, "for (int32_t e = 0; e < d; ++e) D = D + gv[e] * o[e];",
+     "for (int32_t e = 0; e < d; ++e) D = D + gv[e];", BWD),
     # training-free PCA projection
     ("pca_uncentred", P, "    Xc = X - mean\n", "    Xc = X\n", PCA),
     ("pca_smallest_first", P, 'order = np.argsort(-lam, kind="stable")',
@@ -134,7 +152,7 @@ MUTANTS = [
     ("pca_divides_by_n_minus_1", P, "C = (Xc.T @ Xc) / N", "C = (Xc.T @ Xc) / (N - 1)", PCA),
 ]
 
-PIN_FILES = (NUM, WARD, SEL, PCA)
+PIN_FILES = (NUM, WARD, SEL, PCA, BWD)
 
 
 def _copy(dst):
