@@ -9,8 +9,8 @@ import numpy as np
 import pytest
 
 from clustered_key_indexing_b200 import _lib
-from clustered_key_indexing_b200._lib import (LSA_EINVAL, LSA_EUNSUPPORTED, LSA_OK, lsa_cache,
-                                              lsa_cfg, lsa_tree)
+from clustered_key_indexing_b200._lib import (LSA_EINVAL, LSA_ENOSPACE, LSA_EUNSUPPORTED, LSA_OK,
+                                              lsa_cache, lsa_cfg, lsa_decode, lsa_tree)
 
 
 @pytest.fixture(scope="module")
@@ -82,6 +82,79 @@ def test_compute_calls_reject_bad_arguments_before_any_launch(L):
     assert L.lsa_select(None, 0, 1, 4, None, None, None, ctypes.byref(c), None, None, None, 0, None) == LSA_EINVAL
     assert L.lsa_prefill(None, None, None, 16, 4, 1, None, None, ctypes.byref(c), None, None, None, 0,
                          None, 0, None) == LSA_EINVAL
+
+
+def _fake(addr=0x10000):
+    """A non-NULL, 16-byte aligned device address that no call below reaches
+    (each is refused on the host before any CUDA call)."""
+    return ctypes.c_void_p(addr)
+
+
+def _decode_state(batch=2, hkv=2, hq=8, cap=1024, shared_len=0):
+    d = lsa_decode()
+    d.batch, d.hkv, d.hq, d.cap, d.shared_len = batch, hkv, hq, cap, shared_len
+    d.K = d.V = d.U_blk = _fake().value
+    d.K_shared = d.V_shared = _fake().value if shared_len else None
+    c = d.cache
+    c.hkv, c.cap_units, c.cap_buckets = batch * hkv, cap // 4, cap // 512 * 64
+    for f in ("bucket_of_unit", "members", "offsets", "cnt_lr", "minlr", "maxpos", "sum", "cent", "units"):
+        setattr(c, f, _fake().value)
+    return d
+
+
+def _no_gpu():
+    import torch
+    return not torch.cuda.is_available()
+
+
+@pytest.mark.skipif(not _no_gpu(), reason="passes fake device addresses: runs only where no GPU is present")
+def test_host_buffer_pca_and_decode_calls_reject_bad_arguments(L):
+    c = lsa_cfg()
+    L.lsa_cfg_default(ctypes.byref(c))
+    f = _fake()
+    # training-free projection: NULLs, sizes, d_latent range, K alignment, workspace
+    assert L.lsa_fit_pca(None, 16, 1, 64, f, None, f, 1 << 30, None) == LSA_EINVAL
+    assert L.lsa_fit_pca(f, 0, 1, 64, f, None, f, 1 << 30, None) == LSA_EINVAL
+    assert L.lsa_fit_pca(f, 16, 1, 0, f, None, f, 1 << 30, None) == LSA_EINVAL
+    assert L.lsa_fit_pca(f, 16, 1, 129, f, None, f, 1 << 30, None) == LSA_EINVAL
+    assert L.lsa_fit_pca(_fake(0x10008), 16, 1, 64, f, None, f, 1 << 30, None) == LSA_EINVAL
+    assert L.lsa_fit_pca(f, 16, 1, 64, f, None, f, 0, None) == LSA_ENOSPACE
+    assert L.lsa_fit_pca_workspace_bytes(16, 1) > 0 and L.lsa_fit_pca_workspace_bytes(0, 1) == 0
+    # prefill from host buffers: NULL host / device pointers, T, workspace
+    args = [f] * 8
+    assert L.lsa_prefill_host(None, f, f, f, *args[4:], 4096, 4, 1, f, f, ctypes.byref(c), None, None,
+                              0, f, 1 << 40, None, None, None) == LSA_EINVAL
+    assert L.lsa_prefill_host(*args, 4096, 4, 1, None, f, ctypes.byref(c), None, None,
+                              0, f, 1 << 40, None, None, None) == LSA_EINVAL
+    assert L.lsa_prefill_host(*args, 0, 4, 1, f, f, ctypes.byref(c), None, None,
+                              0, f, 1 << 40, None, None, None) == LSA_EINVAL
+    assert L.lsa_prefill_host(*args, 4096, 4, 1, f, f, ctypes.byref(c), None, None,
+                              0, f, 0, None, None, None) == LSA_ENOSPACE
+    # decode: the state's shape, then the call's own arguments
+    assert L.lsa_decode_step(None, f, f, f, f, f, ctypes.byref(c), f, None, f, 1 << 40, None) == LSA_EINVAL
+    for kw, want in ((dict(batch=0), LSA_EUNSUPPORTED), (dict(hq=6, hkv=4), LSA_EINVAL),
+                     (dict(hq=6, hkv=2), LSA_EUNSUPPORTED), (dict(cap=1000), LSA_EINVAL),
+                     (dict(shared_len=256), LSA_EINVAL)):
+        d = _decode_state(**kw)
+        if "cap" in kw:
+            d.cache.cap_units, d.cache.cap_buckets = 250, 64
+        assert L.lsa_decode_step(ctypes.byref(d), f, f, f, f, f, ctypes.byref(c), f, None, f,
+                                 1 << 40, None) == want, kw
+    d = _decode_state(shared_len=512)
+    d.K_shared = None
+    assert L.lsa_decode_load(ctypes.byref(d), 0, 600, f, ctypes.byref(c), f, 1 << 40, None) == LSA_EINVAL
+    d = _decode_state()
+    d.cache.cent = None
+    assert L.lsa_decode_load(ctypes.byref(d), 0, 600, f, ctypes.byref(c), f, 1 << 40, None) == LSA_EINVAL
+    d = _decode_state(shared_len=512)
+    assert L.lsa_decode_load(ctypes.byref(d), 2, 600, f, ctypes.byref(c), f, 1 << 40, None) == LSA_EINVAL
+    assert L.lsa_decode_load(ctypes.byref(d), 0, 1024, f, ctypes.byref(c), f, 1 << 40, None) == LSA_ENOSPACE
+    assert L.lsa_decode_load(ctypes.byref(d), 0, 300, f, ctypes.byref(c), f, 1 << 40, None) == LSA_EINVAL
+    assert L.lsa_decode_load(ctypes.byref(d), 0, 600, f, ctypes.byref(c), f, 0, None) == LSA_ENOSPACE
+    assert L.lsa_decode_workspace_bytes(ctypes.byref(c), ctypes.byref(d)) > 0
+    d.len[1] = 1024
+    assert L.lsa_decode_step(ctypes.byref(d), f, f, f, f, f, ctypes.byref(c), f, None, f,
+                             1 << 40, None) == LSA_ENOSPACE
 
 
 def test_prefill_chunk_is_whole_waves_of_the_candidate_kernel(L):
