@@ -40,6 +40,9 @@ MUTANTS = [
     ("query_group_strided", C, "latent_of(Q + (t * hq + g * G + i) * (int64_t)d",
      "latent_of(Q + (t * hq + g + i * hkv) * (int64_t)d", NUM),
     ("query_mean_not_divided", C, "lsao_bf16_rne(acc[c] / (double)G)", "lsao_bf16_rne(acc[c])", NUM),
+    ("latent_norm_not_square_rooted", C,
+     "    double nrm = sqrt(n2);\n    for (int32_t c = 0; c < dl; ++c) z[c] = (nrm > 0.0) ? v[c] / nrm : 0.0;",
+     "    double nrm = n2;\n    for (int32_t c = 0; c < dl; ++c) z[c] = (nrm > 0.0) ? v[c] / nrm : 0.0;", NUM),
     # bf16 rounding
     ("bf16_truncates", C, "double r = nearbyint(ldexp(a, -ulp_exp));",
      "double r = floor(ldexp(a, -ulp_exp));", NUM),
@@ -59,6 +62,9 @@ MUTANTS = [
     ("ward_buckets_numbered_descending", C,
      "int32_t rank = 0;\n        for (int32_t a = 0; a < n; ++a) {",
      "int32_t rank = 0;\n        for (int32_t a = n - 1; a >= 0; --a) {", WARD),
+    ("cluster_sum_skips_first_member", C, "    for (int32_t i = 0; i < w->size[a]; ++i) {",
+     "    for (int32_t i = 1; i < w->size[a]; ++i) {", WARD),
+    ("merge_loses_a_member", C, "w->size[a] = na + nb;", "w->size[a] = na + nb - 1;", WARD),
     # bucket cache (essay ch. 2-3)
     ("ragged_block_bucket_count_floored", C,
      "int32_t m = (int32_t)(((int64_t)n * bpb + bu - 1) / bu);",
@@ -80,6 +86,10 @@ MUTANTS = [
      "M[node] = (has_b && M[b] > M[a]) ? M[b] : M[a];", SEL),
     ("tree_stop_level_off_by_one", C, "((int64_t)1 << Lstar) < k && Lstar < 62) ++Lstar;",
      "((int64_t)1 << Lstar) <= k && Lstar < 62) ++Lstar;", SEL),
+    ("tree_leaf_range_one_short", C, "int64_t b0 = bm2[i] << Lstar, b1 = (bm2[i] + 1) << Lstar;",
+     "int64_t b0 = bm2[i] << Lstar, b1 = ((bm2[i] + 1) << Lstar) - 1;", SEL),
+    ("tree_beam_keeps_one_fewer", C, "int32_t keep = nl < beam ? nl : beam;",
+     "int32_t keep = nl < beam ? nl : (beam > 1 ? beam - 1 : 1);", SEL),
     # selection and index assembly (essay ch. 3, 5)
     ("equal_scores_take_higher_id", C, "return (a->id < b->id) ? -1 : (a->id > b->id);",
      "return (a->id > b->id) ? -1 : (a->id < b->id);", SEL),
@@ -102,6 +112,8 @@ MUTANTS = [
      "int64_t lim = t - W + 1;", SEL),
     ("window_one_short", C, "int64_t w0 = t - W + 1 > S ? t - W + 1 : S;",
      "int64_t w0 = t - W + 2 > S ? t - W + 2 : S;", SEL),
+    ("window_excludes_t", C, "for (int64_t p = w0; p <= t; ++p) out[o2++] = (int32_t)p;",
+     "for (int64_t p = w0; p < t; ++p) out[o2++] = (int32_t)p;", SEL),
     ("sinks_exclude_t", C, "for (int32_t i = 0; i < S && i <= t; ++i) out[i] = i;",
      "for (int32_t i = 0; i < S && i < t; ++i) out[i] = i;", SEL),
     ("partial_weight_counts_sinks", C, "if (p >= S && p <= lim) ++w;", "if (p <= lim) ++w;", SEL),
@@ -143,6 +155,7 @@ MUTANTS = [
      "for (int32_t e = 0; e < d; ++e) D = D + gv[e];", BWD),
     # training-free PCA projection
     ("pca_uncentred", P, "    Xc = X - mean\n", "    Xc = X\n", PCA),
+    ("pca_mean_over_wrong_count", P, "mean = X.sum(axis=0) / N", "mean = X.sum(axis=0) / (N + 1)", PCA),
     ("pca_smallest_first", P, 'order = np.argsort(-lam, kind="stable")',
      'order = np.argsort(lam, kind="stable")', PCA),
     ("pca_directions_as_rows", P,

@@ -7,8 +7,8 @@ of 4 query heads; single-key lists (a closed form); the flat fill is a top set
 under independently computed exact scores; structural invariants of each index
 row; rows written out by hand on a hand-built cache (a bucket holding sink
 keys, exact score ties); tree with a beam wider than every level equals flat;
-beam 1 equals a greedy single-path descent written here; comparison counts
-O(T/8) vs O(log T).
+beam 1 equals a greedy single-path descent and beams 2 and 3 a plain beam
+search, both written here; comparison counts O(T/8) vs O(log T).
 """
 import numpy as np
 import pytest
@@ -216,6 +216,43 @@ def test_tree_beam1_is_greedy_descent(built):
         allowed = set(p for b in leaves for p in _weights(cache, 0, b, t, c1))
         assert set(lr.tolist()) <= allowed
         assert len(lr) == min(c1.k, len(allowed))
+
+
+def _beam_leaves(tree, cache, y, t, cfg, beam, lstar):
+    """Beam descent written as a plain search: from the root to level L*,
+    score the eligible children of the kept nodes exactly and keep the best
+    `beam` (score desc, node index asc); return the buckets below them."""
+    ln, lo = tree["level_n"], tree["level_off"]
+    top = len(ln) - 1
+    if tree["minlr"][0, lo[top]] > t - cfg.window:
+        return []
+    kept = [0]
+    for lvl in range(top, lstar, -1):
+        cands = []
+        for node in kept:
+            for ch in (2 * node, 2 * node + 1):
+                if ch < ln[lvl - 1] and tree["minlr"][0, lo[lvl - 1] + ch] <= t - cfg.window:
+                    cands.append((-_score_exact(y, tree["cent"][0, lo[lvl - 1] + ch]), ch))
+        kept = [ch for _, ch in sorted(cands)[:beam]]
+    return sorted(b for n in kept for b in range(n << lstar, min((n + 1) << lstar, cache["NB"])))
+
+
+@pytest.mark.parametrize("beam", [2, 3])
+def test_tree_beam_b_is_a_plain_beam_search(built, beam):
+    inp, cfg, cache = built
+    tr = oracle.build_tree(cache)
+    k = 16 * beam * 2                    # L* = 2: beam * 8 * 2^2 = k
+    cb = oracle.Cfg(k=k, sinks=4, window=256, beam=beam, mode=1)
+    tpos = np.array([700, 1500, 2600, 3333, 4095])
+    Y = oracle.query_latent(inp["Q"][tpos], inp["Wq"], 1, 0)
+    idx, _, _ = oracle.select(cache, Y, tpos, cb, tree=tr, G=4)
+    for qi, t in enumerate(tpos):
+        leaves = _beam_leaves(tr, cache, Y[qi, 0], t, cb, beam, 2)
+        assert len(leaves) == 4 * beam
+        lr = _check_row(idx[qi, 0], t, cb)
+        allowed = set(p for b in leaves for p in _weights(cache, 0, b, t, cb))
+        assert set(lr.tolist()) <= allowed
+        assert len(lr) == min(cb.k, len(allowed))
 
 
 def test_tree_structure_and_log_comparisons(built):
