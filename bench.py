@@ -482,7 +482,7 @@ def run_lsa(args):
             inp = {"Wk": Wk_np, "Wq": Wq_np, "K": bits_of(hK[:, :1]), "V": bits_of(hV[:, :1]),
                    "Q": bits_of(hQ)}
         per_layer, desc, spent = oracle_sample(inp, c, n_blocks=None if T <= 131072 else 64,
-                                               n_queries=256 if T <= 131072 else 64)
+                                               n_queries=2048 if T <= 131072 else 64)
         cpu = {"value": T / per_layer, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": desc,
                "sample_seconds": spent}
 
