@@ -24,6 +24,24 @@ def _stream(stream=None):
     return ctypes.c_void_p(s.cuda_stream)
 
 
+BF16, F32, I32 = torch.bfloat16, torch.float32, torch.int32
+W_SHAPE = (128, 64)  # W_k, W_q: d_head x d_latent
+
+
+def _spec(t, name, dtype, shape=None):
+    """One tensor argument's dtype and, where given, its shape (None entries
+    match any size); the library reads every argument as this dense layout,
+    so a mismatch is refused before any call."""
+    if t is None:
+        return
+    if t.dtype != dtype:
+        raise TypeError(f"{name}: expected {dtype}, got {t.dtype}")
+    if shape is not None and (t.dim() != len(shape) or
+                              any(n is not None and t.shape[i] != n for i, n in enumerate(shape))):
+        want = tuple("*" if n is None else n for n in shape)
+        raise ValueError(f"{name}: expected shape {want}, got {tuple(t.shape)}")
+
+
 def _need_cuda(*ts):
     for t in ts:
         if t is not None and not t.is_cuda:
@@ -128,6 +146,8 @@ def check_device_error():
 
 def build_buckets(K: torch.Tensor, W_k: torch.Tensor, cfg: Config, cache: Cache, stream=None):
     """lsa_build_buckets: key latents, pooling, Ward buckets, centroids."""
+    _spec(K, "K", BF16, (None, None, 128))
+    _spec(W_k, "W_k", F32, W_SHAPE)
     _need_cuda(K, W_k)
     T, hkv, _ = K.shape
     check(lib().lsa_build_buckets(_ptr(K), T, hkv, _ptr(W_k), ctypes.byref(cfg.c()),
@@ -145,6 +165,8 @@ def build_tree(cache: Cache, cfg: Config, tree: Tree | None = None, stream=None)
 
 def query_latent(Q: torch.Tensor, W_q: torch.Tensor, hkv: int, cfg: Config, stream=None):
     """lsa_query_latent: bf16 latents [nq, hkv, 64] (mean) or [nq, hq, 64] (native)."""
+    _spec(Q, "Q", BF16, (None, None, 128))
+    _spec(W_q, "W_q", F32, W_SHAPE)
     _need_cuda(Q, W_q)
     nq, hq, _ = Q.shape
     Y = torch.empty((nq, hkv if cfg.agg == 0 else hq, cfg.d_latent), dtype=torch.bfloat16, device=Q.device)
@@ -161,8 +183,13 @@ def select(Q: torch.Tensor, t0: int, W_q: torch.Tensor, cache: Cache, cfg: Confi
            tree: Tree | None = None, idx: torch.Tensor | None = None, Y_out: torch.Tensor | None = None,
            ws: torch.Tensor | None = None, stream=None) -> torch.Tensor:
     """lsa_select: index lists [nq, hkv, S + k + W] for positions t0 .. t0+nq-1."""
-    _need_cuda(Q, W_q)
+    _spec(Q, "Q", BF16, (None, None, 128))
+    _spec(W_q, "W_q", F32, W_SHAPE)
     nq, hq, _ = Q.shape
+    _spec(idx, "idx", I32, (nq, cache.hkv, cfg.row))
+    _spec(Y_out, "Y_out", BF16, (nq, cache.hkv if cfg.agg == 0 else hq, 64))
+    _spec(ws, "ws", torch.uint8, (None,))
+    _need_cuda(Q, W_q, idx, Y_out, ws)
     if idx is None:
         idx = torch.empty((nq, cache.hkv, cfg.row), dtype=torch.int32, device=Q.device)
     need = select_workspace_bytes(cfg, nq, hq, cache)
@@ -176,9 +203,14 @@ def select(Q: torch.Tensor, t0: int, W_q: torch.Tensor, cache: Cache, cfg: Confi
 
 def sparse_attn(Q, K, V, idx, T: int | None = None, O=None, stream=None) -> torch.Tensor:
     """lsa_sparse_attn: exact softmax attention over index lists."""
-    _need_cuda(Q, K, V, idx)
+    _spec(Q, "Q", BF16, (None, None, 128))
+    _spec(K, "K", BF16, (None, None, 128))
+    _spec(V, "V", BF16, tuple(K.shape))
     nq, hq, d = Q.shape
     hkv = K.shape[1]
+    _spec(idx, "idx", I32, (nq, hkv, None))
+    _spec(O, "O", BF16, (nq, hq, 128))
+    _need_cuda(Q, K, V, idx, O)
     if O is None:
         O = torch.empty((nq, hq, d), dtype=torch.bfloat16, device=Q.device)
     T = K.shape[0] if T is None else T
@@ -194,9 +226,15 @@ def select_attn_workspace_bytes(nq: int, hq: int) -> int:
 def select_attn(Q, K, V, idx, t0: int, cfg: Config, T: int | None = None, O=None, ws=None,
                 stream=None) -> torch.Tensor:
     """lsa_select_attn: attention over lsa_select's index rows (window as a band)."""
-    _need_cuda(Q, K, V, idx)
+    _spec(Q, "Q", BF16, (None, None, 128))
+    _spec(K, "K", BF16, (None, None, 128))
+    _spec(V, "V", BF16, tuple(K.shape))
     nq, hq, d = Q.shape
     hkv = K.shape[1]
+    _spec(idx, "idx", I32, (nq, hkv, cfg.row))
+    _spec(O, "O", BF16, (nq, hq, 128))
+    _spec(ws, "ws", torch.uint8, (None,))
+    _need_cuda(Q, K, V, idx, O, ws)
     if O is None:
         O = torch.empty((nq, hq, d), dtype=torch.bfloat16, device=Q.device)
     T = K.shape[0] if T is None else T
@@ -213,6 +251,7 @@ def fit_pca(K: torch.Tensor, d_latent: int = 64, stream=None):
     """lsa_fit_pca: the training-free projection, the leading d_latent
     principal directions of the keys K [T, hkv, 128] (all heads).  Returns
     (W fp32 [128, d_latent], eigenvalues fp64 [128], descending)."""
+    _spec(K, "K", BF16, (None, None, 128))
     _need_cuda(K)
     T, hkv = int(K.shape[0]), int(K.shape[1])
     W = torch.empty((128, d_latent), dtype=torch.float32, device=K.device)
@@ -235,8 +274,14 @@ def prefill_workspace_bytes(cfg: Config, T: int, hq: int, hkv: int, chunk: int) 
 def prefill(Q, K, V, W_k, W_q, cfg: Config, cache: Cache | None = None, tree: Tree | None = None,
             O=None, chunk: int = 16384, ws=None, stream=None) -> torch.Tensor:
     """lsa_prefill: a whole LSA attention layer over a T-token prompt."""
-    _need_cuda(Q, K, V, W_k, W_q)
+    _spec(Q, "Q", BF16, (None, None, 128))
     T, hq, d = Q.shape
+    _spec(K, "K", BF16, (T, None, 128))
+    _spec(V, "V", BF16, tuple(K.shape))
+    _spec(W_k, "W_k", F32, W_SHAPE)
+    _spec(W_q, "W_q", F32, W_SHAPE)
+    _spec(O, "O", BF16, (T, hq, 128))
+    _need_cuda(Q, K, V, W_k, W_q, O)
     hkv = K.shape[1]
     cache = cache or Cache(hkv, T, cfg, device=Q.device)
     if cfg.mode == 1 and tree is None:
@@ -260,11 +305,21 @@ def prefill_host(hQ, hK, hV, W_k, W_q, cfg: Config, hO=None, dev_bufs=None, cach
     host O, uploads and downloads overlapped with the compute.  dev_bufs:
     optional (Q, K, V, O) device buffers; streams: the compute stream (default
     current) and two copy streams (default: new ones)."""
-    _need_cuda(W_k, W_q)
-    for t in (hQ, hK, hV):
-        if t.is_cuda or not t.is_pinned():
-            raise ValueError("lsa_prefill_host takes pinned host tensors")
+    _spec(hQ, "hQ", BF16, (None, None, 128))
     T, hq, d = hQ.shape
+    _spec(hK, "hK", BF16, (T, None, 128))
+    _spec(hV, "hV", BF16, tuple(hK.shape))
+    _spec(hO, "hO", BF16, tuple(hQ.shape))
+    _spec(W_k, "W_k", F32, W_SHAPE)
+    _spec(W_q, "W_q", F32, W_SHAPE)
+    if dev_bufs is not None:
+        for name, t, like in zip(("Q", "K", "V", "O"), dev_bufs, (hQ, hK, hV, hQ)):
+            _spec(t, name, BF16, tuple(like.shape))
+        _need_cuda(*dev_bufs)
+    _need_cuda(W_k, W_q)
+    for t in (hQ, hK, hV) + ((hO,) if hO is not None else ()):
+        if t.is_cuda or not t.is_pinned() or not t.is_contiguous():
+            raise ValueError("lsa_prefill_host takes contiguous pinned host tensors")
     hkv = hK.shape[1]
     dev = W_k.device
     if hO is None:
@@ -314,6 +369,8 @@ class Decode:
         d.batch, d.hkv, d.hq, d.cap = batch, hkv, hq, cap
         d.K, d.V, d.U_blk = self.K.data_ptr(), self.V.data_ptr(), self.U_blk.data_ptr()
         if shared is not None:
+            _spec(shared[0], "K_shared", BF16, (None, hkv, 128))
+            _spec(shared[1], "V_shared", BF16, tuple(shared[0].shape))
             _need_cuda(*shared)
             d.K_shared, d.V_shared, d.shared_len = shared[0].data_ptr(), shared[1].data_ptr(), sl
         d.cache = self.cache.c
@@ -332,6 +389,11 @@ class Decode:
     def load(self, r: int, K: torch.Tensor, V: torch.Tensor, W_k: torch.Tensor, stream=None):
         """Install a prompt as request r: K/V [n, hkv, 128], or with a shared
         prefix the prompt's tokens after it (the prompt holds shared_len + n)."""
+        hkv = self.K.shape[2]
+        _spec(K, "K", BF16, (None, hkv, 128))
+        _spec(V, "V", BF16, tuple(K.shape))
+        _spec(W_k, "W_k", F32, W_SHAPE)
+        _need_cuda(W_k)
         n = K.shape[0]
         self.K[r, :n].copy_(K)
         self.V[r, :n].copy_(V)
@@ -341,7 +403,15 @@ class Decode:
 
     def step(self, q, k, v, W_k, W_q, o=None, idx_out=None, stream=None):
         """One token per request: q [batch, hq, 128], k/v [batch, hkv, 128]."""
-        _need_cuda(q, k, v, W_k, W_q)
+        b, hkv, hq = int(self.d.batch), int(self.d.hkv), int(self.d.hq)
+        _spec(q, "q", BF16, (b, hq, 128))
+        _spec(k, "k", BF16, (b, hkv, 128))
+        _spec(v, "v", BF16, (b, hkv, 128))
+        _spec(W_k, "W_k", F32, W_SHAPE)
+        _spec(W_q, "W_q", F32, W_SHAPE)
+        _spec(o, "o", BF16, (b, hq, 128))
+        _spec(idx_out, "idx_out", I32, (b, hkv, self.cfg.row))
+        _need_cuda(q, k, v, W_k, W_q, o, idx_out)
         if o is None:
             o = torch.empty_like(q)
         check(lib().lsa_decode_step(ctypes.byref(self.d), _ptr(q), _ptr(k), _ptr(v), _ptr(W_k), _ptr(W_q),

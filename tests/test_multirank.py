@@ -50,7 +50,7 @@ def _rank(rank, world, port, out):
 def test_two_rank_timing_and_sharding():
     world = 2
     port = _free_port()
-    with mp.Manager() as mgr:
+    with mp.get_context("spawn").Manager() as mgr:
         out = mgr.dict()
         mp.start_processes(_rank, args=(world, port, out), nprocs=world, join=True, start_method="spawn")
         res = dict(out)
