@@ -162,9 +162,12 @@ def peaks():
 
 # ------------------------------------------------------------ CPU oracle
 
-def oracle_sample(inp, c, n_blocks=None, n_queries=32, seed=0):
+def oracle_sample(inp, c, n_blocks=None, n_queries=32, seed=0, full=None):
     """Time the oracle on one kv-head: the build of `n_blocks` cluster blocks
     (all if None) and select + attention for `n_queries` stratified positions.
+    `full`: an optional dict that keeps the whole head's cache (the query
+    sample needs it) between calls on the same inputs; that build is not
+    part of the timed sample.
     Returns (seconds per layer extrapolated to T x hkv, description)."""
     import oracle
     T, hkv = c["T"], c["hkv"]
@@ -179,9 +182,14 @@ def oracle_sample(inp, c, n_blocks=None, n_queries=32, seed=0):
     tree = oracle.build_tree(cache) if c["mode"] == 1 else None
     t_build = time.perf_counter() - t0
     if Tb < T:  # the query sample needs the whole head's cache
-        U = oracle.key_latent_pool(K1, inp["Wk"], 4)
-        cache = oracle.build_cache(U, T, ocfg)
-        tree = oracle.build_tree(cache) if c["mode"] == 1 else None
+        if full is not None and "cache" in full:
+            cache, tree = full["cache"], full["tree"]
+        else:
+            U = oracle.key_latent_pool(K1, inp["Wk"], 4)
+            cache = oracle.build_cache(U, T, ocfg)
+            tree = oracle.build_tree(cache) if c["mode"] == 1 else None
+            if full is not None:
+                full["cache"], full["tree"] = cache, tree
     rng = np.random.default_rng(seed)
     lo = c["window"] + c["sinks"]
     tpos = np.sort(rng.choice(np.arange(lo, T), size=n_queries, replace=False))
@@ -251,8 +259,9 @@ def run_reference(args):
     inp = synth.layer_inputs(args.workload, seed=0, T=c["T"], parts=("Q", "K", "V"))
     vals = []
     desc = ""
+    full = {}
     for i in range(args.warmup + args.steps):
-        per_layer, desc, _ = oracle_sample(inp, c, n_blocks=8, n_queries=4, seed=i)
+        per_layer, desc, _ = oracle_sample(inp, c, n_blocks=8, n_queries=16, seed=i, full=full)
         if i >= args.warmup:
             vals.append(c["T"] / per_layer)
     v = statistics.median(vals)
