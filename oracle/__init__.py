@@ -62,6 +62,11 @@ def _L():
         lib.lsao_bf16_rne.restype = ctypes.c_uint16
         lib.lsao_bf16_rne.argtypes = [ctypes.c_double]
         lib.lsao_bf16_rne_array.argtypes = [P, i64, P]
+        lib.lsao_e4m3_rne.restype = ctypes.c_uint8
+        lib.lsao_e4m3_rne.argtypes = [ctypes.c_double]
+        lib.lsao_e4m3_to_double.restype = ctypes.c_double
+        lib.lsao_e4m3_to_double.argtypes = [ctypes.c_uint8]
+        lib.lsao_cent_fp8.argtypes = [P, i64, i32, P]
         lib.lsao_key_latent_pool.argtypes = [P, i64, i32, i32, P, i32, i32, P]
         lib.lsao_query_latent.argtypes = [P, i64, i32, i32, i32, P, i32, i32, P]
         lib.lsao_ward_delta.restype = ctypes.c_double
@@ -141,6 +146,49 @@ def bf16_rne(x) -> np.ndarray:
     out = np.empty(x.shape, np.uint16)
     _L().lsao_bf16_rne_array(_p(x), x.size, _p(out))
     return out
+
+
+# -------------------------------------------------- fp8 centroids (ch. 8)
+
+FP8_SCALE_EXP = 8   # a component c is stored as the e4m3 code of 2^8 * c
+
+
+def e4m3_rne(x) -> np.ndarray:
+    """fp64 values straight to OCP e4m3 codes (uint8), ties to even,
+    saturating at +-448."""
+    x = _c(np.atleast_1d(x), np.float64)
+    L = _L()
+    return np.array([L.lsao_e4m3_rne(float(v)) for v in x.ravel()], np.uint8).reshape(x.shape)
+
+
+def e4m3_to_f64(codes) -> np.ndarray:
+    c = np.atleast_1d(np.asarray(codes, np.uint8))
+    L = _L()
+    return np.array([L.lsao_e4m3_to_double(int(v)) for v in c.ravel()], np.float64).reshape(c.shape)
+
+
+def cent_fp8(cache: dict) -> np.ndarray:
+    """FP8 centroid cache (essay ch. 8: the bucket cache stacks with FP8
+    quantisation): per bucket, the e4m3 code of 2^8 * s / |s| for its fp64
+    unit sum s, rounded straight from fp64.  Returns uint8 [H, NB, dl]."""
+    s = _c(cache["sum"], np.float64)
+    H, NB, dl = s.shape
+    out = np.empty((H, NB, dl), np.uint8)
+    _L().lsao_cent_fp8(_p(s), H * NB, dl, _p(out))
+    return out
+
+
+def fp8_as_bf16(codes: np.ndarray) -> np.ndarray:
+    """The values 2^-8 * e4m3(code) as bf16 bits (exact: 4 significant bits
+    and exponents in bf16's range), so that the bf16 selection scores the FP8
+    centroids exactly."""
+    return bf16_rne(np.ldexp(e4m3_to_f64(codes), -FP8_SCALE_EXP)).reshape(np.shape(codes))
+
+
+def with_fp8_centroids(cache: dict) -> dict:
+    """The cache with its centroids replaced by the FP8 ones (as exact bf16
+    values): selecting on it scores every bucket against its FP8 centroid."""
+    return dict(cache, cent=fp8_as_bf16(cent_fp8(cache)))
 
 
 # ----------------------------------------------------------- latents (ch. 2)

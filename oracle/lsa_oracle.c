@@ -27,6 +27,8 @@
  *   [DA2] tutorial "隐空间稀疏注意力 (LSA)" (diosapp.com.cn), section 二
  *         "LSA 怎么工作": the query is projected into the same latent space;
  *         exact softmax attention over the gathered keys, scale 1/sqrt(d).
+ *   [CC8] same essay, ch. 8 "亚平方版图上的新坐标": the bucket cache is
+ *         compatible with FP8 / INT4 quantisation.
  *   [W63] Ward, "Hierarchical Grouping to Optimize an Objective Function",
  *         JASA 1963 (cited in the essay's references): merge the pair whose
  *         union increases the within-cluster sum of squares least.
@@ -83,6 +85,67 @@ uint16_t lsao_bf16_rne(double x)
 void lsao_bf16_rne_array(const double* x, int64_t n, uint16_t* out)
 {
     for (int64_t i = 0; i < n; ++i) out[i] = lsao_bf16_rne(x[i]);
+}
+
+/* ----------------------------------------------------- fp8 e4m3 [CC8] */
+
+/*
+ * FP8 (e4m3) centroid cache [CC8]: the essay's closing chapter names FP8 and
+ * INT4 quantisation of the bucket cache as compatible with the method.
+ * Reading: a centroid component c (|c| <= 1) is stored as the e4m3 code of
+ * 2^8 * c, rounded to nearest, ties to even, from the fp64 normalised value
+ * (no intermediate bf16); |2^8 c| <= 256 < 448, so no code saturates; its
+ * value is the code's value times 2^-8.  e4m3 (OCP FP8 E4M3, "fn"): 1 sign,
+ * 4 exponent bits (bias 7), 3 mantissa bits, no infinities, largest finite
+ * 448, smallest subnormal 2^-9; exponent field 0 holds the subnormals m 2^-9.
+ * Every such value times 2^-8 is a bf16 number, so a bf16 array can carry it
+ * exactly.
+ */
+double lsao_e4m3_to_double(uint8_t code)
+{
+    int s = code >> 7, e = (code >> 3) & 15, m = code & 7;
+    double v;
+    if (e == 15 && m == 7) return NAN;
+    if (e == 0) v = ldexp((double)m, -9);
+    else v = ldexp(1.0 + m / 8.0, e - 7);
+    return s ? -v : v;
+}
+
+/* Round a double straight to e4m3, ties to even, saturating at +-448. */
+uint8_t lsao_e4m3_rne(double x)
+{
+    if (isnan(x)) return 0x7F;
+    uint8_t sign = signbit(x) ? 0x80 : 0;
+    double a = fabs(x);
+    if (a == 0.0) return sign;
+    int e;
+    frexp(a, &e);                 /* a in [2^(e-1), 2^e) */
+    int ulp_exp = e - 4;          /* spacing of 4-significant-bit numbers */
+    if (e - 1 < -6) ulp_exp = -9; /* subnormal spacing 2^-9 */
+    double r = nearbyint(ldexp(a, -ulp_exp)) ; /* exact scale, RNE */
+    double y = ldexp(r, ulp_exp);
+    if (y > 448.0) y = 448.0;
+    /* encode y (exactly representable now) */
+    int ye;
+    if (y < ldexp(1.0, -6)) return (uint8_t)(sign | (uint8_t)ldexp(y, 9)); /* subnormal or zero */
+    frexp(y, &ye);                /* y in [2^(ye-1), 2^ye) */
+    int E = ye - 1 + 7;
+    int M = (int)ldexp(y, -(ye - 1) + 3) - 8;
+    return (uint8_t)(sign | (uint8_t)(E << 3) | (uint8_t)M);
+}
+
+/* FP8 centroids of n fp64 bucket sums [n, dl]: code of 2^8 * s / |s| per
+ * component (0 for an empty sum). */
+void lsao_cent_fp8(const double* sum, int64_t n, int32_t dl, uint8_t* out)
+{
+    for (int64_t b = 0; b < n; ++b) {
+        const double* s = sum + b * dl;
+        double n2 = 0.0;
+        for (int32_t c = 0; c < dl; ++c) n2 = n2 + s[c] * s[c];
+        double nrm = sqrt(n2);
+        for (int32_t c = 0; c < dl; ++c)
+            out[b * dl + c] = lsao_e4m3_rne(nrm > 0.0 ? ldexp(s[c] / nrm, 8) : 0.0);
+    }
 }
 
 /* ------------------------------------------------------- latent [CC2][DA2] */

@@ -25,6 +25,7 @@ WARD = "test_oracle_ward.py"
 SEL = "test_oracle_select_attn.py"
 PCA = "test_oracle_pca.py"
 BWD = "test_oracle_backward.py"
+FP8 = "test_oracle_fp8.py"
 
 # (name, file, original text, mutated text, pin file that must fail)
 MUTANTS = [
@@ -163,9 +164,20 @@ MUTANTS = [
      "return np.ascontiguousarray(V.T[:, :d_latent], dtype=np.float32), lam, V", PCA),
     ("pca_sign_flipped", P, "        if V[i, j] < 0:\n", "        if V[i, j] > 0:\n", PCA),
     ("pca_divides_by_n_minus_1", P, "C = (Xc.T @ Xc) / N", "C = (Xc.T @ Xc) / (N - 1)", PCA),
+    # FP8 centroid cache (essay ch. 8)
+    ("e4m3_ties_away_from_zero", C, "double r = nearbyint(ldexp(a, -ulp_exp)) ;",
+     "double r = round(ldexp(a, -ulp_exp)) ;", FP8),
+    ("e4m3_exponent_bias_8", C, "int E = ye - 1 + 7;", "int E = ye - 1 + 8;", FP8),
+    ("e4m3_subnormal_range_one_short", C, "if (e - 1 < -6) ulp_exp = -9;", "if (e - 1 < -7) ulp_exp = -9;", FP8),
+    ("e4m3_no_saturation", C, "if (y > 448.0) y = 448.0;", "if (y > 480.0) y = 480.0;", FP8),
+    ("fp8_scale_2_7", C, "ldexp(s[c] / nrm, 8)", "ldexp(s[c] / nrm, 7)", FP8),
+    ("fp8_centroid_not_normalised", C, "lsao_e4m3_rne(nrm > 0.0 ? ldexp(s[c] / nrm, 8) : 0.0)",
+     "lsao_e4m3_rne(nrm > 0.0 ? ldexp(s[c], 8) : 0.0)", FP8),
+    ("fp8_decoded_without_scale", P, "bf16_rne(np.ldexp(e4m3_to_f64(codes), -FP8_SCALE_EXP))",
+     "bf16_rne(e4m3_to_f64(codes))", FP8),
 ]
 
-PIN_FILES = (NUM, WARD, SEL, PCA, BWD)
+PIN_FILES = (NUM, WARD, SEL, PCA, BWD, FP8)
 
 
 def _copy(dst):
