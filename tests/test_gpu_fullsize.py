@@ -9,9 +9,9 @@ samples it can compute one by one:
 * one kv-head's whole bucket cache (and tree), bit-exact: the oracle
   clusters that head's keys alone (Ward per 512-key block, essay "《卡片柜》"
   ch. 2);
-* the index rows of that head for sampled query positions in the first
-  chunk, a middle chunk and the ragged last chunk (first and last row of
-  each chunk included), bit-exact (ch. 3-4);
+* the index rows of that head for 128 sampled query positions in each of
+  the first chunk, a middle chunk and the ragged last chunk (first and last
+  row of each chunk included), bit-exact (ch. 3-4);
 * the attention output of the head's GQA group at those positions, within
   max |err| 2e-2 and mean |err| 2e-3 of the fp64 oracle (tutorial
   "隐空间稀疏注意力" section 二).
@@ -99,7 +99,7 @@ def _assert_head_cache(cache, h, U, oc):
         assert np.array_equal(got, oc["members"][0][off[:-1][m] + i]), i
 
 
-def _run_sampled(lsa, L, cfg, heads, n_per_chunk=6, seed=0):
+def _run_sampled(lsa, L, cfg, heads, n_per_chunk=128, seed=0):
     """Run the benchmark's launch sequence on three chunks and check sampled
     rows of `heads` against the oracle."""
     c = L.c
@@ -181,12 +181,44 @@ def test_prefill_128k_sampled(lsa, layer_128k, agg):
 
 
 def test_prefill_1m_flat_sampled(lsa, layer_1m):
-    """2^20 tokens, flat search (the wave-aligned multi-chunk candidate path)."""
+    """2^20 tokens, flat search (the wave-aligned multi-chunk candidate path),
+    kv-heads 1 and 5."""
     cfg = _cfg(lsa, layer_1m.c)
-    _run_sampled(lsa, layer_1m, cfg, heads=(5,), seed=1)
+    _run_sampled(lsa, layer_1m, cfg, heads=(1, 5), seed=1)
 
 
 def test_prefill_1m_tree_sampled(lsa, layer_1m):
-    """2^20 tokens, tree search with beam 2."""
+    """2^20 tokens, tree search with beam 2, kv-heads 1 and 5."""
     cfg = _cfg(lsa, dict(layer_1m.c, mode=1))
-    _run_sampled(lsa, layer_1m, cfg, heads=(5,), seed=2)
+    _run_sampled(lsa, layer_1m, cfg, heads=(1, 5), seed=2)
+
+
+def test_prefill_128k_exact_fallback(lsa, layer_128k):
+    """The exact fallback at full size.  Two kv-heads of the 128K layer are
+    replaced: kv-head 3's keys are all zero (every centroid is 0, so every
+    eligible bucket ties at score 0 and the candidate list overflows) and
+    kv-head 6's keys are 4 x one of three centres, with no noise (few
+    distinct scores, so wide bands of exactly tied buckets at the cut).  Rows
+    whose ranking the tensor-core scores cannot settle take the exact fp64
+    fallback kernel; their index rows must still equal the oracle's bit for
+    bit, and the fallback must have run."""
+    from clustered_key_indexing_b200._lib import lib
+    base = layer_128k
+    c = base.c
+    L = Layer.__new__(Layer)
+    L.c, L.Q, L.V, L.Wk, L.Wq, L.Wk_np, L.Wq_np = base.c, base.Q, base.V, base.Wk, base.Wq, base.Wk_np, base.Wq_np
+    L._heads = {}
+    K = base.K.clone()
+    K[:, 3] = 0
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(7)
+    mu = torch.from_numpy(synth.centres(0, c["n_centres"], c["d"])[:3]).cuda()
+    ci = torch.randint(0, 3, (c["T"],), generator=gen, device="cuda")
+    K[:, 6] = (4.0 * mu[ci]).to(torch.bfloat16)
+    L.K = K
+    cfg = _cfg(lsa, c)
+    lib().lsa_fallback_rows()  # reset the counter
+    _run_sampled(lsa, L, cfg, heads=(3, 6, 0), n_per_chunk=64, seed=3)
+    assert lib().lsa_fallback_rows() > 0
+    del L, K
+    torch.cuda.empty_cache()
