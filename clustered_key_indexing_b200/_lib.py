@@ -108,6 +108,11 @@ def lib():
         L.lsa_fit_pca_workspace_bytes.argtypes = [i64, i32]
         L.lsa_fit_pca_workspace_bytes.restype = sz
         L.lsa_fit_pca.argtypes = [vp, i64, i32, i32, vp, vp, vp, sz, vp]
+        L.lsa_l2_read_sink_bytes.argtypes = [i32]
+        L.lsa_l2_read_sink_bytes.restype = sz
+        L.lsa_l2_read_bytes.argtypes = [sz, i32]
+        L.lsa_l2_read_bytes.restype = i64
+        L.lsa_l2_read.argtypes = [vp, sz, i32, i32, vp, vp]
         for name in exported_names():
             if getattr(L, name).restype is ctypes.c_int:
                 getattr(L, name).restype = i32

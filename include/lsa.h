@@ -226,6 +226,24 @@ void lsa_timing_begin(void);
 void lsa_timing_end(void);
 lsa_status lsa_timing_get(const char* name, double* total_ms, int64_t* launches);
 
+/*
+ * L2-to-SM read bandwidth (measurement; no counterpart on the pages).  The
+ * gathered attention re-reads K/V rows that stay in L2, so its bound is the
+ * rate at which the SMs can read from L2, which this kernel measures:
+ * lsa_l2_read streams the device buffer `buf` (16-byte aligned, at least
+ * 128 KiB; choose it well under the L2 size so it stays resident) `passes`
+ * times with 16-byte loads that bypass L1, from `ctas` CTAs of 512 threads,
+ * and writes one word per thread to `sink` (device, at least
+ * lsa_l2_read_sink_bytes(ctas) bytes).  lsa_l2_read_bytes() gives the bytes
+ * one launch reads (whole 128 KiB chunks of the buffer, each once a pass);
+ * the caller times the launch with CUDA events on `stream`.  LSA_EINVAL on
+ * NULL, misaligned or too small buffers or passes/ctas out of range.
+ */
+size_t lsa_l2_read_sink_bytes(int32_t ctas);
+int64_t lsa_l2_read_bytes(size_t bytes, int32_t passes);
+lsa_status lsa_l2_read(const void* buf, size_t bytes, int32_t passes, int32_t ctas, uint32_t* sink,
+                       void* stream);
+
 /* ------------------------------------------------------- (4) attention */
 
 /*

@@ -98,10 +98,14 @@ def _tokens(seed, kind, t0, t1, heads, d, mu, scale):
 
 
 def layer_inputs(name: str = "prefill-4k", seed: int = 0, T: int | None = None,
-                 parts=("Q", "K", "V")) -> dict:
+                 parts=("Q", "K", "V"), hkv: int | None = None) -> dict:
     """Q [T, hq, d], K/V [T, hkv, d] as bf16 bits, W_k/W_q fp32 [d, dl].
-    `T` overrides the configuration's length (a prefix of the same stream)."""
+    `T` overrides the configuration's length (a prefix of the same stream);
+    `hkv` draws that many kv-heads (and their hkv * hq / hkv query heads) of
+    the same recipe instead (another stream than the full layer's)."""
     c = CONFIGS[name]
+    if hkv is not None:
+        c = dict(c, hkv=hkv, hq=hkv * (c["hq"] // c["hkv"]))
     T = c["T"] if T is None else T
     mu = centres(seed, c["n_centres"], c["d"])
     Wk, Wq = projections(seed, c["d"], c["dl"])
