@@ -108,6 +108,7 @@ def lib():
         L.lsa_fit_pca_workspace_bytes.argtypes = [i64, i32]
         L.lsa_fit_pca_workspace_bytes.restype = sz
         L.lsa_fit_pca.argtypes = [vp, i64, i32, i32, vp, vp, vp, sz, vp]
+        L.lsa_attn_backward.argtypes = [vp, vp, vp, vp, vp, vp, i64, i32, i32, i32, i64, vp, vp, vp, vp]
         for name in exported_names():
             if getattr(L, name).restype is ctypes.c_int:
                 getattr(L, name).restype = i32

@@ -8,3 +8,4 @@
 #include "lsa_decode.cu"
 #include "lsa_noalloc.cu"
 #include "lsa_pca.cu"
+#include "lsa_bwd.cu"
