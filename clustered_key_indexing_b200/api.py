@@ -223,9 +223,17 @@ def attn_backward(Q, K, V, O, dO, idx, T: int | None = None, dK=None, dV=None, s
     """lsa_attn_backward: gradients of the sparse attention over saved index
     lists.  Returns (dQ [nq, hq, 128], dK, dV [T, hkv, 128]), fp32; dK and dV
     are added to when given (so query chunks accumulate), else zero-started."""
-    _need_cuda(Q, K, V, O, dO, idx)
+    _spec(Q, "Q", BF16, (None, None, 128))
     nq, hq, d = Q.shape
+    _spec(O, "O", BF16, tuple(Q.shape))
+    _spec(dO, "dO", BF16, tuple(Q.shape))
+    _spec(K, "K", BF16, (None, None, 128))
+    _spec(V, "V", BF16, tuple(K.shape))
     hkv = K.shape[1]
+    _spec(idx, "idx", I32, (nq, hkv, None))
+    _spec(dK, "dK", F32, tuple(K.shape))
+    _spec(dV, "dV", F32, tuple(K.shape))
+    _need_cuda(Q, K, V, O, dO, idx, dK, dV)
     T = K.shape[0] if T is None else T
     dQ = torch.empty((nq, hq, d), dtype=torch.float32, device=Q.device)
     if dK is None:

@@ -138,6 +138,15 @@ def test_bad_arguments(lsa):
         lsa.attn_backward(Q, K, K, Q, Q, idx)        # hq / hkv = 3
     assert e.value.status == LSA_EUNSUPPORTED
     Q4 = to_dev_bf16(_bf16(rng, (2, 4, 128)))
-    with pytest.raises(LSAError) as e:
-        lsa.attn_backward(Q4[:, :, 1:], K, K, Q4, Q4, idx)   # misaligned rows
-    assert e.value.status in (LSA_EINVAL, LSA_EUNSUPPORTED)
+    with pytest.raises(ValueError):                            # rows of 127: refused by the binding
+        lsa.attn_backward(Q4[:, :, 1:], K, K, Q4, Q4, idx)
+    with pytest.raises(LSAError) as e:                         # NULL dQ pointer: refused by the library
+        from clustered_key_indexing_b200._lib import lib
+        import ctypes
+        p = ctypes.c_void_p
+        st = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+        from clustered_key_indexing_b200._lib import check
+        check(lib().lsa_attn_backward(p(Q4.data_ptr()), p(K.data_ptr()), p(K.data_ptr()), p(Q4.data_ptr()),
+                                      p(Q4.data_ptr()), p(idx.data_ptr()), 2, 4, 2, 4, 8, None, None, None, st),
+              "lsa_attn_backward")
+    assert e.value.status == LSA_EINVAL
