@@ -88,6 +88,8 @@ def parse():
     p.add_argument("--no-tree", action="store_true", help="skip the tree-search timing on the prefill line")
     p.add_argument("--no-decode", action="store_true", help="skip the decode block on the 1M prefill line")
     p.add_argument("--pca", action="store_true", help="time the training-free projection fit on the workload's keys")
+    p.add_argument("--backward", action="store_true",
+                   help="time the sparse-attention backward over the layer's saved index rows")
     return p.parse_args()
 
 
@@ -876,6 +878,130 @@ def run_pca(args):
         })
 
 
+def oracle_backward_sample(inp, c, n_queries=16, seed=0):
+    """Time the oracle's attention backward on one kv-head: rows of
+    `n_queries` stratified positions from the oracle's own selection, O from
+    the oracle's forward, then oracle.attention_backward over those rows.
+    Returns (seconds per layer extrapolated to T x hkv, description)."""
+    import oracle
+    T, hkv = c["T"], c["hkv"]
+    G = c["hq"] // hkv
+    ocfg = oracle.Cfg(k=c["k"], sinks=c["sinks"], window=c["window"], beam=c["beam"],
+                      mode=c["mode"], agg=c["agg"])
+    K1 = np.ascontiguousarray(inp["K"][:, :1])
+    V1 = np.ascontiguousarray(inp["V"][:, :1])
+    cache = oracle.build_cache(oracle.key_latent_pool(K1, inp["Wk"], 4), T, ocfg)
+    tree = oracle.build_tree(cache) if c["mode"] == 1 else None
+    rng = np.random.default_rng(seed)
+    lo = c["window"] + c["sinks"]
+    tpos = np.sort(rng.choice(np.arange(lo, T), size=n_queries, replace=False))
+    Qs = np.ascontiguousarray(inp["Q"][tpos][:, :G])
+    Y = oracle.query_latent(Qs, inp["Wq"], 1, c["agg"])
+    idx, _, _ = oracle.select(cache, Y, tpos, ocfg, tree=tree, G=G)
+    dO = rng.standard_normal(Qs.shape)
+    t0 = time.perf_counter()
+    oracle.attention_backward(Qs, K1, V1, idx, dO)
+    t_q = (time.perf_counter() - t0) / n_queries
+    desc = (f"1 of {hkv} kv-heads: attention backward over the oracle's own rows at {n_queries} stratified "
+            f"query positions (G={G} heads), extrapolated to T={T} x {hkv} heads")
+    return t_q * T * hkv, desc
+
+
+def run_backward(args):
+    """The sparse-attention backward (lsa_attn_backward) over a prefill
+    layer's saved index rows: one step = dQ, dK, dV of all T queries, with dK
+    and dV zeroed first.  The rows and the forward output O come from the
+    library's own selection and attention before the timed region."""
+    import torch
+
+    import clustered_key_indexing_b200 as lsa
+
+    world, rank, local = dist_setup(args)
+    c = workload_cfg(args)
+    T, hkv, hq = c["T"], c["hkv"], c["hq"]
+    cfg = lsa.Config(k=c["k"], sinks=c["sinks"], window=c["window"], beam=c["beam"],
+                     mode=c["mode"], agg=c["agg"])
+    dev = torch.device("cuda", torch.cuda.current_device())
+    if T > 131072:
+        raise SystemExit("--backward keeps every query's index row: use a workload of at most 131072 tokens")
+    inp = synth.layer_inputs(args.workload, seed=rank, T=T)
+
+    def on_dev(bits):
+        return torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).to(dev)
+
+    Q, K, V = on_dev(inp["Q"]), on_dev(inp["K"]), on_dev(inp["V"])
+    Wk, Wq = torch.from_numpy(inp["Wk"]).to(dev), torch.from_numpy(inp["Wq"]).to(dev)
+    cache = lsa.Cache(hkv, T, cfg, device=dev)
+    tree = lsa.Tree(cache, device=dev) if cfg.mode == 1 else None
+    lsa.build_buckets(K, Wk, cfg, cache)
+    if tree is not None:
+        lsa.build_tree(cache, cfg, tree)
+    idx = torch.empty((T, hkv, cfg.row), dtype=torch.int32, device=dev)
+    chunk = lsa.prefill_chunk(cfg, T, hq, hkv, args.chunk)
+    for t0 in range(0, T, chunk):
+        n = min(chunk, T - t0)
+        lsa.select(Q[t0:t0 + n], t0, Wq, cache, cfg, tree=tree, idx=idx[t0:t0 + n])
+    O = lsa.sparse_attn(Q, K, V, idx)
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(1000 + rank)
+    dO = torch.randn(Q.shape, generator=gen, device=dev, dtype=torch.float32).to(torch.bfloat16)
+    dQ = torch.empty((T, hq, 128), dtype=torch.float32, device=dev)
+    dK = torch.zeros((T, hkv, 128), dtype=torch.float32, device=dev)
+    dV = torch.zeros_like(dK)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        dK.zero_()
+        dV.zero_()
+        lsa.attn_backward(Q, K, V, O, dO, idx, dK=dK, dV=dV)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    lsa.check_device_error()
+    clocks = Clocks(torch.cuda.current_device())
+    kt = lsa.KernelTimer()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with kt:
+        e0.record(stream)
+        for _ in range(args.steps):
+            step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+    clk = clocks.stop()
+    lsa.check_device_error()
+    ms = max_over_ranks(e0.elapsed_time(e1), world, dev) / args.steps
+    bms, bn = kt.get("attn_bwd_kernel")
+    bwd_ms = bms / max(bn, 1)
+    # algorithmic bytes per valid index entry: the K row twice (statistics,
+    # then gradients) and the V row once, 256 B each, plus the fp32 dK and dV
+    # rows added to (2 x 512 B)
+    n_valid = int((idx >= 0).sum())
+    bytes_ = n_valid * (3 * 256 + 2 * 512.0)
+    pk, src = peaks()
+    achieved = bytes_ / (bwd_ms / 1e3) / 1e9
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu:
+        per_layer, desc = oracle_backward_sample(inp, c)
+        cpu = {"value": T / per_layer, "unit": "tokens/s", "cores": 1, "kind": "oracle", "sample": desc}
+    if rank == 0:
+        emit_json({
+            "metric": "LSA attention backward tokens/s", "value": job_rate(world, T, ms), "unit": "tokens/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
+            "config": {"workload": args.workload, "T": T, "hkv": hkv, "hq": hq, "k": c["k"], "sinks": c["sinks"],
+                       "window": c["window"], "index_entries": n_valid,
+                       "l2": "no flush: per-step K/V gathers and dK/dV (fp32) are larger than L2"},
+            "clocks": clk, "gpu_launches": args.steps, "e2e": None,
+            "kernels": {"attn_bwd_kernel": bwd_ms},
+            "roofline": {"kernel": "attn_bwd_kernel", "bound": "hbm", "achieved": achieved,
+                         "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": achieved / pk["hbm_gbs"],
+                         "traffic": None, "peak_source": src, "bytes_per_launch": bytes_},
+            "cpu_baseline": cpu,
+        })
+
+
 def ctypes_ref(x):
     import ctypes
     return ctypes.byref(x)
@@ -892,6 +1018,8 @@ if __name__ == "__main__":
         run_reference(a)
     elif a.pca:
         run_pca(a)
+    elif a.backward:
+        run_backward(a)
     elif a.workload.startswith("decode"):
         run_decode(a)
     else:

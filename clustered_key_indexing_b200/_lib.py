@@ -113,6 +113,7 @@ def lib():
         L.lsa_l2_read_bytes.argtypes = [sz, i32]
         L.lsa_l2_read_bytes.restype = i64
         L.lsa_l2_read.argtypes = [vp, sz, i32, i32, vp, vp]
+        L.lsa_attn_backward.argtypes = [vp, vp, vp, vp, vp, vp, i64, i32, i32, i32, i64, vp, vp, vp, vp]
         for name in exported_names():
             if getattr(L, name).restype is ctypes.c_int:
                 getattr(L, name).restype = i32

@@ -219,6 +219,33 @@ def sparse_attn(Q, K, V, idx, T: int | None = None, O=None, stream=None) -> torc
     return O
 
 
+def attn_backward(Q, K, V, O, dO, idx, T: int | None = None, dK=None, dV=None, stream=None):
+    """lsa_attn_backward: gradients of the sparse attention over saved index
+    lists.  Returns (dQ [nq, hq, 128], dK, dV [T, hkv, 128]), fp32; dK and dV
+    are added to when given (so query chunks accumulate), else zero-started."""
+    _spec(Q, "Q", BF16, (None, None, 128))
+    nq, hq, d = Q.shape
+    _spec(O, "O", BF16, tuple(Q.shape))
+    _spec(dO, "dO", BF16, tuple(Q.shape))
+    _spec(K, "K", BF16, (None, None, 128))
+    _spec(V, "V", BF16, tuple(K.shape))
+    hkv = K.shape[1]
+    _spec(idx, "idx", I32, (nq, hkv, None))
+    _spec(dK, "dK", F32, tuple(K.shape))
+    _spec(dV, "dV", F32, tuple(K.shape))
+    _need_cuda(Q, K, V, O, dO, idx, dK, dV)
+    T = K.shape[0] if T is None else T
+    dQ = torch.empty((nq, hq, d), dtype=torch.float32, device=Q.device)
+    if dK is None:
+        dK = torch.zeros((K.shape[0], hkv, d), dtype=torch.float32, device=Q.device)
+    if dV is None:
+        dV = torch.zeros((V.shape[0], hkv, d), dtype=torch.float32, device=Q.device)
+    check(lib().lsa_attn_backward(_ptr(Q), _ptr(K), _ptr(V), _ptr(O), _ptr(dO), _ptr(idx), nq, hq, hkv,
+                                  idx.shape[2], T, _ptr(dQ), _ptr(dK), _ptr(dV), _stream(stream)),
+          "lsa_attn_backward")
+    return dQ, dK, dV
+
+
 def select_attn_workspace_bytes(nq: int, hq: int) -> int:
     return int(lib().lsa_select_attn_workspace_bytes(nq, hq))
 

@@ -9,3 +9,4 @@
 #include "lsa_noalloc.cu"
 #include "lsa_pca.cu"
 #include "lsa_probe.cu"
+#include "lsa_bwd.cu"

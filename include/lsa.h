@@ -454,6 +454,30 @@ lsa_status lsa_fit_pca(const uint16_t* K, int64_t T, int32_t hkv, int32_t d_late
                        float* W_out, double* eig_out, void* ws, size_t ws_bytes,
                        void* stream);
 
+/*
+ * Gradient of the sparse attention over saved index lists [tutorial
+ * "隐空间稀疏注意力 (LSA)", section 二: the attention; essay "《卡片柜》",
+ * ch. 6: the natively trained variant's backward keeps every query's
+ * selected key indices].  The selection carries no gradient.  For every
+ * (query, head h) with row idx[q, h / G, :] (entries < 0 are padding), with
+ * s_j = q.k_j / sqrt(d), p = softmax(s) and D = dO . O:
+ *   dQ[q, h]  = (1/sqrt(d)) sum_j p_j (dO . v_j - D) k_j      (written)
+ *   dK[j, g] += (1/sqrt(d)) p_j (dO . v_j - D) q              (added)
+ *   dV[j, g] += p_j dO                                        (added)
+ * Q, O, dO [nq, hq, d_head] bf16 (O: the forward's output for the same rows);
+ * K, V [T, hkv, d_head] bf16; all five 16-byte aligned.  idx [nq, hkv, n_idx]
+ * int32; an entry >= T raises the device error word (LSA_EDEVICE at the next
+ * lsa_check_device_error) and is skipped.  dQ [nq, hq, d_head] fp32; dK, dV
+ * [T, hkv, d_head] fp32, 8-byte aligned, accumulated into so that query
+ * chunks add up: the caller zeroes them first.  fp32 accumulation; P and dS
+ * enter the tensor-core products rounded to bf16.  Asynchronous on `stream`;
+ * no workspace.  hq / hkv must be 1, 2, 4 or 8.
+ */
+lsa_status lsa_attn_backward(const uint16_t* Q, const uint16_t* K, const uint16_t* V,
+                             const uint16_t* O, const uint16_t* dO, const int32_t* idx,
+                             int64_t nq, int32_t hq, int32_t hkv, int32_t n_idx, int64_t T,
+                             float* dQ, float* dK, float* dV, void* stream);
+
 #ifdef __cplusplus
 }
 #endif
