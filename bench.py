@@ -87,6 +87,7 @@ def parse():
     p.add_argument("--no-cpu", action="store_true")
     p.add_argument("--no-tree", action="store_true", help="skip the tree-search timing on the prefill line")
     p.add_argument("--no-decode", action="store_true", help="skip the decode block on the 1M prefill line")
+    p.add_argument("--fp8", action="store_true", help="decode: FP8 (e4m3) centroid cache for the flat scan")
     p.add_argument("--pca", action="store_true", help="time the training-free projection fit on the workload's keys")
     p.add_argument("--backward", action="store_true",
                    help="time the sparse-attention backward over the layer's saved index rows")
@@ -702,16 +703,17 @@ def decode_measure(args, world, rank, dev):
     Wk, Wq = torch.from_numpy(Wk_np).to(dev), torch.from_numpy(Wq_np).to(dev)
     ccfg = cfg.c()
     cw = dict(c, batch=B)
+    fp8 = bool(getattr(args, "fp8", False)) and cfg.mode == 0
     if c.get("shared_prefix"):
         # one shared K/V for the prompt's whole blocks but the last, every
         # request's own tokens after it
         sl = 512 * ((n0 - 512) // 512)
         shared = synth.device_shared_prefix(cw, rank, dev, sl)
-        dec = lsa.Decode(B, hkv, hq, cap, cfg, device=dev, shared=shared)
+        dec = lsa.Decode(B, hkv, hq, cap, cfg, device=dev, shared=shared, fp8=fp8)
         q, kk, vv = synth.device_decode_tails(cw, rank, dev, sl, n0, nsteps, dec.K, dec.V)
     else:
         sl = 0
-        dec = lsa.Decode(B, hkv, hq, cap, cfg, device=dev)
+        dec = lsa.Decode(B, hkv, hq, cap, cfg, device=dev, fp8=fp8)
         q, kk, vv = synth.device_decode(cw, rank, dev, n0, nsteps, dec.K, dec.V)
     for r in range(B):
         check(lib().lsa_decode_load(ctypes_ref(dec.d), r, n0, ctypes_ptr(Wk), ctypes_ref(ccfg),
@@ -759,7 +761,7 @@ def decode_measure(args, world, rank, dev):
             kernels[name] = {"ms_per_step": kms / args.steps, "launches_per_step": kn / args.steps}
     lsa.check_device_error()
     # algorithmic bytes per step: the centroids the search must read (128 B,
-    # with a 4-byte record) -- flat: every eligible bucket; tree: the children
+    # FP8 64 B, with a 4-byte record) -- flat: every eligible bucket; tree: the children
     # of the beam at every level above L* plus the B * 2^L* leaves under the
     # final beam -- the gathered K/V rows of every index entry (512 B), Q and O
     row = cfg.row
@@ -777,7 +779,7 @@ def decode_measure(args, world, rank, dev):
             nb = min(nb, 64 * ((pos + 1) // 512))
             if cfg.mode == 1:
                 nb = min(nb, tree_nodes)
-            byts += hkv * (nb * 132 + row * 512) + 2 * hq * c["d"] * 2
+            byts += hkv * (nb * (68 if fp8 else 132) + row * 512) + 2 * hq * c["d"] * 2
     byts /= args.steps
     pk, src = peaks()
     achieved = byts / (ms_step / 1e3) / 1e9
@@ -791,6 +793,7 @@ def decode_measure(args, world, rank, dev):
         "config": {"workload": args.workload, "batch": c["batch"], "context": T, "shared_prefix": sl, "hkv": hkv,
                    "hq": hq, "k": c["k"], "sinks": c["sinks"], "window": c["window"],
                    "search": "flat" if c["mode"] == 0 else f"tree(beam={c['beam']})",
+                   "centroids": "fp8 e4m3 (64 B)" if fp8 else "bf16 (128 B)",
                    "parallelism": f"requests split over {world} GPU(s)" if world > 1 else "1 GPU",
                    "inputs": "device-drawn (torch Philox), same recipe as synth",
                    "l2": f"no flush: per-step centroid scan ({byts / 1e9:.1f} GB) is larger than L2"},

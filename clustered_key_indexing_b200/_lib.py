@@ -31,7 +31,7 @@ class lsa_cache(ctypes.Structure):
     _fields_ = [("hkv", i32), ("n_tokens", i64), ("cap_units", i64), ("cap_buckets", i64),
                 ("U", vp), ("bucket_of_unit", vp), ("members", vp), ("offsets", vp),
                 ("cnt_lr", vp), ("minlr", vp), ("maxpos", vp), ("sum", vp), ("cent", vp),
-                ("units", vp)]
+                ("units", vp), ("cent8", vp)]
 
 
 class lsa_tree(ctypes.Structure):

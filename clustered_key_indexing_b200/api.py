@@ -79,7 +79,9 @@ class Cache:
     `cap_tokens` tokens per head."""
 
     def __init__(self, hkv: int, cap_tokens: int, cfg: Config | None = None, device="cuda",
-                 with_units: bool = True):
+                 with_units: bool = True, fp8: bool = False):
+        """fp8: also keep FP8 (e4m3) centroids, which the flat decode step
+        then scores (lsa_cache.cent8)."""
         cfg = cfg or Config()
         cc = cfg.c()
         L = lib()
@@ -99,10 +101,11 @@ class Cache:
         self.sum = torch.zeros((hkv, self.cap_buckets, dl), dtype=torch.float64, **z)
         self.cent = torch.zeros((hkv, self.cap_buckets, dl), dtype=torch.bfloat16, **z)
         self.units = torch.zeros((hkv, self.cap_buckets), dtype=torch.int32, **z)
+        self.cent8 = torch.zeros((hkv, self.cap_buckets, dl), dtype=torch.uint8, **z) if fp8 else None
         self.c = _lib.lsa_cache(hkv, 0, self.cap_units, self.cap_buckets, *[
             t.data_ptr() for t in (self.U, self.bucket_of_unit, self.members, self.offsets,
                                    self.cnt_lr, self.minlr, self.maxpos, self.sum, self.cent,
-                                   self.units)])
+                                   self.units)], self.cent8.data_ptr() if fp8 else None)
 
     @property
     def n_tokens(self) -> int:
@@ -376,10 +379,12 @@ class Decode:
     (request, kv-head) pairs, the per-request block ring, and (tree mode) the
     tree.  `load` installs a prompt, `step` decodes one token per request."""
 
-    def __init__(self, batch: int, hkv: int, hq: int, cap: int, cfg: Config, device="cuda", shared=None):
+    def __init__(self, batch: int, hkv: int, hq: int, cap: int, cfg: Config, device="cuda", shared=None,
+                 fp8: bool = False):
         """`shared`: optional (K_shared, V_shared) [shared_len, hkv, 128], a
         prefix every request starts with (shared_len a multiple of 512); the
-        pools then hold each request's tokens from shared_len on."""
+        pools then hold each request's tokens from shared_len on.  `fp8`: the
+        cache keeps FP8 centroids and the flat search scores those."""
         if cap % 512:
             raise ValueError("cap must be a multiple of 512")
         self.cfg = cfg
@@ -390,7 +395,7 @@ class Decode:
         self.K = torch.zeros((batch, cap - sl, hkv, 128), dtype=torch.bfloat16, **z)
         self.V = torch.zeros((batch, cap - sl, hkv, 128), dtype=torch.bfloat16, **z)
         self.U_blk = torch.zeros((batch * hkv, 128, 64), dtype=torch.float64, **z)
-        self.cache = Cache(batch * hkv, cap, cfg, device=device, with_units=False)
+        self.cache = Cache(batch * hkv, cap, cfg, device=device, with_units=False, fp8=fp8)
         self.tree = Tree(self.cache, device=device) if cfg.mode == 1 else None
         d = _lib.lsa_decode()
         d.batch, d.hkv, d.hq, d.cap = batch, hkv, hq, cap

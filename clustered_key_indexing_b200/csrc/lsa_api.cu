@@ -145,8 +145,8 @@ static lsa_status check_cache(const lsa_cache* c, bool need_built) {
     if (c->cap_buckets < ceil_div<int64_t>(c->cap_units, kUnitsPerBlock) * kBucketsPerBlock)
         return set_error(LSA_EINVAL, "cache: cap_buckets < 64 * ceil(cap_units / 128)");
     if (c->cap_units > (int64_t)1 << 30) return set_error(LSA_EUNSUPPORTED, "cache: more than 2^30 units");
-    if (!aligned16(c->cent) || !aligned16(c->sum) || !aligned16(c->U))
-        return set_error(LSA_EINVAL, "cache: U, sum and cent must be 16-byte aligned");
+    if (!aligned16(c->cent) || !aligned16(c->sum) || !aligned16(c->U) || !aligned16(c->cent8))
+        return set_error(LSA_EINVAL, "cache: U, sum, cent and cent8 must be 16-byte aligned");
     if (need_built && c->n_tokens <= 0) return set_error(LSA_EINVAL, "cache: not built (n_tokens == 0)");
     if (c->n_tokens > c->cap_units * kPool) return set_error(LSA_EINVAL, "cache: n_tokens beyond capacity");
     return LSA_OK;

@@ -245,6 +245,7 @@ struct WardArgs {
     double* sum;
     uint16_t* cent;
     int32_t* units;
+    uint8_t* cent8;      // optional FP8 centroids (NULL: none)
 };
 
 __device__ __forceinline__ int tri_index(int i, int j) {  // i < j < 128
@@ -490,6 +491,11 @@ __global__ void __launch_bounds__(128, 1) ward_kernel(WardArgs a) {
         uint16_t* cb = a.cent + (hb0 + b) * kDL;
         for (int c = 0; c < kDL; ++c)
             cb[c] = f64_to_bf16_rne(nrm > 0.0 ? __ddiv_rn(sb[c], nrm) : 0.0);
+        if (a.cent8) {  // e4m3 of 2^8 times the same fp64 component (exact scaling)
+            uint8_t* c8 = a.cent8 + (hb0 + b) * kDL;
+            for (int c = 0; c < kDL; ++c)
+                c8[c] = f64_to_e4m3_rne(nrm > 0.0 ? __ddiv_rn(sb[c], nrm) * 256.0 : 0.0);
+        }
     }
     if (tid >= m && tid < kBucketsPerBlock) {
         const int64_t b = blk * kBucketsPerBlock + tid;
@@ -501,6 +507,7 @@ __global__ void __launch_bounds__(128, 1) ward_kernel(WardArgs a) {
         for (int c = 0; c < kDL; ++c) {
             a.sum[(hb0 + b) * kDL + c] = 0.0;
             a.cent[(hb0 + b) * kDL + c] = 0;
+            if (a.cent8) a.cent8[(hb0 + b) * kDL + c] = 0;
         }
     }
     if (tid == 0) offs[(blk + 1) * kBucketsPerBlock] = (int32_t)(u0 + n);
@@ -510,7 +517,7 @@ static void fill_ward_cache(WardArgs& a, const lsa_cache* c) {
     a.cap_units = c->cap_units; a.cap_buckets = c->cap_buckets;
     a.bucket_of_unit = c->bucket_of_unit; a.members = c->members; a.offsets = c->offsets;
     a.cnt_lr = c->cnt_lr; a.minlr = c->minlr; a.maxpos = c->maxpos; a.sum = c->sum; a.cent = c->cent;
-    a.units = c->units;
+    a.units = c->units; a.cent8 = c->cent8;
 }
 
 static size_t ward_smem() {
@@ -565,8 +572,8 @@ lsa_status launch_ward_jobs(const lsa_cache* c, const double* U_blk, int32_t hkv
 
 // Mark bucket slots [b0, b1) of every head empty.
 __global__ void clear_slots_kernel(int32_t* cnt_lr, int32_t* minlr, int32_t* maxpos, double* sum,
-                                   uint16_t* cent, int32_t* units, int64_t cap_buckets, int64_t b0,
-                                   int64_t b1, int32_t hkv) {
+                                   uint16_t* cent, int32_t* units, uint8_t* cent8, int64_t cap_buckets,
+                                   int64_t b0, int64_t b1, int32_t hkv) {
     const int64_t span = b1 - b0;
     const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     if (i >= span * hkv * kDL) return;
@@ -575,6 +582,7 @@ __global__ void clear_slots_kernel(int32_t* cnt_lr, int32_t* minlr, int32_t* max
     const int64_t hb = h * cap_buckets + b;
     sum[hb * kDL + c] = 0.0;
     cent[hb * kDL + c] = 0;
+    if (cent8) cent8[hb * kDL + c] = 0;
     if (c == 0) {
         cnt_lr[hb] = 0;
         minlr[hb] = kIMax;
@@ -587,7 +595,7 @@ lsa_status launch_clear_slots(const lsa_cache* c, int64_t b0, int64_t b1, cudaSt
     if (b1 <= b0) return LSA_OK;
     const int64_t n = (b1 - b0) * c->hkv * kDL;
     clear_slots_kernel<<<(unsigned)ceil_div<int64_t>(n, 256), 256, 0, st>>>(
-        c->cnt_lr, c->minlr, c->maxpos, c->sum, c->cent, c->units, c->cap_buckets, b0, b1, c->hkv);
+        c->cnt_lr, c->minlr, c->maxpos, c->sum, c->cent, c->units, c->cent8, c->cap_buckets, b0, b1, c->hkv);
     return check_launch("clear_slots_kernel");
 }
 

@@ -74,6 +74,48 @@ __device__ __forceinline__ uint16_t f64_to_bf16_rne(double x) {
     return (uint16_t)(sign | (uint16_t)(__float_as_uint(f) >> 16));
 }
 
+// OCP FP8 E4M3 ("fn": bias 7, 3 mantissa bits, no infinities, largest
+// finite 448, exponent field 0 = subnormals m * 2^-9).  Round a double to
+// the nearest code, ties to the even mantissa, saturating at +-448: normal
+// magnitudes keep the top 3 of the 52 mantissa bits (a carry out of them
+// moves to the next exponent), magnitudes below 2^-6 are the integer
+// nearest a * 2^9 (0 .. 8, where 8 is the smallest normal, code 0x08).
+__device__ __forceinline__ uint8_t f64_to_e4m3_rne(double x) {
+    if (isnan(x)) return 0x7F;
+    const uint8_t sign = signbit(x) ? 0x80 : 0;
+    const double a = fabs(x);
+    if (a == 0.0) return sign;
+    const unsigned long long b = (unsigned long long)__double_as_longlong(a);
+    const int e = (int)(b >> 52) - 1023;  // a in [2^e, 2^(e+1))
+    if (e >= -6) {
+        if (e > 8) return (uint8_t)(sign | 0x7E);
+        const unsigned long long mant = b & ((1ull << 52) - 1ull);
+        uint32_t q = ((uint32_t)(e + 7) << 3) | (uint32_t)(mant >> 49);
+        const unsigned long long rem = mant & ((1ull << 49) - 1ull), half = 1ull << 48;
+        if (rem > half || (rem == half && (q & 1u))) ++q;
+        return (uint8_t)(sign | (q > 0x7Eu ? 0x7Eu : q));
+    }
+    return (uint8_t)(sign | (uint8_t)__double2int_rn(a * 512.0));  // exact scaling, then nearest even
+}
+
+// Value of an e4m3 code (the NaN codes are never written).
+__device__ __forceinline__ double e4m3_to_f64(uint32_t c) {
+    const int e = (int)((c >> 3) & 15u), m = (int)(c & 7u);
+    const double v = e == 0 ? (double)m * 0x1p-9 : ldexp((double)(8 + m), e - 10);
+    return (c & 0x80u) ? -v : v;
+}
+
+// Exact score of a bf16 latent and an FP8 centroid (values 2^-8 * e4m3):
+// every product of a bf16 and an e4m3 value is exact in fp64; ascending
+// index order, as for two bf16 latents.
+__device__ __forceinline__ double dot_bf16_fp8_exact(const uint16_t* __restrict__ y,
+                                                     const uint8_t* __restrict__ c) {
+    double s = 0.0;
+#pragma unroll 8
+    for (int i = 0; i < kDL; ++i) s = fma(bf16_to_f64(y[i]), e4m3_to_f64(c[i]) * 0x1p-8, s);
+    return s;
+}
+
 // Exact score of two bf16 latents: every product of two bf16 values is exact
 // in fp64; the sum runs in ascending index order.
 __device__ __forceinline__ double dot_bf16_exact(const uint16_t* __restrict__ y,

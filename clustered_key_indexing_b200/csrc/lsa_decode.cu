@@ -24,6 +24,7 @@
 // rescoring, weighted radix select, key emission in bucket-id order.  Rows
 // whose kept bins overflow shared memory take exact fp64 scores of every
 // eligible bucket in a global slot.
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -404,6 +405,172 @@ __global__ void __launch_bounds__(128) decode_score_kernel(const __grid_constant
         if (shist[i]) atomicAdd(a.hist + row * kDecBins + i, shist[i]);
 }
 
+// The same scan over FP8 centroids (lsa_cache.cent8: e4m3 codes of 2^8 c,
+// 64 bytes per bucket).  TMA brings 256-row tiles of the codes (16 KB, no
+// swizzle) through a 6-stage ring; each lane converts its rows' codes to
+// fp16 pairs (exact) and scores them with fp16 mma.sync against the row's
+// query latents (bf16 -> fp16: exact for components >= 2^-14, the smaller
+// ones move a score by under 2^-21) with fp32 accumulation.  The MMA's K
+// order is a permutation of the 64 dims, the same on both operands: lane
+// (g, t) takes dims 16 t .. 16 t + 15 of its two centroid rows with one
+// 16-byte load each (rows 64 bytes apart: a quarter-warp reads 128
+// contiguous bytes), k-step kk of the MMA covering dims 16 t + 4 kk .. + 3.
+// Scores come out times 2^8 and are scaled back exactly.  Their error stays
+// below 1e-5 < e, and |score| <= 1.07 |y| (an e4m3 component is within
+// 2^-4 of its value relative, so |c8| <= 1.0625 + 2^-17): the row radius
+// grows by that factor and the binning, keep and exact fp64 rescoring
+// (against the same FP8 values) are unchanged.
+constexpr int kDec8Stages = 6;
+constexpr size_t kDec8ScanSmem = 1024 + (size_t)kDec8Stages * kDecTile * kDL + kDecTile * 4 + 64;
+
+__device__ __forceinline__ float row_radius8(const uint16_t* y, int ng) {
+    float R = 0.f;
+    for (int g = 0; g < ng; ++g) {
+        float n2 = 0.f;
+        for (int i = 0; i < kDL; ++i) { const float v = bf16_to_f32(y[g * kDL + i]); n2 += v * v; }
+        R = fmaxf(R, sqrtf(n2));
+    }
+    return fmaxf(0.25f, fminf(1.14f, R * 1.07f + 1e-6f));
+}
+
+__device__ __forceinline__ uint32_t bf16_pair_to_f16x2(uint16_t lo, uint16_t hi) {
+    const __half2 h = __floats2half2_rn(bf16_to_f32(lo), bf16_to_f32(hi));
+    return *reinterpret_cast<const uint32_t*>(&h);
+}
+
+template <int NG>
+__global__ void __launch_bounds__(128) decode_score8_kernel(const __grid_constant__ CUtensorMap tmC, DecScoreArgs a) {
+    extern __shared__ uint8_t dsm_raw[];
+    uint8_t* dsm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsm_raw) + 1023) & ~(uintptr_t)1023);
+    uint8_t* ring = dsm;
+    float* best_s = reinterpret_cast<float*>(ring + kDec8Stages * kDecTile * kDL);  // [kDecTile]
+    uint64_t* bars = reinterpret_cast<uint64_t*>(best_s + kDecTile);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + kDec8Stages);
+    __shared__ float rad;
+    __shared__ uint32_t shist[kDecBins];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int64_t row = blockIdx.y;
+    const int64_t r = row / a.hkv;
+    const int64_t t = a.pos[r];
+    const int64_t lim = t - a.W;
+    const int64_t ncol = lim < 0 ? 0 : min(a.cap_buckets, (int64_t)kBucketsPerBlock * (lim / kBlockKeys + 1));
+    const int64_t c0 = (int64_t)blockIdx.x * kDecScanCols;
+    if (c0 >= ncol) return;
+    const int64_t cend = min(ncol, c0 + kDecScanCols);
+    const int ntiles = (int)((cend - c0 + kDecTile - 1) / kDecTile);
+    const uint32_t bar0 = smem_u32(bars);
+    constexpr uint32_t kTileB = kDecTile * kDL;  // 16 KB
+    for (int i = tid; i < kDecBins; i += 128) shist[i] = 0u;
+    if (tid == 0) {
+        for (int s = 0; s < kDec8Stages; ++s) mbar_init(bar0 + 8u * s, 1);
+        *abort_flag = 0;
+        fence_barrier_init();
+    }
+    const uint16_t* yb = a.Y + (row * NG) * kDL;
+    if (tid == 0) rad = row_radius8(yb, NG);
+    // B operand in the permuted K order: k-step kk, lane (g, t): dims
+    // 16 t + 4 kk + {0, 1} (b0) and + {2, 3} (b1) of latent row g
+    const int gq = lane >> 2, tq = lane & 3;
+    uint32_t yq[4][2];
+#pragma unroll
+    for (int kk = 0; kk < 4; ++kk) {
+        const uint16_t* yr = yb + gq * kDL + 16 * tq + 4 * kk;
+        yq[kk][0] = gq < NG ? bf16_pair_to_f16x2(yr[0], yr[1]) : 0u;
+        yq[kk][1] = gq < NG ? bf16_pair_to_f16x2(yr[2], yr[3]) : 0u;
+    }
+    __syncthreads();
+    const int64_t rowbase = row * a.cap_buckets;
+    if (tid == 0) {
+        for (int i = 0; i < kDec8Stages && i < ntiles; ++i) {
+            mbar_expect_tx(bar0 + 8u * i, kTileB);
+            tma_load_2d(smem_u32(ring + i * kTileB), &tmC, 0, (int32_t)(rowbase + c0 + i * kDecTile), bar0 + 8u * i);
+        }
+    }
+    const float R = rad;
+    const int64_t hb0 = rowbase;
+    const int64_t frontier = ncol - kBucketsPerBlock;
+    int done = 0;
+    for (int it = 0; it < ntiles; ++it) {
+        const int s = it % kDec8Stages;
+        const int64_t tb0 = c0 + (int64_t)it * kDecTile;
+        int32_t clr_pre[kDecTile / 128];
+#pragma unroll
+        for (int u = 0; u < kDecTile / 128; ++u) {
+            const int64_t b = tb0 + tid + 128 * u;
+            clr_pre[u] = b < cend ? __ldg(a.cnt_lr + hb0 + b) : 0;
+        }
+        const bool ok = mbar_wait(bar0 + 8u * s, (uint32_t)(it / kDec8Stages) & 1u, abort_flag);
+        if (!__syncthreads_and(ok)) break;
+        const uint8_t* tile = ring + s * kTileB;
+#pragma unroll
+        for (int mt = 0; mt < 4; ++mt) {
+            const int m0 = 64 * warp + 16 * mt;
+            const uint4 ra = *reinterpret_cast<const uint4*>(tile + (m0 + gq) * kDL + 16 * tq);
+            const uint4 rb = *reinterpret_cast<const uint4*>(tile + (m0 + gq + 8) * kDL + 16 * tq);
+            const uint32_t wa[4] = {ra.x, ra.y, ra.z, ra.w}, wb[4] = {rb.x, rb.y, rb.z, rb.w};
+            float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+                const uint32_t af[4] = {e4m3x2_to_f16x2(wa[kk] & 0xFFFFu), e4m3x2_to_f16x2(wb[kk] & 0xFFFFu),
+                                        e4m3x2_to_f16x2(wa[kk] >> 16), e4m3x2_to_f16x2(wb[kk] >> 16)};
+                mma_16816_f16(acc, af, yq[kk][0], yq[kk][1]);
+            }
+            float b0 = NG > 1 ? fmaxf(acc[0], acc[1]) : acc[0];
+            float b1 = NG > 1 ? fmaxf(acc[2], acc[3]) : acc[2];
+            if (NG > 2) {
+                b0 = fmaxf(b0, __shfl_xor_sync(0xffffffffu, b0, 1));
+                b1 = fmaxf(b1, __shfl_xor_sync(0xffffffffu, b1, 1));
+            }
+            if (NG > 4) {
+                b0 = fmaxf(b0, __shfl_xor_sync(0xffffffffu, b0, 2));
+                b1 = fmaxf(b1, __shfl_xor_sync(0xffffffffu, b1, 2));
+            }
+            if (tq == 0) {
+                best_s[m0 + gq] = b0 * 0x1p-8f;
+                best_s[m0 + gq + 8] = b1 * 0x1p-8f;
+            }
+        }
+        __syncthreads();
+        if (tid == 0 && it + kDec8Stages < ntiles) {
+            fence_proxy_async_smem();
+            mbar_expect_tx(bar0 + 8u * s, kTileB);
+            tma_load_2d(smem_u32(ring + s * kTileB), &tmC, 0, (int32_t)(rowbase + c0 + (it + kDec8Stages) * kDecTile),
+                        bar0 + 8u * s);
+        }
+#pragma unroll
+        for (int u = 0; u < kDecTile / 128; ++u) {
+            const int j = tid + 128 * u;
+            const int64_t b = tb0 + j;
+            if (b >= cend) break;
+            const int32_t clr = clr_pre[u];
+            int w = clr;
+            if (b >= frontier) {
+                const int32_t mlr = __ldg(a.minlr + hb0 + b), mxp = __ldg(a.maxpos + hb0 + b);
+                w = 0;
+                if ((int64_t)mlr <= lim)
+                    w = (int64_t)mxp <= lim ? clr : weight_units(b, __ldg(a.units + hb0 + b), lim, a.S, a.T_built);
+            }
+            const int bn = score_to_bin(best_s[j], R);
+            a.bin[row * a.ld + b] = (uint16_t)bn;
+            a.wt[row * a.ld + b] = (uint8_t)w;
+            if (w > 0) atomicAdd(&shist[bn], (uint32_t)w);
+        }
+        __syncthreads();
+        done = it + 1;
+    }
+    if (tid == 0 && *abort_flag) {
+        const int issued = min(ntiles, done + kDec8Stages);
+        for (int i = done; i < issued; ++i)
+            mbar_wait(bar0 + 8u * (i % kDec8Stages), (uint32_t)(i / kDec8Stages) & 1u, abort_flag, false);
+    }
+    __syncthreads();
+    long long tc;
+    const int jc = dec_cut_block(shist, a.k, &tc);
+    if (tid == 0 && tc) atomicAdd(a.tot + row, (unsigned long long)tc);
+    for (int i = jc + tid; i < kDecBins; i += 128)
+        if (shist[i]) atomicAdd(a.hist + row * kDecBins + i, shist[i]);
+}
+
 // ------------------------------------------------------ flat decode cut
 
 // Slots of chunk [c0, c0 + kDecScanCols) of a row with a key in [S, t - W]
@@ -584,7 +751,8 @@ __global__ void __launch_bounds__(kSelThreads) decode_resolve_kernel(DecResolveA
         const int64_t hb0 = (int64_t)r.h * d.cap_buckets;
         for (int i = tid; i < n; i += kSelThreads) {
             const int64_t b = sh.cid[i];
-            sh.csc[i] = exact_row(sh.ylat, ng, a.cent + (hb0 + b) * kDL);
+            sh.csc[i] = a.cent8 ? exact_row8(sh.ylat, ng, a.cent8 + (hb0 + b) * kDL)
+                                : exact_row(sh.ylat, ng, a.cent + (hb0 + b) * kDL);
             sh.cw[i] = wrow[b];
         }
         __syncthreads();
@@ -598,7 +766,9 @@ __global__ void __launch_bounds__(kSelThreads) decode_resolve_kernel(DecResolveA
     double* fs = d.slot + row * d.ld;
     const int64_t hb0 = (int64_t)r.h * d.cap_buckets;
     for (int64_t b = tid; b < ncol; b += kSelThreads)
-        fs[b] = wrow[b] > 0 ? exact_row(sh.ylat, ng, a.cent + (hb0 + b) * kDL) : 0.0;
+        fs[b] = wrow[b] == 0 ? 0.0
+                : a.cent8 ? exact_row8(sh.ylat, ng, a.cent8 + (hb0 + b) * kDL)
+                          : exact_row(sh.ylat, ng, a.cent + (hb0 + b) * kDL);
     __syncthreads();
     radix_fill(
         ncol, a.k, [&](int64_t i) { return fs[i]; }, [&](int64_t i) { return (int)wrow[i]; },
@@ -666,6 +836,7 @@ static lsa_cache request_view(const lsa_decode* d, int32_t r) {
     v.sum += h0 * v.cap_buckets * kDL;
     v.cent += h0 * v.cap_buckets * kDL;
     v.units += h0 * v.cap_buckets;
+    if (v.cent8) v.cent8 += h0 * v.cap_buckets * kDL;
     return v;
 }
 
@@ -728,6 +899,7 @@ static void fill_select_args(SelectArgs& a, const lsa_decode* d, const lsa_cfg* 
     }
     a.Y = Y; a.nqc = d->batch; a.t_first = 0; a.idx = idx;
     a.decode = 1;
+    a.cent8 = cfg->mode == 0 ? c.cent8 : nullptr;  // the flat decode search scores the FP8 centroids
     for (int r = 0; r < d->batch; ++r) a.pos[r] = d->len[r];
 }
 
@@ -854,13 +1026,25 @@ lsa_status lsa_decode_step(lsa_decode* d, const uint16_t* q, const uint16_t* k, 
         dim3 grid((unsigned)ceil_div<int64_t>(d->cache.cap_buckets, kDecScanCols), (unsigned)rows);
         const int ng = cfg->agg ? d->hq / d->hkv : 1;
         CUtensorMap tmC;
-        if ((s = make_rows64_map(&tmC, d->cache.cent, rows * d->cache.cap_buckets, kDecTile)) != LSA_OK) return s;
-        auto kern = ng == 1 ? decode_score_kernel<1> : ng == 2 ? decode_score_kernel<2>
-                  : ng == 4 ? decode_score_kernel<4> : decode_score_kernel<8>;
-        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kDecScanSmem);
-        {
-            KTime kt_("decode_score_kernel", st);
-            kern<<<grid, 128, kDecScanSmem, st>>>(tmC, sa);
+        if (d->cache.cent8) {
+            if ((s = make_rows64_u8_map(&tmC, d->cache.cent8, rows * d->cache.cap_buckets, kDecTile)) != LSA_OK)
+                return s;
+            auto kern = ng == 1 ? decode_score8_kernel<1> : ng == 2 ? decode_score8_kernel<2>
+                      : ng == 4 ? decode_score8_kernel<4> : decode_score8_kernel<8>;
+            cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kDec8ScanSmem);
+            {
+                KTime kt_("decode_score_kernel", st);
+                kern<<<grid, 128, kDec8ScanSmem, st>>>(tmC, sa);
+            }
+        } else {
+            if ((s = make_rows64_map(&tmC, d->cache.cent, rows * d->cache.cap_buckets, kDecTile)) != LSA_OK) return s;
+            auto kern = ng == 1 ? decode_score_kernel<1> : ng == 2 ? decode_score_kernel<2>
+                      : ng == 4 ? decode_score_kernel<4> : decode_score_kernel<8>;
+            cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kDecScanSmem);
+            {
+                KTime kt_("decode_score_kernel", st);
+                kern<<<grid, 128, kDecScanSmem, st>>>(tmC, sa);
+            }
         }
         if ((s = check_launch("decode_score_kernel")) != LSA_OK) return s;
         DecKeepArgs ka{};

@@ -602,6 +602,28 @@ __device__ __forceinline__ double exact_row(const uint16_t* ylat, int ng, const 
     return best;
 }
 
+// exact_row against an FP8 centroid (64 e4m3 codes of 2^8 c): products of a
+// bf16 and a 2^-8 e4m3 value are exact in fp64, ascending dimension order.
+__device__ __forceinline__ double exact_row8(const uint16_t* ylat, int ng, const uint8_t* c8) {
+    uint4 cv[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) cv[i] = __ldg(reinterpret_cast<const uint4*>(c8) + i);
+    double best = -CUDART_INF;
+    for (int g = 0; g < ng; ++g) {
+        const uint16_t* y = ylat + g * kDL;
+        double s = 0.0;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const uint32_t wv[4] = {cv[i].x, cv[i].y, cv[i].z, cv[i].w};
+#pragma unroll
+            for (int e = 0; e < 16; ++e)
+                s = fma(bf16_to_f64(y[16 * i + e]), e4m3_to_f64((wv[e >> 2] >> (8 * (e & 3))) & 0xFFu) * 0x1p-8, s);
+        }
+        best = s > best ? s : best;
+    }
+    return best;
+}
+
 // exact_row for four centroids at once: four independent fma chains (each
 // in ascending dimension order, so every score equals exact_row's).
 __device__ __forceinline__ void exact_rows4(const uint16_t* ylat, int ng, const uint16_t* const (&c)[4],

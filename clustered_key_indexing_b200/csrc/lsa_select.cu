@@ -55,6 +55,7 @@ struct SelectArgs {
     const int32_t* minlr;
     const int32_t* maxpos;
     const uint16_t* cent;
+    const uint8_t* cent8;  // decode, flat search: FP8 centroids scored instead of cent (NULL: bf16)
     int64_t cap_units, cap_buckets, NB, T_built;
     // tree (mode 1)
     const int32_t* tminlr;

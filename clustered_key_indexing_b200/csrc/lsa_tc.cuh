@@ -236,4 +236,32 @@ static lsa_status make_rows64_map(CUtensorMap* map, const uint16_t* base, int64_
     return LSA_OK;
 }
 
+// Tensor map of a row-major [rows, 64] byte matrix (FP8 centroids, 64-byte
+// rows), box of `box_rows` x 64 bytes, no swizzle.
+static lsa_status make_rows64_u8_map(CUtensorMap* map, const uint8_t* base, int64_t rows, int box_rows) {
+    using EncodeFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+    static EncodeFn encode = nullptr;
+    if (!encode) {
+        void* fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess || !fn ||
+            q != cudaDriverEntryPointSuccess)
+            return set_error(LSA_ECUDA, "cuTensorMapEncodeTiled is not available");
+        encode = reinterpret_cast<EncodeFn>(fn);
+    }
+    if (rows <= 0 || ((uintptr_t)base & 15u) != 0)
+        return set_error(LSA_EINVAL, "tensor map: need rows > 0 and a 16-byte aligned base");
+    const cuuint64_t dims[2] = {(cuuint64_t)kDL, (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)kDL};
+    const cuuint32_t box[2] = {(cuuint32_t)kDL, (cuuint32_t)box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    const CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(base), dims, strides, box,
+                              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return set_error(LSA_ECUDA, "cuTensorMapEncodeTiled (u8) failed (%d)", (int)r);
+    return LSA_OK;
+}
+
 }  // namespace lsa

@@ -98,6 +98,17 @@ typedef struct lsa_cache {
     int32_t*  units;           /* [hkv, cap_buckets] member units packed: bits
                                   7i..7i+6 = i-th member's unit index within its
                                   128-unit block (ascending), bits 28..30 = count */
+    uint8_t*  cent8;           /* optional (NULL = none), [hkv, cap_buckets,
+                                  d_latent], 16-byte aligned: FP8 centroids, the
+                                  OCP e4m3 code of 2^8 * c for each component c
+                                  of the normalised centroid, rounded to nearest
+                                  even straight from fp64 [ch. 8: the bucket
+                                  cache stacks with FP8 quantisation].  When
+                                  present, every build call writes them and the
+                                  flat decode step (lsa_decode_step, mode 0)
+                                  scores the buckets against them (64 bytes per
+                                  bucket instead of 128); prefill selection
+                                  (lsa_select) always scores the bf16 cent.    */
 } lsa_cache;
 
 #define LSA_MAX_LEVELS 48

@@ -30,17 +30,19 @@ def reqs():
     return [synth.layer_inputs("decode-small", seed=r) for r in range(len(PROMPTS))]
 
 
-def _run_decode(lsa, Kl, Vl, Ql, Wk_np, Wq_np, cfg, shared_len=0):
+def _run_decode(lsa, Kl, Vl, Ql, Wk_np, Wq_np, cfg, shared_len=0, fp8=False):
     """Decode STEPS tokens per request after PROMPTS, checking index rows and
     outputs against the oracle over the logical keys Kl[r] (the shared prefix
-    then the request's own tokens)."""
+    then the request's own tokens).  fp8: the cache keeps FP8 centroids,
+    which the flat search scores; the oracle then selects on its own FP8
+    centroids (essay ch. 8), and the library's FP8 codes must equal them."""
     c = synth.CONFIGS["decode-small"]
     hkv, hq, cap = c["hkv"], c["hq"], c["T"]
     Wk, Wq = to_dev(Wk_np), to_dev(Wq_np)  # one W_k / W_q per layer
     shared = None
     if shared_len:
         shared = (to_dev_bf16(Kl[0][:shared_len]), to_dev_bf16(Vl[0][:shared_len]))
-    dec = lsa.Decode(len(PROMPTS), hkv, hq, cap, cfg, shared=shared)
+    dec = lsa.Decode(len(PROMPTS), hkv, hq, cap, cfg, shared=shared, fp8=fp8)
     for r, n in enumerate(PROMPTS):
         dec.load(r, to_dev_bf16(Kl[r][shared_len:n]), to_dev_bf16(Vl[r][shared_len:n]), Wk)
     check_at = {0, 1, 2, 19, STEPS - 1}
@@ -66,8 +68,13 @@ def _run_decode(lsa, Kl, Vl, Ql, Wk_np, Wq_np, cfg, shared_len=0):
             if key not in caches:
                 U = oracle.key_latent_pool(Kl[r][:tb], Wk_np, 4)
                 oc = oracle.build_cache(U, tb, ocfg)
-                caches[key] = (oc, oracle.build_tree(oc) if cfg.mode == 1 else None)
-            oc, ot = caches[key]
+                caches[key] = (oracle.with_fp8_centroids(oc) if fp8 else oc,
+                               oracle.build_tree(oc) if cfg.mode == 1 else None, oc)
+            oc, ot, plain = caches[key]
+            if fp8:   # the library's FP8 codes of the request's complete blocks
+                nb = tb // 512 * 64
+                got8 = dec.cache.cent8[r * hkv:(r + 1) * hkv, :nb].cpu().numpy()
+                assert np.array_equal(got8, oracle.cent_fp8(plain)), (s, r)
             Qt = Ql[r][t:t + 1]
             Y = oracle.query_latent(Qt, Wq_np, hkv, cfg.agg)
             oidx, _, _ = oracle.select(oc, Y, np.array([t]), ocfg, tree=ot, G=hq // hkv)
@@ -97,3 +104,16 @@ def test_decode_shared_prefix_matches_oracle(lsa, reqs, mode):
     Kl = [np.concatenate([reqs[0]["K"][:sl], x["K"][sl:]]) for x in reqs]
     Vl = [np.concatenate([reqs[0]["V"][:sl], x["V"][sl:]]) for x in reqs]
     _run_decode(lsa, Kl, Vl, [x["Q"] for x in reqs], reqs[0]["Wk"], reqs[0]["Wq"], cfg, shared_len=sl)
+
+
+@pytest.mark.parametrize("agg,shared", [(0, False), (1, False), (0, True)])
+def test_decode_fp8_centroids_match_oracle(lsa, reqs, agg, shared):
+    """Flat decode over FP8 (e4m3) centroids: the library's codes equal the
+    oracle's, and the selection equals the oracle's selection on them, bit
+    for bit (products of bf16 and e4m3 values are exact in fp64)."""
+    c = synth.CONFIGS["decode-small"]
+    cfg = lsa.Config(k=c["k"], sinks=c["sinks"], window=600, beam=c["beam"], mode=0, agg=agg)
+    sl = 512 if shared else 0
+    Kl = [np.concatenate([reqs[0]["K"][:sl], x["K"][sl:]]) for x in reqs]
+    Vl = [np.concatenate([reqs[0]["V"][:sl], x["V"][sl:]]) for x in reqs]
+    _run_decode(lsa, Kl, Vl, [x["Q"] for x in reqs], reqs[0]["Wk"], reqs[0]["Wq"], cfg, shared_len=sl, fp8=True)

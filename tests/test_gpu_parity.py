@@ -28,11 +28,11 @@ def lsa():
     return m
 
 
-def _build_both(lsa, name, T, cfg, seed=0):
+def _build_both(lsa, name, T, cfg, seed=0, fp8=False):
     inp = synth.layer_inputs(name, seed=seed, T=T)
     hkv = inp["K"].shape[1]
     K = to_dev_bf16(inp["K"])
-    cache = lsa.Cache(hkv, T, cfg)
+    cache = lsa.Cache(hkv, T, cfg, fp8=fp8)
     lsa.build_buckets(K, to_dev(inp["Wk"]), cfg, cache)
     torch.cuda.synchronize()
     lsa.check_device_error()
@@ -73,6 +73,16 @@ def test_build_bit_exact_8_heads(lsa):
     cfg = lsa.Config(k=2048, sinks=4, window=1024)
     _, cache, U, oc = _build_both(lsa, "prefill-128k", 8192 + 100, cfg)
     _assert_cache_equal(cache, U, oc)
+
+
+@pytest.mark.parametrize("T", [4096, 1000, 7])
+def test_build_fp8_centroids_bit_exact(lsa, T):
+    """A cache with FP8 centroids: the e4m3 codes of 2^8 c equal the
+    oracle's (essay ch. 8), and the rest of the cache is unchanged."""
+    cfg = lsa.Config(k=512, sinks=4, window=256)
+    _, cache, U, oc = _build_both(lsa, "prefill-4k", T, cfg, fp8=True)
+    _assert_cache_equal(cache, U, oc)
+    assert np.array_equal(cache.cent8[:, :oc["NB"]].cpu().numpy(), oracle.cent_fp8(oc))
 
 
 def test_build_degenerate_keys(lsa):
