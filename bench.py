@@ -635,8 +635,11 @@ def run_lsa(args):
                    "Q": bits_of(P.hQ)}
         else:
             inp = P.inp
-        per_layer, desc, spent = oracle_sample(inp, dict(c, hkv=hkv, hq=hq), n_blocks=None if T <= 131072 else 64,
-                                               n_queries=2048 if T <= 131072 else 64)
+        # about 10-20 s of oracle work: 128K: head 0's whole build + 2048
+        # positions; 1M: 512 blocks + 640 positions (the head's whole cache,
+        # which the positions need, is built outside the timed sample)
+        per_layer, desc, spent = oracle_sample(inp, dict(c, hkv=hkv, hq=hq), n_blocks=None if T <= 131072 else 512,
+                                               n_queries=2048 if T <= 131072 else 640)
         cpu = {"value": T / per_layer, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": desc,
                "sample_seconds": spent}
 
