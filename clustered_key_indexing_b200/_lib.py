@@ -113,6 +113,13 @@ def lib():
         L.lsa_l2_read_bytes.argtypes = [sz, i32]
         L.lsa_l2_read_bytes.restype = i64
         L.lsa_l2_read.argtypes = [vp, sz, i32, i32, vp, vp]
+        L.lsa_shard_cand_cap.argtypes = [P(lsa_cfg)]
+        L.lsa_shard_cand_cap.restype = i32
+        L.lsa_shard_build_buckets.argtypes = [vp, i64, i32, vp, P(lsa_cfg), i64, P(lsa_cache), vp]
+        L.lsa_shard_candidates.argtypes = [vp, i64, i64, i32, vp, P(lsa_cache), i64, P(lsa_cfg), vp, vp, vp, sz, vp]
+        L.lsa_shard_merge.argtypes = [vp, vp, i32, i32, i64, i64, P(lsa_cache), i64, P(lsa_cfg), vp, vp]
+        L.lsa_sparse_attn_partial.argtypes = [vp, vp, vp, vp, i64, i32, i32, i32, i64, i64, vp, vp, vp]
+        L.lsa_lse_combine.argtypes = [vp, vp, i32, i64, i32, vp, vp]
         L.lsa_attn_backward.argtypes = [vp, vp, vp, vp, vp, vp, i64, i32, i32, i32, i64, vp, vp, vp, vp]
         for name in exported_names():
             if getattr(L, name).restype is ctypes.c_int:

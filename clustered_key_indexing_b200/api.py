@@ -452,6 +452,103 @@ class Decode:
         return o
 
 
+# ------------------------------------------------ sequence-sharded layer
+
+def shard_cand_cap(cfg: Config) -> int:
+    """lsa_shard_cand_cap: records per (query, kv-head) row."""
+    return int(lib().lsa_shard_cand_cap(ctypes.byref(cfg.c())))
+
+
+def shard_build_buckets(K: torch.Tensor, W_k: torch.Tensor, cfg: Config, p0: int, cache: Cache, stream=None):
+    """lsa_shard_build_buckets: the cache of a shard's keys K [n, hkv, 128]
+    (global positions p0 ..)."""
+    _spec(K, "K", BF16, (None, None, 128))
+    _spec(W_k, "W_k", F32, W_SHAPE)
+    _need_cuda(K, W_k)
+    n, hkv, _ = K.shape
+    check(lib().lsa_shard_build_buckets(_ptr(K), n, hkv, _ptr(W_k), ctypes.byref(cfg.c()), p0,
+                                        ctypes.byref(cache.c), _stream(stream)), "lsa_shard_build_buckets")
+    return cache
+
+
+def shard_candidates(Q: torch.Tensor, t0: int, W_q: torch.Tensor, cache: Cache, p0: int, cfg: Config,
+                     rec=None, rec_n=None, ws=None, stream=None):
+    """lsa_shard_candidates: the shard's own fill as records.  Returns (rec
+    int32 [nq, hkv, cap, 4] -- each record's 16 bytes: id, taken, fp64
+    score --, rec_n int32 [nq, hkv])."""
+    _spec(Q, "Q", BF16, (None, None, 128))
+    _spec(W_q, "W_q", F32, W_SHAPE)
+    nq, hq, _ = Q.shape
+    cap = shard_cand_cap(cfg)
+    _spec(rec, "rec", I32, (nq, cache.hkv, cap, 4))
+    _spec(rec_n, "rec_n", I32, (nq, cache.hkv))
+    _need_cuda(Q, W_q, rec, rec_n, ws)
+    if rec is None:
+        rec = torch.empty((nq, cache.hkv, cap, 4), dtype=I32, device=Q.device)
+    if rec_n is None:
+        rec_n = torch.empty((nq, cache.hkv), dtype=I32, device=Q.device)
+    need = select_workspace_bytes(cfg, nq, hq, cache)
+    if ws is None or ws.numel() < need:
+        ws = torch.empty(max(need, 1), dtype=torch.uint8, device=Q.device)
+    check(lib().lsa_shard_candidates(_ptr(Q), t0, nq, hq, _ptr(W_q), ctypes.byref(cache.c), p0,
+                                     ctypes.byref(cfg.c()), _ptr(rec), _ptr(rec_n), _ptr(ws), ws.numel(),
+                                     _stream(stream)), "lsa_shard_candidates")
+    return rec, rec_n
+
+
+def shard_merge(rec_all: torch.Tensor, rec_n_all: torch.Tensor, rank: int, t0: int, cache: Cache, p0: int,
+                cfg: Config, idx=None, stream=None) -> torch.Tensor:
+    """lsa_shard_merge: shard `rank`'s part of the index rows [nq, hkv, S+k+W]
+    from every shard's records (rec_all [world, nq, hkv, cap, 4], rec_n_all
+    [world, nq, hkv])."""
+    _spec(rec_all, "rec_all", I32, (None, None, cache.hkv, shard_cand_cap(cfg), 4))
+    world, nq = int(rec_all.shape[0]), int(rec_all.shape[1])
+    _spec(rec_n_all, "rec_n_all", I32, (world, nq, cache.hkv))
+    _spec(idx, "idx", I32, (nq, cache.hkv, cfg.row))
+    _need_cuda(rec_all, rec_n_all, idx)
+    if idx is None:
+        idx = torch.empty((nq, cache.hkv, cfg.row), dtype=I32, device=rec_all.device)
+    check(lib().lsa_shard_merge(_ptr(rec_all), _ptr(rec_n_all), world, rank, t0, nq, ctypes.byref(cache.c), p0,
+                                ctypes.byref(cfg.c()), _ptr(idx), _stream(stream)), "lsa_shard_merge")
+    return idx
+
+
+def sparse_attn_partial(Q, K, V, idx, p0: int, O_part=None, lse=None, stream=None):
+    """lsa_sparse_attn_partial: (O_part fp32 [nq, hq, 128], lse fp32 [nq, hq])
+    over a shard's entries (global positions p0 .. p0 + K.shape[0] - 1)."""
+    _spec(Q, "Q", BF16, (None, None, 128))
+    _spec(K, "K", BF16, (None, None, 128))
+    _spec(V, "V", BF16, tuple(K.shape))
+    nq, hq, _ = Q.shape
+    hkv = K.shape[1]
+    _spec(idx, "idx", I32, (nq, hkv, None))
+    _spec(O_part, "O_part", F32, (nq, hq, 128))
+    _spec(lse, "lse", F32, (nq, hq))
+    _need_cuda(Q, K, V, idx, O_part, lse)
+    if O_part is None:
+        O_part = torch.empty((nq, hq, 128), dtype=F32, device=Q.device)
+    if lse is None:
+        lse = torch.empty((nq, hq), dtype=F32, device=Q.device)
+    check(lib().lsa_sparse_attn_partial(_ptr(Q), _ptr(K), _ptr(V), _ptr(idx), nq, hq, hkv, idx.shape[2], p0,
+                                        K.shape[0], _ptr(O_part), _ptr(lse), _stream(stream)),
+          "lsa_sparse_attn_partial")
+    return O_part, lse
+
+
+def lse_combine(O_parts, lse_parts, O=None, stream=None) -> torch.Tensor:
+    """lsa_lse_combine: bf16 O [nq, hq, 128] from every shard's (O_r, L_r)."""
+    _spec(O_parts, "O_parts", F32, (None, None, None, 128))
+    world, nq, hq, _ = O_parts.shape
+    _spec(lse_parts, "lse_parts", F32, (world, nq, hq))
+    _spec(O, "O", BF16, (nq, hq, 128))
+    _need_cuda(O_parts, lse_parts, O)
+    if O is None:
+        O = torch.empty((nq, hq, 128), dtype=BF16, device=O_parts.device)
+    check(lib().lsa_lse_combine(_ptr(O_parts), _ptr(lse_parts), world, nq, hq, _ptr(O), _stream(stream)),
+          "lsa_lse_combine")
+    return O
+
+
 class KernelTimer:
     """Context manager around lsa_timing_begin / lsa_timing_end; get(name)
     returns (total ms, launches) of one kernel recorded inside it."""

@@ -94,7 +94,7 @@ lsa_status launch_tree_update(const lsa_cache* c, lsa_tree* t, int64_t b0, int64
 size_t select_ws_bytes(const lsa_cfg* cfg, int64_t nq, int32_t hq, int32_t hkv, int64_t NB);
 lsa_status run_select(const uint16_t* Q, int64_t t0, int64_t nq, int32_t hq, const float* W_q,
                       const lsa_cache* c, const lsa_tree* tree, const lsa_cfg* cfg, int32_t* idx,
-                      uint16_t* Y_out, void* ws, size_t ws_bytes, cudaStream_t st);
+                      uint16_t* Y_out, void* ws, size_t ws_bytes, cudaStream_t st, const ShardOut* so);
 lsa_status launch_attn(const uint16_t* Q, const uint16_t* K, const uint16_t* V, const int32_t* idx,
                        int64_t nq, int32_t hq, int32_t hkv, int32_t n_idx, int64_t T, uint16_t* O,
                        cudaStream_t st, int64_t kv_q_stride, int split, int32_t n_use, const float* Ow,
@@ -328,7 +328,7 @@ lsa_status lsa_select(const uint16_t* Q, int64_t t0, int64_t nq, int32_t hq, con
             return set_error(LSA_EINVAL, "lsa_select: tree layout does not match the cache");
     }
     if (!ws && ws_bytes > 0) return set_error(LSA_EINVAL, "lsa_select: ws is NULL");
-    return run_select(Q, t0, nq, hq, W_q, cache, tree, cfg, idx, Y_out, ws, ws_bytes, (cudaStream_t)stream);
+    return run_select(Q, t0, nq, hq, W_q, cache, tree, cfg, idx, Y_out, ws, ws_bytes, (cudaStream_t)stream, nullptr);
 }
 
 lsa_status lsa_sparse_attn(const uint16_t* Q, const uint16_t* K, const uint16_t* V, const int32_t* idx,

@@ -46,6 +46,9 @@ struct AttnArgs {
     int64_t shared_len;   // ... positions below it are read there; 0 = none
     uint16_t* O;
     float scale_log2;
+    int64_t pos0;         // index entries are positions pos0 .. pos0 + T - 1 (K/V row p - pos0)
+    float* Opart;         // optional (SPLIT == 1, Ow == NULL): normalised fp32 O [nq, hq, 128] ...
+    float* lse_out;       // ... and the base-2 log-sum-exp of the scaled scores [nq, hq], instead of O
 };
 
 __device__ __forceinline__ uint32_t swz(int row, int chunk) {
@@ -93,9 +96,14 @@ __global__ void __launch_bounds__(32 * (SPLIT == 1 ? kAttnWarps : SPLIT), SPLIT 
     auto tile_pos = [&](int tile) -> int {
         const int e = tile * kTileKeys + (lane & 15);
         int p = (tile < ntiles && e < a.n_use) ? __ldg(list + e) : -1;
-        if (p >= a.T) {
-            raise_device_error(kErrIndexRange);
-            p = -1;
+        if (p >= 0) {
+            const int64_t pl = (int64_t)p - a.pos0;
+            if (pl < 0 || pl >= a.T) {
+                raise_device_error(kErrIndexRange);
+                p = -1;
+            } else {
+                p = (int)pl;
+            }
         }
         return p;
     };
@@ -259,6 +267,31 @@ __global__ void __launch_bounds__(32 * (SPLIT == 1 ? kAttnWarps : SPLIT), SPLIT 
             const __nv_bfloat16 ob = __float2bfloat16_rn(out);
             a.O[(r0 + hh) * kD + d] = *reinterpret_cast<const uint16_t*>(&ob);
         }
+    } else if (SPLIT == 1 && a.Opart != nullptr) {
+        // partial attention of a shard: normalised fp32 O and the base-2
+        // log-sum-exp of each head (-inf, with O = 0, for an empty list)
+        const float inv0 = l_run[0] > 0.f ? 1.f / l_run[0] : 0.f;
+        const float inv1 = l_run[1] > 0.f ? 1.f / l_run[1] : 0.f;
+        float* op = reinterpret_cast<float*>(wbuf);  // [8][128]
+#pragma unroll
+        for (int mt = 0; mt < 8; ++mt) {
+            const int d0 = mt * 16 + gq;
+            op[(2 * tq) * kD + d0] = o[mt][0] * inv0;
+            op[(2 * tq + 1) * kD + d0] = o[mt][1] * inv1;
+            op[(2 * tq) * kD + d0 + 8] = o[mt][2] * inv0;
+            op[(2 * tq + 1) * kD + d0 + 8] = o[mt][3] * inv1;
+        }
+        const int64_t r0 = q * a.hq + g * G;
+        if (gq == 0) {
+            if (2 * tq < G)
+                a.lse_out[r0 + 2 * tq] = l_run[0] > 0.f ? m_run[0] + log2f(l_run[0]) : -CUDART_INF_F;
+            if (2 * tq + 1 < G)
+                a.lse_out[r0 + 2 * tq + 1] = l_run[1] > 0.f ? m_run[1] + log2f(l_run[1]) : -CUDART_INF_F;
+        }
+        __syncwarp();
+        float* orow = a.Opart + r0 * (int64_t)kD;
+        for (int c = lane; c < G * kD / 4; c += 32)
+            reinterpret_cast<float4*>(orow)[c] = reinterpret_cast<const float4*>(op)[c];
     } else if constexpr (SPLIT == 1) {
         // normalise and stage O (heads x dims, bf16) for a coalesced store
         const float inv0 = l_run[0] > 0.f ? 1.f / l_run[0] : 0.f;
@@ -315,6 +348,28 @@ __global__ void __launch_bounds__(32 * (SPLIT == 1 ? kAttnWarps : SPLIT), SPLIT 
             a.O[(q * a.hq + g * G + hh) * (int64_t)kD + d] = *reinterpret_cast<const uint16_t*>(&ob);
         }
     }
+}
+
+// Partial attention of one sequence shard: entries are positions p0 ..
+// p0 + n_keys - 1 of K/V rows 0 .. n_keys - 1; writes the normalised fp32 O
+// and base-2 log-sum-exp per (query, head).
+lsa_status launch_attn_partial(const uint16_t* Q, const uint16_t* K, const uint16_t* V, const int32_t* idx,
+                               int64_t nq, int32_t hq, int32_t hkv, int32_t n_idx, int64_t p0, int64_t n_keys,
+                               float* Opart, float* lse, cudaStream_t st) {
+    if (nq <= 0) return LSA_OK;
+    AttnArgs a{};
+    a.Q = Q; a.K = K; a.V = V; a.idx = idx; a.nq = nq; a.hq = hq; a.hkv = hkv; a.n_idx = n_idx;
+    a.n_use = n_idx; a.T = n_keys; a.pos0 = p0; a.kv_q_stride = 0;
+    a.Opart = Opart; a.lse_out = lse;
+    a.scale_log2 = 1.4426950408889634f / sqrtf((float)kD);
+    const int64_t rows = nq * hkv;
+    const size_t smem = (size_t)kAttnWarps * kWarpBytes;
+    cudaFuncSetAttribute(attn_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    {
+        KTime kt_("attn_kernel", st);
+        attn_kernel<1><<<(unsigned)ceil_div<int64_t>(rows, kAttnWarps), 32 * kAttnWarps, smem, st>>>(a);
+    }
+    return check_launch("attn_kernel(partial)");
 }
 
 // n_use < 0: every entry of each list; Ow / lse: optional partial state of

@@ -500,6 +500,15 @@ flat_cand_kernel(const __grid_constant__ CUtensorMap tmF, PassArgs a) {
 constexpr int kResWarps = 4;
 constexpr int kBandCap = 128;  // buckets ranked on exact scores per row
 
+// One record of a shard's local fill (sequence-sharded selection): a bucket
+// the shard's own fill of k keys took, its global id, the keys it took and
+// its exact fp64 score.
+struct ShardRec {
+    int32_t bucket;
+    int32_t taken;
+    double score;
+};
+
 struct ResolveArgs {
     const int4* meta;        // [hkv, NB] (minlr, maxpos, cnt_lr, packed member units)
     const uint16_t* cent;
@@ -514,6 +523,12 @@ struct ResolveArgs {
     int32_t* ovf_rows;
     int32_t* ovf_count;
     int32_t ovf_cap;
+    // candidate-record mode (rec != NULL): no index rows; per row the taken
+    // buckets as records [rows, rec_cap] in ascending id, ids offset by id_base
+    ShardRec* rec;
+    int32_t* rec_n;
+    int32_t rec_cap;
+    int64_t id_base;
 };
 
 // meta[h * NB + b] = (minlr, maxpos, cnt_lr, units) of bucket b < NB: one 16-byte
@@ -705,6 +720,9 @@ __device__ __forceinline__ float warp_maxf(float v) {
     return v;
 }
 
+// CANDS: write the row's taken buckets as records (ascending id, exact
+// scores) instead of its index row.
+template <bool CANDS>
 __global__ void __launch_bounds__(32 * kResWarps, 3) flat_resolve_kernel(ResolveArgs a) {
     extern __shared__ __align__(16) uint8_t rsm[];
     const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
@@ -717,23 +735,29 @@ __global__ void __launch_bounds__(32 * kResWarps, 3) flat_resolve_kernel(Resolve
     const int64_t lim = t - a.W;
     int32_t* out = a.idx + row * (int64_t)(a.S + a.k + a.W);
 
-    // sinks and window (16-byte stores when the row layout keeps them aligned)
-    for (int i = lane; i < a.S; i += 32) out[i] = (i <= t) ? i : -1;
-    const int64_t w0 = max((int64_t)a.S, t - a.W + 1);
-    const int nw = t >= a.S ? (int)(t - w0 + 1) : 0;
-    int32_t* wout = out + a.S + a.k;
-    if ((((uintptr_t)wout) & 15u) == 0u && (a.W & 3) == 0) {
-        for (int i4 = lane; i4 < a.W / 4; i4 += 32) {
-            const int i = 4 * i4;
-            reinterpret_cast<int4*>(wout)[i4] =
-                make_int4(i < nw ? (int)w0 + i : -1, i + 1 < nw ? (int)w0 + i + 1 : -1,
-                          i + 2 < nw ? (int)w0 + i + 2 : -1, i + 3 < nw ? (int)w0 + i + 3 : -1);
+    if constexpr (!CANDS) {
+        // sinks and window (16-byte stores when the row layout keeps them aligned)
+        for (int i = lane; i < a.S; i += 32) out[i] = (i <= t) ? i : -1;
+        const int64_t w0 = max((int64_t)a.S, t - a.W + 1);
+        const int nw = t >= a.S ? (int)(t - w0 + 1) : 0;
+        int32_t* wout = out + a.S + a.k;
+        if ((((uintptr_t)wout) & 15u) == 0u && (a.W & 3) == 0) {
+            for (int i4 = lane; i4 < a.W / 4; i4 += 32) {
+                const int i = 4 * i4;
+                reinterpret_cast<int4*>(wout)[i4] =
+                    make_int4(i < nw ? (int)w0 + i : -1, i + 1 < nw ? (int)w0 + i + 1 : -1,
+                              i + 2 < nw ? (int)w0 + i + 2 : -1, i + 3 < nw ? (int)w0 + i + 3 : -1);
+            }
+        } else {
+            for (int i = lane; i < a.W; i += 32) wout[i] = i < nw ? (int32_t)(w0 + i) : -1;
         }
-    } else {
-        for (int i = lane; i < a.W; i += 32) wout[i] = i < nw ? (int32_t)(w0 + i) : -1;
     }
     if (lim < a.S) {
-        for (int i = lane; i < a.k; i += 32) out[a.S + i] = -1;
+        if constexpr (CANDS) {
+            if (lane == 0) a.rec_n[row] = 0;
+        } else {
+            for (int i = lane; i < a.k; i += 32) out[a.S + i] = -1;
+        }
         return;
     }
     const int n = a.cand_n[row];
@@ -921,6 +945,34 @@ __global__ void __launch_bounds__(32 * kResWarps, 3) flat_resolve_kernel(Resolve
         if (lane == 0) push_fallback(a, row);
         return;
     }
+    if constexpr (CANDS) {
+        // records of the taken buckets, ascending id, with their exact scores
+        const int ng = a.agg ? a.G : 1;
+        const uint16_t* ysrc = a.agg ? a.Y + (q * (int64_t)a.hkv * a.G + (int64_t)h * a.G) * kDL
+                                     : a.Y + row * kDL;
+        __syncwarp();
+        for (int i = lane; i < ng * kDL; i += 32) sw.ylat[i] = ysrc[i];
+        __syncwarp();
+        ShardRec* rec = a.rec + row * (int64_t)a.rec_cap;
+        int nrec = 0;
+        for (int base = 0; base < m; base += 32) {
+            const int i = base + lane;
+            const int tk = i < m ? sw.w[i] : 0;
+            const unsigned bal = __ballot_sync(0xffffffffu, tk > 0);
+            const int pos = nrec + __popc(bal & ((1u << lane) - 1u));
+            if (tk > 0 && pos < a.rec_cap) {
+                const int col = sw.cs[i].x;
+                rec[pos] = ShardRec{(int32_t)(a.id_base + col), tk,
+                                    exact_row(sw.ylat, ng, a.cent + (hb0 + col) * kDL)};
+            }
+            nrec += __popc(bal);
+        }
+        if (lane == 0) {
+            a.rec_n[row] = min(nrec, a.rec_cap);
+            if (nrec > a.rec_cap) raise_device_error(kErrSelectOverflow);
+        }
+        return;
+    }
     // emit keys in ascending bucket id (candidates are already in that order)
     int run = 0;
     for (int base = 0; base < m; base += 32) {
@@ -987,11 +1039,12 @@ lsa_status launch_flat(const PassArgs& pa, const ResolveArgs& ra, const CUtensor
     }
     if ((s = check_launch("flat_cand_kernel")) != LSA_OK) return s;
     const size_t smem_r = sizeof(ResWarp) * kResWarps;
-    cudaFuncSetAttribute(flat_resolve_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_r);
+    auto kr = ra.rec ? flat_resolve_kernel<true> : flat_resolve_kernel<false>;
+    cudaFuncSetAttribute(kr, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_r);
     const int64_t rows = pa.nqc * pa.hkv;
     {
         KTime kt_("flat_resolve_kernel", st);
-        flat_resolve_kernel<<<(unsigned)ceil_div<int64_t>(rows, kResWarps), 32 * kResWarps, smem_r, st>>>(ra);
+        kr<<<(unsigned)ceil_div<int64_t>(rows, kResWarps), 32 * kResWarps, smem_r, st>>>(ra);
     }
     return check_launch("flat_resolve_kernel");
 }

@@ -10,3 +10,4 @@
 #include "lsa_pca.cu"
 #include "lsa_probe.cu"
 #include "lsa_bwd.cu"
+#include "lsa_shard.cu"

@@ -79,6 +79,11 @@ struct SelectArgs {
     // each request has its own position
     int32_t decode;
     int64_t pos[LSA_MAX_BATCH];
+    // candidate-record mode of the flat fallback (sequence-sharded selection)
+    ShardRec* rec;
+    int32_t* rec_n;
+    int32_t rec_cap;
+    int64_t id_base;
 };
 
 __device__ __forceinline__ unsigned long long order_key(double s) {
@@ -627,8 +632,41 @@ lsa_status launch_tree_select(const SelectArgs& a, int64_t nrows, cudaStream_t s
     return check_launch("tree_warp_kernel");
 }
 
+// Records (ascending id) of the buckets of [0, ncol) with taken count tk(b) >
+// 0 and exact score sc(b), for the candidate-record mode.
+template <typename TkOf, typename ScOf>
+__device__ void emit_records(const SelectArgs& a, int64_t row, int64_t ncol, TkOf tkof, ScOf scof,
+                             SelShared& sh) {
+    ShardRec* rec = a.rec + row * (int64_t)a.rec_cap;
+    int64_t base = 0;
+    constexpr int per = 8;
+    for (int64_t c0 = 0; c0 < ncol; c0 += (int64_t)per * kSelThreads) {
+        const int64_t b0 = c0 + (int64_t)threadIdx.x * per;
+        int mine = 0;
+#pragma unroll
+        for (int i = 0; i < per; ++i) mine += (b0 + i < ncol && tkof(b0 + i) > 0) ? 1 : 0;
+        int tot;
+        int o = block_exscan(mine, &tot, sh.sh4);
+#pragma unroll
+        for (int i = 0; i < per; ++i) {
+            const int64_t b = b0 + i;
+            if (b < ncol && tkof(b) > 0) {
+                if (base + o < a.rec_cap) rec[base + o] = ShardRec{(int32_t)(a.id_base + b), tkof(b), scof(b)};
+                ++o;
+            }
+        }
+        base += tot;
+    }
+    if (threadIdx.x == 0) {
+        a.rec_n[row] = (int32_t)min(base, (int64_t)a.rec_cap);
+        if (base > a.rec_cap) raise_device_error(kErrSelectOverflow);
+    }
+}
+
 // Rows whose candidate band overflowed: exact scores of every eligible
-// bucket in a global slot (one per CTA), then the same radix fill.
+// bucket in a global slot (one per CTA), then the same radix fill.  CANDS:
+// the taken buckets as records instead of the index row.
+template <bool CANDS>
 __global__ void __launch_bounds__(kSelThreads) select_fallback_kernel(SelectArgs a) {
     __shared__ SelShared sh;
     const int tid = threadIdx.x;
@@ -661,7 +699,11 @@ __global__ void __launch_bounds__(kSelThreads) select_fallback_kernel(SelectArgs
                 ncol, a.k, [&](int64_t i) { return fs[i]; }, [&](int64_t i) { return (int)fw[i]; },
                 [&](int64_t i, int tk) { fw[i] = tk; }, sh);
         __syncthreads();
-        emit_range(a, r, ncol, [&](int64_t b) -> int { return fw[b]; }, sh);
+        if constexpr (CANDS)
+            emit_records(a, row, ncol, [&](int64_t b) -> int { return fw[b]; },
+                         [&](int64_t b) -> double { return fs[b]; }, sh);
+        else
+            emit_range(a, r, ncol, [&](int64_t b) -> int { return fw[b]; }, sh);
     }
 }
 
@@ -759,9 +801,18 @@ static int lstar_of(const lsa_cfg* cfg) {
     return l;
 }
 
+// Candidate-record output of a flat selection (sequence-sharded selection):
+// per (query, kv-head) row, the buckets its own fill of k keys took.
+struct ShardOut {
+    ShardRec* rec;      // [nq, hkv, cap]
+    int32_t* rec_n;     // [nq, hkv]
+    int32_t cap;
+    int64_t id_base;    // added to local bucket ids
+};
+
 lsa_status run_select(const uint16_t* Q, int64_t t0, int64_t nq, int32_t hq, const float* W_q,
                       const lsa_cache* c, const lsa_tree* tree, const lsa_cfg* cfg, int32_t* idx,
-                      uint16_t* Y_out, void* ws, size_t ws_bytes, cudaStream_t st) {
+                      uint16_t* Y_out, void* ws, size_t ws_bytes, cudaStream_t st, const ShardOut* so) {
     const int32_t hkv = c->hkv;
     const int64_t NU = ceil_div<int64_t>(c->n_tokens, kPool);
     const int64_t NB = ceil_div<int64_t>(NU, kUnitsPerBlock) * kBucketsPerBlock;
@@ -785,6 +836,8 @@ lsa_status run_select(const uint16_t* Q, int64_t t0, int64_t nq, int32_t hq, con
     a.ld = p.ld;
     a.ovf_rows = w.ovf_rows; a.ovf_count = w.ovf_count; a.ovf_cap = (int32_t)(p.chunk * hkv);
     a.fb_score = w.fb_score; a.fb_w = w.fb_w;
+    if (so && cfg->mode != 0) return set_error(LSA_EUNSUPPORTED, "candidate records: flat search only");
+    if (so) { a.rec_cap = so->cap; a.id_base = so->id_base; }
 
     CUtensorMap tmF, tmS;
     if (cfg->mode == 0) {
@@ -800,7 +853,8 @@ lsa_status run_select(const uint16_t* Q, int64_t t0, int64_t nq, int32_t hq, con
         uint16_t* Y = Y_out ? Y_out + c0 * p.hy * kDL : w.Y;
         lsa_status s = launch_query_latent(Q + c0 * hq * kD, nqc, hq, hkv, W_q, cfg->agg, Y, st);
         if (s != LSA_OK) return s;
-        a.Y = Y; a.nqc = nqc; a.t_first = t0 + c0; a.idx = idx + c0 * hkv * row_len;
+        a.Y = Y; a.nqc = nqc; a.t_first = t0 + c0; a.idx = idx ? idx + c0 * hkv * row_len : nullptr;
+        if (so) { a.rec = so->rec + c0 * hkv * so->cap; a.rec_n = so->rec_n + c0 * hkv; }
         if (cfg->mode == 1) {
             if ((s = launch_tree_select(a, nqc * hkv, st)) != LSA_OK) return s;
             continue;
@@ -819,10 +873,12 @@ lsa_status run_select(const uint16_t* Q, int64_t t0, int64_t nq, int32_t hq, con
         ra.W = cfg->window; ra.Y = Y; ra.nqc = nqc; ra.t_first = t0 + c0; ra.tau = w.tau;
         ra.cand = w.cand; ra.cand_n = w.cand_n; ra.idx = a.idx;
         ra.ovf_rows = w.ovf_rows; ra.ovf_count = w.ovf_count; ra.ovf_cap = a.ovf_cap;
+        ra.rec = a.rec; ra.rec_n = a.rec_n; ra.rec_cap = a.rec_cap; ra.id_base = a.id_base;
         if ((s = launch_flat(pa, ra, tmF, tmS, st)) != LSA_OK) return s;
         {
             KTime kt_("select_fallback_kernel", st);
-            select_fallback_kernel<<<(unsigned)p.fb_slots, kSelThreads, 0, st>>>(a);
+            if (so) select_fallback_kernel<true><<<(unsigned)p.fb_slots, kSelThreads, 0, st>>>(a);
+            else select_fallback_kernel<false><<<(unsigned)p.fb_slots, kSelThreads, 0, st>>>(a);
         }
         if ((s = check_launch("select_fallback_kernel")) != LSA_OK) return s;
     }

@@ -489,6 +489,98 @@ lsa_status lsa_attn_backward(const uint16_t* Q, const uint16_t* K, const uint16_
                              int64_t nq, int32_t hq, int32_t hkv, int32_t n_idx, int64_t T,
                              float* dQ, float* dK, float* dV, void* stream);
 
+/* ------------------------------------------------- sequence-sharded layer */
+
+/*
+ * The layer split over the GPUs of a job by sequence position, as the pages'
+ * deployments split the context (news page "开源内容": DCP8 / CP8 context
+ * parallelism).  Shard r of a job holds the keys of positions [p0, p1): whole
+ * 512-key blocks (p0 a multiple of 512; the last shard may end ragged), its
+ * K/V rows 0 .. p1 - p0 - 1 and the bucket cache of those keys (positions
+ * local to the shard).  Every shard sees every query position.  Flat search
+ * only.  Per chunk of queries [t0, t0 + nq):
+ *   1. lsa_shard_candidates on every shard;
+ *   2. the caller all-gathers the records and counts (rank order);
+ *   3. lsa_shard_merge on every shard -> its part of every index row;
+ *   4. lsa_sparse_attn_partial on every shard -> (O_r, L_r);
+ *   5. the caller all-gathers the partials; lsa_lse_combine -> O.
+ * The union over shards of the index rows' valid entries equals lsa_select's
+ * row for the whole context (sinks in the first shard, long-range keys in
+ * ascending bucket id shard by shard, the window in position order), and O
+ * is the attention over that union.
+ */
+
+/* Records per (query, kv-head) row of a candidate list: k / 4 + 4 (every
+ * bucket a fill takes, except at most the one holding the window's edge, a
+ * sink unit or the ragged last unit, holds at least one whole 4-key unit of
+ * eligible keys).  0 if cfg is invalid. */
+int32_t lsa_shard_cand_cap(const lsa_cfg* cfg);
+
+/*
+ * lsa_shard_build_buckets -- lsa_build_buckets over a shard's n keys K
+ * [n, hkv, d_head] (positions p0 .. p0 + n - 1): sinks count only in the
+ * first shard (p0 = 0).  Errors as lsa_build_buckets; LSA_EINVAL if p0 is
+ * not a multiple of 512; LSA_EUNSUPPORTED for sinks > 512.
+ */
+lsa_status lsa_shard_build_buckets(const uint16_t* K, int64_t n, int32_t hkv, const float* W_k,
+                                   const lsa_cfg* cfg, int64_t p0, lsa_cache* cache, void* stream);
+
+/*
+ * lsa_shard_candidates -- the shard's own flat fill [essay ch. 3] of k keys
+ * for query positions t0 .. t0 + nq - 1 (global), over its cache built by
+ * lsa_shard_build_buckets: per (query, kv-head) row the buckets that fill
+ * takes, as 16-byte records {int32 global bucket id (64 p0 / 512 + local),
+ * int32 keys taken, double exact fp64 score}, in ascending id, into rec
+ * [nq, hkv, lsa_shard_cand_cap(cfg)] (device, 16-byte aligned); rec_n
+ * [nq, hkv] int32 the counts.  Q [nq, hq, d_head] bf16 (the chunk's rows),
+ * W_q as lsa_select; ws / ws_bytes >= lsa_select_workspace_bytes(cfg, nq,
+ * hq, cache).  The global fill takes a bucket only if its shard's own fill
+ * does, and at most the keys that one takes, so these records carry every
+ * decision of the global fill.  LSA_EUNSUPPORTED for tree mode.
+ */
+lsa_status lsa_shard_candidates(const uint16_t* Q, int64_t t0, int64_t nq, int32_t hq,
+                                const float* W_q, const lsa_cache* cache, int64_t p0,
+                                const lsa_cfg* cfg, void* rec, int32_t* rec_n, void* ws,
+                                size_t ws_bytes, void* stream);
+
+/*
+ * lsa_shard_merge -- the global fill of k keys over every shard's records
+ * (rec_all [world, nq, hkv, cap], rec_n_all [world, nq, hkv], in rank order,
+ * as an all-gather leaves them): weighted radix select on the exact scores,
+ * score desc, global bucket id asc, exactly k keys.  Writes shard `rank`'s
+ * part of each row into idx [nq, hkv, S + k + W] (global positions): the
+ * sinks (first shard only), the keys its buckets give in [S, t - W] in
+ * ascending bucket id (each bucket's lowest first), and the window
+ * positions [max(S, t - W + 1), t] inside [p0, p0 + n_tokens); every part
+ * packed at its segment's start, -1 after.  `cache` is the shard's own.
+ * LSA_EUNSUPPORTED if world * cap records do not fit shared memory.
+ */
+lsa_status lsa_shard_merge(const void* rec_all, const int32_t* rec_n_all, int32_t world,
+                           int32_t rank, int64_t t0, int64_t nq, const lsa_cache* cache,
+                           int64_t p0, const lsa_cfg* cfg, int32_t* idx, void* stream);
+
+/*
+ * lsa_sparse_attn_partial -- lsa_sparse_attn over a shard's part of the
+ * index rows: entries are global positions p0 .. p0 + n_keys - 1 of the K/V
+ * rows 0 .. n_keys - 1 given here (others raise the device error word and
+ * are skipped).  Writes the normalised fp32 O_part [nq, hq, d_head]
+ * (16-byte aligned) and lse [nq, hq] fp32, the base-2 log-sum-exp of the
+ * scores scaled by log2(e) / sqrt(d_head) (-inf and O = 0 for an empty row).
+ */
+lsa_status lsa_sparse_attn_partial(const uint16_t* Q, const uint16_t* K, const uint16_t* V,
+                                   const int32_t* idx, int64_t nq, int32_t hq, int32_t hkv,
+                                   int32_t n_idx, int64_t p0, int64_t n_keys, float* O_part,
+                                   float* lse, void* stream);
+
+/*
+ * lsa_lse_combine -- the shards' partial attentions merged into O [nq, hq,
+ * d_head] bf16: O = sum_r 2^(L_r - M) O_r / sum_r 2^(L_r - M), M = max_r L_r
+ * (fp32), from O_parts [world, nq, hq, d_head] and lse_parts [world, nq, hq]
+ * as lsa_sparse_attn_partial writes them.  Rows no shard attends give 0.
+ */
+lsa_status lsa_lse_combine(const float* O_parts, const float* lse_parts, int32_t world, int64_t nq,
+                           int32_t hq, uint16_t* O, void* stream);
+
 #ifdef __cplusplus
 }
 #endif
