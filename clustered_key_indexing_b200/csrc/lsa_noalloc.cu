@@ -60,18 +60,36 @@ extern "C" lsa_status lsa_select_noalloc(const uint16_t* Q, int64_t t0, int64_t 
                                          const float* W_q, const lsa_cache* cache,
                                          const lsa_tree* tree, const lsa_cfg* cfg, int32_t* idx,
                                          void* stream) {
-    // size check before anything touches the device
+    // size checks before anything touches the device.  Part of the flat
+    // search's scratch grows with the cache (about 1 KB per bucket slot and
+    // kv-head group of 8 heads), not with nq: if even one query does not fit,
+    // splitting the query range cannot help.
     const size_t need = lsa_select_workspace_bytes(cfg, nq, hq, cache);
     if (need == 0) {
         lsa_status s = lsa_cfg_check(cfg);
         if (s != LSA_OK) return s;
         return set_error(LSA_EINVAL, "lsa_select_noalloc: invalid cache or nq");
     }
-    if (need > kNoAllocScratchBytes)
+    if (need > kNoAllocScratchBytes) {
+        const size_t one = lsa_select_workspace_bytes(cfg, 1, hq, cache);
+        if (one > kNoAllocScratchBytes)
+            return set_error(LSA_ENOSPACE,
+                             "lsa_select_noalloc: the cache is too large for the built-in scratch: flat search "
+                             "over it needs %zu bytes even for one query, the scratch holds %zu (about 512K "
+                             "tokens at 8 kv-heads is the largest flat-mode cache; tree mode has no such limit)",
+                             one, kNoAllocScratchBytes);
         return set_error(LSA_ENOSPACE,
                          "lsa_select_noalloc: this call needs %zu scratch bytes; the built-in scratch holds "
                          "%zu (split the queries into smaller ranges)",
                          need, kNoAllocScratchBytes);
+    }
+    // the scratch address is the current device's: the stream must be one
+    // of that device's streams
+    int dev = 0, sdev = 0;
+    if (cudaGetDevice(&dev) == cudaSuccess && cudaStreamGetDevice((cudaStream_t)stream, &sdev) == cudaSuccess &&
+        sdev != dev)
+        return set_error(LSA_EINVAL, "lsa_select_noalloc: the stream belongs to device %d, the current device is %d",
+                         sdev, dev);
     void* ws = nullptr;
     lsa_status s = noalloc_scratch(&ws);
     if (s != LSA_OK) return s;

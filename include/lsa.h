@@ -378,7 +378,14 @@ lsa_status lsa_decode_step(lsa_decode* d, const uint16_t* q, const uint16_t* k,
  * this library reserves until the process exits.
  *   - A request whose lsa_select_workspace_bytes() exceeds that size is
  *     refused with LSA_ENOSPACE (split the query range into smaller calls;
- *     e.g. 512 queries fit at 131072 keys x 8 kv-heads).
+ *     e.g. 512 queries fit at 131072 keys x 8 kv-heads).  Flat search also
+ *     needs scratch that grows with the cache, about 1 KB per bucket slot
+ *     for 8 kv-heads, whatever nq: the largest flat-mode cache is about 512K
+ *     tokens at 8 kv-heads, and a larger one is refused with LSA_ENOSPACE
+ *     and a message saying so.  Tree mode's scratch does not grow with the
+ *     cache.
+ *   - `stream` must belong to the current device (the scratch address is
+ *     that device's); another device's stream gives LSA_EINVAL.
  *   - The first call on a device looks up the array's device address
  *     (cudaGetSymbolAddress, with that device current); make that first
  *     call before any stream capture.
