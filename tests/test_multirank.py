@@ -1,10 +1,13 @@
 """The multi-rank host logic of bench.py and the kv-head split on CPU ranks (gloo, 127.0.0.1).
 
-The LSA layer shards without a data-path collective (each rank runs its own
-layer or decode batch: weak scaling), so the only cross-rank steps are the
-timing reduction and the job throughput.  Checked here: every rank gets the
-slowest rank's time, the job rate counts every rank's units at that time,
-ranks draw distinct inputs, and the reference arm does no work off rank 0.
+The LSA layer shards without a data-path collective: each rank takes hkv / N
+kv-heads of the layer (decode: a slice of the requests), so the only
+cross-rank steps of the benchmark are the timing reduction and the job
+throughput.  Checked here: every rank gets the slowest rank's time, the job
+rate counts every rank's units at that time, ranks draw distinct inputs, the
+reference arm does no work off rank 0, the head and request ranges partition
+the layer, and a two-rank kv-head split (the oracle's arithmetic per rank)
+reproduces the whole layer's output.
 """
 import os
 import socket
