@@ -43,25 +43,29 @@ constexpr float kScoreErr = 1e-4f;   // bound on |fp32 score - exact score|
 // The flat pass runs on the 5th-generation tensor cores in two kernels per
 // chunk, both TMA -> shared memory -> tcgen05.mma (bf16 in, fp32 accumulate
 // in TMEM) -> tcgen05.ld, with one producer thread (warp 0), one MMA thread
-// (warp 1, which also owns the TMEM allocation) and epilogue warps that own
-// one latent row per thread (TMEM lane quarter = warp % 4):
+// (warp 1, which also owns the TMEM allocation) and sixteen epilogue warps
+// (TMEM lane quarter = warp % 4):
 //   flat_sample_kernel  256 rows (two M = 128 blocks) x 128 sampled centroids
-//       per tile; per-row histogram of the sampled scores -> tau;
+//       per tile, two epilogue threads per row, one per 64-column half of a
+//       tile; per-row histogram of the sampled scores (both threads of a row
+//       count into it) -> tau;
 //   flat_cand_kernel    512 rows (four blocks) x 64 centroids per tile, plus
 //       one K = 16 step that adds -tau to every row (A holds -tau in its first
 //       extra column, B a 1 there), so TMEM holds s - tau and a hit is a clear
-//       sign bit; hits are appended in ascending bucket id.  Each epilogue
-//       thread takes a whole tile row into registers with one TMEM load, and
-//       the buffer goes back to the MMA thread before the scan.  (Two blocks
-//       of 128 columns halve the operand bytes per score but leave half the
-//       epilogue warps, which then bound the kernel.)
+//       sign bit; hits are appended in ascending bucket id.  One epilogue
+//       thread per row takes a whole tile row into registers with one TMEM
+//       load, and the buffer goes back to the MMA thread before the scan.
+//       (Two blocks of 128 columns read a third fewer operand bytes per
+//       score; with a thread per 64-column half of a row and a per-tile
+//       exchange of hit counts between the two, they ran 14% slower.)
 constexpr uint32_t kTcABytes = 128 * kDL * 2;      // one M = 128 block of latents, 128-byte swizzle
 constexpr uint32_t kTcAxBytes = 128 * 16 * 2;      // extra K = 16 of a block, no swizzle
 constexpr int kHBins = 256;                        // sample histogram bins per row (16-bit counts)
 
 constexpr int kSmBlocks = 2, kSmCols = 128, kSmStages = 3;
 constexpr int kSmRows = 128 * kSmBlocks;
-constexpr int kSmThreads = 64 + kSmRows;
+constexpr int kSmEpi = 2 * kSmRows;                  // epilogue threads: two per row
+constexpr int kSmThreads = 64 + kSmEpi;
 constexpr uint32_t kSmBBytes = kSmCols * kDL * 2;
 constexpr uint32_t kSmHistBytes = kHBins / 2 * kSmRows * 4;  // [bin / 2][row] words, two counts each
 constexpr size_t kSmSmemBytes = 1024 + kSmBlocks * kTcABytes + kSmStages * kSmBBytes + kSmHistBytes + 256;
@@ -263,15 +267,16 @@ flat_sample_kernel(const __grid_constant__ CUtensorMap tmS, PassArgs a) {
     const int ntiles = (int)ceil_div<int64_t>(ceil_div<int64_t>(ncol_max, kSampleStride), kSmCols);
 
     if (tid == 0) {
-        bar.init(kSmRows);
+        bar.init(kSmEpi);
         *abort_flag = 0;
         fence_barrier_init();
     }
     if (warp == 1) tmem_alloc(smem_u32(tmem_slot), 512);
     for (int i = tid; i < kHBins / 2 * kSmRows; i += kSmThreads) hist[i] = 0u;
-    const int quarter = warp & 3, blk = (warp - 2) >> 2;
+    // epilogue warps 2 .. 17: TMEM lane quarter warp % 4, then column half, then block
+    const int quarter = warp & 3, half = ((warp - 2) >> 2) & 1, blk = (warp - 2) >> 3;
     const int r = blk * 128 + quarter * 32 + lane;  // epilogue row of this thread
-    if (warp >= 2) fill_a_row<G>(sA, a, q0, h, r);
+    if (warp >= 2 && half == 0) fill_a_row<G>(sA, a, q0, h, r);
     fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
@@ -284,7 +289,8 @@ flat_sample_kernel(const __grid_constant__ CUtensorMap tmS, PassArgs a) {
         if (lane == 0) tc_mma<kSmBlocks, kSmCols, kSmStages, false>(tmem, sA, sB, nullptr, nullptr, ntiles, bar, abort_flag);
     } else {
         const EpiRow e = epi_row<G>(a, q0, h, r);
-        const uint32_t trow = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(blk * kSmCols);
+        const uint32_t trow =
+            tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(blk * kSmCols + half * (kSmCols / 2));
         // R bounds |score| of the row: |s| <= |y| |c| < 1.01 |y| (|c| <= 1 + 2^-8)
         float n2 = 0.f;
         {
@@ -319,51 +325,49 @@ flat_sample_kernel(const __grid_constant__ CUtensorMap tmS, PassArgs a) {
         const float boff = -lo * bsc - 0.5f + 12582912.0f;
         const int ns_row = e.owner ? (e.ncol + kSampleStride - 1) / kSampleStride : 0;
 
-        uint32_t va[32], vb[32];
         // one count per sampled bucket (buckets hold 8 keys on average: a
-        // block's 512 keys in 64); 16-bit counts, two bins per word
+        // block's 512 keys in 64); 16-bit counts, two bins per word.  Bin 0
+        // is not counted: every valid sample lands in some bin, so its count
+        // is ns_row less the others
         for (int it = 0; it < ntiles; ++it) {
             const int b = it & 1;
             if (!__all_sync(0xffffffffu, mbar_wait(bar.tfull(b), (uint32_t)(it >> 1) & 1u, abort_flag))) break;
             tc_fence_after();
-            const uint32_t tb = trow + (uint32_t)(b * kSmBlocks * kSmCols);
-            auto chunk = [&](uint32_t (&v)[32], uint32_t (&vn)[32], int c) {
-                if (c + 1 < kSmCols / 32) tmem_ld32_async(tb + (uint32_t)((c + 1) * 32), vn);
-                group_max<G>(v);
-                const int nval = min(32, max(0, ns_row - (it * kSmCols + c * 32)));
+            uint32_t v[64];
+            tmem_ld64(trow + (uint32_t)(b * kSmBlocks * kSmCols), v);
+            tc_fence_before();
+            mbar_arrive(bar.tempty(b));
+#pragma unroll
+            for (int c = 0; c < 2; ++c) {
+                uint32_t(&vv)[32] = *reinterpret_cast<uint32_t(*)[32]>(v + 32 * c);
+                group_max<G>(vv);
+                const int nval = min(32, max(0, ns_row - (it * kSmCols + half * (kSmCols / 2) + c * 32)));
 #pragma unroll
                 for (int i = 0; i < 32; ++i) {
                     const int bin =
-                        min(kHBins - 1, max(0, __float_as_int(fmaf(__uint_as_float(v[i]), bsc, boff)) - 0x4B400000));
-                    if (i < nval) atomicAdd(&hist[(bin >> 1) * kSmRows + r], 1u << ((bin & 1) << 4));
+                        min(kHBins - 1, max(0, __float_as_int(fmaf(__uint_as_float(vv[i]), bsc, boff)) - 0x4B400000));
+                    if (i < nval && bin > 0) atomicAdd(&hist[(bin >> 1) * kSmRows + r], 1u << ((bin & 1) << 4));
                 }
-                if (c + 1 < kSmCols / 32) tmem_wait_ld(vn);
-            };
-            tmem_ld32_async(tb, va);
-            tmem_wait_ld(va);
-#pragma unroll 1
-            for (int c = 0; c < kSmCols / 32; c += 2) {
-                chunk(va, vb, c);
-                chunk(vb, va, c + 1);
             }
-            tc_fence_before();
-            mbar_arrive(bar.tempty(b));
         }
+        // both halves' counts are in before the row's tau is read off
+        asm volatile("bar.sync 1, %0;\n" ::"n"(kSmEpi) : "memory");
         // tau: lower edge of the bin where the sampled key estimate (8 keys
         // per bucket, every 8th bucket) from the top first reaches
         // kOversample * k, rounded down to bf16 (it enters the extra K step
         // of the candidate kernel); -inf if never (an upper-range row whose
         // target lies below 0 gets 0: bin 0 holds every score below 0)
         float tau = -CUDART_INF_F;
-        if (!take_all) {
+        if (!take_all && half == 0) {
             long long cum = 0;
             const long long need = ((long long)kOversample * a.k + 63) / 64;  // sampled buckets
-            for (int bn = kHBins - 1; bn >= 0; --bn) {
+            for (int bn = kHBins - 1; bn >= 1; --bn) {
                 cum += (hist[(bn >> 1) * kSmRows + r] >> ((bn & 1) << 4)) & 0xFFFFu;
                 if (cum >= need) { tau = lo + bn * ((R - lo) / kHBins); break; }
             }
+            if (tau == -CUDART_INF_F && ns_row >= need) tau = lo;  // reached in bin 0
         }
-        if (e.owner) a.tau[e.orow] = bf16_floor(tau);
+        if (e.owner && half == 0) a.tau[e.orow] = bf16_floor(tau);
     }
     tc_fence_before();
     __syncthreads();
