@@ -89,6 +89,27 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
         : "memory");
 }
 
+// 3-D tiled TMA load (coordinates innermost first); x must keep x * element
+// size a multiple of 16 bytes (every caller passes x = 0 or 64 for 16-bit
+// elements).
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, int32_t x, int32_t y, int32_t z,
+                                            uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3, %4}], [%5];\n" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(bar)
+        : "memory");
+}
+
+// Shared-memory matrix descriptor of an MN-major operand with the 128-byte
+// swizzle: each K index is one 128-byte row of 64 MN elements (16-byte chunk
+// c of row r at c ^ (r & 7)), 8-row groups `sbo` bytes apart along K, blocks
+// of 64 MN elements `lbo` bytes apart; the tile base must be 1024-byte aligned.
+__device__ __forceinline__ uint64_t sw128_mn_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+    return (uint64_t)((saddr >> 4) & 0x3FFF) | ((uint64_t)((lbo >> 4) & 0x3FFF) << 16) |
+           ((uint64_t)((sbo >> 4) & 0x3FFF) << 32) | ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
+}
+
 // Shared-memory matrix descriptor of a K-major operand stored as 128-byte
 // rows with the 128-byte swizzle (16-byte chunk c of row r at c ^ (r & 7)),
 // 8-row groups 1024 bytes apart; the tile base must be 1024-byte aligned.
@@ -112,6 +133,18 @@ __device__ __forceinline__ void umma_bf16(uint32_t dtmem, uint64_t adesc, uint64
         "{\n .reg .pred p;\n setp.ne.u32 p, %4, 0;\n"
         " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(dtmem),
         "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// D[tmem] (+)= A[tmem] * B[smem]^T, issued by one thread.  A is K-major in
+// tensor memory: row m in lane m, 32-bit column j holding K elements 2j (low
+// half) and 2j + 1 (high half); `atmem` addresses the column of this K step.
+__device__ __forceinline__ void umma_bf16_ts(uint32_t dtmem, uint32_t atmem, uint64_t bdesc, uint32_t idesc,
+                                             uint32_t accumulate) {
+    asm volatile(
+        "{\n .reg .pred p;\n setp.ne.u32 p, %4, 0;\n"
+        " tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n}\n" ::"r"(dtmem),
+        "r"(atmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
         : "memory");
 }
 
@@ -207,22 +240,72 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
     for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
 
-// Tensor map of a row-major [rows, 64] bf16 matrix (128-byte rows), box of
-// `box_rows` x 64, 128-byte swizzle; cuTensorMapEncodeTiled is taken from the
-// driver through the runtime, so the library does not link libcuda.
-static lsa_status make_rows64_map(CUtensorMap* map, const uint16_t* base, int64_t rows, int box_rows) {
-    using EncodeFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-    static EncodeFn encode = nullptr;
+// This thread's lane, 32 consecutive 32-bit columns from `taddr` on
+// (warp-collective; the warp writes lanes 32 * (warp % 4) .. + 31).
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+        "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};\n" ::"r"(taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
+        "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]),
+        "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]),
+        "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+        : "memory");
+}
+
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};\n" ::"r"(
+            taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
+        "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+        : "memory");
+}
+
+// Wait until this thread's tensor-memory stores have completed.
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;\n" ::: "memory"); }
+
+// cuTensorMapEncodeTiled, taken from the driver through the runtime (the
+// library does not link libcuda); nullptr if unavailable.
+using TensorMapEncodeFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                       const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                       CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+static TensorMapEncodeFn tensor_map_encoder() {
+    static TensorMapEncodeFn encode = nullptr;
     if (!encode) {
         void* fn = nullptr;
         cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess || !fn ||
-            q != cudaDriverEntryPointSuccess)
-            return set_error(LSA_ECUDA, "cuTensorMapEncodeTiled is not available");
-        encode = reinterpret_cast<EncodeFn>(fn);
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) == cudaSuccess && fn &&
+            q == cudaDriverEntryPointSuccess)
+            encode = reinterpret_cast<TensorMapEncodeFn>(fn);
     }
+    return encode;
+}
+
+// Tensor map of one kv-head's rows of K or V [T, hkv, 128] bf16: dimensions
+// (dim, kv-head, position), box of 64 dims x 1 head x `box_keys` positions,
+// 128-byte swizzle, so one box is a [box_keys, 64] tile of 128-byte rows.
+static lsa_status make_kv_map(CUtensorMap* map, const uint16_t* base, int64_t T, int32_t hkv, int box_keys) {
+    const TensorMapEncodeFn encode = tensor_map_encoder();
+    if (!encode) return set_error(LSA_ECUDA, "cuTensorMapEncodeTiled is not available");
+    if (T <= 0 || hkv <= 0 || ((uintptr_t)base & 15u) != 0)
+        return set_error(LSA_EINVAL, "tensor map: need T > 0, hkv > 0 and a 16-byte aligned base");
+    const cuuint64_t dims[3] = {(cuuint64_t)kD, (cuuint64_t)hkv, (cuuint64_t)T};
+    const cuuint64_t strides[2] = {(cuuint64_t)kD * 2, (cuuint64_t)hkv * kD * 2};
+    const cuuint32_t box[3] = {64, 1, (cuuint32_t)box_keys};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    const CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<uint16_t*>(base), dims, strides,
+                              box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return set_error(LSA_ECUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+    return LSA_OK;
+}
+
+// Tensor map of a row-major [rows, 64] bf16 matrix (128-byte rows), box of
+// `box_rows` x 64, 128-byte swizzle.
+static lsa_status make_rows64_map(CUtensorMap* map, const uint16_t* base, int64_t rows, int box_rows) {
+    const TensorMapEncodeFn encode = tensor_map_encoder();
+    if (!encode) return set_error(LSA_ECUDA, "cuTensorMapEncodeTiled is not available");
     if (rows <= 0 || ((uintptr_t)base & 15u) != 0)
         return set_error(LSA_EINVAL, "tensor map: need rows > 0 and a 16-byte aligned base");
     const cuuint64_t dims[2] = {(cuuint64_t)kDL, (cuuint64_t)rows};
@@ -239,18 +322,8 @@ static lsa_status make_rows64_map(CUtensorMap* map, const uint16_t* base, int64_
 // Tensor map of a row-major [rows, 64] byte matrix (FP8 centroids, 64-byte
 // rows), box of `box_rows` x 64 bytes, no swizzle.
 static lsa_status make_rows64_u8_map(CUtensorMap* map, const uint8_t* base, int64_t rows, int box_rows) {
-    using EncodeFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-    static EncodeFn encode = nullptr;
-    if (!encode) {
-        void* fn = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess || !fn ||
-            q != cudaDriverEntryPointSuccess)
-            return set_error(LSA_ECUDA, "cuTensorMapEncodeTiled is not available");
-        encode = reinterpret_cast<EncodeFn>(fn);
-    }
+    const TensorMapEncodeFn encode = tensor_map_encoder();
+    if (!encode) return set_error(LSA_ECUDA, "cuTensorMapEncodeTiled is not available");
     if (rows <= 0 || ((uintptr_t)base & 15u) != 0)
         return set_error(LSA_EINVAL, "tensor map: need rows > 0 and a 16-byte aligned base");
     const cuuint64_t dims[2] = {(cuuint64_t)kDL, (cuuint64_t)rows};

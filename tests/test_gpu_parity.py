@@ -330,3 +330,31 @@ def test_tree_exponent_spread_fallback(lsa, scale_q, scale_k):
     Y = oracle.query_latent(inp["Q"][tpos], Wq, 1, 0)
     oidx, _, _ = oracle.select(oc, Y, tpos, ocfg, tree=oracle.build_tree(oc), G=4)
     assert np.array_equal(idx.cpu().numpy()[tpos], oidx)
+
+
+def test_select_attn_band_with_growing_scores(lsa):
+    """Scores that grow along the window by far more than 2^8 per 64-key tile
+    move the band kernel's running max on every tile (its rescaling path);
+    the output still matches the oracle attention over the same index rows."""
+    T, hkv, G, t0, nq = 2100, 1, 4, 1500, 300
+    rng = np.random.default_rng(11)
+    u = rng.standard_normal(128)
+    u /= np.linalg.norm(u)
+    pos = np.arange(T, dtype=np.float64)
+    K = synth.f32_to_bf16_bits(
+        (0.5 * pos)[:, None, None] * u[None, None, :] + 0.05 * rng.standard_normal((T, hkv, 128)))
+    V = synth.f32_to_bf16_bits(rng.standard_normal((T, hkv, 128)))
+    Q = synth.f32_to_bf16_bits(4.0 * u[None, None, :] + 0.05 * rng.standard_normal((nq, hkv * G, 128)))
+    inp = synth.layer_inputs("prefill-4k", T=T)
+    cfg = lsa.Config(k=64, sinks=4, window=1024)
+    dK, dV = to_dev_bf16(K), to_dev_bf16(V)
+    cache = lsa.Cache(hkv, T, cfg)
+    lsa.build_buckets(dK, to_dev(inp["Wk"]), cfg, cache)
+    dQ = to_dev_bf16(Q)
+    idx = lsa.select(dQ, t0, to_dev(inp["Wq"]), cache, cfg)
+    O = lsa.select_attn(dQ, dK, dV, idx, t0, cfg, T)
+    torch.cuda.synchronize()
+    lsa.check_device_error()
+    ref = oracle.attention(Q, K, V, idx.cpu().numpy())
+    mx, mean = _attn_err(O, ref)
+    assert mx <= ATOL_MAX and mean <= ATOL_MEAN, (mx, mean)
