@@ -326,9 +326,7 @@ flat_sample_kernel(const __grid_constant__ CUtensorMap tmS, PassArgs a) {
         const int ns_row = e.owner ? (e.ncol + kSampleStride - 1) / kSampleStride : 0;
 
         // one count per sampled bucket (buckets hold 8 keys on average: a
-        // block's 512 keys in 64); 16-bit counts, two bins per word.  Bin 0
-        // is not counted: every valid sample lands in some bin, so its count
-        // is ns_row less the others
+        // block's 512 keys in 64); 16-bit counts, two bins per word
         for (int it = 0; it < ntiles; ++it) {
             const int b = it & 1;
             if (!__all_sync(0xffffffffu, mbar_wait(bar.tfull(b), (uint32_t)(it >> 1) & 1u, abort_flag))) break;
@@ -346,7 +344,7 @@ flat_sample_kernel(const __grid_constant__ CUtensorMap tmS, PassArgs a) {
                 for (int i = 0; i < 32; ++i) {
                     const int bin =
                         min(kHBins - 1, max(0, __float_as_int(fmaf(__uint_as_float(vv[i]), bsc, boff)) - 0x4B400000));
-                    if (i < nval && bin > 0) atomicAdd(&hist[(bin >> 1) * kSmRows + r], 1u << ((bin & 1) << 4));
+                    if (i < nval) atomicAdd(&hist[(bin >> 1) * kSmRows + r], 1u << ((bin & 1) << 4));
                 }
             }
         }
@@ -361,11 +359,10 @@ flat_sample_kernel(const __grid_constant__ CUtensorMap tmS, PassArgs a) {
         if (!take_all && half == 0) {
             long long cum = 0;
             const long long need = ((long long)kOversample * a.k + 63) / 64;  // sampled buckets
-            for (int bn = kHBins - 1; bn >= 1; --bn) {
+            for (int bn = kHBins - 1; bn >= 0; --bn) {
                 cum += (hist[(bn >> 1) * kSmRows + r] >> ((bn & 1) << 4)) & 0xFFFFu;
                 if (cum >= need) { tau = lo + bn * ((R - lo) / kHBins); break; }
             }
-            if (tau == -CUDART_INF_F && ns_row >= need) tau = lo;  // reached in bin 0
         }
         if (e.owner && half == 0) a.tau[e.orow] = bf16_floor(tau);
     }
