@@ -49,18 +49,13 @@ METRIC = "LSA layer prefill tokens/s"
 UNIT = "tokens/s"
 
 # ncu DRAM bytes (read + write) per (query, kv-head) of the gather attention
-# kernel, averaged over the seven launches of one timed step of the workload
-# (the committed ncu summary of attn_kernel gives the command); reported as
+# kernel, summed over the 56 launches of one whole step of the workload (the
+# committed launch-list summary of the 1M line gives the command); reported as
 # `traffic` only while the kernel's source (the text from its template header
 # to its launcher, hashed) is the one that capture measured.
-ATTN_TRAFFIC = {"kernel_sha256_prefix": "d24e17fa489f0fb0", "bytes_per_query_kvhead": 19224.3,
-                "workload": "prefill-128k"}
+ATTN_TRAFFIC = {"kernel_sha256_prefix": "2e3df2e5bd8b2f99", "bytes_per_query_kvhead": 310348.7,
+                "workload": "prefill-1m"}
 
-
-# Peak of the L2-to-SM read path on this machine's B200s, from ncu's
-# l1tex__m_xbar2l1tex_read_bytes.sum.per_second (12.905 TB/s) and its
-# pct_of_peak_sustained_elapsed (37.04%) for the gather attention kernel.
-L2_TO_SM_PEAK_GBS = 12904.99 / 0.3703643
 
 
 def attn_kernel_hash():
