@@ -102,7 +102,7 @@ def workload_cfg(args):
     return c
 
 
-def config_json(args, c, world, chunk=None, split="none"):
+def config_json(args, c, world, split="none"):
     par = {"none": "1 GPU", "heads": f"kv-heads split over {world} GPUs ({c['hkv'] // world} each, no collective)",
            "replicas": f"replicas x{world} (one layer per GPU)"}[split]
     return {
@@ -110,7 +110,7 @@ def config_json(args, c, world, chunk=None, split="none"):
         "d_latent": c["dl"], "k": c["k"], "sinks": c["sinks"], "window": c["window"],
         "search": "flat" if c["mode"] == 0 else f"tree(beam={c['beam']})",
         "query_score": "group-mean" if c["agg"] == 0 else "max-over-heads (native)",
-        "query_chunk": chunk or args.chunk, "parallelism": par,
+        "parallelism": par,
         "l2": "no flush: per-step inputs (Q/K/V) are larger than L2",
         "inputs": "host-drawn (numpy PCG64)" if c["T"] <= 131072 else "device-drawn (torch Philox), same recipe",
     }
@@ -642,7 +642,7 @@ def run_lsa(args):
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": scaling,
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": config_json(args, c, world, P.chunk, P.split), "clocks": clk, "e2e": e2e,
+        "config": config_json(args, c, world, P.split), "query_chunk": P.chunk, "clocks": clk, "e2e": e2e,
         "gpu_launches": int(launches), "roofline": roofline, "roofline_scoring": roofline_scoring,
         "tree": tree_line, "kernels": kernels, "cpu_baseline": cpu,
         "stages_ms_per_step": stages, "select_fallback_rows_per_step": fallback_rows / args.steps,
