@@ -1,27 +1,26 @@
-// lsa_select.cu -- query scoring, long-range selection and index assembly of
-// the LSA path on sm_100a [essay "《卡片柜》——当注意力学会先查目录再翻书",
-// ch. 3 (flat search, sinks, window) and ch. 4 (tree beam search); ch. 5 for
-// the native max-over-heads score].
+// lsa_select.cu -- long-range selection and index assembly of the LSA path
+// on sm_100a [essay "《卡片柜》——当注意力学会先查目录再翻书", ch. 3 (flat
+// search, sinks, window) and ch. 4 (tree beam search); ch. 5 for the native
+// max-over-heads score].
 //
-// Flat search runs in three kernels per chunk of query positions:
-//   score_kernel    bf16 tensor-core contraction (mma.sync m16n8k16, fp32
-//                   accumulate) of query latents against centroid tiles;
-//   select_kernel   one CTA per (query, kv-head): weighted histogram of the
-//                   fp32 scores locates the k-th key's score bin, the band of
-//                   candidates at or above the bin below it is rescored
-//                   exactly in fp64, a weighted radix select on the exact
-//                   scores finds the cut (score desc, bucket id asc), and the
-//                   chosen buckets' keys are written in ascending bucket id;
-//   select_fallback for rows whose candidate band overflows shared memory:
-//                   exact scores of every eligible bucket in a global slot,
-//                   same radix select.
-// Tree search is a mode of select_kernel: beam descent over the node
-// centroids with exact scores, then the same fill over the final leaves.
+//   tree_warp_kernel        tree search, one warp per (query, kv-head): beam
+//                           descent over the node centroids with exact fp64
+//                           scores, then exact scores of the leaves below the
+//                           final beam and a weighted radix fill of k keys;
+//   select_fallback_kernel  the exact flat search for the rows the flat
+//                           resolve flags (band below tau, or a candidate
+//                           list that overflowed): exact scores of every
+//                           eligible bucket in a global slot, the same fill;
+//   run_select              the selection driver: query latents, then per
+//                           chunk of query positions the flat kernels of
+//                           lsa_flat.cuh (tcgen05 scores, candidates, resolve)
+//                           or the tree kernel, then the fallback.
+// The record modes of the resolve and fallback kernels write a shard's taken
+// buckets with their exact scores instead of index rows (sequence sharding).
 //
-// Exactness: the fp32 scores only steer which buckets are rescored.  Their
-// error is below 64 * 2^-23 * |y||c| < 1e-5; a histogram bin is 1.04e-3 wide,
-// so every bucket whose exact score can reach the cut lies in the two bins
-// kept, and the decision itself is taken on exact fp64 scores.
+// Exactness: every ranking decision is taken on exact fp64 scores (score
+// desc, bucket id asc); fp32 tensor-core scores only steer which buckets are
+// rescored (lsa_flat.cuh states the bound).
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -43,10 +42,7 @@ __host__ __device__ __forceinline__ int64_t flat_ncol(int64_t t, int32_t W, int6
 // ------------------------------------------------------------- selection
 
 constexpr int kSelThreads = 128;
-constexpr int kCap = 1024;      // candidates held in shared memory
-constexpr int kBins = 2048;     // fp32 score bins over [-1.0625, 1.0625)
-constexpr float kBinLo = -1.0625f;
-constexpr float kBinScale = 2048.0f / 2.125f;
+constexpr int kCap = 1024;      // candidates held in shared memory (fallback, decode resolve); decode keep slots per row chunk
 
 struct SelectArgs {
     const int32_t* offsets;
@@ -90,11 +86,6 @@ __device__ __forceinline__ unsigned long long order_key(double s) {
     s = s + 0.0;  // -0 -> +0
     const unsigned long long u = (unsigned long long)__double_as_longlong(s);
     return (u >> 63) ? ~u : (u | 0x8000000000000000ull);
-}
-
-__device__ __forceinline__ int score_bin(float s) {
-    int b = __float2int_rd((s - kBinLo) * kBinScale);
-    return b < 0 ? 0 : (b >= kBins ? kBins - 1 : b);
 }
 
 // Number of keys of bucket b (head h) in [S, lim].
@@ -158,9 +149,9 @@ __device__ __forceinline__ int block_exscan(int v, int* total, int* sh4) {
 
 struct SelShared {
     // 8-byte members first: every field below stays naturally aligned
-    unsigned long long hist[kBins];   // packed (count << 32 | weight)
     double csc[kCap];
     long long above;                  // radix select: weight strictly above the prefix
+    unsigned int hist[256];           // radix select: weight per digit
     int cid[kCap];
     int cw[kCap];
     int ctk[kCap];
@@ -175,7 +166,7 @@ struct SelShared {
 template <typename GetS, typename GetW, typename SetTk>
 __device__ void radix_fill(int64_t n, int k, GetS gs, GetW gw, SetTk st, SelShared& sh) {
     const int tid = threadIdx.x, lane = tid & 31;
-    unsigned int* h256 = reinterpret_cast<unsigned int*>(sh.hist);
+    unsigned int* h256 = sh.hist;
     unsigned long long prefix = 0;
     long long above = 0;
     for (int pass = 0; pass < 8; ++pass) {
