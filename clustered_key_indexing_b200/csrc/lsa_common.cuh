@@ -105,27 +105,6 @@ __device__ __forceinline__ double e4m3_to_f64(uint32_t c) {
     return (c & 0x80u) ? -v : v;
 }
 
-// Exact score of a bf16 latent and an FP8 centroid (values 2^-8 * e4m3):
-// every product of a bf16 and an e4m3 value is exact in fp64; ascending
-// index order, as for two bf16 latents.
-__device__ __forceinline__ double dot_bf16_fp8_exact(const uint16_t* __restrict__ y,
-                                                     const uint8_t* __restrict__ c) {
-    double s = 0.0;
-#pragma unroll 8
-    for (int i = 0; i < kDL; ++i) s = fma(bf16_to_f64(y[i]), e4m3_to_f64(c[i]) * 0x1p-8, s);
-    return s;
-}
-
-// Exact score of two bf16 latents: every product of two bf16 values is exact
-// in fp64; the sum runs in ascending index order.
-__device__ __forceinline__ double dot_bf16_exact(const uint16_t* __restrict__ y,
-                                                 const uint16_t* __restrict__ c) {
-    double s = 0.0;
-#pragma unroll 8
-    for (int i = 0; i < kDL; ++i) s = fma(bf16_to_f64(y[i]), bf16_to_f64(c[i]), s);
-    return s;
-}
-
 template <typename T>
 __host__ __device__ __forceinline__ T ceil_div(T a, T b) { return (a + b - 1) / b; }
 

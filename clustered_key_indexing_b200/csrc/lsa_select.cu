@@ -116,16 +116,6 @@ __device__ void emit_bucket(const SelectArgs& a, int h, int64_t b, int tk, int64
     }
 }
 
-// Exact (fp64) score of node centroid c against the query latent(s) in shared memory.
-__device__ __forceinline__ double exact_score(const uint16_t* ylat, int ng, const uint16_t* c) {
-    double best = -CUDART_INF;
-    for (int g = 0; g < ng; ++g) {
-        const double v = dot_bf16_exact(ylat + g * kDL, c);
-        best = v > best ? v : best;
-    }
-    return best;
-}
-
 // Block-wide exclusive scan of one int per thread; returns the prefix and the total.
 __device__ __forceinline__ int block_exscan(int v, int* total, int* sh4) {
     const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
