@@ -608,6 +608,10 @@ def run_lsa(args):
     if roofline_scoring:
         roofline_scoring["note"] = ("tcgen05 scores of every eligible centroid; the epilogue appends the candidates "
                                     "(score >= tau, about 2k keys' buckets per row)")
+    roofline_band = roof("band_attn_kernel")
+    if roofline_band:
+        roofline_band["note"] = ("tcgen05 window attention: S = Q K^T and O = P V in tensor memory; achieved = "
+                                 "4 x 128 FLOP per valid (window entry, query head)")
 
     # tree search over the same layer, timed on its own
     tree_line = None
@@ -644,6 +648,7 @@ def run_lsa(args):
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": config_json(args, c, world, P.split), "query_chunk": P.chunk, "clocks": clk, "e2e": e2e,
         "gpu_launches": int(launches), "roofline": roofline, "roofline_scoring": roofline_scoring,
+        "roofline_band": roofline_band,
         "tree": tree_line, "kernels": kernels, "cpu_baseline": cpu,
         "stages_ms_per_step": stages, "select_fallback_rows_per_step": fallback_rows / args.steps,
     }
